@@ -1,0 +1,391 @@
+"""Pins of the fp64 oracle against facts fixed by the pages and by mathematics.
+
+Each test checks the oracle against something other than itself: a closed form
+(linear attention), a hand-worked example, brute-force scalar loops, central
+finite differences, an SVD, or an invariance the method must have.  None of
+these needs a GPU.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle as orc
+from synth_inputs import make_config
+
+RNG = np.random.default_rng(12345)
+KINDS = ["linear", "mlp2_gelu", "swiglu"]
+LOSSES = ["mse", "neg_dot"]
+
+
+def rand(*shape, scale=1.0):
+    return RNG.standard_normal(shape) * scale
+
+
+def cfg_for(kind, loss, **kw):
+    base = dict(inner=kind, loss=loss, opt="gd", dtype="f32", d=4, h=6, N=8, key_instnorm=False,
+                weight_l2norm=False, eta_mode="per_token")
+    base.update(kw)
+    return make_config(**base)
+
+
+def rand_w(kind, d, h, scale=0.5):
+    return {name: rand(r, c, scale=scale) for name, r, c in orc.matrix_shapes(kind, d, h)}
+
+
+# ---------------------------------------------------------------- activations
+def test_gelu_textbook_values():
+    # GELU(x) = x * Phi(x); Phi(1) = 0.8413447460685429 (standard normal CDF)
+    x = np.array([0.0, 1.0, -1.0, 8.0, -8.0])
+    g = orc.gelu(x)
+    assert g[0] == 0.0
+    assert abs(g[1] - 0.8413447460685429) < 1e-15
+    assert abs(g[2] + 0.15865525393145707) < 1e-15
+    assert abs(g[3] - 8.0) < 1e-12 and abs(g[4]) < 1e-12
+
+
+def test_silu_textbook_values():
+    x = np.array([0.0, 1.0, -1.0])
+    s = orc.silu(x)
+    assert s[0] == 0.0
+    assert abs(s[1] - 1.0 / (1.0 + math.exp(-1.0))) < 1e-15
+    assert abs(s[2] + 1.0 / (1.0 + math.exp(1.0))) < 1e-15
+
+
+@pytest.mark.parametrize("fn,dfn", [(orc.gelu, orc.gelu_prime), (orc.silu, orc.silu_prime)])
+def test_activation_derivatives_by_finite_difference(fn, dfn):
+    x = np.linspace(-6, 6, 97)
+    eps = 1e-6
+    fd = (fn(x + eps) - fn(x - eps)) / (2 * eps)
+    assert np.max(np.abs(fd - dfn(x))) < 1e-8
+
+
+# ---------------------------------------------------------------- brute-force forward
+def _brute_forward(kind, W, x):
+    """Scalar loops with math.erf / math.exp on one token (no numpy linear algebra)."""
+    def gelu(z):
+        return 0.5 * z * (1.0 + math.erf(z / math.sqrt(2.0)))
+
+    def silu(z):
+        return z / (1.0 + math.exp(-z))
+
+    def matvec(M, v):
+        return [sum(M[i][j] * v[j] for j in range(len(v))) for i in range(len(M))]
+
+    if kind == "linear":
+        return matvec(W["W"].tolist(), x)
+    if kind == "mlp2_gelu":
+        hid = [gelu(z) for z in matvec(W["W1"].tolist(), x)]
+        return matvec(W["W2"].tolist(), hid)
+    z1 = matvec(W["W1"].tolist(), x)
+    z3 = matvec(W["W3"].tolist(), x)
+    hid = [silu(a) * b for a, b in zip(z1, z3)]
+    return matvec(W["W2"].tolist(), hid)
+
+
+@pytest.mark.parametrize("kind", KINDS)
+def test_inner_forward_matches_scalar_loops(kind):
+    d, h = 5, 7
+    W = rand_w(kind, d, h)
+    X = rand(6, d)
+    Y = orc.inner_forward(kind, W, X)[0]
+    for i in range(X.shape[0]):
+        ref = _brute_forward(kind, W, X[i].tolist())
+        assert np.allclose(Y[i], ref, rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------- gradients
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("loss", LOSSES)
+def test_gradients_by_central_finite_differences(kind, loss):
+    d, h, n = 4, 6, 8
+    W = rand_w(kind, d, h)
+    X, V = rand(n, d), rand(n, d)
+    eta = np.abs(rand(n)) + 0.1
+
+    def L(Wd):
+        return orc.loss_value(loss, orc.inner_forward(kind, Wd, X)[0], V, eta)
+
+    Vhat, cache = orc.inner_forward(kind, W, X)
+    G = orc.inner_backward(kind, W, cache, orc.loss_grad(loss, Vhat, V, eta))
+    eps = 1e-6
+    for name, M in W.items():
+        fd = np.zeros_like(M)
+        for idx in np.ndindex(M.shape):
+            Wp = {k: v.copy() for k, v in W.items()}
+            Wm = {k: v.copy() for k, v in W.items()}
+            Wp[name][idx] += eps
+            Wm[name][idx] -= eps
+            fd[idx] = (L(Wp) - L(Wm)) / (2 * eps)
+        rel = np.linalg.norm(fd - G[name]) / np.linalg.norm(G[name])
+        assert rel < 1e-7, (name, rel)
+
+
+# ---------------------------------------------------------------- closed forms
+def _linear_attention_state(W0, K, V, eta):
+    """W0 + sum_i eta_i v_i k_i^T, accumulated token by token with outer products."""
+    W = W0.copy()
+    for i in range(K.shape[0]):
+        W += eta[i] * np.outer(V[i], K[i])
+    return W
+
+
+@pytest.mark.parametrize("chunk", [0, 3, 5, 16])
+def test_linear_dot_is_linear_attention(chunk):
+    # linear inner model + negative dot loss + plain step: W* = W0 + V^T diag(eta) K and O = Q W*^T,
+    # whatever the chunking, because the gradient does not depend on W.
+    d, n = 5, 16
+    cfg = cfg_for("linear", "neg_dot", d=d, h=d, N=n, chunk=chunk)
+    Q, K, V = rand(n, d), rand(n, d), rand(n, d)
+    eta = np.abs(rand(n))
+    W0 = rand(d, d)
+    O, Ws = orc.forward_head(cfg, Q, K, V, eta, W0.reshape(-1))
+    Wref = _linear_attention_state(W0, K, V, eta)
+    assert np.allclose(Ws.reshape(d, d), Wref, rtol=1e-12, atol=1e-12)
+    Oref = np.array([[sum(Wref[r, c] * Q[i, c] for c in range(d)) for r in range(d)] for i in range(n)])
+    assert np.allclose(O, Oref, rtol=1e-12, atol=1e-12)
+
+
+def test_linear_dot_causal_is_chunkwise_causal_linear_attention():
+    d, n, C = 4, 10, 3
+    cfg = cfg_for("linear", "neg_dot", d=d, h=d, N=n, chunk=C, causal=1)
+    Q, K, V = rand(n, d), rand(n, d), rand(n, d)
+    eta = np.abs(rand(n))
+    W0 = rand(d, d)
+    O, Ws = orc.forward_head(cfg, Q, K, V, eta, W0.reshape(-1))
+    for s in range(0, n, C):
+        Wc = _linear_attention_state(W0, K[:s], V[:s], eta[:s])  # only earlier chunks
+        for i in range(s, min(s + C, n)):
+            assert np.allclose(O[i], Wc @ Q[i], rtol=1e-12, atol=1e-12)
+    assert np.allclose(Ws.reshape(d, d), _linear_attention_state(W0, K, V, eta), rtol=1e-12, atol=1e-12)
+
+
+def test_linear_mse_closed_form():
+    # V_hat = K W0^T; dL/dV_hat = 2 eta (V_hat - V)/(n d); W* = W0 - sum_i 2 eta_i/(n d) (W0 k_i - v_i) k_i^T
+    d, n = 4, 9
+    cfg = cfg_for("linear", "mse", d=d, h=d, N=n)
+    Q, K, V = rand(n, d), rand(n, d), rand(n, d)
+    eta = np.abs(rand(n))
+    W0 = rand(d, d)
+    _, Ws = orc.forward_head(cfg, Q, K, V, eta, W0.reshape(-1))
+    G = np.zeros((d, d))
+    for i in range(n):
+        G += 2.0 * eta[i] / (n * d) * np.outer(W0 @ K[i] - V[i], K[i])
+    assert np.allclose(Ws.reshape(d, d), W0 - G, rtol=1e-12, atol=1e-12)
+
+
+def test_linear_mse_eta_is_a_rescaling_of_k_and_v():
+    # ViT3 digest, guideline 3: for a linear inner model with MSE, eta is equivalent to scaling K and V.
+    # With W0 = 0:  O(eta * a * b; K, V) == O(eta; a K, b V).
+    d, n, a, b, eta0 = 4, 7, 1.7, -0.6, 0.8
+    Q, K, V = rand(n, d), rand(n, d), rand(n, d)
+    W0 = np.zeros(d * d)
+    c1 = cfg_for("linear", "mse", d=d, h=d, N=n, eta_mode="scalar", eta_scalar=eta0 * a * b)
+    c2 = cfg_for("linear", "mse", d=d, h=d, N=n, eta_mode="scalar", eta_scalar=eta0)
+    O1, _ = orc.forward_head(c1, Q, K, V, None, W0)
+    O2, _ = orc.forward_head(c2, Q, a * K, b * V, None, W0)
+    assert np.allclose(O1, O2, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("name", ["neg_dot", "mse"])
+def test_hand_worked_linear_example(repo_root, name):
+    g = json.load(open(os.path.join(repo_root, "tests", "golden", "linear_two_tokens.json")))
+    d = g["d"]
+    K, V, eta = np.array(g["K"], float), np.array(g["V"], float), np.array(g["eta"], float)
+    W0 = np.array(g["W0"], float)
+    q = np.array(g["q"], float)[None, :]
+    cfg = cfg_for("linear", name, d=d, h=d, N=2, Nq=1)
+    O, Ws = orc.forward_head(cfg, q, K, V, eta, W0.reshape(-1))
+    case = g["cases"][name]
+    assert np.allclose(Ws.reshape(d, d), np.array(case["W_star"]), rtol=0, atol=1e-14)
+    assert np.allclose(O[0], np.array(case["O"]), rtol=0, atol=1e-14)
+
+
+# ---------------------------------------------------------------- special cases
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("loss", LOSSES)
+@pytest.mark.parametrize("rownorm", [False, True])
+def test_eta_zero_reduces_to_initial_weights(kind, loss, rownorm):
+    d, h, n = 4, 6, 9
+    cfg = cfg_for(kind, loss, d=d, h=h, N=n, eta_mode="scalar", eta_scalar=0.0, weight_l2norm=rownorm,
+                  key_instnorm=True)
+    Q, K, V = rand(n, d), rand(n, d), rand(n, d)
+    W = rand_w(kind, d, h)
+    w0 = orc.pack(kind, d, h, W)
+    O, Ws = orc.forward_head(cfg, Q, K, V, None, w0)
+    Wexp = {k: (orc.row_l2_normalize(v) if rownorm else v) for k, v in W.items()}
+    assert np.allclose(Ws, orc.pack(kind, d, h, Wexp), rtol=1e-14, atol=1e-14)
+    for i in range(n):
+        assert np.allclose(O[i], _brute_forward(kind, Wexp, Q[i].tolist()), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("opt", ["gd", "momentum", "muon", "momentum_muon"])
+def test_causal_with_chunk_n_equals_single_chunk(kind, opt):
+    # apply-before-update: W* is that of the non-causal single chunk; O reads W0 (reading R16).
+    d, h, n = 4, 6, 10
+    kw = dict(d=d, h=h, N=n, opt=opt, weight_l2norm=True)
+    Q, K, V = rand(n, d), rand(n, d), rand(n, d)
+    eta = np.abs(rand(n)) * 0.1
+    W = rand_w(kind, d, h)
+    w0 = orc.pack(kind, d, h, W)
+    Oc, Wc = orc.forward_head(cfg_for(kind, "neg_dot", chunk=n, causal=1, **kw), Q, K, V, eta, w0)
+    On, Wn = orc.forward_head(cfg_for(kind, "neg_dot", chunk=0, causal=0, **kw), Q, K, V, eta, w0)
+    assert np.allclose(Wc, Wn, rtol=1e-13, atol=1e-13)
+    for i in range(n):
+        assert np.allclose(Oc[i], _brute_forward(kind, W, Q[i].tolist()), rtol=1e-12, atol=1e-12)
+
+
+def test_causal_prefix_consistency():
+    # the causal output of chunk c is F applied with the weights a non-causal chunked run
+    # reaches on the first c chunks (no future leakage, LaCT analysis "Order of operations").
+    kind, d, h, n, C = "swiglu", 4, 6, 12, 4
+    kw = dict(d=d, h=h, opt="momentum", weight_l2norm=True)
+    Q, K, V = rand(n, d), rand(n, d), rand(n, d)
+    eta = np.abs(rand(n)) * 0.1
+    w0 = orc.pack(kind, d, h, rand_w(kind, d, h))
+    Oc, _ = orc.forward_head(cfg_for(kind, "neg_dot", N=n, chunk=C, causal=1, **kw), Q, K, V, eta, w0)
+    for c in range(1, n // C):
+        s = c * C
+        cfgp = cfg_for(kind, "neg_dot", N=s, Nq=C, chunk=C, causal=0, **kw)
+        Op, _ = orc.forward_head(cfgp, Q[s:s + C], K[:s], V[:s], eta[:s], w0)
+        assert np.allclose(Oc[s:s + C], Op, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- optimizer pieces
+def _quintic_on_singular_values(G, iters, coeff):
+    a, b, c = coeff
+    U, S, Vt = np.linalg.svd(G, full_matrices=False)
+    s = S / (np.linalg.norm(G) + 1e-7)
+    for _ in range(iters):
+        s = a * s + b * s ** 3 + c * s ** 5
+    return (U * s) @ Vt
+
+
+@pytest.mark.parametrize("shape", [(6, 10), (10, 6), (7, 7)])
+@pytest.mark.parametrize("iters", [0, 1, 5])
+def test_newton_schulz_is_a_polynomial_of_the_singular_values(shape, iters):
+    coeff = (3.4445, -4.7750, 2.0315)
+    G = rand(*shape)
+    X = orc.newton_schulz(G, iters, coeff)
+    assert np.allclose(X, _quintic_on_singular_values(G, iters, coeff), rtol=1e-10, atol=1e-12)
+
+
+def test_newton_schulz_orientation_and_zero_iterations():
+    coeff = (3.4445, -4.7750, 2.0315)
+    G = rand(5, 9)
+    assert np.allclose(orc.newton_schulz(G.T, 5, coeff), orc.newton_schulz(G, 5, coeff).T, rtol=1e-12, atol=1e-14)
+    assert np.allclose(orc.newton_schulz(G, 0, coeff), G / (np.linalg.norm(G) + 1e-7), rtol=1e-14, atol=0)
+
+
+def test_newton_schulz_cubic_converges_to_polar_factor():
+    # classical cubic (1.5, -0.5, 0) on a well-conditioned matrix converges to U V^T
+    U, _ = np.linalg.qr(rand(6, 6))
+    Vt = np.linalg.qr(rand(9, 9))[0][:6]
+    G = (U * np.linspace(0.3, 1.0, 6)) @ Vt
+    X = orc.newton_schulz(G, 40, (1.5, -0.5, 0.0))
+    assert np.allclose(X @ X.T, np.eye(6), atol=1e-10)
+    assert np.allclose(X, U @ Vt, atol=1e-10)
+
+
+def test_momentum_two_chunk_closed_form():
+    # linear + dot: the chunk gradient G_c = -sum eta_i v_i k_i^T does not depend on W, so
+    # W1 = W0 - G0 and W2 = W1 - (beta G0 + G1).
+    d, n, C, beta = 3, 8, 4, 0.9
+    cfg = cfg_for("linear", "neg_dot", d=d, h=d, N=n, chunk=C, opt="momentum", momentum=beta)
+    Q, K, V = rand(n, d), rand(n, d), rand(n, d)
+    eta = np.abs(rand(n))
+    W0 = rand(d, d)
+    _, Ws = orc.forward_head(cfg, Q, K, V, eta, W0.reshape(-1))
+    G0 = -sum(eta[i] * np.outer(V[i], K[i]) for i in range(C))
+    G1 = -sum(eta[i] * np.outer(V[i], K[i]) for i in range(C, n))
+    W2 = (W0 - G0) - (beta * G0 + G1)
+    assert np.allclose(Ws.reshape(d, d), W2, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("kind", KINDS)
+def test_momentum_zero_is_plain_step(kind):
+    d, h, n = 4, 6, 12
+    Q, K, V = rand(n, d), rand(n, d), rand(n, d)
+    eta = np.abs(rand(n)) * 0.3
+    w0 = orc.pack(kind, d, h, rand_w(kind, d, h))
+    a = orc.forward_head(cfg_for(kind, "neg_dot", N=n, chunk=4, opt="momentum", momentum=0.0), Q, K, V, eta, w0)
+    b = orc.forward_head(cfg_for(kind, "neg_dot", N=n, chunk=4, opt="gd"), Q, K, V, eta, w0)
+    assert np.allclose(a[0], b[0], rtol=1e-13, atol=1e-13) and np.allclose(a[1], b[1], rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("kind", KINDS)
+def test_row_norm_gives_unit_rows_and_is_idempotent(kind):
+    d, h, n = 4, 6, 9
+    cfg = cfg_for(kind, "neg_dot", d=d, h=h, N=n, weight_l2norm=True, opt="muon")
+    Q, K, V = rand(n, d), rand(n, d), rand(n, d)
+    _, Ws = orc.forward_head(cfg, Q, K, V, np.abs(rand(n)), orc.pack(kind, d, h, rand_w(kind, d, h)))
+    W = orc.unpack(kind, d, h, Ws)
+    for name, M in W.items():
+        assert np.allclose(np.sqrt((M * M).sum(axis=1)), 1.0, atol=1e-13), name
+        assert np.allclose(orc.row_l2_normalize(M), M, atol=1e-15)
+
+
+# ---------------------------------------------------------------- instance norm
+def test_instance_norm_moments():
+    K = rand(50, 6) * 3 + 2
+    Kt = orc.instance_norm(K, 0.0)
+    assert np.allclose(Kt.mean(axis=0), 0.0, atol=1e-13)
+    assert np.allclose((Kt ** 2).mean(axis=0), 1.0, atol=1e-12)
+
+
+@pytest.mark.parametrize("kind", KINDS)
+def test_key_instance_norm_removes_per_channel_shift_and_scale(kind):
+    # TTT vs Sleep, "Side one": a constant per-channel key shift must not change the layer.
+    d, h, n = 5, 6, 11
+    Q, K, V = rand(n, d), rand(n, d), rand(n, d)
+    w0 = orc.pack(kind, d, h, rand_w(kind, d, h))
+    cfg = cfg_for(kind, "mse", d=d, h=h, N=n, key_instnorm=True, in_eps=0.0, eta_mode="scalar")
+    O1, W1 = orc.forward_head(cfg, Q, K, V, None, w0)
+    shift = rand(1, d) * 5
+    O2, W2 = orc.forward_head(cfg, Q, K + shift, V, None, w0)
+    scale = np.abs(rand(1, d)) + 0.5
+    O3, W3 = orc.forward_head(cfg, Q, K * scale, V, None, w0)
+    for O, Wx in ((O2, W2), (O3, W3)):
+        assert np.allclose(O, O1, rtol=1e-10, atol=1e-10)
+        assert np.allclose(Wx, W1, rtol=1e-10, atol=1e-10)
+
+
+# ---------------------------------------------------------------- token-set semantics
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("loss", LOSSES)
+def test_single_chunk_is_invariant_to_token_permutation(kind, loss):
+    # LaCT analysis, "Nonlinear memory": a large-chunk update treats the tokens as a set.
+    d, h, n = 4, 6, 13
+    Q, K, V = rand(n, d), rand(n, d), rand(n, d)
+    eta = np.abs(rand(n))
+    w0 = orc.pack(kind, d, h, rand_w(kind, d, h))
+    cfg = cfg_for(kind, loss, d=d, h=h, N=n, key_instnorm=True, weight_l2norm=True, opt="muon")
+    O1, W1 = orc.forward_head(cfg, Q, K, V, eta, w0)
+    p = RNG.permutation(n)
+    O2, W2 = orc.forward_head(cfg, Q, K[p], V[p], eta[p], w0)
+    assert np.allclose(O1, O2, rtol=1e-11, atol=1e-11) and np.allclose(W1, W2, rtol=1e-11, atol=1e-11)
+
+
+def test_chunk_bounds_cover_tokens_once():
+    assert orc.chunk_bounds(10, 0) == [(0, 10)]
+    assert orc.chunk_bounds(10, 10) == [(0, 10)]
+    assert orc.chunk_bounds(10, 4) == [(0, 4), (4, 8), (8, 10)]
+    b = orc.chunk_bounds(1029120, 131072)
+    assert len(b) == 8 and b[-1] == (917504, 1029120) and b[-1][1] - b[-1][0] == 111616
+
+
+def test_forward_all_heads_matches_per_head():
+    cfg = make_config(B=2, H=2, N=9, d=4, h=6, inner="swiglu", loss="neg_dot", opt="momentum",
+                      chunk=4, eta_mode="per_token", dtype="f32", data="lact")
+    from synth_inputs import gen_inputs
+    x = gen_inputs(cfg)
+    O, W = orc.forward(cfg, x["Q"], x["K"], x["V"], x["eta"], x["W0"])
+    for b in range(2):
+        for hh in range(2):
+            o, w = orc.forward_head(cfg, x["Q"][b, hh].double().numpy(), x["K"][b, hh].double().numpy(),
+                                    x["V"][b, hh].double().numpy(), x["eta"][b, hh].double().numpy(),
+                                    x["W0"][hh].double().numpy())
+            assert np.array_equal(O[b, hh], o) and np.array_equal(W[b, hh], w)
