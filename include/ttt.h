@@ -1,0 +1,141 @@
+/*
+ * ttt.h -- C ABI of the B200 (sm_100a) TTT-layer forward pass.
+ *
+ * The TTT (test-time training) layer replaces Softmax attention: the keys and
+ * values of a chunk form a small training set, a fast-weight inner model F_W
+ * takes one full-batch gradient step on a reconstruction loss over it, and the
+ * queries then read the updated weights, O = F_{W*}(Q).
+ *   Source: ViT3 digest ("ViT^3 test-time training for vision"), section 02,
+ *   update equation  V_hat = F_W(K_B); W <- W - eta dL(V_hat, V_B)/dW; O = F_{W*}(Q);
+ *   LaCT analysis ("Test-Time Training Done Right"), sections "Fast weights",
+ *   "Nonlinear memory complements local attention" and "Order of operations".
+ *
+ * Conventions
+ *   - Every matrix is row-major.  Fast weights are stored PyTorch-Linear style,
+ *     [out, in], and applied to row vectors as x W^T.  Per head they are packed
+ *     one after the other (P floats per head):
+ *        TTT_INNER_LINEAR     [W  (d x d)]
+ *        TTT_INNER_MLP2_GELU  [W1 (h x d) | W2 (d x h)]         F(x) = GELU(x W1^T) W2^T
+ *        TTT_INNER_SWIGLU     [W1 (h x d) | W3 (h x d) | W2 (d x h)]
+ *                                                    F(x) = (SiLU(x W1^T) * x W3^T) W2^T
+ *   - Q [B,H,Nq,d], K [B,H,N,d], V [B,H,N,d] and O [B,H,Nq,d] in `dtype`
+ *     (fp32 or bf16); eta [B,H,N] fp32; W0 [H,P] fp32 (shared by every batch
+ *     entry); W_out [B,H,P] fp32.
+ *   - Losses, summed over the chunk's tokens with the per-token learning rate eta_i:
+ *        TTT_LOSS_MSE      L = sum_i eta_i ||F(k_i) - v_i||^2 / (n_chunk * d)
+ *        TTT_LOSS_NEG_DOT  L = -sum_i eta_i <F(k_i), v_i>
+ *   - One step per chunk: G -> [momentum M <- beta M + G] -> [Muon: Newton-Schulz]
+ *     -> W <- W - lr U -> [each row of each matrix scaled to unit L2 norm].
+ *   - causal = 1 (needs Nq == N): per chunk, first O_c = F_W(Q_c), then update.
+ *     causal = 0: update over every chunk in order, then O = F_{W*}(Q).
+ *   - Nothing persists between calls: momentum starts at zero in every call.
+ *
+ * Ownership and threading
+ *   The caller owns every buffer (inputs, outputs and the workspace); the handle
+ *   owns only host-side state.  Device pointers must be 16-byte aligned and
+ *   contiguous.  ttt_forward only enqueues work on `stream` and returns; it
+ *   allocates nothing.  One handle must not be used on two streams at once.
+ *
+ * Errors
+ *   Calls return TTT_OK (0) or a negative status.  Argument errors are found on
+ *   the host before anything is enqueued.  Conditions found on the device
+ *   (non-finite outputs, a bounded wait that ran out) are recorded in a status
+ *   word at the start of the workspace and returned by ttt_query_status.
+ *   Nothing traps or asserts on the device.
+ */
+#ifndef TTT_H_
+#define TTT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TTT_OK 0
+#define TTT_ERR_INVALID_ARG (-1) /* null pointer, bad shape, causal with Nq != N, ... */
+#define TTT_ERR_UNSUPPORTED (-2) /* a valid combination this build does not implement */
+#define TTT_ERR_CUDA (-3)        /* a CUDA runtime call failed */
+#define TTT_ERR_NONFINITE (-4)   /* O or W* holds Inf or NaN (device status word) */
+#define TTT_ERR_TIMEOUT (-5)     /* a bounded device-side wait ran out (device status word) */
+#define TTT_ERR_WORKSPACE (-6)   /* workspace too small or misaligned */
+
+typedef enum { TTT_INNER_LINEAR = 0, TTT_INNER_MLP2_GELU = 1, TTT_INNER_SWIGLU = 2 } ttt_inner_kind;
+typedef enum { TTT_LOSS_MSE = 0, TTT_LOSS_NEG_DOT = 1 } ttt_loss_kind;
+typedef enum {
+  TTT_OPT_GD = 0,            /* U = G */
+  TTT_OPT_MOMENTUM = 1,      /* M <- beta M + G; U = M */
+  TTT_OPT_MUON = 2,          /* U = NS(G) */
+  TTT_OPT_MOMENTUM_MUON = 3  /* M <- beta M + G; U = NS(M) */
+} ttt_opt_kind;
+typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
+
+#define TTT_FLAG_KEY_INSTNORM 1u  /* normalise each key channel over the chunk's tokens */
+#define TTT_FLAG_WEIGHT_L2NORM 2u /* unit L2 norm for every weight row after each update */
+
+typedef struct ttt_config {
+  int32_t B, H;       /* batch entries and heads */
+  int32_t N, Nq;      /* key/value tokens and query tokens */
+  int32_t d, h;       /* head dim and inner hidden width (ignored for LINEAR) */
+  int32_t chunk;      /* tokens per update; <= 0 or >= N means one chunk of N */
+  int32_t causal;     /* 1: apply-then-update per chunk (needs Nq == N) */
+  int32_t inner;      /* ttt_inner_kind */
+  int32_t loss;       /* ttt_loss_kind */
+  int32_t opt;        /* ttt_opt_kind */
+  int32_t dtype;      /* ttt_dtype of Q, K, V and O */
+  uint32_t flags;     /* TTT_FLAG_* */
+  float eta_scalar;   /* learning rate of every token when eta == NULL */
+  float lr;           /* multiplies the update U (default 1) */
+  float momentum;     /* beta of the momentum optimizers */
+  int32_t ns_iters;   /* Newton-Schulz iterations (default 5) */
+  float ns_coeff[3];  /* quintic (a, b, c), default (3.4445, -4.7750, 2.0315) */
+  float in_eps;       /* instance-norm epsilon (default 1e-5) */
+} ttt_config;
+
+typedef struct ttt_handle ttt_handle;
+
+/* Fill `cfg` with defaults (lr 1, momentum 0.9, 5 NS iterations with the Muon
+ * quintic, in_eps 1e-5, eta_scalar 1); shapes are zero and must be set. */
+void ttt_config_init(ttt_config* cfg);
+
+/* Validate `cfg` and build a handle.  Host only; no device work.  Returns
+ * TTT_ERR_INVALID_ARG / TTT_ERR_UNSUPPORTED and leaves *out NULL on failure. */
+int ttt_create(const ttt_config* cfg, ttt_handle** out);
+
+/* Fast-weight floats per head (P). */
+int64_t ttt_param_count(const ttt_handle* handle);
+
+/* Device workspace bytes ttt_forward needs (256-byte aligned buffer). */
+size_t ttt_workspace_size(const ttt_handle* handle);
+
+/* Enqueue one TTT-layer forward pass on `stream` (a cudaStream_t; NULL = legacy
+ * default stream).  All pointers are device pointers.  eta may be NULL (then
+ * cfg.eta_scalar is every token's rate); W_out may be NULL.  O and W_out are
+ * fully overwritten.  Returns without waiting for the GPU. */
+int ttt_forward(ttt_handle* handle, const void* Q, const void* K, const void* V, const float* eta,
+                const float* W0, void* O, float* W_out, void* workspace, size_t workspace_bytes,
+                void* stream);
+
+/* The same pass on HOST buffers (pinned memory gives asynchronous copies):
+ * copies the inputs into the front of `device_staging`, runs ttt_forward and
+ * copies O (and W_out when non-NULL) back, all enqueued on `stream`.  The host
+ * outputs are valid after the stream is synchronised. */
+size_t ttt_host_staging_size(const ttt_handle* handle);
+int ttt_forward_host(ttt_handle* handle, const void* Q, const void* K, const void* V, const float* eta,
+                     const float* W0, void* O, float* W_out, void* device_staging, size_t staging_bytes,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream`, read the device status word of `workspace` and clear
+ * it.  Returns TTT_OK, TTT_ERR_NONFINITE, TTT_ERR_TIMEOUT or TTT_ERR_CUDA. */
+int ttt_query_status(ttt_handle* handle, void* workspace, void* stream);
+
+void ttt_destroy(ttt_handle* handle);
+
+/* Static text for a status code. */
+const char* ttt_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TTT_H_ */

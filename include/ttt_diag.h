@@ -1,0 +1,31 @@
+/*
+ * ttt_diag.h -- diagnostic entry points of the TTT-layer library.
+ *
+ * These exercise single building blocks of the forward pass so that they can be
+ * checked in isolation against a library routine.  They are not part of the
+ * layer's statement of the problem (no page defines them).
+ */
+#ifndef TTT_DIAG_H_
+#define TTT_DIAG_H_
+
+#include "ttt.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* One batched GEMM through the library's tcgen05 tensor-core engine:
+ *   C[s][z] = sum over the k-blocks of split s of  A[z] * B[z]^T
+ * elem_bytes 2: A, B bf16 (kind::f16); 4: A, B fp32 read as tf32 (kind::tf32), K-major only
+ * (TTT_ERR_UNSUPPORTED otherwise).
+ * A is [batches][M][K] when a_mn == 0 (K-major) and [batches][K][M] when a_mn == 1
+ * (MN-major); B likewise with N.  C is fp32 [splits][batches][M][N], written for
+ * every element.  bn is the output tile width (64/128/256 for bf16, 128/256 for
+ * fp32).  Rows of A/B must be 16-byte multiples.  Enqueued on `stream`. */
+int ttt_selftest_gemm(int elem_bytes, int a_mn, int b_mn, int bn, int M, int N, int K, int batches, int splits,
+                      const void* A, const void* B, float* C, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TTT_DIAG_H_ */

@@ -1,0 +1,92 @@
+"""The C-ABI library: loads, exports every function include/*.h declares, and
+validates configurations on the host (no GPU needed for any of this)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from synth_inputs import make_config, workload, WORKLOADS
+
+
+def _declared(repo_root):
+    names = set()
+    for f in os.listdir(os.path.join(repo_root, "include")):
+        if f.endswith(".h"):
+            text = open(os.path.join(repo_root, "include", f)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            for m in re.finditer(r"\b(ttt_[a-z0-9_]+)\s*\(", text):
+                names.add(m.group(1))
+    return names
+
+
+def test_library_exports_every_declared_function(repo_root):
+    from weight_sequence_mixing_b200 import binding
+    names = _declared(repo_root)
+    assert {"ttt_create", "ttt_forward", "ttt_destroy", "ttt_workspace_size"} <= names
+    lib = ctypes.CDLL(binding._LIB_PATH)
+    for n in sorted(names):
+        assert hasattr(lib, n), n
+    assert names <= set(binding.EXPORTED)
+
+
+def _create(cfg_c):
+    from weight_sequence_mixing_b200 import binding
+    h = ctypes.c_void_p()
+    st = binding.LIB.ttt_create(ctypes.byref(cfg_c), ctypes.byref(h))
+    return st, h
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_every_workload_configuration_is_accepted(name):
+    from weight_sequence_mixing_b200 import binding
+    cfg = workload(name)
+    st, h = _create(binding.make_config(cfg))
+    assert st == 0, binding.status_string(st)
+    P = binding.LIB.ttt_param_count(h)
+    expect = {"linear": 1, "mlp2_gelu": 2, "swiglu": 3}[cfg["inner"]] * cfg["d"] * cfg["h"]
+    assert P == expect
+    assert binding.LIB.ttt_workspace_size(h) >= 256
+    assert binding.LIB.ttt_host_staging_size(h) > 0
+    binding.LIB.ttt_destroy(h)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(B=0), dict(N=0), dict(d=0), dict(causal=1, Nq=7),
+])
+def test_invalid_configurations_are_rejected(bad):
+    from weight_sequence_mixing_b200 import binding
+    kw = dict(N=16, d=64, h=128, dtype="bf16")
+    kw.update(bad)
+    c = binding.make_config(make_config(**kw))
+    st, h = _create(c)
+    assert st == binding.TTT_ERR_INVALID_ARG and not h.value
+
+
+def test_invalid_enum_and_flag_values_are_rejected():
+    from weight_sequence_mixing_b200 import binding
+    for field, value in (("inner", 7), ("loss", -1), ("opt", 9), ("dtype", 5), ("flags", 64), ("ns_iters", -1)):
+        c = binding.make_config(make_config(N=16, d=64, h=128))
+        setattr(c, field, value)
+        st, h = _create(c)
+        assert st == binding.TTT_ERR_INVALID_ARG, field
+
+
+def test_forward_rejects_null_and_small_workspace_without_touching_the_gpu():
+    from weight_sequence_mixing_b200 import binding
+    st, h = _create(binding.make_config(make_config(N=16, d=64, h=128)))
+    assert st == 0
+    lib = binding.LIB
+    fake = ctypes.c_void_p(4096)
+    assert lib.ttt_forward(h, None, fake, fake, None, fake, fake, None, fake, 1 << 30, None) == binding.TTT_ERR_INVALID_ARG
+    assert lib.ttt_forward(h, fake, fake, fake, None, fake, fake, None, fake, 16, None) == binding.TTT_ERR_WORKSPACE
+    misaligned = ctypes.c_void_p(4096 + 8)
+    assert lib.ttt_forward(h, misaligned, fake, fake, None, fake, fake, None, fake, 1 << 30, None) == binding.TTT_ERR_INVALID_ARG
+    lib.ttt_destroy(h)
+
+
+def test_status_strings():
+    from weight_sequence_mixing_b200 import binding
+    for s in range(-6, 1):
+        assert binding.status_string(s) and binding.status_string(s) != "unknown status"
+    assert binding.status_string(-99) == "unknown status"

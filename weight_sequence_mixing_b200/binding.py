@@ -1,0 +1,197 @@
+"""ctypes binding of libttt_b200.so (the C ABI declared in include/ttt.h).
+
+Argument marshalling only: every step of the TTT forward pass runs in the CUDA
+library.  torch tensors are used for device memory and streams.  There is no
+CPU fallback: if the library is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, field
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libttt_b200.so")
+
+TTT_OK = 0
+TTT_ERR_INVALID_ARG = -1
+TTT_ERR_UNSUPPORTED = -2
+TTT_ERR_CUDA = -3
+TTT_ERR_NONFINITE = -4
+TTT_ERR_TIMEOUT = -5
+TTT_ERR_WORKSPACE = -6
+
+INNER = {"linear": 0, "mlp2_gelu": 1, "swiglu": 2}
+LOSS = {"mse": 0, "neg_dot": 1}
+OPT = {"gd": 0, "momentum": 1, "muon": 2, "momentum_muon": 3}
+DTYPE = {"f32": 0, "bf16": 1}
+FLAG_KEY_INSTNORM = 1
+FLAG_WEIGHT_L2NORM = 2
+
+EXPORTED = [
+    "ttt_config_init", "ttt_create", "ttt_param_count", "ttt_workspace_size", "ttt_forward",
+    "ttt_host_staging_size", "ttt_forward_host", "ttt_query_status", "ttt_destroy", "ttt_status_string",
+    "ttt_selftest_gemm",
+]
+
+
+class TTTConfig(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32), ("Nq", ctypes.c_int32),
+        ("d", ctypes.c_int32), ("h", ctypes.c_int32), ("chunk", ctypes.c_int32), ("causal", ctypes.c_int32),
+        ("inner", ctypes.c_int32), ("loss", ctypes.c_int32), ("opt", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("flags", ctypes.c_uint32), ("eta_scalar", ctypes.c_float), ("lr", ctypes.c_float),
+        ("momentum", ctypes.c_float), ("ns_iters", ctypes.c_int32), ("ns_coeff", ctypes.c_float * 3),
+        ("in_eps", ctypes.c_float),
+    ]
+
+
+class TTTError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"CUDA library {_LIB_PATH} is missing: build it with weight_sequence_mixing_b200.build")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    cfgp = ctypes.POINTER(TTTConfig)
+    sig = {
+        "ttt_config_init": (None, [cfgp]),
+        "ttt_create": (i32, [cfgp, ctypes.POINTER(vp)]),
+        "ttt_param_count": (i64, [vp]),
+        "ttt_workspace_size": (sz, [vp]),
+        "ttt_forward": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "ttt_host_staging_size": (sz, [vp]),
+        "ttt_forward_host": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, sz, vp]),
+        "ttt_query_status": (i32, [vp, vp, vp]),
+        "ttt_destroy": (None, [vp]),
+        "ttt_status_string": (ctypes.c_char_p, [i32]),
+        "ttt_selftest_gemm": (i32, [i32] * 9 + [vp, vp, vp, vp]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+LIB = _load()
+
+
+def status_string(status: int) -> str:
+    return LIB.ttt_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != TTT_OK:
+        raise TTTError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def make_config(cfg: dict) -> TTTConfig:
+    """C config from a workload dict (see synth_inputs.make_config for the keys)."""
+    c = TTTConfig()
+    LIB.ttt_config_init(ctypes.byref(c))
+    c.B, c.H, c.N, c.Nq = cfg["B"], cfg["H"], cfg["N"], cfg["Nq"]
+    c.d, c.h = cfg["d"], cfg["h"]
+    c.chunk, c.causal = int(cfg["chunk"] or 0), int(cfg["causal"])
+    c.inner, c.loss, c.opt = INNER[cfg["inner"]], LOSS[cfg["loss"]], OPT[cfg["opt"]]
+    c.dtype = DTYPE[cfg["dtype"]]
+    c.flags = (FLAG_KEY_INSTNORM if cfg["key_instnorm"] else 0) | (FLAG_WEIGHT_L2NORM if cfg["weight_l2norm"] else 0)
+    c.eta_scalar = float(cfg["eta_scalar"])
+    c.lr = float(cfg["lr"])
+    c.momentum = float(cfg["momentum"])
+    c.ns_iters = int(cfg["ns_iters"])
+    for i in range(3):
+        c.ns_coeff[i] = float(cfg["ns_coeff"][i])
+    c.in_eps = float(cfg["in_eps"])
+    return c
+
+
+@dataclass
+class TTTLayer:
+    """One configured TTT layer: a C handle plus its device workspace."""
+    cfg: dict
+    device: str = "cuda"
+    _handle: ctypes.c_void_p = field(default=None, repr=False)
+    workspace: torch.Tensor = field(default=None, repr=False)
+
+    def __post_init__(self):
+        self._c = make_config(self.cfg)
+        h = ctypes.c_void_p()
+        _check(LIB.ttt_create(ctypes.byref(self._c), ctypes.byref(h)), "ttt_create")
+        self._handle = h
+        self.P = int(LIB.ttt_param_count(h))
+        ws = int(LIB.ttt_workspace_size(h))
+        self.workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=self.device)
+
+    def close(self):
+        if self._handle:
+            LIB.ttt_destroy(self._handle)
+            self._handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def io_dtype(self):
+        return torch.float32 if self.cfg["dtype"] == "f32" else torch.bfloat16
+
+    def forward(self, Q, K, V, eta, W0, O=None, W_out=None, stream=None, check=True):
+        """Enqueue the layer on `stream`; returns (O, W_out).  With check=True the
+        stream is synchronised and the device status word is checked."""
+        c = self.cfg
+        if O is None:
+            O = torch.empty((c["B"], c["H"], c["Nq"], c["d"]), dtype=self.io_dtype, device=self.device)
+        if W_out is None:
+            W_out = torch.empty((c["B"], c["H"], self.P), dtype=torch.float32, device=self.device)
+        for t in (Q, K, V, W0, O, W_out) + ((eta,) if eta is not None else ()):
+            if not t.is_contiguous() or t.device.type != "cuda":
+                raise ValueError("tensors must be contiguous CUDA tensors")
+        st = _stream_ptr(stream)
+        _check(LIB.ttt_forward(self._handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W0), _ptr(O), _ptr(W_out),
+                               _ptr(self.workspace), self.workspace.numel(), st), "ttt_forward")
+        if check:
+            self.check_status(stream)
+        return O, W_out
+
+    def check_status(self, stream=None):
+        _check(LIB.ttt_query_status(self._handle, _ptr(self.workspace), _stream_ptr(stream)), "device status")
+
+    # ---- host-buffer entry point (copies inside the library call)
+    def staging(self):
+        n = int(LIB.ttt_host_staging_size(self._handle))
+        return torch.empty(max(n, 256), dtype=torch.uint8, device=self.device)
+
+    def forward_host(self, Q, K, V, eta, W0, O, W_out, staging, stream=None):
+        """Host (ideally pinned) CPU tensors in and out; enqueued on `stream`."""
+        st = _stream_ptr(stream)
+        _check(LIB.ttt_forward_host(self._handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W0), _ptr(O),
+                                    _ptr(W_out), _ptr(staging), staging.numel(), _ptr(self.workspace),
+                                    self.workspace.numel(), st), "ttt_forward_host")
+
+
+def selftest_gemm(A, B, elem_bytes, a_mn, b_mn, bn, M, N, K, batches, splits, stream=None):
+    """Diagnostic: C[s][z] = A[z] B[z]^T through the tcgen05 engine (see ttt_diag.h)."""
+    C = torch.full((splits, batches, M, N), float("nan"), dtype=torch.float32, device=A.device)
+    _check(LIB.ttt_selftest_gemm(elem_bytes, int(a_mn), int(b_mn), bn, M, N, K, batches, splits, _ptr(A), _ptr(B),
+                                 _ptr(C), _stream_ptr(stream)), "ttt_selftest_gemm")
+    return C

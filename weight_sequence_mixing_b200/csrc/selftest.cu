@@ -1,0 +1,86 @@
+// Diagnostic entry point: one plain tcgen05 GEMM through the same engine the
+// TTT path uses, so the operand layouts (K-major / MN-major, bf16 / tf32),
+// ragged edges, batching and split-K can be checked against a library matmul.
+#include "../../include/ttt_diag.h"
+#include "tc_gemm.cuh"
+
+namespace ttt {
+namespace {
+
+struct EpiStorePartial {
+  float* out;  // [splits][batches][M][N]
+  int M, N, batches;
+  template <int BN0, int BN1>
+  __device__ void run(const EpiCtx& c) const {
+    float* rowp = out + ((static_cast<int64_t>(c.split) * batches + c.z) * M + c.m) * N;
+#pragma unroll 1
+    for (int cc = 0; cc < BN0; cc += 32) {
+      float v[32];
+      tmem_ld32(c.taddr + cc, v);
+      if (c.m < M) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c.n0 + cc + j < N) rowp[c.n0 + cc + j] = v[j];
+      }
+    }
+  }
+};
+
+template <int BN, bool AMN, bool BMN, int EB>
+int run_one(const void* A, const void* B, float* C, int M, int N, int K, int batches, int splits,
+            cudaStream_t st) {
+  CUtensorMap ta, tb;
+  const int run = 128 / EB;
+  // A: K-major [batch][M][K]; MN-major [batch][K][M].  Same for B with N.
+  bool ok = AMN ? make_tmap(&ta, A, EB, M, K, batches, M, static_cast<int64_t>(M) * K, run)
+                : make_tmap(&ta, A, EB, K, M, batches, K, static_cast<int64_t>(M) * K, 128);
+  ok = ok && (BMN ? make_tmap(&tb, B, EB, N, K, batches, N, static_cast<int64_t>(N) * K, run)
+                  : make_tmap(&tb, B, EB, K, N, batches, K, static_cast<int64_t>(N) * K, BN));
+  if (!ok) return TTT_ERR_INVALID_ARG;
+  TcGeom g;
+  g.m_tiles0 = (M + 127) / 128;
+  g.n_tiles = (N + BN - 1) / BN;
+  g.M0 = M;
+  g.N = N;
+  g.kblocks = (K + run - 1) / run;
+  g.batches = batches;
+  g.kb_per_split = (g.kblocks + splits - 1) / splits;
+  g.splits = (g.kblocks + g.kb_per_split - 1) / g.kb_per_split;
+  if (g.splits != splits) return TTT_ERR_INVALID_ARG;  // every split must own at least one k-block
+  EpiStorePartial epi{C, M, N, batches};
+  cudaError_t e = launch_tc_gemm<BN, 0, AMN, BMN, EB, 4>(ta, tb, ta, tb, g, epi, nullptr, st);
+  return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+
+template <int BN, int EB>
+int dispatch_major(int a_mn, int b_mn, const void* A, const void* B, float* C, int M, int N, int K, int batches,
+                   int splits, cudaStream_t st) {
+  if constexpr (EB == 4) {
+    if (a_mn || b_mn) return TTT_ERR_UNSUPPORTED;
+    return run_one<BN, false, false, EB>(A, B, C, M, N, K, batches, splits, st);
+  } else {
+  if (!a_mn && !b_mn) return run_one<BN, false, false, EB>(A, B, C, M, N, K, batches, splits, st);
+  if (!a_mn && b_mn) return run_one<BN, false, true, EB>(A, B, C, M, N, K, batches, splits, st);
+  if (a_mn && !b_mn) return run_one<BN, true, false, EB>(A, B, C, M, N, K, batches, splits, st);
+  return run_one<BN, true, true, EB>(A, B, C, M, N, K, batches, splits, st);
+  }
+}
+
+}  // namespace
+}  // namespace ttt
+
+extern "C" int ttt_selftest_gemm(int elem_bytes, int a_mn, int b_mn, int bn, int M, int N, int K, int batches,
+                                 int splits, const void* A, const void* B, float* C, void* stream) {
+  using namespace ttt;
+  if (!A || !B || !C || M <= 0 || N <= 0 || K <= 0 || batches <= 0 || splits <= 0) return TTT_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (elem_bytes == 2) {
+    if (bn == 64) return dispatch_major<64, 2>(a_mn, b_mn, A, B, C, M, N, K, batches, splits, st);
+    if (bn == 128) return dispatch_major<128, 2>(a_mn, b_mn, A, B, C, M, N, K, batches, splits, st);
+    if (bn == 256) return dispatch_major<256, 2>(a_mn, b_mn, A, B, C, M, N, K, batches, splits, st);
+  } else if (elem_bytes == 4) {
+    if (bn == 128) return dispatch_major<128, 4>(a_mn, b_mn, A, B, C, M, N, K, batches, splits, st);
+    if (bn == 256) return dispatch_major<256, 4>(a_mn, b_mn, A, B, C, M, N, K, batches, splits, st);
+  }
+  return TTT_ERR_UNSUPPORTED;
+}

@@ -1,0 +1,127 @@
+// C ABI of the TTT-layer forward pass: argument validation, workspace sizing,
+// the device status word and the host-buffer wrapper.  The forward pass itself
+// is planned and enqueued by the path selected in ttt_path.cuh.
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "../../include/ttt.h"
+#include "ttt_plan.cuh"
+
+using namespace ttt;
+
+extern "C" void ttt_config_init(ttt_config* c) {
+  if (!c) return;
+  std::memset(c, 0, sizeof(*c));
+  c->chunk = 0;
+  c->inner = TTT_INNER_MLP2_GELU;
+  c->loss = TTT_LOSS_MSE;
+  c->opt = TTT_OPT_GD;
+  c->dtype = TTT_BF16;
+  c->eta_scalar = 1.0f;
+  c->lr = 1.0f;
+  c->momentum = 0.9f;
+  c->ns_iters = 5;
+  c->ns_coeff[0] = 3.4445f;
+  c->ns_coeff[1] = -4.7750f;
+  c->ns_coeff[2] = 2.0315f;
+  c->in_eps = 1e-5f;
+}
+
+extern "C" int ttt_create(const ttt_config* cfg, ttt_handle** out) {
+  if (!out) return TTT_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!cfg) return TTT_ERR_INVALID_ARG;
+  Plan plan;
+  int st = plan_build(*cfg, &plan);
+  if (st != TTT_OK) return st;
+  ttt_handle* h = new (std::nothrow) ttt_handle;
+  if (!h) return TTT_ERR_INVALID_ARG;
+  h->plan = plan;
+  *out = h;
+  return TTT_OK;
+}
+
+extern "C" int64_t ttt_param_count(const ttt_handle* h) { return h ? h->plan.P : 0; }
+
+extern "C" size_t ttt_workspace_size(const ttt_handle* h) { return h ? h->plan.ws_bytes : 0; }
+
+extern "C" int ttt_forward(ttt_handle* h, const void* Q, const void* K, const void* V, const float* eta,
+                           const float* W0, void* O, float* W_out, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  if (!h || !Q || !K || !V || !W0 || !O) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {Q, K, V, eta, W0, O, W_out};
+  for (const void* p : ptrs)
+    if (p && (reinterpret_cast<uintptr_t>(p) & 15) != 0) return TTT_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) != 0 || workspace_bytes < h->plan.ws_bytes)
+    return TTT_ERR_WORKSPACE;
+  Io io{Q, K, V, eta, W0, O, W_out};
+  return plan_run(h->plan, io, workspace, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" size_t ttt_host_staging_size(const ttt_handle* h) { return h ? h->plan.staging_bytes : 0; }
+
+extern "C" int ttt_forward_host(ttt_handle* h, const void* Q, const void* K, const void* V, const float* eta,
+                                const float* W0, void* O, float* W_out, void* staging, size_t staging_bytes,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  if (!h || !Q || !K || !V || !W0 || !O) return TTT_ERR_INVALID_ARG;
+  const Plan& p = h->plan;
+  if (!staging || (reinterpret_cast<uintptr_t>(staging) & 255) != 0 || staging_bytes < p.staging_bytes)
+    return TTT_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(staging);
+  void* dQ = base + p.stg_q;
+  void* dK = base + p.stg_k;
+  void* dV = base + p.stg_v;
+  float* dEta = eta ? reinterpret_cast<float*>(base + p.stg_eta) : nullptr;
+  float* dW0 = reinterpret_cast<float*>(base + p.stg_w0);
+  void* dO = base + p.stg_o;
+  float* dW = W_out ? reinterpret_cast<float*>(base + p.stg_w) : nullptr;
+  const size_t es = p.cfg.dtype == TTT_F32 ? 4 : 2;
+  const size_t nq = static_cast<size_t>(p.cfg.B) * p.cfg.H * p.cfg.Nq * p.cfg.d * es;
+  const size_t nk = static_cast<size_t>(p.cfg.B) * p.cfg.H * p.cfg.N * p.cfg.d * es;
+  const size_t ne = static_cast<size_t>(p.cfg.B) * p.cfg.H * p.cfg.N * 4;
+  const size_t nw0 = static_cast<size_t>(p.cfg.H) * p.P * 4;
+  const size_t nw = static_cast<size_t>(p.cfg.B) * p.cfg.H * p.P * 4;
+  if (cudaMemcpyAsync(dQ, Q, nq, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(dK, K, nk, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(dV, V, nk, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      (eta && cudaMemcpyAsync(dEta, eta, ne, cudaMemcpyHostToDevice, st) != cudaSuccess) ||
+      cudaMemcpyAsync(dW0, W0, nw0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return TTT_ERR_CUDA;
+  int r = ttt_forward(h, dQ, dK, dV, dEta, dW0, dO, dW, workspace, workspace_bytes, stream);
+  if (r != TTT_OK) return r;
+  if (cudaMemcpyAsync(O, dO, nq, cudaMemcpyDeviceToHost, st) != cudaSuccess) return TTT_ERR_CUDA;
+  if (W_out && cudaMemcpyAsync(W_out, dW, nw, cudaMemcpyDeviceToHost, st) != cudaSuccess) return TTT_ERR_CUDA;
+  return TTT_OK;
+}
+
+extern "C" int ttt_query_status(ttt_handle* h, void* workspace, void* stream) {
+  if (!h || !workspace) return TTT_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return TTT_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return TTT_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, sizeof(unsigned), st) != cudaSuccess) return TTT_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return TTT_ERR_CUDA;
+  if (word & kStatusTimeout) return TTT_ERR_TIMEOUT;
+  if (word & kStatusBadLaunch) return TTT_ERR_CUDA;
+  if (word & kStatusNonFinite) return TTT_ERR_NONFINITE;
+  return TTT_OK;
+}
+
+extern "C" void ttt_destroy(ttt_handle* h) { delete h; }
+
+extern "C" const char* ttt_status_string(int s) {
+  switch (s) {
+    case TTT_OK: return "ok";
+    case TTT_ERR_INVALID_ARG: return "invalid argument";
+    case TTT_ERR_UNSUPPORTED: return "unsupported configuration";
+    case TTT_ERR_CUDA: return "CUDA error";
+    case TTT_ERR_NONFINITE: return "non-finite values in the outputs";
+    case TTT_ERR_TIMEOUT: return "a bounded device wait ran out";
+    case TTT_ERR_WORKSPACE: return "workspace too small or misaligned";
+    default: return "unknown status";
+  }
+}

@@ -1,0 +1,59 @@
+// Validation, chunking and workspace carving of a TTT layer configuration.
+#include <cmath>
+
+#include "ttt_plan.cuh"
+
+namespace ttt {
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int plan_build(const ttt_config& c, Plan* p) {
+  if (c.B < 1 || c.H < 1 || c.N < 1 || c.Nq < 1 || c.d < 1) return TTT_ERR_INVALID_ARG;
+  if (c.inner < TTT_INNER_LINEAR || c.inner > TTT_INNER_SWIGLU) return TTT_ERR_INVALID_ARG;
+  if (c.loss < TTT_LOSS_MSE || c.loss > TTT_LOSS_NEG_DOT) return TTT_ERR_INVALID_ARG;
+  if (c.opt < TTT_OPT_GD || c.opt > TTT_OPT_MOMENTUM_MUON) return TTT_ERR_INVALID_ARG;
+  if (c.dtype != TTT_F32 && c.dtype != TTT_BF16) return TTT_ERR_INVALID_ARG;
+  if (c.causal != 0 && c.causal != 1) return TTT_ERR_INVALID_ARG;
+  if (c.causal && c.Nq != c.N) return TTT_ERR_INVALID_ARG;
+  if (c.inner != TTT_INNER_LINEAR && c.h < 1) return TTT_ERR_INVALID_ARG;
+  if ((c.flags & ~(TTT_FLAG_KEY_INSTNORM | TTT_FLAG_WEIGHT_L2NORM)) != 0) return TTT_ERR_INVALID_ARG;
+  if (c.ns_iters < 0 || c.ns_iters > 100) return TTT_ERR_INVALID_ARG;
+  if (!std::isfinite(c.eta_scalar) || !std::isfinite(c.lr) || !std::isfinite(c.momentum) ||
+      !std::isfinite(c.in_eps) || c.in_eps < 0.0f)
+    return TTT_ERR_INVALID_ARG;
+  for (float v : c.ns_coeff)
+    if (!std::isfinite(v)) return TTT_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(c.B) * c.H > 65535) return TTT_ERR_UNSUPPORTED;
+  if (c.d > 4096 || c.h > 16384) return TTT_ERR_UNSUPPORTED;
+
+  p->cfg = c;
+  const int64_t d = c.d, h = c.inner == TTT_INNER_LINEAR ? c.d : c.h;
+  p->cfg.h = static_cast<int32_t>(h);
+  p->P = c.inner == TTT_INNER_LINEAR ? d * d : c.inner == TTT_INNER_MLP2_GELU ? 2 * d * h : 3 * d * h;
+  p->BH = c.B * c.H;
+  p->chunk = (c.chunk <= 0 || c.chunk >= c.N) ? c.N : c.chunk;
+  p->nchunks = (c.N + p->chunk - 1) / p->chunk;
+  p->path = c.dtype == TTT_F32 ? kPathF32 : kPathBf16;
+
+  // host staging: inputs then outputs, each 256-byte aligned
+  const size_t es = c.dtype == TTT_F32 ? 4 : 2;
+  size_t o = 0;
+  p->stg_q = o; o = align_up(o + size_t(p->BH) * c.Nq * d * es, 256);
+  p->stg_k = o; o = align_up(o + size_t(p->BH) * c.N * d * es, 256);
+  p->stg_v = o; o = align_up(o + size_t(p->BH) * c.N * d * es, 256);
+  p->stg_eta = o; o = align_up(o + size_t(p->BH) * c.N * 4, 256);
+  p->stg_w0 = o; o = align_up(o + size_t(c.H) * p->P * 4, 256);
+  p->stg_o = o; o = align_up(o + size_t(p->BH) * c.Nq * d * es, 256);
+  p->stg_w = o; o = align_up(o + size_t(p->BH) * p->P * 4, 256);
+  p->staging_bytes = o;
+
+  int st = p->path == kPathF32 ? plan_layout_f32(p) : plan_layout_bf16(p);
+  return st;
+}
+
+int plan_run(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
+  if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return TTT_ERR_CUDA;  // status word
+  return p.path == kPathF32 ? run_f32(p, io, ws, st) : run_bf16(p, io, ws, st);
+}
+
+}  // namespace ttt

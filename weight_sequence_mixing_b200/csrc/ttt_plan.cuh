@@ -1,0 +1,51 @@
+// Host-side plan of one configured TTT layer: validated sizes, chunking,
+// which device path runs it, and the carving of the caller's workspace.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/ttt.h"
+#include "ptx.cuh"
+
+namespace ttt {
+
+struct Io {
+  const void* Q;
+  const void* K;
+  const void* V;
+  const float* eta;
+  const float* W0;
+  void* O;
+  float* W_out;
+};
+
+enum PathKind : int { kPathF32 = 0, kPathBf16 = 1 };
+
+struct Plan {
+  ttt_config cfg{};
+  int64_t P = 0;       // fast-weight floats per head
+  int BH = 0;          // B * H
+  int chunk = 0;       // tokens per chunk (== N for one chunk)
+  int nchunks = 0;
+  int path = kPathF32;
+  size_t ws_bytes = 0;
+  // host-staging layout (ttt_forward_host)
+  size_t staging_bytes = 0, stg_q = 0, stg_k = 0, stg_v = 0, stg_eta = 0, stg_w0 = 0, stg_o = 0, stg_w = 0;
+  // workspace layout: byte offsets into the caller's workspace
+  size_t off[32] = {};
+};
+
+int plan_build(const ttt_config& cfg, Plan* plan);
+int plan_run(const Plan& plan, const Io& io, void* workspace, cudaStream_t st);
+
+// per-path workspace layout and launch sequence
+int plan_layout_f32(Plan* plan);
+int plan_layout_bf16(Plan* plan);
+int run_f32(const Plan& plan, const Io& io, void* workspace, cudaStream_t st);
+int run_bf16(const Plan& plan, const Io& io, void* workspace, cudaStream_t st);
+
+}  // namespace ttt
+
+struct ttt_handle {
+  ttt::Plan plan;
+};
