@@ -1,0 +1,101 @@
+"""bf16 tensor-core CUDA path against the fp64 oracle.
+
+Gate: relative Frobenius error <= 2e-2 per output and per final weight matrix
+(the bf16-input / fp32-accumulate bound of the layer's target).  The change
+of the weights, W* - W0, is also compared (a looser diagnostic bound), since a
+small update hides inside W* when ||W* - W0|| << ||W0||.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from synth_inputs import gen_inputs, make_config, matrix_shapes, workload
+from tests.parity_util import compare, rel_fro, run_gpu
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-2
+DW_TOL = 5e-2
+
+
+def _check(errs, tol=TOL):
+    for k, v in errs.items():
+        assert v <= tol, f"{k}: relative Frobenius error {v:.3e} > {tol}"
+
+
+def _delta_w_check(cfg, x, heads=None):
+    Og, Wg = run_gpu(cfg, x)
+    Or, Wr = orc.forward(cfg, x["Q"], x["K"], x["V"], x["eta"], x["W0"], heads=heads)
+    sel = heads or [(b, h) for b in range(cfg["B"]) for h in range(cfg["H"])]
+    W0 = x["W0"].double().numpy()
+    out = {"O": max(rel_fro(Og[b, h], Or[b, h]) for b, h in sel)}
+    off = 0
+    for name, r, c in matrix_shapes(cfg):
+        sl = slice(off, off + r * c)
+        out[name] = max(rel_fro(Wg[b, h, sl], Wr[b, h, sl]) for b, h in sel)
+        if not cfg["weight_l2norm"]:
+            out["d" + name] = max(rel_fro(Wg[b, h, sl] - W0[h, sl], Wr[b, h, sl] - W0[h, sl]) for b, h in sel)
+        off += r * c
+    return out
+
+
+SMALL = [
+    dict(inner="swiglu", loss="neg_dot", opt="gd", d=128, h=256, N=300),
+    dict(inner="swiglu", loss="neg_dot", opt="momentum", d=128, h=128, N=450, chunk=128, causal=1, weight_l2norm=True),
+    dict(inner="swiglu", loss="neg_dot", opt="muon", d=128, h=256, N=384, weight_l2norm=True),
+    dict(inner="swiglu", loss="neg_dot", opt="momentum_muon", d=128, h=256, N=700, chunk=256, Nq=200,
+         weight_l2norm=True),
+    dict(inner="swiglu", loss="neg_dot", opt="gd", d=256, h=512, N=520, Nq=130, eta_mode="scalar",
+         eta_scalar=0.002),
+    dict(inner="mlp2_gelu", loss="mse", opt="gd", d=64, h=256, N=700, key_instnorm=True, data="vit",
+         eta_mode="scalar", eta_scalar=1.0),
+    dict(inner="mlp2_gelu", loss="mse", opt="momentum", d=64, h=128, N=333, chunk=128, key_instnorm=True,
+         data="vit", eta_mode="scalar"),
+    dict(inner="mlp2_gelu", loss="neg_dot", opt="momentum", d=128, h=256, N=400, chunk=256, weight_l2norm=True),
+    dict(inner="linear", loss="neg_dot", opt="gd", d=128, h=128, N=260),
+    dict(inner="linear", loss="mse", opt="momentum_muon", d=128, h=128, N=390, chunk=128, weight_l2norm=True),
+]
+
+
+@pytest.mark.parametrize("kw", SMALL, ids=lambda kw: "-".join(f"{v}" for v in kw.values()))
+def test_small_bf16_variants(kw):
+    base = dict(B=2, H=2, dtype="bf16", data="lact", eta_mode="per_token", seed=91)
+    base.update(kw)
+    cfg = make_config(**base)
+    errs = _delta_w_check(cfg, gen_inputs(cfg))
+    for k, v in errs.items():
+        tol = DW_TOL if k.startswith("d") else TOL
+        assert v <= tol, f"{k}: relative Frobenius error {v:.3e} > {tol}"
+
+
+def test_causal_chunk_n_equals_single_chunk_weights_on_gpu():
+    # apply-before-update with one chunk: W* equals the non-causal single chunk's,
+    # and O reads the initial weights (the non-causal eta = 0 output).
+    kw = dict(B=1, H=2, N=256, d=128, h=128, inner="swiglu", loss="neg_dot", opt="momentum", dtype="bf16",
+              weight_l2norm=False, data="lact", eta_mode="per_token", seed=5)
+    x = gen_inputs(make_config(**kw))
+    Oc, Wc = run_gpu(make_config(chunk=256, causal=1, **kw), x)
+    On, Wn = run_gpu(make_config(chunk=0, causal=0, **kw), x)
+    assert rel_fro(Wc, Wn) < 1e-6
+    x0 = dict(x)
+    x0["eta"] = torch.zeros_like(x["eta"])
+    O0, _ = run_gpu(make_config(chunk=0, causal=0, **kw), x0)
+    assert rel_fro(Oc, O0) < 1e-6
+
+
+# ---------------------------------------------------------------- full-size workloads
+FULL = {
+    "vit3s_1248_mlp2_n6084": None,
+    "lact_lm_causal_n32k_c2048": None,
+    "lact_nvs_n196k_d512": None,
+    "lact_scene_n1m_c131k": [(0, 0), (0, 3)],
+}
+
+
+@pytest.mark.parametrize("name", list(FULL))
+def test_full_size_workload(name):
+    cfg = workload(name)
+    heads = FULL[name]
+    errs = compare(cfg, heads=heads)
+    print(name, {k: f"{v:.2e}" for k, v in errs.items()})
+    _check(errs)

@@ -1,0 +1,377 @@
+// Fused epilogues of the tcgen05 GEMMs of the bf16 TTT path.
+//
+// Each functor runs on the 4 epilogue warps of a CTA with one output row per
+// thread (TMEM lane = tile row) and reads its accumulators 32 columns at a time
+// with tcgen05.ld (a warp-collective: every thread of the warp executes every
+// load, rows outside the problem only skip their stores).
+#pragma once
+#include <cuda_bf16.h>
+
+#include "tc_gemm.cuh"
+
+namespace ttt {
+
+using bf16 = __nv_bfloat16;
+
+// ------------------------------------------------------------------ helpers
+__device__ __forceinline__ float gelu_dev(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+__device__ __forceinline__ float gelu_grad_dev(float x) {
+  return 0.5f * (1.0f + erff(x * 0.70710678118654752f)) + x * 0.39894228040143268f * __expf(-0.5f * x * x);
+}
+__device__ __forceinline__ float sigmoid_dev(float x) { return 1.0f / (1.0f + __expf(-x)); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// 32 floats -> 32 bf16 at a 16-byte aligned address
+__device__ __forceinline__ void store_bf16x32(bf16* dst, const float (&v)[32]) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 u;
+    u.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    u.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    u.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    u.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    d4[q] = u;
+  }
+}
+
+__device__ __forceinline__ void load_bf16x32(const bf16* src, float (&v)[32]) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 u = s4[q];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      __nv_bfloat162 p = *reinterpret_cast<const __nv_bfloat162*>(&w[j]);
+      float2 f = __bfloat1622float2(p);
+      v[8 * q + 2 * j] = f.x;
+      v[8 * q + 2 * j + 1] = f.y;
+    }
+  }
+}
+
+__device__ __forceinline__ void store_f32x32(float* dst, const float (&v)[32]) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+__device__ __forceinline__ void load_f32x32(const float* src, float (&v)[32]) {
+  const float4* s4 = reinterpret_cast<const float4*>(src);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    float4 f = s4[q];
+    v[4 * q] = f.x;
+    v[4 * q + 1] = f.y;
+    v[4 * q + 2] = f.z;
+    v[4 * q + 3] = f.w;
+  }
+}
+
+__device__ __forceinline__ void zero32(float (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+}
+
+// ------------------------------------------------------------------ split-K partials
+// out[split][z][row0_p + m][n] (fp32), rows_p valid rows of problem p; N columns.
+struct EpiPartial {
+  float* out;
+  int64_t split_stride, z_stride;  // elements
+  int ld;                          // row length (= N)
+  int row0[2], rows[2];
+  template <int BN0, int BN1>
+  __device__ void run(const EpiCtx& c) const {
+    const bool ok = c.m < rows[c.problem];
+    float* rowp = out + c.split * split_stride + c.z * z_stride + int64_t(row0[c.problem] + c.m) * ld + c.n0;
+#pragma unroll 1
+    for (int cc = 0; cc < BN0; cc += 32) {
+      float v[32];
+      tmem_ld32(c.taddr + cc, v);
+      if (ok && c.n0 + cc < ld) store_f32x32(rowp + cc, v);
+    }
+  }
+};
+
+// ------------------------------------------------------------------ token phase, dot loss
+// Two products per 128-token tile and 128-wide hidden block j0 = 128*tile_n:
+//   SwiGLU: D0 = X [W1_blk ; W3_blk]^T (256 cols: z1 | z3), D1 = V W2[:, blk] (128 cols: p)
+//   MLP2  : D0 = X W1_blk^T           (128 cols: z),       D1 = V W2[:, blk] (128 cols: p)
+// With dL/dV_hat_t = -eta_t v_t (negative dot loss, LaCT analysis "Nonlinear memory"):
+//   dH = -eta_t p.  SwiGLU: H' = -eta_t SiLU(z1) z3, dZ3 = dH SiLU(z1), dZ1 = dH z3 SiLU'(z1).
+//   MLP2  : H' = -eta_t GELU(z), dZ = dH GELU'(z).
+// H' (so that the W2 gradient is V^T H') goes to Hp [z][t][h]; dZ1/dZ3 to dZ
+// [z][t][2h] blocked as [blk][dZ1 128 | dZ3 128] (SwiGLU) or dZ [z][t][h] (MLP2).
+// Rows t >= rows_valid (past the chunk's last token) are written as zeros.
+template <bool SWIGLU>
+struct EpiTokenDot {
+  bf16* Hp;
+  bf16* dZ;
+  int h;                 // hidden width
+  int rows_valid;        // tokens in the chunk
+  int64_t hp_zs, dz_zs;  // per-z strides (elements)
+  const float* eta;      // [z][N] or null
+  int64_t eta_zs;
+  int t0;                // chunk's first token (eta index)
+  float eta_scalar;
+  template <int BN0, int BN1>
+  __device__ void run(const EpiCtx& c) const {
+    const bool valid = c.m < rows_valid;
+    const float e = valid ? (eta ? eta[c.z * eta_zs + t0 + c.m] : eta_scalar) : 0.0f;
+    const int blk = c.n0 / BN0;
+    bf16* hrow = Hp + c.z * hp_zs + int64_t(c.m) * h + blk * 128;
+    bf16* drow = dZ + c.z * dz_zs + int64_t(c.m) * (SWIGLU ? 2 * h : h) + blk * (SWIGLU ? 256 : 128);
+#pragma unroll 1
+    for (int cc = 0; cc < 128; cc += 32) {
+      float z1[32], z3[32], p[32];
+      tmem_ld32(c.taddr + cc, z1);
+      if constexpr (SWIGLU) tmem_ld32(c.taddr + 128 + cc, z3);
+      tmem_ld32(c.taddr + BN0 + cc, p);
+      float hv[32], d1[32], d3[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float dh = -e * p[j];
+        if constexpr (SWIGLU) {
+          const float s = sigmoid_dev(z1[j]);
+          const float a = z1[j] * s;
+          hv[j] = -e * a * z3[j];
+          d3[j] = dh * a;
+          d1[j] = dh * z3[j] * s * (1.0f + z1[j] * (1.0f - s));
+        } else {
+          hv[j] = -e * gelu_dev(z1[j]);
+          d1[j] = dh * gelu_grad_dev(z1[j]);
+          d3[j] = 0.0f;
+        }
+      }
+      store_bf16x32(hrow + cc, hv);
+      store_bf16x32(drow + cc, d1);
+      if constexpr (SWIGLU) store_bf16x32(drow + 128 + cc, d3);
+    }
+  }
+};
+
+// ------------------------------------------------------------------ token phase, MSE (MLP2)
+// Z = X W1^T tile: H = GELU(Z) and G' = GELU'(Z) (bf16), zeros past the chunk.
+struct EpiGeluSave {
+  bf16* H;
+  bf16* Gp;
+  int ld;  // h
+  int rows_valid;
+  int64_t zs;
+  template <int BN0, int BN1>
+  __device__ void run(const EpiCtx& c) const {
+    const bool valid = c.m < rows_valid;
+    bf16* hrow = H + c.z * zs + int64_t(c.m) * ld + c.n0;
+    bf16* grow = Gp + c.z * zs + int64_t(c.m) * ld + c.n0;
+#pragma unroll 1
+    for (int cc = 0; cc < BN0; cc += 32) {
+      float v[32], a[32], g[32];
+      tmem_ld32(c.taddr + cc, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        a[j] = valid ? gelu_dev(v[j]) : 0.0f;
+        g[j] = valid ? gelu_grad_dev(v[j]) : 0.0f;
+      }
+      store_bf16x32(hrow + cc, a);
+      store_bf16x32(grow + cc, g);
+    }
+  }
+};
+
+// V_hat tile -> dL/dV_hat = coef * eta_t * (V_hat - V) (MSE, mean over the chunk's
+// n*d elements: coef = 2/(n d)); zeros past the chunk.
+struct EpiMseGrad {
+  bf16* dY;
+  int d;
+  int rows_valid;
+  int64_t zs;
+  const bf16* V;  // [z][N][d]
+  int64_t v_zs;
+  int t0;
+  const float* eta;
+  int64_t eta_zs;
+  float eta_scalar, coef;
+  template <int BN0, int BN1>
+  __device__ void run(const EpiCtx& c) const {
+    const bool valid = c.m < rows_valid;
+    const float e = valid ? (eta ? eta[c.z * eta_zs + t0 + c.m] : eta_scalar) * coef : 0.0f;
+    bf16* yrow = dY + c.z * zs + int64_t(c.m) * d + c.n0;
+    const bf16* vrow = V + c.z * v_zs + int64_t(t0 + (valid ? c.m : 0)) * d + c.n0;
+#pragma unroll 1
+    for (int cc = 0; cc < BN0; cc += 32) {
+      float v[32], t[32];
+      tmem_ld32(c.taddr + cc, v);
+      if (c.n0 + cc >= d) continue;
+      if (valid) load_bf16x32(vrow + cc, t);
+      else zero32(t);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = e * (v[j] - t[j]);
+      store_bf16x32(yrow + cc, v);
+    }
+  }
+};
+
+// dH tile -> dZ = dH * G' (G' saved by EpiGeluSave)
+struct EpiMulSaved {
+  bf16* dZ;
+  const bf16* Gp;
+  int ld;
+  int64_t zs;
+  template <int BN0, int BN1>
+  __device__ void run(const EpiCtx& c) const {
+    bf16* zrow = dZ + c.z * zs + int64_t(c.m) * ld + c.n0;
+    const bf16* grow = Gp + c.z * zs + int64_t(c.m) * ld + c.n0;
+#pragma unroll 1
+    for (int cc = 0; cc < BN0; cc += 32) {
+      float v[32], g[32];
+      tmem_ld32(c.taddr + cc, v);
+      load_bf16x32(grow + cc, g);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] *= g[j];
+      store_bf16x32(zrow + cc, v);
+    }
+  }
+};
+
+// ------------------------------------------------------------------ apply on queries
+// First layer of F_W(Q): SwiGLU tiles hold [z1 (128) | z3 (128)] of hidden block
+// n0/256 -> H = SiLU(z1) z3; MLP2 tiles hold z -> H = GELU(z).  Rows >= rows_valid skipped.
+template <bool SWIGLU>
+struct EpiApplyAct {
+  bf16* Hq;
+  int h;
+  int rows_valid;
+  int64_t zs;
+  template <int BN0, int BN1>
+  __device__ void run(const EpiCtx& c) const {
+    const bool valid = c.m < rows_valid;
+    if constexpr (SWIGLU) {
+      bf16* row = Hq + c.z * zs + int64_t(c.m) * h + (c.n0 / BN0) * 128;
+#pragma unroll 1
+      for (int cc = 0; cc < 128; cc += 32) {
+        float z1[32], z3[32];
+        tmem_ld32(c.taddr + cc, z1);
+        tmem_ld32(c.taddr + 128 + cc, z3);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) z1[j] = z1[j] * sigmoid_dev(z1[j]) * z3[j];
+        if (valid) store_bf16x32(row + cc, z1);
+      }
+    } else {
+      bf16* row = Hq + c.z * zs + int64_t(c.m) * h + c.n0;
+#pragma unroll 1
+      for (int cc = 0; cc < BN0; cc += 32) {
+        float z[32];
+        tmem_ld32(c.taddr + cc, z);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) z[j] = gelu_dev(z[j]);
+        if (valid && c.n0 + cc < h) store_bf16x32(row + cc, z);
+      }
+    }
+  }
+};
+
+// Output rows of O (row0 + m for m < rows_valid), bf16 or fp32, with the
+// non-finite check of the layer's output.
+template <typename OutT>
+struct EpiStoreOut {
+  OutT* O;
+  int d;
+  int rows_valid, row0;
+  int64_t zs;
+  unsigned* status;
+  template <int BN0, int BN1>
+  __device__ void run(const EpiCtx& c) const {
+    const bool valid = c.m < rows_valid;
+    OutT* row = O + c.z * zs + int64_t(row0 + c.m) * d + c.n0;
+    bool bad = false;
+#pragma unroll 1
+    for (int cc = 0; cc < BN0; cc += 32) {
+      float v[32];
+      tmem_ld32(c.taddr + cc, v);
+      if (!valid || c.n0 + cc >= d) continue;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) bad |= !isfinite(v[j]);
+      if constexpr (sizeof(OutT) == 2) store_bf16x32(reinterpret_cast<bf16*>(row + cc), v);
+      else store_f32x32(reinterpret_cast<float*>(row + cc), v);
+    }
+    if (bad) set_status(status, kStatusNonFinite);
+  }
+};
+
+// ------------------------------------------------------------------ Newton-Schulz (fp32 / tf32)
+// S = X X^T
+struct EpiStoreF32 {
+  float* out;
+  int ld, rows;
+  int64_t zs;
+  template <int BN0, int BN1>
+  __device__ void run(const EpiCtx& c) const {
+    float* row = out + c.z * zs + int64_t(c.m) * ld + c.n0;
+#pragma unroll 1
+    for (int cc = 0; cc < BN0; cc += 32) {
+      float v[32];
+      tmem_ld32(c.taddr + cc, v);
+      if (c.m < rows && c.n0 + cc < ld) store_f32x32(row + cc, v);
+    }
+  }
+};
+
+// T = b S + c (S S)
+struct EpiNsPoly {
+  float* T;
+  const float* S;
+  int ld, rows;
+  int64_t zs;
+  float b, cc_;
+  template <int BN0, int BN1>
+  __device__ void run(const EpiCtx& c) const {
+    float* trow = T + c.z * zs + int64_t(c.m) * ld + c.n0;
+    const float* srow = S + c.z * zs + int64_t(c.m) * ld + c.n0;
+#pragma unroll 1
+    for (int cc = 0; cc < BN0; cc += 32) {
+      float v[32], s[32];
+      tmem_ld32(c.taddr + cc, v);
+      if (c.m >= rows || c.n0 + cc >= ld) continue;
+      load_f32x32(srow + cc, s);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = b * s[j] + cc_ * v[j];
+      store_f32x32(trow + cc, v);
+    }
+  }
+};
+
+// X' = a X + T X, stored as X' [m][n] and X'^T [n][m]
+struct EpiNsUpdate {
+  float* Xn;
+  float* XnT;
+  const float* X;
+  int m, n;
+  int64_t zs;
+  float a;
+  template <int BN0, int BN1>
+  __device__ void run(const EpiCtx& c) const {
+    const bool valid = c.m < m;
+    float* row = Xn + c.z * zs + int64_t(c.m) * n + c.n0;
+    const float* xrow = X + c.z * zs + int64_t(c.m) * n + c.n0;
+    float* colT = XnT + c.z * zs + int64_t(c.n0) * m + c.m;
+#pragma unroll 1
+    for (int cc = 0; cc < BN0; cc += 32) {
+      float v[32], x[32];
+      tmem_ld32(c.taddr + cc, v);
+      if (!valid || c.n0 + cc >= n) continue;
+      load_f32x32(xrow + cc, x);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = a * x[j] + v[j];
+      store_f32x32(row + cc, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) colT[int64_t(cc + j) * m] = v[j];  // coalesced across the warp's rows
+    }
+  }
+};
+
+}  // namespace ttt

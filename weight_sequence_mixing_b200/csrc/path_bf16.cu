@@ -1,5 +1,752 @@
+// bf16 path of the TTT layer: tcgen05 tensor-core GEMMs (bf16 operands, fp32
+// accumulation in TMEM) with the elementwise steps fused into their epilogues.
+//
+// Per chunk c (tokens [t0, t0+n), all heads batched, z = b*H + h):
+//   token phase  : one GEMM launch over 128-token x 128-hidden tiles computes the
+//                  inner forward on the keys and the loss backprop to the hidden
+//                  layer (epilogue: SiLU / GELU gating, eta_i folding), writing the
+//                  bf16 activations the weight gradient needs
+//   weight grads : one grouped launch of token-reduction GEMMs (MN-major operands,
+//                  split-K over tokens, fp32 partials, deterministic reduction)
+//   optimizer    : split reduction + momentum, [Newton-Schulz on tf32 tensor cores],
+//                  W <- W - lr U, row L2-norm, bf16 copies of the new weights
+//   apply        : O = F_W(Q) as two GEMMs (first layer + gating, second layer)
+// Non-causal layers update over every chunk and apply once; causal layers apply
+// with the current weights before each chunk's update.
+// Source: ViT3 digest section 02 (update equation; forward on keys, loss
+// backward, forward on queries); LaCT analysis "Nonlinear memory complements local
+// attention" (SwiGLU fast weights, negative dot loss, per-token learning rates,
+// momentum / Muon, L2 normalisation) and "Order of operations".
+#include <algorithm>
+
+#include "epilogues.cuh"
 #include "ttt_plan.cuh"
+
 namespace ttt {
-int plan_layout_bf16(Plan* p) { p->ws_bytes = 256; return TTT_OK; }
-int run_bf16(const Plan&, const Io&, void*, cudaStream_t) { return TTT_ERR_UNSUPPORTED; }
+namespace {
+
+// ------------------------------------------------------------------ workspace
+enum BBuf {
+  xWf,     // fp32 master weights [Z][P] (canonical packed layout)
+  xMom,    // fp32 momentum, gradient layout [Z][GR][d]
+  xU,      // fp32 update direction, gradient layout [Z][GR][d]
+  xRowSq,  // fp32 [Z][GR] squared row norms of U
+  xInvN,   // fp32 [Z][nmat] 1/(||U_k||_F + 1e-7)
+  xPart,   // fp32 split-K partials [S][Z][GR][d]
+  xFirst,  // bf16 first-layer weights [Z][R1][d] (SwiGLU: blocks [W1 128 | W3 128])
+  xW2T,    // bf16 W2^T [Z][h][d]
+  xW2,     // bf16 W2 [Z][d][h]
+  xKn,     // bf16 instance-normalised keys [Z][Cp][d]
+  xAct0,   // bf16 activations [Z][Cp][h]   (H' or H)
+  xAct1,   // bf16 activations [Z][Cp][2h]  (dZ13, dZ)
+  xAct2,   // bf16 [Z][Cp][h]  (GELU' for MSE)
+  xDY,     // bf16 [Z][Cp][d]  (dL/dV_hat for MSE / linear)
+  xHq,     // bf16 apply hidden [Z][Rq][h]
+  xNX, xNXT, xNX2, xNXT2, xNS, xNT,  // fp32 Newton-Schulz buffers [Z*nmat][...]
+  kNumBBuf
+};
+
+struct Dims {
+  int Z, H, N, Nq, d, h, Cp, Rq, GR, R1, nmat, m, n, splits;
+  bool src_t;  // Newton-Schulz input is the transpose of the gradient-layout source
+};
+
+Dims dims_of(const Plan& p) {
+  const ttt_config& c = p.cfg;
+  Dims D{};
+  D.Z = p.BH;
+  D.H = c.H;
+  D.N = c.N;
+  D.Nq = c.Nq;
+  D.d = c.d;
+  D.h = c.h;
+  D.Cp = (p.chunk + 127) / 128 * 128;
+  D.Rq = c.causal ? D.Cp : (c.Nq + 127) / 128 * 128;
+  switch (c.inner) {
+    case TTT_INNER_LINEAR: D.GR = c.d; D.R1 = c.d; D.nmat = 1; break;
+    case TTT_INNER_MLP2_GELU: D.GR = 2 * c.h; D.R1 = c.h; D.nmat = 2; break;
+    default: D.GR = 3 * c.h; D.R1 = 2 * c.h; D.nmat = 3; break;
+  }
+  const int rows_src = c.inner == TTT_INNER_LINEAR ? c.d : c.h;
+  D.src_t = rows_src > c.d;
+  D.m = std::min(rows_src, c.d);
+  D.n = std::max(rows_src, c.d);
+  D.splits = int(p.off[kNumBBuf]);
+  return D;
 }
+
+int bn_for(int n) { return n % 256 == 0 ? 256 : n % 128 == 0 ? 128 : 64; }
+
+// ------------------------------------------------------------------ small kernels
+// Per canonical weight row: which matrix, its length, and where its gradient /
+// Newton-Schulz rows live.
+struct RowMap {
+  int inner, d, h, GR;
+  int64_t P;
+  __host__ __device__ int nrows() const {
+    return inner == TTT_INNER_LINEAR ? d : inner == TTT_INNER_MLP2_GELU ? h + d : 2 * h + d;
+  }
+  // matrix index k, row inside it, row length, offset of the matrix in the packed layout
+  __device__ void locate(int R, int& k, int& r, int& len, int64_t& off) const {
+    if (inner == TTT_INNER_LINEAR) { k = 0; r = R; len = d; off = 0; return; }
+    if (inner == TTT_INNER_MLP2_GELU) {
+      if (R < h) { k = 0; r = R; len = d; off = 0; }
+      else { k = 1; r = R - h; len = h; off = int64_t(h) * d; }
+      return;
+    }
+    if (R < h) { k = 0; r = R; len = d; off = 0; }
+    else if (R < 2 * h) { k = 1; r = R - h; len = d; off = int64_t(h) * d; }
+    else { k = 2; r = R - 2 * h; len = h; off = 2 * int64_t(h) * d; }
+  }
+  __device__ bool is_w2(int k) const { return inner != TTT_INNER_LINEAR && k == (inner == TTT_INNER_SWIGLU ? 2 : 1); }
+  // gradient-layout row of row r of a first-layer matrix k (W1, W3 or linear W)
+  __device__ int grad_row(int k, int r) const {
+    if (inner == TTT_INNER_LINEAR) return r;
+    if (inner == TTT_INNER_MLP2_GELU) return h + r;
+    return h + 256 * (r / 128) + (k == 1 ? 128 : 0) + (r % 128);
+  }
+  // bf16 first-layer row of row r of matrix k
+  __device__ int first_row(int k, int r) const {
+    if (inner == TTT_INNER_SWIGLU) return 256 * (r / 128) + (k == 1 ? 128 : 0) + (r % 128);
+    return r;
+  }
+};
+
+__global__ void init_weights_kernel(int Z, int H, int64_t P, const float* W0, float* W) {
+  const int64_t total = int64_t(Z) * P;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x)
+    W[i] = W0[int64_t(int(i / P) % H) * P + i % P];
+}
+
+// One warp per canonical weight row: [W -= lr U] -> [row L2-norm] -> bf16 copies
+// (+ the non-finite check of the layer's weights).
+//   mode 0: no update (initial weights)
+//   mode 1: U from the gradient layout
+//   mode 2: U from the Newton-Schulz result (X [m][n], XT [n][m] per matrix)
+__global__ void finish_rows_kernel(RowMap rm, int mode, float lr, bool rownorm, float* Wf, const float* U,
+                                   const float* X, const float* XT, int m, int n, bool src_t, bf16* First, bf16* W2T,
+                                   bf16* W2, unsigned* status) {
+  const int z = blockIdx.y;
+  const int R = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  if (R >= rm.nrows()) return;
+  const int lane = threadIdx.x & 31;
+  int k, r, len;
+  int64_t off;
+  rm.locate(R, k, r, len, off);
+  float* w = Wf + z * rm.P + off + int64_t(r) * len;
+  const bool w2 = rm.is_w2(k);
+  const int nmat = rm.inner == TTT_INNER_LINEAR ? 1 : rm.inner == TTT_INNER_MLP2_GELU ? 2 : 3;
+  if (mode == 1) {
+    const float* Uz = U + int64_t(z) * rm.GR * rm.d;
+    if (!w2) {
+      const float* u = Uz + int64_t(rm.grad_row(k, r)) * rm.d;
+      for (int i = lane; i < len; i += 32) w[i] -= lr * u[i];
+    } else {  // W2 row r = column r of the G2^T rows [0, h)
+      for (int i = lane; i < len; i += 32) w[i] -= lr * Uz[int64_t(i) * rm.d + r];
+    }
+  } else if (mode == 2) {
+    const int64_t mn = int64_t(m) * n;
+    const float* Xk = X + (int64_t(z) * nmat + k) * mn;
+    const float* XTk = XT + (int64_t(z) * nmat + k) * mn;
+    // result in the source orientation is (src_t ? XT : X); W2 rows are its columns
+    const float* src = w2 ? (src_t ? Xk : XTk) : (src_t ? XTk : Xk);
+    const float* u = src + int64_t(r) * len;
+    for (int i = lane; i < len; i += 32) w[i] -= lr * u[i];
+  }
+  float inv = 1.0f;
+  if (rownorm) {
+    float s = 0.f;
+    for (int i = lane; i < len; i += 32) s += w[i] * w[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    inv = 1.0f / fmaxf(sqrtf(s), 1e-12f);
+  }
+  bool bad = false;
+  if (!w2) {
+    bf16* f = First + (int64_t(z) * (rm.inner == TTT_INNER_SWIGLU ? 2 * rm.h : (rm.inner == TTT_INNER_LINEAR ? rm.d : rm.h)) +
+                       rm.first_row(k, r)) * rm.d;
+    for (int i = lane; i < len; i += 32) {
+      const float v = w[i] * inv;
+      w[i] = v;
+      bad |= !isfinite(v);
+      f[i] = __float2bfloat16_rn(v);
+    }
+  } else {
+    bf16* w2row = W2 + (int64_t(z) * rm.d + r) * rm.h;
+    bf16* w2t = W2T + int64_t(z) * rm.h * rm.d + r;
+    for (int i = lane; i < len; i += 32) {
+      const float v = w[i] * inv;
+      w[i] = v;
+      bad |= !isfinite(v);
+      const bf16 b = __float2bfloat16_rn(v);
+      w2row[i] = b;
+      w2t[int64_t(i) * rm.d] = b;
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(status, kStatusNonFinite);
+}
+
+// One warp per gradient row: sum the split-K partials in split order, momentum,
+// write the update direction U and its squared norm.
+__global__ void reduce_grad_kernel(int Z, int GR, int d, int splits, const float* part, bool momentum, float beta,
+                                   float* Mom, float* U, float* rowsq) {
+  const int z = blockIdx.y;
+  const int g = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  if (g >= GR) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t(z) * GR + g) * d;
+  const int64_t sstride = int64_t(Z) * GR * d;
+  float sq = 0.f;
+  for (int i = lane * 4; i < d; i += 128) {
+    float4 acc = *reinterpret_cast<const float4*>(part + row + i);
+    for (int s = 1; s < splits; ++s) {
+      const float4 t = *reinterpret_cast<const float4*>(part + s * sstride + row + i);
+      acc.x += t.x; acc.y += t.y; acc.z += t.z; acc.w += t.w;
+    }
+    if (momentum) {
+      float4 m = *reinterpret_cast<const float4*>(Mom + row + i);
+      m.x = beta * m.x + acc.x; m.y = beta * m.y + acc.y; m.z = beta * m.z + acc.z; m.w = beta * m.w + acc.w;
+      *reinterpret_cast<float4*>(Mom + row + i) = m;
+      acc = m;
+    }
+    *reinterpret_cast<float4*>(U + row + i) = acc;
+    sq += acc.x * acc.x + acc.y * acc.y + acc.z * acc.z + acc.w * acc.w;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  if (lane == 0 && rowsq) rowsq[int64_t(z) * GR + g] = sq;
+}
+
+// 1/(||U_k||_F + 1e-7) per (z, matrix k), summing row norms in a fixed order.
+__global__ void ns_norm_kernel(RowMap rm, int nmat, const float* rowsq, float* invn) {
+  __shared__ float red[256];
+  const int z = blockIdx.x / nmat, k = blockIdx.x % nmat;
+  const int rows_src = rm.inner == TTT_INNER_LINEAR ? rm.d : rm.h;
+  const bool w2 = rm.is_w2(k);
+  float s = 0.f;
+  for (int r = threadIdx.x; r < rows_src; r += blockDim.x)
+    s += rowsq[int64_t(z) * rm.GR + (w2 ? r : rm.grad_row(k, r))];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) invn[blockIdx.x] = 1.0f / (sqrtf(red[0]) + 1e-7f);
+}
+
+// Newton-Schulz input of matrix k: its gradient-layout source M_src [rows_src][d]
+// scaled by invn, written in source orientation to A and transposed to B.
+// (X0, X0^T) = src_t ? (B, A) : (A, B).
+__global__ void ns_prep_kernel(RowMap rm, int nmat, const float* U, const float* invn, float* A, float* Bt) {
+  __shared__ float tile[32][33];
+  const int zk = blockIdx.z, z = zk / nmat, k = zk % nmat;
+  const int rows_src = rm.inner == TTT_INNER_LINEAR ? rm.d : rm.h;
+  const int d = rm.d;
+  const bool w2 = rm.is_w2(k);
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  const float s = invn[zk];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8 threads
+  const int64_t mn = int64_t(rows_src) * d;
+  for (int j = ty; j < 32; j += 8) {
+    const int r = r0 + j, c = c0 + tx;
+    float v = 0.f;
+    if (r < rows_src && c < d) {
+      const int g = w2 ? r : rm.grad_row(k, r);
+      v = U[(int64_t(z) * rm.GR + g) * d + c] * s;
+      A[zk * mn + int64_t(r) * d + c] = v;
+    }
+    tile[j][tx] = v;
+  }
+  __syncthreads();
+  for (int j = ty; j < 32; j += 8) {
+    const int c = c0 + j, r = r0 + tx;
+    if (r < rows_src && c < d) Bt[zk * mn + int64_t(c) * rows_src + r] = tile[tx][j];
+  }
+}
+
+// bf16 key instance-norm over the chunk's tokens: per (z, 64-channel group)
+__global__ void instnorm_bf16_kernel(int n, int Cp, int d, const bf16* K, int64_t k_zs, int t0, float eps, bf16* Kn,
+                                     int64_t kn_zs) {
+  __shared__ float red[8][64];
+  __shared__ float stat[2][64];
+  const int z = blockIdx.y, c0 = blockIdx.x * 64;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;  // 8 warps; each lane owns channels c0+2l, c0+2l+1
+  const bf16* src = K + z * k_zs + int64_t(t0) * d + c0 + 2 * lane;
+  float s0 = 0.f, s1 = 0.f;
+  for (int r = w; r < n; r += 8) {
+    const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(src + int64_t(r) * d));
+    s0 += v.x;
+    s1 += v.y;
+  }
+  red[w][2 * lane] = s0;
+  red[w][2 * lane + 1] = s1;
+  __syncthreads();
+  if (threadIdx.x < 64) {
+    float t = 0.f;
+    for (int j = 0; j < 8; ++j) t += red[j][threadIdx.x];
+    stat[0][threadIdx.x] = t / float(n);
+  }
+  __syncthreads();
+  const float m0 = stat[0][2 * lane], m1 = stat[0][2 * lane + 1];
+  float q0 = 0.f, q1 = 0.f;
+  for (int r = w; r < n; r += 8) {
+    const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(src + int64_t(r) * d));
+    q0 += (v.x - m0) * (v.x - m0);
+    q1 += (v.y - m1) * (v.y - m1);
+  }
+  __syncthreads();
+  red[w][2 * lane] = q0;
+  red[w][2 * lane + 1] = q1;
+  __syncthreads();
+  if (threadIdx.x < 64) {
+    float t = 0.f;
+    for (int j = 0; j < 8; ++j) t += red[j][threadIdx.x];
+    stat[1][threadIdx.x] = rsqrtf(t / float(n) + eps);
+  }
+  __syncthreads();
+  const float r0 = stat[1][2 * lane], r1 = stat[1][2 * lane + 1];
+  bf16* dst = Kn + z * kn_zs + c0 + 2 * lane;
+  for (int r = w; r < Cp; r += 8) {
+    float a = 0.f, b = 0.f;
+    if (r < n) {
+      const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(src + int64_t(r) * d));
+      a = (v.x - m0) * r0;
+      b = (v.y - m1) * r1;
+    }
+    *reinterpret_cast<__nv_bfloat162*>(dst + int64_t(r) * d) = __floats2bfloat162_rn(a, b);
+  }
+}
+
+// linear + negative dot loss: dY = -eta_t v_t for the chunk's rows (zeros past it)
+__global__ void neg_eta_rows_kernel(int n, int Cp, int d, const bf16* V, int64_t v_zs, int t0, const float* eta,
+                                    int64_t eta_zs, float eta_scalar, bf16* dY, int64_t y_zs) {
+  const int z = blockIdx.y;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < int64_t(Cp) * d; i += int64_t(gridDim.x) * blockDim.x) {
+    const int r = int(i / d), c = int(i % d);
+    float v = 0.f;
+    if (r < n) {
+      const float e = eta ? eta[z * eta_zs + t0 + r] : eta_scalar;
+      v = -e * __bfloat162float(V[z * v_zs + int64_t(t0 + r) * d + c]);
+    }
+    dY[z * y_zs + i] = __float2bfloat16_rn(v);
+  }
+}
+
+// ------------------------------------------------------------------ host helpers
+struct BView {
+  uint8_t* base;
+  unsigned* status;
+  template <typename T>
+  T* at(const Plan& p, int i) const { return reinterpret_cast<T*>(base + p.off[i]); }
+};
+
+#define TRY(x)                       \
+  do {                               \
+    int _r = (x);                    \
+    if (_r != TTT_OK) return _r;     \
+  } while (0)
+#define TRY_CUDA(x)                               \
+  do {                                            \
+    if ((x) != cudaSuccess) return TTT_ERR_CUDA;  \
+  } while (0)
+
+// A TMA map plus the box it was encoded with (checked against every launch).
+struct TM {
+  CUtensorMap m;
+  int box = 0;
+  int eb = 0;
+};
+
+// row-major [Z][rows][cols] view as a TMA map; box rows `box`
+int tmap(TM* t, const void* p, int eb, int64_t cols, int64_t rows, int64_t Z, int box) {
+  t->box = box;
+  t->eb = eb;
+  return make_tmap(&t->m, p, eb, cols, rows, Z, cols, cols * rows, box) ? TTT_OK : TTT_ERR_INVALID_ARG;
+}
+
+// Launch through the engine after checking that every map's box matches the
+// tile the kernel loads (K-major: the tile's rows; MN-major: 128/EB rows), so the
+// bytes a stage expects are exactly the bytes TMA delivers.
+template <int BN0, int BN1, bool AMN, bool BMN, int EB, int STAGES, class Epi>
+int gemm(const TM& a0, const TM& b0, const TM& a1, const TM& b1, const TcGeom& g, const Epi& e, unsigned* status,
+         cudaStream_t st) {
+  const int run = 128 / EB;
+  const int ra = AMN ? run : 128;
+  const int rb0 = BMN ? run : BN0;
+  const int rb1 = BMN ? run : (BN1 > 0 ? BN1 : BN0);
+  const bool second = BN1 > 0 || g.m_tiles1 > 0;
+  if (a0.box != ra || b0.box != rb0 || a0.eb != EB || b0.eb != EB) return TTT_ERR_INVALID_ARG;
+  if (second && (a1.box != ra || b1.box != rb1 || a1.eb != EB || b1.eb != EB)) return TTT_ERR_INVALID_ARG;
+  if (g.kblocks <= 0 || g.kb_per_split <= 0) return TTT_ERR_INVALID_ARG;
+  return launch_tc_gemm<BN0, BN1, AMN, BMN, EB, STAGES>(a0.m, b0.m, a1.m, b1.m, g, e, status, st) == cudaSuccess
+             ? TTT_OK
+             : TTT_ERR_CUDA;
+}
+
+TcGeom geom(int mt0, int mt1, int nt, int kblocks, int Z, int splits) {
+  TcGeom g;
+  g.m_tiles0 = mt0;
+  g.m_tiles1 = mt1;
+  g.n_tiles = nt;
+  g.kblocks = kblocks;
+  g.batches = Z;
+  g.kb_per_split = (kblocks + splits - 1) / splits;
+  g.splits = (kblocks + g.kb_per_split - 1) / g.kb_per_split;
+  return g;
+}
+
+struct Ctx {
+  const Plan& p;
+  Dims D;
+  BView v;
+  const Io& io;
+  cudaStream_t st;
+  RowMap rm;
+  TM tK, tV, tKmn, tVmn, tQ, tFirst, tW2T, tW2;
+  int bn_first = 0;
+};
+
+// update-direction -> weights (+ Newton-Schulz when the optimizer is Muon)
+int optimizer_step(Ctx& c) {
+  const Plan& p = c.p;
+  const Dims& D = c.D;
+  const ttt_config& cfg = p.cfg;
+  const bool mom = cfg.opt == TTT_OPT_MOMENTUM || cfg.opt == TTT_OPT_MOMENTUM_MUON;
+  const bool muon = cfg.opt == TTT_OPT_MUON || cfg.opt == TTT_OPT_MOMENTUM_MUON;
+  {
+    dim3 g((D.GR + 7) / 8, D.Z);
+    reduce_grad_kernel<<<g, 256, 0, c.st>>>(D.Z, D.GR, D.d, D.splits, c.v.at<float>(p, xPart), mom, cfg.momentum,
+                                            c.v.at<float>(p, xMom), c.v.at<float>(p, xU),
+                                            muon ? c.v.at<float>(p, xRowSq) : nullptr);
+    TRY_CUDA(cudaGetLastError());
+  }
+  float* X = c.v.at<float>(p, xNX);
+  float* XT = c.v.at<float>(p, xNXT);
+  if (muon) {
+    const int ZK = D.Z * D.nmat;
+    ns_norm_kernel<<<ZK, 256, 0, c.st>>>(c.rm, D.nmat, c.v.at<float>(p, xRowSq), c.v.at<float>(p, xInvN));
+    const int rows_src = cfg.inner == TTT_INNER_LINEAR ? D.d : D.h;
+    dim3 g((D.d + 31) / 32, (rows_src + 31) / 32, ZK);
+    float* A = D.src_t ? XT : X;
+    float* B = D.src_t ? X : XT;
+    ns_prep_kernel<<<g, 256, 0, c.st>>>(c.rm, D.nmat, c.v.at<float>(p, xU), c.v.at<float>(p, xInvN), A, B);
+    TRY_CUDA(cudaGetLastError());
+    float* X2 = c.v.at<float>(p, xNX2);
+    float* XT2 = c.v.at<float>(p, xNXT2);
+    float* S = c.v.at<float>(p, xNS);
+    float* T = c.v.at<float>(p, xNT);
+    const int m = D.m, n = D.n;
+    TM tS, tT;
+    TRY(tmap(&tS, S, 4, m, m, ZK, 128));
+    TRY(tmap(&tT, T, 4, m, m, ZK, 128));
+    const float a = cfg.ns_coeff[0], b = cfg.ns_coeff[1], cc = cfg.ns_coeff[2];
+    for (int it = 0; it < cfg.ns_iters; ++it) {
+      TM tX, tXT;
+      TRY(tmap(&tX, X, 4, n, m, ZK, 128));
+      TRY(tmap(&tXT, XT, 4, m, n, ZK, 128));
+      // S = X X^T
+      EpiStoreF32 e1{S, m, m, int64_t(m) * m};
+      TRY((gemm<128, 0, false, false, 4, 4>(tX, tX, tX, tX, geom(m / 128, 0, m / 128, n / 32, ZK, 1),
+                                                          e1, c.v.status, c.st)));
+      // T = b S + c S S   (S symmetric: S^T = S serves as the K-major B operand)
+      EpiNsPoly e2{T, S, m, m, int64_t(m) * m, b, cc};
+      TRY((gemm<128, 0, false, false, 4, 4>(tS, tS, tS, tS, geom(m / 128, 0, m / 128, m / 32, ZK, 1),
+                                                          e2, c.v.status, c.st)));
+      // X' = a X + T X  (B operand X^T [n][m] is K-major); stores X' and X'^T
+      EpiNsUpdate e3{X2, XT2, X, m, n, int64_t(m) * n, a};
+      TRY((gemm<128, 0, false, false, 4, 4>(tT, tXT, tT, tXT, geom(m / 128, 0, n / 128, m / 32, ZK, 1),
+                                                          e3, c.v.status, c.st)));
+      std::swap(X, X2);
+      std::swap(XT, XT2);
+    }
+  }
+  dim3 g((c.rm.nrows() + 7) / 8, D.Z);
+  finish_rows_kernel<<<g, 256, 0, c.st>>>(c.rm, muon ? 2 : 1, cfg.lr, (cfg.flags & TTT_FLAG_WEIGHT_L2NORM) != 0,
+                                          c.v.at<float>(p, xWf), c.v.at<float>(p, xU), X, XT, D.m, D.n, D.src_t,
+                                          c.v.at<bf16>(p, xFirst), c.v.at<bf16>(p, xW2T), c.v.at<bf16>(p, xW2),
+                                          c.v.status);
+  TRY_CUDA(cudaGetLastError());
+  return TTT_OK;
+}
+
+// one chunk's weight update: tokens [t0, t0+n)
+int update_chunk(Ctx& c, int t0, int n) {
+  const Plan& p = c.p;
+  const Dims& D = c.D;
+  const ttt_config& cfg = p.cfg;
+  const int Z = D.Z, d = D.d, h = D.h, Cp = D.Cp;
+  const bf16* K = static_cast<const bf16*>(c.io.K);
+  const bf16* V = static_cast<const bf16*>(c.io.V);
+  // keys: the input (token offset t0) or their instance-normalised copy (offset 0)
+  const TM* tX = &c.tK;
+  const TM* tXmn = &c.tKmn;
+  int xoff = t0;
+  TM tKn, tKnmn;
+  if (cfg.flags & TTT_FLAG_KEY_INSTNORM) {
+    bf16* Kn = c.v.at<bf16>(p, xKn);
+    instnorm_bf16_kernel<<<dim3(d / 64, Z), 256, 0, c.st>>>(n, Cp, d, K, int64_t(D.N) * d, t0, cfg.in_eps, Kn,
+                                                            int64_t(Cp) * d);
+    TRY_CUDA(cudaGetLastError());
+    TRY(tmap(&tKn, Kn, 2, d, Cp, Z, 128));
+    TRY(tmap(&tKnmn, Kn, 2, d, Cp, Z, 64));
+    tX = &tKn;
+    tXmn = &tKnmn;
+    xoff = 0;
+  }
+  bf16* A0 = c.v.at<bf16>(p, xAct0);
+  bf16* A1 = c.v.at<bf16>(p, xAct1);
+  bf16* A2 = c.v.at<bf16>(p, xAct2);
+  bf16* DY = c.v.at<bf16>(p, xDY);
+  float* part = c.v.at<float>(p, xPart);
+  const int64_t pz = int64_t(D.GR) * d, ps = int64_t(Z) * pz;
+  const int kbt = Cp / 64;  // token k-blocks of the weight-gradient GEMMs
+  const int bnd = bn_for(d);
+  unsigned* status = c.v.status;
+  const int mt = Cp / 128;
+
+  if (cfg.inner == TTT_INNER_SWIGLU) {
+    // token phase: [z1 | z3] = X [W1;W3]_blk^T, p = V W2[:, blk]  -> H', dZ13
+    EpiTokenDot<true> e{A0, A1, h, n, int64_t(Cp) * h, int64_t(Cp) * 2 * h, c.io.eta, D.N, t0, cfg.eta_scalar};
+    TcGeom g = geom(mt, 0, h / 128, d / 64, Z, 1);
+    g.a0.mn = xoff;
+    g.a1.mn = t0;
+    TRY((gemm<256, 128, false, false, 2, 2>(*tX, c.tFirst, c.tV, c.tW2T, g, e, status, c.st)));
+    // weight gradients: G2^T = H'^T V  (rows [0,h)),  G13 = dZ13^T X  (rows [h, 3h))
+    TM tH, tD;
+    TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
+    TRY(tmap(&tD, A1, 2, 2 * h, Cp, Z, 64));
+    TcGeom gg = geom(h / 128, 2 * h / 128, d / bnd, kbt, Z, D.splits);
+    gg.b0.k = t0;
+    gg.b1.k = xoff;
+    EpiPartial ep{part, ps, pz, d, {0, h}, {h, 2 * h}};
+    if (bnd == 256) TRY((gemm<256, 0, true, true, 2, 4>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st)));
+    else if (bnd == 128) TRY((gemm<128, 0, true, true, 2, 6>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st)));
+    else TRY((gemm<64, 0, true, true, 2, 4>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st)));
+  } else if (cfg.inner == TTT_INNER_MLP2_GELU && cfg.loss == TTT_LOSS_NEG_DOT) {
+    EpiTokenDot<false> e{A0, A1, h, n, int64_t(Cp) * h, int64_t(Cp) * h, c.io.eta, D.N, t0, cfg.eta_scalar};
+    TcGeom g = geom(mt, 0, h / 128, d / 64, Z, 1);
+    g.a0.mn = xoff;
+    g.a1.mn = t0;
+    TRY((gemm<128, 128, false, false, 2, 3>(*tX, c.tFirst, c.tV, c.tW2T, g, e, status, c.st)));
+    TM tH, tD;
+    TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
+    TRY(tmap(&tD, A1, 2, h, Cp, Z, 64));
+    TcGeom gg = geom(h / 128, h / 128, d / bnd, kbt, Z, D.splits);
+    gg.b0.k = t0;
+    gg.b1.k = xoff;
+    EpiPartial ep{part, ps, pz, d, {0, h}, {h, h}};
+    if (bnd == 256) TRY((gemm<256, 0, true, true, 2, 4>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st)));
+    else if (bnd == 128) TRY((gemm<128, 0, true, true, 2, 6>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st)));
+    else TRY((gemm<64, 0, true, true, 2, 4>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st)));
+  } else if (cfg.inner == TTT_INNER_MLP2_GELU) {  // MSE
+    // Z = X W1^T -> H = GELU(Z), G' = GELU'(Z)
+    EpiGeluSave e1{A0, A2, h, n, int64_t(Cp) * h};
+    TcGeom g1 = geom(mt, 0, h / bn_for(h), d / 64, Z, 1);
+    g1.a0.mn = xoff;
+    if (bn_for(h) == 256) TRY((gemm<256, 0, false, false, 2, 4>(*tX, c.tFirst, *tX, c.tFirst, g1, e1, status, c.st)));
+    else TRY((gemm<128, 0, false, false, 2, 4>(*tX, c.tFirst, *tX, c.tFirst, g1, e1, status, c.st)));
+    // V_hat = H W2^T -> dY = 2 eta (V_hat - V)/(n d)
+    TM tHk, tY, tYmn, tH, tD;
+    TRY(tmap(&tHk, A0, 2, h, Cp, Z, 128));
+    EpiMseGrad e2{DY, d, n, int64_t(Cp) * d, V, int64_t(D.N) * d, t0, c.io.eta, D.N, cfg.eta_scalar,
+                  2.0f / (float(n) * float(d))};
+    TcGeom g2 = geom(mt, 0, d / bnd, h / 64, Z, 1);
+    if (bnd == 256) TRY((gemm<256, 0, false, false, 2, 4>(tHk, c.tW2, tHk, c.tW2, g2, e2, status, c.st)));
+    else if (bnd == 128) TRY((gemm<128, 0, false, false, 2, 4>(tHk, c.tW2, tHk, c.tW2, g2, e2, status, c.st)));
+    else TRY((gemm<64, 0, false, false, 2, 4>(tHk, c.tW2, tHk, c.tW2, g2, e2, status, c.st)));
+    // dH = dY W2 -> dZ = dH G'
+    TRY(tmap(&tY, DY, 2, d, Cp, Z, 128));
+    EpiMulSaved e3{A1, A2, h, int64_t(Cp) * h};
+    TcGeom g3 = geom(mt, 0, h / bn_for(h), d / 64, Z, 1);
+    if (bn_for(h) == 256) TRY((gemm<256, 0, false, false, 2, 4>(tY, c.tW2T, tY, c.tW2T, g3, e3, status, c.st)));
+    else TRY((gemm<128, 0, false, false, 2, 4>(tY, c.tW2T, tY, c.tW2T, g3, e3, status, c.st)));
+    // G2^T = H^T dY (rows [0,h)), G1 = dZ^T X (rows [h,2h))
+    TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
+    TRY(tmap(&tYmn, DY, 2, d, Cp, Z, 64));
+    TRY(tmap(&tD, A1, 2, h, Cp, Z, 64));
+    TcGeom gg = geom(h / 128, h / 128, d / bnd, kbt, Z, D.splits);
+    gg.b1.k = xoff;
+    EpiPartial ep{part, ps, pz, d, {0, h}, {h, h}};
+    if (bnd == 256) TRY((gemm<256, 0, true, true, 2, 4>(tH, tYmn, tD, *tXmn, gg, ep, status, c.st)));
+    else if (bnd == 128) TRY((gemm<128, 0, true, true, 2, 6>(tH, tYmn, tD, *tXmn, gg, ep, status, c.st)));
+    else TRY((gemm<64, 0, true, true, 2, 4>(tH, tYmn, tD, *tXmn, gg, ep, status, c.st)));
+  } else {  // linear
+    if (cfg.loss == TTT_LOSS_MSE) {
+      EpiMseGrad e2{DY, d, n, int64_t(Cp) * d, V, int64_t(D.N) * d, t0, c.io.eta, D.N, cfg.eta_scalar,
+                    2.0f / (float(n) * float(d))};
+      TcGeom g2 = geom(mt, 0, d / bnd, d / 64, Z, 1);
+      g2.a0.mn = xoff;
+      if (bnd == 256) TRY((gemm<256, 0, false, false, 2, 4>(*tX, c.tFirst, *tX, c.tFirst, g2, e2, status, c.st)));
+      else if (bnd == 128) TRY((gemm<128, 0, false, false, 2, 4>(*tX, c.tFirst, *tX, c.tFirst, g2, e2, status, c.st)));
+      else TRY((gemm<64, 0, false, false, 2, 4>(*tX, c.tFirst, *tX, c.tFirst, g2, e2, status, c.st)));
+    } else {
+      neg_eta_rows_kernel<<<dim3(64, Z), 256, 0, c.st>>>(n, Cp, d, V, int64_t(D.N) * d, t0, c.io.eta, D.N,
+                                                         cfg.eta_scalar, DY, int64_t(Cp) * d);
+      TRY_CUDA(cudaGetLastError());
+    }
+    TM tYmn;
+    TRY(tmap(&tYmn, DY, 2, d, Cp, Z, 64));
+    TcGeom gg = geom(d / 128, 0, d / bnd, kbt, Z, D.splits);
+    gg.b0.k = xoff;
+    EpiPartial ep{part, ps, pz, d, {0, 0}, {d, 0}};
+    if (bnd == 256) TRY((gemm<256, 0, true, true, 2, 4>(tYmn, *tXmn, tYmn, *tXmn, gg, ep, status, c.st)));
+    else if (bnd == 128) TRY((gemm<128, 0, true, true, 2, 6>(tYmn, *tXmn, tYmn, *tXmn, gg, ep, status, c.st)));
+    else TRY((gemm<64, 0, true, true, 2, 4>(tYmn, *tXmn, tYmn, *tXmn, gg, ep, status, c.st)));
+  }
+  return optimizer_step(c);
+}
+
+// O rows [row0, row0 + rows) = F_W(Q rows [row0, row0 + rows))
+int apply_rows(Ctx& c, int row0, int rows) {
+  const Plan& p = c.p;
+  const Dims& D = c.D;
+  const ttt_config& cfg = p.cfg;
+  const int Z = D.Z, d = D.d, h = D.h;
+  const int mt = (rows + 127) / 128;
+  const int bnd = bn_for(d);
+  unsigned* status = c.v.status;
+  bf16* O = static_cast<bf16*>(c.io.O);
+  EpiStoreOut<bf16> eo{O, d, rows, row0, int64_t(D.Nq) * d, status};
+  if (cfg.inner == TTT_INNER_LINEAR) {
+    TcGeom g = geom(mt, 0, d / bnd, d / 64, Z, 1);
+    g.a0.mn = row0;
+    if (bnd == 256) TRY((gemm<256, 0, false, false, 2, 4>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, eo, status, c.st)));
+    else if (bnd == 128) TRY((gemm<128, 0, false, false, 2, 4>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, eo, status, c.st)));
+    else TRY((gemm<64, 0, false, false, 2, 4>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, eo, status, c.st)));
+    return TTT_OK;
+  }
+  bf16* Hq = c.v.at<bf16>(p, xHq);
+  if (cfg.inner == TTT_INNER_SWIGLU) {
+    EpiApplyAct<true> e{Hq, h, rows, int64_t(D.Rq) * h};
+    TcGeom g = geom(mt, 0, h / 128, d / 64, Z, 1);
+    g.a0.mn = row0;
+    TRY((gemm<256, 0, false, false, 2, 4>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, e, status, c.st)));
+  } else {
+    EpiApplyAct<false> e{Hq, h, rows, int64_t(D.Rq) * h};
+    const int bnh = c.bn_first;
+    TcGeom g = geom(mt, 0, h / bnh, d / 64, Z, 1);
+    g.a0.mn = row0;
+    if (bnh == 256) TRY((gemm<256, 0, false, false, 2, 4>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, e, status, c.st)));
+    else TRY((gemm<128, 0, false, false, 2, 4>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, e, status, c.st)));
+  }
+  TM tHq;
+  TRY(tmap(&tHq, Hq, 2, h, D.Rq, Z, 128));
+  TcGeom g2 = geom(mt, 0, d / bnd, h / 64, Z, 1);
+  if (bnd == 256) TRY((gemm<256, 0, false, false, 2, 4>(tHq, c.tW2, tHq, c.tW2, g2, eo, status, c.st)));
+  else if (bnd == 128) TRY((gemm<128, 0, false, false, 2, 4>(tHq, c.tW2, tHq, c.tW2, g2, eo, status, c.st)));
+  else TRY((gemm<64, 0, false, false, 2, 4>(tHq, c.tW2, tHq, c.tW2, g2, eo, status, c.st)));
+  return TTT_OK;
+}
+
+int choose_splits(const Plan& p, int Cp) {
+  const ttt_config& c = p.cfg;
+  const int d = c.d, h = c.h;
+  const int bnd = bn_for(d);
+  const int rows = c.inner == TTT_INNER_LINEAR ? d : c.inner == TTT_INNER_MLP2_GELU ? 2 * h : 3 * h;
+  const int tiles = rows / 128 * (d / bnd) * p.BH;
+  const int kblocks = Cp / 64;
+  int s = std::max(1, (4 * 148 + tiles - 1) / tiles);
+  s = std::min(s, std::max(1, kblocks / 4));
+  s = std::min(s, 64);
+  // every split must own at least one k-block
+  const int per = (kblocks + s - 1) / s;
+  return (kblocks + per - 1) / per;
+}
+
+}  // namespace
+
+int plan_layout_bf16(Plan* p) {
+  const ttt_config& c = p->cfg;
+  const int d = c.d, h = c.h;
+  // supported shapes of the tensor-core path
+  if (d % 64 != 0) return TTT_ERR_UNSUPPORTED;
+  if (c.inner != TTT_INNER_LINEAR && h % 128 != 0) return TTT_ERR_UNSUPPORTED;
+  if (c.inner == TTT_INNER_SWIGLU && c.loss != TTT_LOSS_NEG_DOT) return TTT_ERR_UNSUPPORTED;
+  const bool muon = c.opt == TTT_OPT_MUON || c.opt == TTT_OPT_MOMENTUM_MUON;
+  if (muon && (d % 128 != 0 || (c.inner != TTT_INNER_LINEAR && h % 128 != 0))) return TTT_ERR_UNSUPPORTED;
+  const int Cp = (p->chunk + 127) / 128 * 128;
+  p->off[kNumBBuf] = size_t(choose_splits(*p, Cp));
+  const Dims D = dims_of(*p);
+  const int64_t Z = D.Z, P = p->P, GR = D.GR, nm = int64_t(D.m) * D.n, mm = int64_t(D.m) * D.m;
+  const int64_t ZK = Z * D.nmat;
+  const bool mlp_mse = c.inner == TTT_INNER_MLP2_GELU && c.loss == TTT_LOSS_MSE;
+  const bool act = c.inner != TTT_INNER_LINEAR;
+  const int64_t bytes[kNumBBuf] = {
+      Z * P * 4,
+      Z * GR * d * 4,
+      Z * GR * d * 4,
+      Z * GR * 4,
+      ZK * 4,
+      int64_t(D.splits) * Z * GR * d * 4,
+      Z * D.R1 * d * 2,
+      act ? Z * h * d * 2 : 0,
+      act ? Z * d * h * 2 : 0,
+      (c.flags & TTT_FLAG_KEY_INSTNORM) ? Z * Cp * d * 2 : 0,
+      act ? Z * Cp * h * 2 : 0,
+      act ? Z * Cp * 2 * h * 2 : 0,
+      mlp_mse ? Z * Cp * h * 2 : 0,
+      (mlp_mse || !act) ? Z * Cp * d * 2 : 0,
+      act ? Z * D.Rq * h * 2 : 0,
+      muon ? ZK * nm * 4 : 0,
+      muon ? ZK * nm * 4 : 0,
+      muon ? ZK * nm * 4 : 0,
+      muon ? ZK * nm * 4 : 0,
+      muon ? ZK * mm * 4 : 0,
+      muon ? ZK * mm * 4 : 0,
+  };
+  size_t o = 256;
+  for (int i = 0; i < kNumBBuf; ++i) {
+    p->off[i] = o;
+    o += (size_t(bytes[i]) + 1023) / 1024 * 1024;
+  }
+  p->ws_bytes = o;
+  return TTT_OK;
+}
+
+int run_bf16(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
+  const ttt_config& cfg = p.cfg;
+  Ctx c{p, dims_of(p), BView{static_cast<uint8_t*>(ws), static_cast<unsigned*>(ws)}, io, st,
+        RowMap{cfg.inner, cfg.d, cfg.h, 0, p.P}};
+  const Dims& D = c.D;
+  c.rm.GR = D.GR;
+  const int Z = D.Z, d = D.d, h = D.h;
+  // tensor maps of the inputs and of the bf16 weight copies
+  TRY(tmap(&c.tK, io.K, 2, d, D.N, Z, 128));
+  TRY(tmap(&c.tV, io.V, 2, d, D.N, Z, 128));
+  TRY(tmap(&c.tKmn, io.K, 2, d, D.N, Z, 64));
+  TRY(tmap(&c.tVmn, io.V, 2, d, D.N, Z, 64));
+  TRY(tmap(&c.tQ, io.Q, 2, d, D.Nq, Z, 128));
+  bf16* First = c.v.at<bf16>(p, xFirst);
+  const int bn_first = cfg.inner == TTT_INNER_SWIGLU ? 256
+                       : cfg.inner == TTT_INNER_MLP2_GELU
+                           ? (cfg.loss == TTT_LOSS_NEG_DOT ? 128 : bn_for(h))
+                           : bn_for(d);
+  c.bn_first = bn_first;
+  TRY(tmap(&c.tFirst, First, 2, d, D.R1, Z, bn_first));
+  if (cfg.inner != TTT_INNER_LINEAR) {
+    TRY(tmap(&c.tW2T, c.v.at<bf16>(p, xW2T), 2, d, h, Z, cfg.loss == TTT_LOSS_NEG_DOT ? 128 : bn_for(h)));
+    TRY(tmap(&c.tW2, c.v.at<bf16>(p, xW2), 2, h, d, Z, bn_for(d)));
+  }
+  // W = W0 per batch entry, zero momentum, bf16 copies
+  init_weights_kernel<<<std::min<int64_t>((int64_t(Z) * p.P + 255) / 256, 4096), 256, 0, st>>>(
+      Z, cfg.H, p.P, io.W0, c.v.at<float>(p, xWf));
+  TRY_CUDA(cudaMemsetAsync(c.v.at<float>(p, xMom), 0, size_t(Z) * D.GR * d * 4, st));
+  {
+    dim3 g((c.rm.nrows() + 7) / 8, Z);
+    finish_rows_kernel<<<g, 256, 0, st>>>(c.rm, 0, 0.f, false, c.v.at<float>(p, xWf), nullptr, nullptr, nullptr, 0, 0,
+                                          false, First, c.v.at<bf16>(p, xW2T), c.v.at<bf16>(p, xW2), c.v.status);
+    TRY_CUDA(cudaGetLastError());
+  }
+  for (int ci = 0; ci < p.nchunks; ++ci) {
+    const int t0 = ci * p.chunk, n = std::min(p.chunk, cfg.N - t0);
+    if (cfg.causal) TRY(apply_rows(c, t0, n));
+    TRY(update_chunk(c, t0, n));
+  }
+  if (!cfg.causal) TRY(apply_rows(c, 0, cfg.Nq));
+  if (io.W_out)
+    TRY_CUDA(cudaMemcpyAsync(io.W_out, c.v.at<float>(p, xWf), size_t(Z) * p.P * 4, cudaMemcpyDeviceToDevice, st));
+  return TTT_OK;
+}
+
+}  // namespace ttt

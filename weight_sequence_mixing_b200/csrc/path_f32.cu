@@ -126,8 +126,8 @@ __global__ void swiglu_back_kernel(int64_t n, float* Z1, const float* Z3, float*
 }
 
 // dY = dL/dV_hat for the chunk; Vhat [Z][n][d] (overwritten), V rows t0.. of [Z][N][d]
-__global__ void loss_grad_kernel(int loss, int Z, int n, int d, float* Y, const float* V, int64_t v_sz, int t0,
-                                 const float* eta, int64_t eta_sz, float eta_scalar) {
+__global__ void loss_grad_kernel(int loss, int Z, int n, int d, float* Y, int64_t y_sz, const float* V, int64_t v_sz,
+                                 int t0, const float* eta, int64_t eta_sz, float eta_scalar) {
   const int64_t total = int64_t(Z) * n * d;
   const float mse_coef = 2.0f / (float(n) * float(d));
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
@@ -135,16 +135,18 @@ __global__ void loss_grad_kernel(int loss, int Z, int n, int d, float* Y, const 
     const int r = int((i / d) % n), c = int(i % d);
     const float v = V[z * v_sz + int64_t(t0 + r) * d + c];
     const float e = eta ? eta[z * eta_sz + t0 + r] : eta_scalar;
-    Y[i] = loss == TTT_LOSS_MSE ? mse_coef * e * (Y[i] - v) : -e * v;
+    float* y = Y + z * y_sz + int64_t(r) * d + c;
+    *y = loss == TTT_LOSS_MSE ? mse_coef * e * (*y - v) : -e * v;
   }
 }
 
 // key instance-norm over the chunk's tokens: one CTA per z
-__global__ void instnorm_kernel(int n, int d, const float* K, int64_t k_sz, int t0, float eps, float* out) {
-  extern __shared__ float red[];  // [2][blockDim]
+__global__ void instnorm_kernel(int n, int d, const float* K, int64_t k_sz, int t0, float eps, float* out,
+                                int64_t out_sz) {
+  extern __shared__ float red[];  // [blockDim]
   const int z = blockIdx.x;
   const float* src = K + z * k_sz + int64_t(t0) * d;
-  float* dst = out + int64_t(z) * n * d;
+  float* dst = out + z * out_sz;
   for (int c0 = 0; c0 < d; c0 += 32) {
     const int c = c0 + (threadIdx.x & 31);
     const int g = threadIdx.x >> 5, G = blockDim.x >> 5;
@@ -300,9 +302,7 @@ int inner_forward(const Plan& p, const F32View& v, cudaStream_t st, MatRef X, in
     case TTT_INNER_MLP2_GELU:
       r = sgemm(st, Z, n, h, d, 1.f, X, rmT(W, P, d), 0.f, none, v.b[bZ1], Rh, h);
       if (r) return r;
-      for (int z = 0; z < 1; ++z) {
-        act_kernel<<<grid_for(int64_t(Z) * Rh), 256, 0, st>>>(0, int64_t(Z) * Rh, v.b[bZ1], v.b[bH]);
-      }
+      act_kernel<<<grid_for(int64_t(Z) * Rh), 256, 0, st>>>(0, int64_t(Z) * Rh, v.b[bZ1], v.b[bH]);
       return sgemm(st, Z, n, d, h, 1.f, rm(v.b[bH], Rh, h), rmT(W + int64_t(h) * d, P, h), 0.f, none, Y, y_sz, y_ld);
     default:
       r = sgemm(st, Z, n, h, d, 1.f, X, rmT(W, P, d), 0.f, none, v.b[bZ1], Rh, h);
@@ -352,7 +352,7 @@ int update_chunk(const Plan& p, const F32View& v, const Io& io, cudaStream_t st,
   // keys (instance-normalised over the chunk's tokens when asked)
   MatRef X{K + int64_t(t0) * d, int64_t(N) * d, d, 1};
   if (c.flags & TTT_FLAG_KEY_INSTNORM) {
-    instnorm_kernel<<<Z, 256, 2 * 256 * sizeof(float), st>>>(n, d, K, int64_t(N) * d, t0, c.in_eps, v.b[bXn]);
+    instnorm_kernel<<<Z, 256, 256 * sizeof(float), st>>>(n, d, K, int64_t(N) * d, t0, c.in_eps, v.b[bXn], Rd);
     if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
     X = rm(v.b[bXn], Rd, d);
   }
@@ -360,7 +360,7 @@ int update_chunk(const Plan& p, const F32View& v, const Io& io, cudaStream_t st,
   r = inner_forward(p, v, st, X, n, v.b[bY], Rd, d);
   if (r) return r;
   const int64_t tot = int64_t(Z) * n * d;
-  loss_grad_kernel<<<grid_for(tot), 256, 0, st>>>(c.loss, Z, n, d, v.b[bY], V, int64_t(N) * d, t0, io.eta,
+  loss_grad_kernel<<<grid_for(tot), 256, 0, st>>>(c.loss, Z, n, d, v.b[bY], Rd, V, int64_t(N) * d, t0, io.eta,
                                                    int64_t(N), c.eta_scalar);
   // backprop into the gradient buffer G [Z][P]
   float* G = v.b[bG];
@@ -420,7 +420,7 @@ int plan_layout_f32(Plan* p) {
   const int64_t Z = p->BH, d = c.d, h = c.h, P = p->P;
   const int64_t R = std::max<int64_t>(p->chunk, c.Nq);  // rows per head in the activation buffers
   const int64_t m = std::min(d, h), n = std::max(d, h);
-  const int64_t sizes[kNumBuf] = {Z * P, Z * P, Z * P, Z * p->chunk * d, Z * R * h, Z * R * h, Z * R * h,
+  const int64_t sizes[kNumBuf] = {Z * P, Z * P, Z * P, Z * R * d, Z * R * h, Z * R * h, Z * R * h,
                                   Z * R * h, Z * R * h, Z * R * d, Z * m * n, Z * m * n, Z * m * m, Z * m * m};
   size_t o = 256;
   for (int i = 0; i < kNumBuf; ++i) {
