@@ -25,6 +25,19 @@ extern "C" {
 int ttt_selftest_gemm(int elem_bytes, int a_mn, int b_mn, int bn, int M, int N, int K, int batches, int splits,
                       const void* A, const void* B, float* C, void* stream);
 
+/* Per-stage timing of a handle's forward calls.  ttt_profile_enable(h, 1)
+ * clears earlier records and starts recording a CUDA event pair around every
+ * kernel launch of later ttt_forward calls, on the stream the kernel runs on;
+ * ttt_profile_enable(h, 0) stops.  ttt_profile_collect synchronises those events
+ * and writes, per stage id s < max_stages, the summed device milliseconds and the
+ * number of launches.  Stage ids and their names: ttt_stage_name(s). */
+int ttt_profile_enable(ttt_handle* handle, int on);
+int ttt_profile_collect(ttt_handle* handle, int max_stages, float* total_ms, int* launches);
+const char* ttt_stage_name(int stage);
+
+/* Kernel launches this handle's forward calls have enqueued since it was created. */
+int64_t ttt_launch_count(const ttt_handle* handle);
+
 #ifdef __cplusplus
 }
 #endif

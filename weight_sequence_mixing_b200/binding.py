@@ -32,8 +32,9 @@ FLAG_WEIGHT_L2NORM = 2
 EXPORTED = [
     "ttt_config_init", "ttt_create", "ttt_param_count", "ttt_workspace_size", "ttt_forward",
     "ttt_host_staging_size", "ttt_forward_host", "ttt_query_status", "ttt_destroy", "ttt_status_string",
-    "ttt_selftest_gemm",
+    "ttt_selftest_gemm", "ttt_profile_enable", "ttt_profile_collect", "ttt_stage_name", "ttt_launch_count",
 ]
+NUM_STAGES = 8
 
 
 class TTTConfig(ctypes.Structure):
@@ -71,6 +72,10 @@ def _load():
         "ttt_destroy": (None, [vp]),
         "ttt_status_string": (ctypes.c_char_p, [i32]),
         "ttt_selftest_gemm": (i32, [i32] * 9 + [vp, vp, vp, vp]),
+        "ttt_profile_enable": (i32, [vp, i32]),
+        "ttt_profile_collect": (i32, [vp, i32, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]),
+        "ttt_stage_name": (ctypes.c_char_p, [i32]),
+        "ttt_launch_count": (i64, [vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -175,6 +180,19 @@ class TTTLayer:
 
     def check_status(self, stream=None):
         _check(LIB.ttt_query_status(self._handle, _ptr(self.workspace), _stream_ptr(stream)), "device status")
+
+    # ---- per-stage device timing (CUDA events around every launch, on its stream)
+    def profile(self, on: bool):
+        _check(LIB.ttt_profile_enable(self._handle, int(bool(on))), "ttt_profile_enable")
+
+    def profile_collect(self) -> dict:
+        ms = (ctypes.c_float * NUM_STAGES)()
+        cnt = (ctypes.c_int * NUM_STAGES)()
+        _check(LIB.ttt_profile_collect(self._handle, NUM_STAGES, ms, cnt), "ttt_profile_collect")
+        return {LIB.ttt_stage_name(i).decode(): (float(ms[i]), int(cnt[i])) for i in range(NUM_STAGES) if cnt[i]}
+
+    def launch_count(self) -> int:
+        return int(LIB.ttt_launch_count(self._handle))
 
     # ---- host-buffer entry point (copies inside the library call)
     def staging(self):

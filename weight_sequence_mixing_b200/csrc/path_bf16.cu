@@ -379,6 +379,7 @@ int gemm(const TM& a0, const TM& b0, const TM& a1, const TM& b1, const TcGeom& g
   if (a0.box != ra || b0.box != rb0 || a0.eb != EB || b0.eb != EB) return TTT_ERR_INVALID_ARG;
   if (second && (a1.box != ra || b1.box != rb1 || a1.eb != EB || b1.eb != EB)) return TTT_ERR_INVALID_ARG;
   if (g.kblocks <= 0 || g.kb_per_split <= 0) return TTT_ERR_INVALID_ARG;
+  StageScope sc(g_stage, st);
   return launch_tc_gemm<BN0, BN1, AMN, BMN, EB, STAGES>(a0.m, b0.m, a1.m, b1.m, g, e, status, st) == cudaSuccess
              ? TTT_OK
              : TTT_ERR_CUDA;
@@ -409,6 +410,7 @@ struct Ctx {
 
 // update-direction -> weights (+ Newton-Schulz when the optimizer is Muon)
 int optimizer_step(Ctx& c) {
+  cudaStream_t st = c.st;
   const Plan& p = c.p;
   const Dims& D = c.D;
   const ttt_config& cfg = p.cfg;
@@ -416,21 +418,30 @@ int optimizer_step(Ctx& c) {
   const bool muon = cfg.opt == TTT_OPT_MUON || cfg.opt == TTT_OPT_MOMENTUM_MUON;
   {
     dim3 g((D.GR + 7) / 8, D.Z);
-    reduce_grad_kernel<<<g, 256, 0, c.st>>>(D.Z, D.GR, D.d, D.splits, c.v.at<float>(p, xPart), mom, cfg.momentum,
-                                            c.v.at<float>(p, xMom), c.v.at<float>(p, xU),
-                                            muon ? c.v.at<float>(p, xRowSq) : nullptr);
+    {
+      StageScope _sc(kStageReduce, st);
+      reduce_grad_kernel<<<g, 256, 0, c.st>>>(D.Z, D.GR, D.d, D.splits, c.v.at<float>(p, xPart), mom, cfg.momentum,
+                                              c.v.at<float>(p, xMom), c.v.at<float>(p, xU),
+                                              muon ? c.v.at<float>(p, xRowSq) : nullptr);
+    }
     TRY_CUDA(cudaGetLastError());
   }
   float* X = c.v.at<float>(p, xNX);
   float* XT = c.v.at<float>(p, xNXT);
   if (muon) {
     const int ZK = D.Z * D.nmat;
-    ns_norm_kernel<<<ZK, 256, 0, c.st>>>(c.rm, D.nmat, c.v.at<float>(p, xRowSq), c.v.at<float>(p, xInvN));
+    {
+      StageScope _sc(kStageNewtonSchulz, st);
+      ns_norm_kernel<<<ZK, 256, 0, c.st>>>(c.rm, D.nmat, c.v.at<float>(p, xRowSq), c.v.at<float>(p, xInvN));
+    }
     const int rows_src = cfg.inner == TTT_INNER_LINEAR ? D.d : D.h;
     dim3 g((D.d + 31) / 32, (rows_src + 31) / 32, ZK);
     float* A = D.src_t ? XT : X;
     float* B = D.src_t ? X : XT;
-    ns_prep_kernel<<<g, 256, 0, c.st>>>(c.rm, D.nmat, c.v.at<float>(p, xU), c.v.at<float>(p, xInvN), A, B);
+    {
+      StageScope _sc(kStageNewtonSchulz, st);
+      ns_prep_kernel<<<g, 256, 0, c.st>>>(c.rm, D.nmat, c.v.at<float>(p, xU), c.v.at<float>(p, xInvN), A, B);
+    }
     TRY_CUDA(cudaGetLastError());
     float* X2 = c.v.at<float>(p, xNX2);
     float* XT2 = c.v.at<float>(p, xNXT2);
@@ -441,6 +452,7 @@ int optimizer_step(Ctx& c) {
     TRY(tmap(&tS, S, 4, m, m, ZK, 128));
     TRY(tmap(&tT, T, 4, m, m, ZK, 128));
     const float a = cfg.ns_coeff[0], b = cfg.ns_coeff[1], cc = cfg.ns_coeff[2];
+    StageCtx stage(kStageNewtonSchulz);
     for (int it = 0; it < cfg.ns_iters; ++it) {
       TM tX, tXT;
       TRY(tmap(&tX, X, 4, n, m, ZK, 128));
@@ -462,16 +474,20 @@ int optimizer_step(Ctx& c) {
     }
   }
   dim3 g((c.rm.nrows() + 7) / 8, D.Z);
-  finish_rows_kernel<<<g, 256, 0, c.st>>>(c.rm, muon ? 2 : 1, cfg.lr, (cfg.flags & TTT_FLAG_WEIGHT_L2NORM) != 0,
-                                          c.v.at<float>(p, xWf), c.v.at<float>(p, xU), X, XT, D.m, D.n, D.src_t,
-                                          c.v.at<bf16>(p, xFirst), c.v.at<bf16>(p, xW2T), c.v.at<bf16>(p, xW2),
-                                          c.v.status);
+  {
+    StageScope _sc(kStageFinish, st);
+    finish_rows_kernel<<<g, 256, 0, c.st>>>(c.rm, muon ? 2 : 1, cfg.lr, (cfg.flags & TTT_FLAG_WEIGHT_L2NORM) != 0,
+                                            c.v.at<float>(p, xWf), c.v.at<float>(p, xU), X, XT, D.m, D.n, D.src_t,
+                                            c.v.at<bf16>(p, xFirst), c.v.at<bf16>(p, xW2T), c.v.at<bf16>(p, xW2),
+                                            c.v.status);
+  }
   TRY_CUDA(cudaGetLastError());
   return TTT_OK;
 }
 
 // one chunk's weight update: tokens [t0, t0+n)
 int update_chunk(Ctx& c, int t0, int n) {
+  cudaStream_t st = c.st;
   const Plan& p = c.p;
   const Dims& D = c.D;
   const ttt_config& cfg = p.cfg;
@@ -485,8 +501,11 @@ int update_chunk(Ctx& c, int t0, int n) {
   TM tKn, tKnmn;
   if (cfg.flags & TTT_FLAG_KEY_INSTNORM) {
     bf16* Kn = c.v.at<bf16>(p, xKn);
-    instnorm_bf16_kernel<<<dim3(d / 64, Z), 256, 0, c.st>>>(n, Cp, d, K, int64_t(D.N) * d, t0, cfg.in_eps, Kn,
-                                                            int64_t(Cp) * d);
+    {
+      StageScope _sc(kStageKeyNorm, st);
+      instnorm_bf16_kernel<<<dim3(d / 64, Z), 256, 0, c.st>>>(n, Cp, d, K, int64_t(D.N) * d, t0, cfg.in_eps, Kn,
+                                                              int64_t(Cp) * d);
+    }
     TRY_CUDA(cudaGetLastError());
     TRY(tmap(&tKn, Kn, 2, d, Cp, Z, 128));
     TRY(tmap(&tKnmn, Kn, 2, d, Cp, Z, 64));
@@ -505,6 +524,7 @@ int update_chunk(Ctx& c, int t0, int n) {
   unsigned* status = c.v.status;
   const int mt = Cp / 128;
 
+  StageCtx stage(kStageTokenPhase);
   if (cfg.inner == TTT_INNER_SWIGLU) {
     // token phase: [z1 | z3] = X [W1;W3]_blk^T, p = V W2[:, blk]  -> H', dZ13
     EpiTokenDot<true> e{A0, A1, h, n, int64_t(Cp) * h, int64_t(Cp) * 2 * h, c.io.eta, D.N, t0, cfg.eta_scalar};
@@ -516,6 +536,7 @@ int update_chunk(Ctx& c, int t0, int n) {
     TM tH, tD;
     TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
     TRY(tmap(&tD, A1, 2, 2 * h, Cp, Z, 64));
+    g_stage = kStageWeightGrad;
     TcGeom gg = geom(h / 128, 2 * h / 128, d / bnd, kbt, Z, D.splits);
     gg.b0.k = t0;
     gg.b1.k = xoff;
@@ -532,6 +553,7 @@ int update_chunk(Ctx& c, int t0, int n) {
     TM tH, tD;
     TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
     TRY(tmap(&tD, A1, 2, h, Cp, Z, 64));
+    g_stage = kStageWeightGrad;
     TcGeom gg = geom(h / 128, h / 128, d / bnd, kbt, Z, D.splits);
     gg.b0.k = t0;
     gg.b1.k = xoff;
@@ -565,6 +587,7 @@ int update_chunk(Ctx& c, int t0, int n) {
     TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
     TRY(tmap(&tYmn, DY, 2, d, Cp, Z, 64));
     TRY(tmap(&tD, A1, 2, h, Cp, Z, 64));
+    g_stage = kStageWeightGrad;
     TcGeom gg = geom(h / 128, h / 128, d / bnd, kbt, Z, D.splits);
     gg.b1.k = xoff;
     EpiPartial ep{part, ps, pz, d, {0, h}, {h, h}};
@@ -581,12 +604,16 @@ int update_chunk(Ctx& c, int t0, int n) {
       else if (bnd == 128) TRY((gemm<128, 0, false, false, 2, 4>(*tX, c.tFirst, *tX, c.tFirst, g2, e2, status, c.st)));
       else TRY((gemm<64, 0, false, false, 2, 4>(*tX, c.tFirst, *tX, c.tFirst, g2, e2, status, c.st)));
     } else {
-      neg_eta_rows_kernel<<<dim3(64, Z), 256, 0, c.st>>>(n, Cp, d, V, int64_t(D.N) * d, t0, c.io.eta, D.N,
-                                                         cfg.eta_scalar, DY, int64_t(Cp) * d);
+      {
+        StageScope _sc(kStageKeyNorm, st);
+        neg_eta_rows_kernel<<<dim3(64, Z), 256, 0, c.st>>>(n, Cp, d, V, int64_t(D.N) * d, t0, c.io.eta, D.N,
+                                                           cfg.eta_scalar, DY, int64_t(Cp) * d);
+      }
       TRY_CUDA(cudaGetLastError());
     }
     TM tYmn;
     TRY(tmap(&tYmn, DY, 2, d, Cp, Z, 64));
+    g_stage = kStageWeightGrad;
     TcGeom gg = geom(d / 128, 0, d / bnd, kbt, Z, D.splits);
     gg.b0.k = xoff;
     EpiPartial ep{part, ps, pz, d, {0, 0}, {d, 0}};
@@ -599,6 +626,7 @@ int update_chunk(Ctx& c, int t0, int n) {
 
 // O rows [row0, row0 + rows) = F_W(Q rows [row0, row0 + rows))
 int apply_rows(Ctx& c, int row0, int rows) {
+  StageCtx stage(kStageApply);
   const Plan& p = c.p;
   const Dims& D = c.D;
   const ttt_config& cfg = p.cfg;
@@ -729,13 +757,19 @@ int run_bf16(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
     TRY(tmap(&c.tW2, c.v.at<bf16>(p, xW2), 2, h, d, Z, bn_for(d)));
   }
   // W = W0 per batch entry, zero momentum, bf16 copies
-  init_weights_kernel<<<std::min<int64_t>((int64_t(Z) * p.P + 255) / 256, 4096), 256, 0, st>>>(
-      Z, cfg.H, p.P, io.W0, c.v.at<float>(p, xWf));
+  {
+    StageScope _sc(kStageOther, st);
+    init_weights_kernel<<<std::min<int64_t>((int64_t(Z) * p.P + 255) / 256, 4096), 256, 0, st>>>(
+        Z, cfg.H, p.P, io.W0, c.v.at<float>(p, xWf));
+  }
   TRY_CUDA(cudaMemsetAsync(c.v.at<float>(p, xMom), 0, size_t(Z) * D.GR * d * 4, st));
   {
     dim3 g((c.rm.nrows() + 7) / 8, Z);
-    finish_rows_kernel<<<g, 256, 0, st>>>(c.rm, 0, 0.f, false, c.v.at<float>(p, xWf), nullptr, nullptr, nullptr, 0, 0,
-                                          false, First, c.v.at<bf16>(p, xW2T), c.v.at<bf16>(p, xW2), c.v.status);
+    {
+      StageScope _sc(kStageFinish, st);
+      finish_rows_kernel<<<g, 256, 0, st>>>(c.rm, 0, 0.f, false, c.v.at<float>(p, xWf), nullptr, nullptr, nullptr, 0, 0,
+                                            false, First, c.v.at<bf16>(p, xW2T), c.v.at<bf16>(p, xW2), c.v.status);
+    }
     TRY_CUDA(cudaGetLastError());
   }
   for (int ci = 0; ci < p.nchunks; ++ci) {

@@ -78,7 +78,10 @@ int sgemm(cudaStream_t st, int Z, int M, int N, int K, float alpha, MatRef A, Ma
           float* C, int64_t cz, int64_t cr) {
   if (M <= 0 || N <= 0) return TTT_OK;
   dim3 grid((N + SG_T - 1) / SG_T, (M + SG_T - 1) / SG_T, Z);
-  sgemm_kernel<<<grid, 256, 0, st>>>(M, N, K, alpha, A, B, beta, Cin, C, cz, cr);
+  {
+    StageScope _sc(kStageOther, st);
+    sgemm_kernel<<<grid, 256, 0, st>>>(M, N, K, alpha, A, B, beta, Cin, C, cz, cr);
+  }
   return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
 }
 
@@ -302,14 +305,20 @@ int inner_forward(const Plan& p, const F32View& v, cudaStream_t st, MatRef X, in
     case TTT_INNER_MLP2_GELU:
       r = sgemm(st, Z, n, h, d, 1.f, X, rmT(W, P, d), 0.f, none, v.b[bZ1], Rh, h);
       if (r) return r;
-      act_kernel<<<grid_for(int64_t(Z) * Rh), 256, 0, st>>>(0, int64_t(Z) * Rh, v.b[bZ1], v.b[bH]);
+      {
+        StageScope _sc(kStageOther, st);
+        act_kernel<<<grid_for(int64_t(Z) * Rh), 256, 0, st>>>(0, int64_t(Z) * Rh, v.b[bZ1], v.b[bH]);
+      }
       return sgemm(st, Z, n, d, h, 1.f, rm(v.b[bH], Rh, h), rmT(W + int64_t(h) * d, P, h), 0.f, none, Y, y_sz, y_ld);
     default:
       r = sgemm(st, Z, n, h, d, 1.f, X, rmT(W, P, d), 0.f, none, v.b[bZ1], Rh, h);
       if (!r) r = sgemm(st, Z, n, h, d, 1.f, X, rmT(W + int64_t(h) * d, P, d), 0.f, none, v.b[bZ3], Rh, h);
       if (r) return r;
-      swiglu_fwd_kernel<<<grid_for(int64_t(Z) * Rh), 256, 0, st>>>(int64_t(Z) * Rh, v.b[bZ1], v.b[bZ3], v.b[bA],
-                                                                   v.b[bH]);
+      {
+        StageScope _sc(kStageOther, st);
+        swiglu_fwd_kernel<<<grid_for(int64_t(Z) * Rh), 256, 0, st>>>(int64_t(Z) * Rh, v.b[bZ1], v.b[bZ3], v.b[bA],
+                                                                     v.b[bH]);
+      }
       return sgemm(st, Z, n, d, h, 1.f, rm(v.b[bH], Rh, h), rmT(W + 2 * int64_t(h) * d, P, h), 0.f, none, Y, y_sz,
                    y_ld);
   }
@@ -325,7 +334,10 @@ int newton_schulz(const Plan& p, const F32View& v, cudaStream_t st, MatRef U, in
   const int64_t mn = int64_t(m) * n, mm = int64_t(m) * m;
   float* X = v.b[bNX];
   float* X2 = v.b[bNX2];
-  ns_normalize_kernel<<<Z, 256, 0, st>>>(m, n, src, X);
+  {
+    StageScope _sc(kStageOther, st);
+    ns_normalize_kernel<<<Z, 256, 0, st>>>(m, n, src, X);
+  }
   if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
   const float a = p.cfg.ns_coeff[0], b = p.cfg.ns_coeff[1], c = p.cfg.ns_coeff[2];
   const MatRef none{nullptr, 0, 0, 0};
@@ -352,7 +364,10 @@ int update_chunk(const Plan& p, const F32View& v, const Io& io, cudaStream_t st,
   // keys (instance-normalised over the chunk's tokens when asked)
   MatRef X{K + int64_t(t0) * d, int64_t(N) * d, d, 1};
   if (c.flags & TTT_FLAG_KEY_INSTNORM) {
-    instnorm_kernel<<<Z, 256, 256 * sizeof(float), st>>>(n, d, K, int64_t(N) * d, t0, c.in_eps, v.b[bXn], Rd);
+    {
+      StageScope _sc(kStageOther, st);
+      instnorm_kernel<<<Z, 256, 256 * sizeof(float), st>>>(n, d, K, int64_t(N) * d, t0, c.in_eps, v.b[bXn], Rd);
+    }
     if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
     X = rm(v.b[bXn], Rd, d);
   }
@@ -360,8 +375,11 @@ int update_chunk(const Plan& p, const F32View& v, const Io& io, cudaStream_t st,
   r = inner_forward(p, v, st, X, n, v.b[bY], Rd, d);
   if (r) return r;
   const int64_t tot = int64_t(Z) * n * d;
-  loss_grad_kernel<<<grid_for(tot), 256, 0, st>>>(c.loss, Z, n, d, v.b[bY], Rd, V, int64_t(N) * d, t0, io.eta,
-                                                   int64_t(N), c.eta_scalar);
+  {
+    StageScope _sc(kStageOther, st);
+    loss_grad_kernel<<<grid_for(tot), 256, 0, st>>>(c.loss, Z, n, d, v.b[bY], Rd, V, int64_t(N) * d, t0, io.eta,
+                                                     int64_t(N), c.eta_scalar);
+  }
   // backprop into the gradient buffer G [Z][P]
   float* G = v.b[bG];
   const float* W = v.b[bW];
@@ -375,7 +393,10 @@ int update_chunk(const Plan& p, const F32View& v, const Io& io, cudaStream_t st,
       r = sgemm(st, Z, d, h, n, 1.f, dYT, rm(v.b[bH], Rh, h), 0.f, none, G + int64_t(h) * d, P, h);  // G2 = dY^T H
       if (!r) r = sgemm(st, Z, n, h, d, 1.f, dY, rm(W + int64_t(h) * d, P, h), 0.f, none, v.b[bdH], Rh, h);  // dH
       if (!r) {
-        gelu_back_kernel<<<grid_for(int64_t(Z) * Rh), 256, 0, st>>>(int64_t(Z) * Rh, v.b[bZ1], v.b[bdH]);
+        {
+          StageScope _sc(kStageOther, st);
+          gelu_back_kernel<<<grid_for(int64_t(Z) * Rh), 256, 0, st>>>(int64_t(Z) * Rh, v.b[bZ1], v.b[bdH]);
+        }
         r = sgemm(st, Z, h, d, n, 1.f, rmT(v.b[bdH], Rh, h), X, 0.f, none, G, P, d);  // G1 = dZ^T X
       }
       break;
@@ -383,7 +404,10 @@ int update_chunk(const Plan& p, const F32View& v, const Io& io, cudaStream_t st,
       r = sgemm(st, Z, d, h, n, 1.f, dYT, rm(v.b[bH], Rh, h), 0.f, none, G + 2 * int64_t(h) * d, P, h);  // G2
       if (!r) r = sgemm(st, Z, n, h, d, 1.f, dY, rm(W + 2 * int64_t(h) * d, P, h), 0.f, none, v.b[bdH], Rh, h);
       if (!r) {
-        swiglu_back_kernel<<<grid_for(int64_t(Z) * Rh), 256, 0, st>>>(int64_t(Z) * Rh, v.b[bZ1], v.b[bZ3], v.b[bdH]);
+        {
+          StageScope _sc(kStageOther, st);
+          swiglu_back_kernel<<<grid_for(int64_t(Z) * Rh), 256, 0, st>>>(int64_t(Z) * Rh, v.b[bZ1], v.b[bZ3], v.b[bdH]);
+        }
         r = sgemm(st, Z, h, d, n, 1.f, rmT(v.b[bZ1], Rh, h), X, 0.f, none, G, P, d);  // G1 = dZ1^T X
       }
       if (!r) r = sgemm(st, Z, h, d, n, 1.f, rmT(v.b[bdH], Rh, h), X, 0.f, none, G + int64_t(h) * d, P, d);  // G3
@@ -404,10 +428,16 @@ int update_chunk(const Plan& p, const F32View& v, const Io& io, cudaStream_t st,
       if (r) return r;
     }
     dim3 g1((m.rows * m.cols + 255) / 256, Z);
-    apply_update_kernel<<<g1, 256, 0, st>>>(m.rows, m.cols, c.lr, U, v.b[bW] + m.off, P);
+    {
+      StageScope _sc(kStageOther, st);
+      apply_update_kernel<<<g1, 256, 0, st>>>(m.rows, m.cols, c.lr, U, v.b[bW] + m.off, P);
+    }
     if (c.flags & TTT_FLAG_WEIGHT_L2NORM) {
       dim3 g2((m.rows + 7) / 8, Z);
-      rownorm_kernel<<<g2, 256, 0, st>>>(m.rows, m.cols, v.b[bW] + m.off, P);
+      {
+        StageScope _sc(kStageOther, st);
+        rownorm_kernel<<<g2, 256, 0, st>>>(m.rows, m.cols, v.b[bW] + m.off, P);
+      }
     }
   }
   return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
@@ -437,7 +467,10 @@ int run_f32(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
   const F32View v = view(p, ws);
   const int Z = p.BH, d = c.d;
   const int64_t P = p.P, Rd = int64_t(p.off[kNumBuf]) * d;
-  init_weights_kernel<<<grid_for(int64_t(Z) * P), 256, 0, st>>>(Z, c.H, P, io.W0, v.b[bW]);
+  {
+    StageScope _sc(kStageOther, st);
+    init_weights_kernel<<<grid_for(int64_t(Z) * P), 256, 0, st>>>(Z, c.H, P, io.W0, v.b[bW]);
+  }
   if (cudaMemsetAsync(v.b[bM], 0, size_t(Z) * P * 4, st) != cudaSuccess) return TTT_ERR_CUDA;
   const float* Q = static_cast<const float*>(io.Q);
   float* O = static_cast<float*>(io.O);
@@ -465,8 +498,14 @@ int run_f32(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
   if (io.W_out &&
       cudaMemcpyAsync(io.W_out, v.b[bW], size_t(Z) * P * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return TTT_ERR_CUDA;
-  nonfinite_kernel<<<grid_for(int64_t(Z) * c.Nq * d), 256, 0, st>>>(int64_t(Z) * c.Nq * d, O, v.status);
-  nonfinite_kernel<<<grid_for(int64_t(Z) * P), 256, 0, st>>>(int64_t(Z) * P, v.b[bW], v.status);
+  {
+    StageScope _sc(kStageOther, st);
+    nonfinite_kernel<<<grid_for(int64_t(Z) * c.Nq * d), 256, 0, st>>>(int64_t(Z) * c.Nq * d, O, v.status);
+  }
+  {
+    StageScope _sc(kStageOther, st);
+    nonfinite_kernel<<<grid_for(int64_t(Z) * P), 256, 0, st>>>(int64_t(Z) * P, v.b[bW], v.status);
+  }
   return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
 }
 

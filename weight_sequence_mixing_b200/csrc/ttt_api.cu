@@ -10,6 +10,11 @@
 
 using namespace ttt;
 
+namespace ttt {
+thread_local Profiler* g_prof = nullptr;
+thread_local int g_stage = kStageOther;
+}
+
 extern "C" void ttt_config_init(ttt_config* c) {
   if (!c) return;
   std::memset(c, 0, sizeof(*c));
@@ -56,7 +61,10 @@ extern "C" int ttt_forward(ttt_handle* h, const void* Q, const void* K, const vo
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) != 0 || workspace_bytes < h->plan.ws_bytes)
     return TTT_ERR_WORKSPACE;
   Io io{Q, K, V, eta, W0, O, W_out};
-  return plan_run(h->plan, io, workspace, static_cast<cudaStream_t>(stream));
+  g_prof = &h->prof;
+  const int r = plan_run(h->plan, io, workspace, static_cast<cudaStream_t>(stream));
+  g_prof = nullptr;
+  return r;
 }
 
 extern "C" size_t ttt_host_staging_size(const ttt_handle* h) { return h ? h->plan.staging_bytes : 0; }
@@ -111,7 +119,47 @@ extern "C" int ttt_query_status(ttt_handle* h, void* workspace, void* stream) {
   return TTT_OK;
 }
 
-extern "C" void ttt_destroy(ttt_handle* h) { delete h; }
+extern "C" void ttt_destroy(ttt_handle* h) {
+  if (!h) return;
+  for (cudaEvent_t e : h->prof.pool) cudaEventDestroy(e);
+  delete h;
+}
+
+extern "C" int ttt_profile_enable(ttt_handle* h, int on) {
+  if (!h) return TTT_ERR_INVALID_ARG;
+  h->prof.on = on != 0;
+  h->prof.used = 0;
+  h->prof.stage_of.clear();
+  return TTT_OK;
+}
+
+extern "C" int ttt_profile_collect(ttt_handle* h, int max_stages, float* total_ms, int* launches) {
+  if (!h || max_stages <= 0 || !total_ms || !launches) return TTT_ERR_INVALID_ARG;
+  for (int i = 0; i < max_stages; ++i) {
+    total_ms[i] = 0.f;
+    launches[i] = 0;
+  }
+  const Profiler& p = h->prof;
+  for (size_t i = 0; i < p.used; ++i) {
+    if (cudaEventSynchronize(p.pool[2 * i + 1]) != cudaSuccess) return TTT_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, p.pool[2 * i], p.pool[2 * i + 1]) != cudaSuccess) return TTT_ERR_CUDA;
+    const int s = p.stage_of[i];
+    if (s >= 0 && s < max_stages) {
+      total_ms[s] += ms;
+      launches[s] += 1;
+    }
+  }
+  return TTT_OK;
+}
+
+extern "C" int64_t ttt_launch_count(const ttt_handle* h) { return h ? h->prof.launches : 0; }
+
+extern "C" const char* ttt_stage_name(int s) {
+  static const char* names[kNumStages] = {"token_phase", "weight_grad", "reduce_momentum", "newton_schulz",
+                                          "finish_rows", "apply",       "key_norm",        "other"};
+  return (s >= 0 && s < kNumStages) ? names[s] : "unknown";
+}
 
 extern "C" const char* ttt_status_string(int s) {
   switch (s) {

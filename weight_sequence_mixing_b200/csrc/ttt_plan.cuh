@@ -5,6 +5,7 @@
 #include <cstdint>
 
 #include "../../include/ttt.h"
+#include "profiler.cuh"
 #include "ptx.cuh"
 
 namespace ttt {
@@ -48,4 +49,5 @@ int run_bf16(const Plan& plan, const Io& io, void* workspace, cudaStream_t st);
 
 struct ttt_handle {
   ttt::Plan plan;
+  ttt::Profiler prof;
 };
