@@ -220,6 +220,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run the workload with N cut to this many key/value tokens (profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -228,6 +230,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     cfg = workload(args.workload)
+    if args.tokens:
+        cfg = cpu_sample_config(cfg, args.tokens)
 
     if args.impl == "reference":
         if rank == 0:
@@ -327,7 +331,7 @@ def main():
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        s, times, sample = time_oracle(cfg, CPU_SAMPLE_TOKENS[args.workload])
+        s, times, sample = time_oracle(cfg, min(cfg["N"], CPU_SAMPLE_TOKENS[args.workload]))
         cpu = {"value": s["B"] * s["N"] / times[0], "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
                "sample": sample, "seconds": times[0]}
 
@@ -345,8 +349,8 @@ def main():
         "vs_baseline": None,
         "dtype": "f32" if cfg["dtype"] == "f32" else "bf16",
         "data": "synthetic (seeded Gaussians of the workload's shapes)",
-        "config": {"workload": args.workload, **{k: cfg[k] for k in ("B", "H", "N", "Nq", "d", "h", "chunk",
-                                                                    "causal", "inner", "loss", "opt")},
+        "config": {"workload": args.workload + (f" cut to {cfg['N']} tokens" if args.tokens else ""),
+                   **{k: cfg[k] for k in ("B", "H", "N", "Nq", "d", "h", "chunk", "causal", "inner", "loss", "opt")},
                    "weight_l2norm": cfg["weight_l2norm"], "key_instnorm": cfg["key_instnorm"],
                    "l2": (f"L2 flushed between steps (256 MiB write); inputs {in_bytes / 2**20:.0f} MiB" if flush
                           else f"inputs {in_bytes / 2**20:.0f} MiB > 2x L2, no flush")},

@@ -1,9 +1,10 @@
 // Fused epilogues of the tcgen05 GEMMs of the bf16 TTT path.
 //
-// Each functor runs on the 4 epilogue warps of a CTA with one output row per
-// thread (TMEM lane = tile row) and reads its accumulators 32 columns at a time
-// with tcgen05.ld (a warp-collective: every thread of the warp executes every
-// load, rows outside the problem only skip their stores).
+// Each functor runs on the epilogue warps of a CTA with one output row per
+// thread (TMEM lane = tile row); a warp handles the 32-column chunks
+// c % nparts == part and reads them with tcgen05.ld (a warp-collective: every
+// thread of the warp executes every load, rows outside the problem only skip
+// their stores).
 #pragma once
 #include <cuda_bf16.h>
 
@@ -18,7 +19,14 @@ __device__ __forceinline__ float gelu_dev(float x) { return 0.5f * x * (1.0f + e
 __device__ __forceinline__ float gelu_grad_dev(float x) {
   return 0.5f * (1.0f + erff(x * 0.70710678118654752f)) + x * 0.39894228040143268f * __expf(-0.5f * x * x);
 }
-__device__ __forceinline__ float sigmoid_dev(float x) { return 1.0f / (1.0f + __expf(-x)); }
+// sigma(x) = (1 + tanh(x/2)) / 2 with the hardware tanh approximation (max rel.
+// error ~2^-11, below the bf16 rounding the results get)
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float sigmoid_dev(float x) { return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
@@ -90,7 +98,7 @@ struct EpiPartial {
     const bool ok = c.m < rows[c.problem];
     float* rowp = out + c.split * split_stride + c.z * z_stride + int64_t(row0[c.problem] + c.m) * ld + c.n0;
 #pragma unroll 1
-    for (int cc = 0; cc < BN0; cc += 32) {
+    for (int cc = 32 * c.part; cc < BN0; cc += 32 * c.nparts) {
       float v[32];
       tmem_ld32(c.taddr + cc, v);
       if (ok && c.n0 + cc < ld) store_f32x32(rowp + cc, v);
@@ -127,7 +135,7 @@ struct EpiTokenDot {
     bf16* hrow = Hp + c.z * hp_zs + int64_t(c.m) * h + blk * 128;
     bf16* drow = dZ + c.z * dz_zs + int64_t(c.m) * (SWIGLU ? 2 * h : h) + blk * (SWIGLU ? 256 : 128);
 #pragma unroll 1
-    for (int cc = 0; cc < 128; cc += 32) {
+    for (int cc = 32 * c.part; cc < 128; cc += 32 * c.nparts) {
       float z1[32], z3[32], p[32];
       tmem_ld32(c.taddr + cc, z1);
       if constexpr (SWIGLU) tmem_ld32(c.taddr + 128 + cc, z3);
@@ -169,7 +177,7 @@ struct EpiGeluSave {
     bf16* hrow = H + c.z * zs + int64_t(c.m) * ld + c.n0;
     bf16* grow = Gp + c.z * zs + int64_t(c.m) * ld + c.n0;
 #pragma unroll 1
-    for (int cc = 0; cc < BN0; cc += 32) {
+    for (int cc = 32 * c.part; cc < BN0; cc += 32 * c.nparts) {
       float v[32], a[32], g[32];
       tmem_ld32(c.taddr + cc, v);
 #pragma unroll
@@ -203,7 +211,7 @@ struct EpiMseGrad {
     bf16* yrow = dY + c.z * zs + int64_t(c.m) * d + c.n0;
     const bf16* vrow = V + c.z * v_zs + int64_t(t0 + (valid ? c.m : 0)) * d + c.n0;
 #pragma unroll 1
-    for (int cc = 0; cc < BN0; cc += 32) {
+    for (int cc = 32 * c.part; cc < BN0; cc += 32 * c.nparts) {
       float v[32], t[32];
       tmem_ld32(c.taddr + cc, v);
       if (c.n0 + cc >= d) continue;
@@ -227,7 +235,7 @@ struct EpiMulSaved {
     bf16* zrow = dZ + c.z * zs + int64_t(c.m) * ld + c.n0;
     const bf16* grow = Gp + c.z * zs + int64_t(c.m) * ld + c.n0;
 #pragma unroll 1
-    for (int cc = 0; cc < BN0; cc += 32) {
+    for (int cc = 32 * c.part; cc < BN0; cc += 32 * c.nparts) {
       float v[32], g[32];
       tmem_ld32(c.taddr + cc, v);
       load_bf16x32(grow + cc, g);
@@ -253,7 +261,7 @@ struct EpiApplyAct {
     if constexpr (SWIGLU) {
       bf16* row = Hq + c.z * zs + int64_t(c.m) * h + (c.n0 / BN0) * 128;
 #pragma unroll 1
-      for (int cc = 0; cc < 128; cc += 32) {
+      for (int cc = 32 * c.part; cc < 128; cc += 32 * c.nparts) {
         float z1[32], z3[32];
         tmem_ld32(c.taddr + cc, z1);
         tmem_ld32(c.taddr + 128 + cc, z3);
@@ -264,7 +272,7 @@ struct EpiApplyAct {
     } else {
       bf16* row = Hq + c.z * zs + int64_t(c.m) * h + c.n0;
 #pragma unroll 1
-      for (int cc = 0; cc < BN0; cc += 32) {
+      for (int cc = 32 * c.part; cc < BN0; cc += 32 * c.nparts) {
         float z[32];
         tmem_ld32(c.taddr + cc, z);
 #pragma unroll
@@ -290,7 +298,7 @@ struct EpiStoreOut {
     OutT* row = O + c.z * zs + int64_t(row0 + c.m) * d + c.n0;
     bool bad = false;
 #pragma unroll 1
-    for (int cc = 0; cc < BN0; cc += 32) {
+    for (int cc = 32 * c.part; cc < BN0; cc += 32 * c.nparts) {
       float v[32];
       tmem_ld32(c.taddr + cc, v);
       if (!valid || c.n0 + cc >= d) continue;
@@ -313,7 +321,7 @@ struct EpiStoreF32 {
   __device__ void run(const EpiCtx& c) const {
     float* row = out + c.z * zs + int64_t(c.m) * ld + c.n0;
 #pragma unroll 1
-    for (int cc = 0; cc < BN0; cc += 32) {
+    for (int cc = 32 * c.part; cc < BN0; cc += 32 * c.nparts) {
       float v[32];
       tmem_ld32(c.taddr + cc, v);
       if (c.m < rows && c.n0 + cc < ld) store_f32x32(row + cc, v);
@@ -333,7 +341,7 @@ struct EpiNsPoly {
     float* trow = T + c.z * zs + int64_t(c.m) * ld + c.n0;
     const float* srow = S + c.z * zs + int64_t(c.m) * ld + c.n0;
 #pragma unroll 1
-    for (int cc = 0; cc < BN0; cc += 32) {
+    for (int cc = 32 * c.part; cc < BN0; cc += 32 * c.nparts) {
       float v[32], s[32];
       tmem_ld32(c.taddr + cc, v);
       if (c.m >= rows || c.n0 + cc >= ld) continue;
@@ -360,7 +368,7 @@ struct EpiNsUpdate {
     const float* xrow = X + c.z * zs + int64_t(c.m) * n + c.n0;
     float* colT = XnT + c.z * zs + int64_t(c.n0) * m + c.m;
 #pragma unroll 1
-    for (int cc = 0; cc < BN0; cc += 32) {
+    for (int cc = 32 * c.part; cc < BN0; cc += 32 * c.nparts) {
       float v[32], x[32];
       tmem_ld32(c.taddr + cc, v);
       if (!valid || c.n0 + cc >= n) continue;

@@ -368,9 +368,9 @@ int tmap(TM* t, const void* p, int eb, int64_t cols, int64_t rows, int64_t Z, in
 // Launch through the engine after checking that every map's box matches the
 // tile the kernel loads (K-major: the tile's rows; MN-major: 128/EB rows), so the
 // bytes a stage expects are exactly the bytes TMA delivers.
-template <int BN0, int BN1, bool AMN, bool BMN, int EB, int STAGES, class Epi>
+template <int BN0, int BN1, bool AMN, bool BMN, int EB, int STAGES, int EW = 4, class Epi>
 int gemm(const TM& a0, const TM& b0, const TM& a1, const TM& b1, const TcGeom& g, const Epi& e, unsigned* status,
-         cudaStream_t st) {
+         cudaStream_t st, bool persistent = false) {
   const int run = 128 / EB;
   const int ra = AMN ? run : 128;
   const int rb0 = BMN ? run : BN0;
@@ -380,7 +380,8 @@ int gemm(const TM& a0, const TM& b0, const TM& a1, const TM& b1, const TcGeom& g
   if (second && (a1.box != ra || b1.box != rb1 || a1.eb != EB || b1.eb != EB)) return TTT_ERR_INVALID_ARG;
   if (g.kblocks <= 0 || g.kb_per_split <= 0) return TTT_ERR_INVALID_ARG;
   StageScope sc(g_stage, st);
-  return launch_tc_gemm<BN0, BN1, AMN, BMN, EB, STAGES>(a0.m, b0.m, a1.m, b1.m, g, e, status, st) == cudaSuccess
+  return launch_tc_gemm<BN0, BN1, AMN, BMN, EB, STAGES, EW>(a0.m, b0.m, a1.m, b1.m, g, e, status, st, persistent) ==
+                 cudaSuccess
              ? TTT_OK
              : TTT_ERR_CUDA;
 }
@@ -531,7 +532,7 @@ int update_chunk(Ctx& c, int t0, int n) {
     TcGeom g = geom(mt, 0, h / 128, d / 64, Z, 1);
     g.a0.mn = xoff;
     g.a1.mn = t0;
-    TRY((gemm<256, 128, false, false, 2, 2>(*tX, c.tFirst, c.tV, c.tW2T, g, e, status, c.st)));
+    TRY((gemm<256, 128, false, false, 2, 2, 8>(*tX, c.tFirst, c.tV, c.tW2T, g, e, status, c.st, true)));
     // weight gradients: G2^T = H'^T V  (rows [0,h)),  G13 = dZ13^T X  (rows [h, 3h))
     TM tH, tD;
     TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
@@ -549,7 +550,7 @@ int update_chunk(Ctx& c, int t0, int n) {
     TcGeom g = geom(mt, 0, h / 128, d / 64, Z, 1);
     g.a0.mn = xoff;
     g.a1.mn = t0;
-    TRY((gemm<128, 128, false, false, 2, 3>(*tX, c.tFirst, c.tV, c.tW2T, g, e, status, c.st)));
+    TRY((gemm<128, 128, false, false, 2, 3, 8>(*tX, c.tFirst, c.tV, c.tW2T, g, e, status, c.st, true)));
     TM tH, tD;
     TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
     TRY(tmap(&tD, A1, 2, h, Cp, Z, 64));
@@ -566,23 +567,23 @@ int update_chunk(Ctx& c, int t0, int n) {
     EpiGeluSave e1{A0, A2, h, n, int64_t(Cp) * h};
     TcGeom g1 = geom(mt, 0, h / bn_for(h), d / 64, Z, 1);
     g1.a0.mn = xoff;
-    if (bn_for(h) == 256) TRY((gemm<256, 0, false, false, 2, 4>(*tX, c.tFirst, *tX, c.tFirst, g1, e1, status, c.st)));
-    else TRY((gemm<128, 0, false, false, 2, 4>(*tX, c.tFirst, *tX, c.tFirst, g1, e1, status, c.st)));
+    if (bn_for(h) == 256) TRY((gemm<256, 0, false, false, 2, 4, 8>(*tX, c.tFirst, *tX, c.tFirst, g1, e1, status, c.st, true)));
+    else TRY((gemm<128, 0, false, false, 2, 4, 8>(*tX, c.tFirst, *tX, c.tFirst, g1, e1, status, c.st, true)));
     // V_hat = H W2^T -> dY = 2 eta (V_hat - V)/(n d)
     TM tHk, tY, tYmn, tH, tD;
     TRY(tmap(&tHk, A0, 2, h, Cp, Z, 128));
     EpiMseGrad e2{DY, d, n, int64_t(Cp) * d, V, int64_t(D.N) * d, t0, c.io.eta, D.N, cfg.eta_scalar,
                   2.0f / (float(n) * float(d))};
     TcGeom g2 = geom(mt, 0, d / bnd, h / 64, Z, 1);
-    if (bnd == 256) TRY((gemm<256, 0, false, false, 2, 4>(tHk, c.tW2, tHk, c.tW2, g2, e2, status, c.st)));
-    else if (bnd == 128) TRY((gemm<128, 0, false, false, 2, 4>(tHk, c.tW2, tHk, c.tW2, g2, e2, status, c.st)));
-    else TRY((gemm<64, 0, false, false, 2, 4>(tHk, c.tW2, tHk, c.tW2, g2, e2, status, c.st)));
+    if (bnd == 256) TRY((gemm<256, 0, false, false, 2, 4, 8>(tHk, c.tW2, tHk, c.tW2, g2, e2, status, c.st, true)));
+    else if (bnd == 128) TRY((gemm<128, 0, false, false, 2, 4, 8>(tHk, c.tW2, tHk, c.tW2, g2, e2, status, c.st, true)));
+    else TRY((gemm<64, 0, false, false, 2, 4, 8>(tHk, c.tW2, tHk, c.tW2, g2, e2, status, c.st, true)));
     // dH = dY W2 -> dZ = dH G'
     TRY(tmap(&tY, DY, 2, d, Cp, Z, 128));
     EpiMulSaved e3{A1, A2, h, int64_t(Cp) * h};
     TcGeom g3 = geom(mt, 0, h / bn_for(h), d / 64, Z, 1);
-    if (bn_for(h) == 256) TRY((gemm<256, 0, false, false, 2, 4>(tY, c.tW2T, tY, c.tW2T, g3, e3, status, c.st)));
-    else TRY((gemm<128, 0, false, false, 2, 4>(tY, c.tW2T, tY, c.tW2T, g3, e3, status, c.st)));
+    if (bn_for(h) == 256) TRY((gemm<256, 0, false, false, 2, 4, 8>(tY, c.tW2T, tY, c.tW2T, g3, e3, status, c.st, true)));
+    else TRY((gemm<128, 0, false, false, 2, 4, 8>(tY, c.tW2T, tY, c.tW2T, g3, e3, status, c.st, true)));
     // G2^T = H^T dY (rows [0,h)), G1 = dZ^T X (rows [h,2h))
     TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
     TRY(tmap(&tYmn, DY, 2, d, Cp, Z, 64));
@@ -600,9 +601,9 @@ int update_chunk(Ctx& c, int t0, int n) {
                     2.0f / (float(n) * float(d))};
       TcGeom g2 = geom(mt, 0, d / bnd, d / 64, Z, 1);
       g2.a0.mn = xoff;
-      if (bnd == 256) TRY((gemm<256, 0, false, false, 2, 4>(*tX, c.tFirst, *tX, c.tFirst, g2, e2, status, c.st)));
-      else if (bnd == 128) TRY((gemm<128, 0, false, false, 2, 4>(*tX, c.tFirst, *tX, c.tFirst, g2, e2, status, c.st)));
-      else TRY((gemm<64, 0, false, false, 2, 4>(*tX, c.tFirst, *tX, c.tFirst, g2, e2, status, c.st)));
+      if (bnd == 256) TRY((gemm<256, 0, false, false, 2, 4, 8>(*tX, c.tFirst, *tX, c.tFirst, g2, e2, status, c.st, true)));
+      else if (bnd == 128) TRY((gemm<128, 0, false, false, 2, 4, 8>(*tX, c.tFirst, *tX, c.tFirst, g2, e2, status, c.st, true)));
+      else TRY((gemm<64, 0, false, false, 2, 4, 8>(*tX, c.tFirst, *tX, c.tFirst, g2, e2, status, c.st, true)));
     } else {
       {
         StageScope _sc(kStageKeyNorm, st);
@@ -639,9 +640,9 @@ int apply_rows(Ctx& c, int row0, int rows) {
   if (cfg.inner == TTT_INNER_LINEAR) {
     TcGeom g = geom(mt, 0, d / bnd, d / 64, Z, 1);
     g.a0.mn = row0;
-    if (bnd == 256) TRY((gemm<256, 0, false, false, 2, 4>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, eo, status, c.st)));
-    else if (bnd == 128) TRY((gemm<128, 0, false, false, 2, 4>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, eo, status, c.st)));
-    else TRY((gemm<64, 0, false, false, 2, 4>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, eo, status, c.st)));
+    if (bnd == 256) TRY((gemm<256, 0, false, false, 2, 4, 8>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, eo, status, c.st, true)));
+    else if (bnd == 128) TRY((gemm<128, 0, false, false, 2, 4, 8>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, eo, status, c.st, true)));
+    else TRY((gemm<64, 0, false, false, 2, 4, 8>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, eo, status, c.st, true)));
     return TTT_OK;
   }
   bf16* Hq = c.v.at<bf16>(p, xHq);
@@ -649,21 +650,21 @@ int apply_rows(Ctx& c, int row0, int rows) {
     EpiApplyAct<true> e{Hq, h, rows, int64_t(D.Rq) * h};
     TcGeom g = geom(mt, 0, h / 128, d / 64, Z, 1);
     g.a0.mn = row0;
-    TRY((gemm<256, 0, false, false, 2, 4>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, e, status, c.st)));
+    TRY((gemm<256, 0, false, false, 2, 4, 8>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, e, status, c.st, true)));
   } else {
     EpiApplyAct<false> e{Hq, h, rows, int64_t(D.Rq) * h};
     const int bnh = c.bn_first;
     TcGeom g = geom(mt, 0, h / bnh, d / 64, Z, 1);
     g.a0.mn = row0;
-    if (bnh == 256) TRY((gemm<256, 0, false, false, 2, 4>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, e, status, c.st)));
-    else TRY((gemm<128, 0, false, false, 2, 4>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, e, status, c.st)));
+    if (bnh == 256) TRY((gemm<256, 0, false, false, 2, 4, 8>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, e, status, c.st, true)));
+    else TRY((gemm<128, 0, false, false, 2, 4, 8>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, e, status, c.st, true)));
   }
   TM tHq;
   TRY(tmap(&tHq, Hq, 2, h, D.Rq, Z, 128));
   TcGeom g2 = geom(mt, 0, d / bnd, h / 64, Z, 1);
-  if (bnd == 256) TRY((gemm<256, 0, false, false, 2, 4>(tHq, c.tW2, tHq, c.tW2, g2, eo, status, c.st)));
-  else if (bnd == 128) TRY((gemm<128, 0, false, false, 2, 4>(tHq, c.tW2, tHq, c.tW2, g2, eo, status, c.st)));
-  else TRY((gemm<64, 0, false, false, 2, 4>(tHq, c.tW2, tHq, c.tW2, g2, eo, status, c.st)));
+  if (bnd == 256) TRY((gemm<256, 0, false, false, 2, 4, 8>(tHq, c.tW2, tHq, c.tW2, g2, eo, status, c.st, true)));
+  else if (bnd == 128) TRY((gemm<128, 0, false, false, 2, 4, 8>(tHq, c.tW2, tHq, c.tW2, g2, eo, status, c.st, true)));
+  else TRY((gemm<64, 0, false, false, 2, 4, 8>(tHq, c.tW2, tHq, c.tW2, g2, eo, status, c.st, true)));
   return TTT_OK;
 }
 

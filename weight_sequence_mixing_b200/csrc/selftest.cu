@@ -14,7 +14,7 @@ struct EpiStorePartial {
   __device__ void run(const EpiCtx& c) const {
     float* rowp = out + ((static_cast<int64_t>(c.split) * batches + c.z) * M + c.m) * N;
 #pragma unroll 1
-    for (int cc = 0; cc < BN0; cc += 32) {
+    for (int cc = 32 * c.part; cc < BN0; cc += 32 * c.nparts) {
       float v[32];
       tmem_ld32(c.taddr + cc, v);
       if (c.m < M) {
@@ -48,7 +48,11 @@ int run_one(const void* A, const void* B, float* C, int M, int N, int K, int bat
   g.splits = (g.kblocks + g.kb_per_split - 1) / g.kb_per_split;
   if (g.splits != splits) return TTT_ERR_INVALID_ARG;  // every split must own at least one k-block
   EpiStorePartial epi{C, M, N, batches};
-  cudaError_t e = launch_tc_gemm<BN, 0, AMN, BMN, EB, 4>(ta, tb, ta, tb, g, epi, nullptr, st);
+  // odd batch counts run one CTA per tile, even ones persistent with 8 epilogue warps,
+  // so both launch shapes of the engine are exercised
+  cudaError_t e = (batches % 2)
+                      ? launch_tc_gemm<BN, 0, AMN, BMN, EB, 4, 4>(ta, tb, ta, tb, g, epi, nullptr, st, false)
+                      : launch_tc_gemm<BN, 0, AMN, BMN, EB, 4, 8>(ta, tb, ta, tb, g, epi, nullptr, st, true);
   return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
 }
 

@@ -1,10 +1,15 @@
 // Warp-specialised tcgen05 GEMM engine for sm_100a.
 //
-// One CTA computes one 128 x BN0 output tile (plus, optionally, a second
-// 128 x BN1 product of the same rows) with the accumulators in TMEM:
-//   warp 0    : TMA producer (one elected thread), STAGES-deep smem ring
-//   warp 1    : TMEM allocator + MMA issuer (one elected thread)
-//   warps 2-5 : epilogue; warp w reads TMEM lanes 32*(w%4) .. +31, one output row per thread
+// A CTA loops over output tiles (persistent when the grid is smaller than the
+// tile count).  Each tile is 128 x BN0 (plus, optionally, a second 128 x BN1
+// product of the same rows) with the accumulators in TMEM:
+//   warp 0       : TMA producer (one elected thread); the STAGES-deep smem ring runs
+//                  on across tiles, so the next tile's operands load during an epilogue
+//   warp 1       : TMEM allocator + MMA issuer (one elected thread)
+//   warps 2..    : EW epilogue warps; warp w reads TMEM lanes 32*(w%4) .. +31 (one
+//                  output row per thread) and the (w-2)/4-th share of the columns
+// Tiles are visited N-tile fastest, then M-tile, then batch and split: the CTAs in
+// flight share their A rows (token tiles read from HBM once) and their K range.
 //
 // Operands are read by TMA from 3-D tensor maps [batch][rows][cols] with 128-byte
 // swizzle; each operand is K-major (K contiguous) or MN-major (M/N contiguous), so
@@ -12,13 +17,14 @@
 // EB is the element size: 2 = bf16 (kind::f16), 4 = fp32 read as tf32 (kind::tf32).
 //
 // Launch modes:
-//   BN1 == 0 : one product per tile; blockIdx.x >= m_tiles0 selects a second,
+//   BN1 == 0 : one product per tile; M-tiles >= m_tiles0 belong to a second,
 //              independent problem (maps A1/B1, M1 rows) that shares N and K.
 //   BN1 > 0  : two products per tile, D0 = A0 B0^T (cols [0,BN0)) and
 //              D1 = A1 B1^T (cols [BN0, BN0+BN1)), both over the same K range.
-// Split-K: blockIdx.z = split * batches + batch; split s reduces k-blocks
-// [s*kb_per_split, (s+1)*kb_per_split).
+// Split-K: split s reduces k-blocks [s*kb_per_split, (s+1)*kb_per_split).
 #pragma once
+#include <algorithm>
+
 #include "ptx.cuh"
 
 namespace ttt {
@@ -44,7 +50,30 @@ struct EpiCtx {
   int z;           // batch entry
   int split;       // split-K index
   int problem;     // 0 or 1 (grouped launches)
+  int part, nparts;  // this warp handles the 32-column chunks c with c % nparts == part
 };
+
+// Tile coordinates of a linear tile index (N-tile fastest).
+struct TileCoord {
+  int problem, m0, n0, z, split, kb_begin, nkb;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const TcGeom& g, int t, int bn0) {
+  TileCoord c;
+  const int mtiles = g.m_tiles0 + g.m_tiles1;
+  const int nt = t % g.n_tiles;
+  int r = t / g.n_tiles;
+  const int mt = r % mtiles;
+  r /= mtiles;
+  c.z = r % g.batches;
+  c.split = r / g.batches;
+  c.problem = mt >= g.m_tiles0 ? 1 : 0;
+  c.m0 = (c.problem ? mt - g.m_tiles0 : mt) * 128;
+  c.n0 = nt * bn0;
+  c.kb_begin = c.split * g.kb_per_split;
+  c.nkb = max(0, min(g.kblocks, c.kb_begin + g.kb_per_split) - c.kb_begin);
+  return c;
+}
 
 __host__ __device__ constexpr int tmem_cols_for(int n) {
   return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512;
@@ -103,36 +132,25 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk) {
   }
 }
 
-template <int BN0, int BN1, bool A_MN, bool B_MN, int EB, int STAGES, class Epi>
-__global__ void __launch_bounds__(192, 1)
+template <int BN0, int BN1, bool A_MN, bool B_MN, int EB, int STAGES, int EW, class Epi>
+__global__ void __launch_bounds__(64 + 32 * EW, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tB0,
                    const __grid_constant__ CUtensorMap tA1, const __grid_constant__ CUtensorMap tB1,
                    const TcGeom g, const Epi epi, unsigned* status) {
   using S = TcShape<BN0, BN1, EB, STAGES>;
+  static_assert(EW % 4 == 0 && EW >= 4 && EW <= 16, "epilogue warps cover the 4 TMEM lane quarters");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tmem_full = empty + STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 1);
+  uint64_t* tmem_empty = tmem_full + 1;
+  uint64_t* drain = tmem_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
-  const int tile = blockIdx.x;
-  const int problem = (BN1 == 0 && tile >= g.m_tiles0) ? 1 : 0;
-  const int m_tile = problem ? tile - g.m_tiles0 : tile;
-  const int m0 = m_tile * S::BM;
-  const int n0 = blockIdx.y * BN0;
-  const int z = blockIdx.z % g.batches;
-  const int split = blockIdx.z / g.batches;
-  const int kb_begin = split * g.kb_per_split;
-  const int kb_end = min(g.kblocks, kb_begin + g.kb_per_split);
-  const int nkb = max(0, kb_end - kb_begin);
-
-  const CUtensorMap* mA = problem ? &tA1 : &tA0;
-  const CUtensorMap* mB = problem ? &tB1 : &tB0;
-  const OpOff oA = problem ? g.a1 : g.a0;
-  const OpOff oB = problem ? g.b1 : g.b0;
+  const int total = (g.m_tiles0 + g.m_tiles1) * g.n_tiles * g.batches * g.splits;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -140,6 +158,8 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(tmem_full, 1);
+    mbar_init(tmem_empty, EW);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -154,33 +174,43 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     if (elect_one()) {
-      tma_prefetch_desc(mA);
-      tma_prefetch_desc(mB);
-      if (BN1 > 0) {
+      tma_prefetch_desc(&tA0);
+      tma_prefetch_desc(&tB0);
+      if (BN1 > 0 || g.m_tiles1 > 0) {
         tma_prefetch_desc(&tA1);
         tma_prefetch_desc(&tB1);
       }
-      int issued = 0;
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % STAGES;
-        const uint32_t ph = (i / STAGES) & 1;
-        if (i >= STAGES && !mbar_wait(&empty[s], ph ^ 1, abort_flag)) break;
-        uint8_t* st = smem + s * S::STAGE_BYTES;
-        mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
-        const int k0 = (kb_begin + i) * S::BK;
-        load_operand<A_MN, EB>(st, mA, &full[s], S::BM, m0 + oA.mn, k0 + oA.k, z);
-        load_operand<B_MN, EB>(st + S::A_BYTES, mB, &full[s], BN0, n0 + oB.mn, k0 + oB.k, z);
-        if constexpr (BN1 > 0) {
-          uint8_t* st1 = st + S::A_BYTES + S::B0_BYTES;
-          load_operand<A_MN, EB>(st1, &tA1, &full[s], S::BM, m0 + g.a1.mn, k0 + g.a1.k, z);
-          load_operand<B_MN, EB>(st1 + S::A_BYTES, &tB1, &full[s], BN1, n0 / BN0 * BN1 + g.b1.mn,
-                                 k0 + g.b1.k, z);
+      int it = 0;
+      bool stop = false;
+      for (int t = blockIdx.x; t < total && !stop; t += gridDim.x) {
+        const TileCoord tc = decode_tile(g, t, BN0);
+        const CUtensorMap* mA = tc.problem ? &tA1 : &tA0;
+        const CUtensorMap* mB = tc.problem ? &tB1 : &tB0;
+        const OpOff oA = tc.problem ? g.a1 : g.a0;
+        const OpOff oB = tc.problem ? g.b1 : g.b0;
+        for (int i = 0; i < tc.nkb; ++i, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (it >= STAGES && !mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
+            stop = true;
+            break;
+          }
+          uint8_t* st = smem + s * S::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
+          const int k0 = (tc.kb_begin + i) * S::BK;
+          load_operand<A_MN, EB>(st, mA, &full[s], S::BM, tc.m0 + oA.mn, k0 + oA.k, tc.z);
+          load_operand<B_MN, EB>(st + S::A_BYTES, mB, &full[s], BN0, tc.n0 + oB.mn, k0 + oB.k, tc.z);
+          if constexpr (BN1 > 0) {
+            uint8_t* st1 = st + S::A_BYTES + S::B0_BYTES;
+            load_operand<A_MN, EB>(st1, &tA1, &full[s], S::BM, tc.m0 + g.a1.mn, k0 + g.a1.k, tc.z);
+            load_operand<B_MN, EB>(st1 + S::A_BYTES, &tB1, &full[s], BN1, tc.n0 / BN0 * BN1 + g.b1.mn,
+                                   k0 + g.b1.k, tc.z);
+          }
         }
-        ++issued;
       }
       if (*abort_flag) {
         // let the copies already in flight land before the CTA's smem is released
-        for (int j = max(0, issued - STAGES); j < issued; ++j) {
+        for (int j = max(0, it - STAGES); j < it; ++j) {
           volatile int never = 0;
           mbar_wait(&full[j % STAGES], (j / STAGES) & 1, &never);
         }
@@ -192,53 +222,74 @@ __global__ void __launch_bounds__(192, 1)
       constexpr uint32_t id0 = make_idesc(128, BN0, fmt, A_MN, B_MN);
       constexpr uint32_t id1 = make_idesc(128, BN1 > 0 ? BN1 : 16, fmt, A_MN, B_MN);
       const uint32_t sbase = smem_u32(smem);
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % STAGES;
-        const uint32_t ph = (i / STAGES) & 1;
-        if (!mbar_wait(&full[s], ph, abort_flag)) break;
+      int it = 0, j = 0;
+      bool stop = false;
+      for (int t = blockIdx.x; t < total && !stop; t += gridDim.x, ++j) {
+        const TileCoord tc = decode_tile(g, t, BN0);
+        // the previous tile's epilogue must have drained the accumulators
+        if (j > 0 && !mbar_wait(tmem_empty, (j - 1) & 1, abort_flag)) break;
         tc_fence_after();
-        const uint32_t a = sbase + s * S::STAGE_BYTES;
-        const uint32_t b = a + S::A_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < S::BK / S::UK; ++kk) {
-          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          const uint64_t da = operand_desc<A_MN, EB>(a, kk);
-          const uint64_t db = operand_desc<B_MN, EB>(b, kk);
-          if constexpr (EB == 2) mma_f16(tmem_base, da, db, id0, acc);
-          else mma_tf32(tmem_base, da, db, id0, acc);
-          if constexpr (BN1 > 0) {
-            const uint32_t a1 = b + S::B0_BYTES;
-            const uint32_t b1 = a1 + S::A_BYTES;
-            const uint64_t da1 = operand_desc<A_MN, EB>(a1, kk);
-            const uint64_t db1 = operand_desc<B_MN, EB>(b1, kk);
-            if constexpr (EB == 2) mma_f16(tmem_base + BN0, da1, db1, id1, acc);
-            else mma_tf32(tmem_base + BN0, da1, db1, id1, acc);
+        for (int i = 0; i < tc.nkb; ++i, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(&full[s], ph, abort_flag)) {
+            stop = true;
+            break;
           }
+          tc_fence_after();
+          const uint32_t a = sbase + s * S::STAGE_BYTES;
+          const uint32_t b = a + S::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < S::BK / S::UK; ++kk) {
+            const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+            const uint64_t da = operand_desc<A_MN, EB>(a, kk);
+            const uint64_t db = operand_desc<B_MN, EB>(b, kk);
+            if constexpr (EB == 2) mma_f16(tmem_base, da, db, id0, acc);
+            else mma_tf32(tmem_base, da, db, id0, acc);
+            if constexpr (BN1 > 0) {
+              const uint32_t a1 = b + S::B0_BYTES;
+              const uint32_t b1 = a1 + S::A_BYTES;
+              const uint64_t da1 = operand_desc<A_MN, EB>(a1, kk);
+              const uint64_t db1 = operand_desc<B_MN, EB>(b1, kk);
+              if constexpr (EB == 2) mma_f16(tmem_base + BN0, da1, db1, id1, acc);
+              else mma_tf32(tmem_base + BN0, da1, db1, id1, acc);
+            }
+          }
+          mma_commit(&empty[s]);
         }
-        mma_commit(&empty[s]);
+        mma_commit(tmem_full);
       }
-      mma_commit(tmem_full);
       if (*abort_flag) {
+        // MMAs in flight finish before TMEM is released
         volatile int never = 0;
-        mbar_wait(tmem_full, 0, &never);  // MMAs in flight finish before TMEM is released
+        mma_commit(drain);
+        mbar_wait(drain, 0, &never);
       }
     }
   } else {
     const int q = warp & 3;
     const int row = q * 32 + static_cast<int>(lane_id());
-    // warp-uniform decision: tcgen05.ld below is a warp-collective instruction
-    const bool ready = __all_sync(0xffffffffu, mbar_wait(tmem_full, 0, abort_flag));
-    if (ready) {
+    int j = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++j) {
+      const TileCoord tc = decode_tile(g, t, BN0);
+      // warp-uniform decision: tcgen05.ld below is a warp-collective instruction
+      const bool ready = __all_sync(0xffffffffu, mbar_wait(tmem_full, j & 1, abort_flag));
+      if (!ready) break;
       tc_fence_after();
       EpiCtx c;
       c.taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       c.row = row;
-      c.m = m0 + row;
-      c.n0 = n0;
-      c.z = z;
-      c.split = split;
-      c.problem = problem;
-      if (nkb > 0) epi.template run<BN0, BN1>(c);
+      c.m = tc.m0 + row;
+      c.n0 = tc.n0;
+      c.z = tc.z;
+      c.split = tc.split;
+      c.problem = tc.problem;
+      c.part = (warp - 2) >> 2;
+      c.nparts = EW / 4;
+      if (tc.nkb > 0) epi.template run<BN0, BN1>(c);
+      tc_fence_before();
+      __syncwarp();
+      if (lane_id() == 0) mbar_arrive(tmem_empty);
     }
   }
 
@@ -264,13 +315,17 @@ PFN_tmapEncodeTiled tmap_encoder();
 bool make_tmap(CUtensorMap* out, const void* base, int eb, int64_t cols, int64_t rows, int64_t batches,
                int64_t row_pitch_elems, int64_t batch_pitch_elems, int box_rows);
 
-template <int BN0, int BN1, bool A_MN, bool B_MN, int EB, int STAGES, class Epi>
+int sm_count();
+
+// persistent = true: at most (SMs x resident CTAs per SM) CTAs loop over the tiles;
+// otherwise one CTA per tile.
+template <int BN0, int BN1, bool A_MN, bool B_MN, int EB, int STAGES, int EW = 4, class Epi>
 cudaError_t launch_tc_gemm(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
                            const CUtensorMap& b1, const TcGeom& g, const Epi& epi, unsigned* status,
-                           cudaStream_t st) {
+                           cudaStream_t st, bool persistent = false) {
   using S = TcShape<BN0, BN1, EB, STAGES>;
   static_assert(MajorCheck<A_MN, B_MN, EB>::ok, "");
-  auto kern = tc_gemm_kernel<BN0, BN1, A_MN, B_MN, EB, STAGES, Epi>;
+  auto kern = tc_gemm_kernel<BN0, BN1, A_MN, B_MN, EB, STAGES, EW, Epi>;
   // TMEM holds 512 columns per SM: request enough shared memory that the CTAs
   // resident on one SM never ask for more columns than exist (an allocation
   // beyond that would stall until a neighbour frees its columns).
@@ -279,16 +334,21 @@ cudaError_t launch_tc_gemm(const CUtensorMap& a0, const CUtensorMap& b0, const C
   constexpr int kMinSmem = kSmemPerSM / (kMaxCtas + 1) - kReservedPerCta + 16;
   constexpr int kSmem = S::SMEM_BYTES > kMinSmem ? S::SMEM_BYTES : kMinSmem;
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
+  constexpr int kCtasPerSm = kSmemPerSM / (kSmem + kReservedPerCta) < kMaxCtas
+                                 ? kSmemPerSM / (kSmem + kReservedPerCta)
+                                 : kMaxCtas;
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  if (g.batches * g.splits > 65535 || g.n_tiles > 65535) return cudaErrorInvalidConfiguration;
-  dim3 grid(g.m_tiles0 + g.m_tiles1, g.n_tiles, g.batches * g.splits);
-  if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
-  kern<<<grid, 192, kSmem, st>>>(a0, b0, a1, b1, g, epi, status);
+  const long long total = static_cast<long long>(g.m_tiles0 + g.m_tiles1) * g.n_tiles * g.batches * g.splits;
+  if (total <= 0) return cudaSuccess;
+  if (total > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  long long grid = total;
+  if (persistent) grid = std::min<long long>(total, static_cast<long long>(sm_count()) * (kCtasPerSm > 0 ? kCtasPerSm : 1));
+  kern<<<static_cast<unsigned>(grid), 64 + 32 * EW, kSmem, st>>>(a0, b0, a1, b1, g, epi, status);
   return cudaGetLastError();
 }
 

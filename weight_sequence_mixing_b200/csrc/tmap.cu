@@ -16,6 +16,17 @@ PFN_tmapEncodeTiled tmap_encoder() {
   return fn;
 }
 
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        n <= 0)
+      n = 148;
+  }
+  return n;
+}
+
 bool make_tmap(CUtensorMap* out, const void* base, int eb, int64_t cols, int64_t rows, int64_t batches,
                int64_t row_pitch_elems, int64_t batch_pitch_elems, int box_rows) {
   PFN_tmapEncodeTiled enc = tmap_encoder();
