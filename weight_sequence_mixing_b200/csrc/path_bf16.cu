@@ -20,6 +20,7 @@
 #include <algorithm>
 
 #include "epilogues.cuh"
+#include "token_phase.cuh"
 #include "ttt_plan.cuh"
 
 namespace ttt {
@@ -486,6 +487,36 @@ int optimizer_step(Ctx& c) {
   return TTT_OK;
 }
 
+// Token phase of the negative-dot update: activations H' and dZ(13) of chunk
+// tokens [t0, t0+n) for the weight-gradient GEMMs (token_phase.cuh).
+int token_phase(Ctx& c, const TM& tX, int xoff, int t0, int n, bf16* Hp, bf16* dZ, bool swiglu) {
+  const Dims& D = c.D;
+  const int Z = D.Z, d = D.d, h = D.h, Cp = D.Cp;
+  const int dzc = swiglu ? 2 * h : h;
+  CUtensorMap sH, sD;
+  if (!make_tmap_ex(&sH, Hp, 2, h, Cp, Z, h, int64_t(Cp) * h, 32, 32, 64) ||
+      !make_tmap_ex(&sD, dZ, 2, dzc, Cp, Z, dzc, int64_t(Cp) * dzc, 32, 32, 64))
+    return TTT_ERR_INVALID_ARG;
+  const int bz = swiglu ? 256 : 128;
+  if (tX.box != 128 || c.tV.box != 128 || c.tW2T.box != 128 || c.tFirst.box != bz) return TTT_ERR_INVALID_ARG;
+  TokGeom g;
+  g.m_tiles = Cp / 128;
+  g.n_tiles = h / 128;
+  g.batches = Z;
+  g.kblocks = d / 64;
+  g.x_off = xoff;
+  g.v_off = t0;
+  g.rows_valid = n;
+  g.t0 = t0;
+  g.eta = c.io.eta;
+  g.eta_zs = D.N;
+  g.eta_scalar = c.p.cfg.eta_scalar;
+  StageScope sc(kStageTokenPhase, c.st);
+  const cudaError_t e = swiglu ? launch_token_dot<true>(tX.m, c.tFirst.m, c.tV.m, c.tW2T.m, sH, sD, g, c.v.status, c.st)
+                               : launch_token_dot<false>(tX.m, c.tFirst.m, c.tV.m, c.tW2T.m, sH, sD, g, c.v.status, c.st);
+  return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+
 // one chunk's weight update: tokens [t0, t0+n)
 int update_chunk(Ctx& c, int t0, int n) {
   cudaStream_t st = c.st;
@@ -527,12 +558,8 @@ int update_chunk(Ctx& c, int t0, int n) {
 
   StageCtx stage(kStageTokenPhase);
   if (cfg.inner == TTT_INNER_SWIGLU) {
-    // token phase: [z1 | z3] = X [W1;W3]_blk^T, p = V W2[:, blk]  -> H', dZ13
-    EpiTokenDot<true> e{A0, A1, h, n, int64_t(Cp) * h, int64_t(Cp) * 2 * h, c.io.eta, D.N, t0, cfg.eta_scalar};
-    TcGeom g = geom(mt, 0, h / 128, d / 64, Z, 1);
-    g.a0.mn = xoff;
-    g.a1.mn = t0;
-    TRY((gemm<256, 128, false, false, 2, 2, 8>(*tX, c.tFirst, c.tV, c.tW2T, g, e, status, c.st, true)));
+    // token phase: p = V W2[:, blk], [z1 | z3] = X [W1;W3]_blk^T  -> H', dZ13
+    TRY(token_phase(c, *tX, xoff, t0, n, A0, A1, true));
     // weight gradients: G2^T = H'^T V  (rows [0,h)),  G13 = dZ13^T X  (rows [h, 3h))
     TM tH, tD;
     TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
@@ -546,11 +573,7 @@ int update_chunk(Ctx& c, int t0, int n) {
     else if (bnd == 128) TRY((gemm<128, 0, true, true, 2, 6>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st)));
     else TRY((gemm<64, 0, true, true, 2, 4>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st)));
   } else if (cfg.inner == TTT_INNER_MLP2_GELU && cfg.loss == TTT_LOSS_NEG_DOT) {
-    EpiTokenDot<false> e{A0, A1, h, n, int64_t(Cp) * h, int64_t(Cp) * h, c.io.eta, D.N, t0, cfg.eta_scalar};
-    TcGeom g = geom(mt, 0, h / 128, d / 64, Z, 1);
-    g.a0.mn = xoff;
-    g.a1.mn = t0;
-    TRY((gemm<128, 128, false, false, 2, 3, 8>(*tX, c.tFirst, c.tV, c.tW2T, g, e, status, c.st, true)));
+    TRY(token_phase(c, *tX, xoff, t0, n, A0, A1, false));
     TM tH, tD;
     TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
     TRY(tmap(&tD, A1, 2, h, Cp, Z, 64));

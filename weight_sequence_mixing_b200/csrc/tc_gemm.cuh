@@ -314,6 +314,9 @@ PFN_tmapEncodeTiled tmap_encoder();
 // Returns false when the view violates a TMA rule (alignment, pitch, extent).
 bool make_tmap(CUtensorMap* out, const void* base, int eb, int64_t cols, int64_t rows, int64_t batches,
                int64_t row_pitch_elems, int64_t batch_pitch_elems, int box_rows);
+// General form: box {box_cols, box_rows}, swizzle span 32 / 64 / 128 bytes (box_cols * eb <= span).
+bool make_tmap_ex(CUtensorMap* out, const void* base, int eb, int64_t cols, int64_t rows, int64_t batches,
+                  int64_t row_pitch_elems, int64_t batch_pitch_elems, int box_cols, int box_rows, int swizzle);
 
 int sm_count();
 
