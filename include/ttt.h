@@ -126,6 +126,31 @@ int ttt_forward_host(ttt_handle* handle, const void* Q, const void* K, const voi
                      const float* W0, void* O, float* W_out, void* device_staging, size_t staging_bytes,
                      void* workspace, size_t workspace_bytes, void* stream);
 
+/* The same pass for callers that cannot allocate device memory (a host framework
+ * that owns every allocation, a latency-critical path where cudaMalloc could stall
+ * the device, code running while a CUDA graph that must stay allocation-free is
+ * being captured).  The pages have no counterpart of this call: it is a property
+ * of this library, not of the layer.
+ *   - The workspace is the library's own static device array of
+ *     TTT_NOALLOC_SCRATCH_BYTES (32 MiB).  Every GPU that loads the library holds
+ *     that array until the process exits.  A layer whose ttt_workspace_size is
+ *     larger is rejected with TTT_ERR_WORKSPACE before anything is enqueued.
+ *   - The call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ *     routine).  The caller passes inputs and outputs exactly as for ttt_forward.
+ *   - The first call on a device looks up the address of that device's array with
+ *     that device current; make that first call before any stream capture begins.
+ *   - Every call on a device shares the one array.  Each call clears what must
+ *     start at zero, but calls whose GPU work overlaps (other streams, other host
+ *     threads) race on the array: serialise them.
+ *   - status_out (optional, device memory, 4 bytes) receives the device status
+ *     bits of this call after it completes on `stream`: 0 = ok, bit 0 = non-finite
+ *     values in O or W*, bit 1 = a bounded device wait ran out.
+ *   - Calls through this entry are not counted or timed by the ttt_profile_* hooks.
+ * Returns TTT_OK or a negative status; enqueue only, like ttt_forward. */
+#define TTT_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int ttt_forward_noalloc(ttt_handle* handle, const void* Q, const void* K, const void* V, const float* eta,
+                        const float* W0, void* O, float* W_out, unsigned* status_out, void* stream);
+
 /* Synchronise `stream`, read the device status word of `workspace` and clear
  * it.  Returns TTT_OK, TTT_ERR_NONFINITE, TTT_ERR_TIMEOUT or TTT_ERR_CUDA. */
 int ttt_query_status(ttt_handle* handle, void* workspace, void* stream);

@@ -33,6 +33,7 @@ EXPORTED = [
     "ttt_config_init", "ttt_create", "ttt_param_count", "ttt_workspace_size", "ttt_forward",
     "ttt_host_staging_size", "ttt_forward_host", "ttt_query_status", "ttt_destroy", "ttt_status_string",
     "ttt_selftest_gemm", "ttt_profile_enable", "ttt_profile_collect", "ttt_stage_name", "ttt_launch_count",
+    "ttt_forward_noalloc",
 ]
 NUM_STAGES = 8
 
@@ -76,6 +77,7 @@ def _load():
         "ttt_profile_collect": (i32, [vp, i32, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]),
         "ttt_stage_name": (ctypes.c_char_p, [i32]),
         "ttt_launch_count": (i64, [vp]),
+        "ttt_forward_noalloc": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -180,6 +182,12 @@ class TTTLayer:
 
     def check_status(self, stream=None):
         _check(LIB.ttt_query_status(self._handle, _ptr(self.workspace), _stream_ptr(stream)), "device status")
+
+    def forward_noalloc(self, Q, K, V, eta, W0, O, W_out=None, status=None, stream=None):
+        """The layer without a workspace argument: the library's own static device
+        scratch stands in for it (for callers that cannot allocate; see ttt.h)."""
+        _check(LIB.ttt_forward_noalloc(self._handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W0), _ptr(O),
+                                       _ptr(W_out), _ptr(status), _stream_ptr(stream)), "ttt_forward_noalloc")
 
     # ---- per-stage device timing (CUDA events around every launch, on its stream)
     def profile(self, on: bool):
