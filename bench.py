@@ -248,12 +248,15 @@ def main():
 
     from weight_sequence_mixing_b200 import binding
 
+    # a dedicated stream: ttt_forward replays a cached CUDA graph of its launches on
+    # any stream but the legacy default one
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
     x = gen_inputs(cfg)
     dev = {k: (v.cuda() if v is not None else None) for k, v in x.items()}
     layer = binding.TTTLayer(cfg)
     O = torch.empty((cfg["B"], cfg["H"], cfg["Nq"], cfg["d"]), dtype=layer.io_dtype, device="cuda")
     W = torch.empty((cfg["B"], cfg["H"], layer.P), dtype=torch.float32, device="cuda")
-    stream = torch.cuda.current_stream()
 
     h2d, d2h = io_bytes(cfg)
     in_bytes = h2d
@@ -263,6 +266,7 @@ def main():
     def step():
         layer.forward(dev["Q"], dev["K"], dev["V"], dev["eta"], dev["W0"], O=O, W_out=W, check=False)
 
+    layer.profile(True)  # per-stage events are part of the captured graphs: warm up with them on
     for _ in range(args.warmup):
         step()
     layer.check_status()
@@ -272,7 +276,7 @@ def main():
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     launches0 = layer.launch_count()
-    layer.profile(True)
+    layer.profile(True)  # clears the warm-up's stage times
     if dist:
         dist.barrier()
     torch.cuda.synchronize()

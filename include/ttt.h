@@ -73,6 +73,7 @@ typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
 
 #define TTT_FLAG_KEY_INSTNORM 1u  /* normalise each key channel over the chunk's tokens */
 #define TTT_FLAG_WEIGHT_L2NORM 2u /* unit L2 norm for every weight row after each update */
+#define TTT_FLAG_DIRECT_LAUNCH 4u /* launch every kernel on each call instead of replaying a cached CUDA graph */
 
 typedef struct ttt_config {
   int32_t B, H;       /* batch entries and heads */
@@ -112,7 +113,12 @@ size_t ttt_workspace_size(const ttt_handle* handle);
 /* Enqueue one TTT-layer forward pass on `stream` (a cudaStream_t; NULL = legacy
  * default stream).  All pointers are device pointers.  eta may be NULL (then
  * cfg.eta_scalar is every token's rate); W_out may be NULL.  O and W_out are
- * fully overwritten.  Returns without waiting for the GPU. */
+ * fully overwritten.  Returns without waiting for the GPU.
+ * On a non-NULL stream that is not being captured, the first call with a given
+ * set of pointers captures the pass into a CUDA graph that later calls with the
+ * same pointers replay (at most 8 pointer sets are kept per handle; the handle
+ * owns the graphs).  TTT_FLAG_DIRECT_LAUNCH turns this off; a stream the caller
+ * is capturing gets the kernels themselves. */
 int ttt_forward(ttt_handle* handle, const void* Q, const void* K, const void* V, const float* eta,
                 const float* W0, void* O, float* W_out, void* workspace, size_t workspace_bytes,
                 void* stream);

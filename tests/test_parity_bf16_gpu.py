@@ -99,3 +99,33 @@ def test_full_size_workload(name):
     errs = compare(cfg, heads=heads)
     print(name, {k: f"{v:.2e}" for k, v in errs.items()})
     _check(errs)
+
+
+@pytest.mark.parametrize("profiled", [False, True])
+def test_graph_replay_matches_direct_launch(profiled):
+    # on a non-default stream ttt_forward captures its launches into a CUDA graph on the
+    # first call and replays it afterwards (two alternating instances when profiling);
+    # every replay must give the bits the direct launches give.
+    from weight_sequence_mixing_b200 import binding
+    kw = dict(B=1, H=2, N=640, chunk=256, Nq=300, d=128, h=256, inner="swiglu", loss="neg_dot",
+              opt="momentum_muon", weight_l2norm=True, dtype="bf16", data="lact", eta_mode="per_token", seed=8)
+    x = gen_inputs(make_config(**kw))
+    d = {k: (v.cuda() if v is not None else None) for k, v in x.items()}
+    direct = binding.TTTLayer(make_config(direct_launch=True, **kw))
+    O0, W0 = direct.forward(d["Q"], d["K"], d["V"], d["eta"], d["W0"])
+    side = torch.cuda.Stream()
+    layer = binding.TTTLayer(make_config(**kw))
+    if profiled:
+        layer.profile(True)
+    O = torch.empty_like(O0)
+    W = torch.empty_like(W0)
+    with torch.cuda.stream(side):
+        for _ in range(4):
+            O.fill_(float("nan"))
+            layer.forward(d["Q"], d["K"], d["V"], d["eta"], d["W0"], O=O, W_out=W, stream=side)
+            assert torch.equal(O, O0) and torch.equal(W, W0)
+    side.synchronize()
+    if profiled:
+        stages = layer.profile_collect()
+        assert stages["token_phase"][1] == 4 * 3 and stages["newton_schulz"][1] > 0
+        assert all(ms > 0 for ms, _ in stages.values())

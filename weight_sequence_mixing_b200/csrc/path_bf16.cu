@@ -20,6 +20,7 @@
 #include <algorithm>
 
 #include "epilogues.cuh"
+#include "ns_fused.cuh"
 #include "token_phase.cuh"
 #include "ttt_plan.cuh"
 
@@ -43,7 +44,7 @@ enum BBuf {
   xAct2,   // bf16 [Z][Cp][h]  (GELU' for MSE)
   xDY,     // bf16 [Z][Cp][d]  (dL/dV_hat for MSE / linear)
   xHq,     // bf16 apply hidden [Z][Rq][h]
-  xNX, xNXT, xNX2, xNXT2, xNS, xNT,  // fp32 Newton-Schulz buffers [Z*nmat][...]
+  xNX, xNXT, xNX2, xNXT2, xNS, xNT, xNS2,  // fp32 Newton-Schulz buffers [Z*nmat][...]
   kNumBBuf
 };
 
@@ -445,34 +446,28 @@ int optimizer_step(Ctx& c) {
       ns_prep_kernel<<<g, 256, 0, c.st>>>(c.rm, D.nmat, c.v.at<float>(p, xU), c.v.at<float>(p, xInvN), A, B);
     }
     TRY_CUDA(cudaGetLastError());
-    float* X2 = c.v.at<float>(p, xNX2);
-    float* XT2 = c.v.at<float>(p, xNXT2);
-    float* S = c.v.at<float>(p, xNS);
-    float* T = c.v.at<float>(p, xNT);
-    const int m = D.m, n = D.n;
-    TM tS, tT;
-    TRY(tmap(&tS, S, 4, m, m, ZK, 128));
-    TRY(tmap(&tT, T, 4, m, m, ZK, 128));
-    const float a = cfg.ns_coeff[0], b = cfg.ns_coeff[1], cc = cfg.ns_coeff[2];
-    StageCtx stage(kStageNewtonSchulz);
-    for (int it = 0; it < cfg.ns_iters; ++it) {
-      TM tX, tXT;
-      TRY(tmap(&tX, X, 4, n, m, ZK, 128));
-      TRY(tmap(&tXT, XT, 4, m, n, ZK, 128));
-      // S = X X^T
-      EpiStoreF32 e1{S, m, m, int64_t(m) * m};
-      TRY((gemm<128, 0, false, false, 4, 4>(tX, tX, tX, tX, geom(m / 128, 0, m / 128, n / 32, ZK, 1),
-                                                          e1, c.v.status, c.st)));
-      // T = b S + c S S   (S symmetric: S^T = S serves as the K-major B operand)
-      EpiNsPoly e2{T, S, m, m, int64_t(m) * m, b, cc};
-      TRY((gemm<128, 0, false, false, 4, 4>(tS, tS, tS, tS, geom(m / 128, 0, m / 128, m / 32, ZK, 1),
-                                                          e2, c.v.status, c.st)));
-      // X' = a X + T X  (B operand X^T [n][m] is K-major); stores X' and X'^T
-      EpiNsUpdate e3{X2, XT2, X, m, n, int64_t(m) * n, a};
-      TRY((gemm<128, 0, false, false, 4, 4>(tT, tXT, tT, tXT, geom(m / 128, 0, n / 128, m / 32, ZK, 1),
-                                                          e3, c.v.status, c.st)));
-      std::swap(X, X2);
-      std::swap(XT, XT2);
+    // all Newton-Schulz iterations of every matrix in one clustered launch
+    NsGeom ng;
+    ng.m = D.m;
+    ng.n = D.n;
+    ng.iters = cfg.ns_iters;
+    ng.a = cfg.ns_coeff[0];
+    ng.b = cfg.ns_coeff[1];
+    ng.c = cfg.ns_coeff[2];
+    ng.X = X;
+    ng.XT = XT;
+    ng.X2 = c.v.at<float>(p, xNX2);
+    ng.XT2 = c.v.at<float>(p, xNXT2);
+    ng.S = c.v.at<float>(p, xNS);
+    ng.T = c.v.at<float>(p, xNT);
+    ng.S2 = c.v.at<float>(p, xNS2);
+    {
+      StageScope sc(kStageNewtonSchulz, st);
+      TRY_CUDA(launch_ns_fused(ZK, ng, c.v.status, st));
+    }
+    if (cfg.ns_iters & 1) {
+      X = ng.X2;
+      XT = ng.XT2;
     }
   }
   dim3 g((c.rm.nrows() + 7) / 8, D.Z);
@@ -569,9 +564,9 @@ int update_chunk(Ctx& c, int t0, int n) {
     gg.b0.k = t0;
     gg.b1.k = xoff;
     EpiPartial ep{part, ps, pz, d, {0, h}, {h, 2 * h}};
-    if (bnd == 256) TRY((gemm<256, 0, true, true, 2, 4>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st)));
-    else if (bnd == 128) TRY((gemm<128, 0, true, true, 2, 6>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st)));
-    else TRY((gemm<64, 0, true, true, 2, 4>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st)));
+    if (bnd == 256) TRY((gemm<256, 0, true, true, 2, 4, 8>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st, true)));
+    else if (bnd == 128) TRY((gemm<128, 0, true, true, 2, 6, 8>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st, true)));
+    else TRY((gemm<64, 0, true, true, 2, 4, 8>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st, true)));
   } else if (cfg.inner == TTT_INNER_MLP2_GELU && cfg.loss == TTT_LOSS_NEG_DOT) {
     TRY(token_phase(c, *tX, xoff, t0, n, A0, A1, false));
     TM tH, tD;
@@ -582,9 +577,9 @@ int update_chunk(Ctx& c, int t0, int n) {
     gg.b0.k = t0;
     gg.b1.k = xoff;
     EpiPartial ep{part, ps, pz, d, {0, h}, {h, h}};
-    if (bnd == 256) TRY((gemm<256, 0, true, true, 2, 4>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st)));
-    else if (bnd == 128) TRY((gemm<128, 0, true, true, 2, 6>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st)));
-    else TRY((gemm<64, 0, true, true, 2, 4>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st)));
+    if (bnd == 256) TRY((gemm<256, 0, true, true, 2, 4, 8>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st, true)));
+    else if (bnd == 128) TRY((gemm<128, 0, true, true, 2, 6, 8>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st, true)));
+    else TRY((gemm<64, 0, true, true, 2, 4, 8>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st, true)));
   } else if (cfg.inner == TTT_INNER_MLP2_GELU) {  // MSE
     // Z = X W1^T -> H = GELU(Z), G' = GELU'(Z)
     EpiGeluSave e1{A0, A2, h, n, int64_t(Cp) * h};
@@ -615,9 +610,9 @@ int update_chunk(Ctx& c, int t0, int n) {
     TcGeom gg = geom(h / 128, h / 128, d / bnd, kbt, Z, D.splits);
     gg.b1.k = xoff;
     EpiPartial ep{part, ps, pz, d, {0, h}, {h, h}};
-    if (bnd == 256) TRY((gemm<256, 0, true, true, 2, 4>(tH, tYmn, tD, *tXmn, gg, ep, status, c.st)));
-    else if (bnd == 128) TRY((gemm<128, 0, true, true, 2, 6>(tH, tYmn, tD, *tXmn, gg, ep, status, c.st)));
-    else TRY((gemm<64, 0, true, true, 2, 4>(tH, tYmn, tD, *tXmn, gg, ep, status, c.st)));
+    if (bnd == 256) TRY((gemm<256, 0, true, true, 2, 4, 8>(tH, tYmn, tD, *tXmn, gg, ep, status, c.st, true)));
+    else if (bnd == 128) TRY((gemm<128, 0, true, true, 2, 6, 8>(tH, tYmn, tD, *tXmn, gg, ep, status, c.st, true)));
+    else TRY((gemm<64, 0, true, true, 2, 4, 8>(tH, tYmn, tD, *tXmn, gg, ep, status, c.st, true)));
   } else {  // linear
     if (cfg.loss == TTT_LOSS_MSE) {
       EpiMseGrad e2{DY, d, n, int64_t(Cp) * d, V, int64_t(D.N) * d, t0, c.io.eta, D.N, cfg.eta_scalar,
@@ -641,9 +636,9 @@ int update_chunk(Ctx& c, int t0, int n) {
     TcGeom gg = geom(d / 128, 0, d / bnd, kbt, Z, D.splits);
     gg.b0.k = xoff;
     EpiPartial ep{part, ps, pz, d, {0, 0}, {d, 0}};
-    if (bnd == 256) TRY((gemm<256, 0, true, true, 2, 4>(tYmn, *tXmn, tYmn, *tXmn, gg, ep, status, c.st)));
-    else if (bnd == 128) TRY((gemm<128, 0, true, true, 2, 6>(tYmn, *tXmn, tYmn, *tXmn, gg, ep, status, c.st)));
-    else TRY((gemm<64, 0, true, true, 2, 4>(tYmn, *tXmn, tYmn, *tXmn, gg, ep, status, c.st)));
+    if (bnd == 256) TRY((gemm<256, 0, true, true, 2, 4, 8>(tYmn, *tXmn, tYmn, *tXmn, gg, ep, status, c.st, true)));
+    else if (bnd == 128) TRY((gemm<128, 0, true, true, 2, 6, 8>(tYmn, *tXmn, tYmn, *tXmn, gg, ep, status, c.st, true)));
+    else TRY((gemm<64, 0, true, true, 2, 4, 8>(tYmn, *tXmn, tYmn, *tXmn, gg, ep, status, c.st, true)));
   }
   return optimizer_step(c);
 }
@@ -698,7 +693,8 @@ int choose_splits(const Plan& p, int Cp) {
   const int rows = c.inner == TTT_INNER_LINEAR ? d : c.inner == TTT_INNER_MLP2_GELU ? 2 * h : 3 * h;
   const int tiles = rows / 128 * (d / bnd) * p.BH;
   const int kblocks = Cp / 64;
-  int s = std::max(1, (4 * 148 + tiles - 1) / tiles);
+  // about two waves of CTAs: long K ranges per split, few partials to reduce
+  int s = std::max(1, (2 * 148 + tiles / 2) / tiles);
   s = std::min(s, std::max(1, kblocks / 4));
   s = std::min(s, 64);
   // every split must own at least one k-block
@@ -744,6 +740,7 @@ int plan_layout_bf16(Plan* p) {
       muon ? ZK * nm * 4 : 0,
       muon ? ZK * nm * 4 : 0,
       muon ? ZK * nm * 4 : 0,
+      muon ? ZK * mm * 4 : 0,
       muon ? ZK * mm * 4 : 0,
       muon ? ZK * mm * 4 : 0,
   };

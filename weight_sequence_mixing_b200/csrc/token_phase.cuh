@@ -232,18 +232,37 @@ __global__ void __launch_bounds__(64 + 32 * TokShape<SWIGLU>::EW, 1)
           if (lane == 0) mbar_arrive(tmem_empty);
         }
         float hv[32], d1[32], d3[32];
+        if constexpr (SWIGLU) {
+          // pairs of columns with the paired fp32 instructions:
+          //   s = SiLU gate sigma(z1) = (1 + tanh(z1/2))/2, a = z1 s, dh = -eta p
+          //   H' = -eta a z3, dZ3 = dh a, dZ1 = dh z3 s (1 + z1 (1 - s))
+          const float2 ne = make_float2(-e, -e), half = make_float2(0.5f, 0.5f), one = make_float2(1.0f, 1.0f),
+                       mone = make_float2(-1.0f, -1.0f);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float z1 = __uint_as_float(r1[i]);
-          const float dh = -e * __uint_as_float(rp[i]);
-          if constexpr (SWIGLU) {
-            const float z3 = __uint_as_float(r3[i]);
-            const float sg = sigmoid_dev(z1);
-            const float a = z1 * sg;
-            hv[i] = -e * a * z3;
-            d3[i] = dh * a;
-            d1[i] = dh * z3 * sg * (1.0f + z1 * (1.0f - sg));
-          } else {
+          for (int i = 0; i < 32; i += 2) {
+            const float2 z1 = make_float2(__uint_as_float(r1[i]), __uint_as_float(r1[i + 1]));
+            const float2 z3 = make_float2(__uint_as_float(r3[i]), __uint_as_float(r3[i + 1]));
+            const float2 p = make_float2(__uint_as_float(rp[i]), __uint_as_float(rp[i + 1]));
+            const float2 hz = mul2(half, z1);
+            const float2 sg = fma2(half, make_float2(tanh_approx(hz.x), tanh_approx(hz.y)), half);
+            const float2 a = mul2(z1, sg);
+            const float2 dh = mul2(ne, p);
+            const float2 h = mul2(mul2(ne, a), z3);
+            const float2 g3 = mul2(dh, a);
+            const float2 u = fma2(z1, fma2(sg, mone, one), one);
+            const float2 g1 = mul2(mul2(dh, z3), mul2(sg, u));
+            hv[i] = h.x;
+            hv[i + 1] = h.y;
+            d3[i] = g3.x;
+            d3[i + 1] = g3.y;
+            d1[i] = g1.x;
+            d1[i + 1] = g1.y;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float z1 = __uint_as_float(r1[i]);
+            const float dh = -e * __uint_as_float(rp[i]);
             hv[i] = -e * gelu_dev(z1);
             d1[i] = dh * gelu_grad_dev(z1);
             d3[i] = 0.0f;
