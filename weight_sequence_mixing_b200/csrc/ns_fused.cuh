@@ -2,10 +2,9 @@
 // memory complements local attention") of a batch of m x n matrices (m <= n), all
 // iterations in one launch:
 //   for it in iters:  S = X X^T;  T = b S + c S S;  X <- a X + T X
-// computed as three plain products, with the polynomial folded into the operands
-// (the epilogues then read nothing from memory):
-//   S = X X^T  (also written as S' = c S + b I);   T' = S S' + a I;   X <- T' X
-// since b S + c S S = S (c S + b I) and a X + T X = (T + a I) X.
+// The fp32 terms b S and a X are added in the epilogues at full precision; the
+// producer prefetches the S or X tile they need into shared memory with TMA while
+// the tile's MMAs run, so the epilogue does not wait on global memory.
 // One thread-block cluster of CS CTAs owns one matrix.  Each step is cut into
 // 128 x 128 output tiles dealt round-robin to the cluster's CTAs and computed on
 // the tf32 tensor cores (fp32 storage, fp32 accumulation in TMEM, two accumulator
@@ -25,13 +24,14 @@ namespace ttt {
 struct NsGeom {
   int m, n, iters;
   float a, b, c;
-  // fp32 buffers, per matrix strides m*n (X, XT, X2, XT2) and m*m (S, S', T')
-  float *X, *XT, *X2, *XT2, *S, *T, *S2;
+  // fp32 buffers, per matrix strides m*n (X, XT, X2, XT2) and m*m (S, T)
+  float *X, *XT, *X2, *XT2, *S, *T;
 };
 
 constexpr int kNsStages = 4;
 constexpr int kNsStage = 2 * 128 * 128;  // A + B tile of 32 fp32 (128 B) per row
-constexpr int kNsSmem = 1024 + kNsStages * kNsStage + 256;
+constexpr int kNsEbuf = 4 * 128 * 128;   // one 128 x 128 fp32 epilogue operand tile (4 boxes of 32 cols)
+constexpr int kNsSmem = 1024 + kNsStages * kNsStage + kNsEbuf + 256;
 
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
@@ -56,7 +56,7 @@ struct NsStep {
 
 __device__ __forceinline__ NsStep ns_step(int step, int it, const NsGeom& g, const CUtensorMap* mX,
                                           const CUtensorMap* mXT, const CUtensorMap* mX2, const CUtensorMap* mXT2,
-                                          const CUtensorMap* mS, const CUtensorMap* mT, const CUtensorMap* mS2) {
+                                          const CUtensorMap* mS, const CUtensorMap* mT) {
   const bool odd = it & 1;
   const CUtensorMap* cx = odd ? mX2 : mX;
   const CUtensorMap* cxt = odd ? mXT2 : mXT;
@@ -68,13 +68,13 @@ __device__ __forceinline__ NsStep ns_step(int step, int it, const NsGeom& g, con
     s.tiles_n = tm;
     s.tiles = tm * tm;
     s.kblocks = g.n / 32;
-  } else if (step == 1) {  // S S'  (S' symmetric: its rows are the K-major B operand), K = m
+  } else if (step == 1) {  // S S  (S symmetric: its rows are the K-major B operand), K = m
     s.A = mS;
-    s.B = mS2;
+    s.B = mS;
     s.tiles_n = tm;
     s.tiles = tm * tm;
     s.kblocks = g.m / 32;
-  } else {  // T' X  (A = T' rows, B = X^T rows [n][m]), K = m
+  } else {  // T X  (A = T rows, B = X^T rows [n][m]), K = m
     s.A = mT;
     s.B = cxt;
     s.tiles_n = tn;
@@ -88,16 +88,19 @@ template <int CS>
 __global__ void __launch_bounds__(192, 1)
     ns_fused_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mXT,
                     const __grid_constant__ CUtensorMap mX2, const __grid_constant__ CUtensorMap mXT2,
-                    const __grid_constant__ CUtensorMap mS, const __grid_constant__ CUtensorMap mT,
-                    const __grid_constant__ CUtensorMap mS2, const NsGeom g, unsigned* status) {
+                    const __grid_constant__ CUtensorMap mS, const __grid_constant__ CUtensorMap mT, const NsGeom g,
+                    unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kNsStages * kNsStage);
+  uint8_t* ebuf = smem + kNsStages * kNsStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ebuf + kNsEbuf);
   uint64_t* empty = full + kNsStages;
   uint64_t* tmem_full = empty + kNsStages;  // [2]: accumulator buffer b holds tile j when j % 2 == b
   uint64_t* tmem_empty = tmem_full + 2;     // [2]
   uint64_t* drain = tmem_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* efull = drain + 1;   // epilogue operand tile landed
+  uint64_t* eempty = efull + 1;  // epilogue done with it
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(eempty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -116,6 +119,8 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(&tmem_empty[0], 4);
     mbar_init(&tmem_empty[1], 4);
     mbar_init(drain, 1);
+    mbar_init(efull, 1);
+    mbar_init(eempty, 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -130,12 +135,14 @@ __global__ void __launch_bounds__(192, 1)
 
   int it_ring = 0;  // producer / MMA position in the smem ring (lane 0 of warps 0 and 1)
   int j_tile = 0;   // tiles this CTA has computed (TMEM phases)
+  int e_use = 0;    // epilogue operand tiles loaded (producer) / consumed (epilogue)
   for (int it = 0; it < g.iters; ++it) {
     for (int step = 0; step < 3; ++step) {
-      const NsStep sp = ns_step(step, it, g, &mX, &mXT, &mX2, &mXT2, &mS, &mT, &mS2);
+      const NsStep sp = ns_step(step, it, g, &mX, &mXT, &mX2, &mXT2, &mS, &mT);
       if (warp == 0) {
         if (lane == 0 && !*abort_flag) {
           fence_proxy_async_global();  // the previous step's generic stores -> these TMA loads
+          const CUtensorMap* eop = step == 1 ? &mS : ((it & 1) ? &mX2 : &mX);  // S for T, X for X'
           for (int t = rank; t < sp.tiles && !*abort_flag; t += CS) {
             const int r0 = (t / sp.tiles_n) * 128, c0 = (t % sp.tiles_n) * 128;
             for (int kb = 0; kb < sp.kblocks; ++kb, ++it_ring) {
@@ -146,6 +153,14 @@ __global__ void __launch_bounds__(192, 1)
               mbar_arrive_expect_tx(&full[s], kNsStage);
               tma_load_3d(st, sp.A, &full[s], kb * 32, r0, zk);
               tma_load_3d(st + 128 * 128, sp.B, &full[s], kb * 32, c0, zk);
+            }
+            // after the tile's operands (so waiting for the previous epilogue never holds
+            // them back): the fp32 tile its epilogue adds, S for T = b S + c S S, X for a X + T X
+            if (step > 0 && !*abort_flag) {
+              if (e_use > 0 && !mbar_wait(eempty, (e_use - 1) & 1, abort_flag)) break;
+              mbar_arrive_expect_tx(efull, kNsEbuf);
+              for (int bx = 0; bx < 4; ++bx) tma_load_3d(ebuf + bx * 128 * 128, eop, efull, c0 + 32 * bx, r0, zk);
+              ++e_use;
             }
           }
         }
@@ -192,26 +207,47 @@ __global__ void __launch_bounds__(192, 1)
           float* nx = odd ? g.X : g.X2;  // X of the next iteration
           float* nxt = odd ? g.XT : g.XT2;
           const uint32_t tacc = taddr + static_cast<uint32_t>(buf * 128);
+          const int lrow = q * 32 + lane;  // row inside the tile (and the prefetched box)
+          if (step > 0) {
+            const bool landed = __all_sync(0xffffffffu, mbar_wait(efull, e_use & 1, abort_flag));
+            if (!landed) break;
+          }
 #pragma unroll 1
           for (int cc = 0; cc < 128; cc += 32) {
             float v[32];
             tmem_ld32(tacc + cc, v);
-            const int dcol = row - (c0 + cc);  // column of this row's diagonal element in the chunk
             if (step == 0) {
               store_f32x32(g.S + zk * mm + int64_t(row) * g.m + c0 + cc, v);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = g.c * v[i] + (i == dcol ? g.b : 0.0f);
-              store_f32x32(g.S2 + zk * mm + int64_t(row) * g.m + c0 + cc, v);
-            } else if (step == 1) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] += (i == dcol ? g.a : 0.0f);
-              store_f32x32(g.T + zk * mm + int64_t(row) * g.m + c0 + cc, v);
             } else {
-              store_f32x32(nx + zk * mn + int64_t(row) * g.n + c0 + cc, v);
-              float* colT = nxt + zk * mn + int64_t(c0 + cc) * g.m + row;
+              // the prefetched fp32 tile: box cc/32, row lrow, 16-byte chunk k at k ^ (lrow & 7)
+              const float4* box = reinterpret_cast<const float4*>(ebuf + (cc / 32) * 128 * 128 + lrow * 128);
+              float e[32];
 #pragma unroll
-              for (int i = 0; i < 32; ++i) colT[int64_t(i) * g.m] = v[i];  // coalesced across the warp
+              for (int k = 0; k < 8; ++k) {
+                const float4 f = box[k ^ (lrow & 7)];
+                e[4 * k] = f.x;
+                e[4 * k + 1] = f.y;
+                e[4 * k + 2] = f.z;
+                e[4 * k + 3] = f.w;
+              }
+              if (step == 1) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = g.b * e[i] + g.c * v[i];
+                store_f32x32(g.T + zk * mm + int64_t(row) * g.m + c0 + cc, v);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = g.a * e[i] + v[i];
+                store_f32x32(nx + zk * mn + int64_t(row) * g.n + c0 + cc, v);
+                float* colT = nxt + zk * mn + int64_t(c0 + cc) * g.m + row;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) colT[int64_t(i) * g.m] = v[i];  // coalesced across the warp
+              }
             }
+          }
+          if (step > 0) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(eempty);
+            ++e_use;
           }
           tc_fence_before();
           __syncwarp();
@@ -239,15 +275,14 @@ __global__ void __launch_bounds__(192, 1)
 // X: Newton-Schulz input (normalised) in g.X / g.XT; result in (g.iters odd ? X2 : X).
 template <int CS>
 cudaError_t launch_ns_fused_cs(int nmat, const NsGeom& g, unsigned* status, cudaStream_t st) {
-  CUtensorMap mX, mXT, mX2, mXT2, mS, mT, mS2;
+  CUtensorMap mX, mXT, mX2, mXT2, mS, mT;
   const int m = g.m, n = g.n;
   if (!make_tmap(&mX, g.X, 4, n, m, nmat, n, int64_t(m) * n, 128) ||
       !make_tmap(&mXT, g.XT, 4, m, n, nmat, m, int64_t(m) * n, 128) ||
       !make_tmap(&mX2, g.X2, 4, n, m, nmat, n, int64_t(m) * n, 128) ||
       !make_tmap(&mXT2, g.XT2, 4, m, n, nmat, m, int64_t(m) * n, 128) ||
       !make_tmap(&mS, g.S, 4, m, m, nmat, m, int64_t(m) * m, 128) ||
-      !make_tmap(&mT, g.T, 4, m, m, nmat, m, int64_t(m) * m, 128) ||
-      !make_tmap(&mS2, g.S2, 4, m, m, nmat, m, int64_t(m) * m, 128))
+      !make_tmap(&mT, g.T, 4, m, m, nmat, m, int64_t(m) * m, 128))
     return cudaErrorInvalidValue;
   auto kern = ns_fused_kernel<CS>;
   static bool configured = false;
@@ -272,7 +307,7 @@ cudaError_t launch_ns_fused_cs(int nmat, const NsGeom& g, unsigned* status, cuda
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, mX, mXT, mX2, mXT2, mS, mT, mS2, g, status);
+  return cudaLaunchKernelEx(&cfg, kern, mX, mXT, mX2, mXT2, mS, mT, g, status);
 }
 
 // Whether a cluster of CS CTAs of this kernel can be resident at all on this device.

@@ -44,7 +44,7 @@ enum BBuf {
   xAct2,   // bf16 [Z][Cp][h]  (GELU' for MSE)
   xDY,     // bf16 [Z][Cp][d]  (dL/dV_hat for MSE / linear)
   xHq,     // bf16 apply hidden [Z][Rq][h]
-  xNX, xNXT, xNX2, xNXT2, xNS, xNT, xNS2,  // fp32 Newton-Schulz buffers [Z*nmat][...]
+  xNX, xNXT, xNX2, xNXT2, xNS, xNT,  // fp32 Newton-Schulz buffers [Z*nmat][...]
   kNumBBuf
 };
 
@@ -460,7 +460,6 @@ int optimizer_step(Ctx& c) {
     ng.XT2 = c.v.at<float>(p, xNXT2);
     ng.S = c.v.at<float>(p, xNS);
     ng.T = c.v.at<float>(p, xNT);
-    ng.S2 = c.v.at<float>(p, xNS2);
     {
       StageScope sc(kStageNewtonSchulz, st);
       TRY_CUDA(launch_ns_fused(ZK, ng, c.v.status, st));
@@ -695,7 +694,9 @@ int choose_splits(const Plan& p, int Cp) {
   const int kblocks = Cp / 64;
   // about two waves of CTAs: long K ranges per split, few partials to reduce
   int s = std::max(1, (2 * 148 + tiles / 2) / tiles);
-  s = std::min(s, std::max(1, kblocks / 4));
+  // each split reduces at least 1024 tokens: below that the fp32 partials it writes
+  // and the reduction reads cost more than the parallelism gains
+  s = std::min(s, std::max(1, kblocks / 16));
   s = std::min(s, 64);
   // every split must own at least one k-block
   const int per = (kblocks + s - 1) / s;
@@ -740,7 +741,6 @@ int plan_layout_bf16(Plan* p) {
       muon ? ZK * nm * 4 : 0,
       muon ? ZK * nm * 4 : 0,
       muon ? ZK * nm * 4 : 0,
-      muon ? ZK * mm * 4 : 0,
       muon ? ZK * mm * 4 : 0,
       muon ? ZK * mm * 4 : 0,
   };
