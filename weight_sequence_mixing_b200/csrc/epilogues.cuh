@@ -128,6 +128,43 @@ struct EpiPartial {
   }
 };
 
+// Unsplit weight gradients straight into the optimizer state (no partials): for
+// gradient-layout row r and column n, U = beta M + G and M = U (momentum) or U = G,
+// and the squared row norms Muon needs (rowsq, zeroed beforehand; at most two
+// warps add to a row, so the sum does not depend on their order).
+struct EpiGradDirect {
+  float* U;
+  float* M;      // momentum buffer or null
+  float* rowsq;  // or null
+  float beta;
+  int64_t z_stride;  // elements per batch entry (GR * ld)
+  int ld;            // d
+  int row0[2], rows[2];
+  template <int BN0, int BN1>
+  __device__ void run(const EpiCtx& c) const {
+    const bool ok = c.m < rows[c.problem];
+    const int64_t off = c.z * z_stride + int64_t(row0[c.problem] + c.m) * ld + c.n0;
+    float sq = 0.0f;
+#pragma unroll 1
+    for (int cc = 32 * c.part; cc < BN0; cc += 32 * c.nparts) {
+      float v[32];
+      tmem_ld32(c.taddr + cc, v);
+      if (!ok || c.n0 + cc >= ld) continue;
+      if (M) {
+        float mv[32];
+        load_f32x32(M + off + cc, mv);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = beta * mv[j] + v[j];
+        store_f32x32(M + off + cc, v);
+      }
+      store_f32x32(U + off + cc, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) sq += v[j] * v[j];
+    }
+    if (rowsq && ok) atomicAdd(rowsq + c.z * (z_stride / ld) + row0[c.problem] + c.m, sq);
+  }
+};
+
 // ------------------------------------------------------------------ token phase, dot loss
 // Two products per 128-token tile and 128-wide hidden block j0 = 128*tile_n:
 //   SwiGLU: D0 = X [W1_blk ; W3_blk]^T (256 cols: z1 | z3), D1 = V W2[:, blk] (128 cols: p)

@@ -23,6 +23,7 @@
 #include "ns_fused.cuh"
 #include "token_phase.cuh"
 #include "ttt_plan.cuh"
+#include "wgrad.cuh"
 
 namespace ttt {
 namespace {
@@ -44,14 +45,18 @@ enum BBuf {
   xAct2,   // bf16 [Z][Cp][h]  (GELU' for MSE)
   xDY,     // bf16 [Z][Cp][d]  (dL/dV_hat for MSE / linear)
   xHq,     // bf16 apply hidden [Z][Rq][h]
+  xKstat,  // fp32 key-norm partial sums [Z][Cp/128][d][2]
   xNX, xNXT, xNX2, xNXT2, xNS, xNT,  // fp32 Newton-Schulz buffers [Z*nmat][...]
   kNumBBuf
 };
 
 struct Dims {
-  int Z, H, N, Nq, d, h, Cp, Rq, GR, R1, nmat, m, n, splits;
+  int Z, H, N, Nq, d, h, Cp, Rq, GR, R1, nmat, m, n, splits, tile_rows;
+  bool direct;  // unsplit gradients go straight into U (and M): no partials, no reduction
   bool src_t;  // Newton-Schulz input is the transpose of the gradient-layout source
 };
+
+int bn_for(int n) { return n % 256 == 0 ? 256 : n % 128 == 0 ? 128 : 64; }
 
 Dims dims_of(const Plan& p) {
   const ttt_config& c = p.cfg;
@@ -74,10 +79,14 @@ Dims dims_of(const Plan& p) {
   D.m = std::min(rows_src, c.d);
   D.n = std::max(rows_src, c.d);
   D.splits = int(p.off[kNumBBuf]);
+  D.tile_rows = int(p.off[kNumBBuf + 1]);
+  const bool muon = c.opt == TTT_OPT_MUON || c.opt == TTT_OPT_MOMENTUM_MUON;
+  // with Muon the squared row norms are summed over the tiles of a row: allow at
+  // most two contributions per row (order-independent)
+  D.direct = D.splits == 1 && !(muon && bn_for(c.d) != c.d);
   return D;
 }
 
-int bn_for(int n) { return n % 256 == 0 ? 256 : n % 128 == 0 ? 128 : 64; }
 
 // ------------------------------------------------------------------ small kernels
 // Per canonical weight row: which matrix, its length, and where its gradient /
@@ -121,7 +130,8 @@ __global__ void init_weights_kernel(int Z, int H, int64_t P, const float* W0, fl
 }
 
 // One warp per canonical weight row: [W -= lr U] -> [row L2-norm] -> bf16 copies
-// (+ the non-finite check of the layer's weights).
+// (+ the non-finite check of the layer's weights).  W2^T is made from the bf16 W2
+// afterwards by transpose_w2_kernel.
 //   mode 0: no update (initial weights)
 //   mode 1: U from the gradient layout
 //   mode 2: U from the Newton-Schulz result (X [m][n], XT [n][m] per matrix)
@@ -175,17 +185,94 @@ __global__ void finish_rows_kernel(RowMap rm, int mode, float lr, bool rownorm, 
     }
   } else {
     bf16* w2row = W2 + (int64_t(z) * rm.d + r) * rm.h;
-    bf16* w2t = W2T + int64_t(z) * rm.h * rm.d + r;
     for (int i = lane; i < len; i += 32) {
       const float v = w[i] * inv;
       w[i] = v;
       bad |= !isfinite(v);
-      const bf16 b = __float2bfloat16_rn(v);
-      w2row[i] = b;
-      w2t[int64_t(i) * rm.d] = b;
+      w2row[i] = __float2bfloat16_rn(v);
     }
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(status, kStatusNonFinite);
+}
+
+// W2^T [z][h][d] from W2 [z][d][h] (bf16) through 32 x 32 shared-memory tiles.
+__global__ void transpose_w2_kernel(int d, int h, const bf16* W2, bf16* W2T) {
+  __shared__ bf16 tile[32][34];
+  const int z = blockIdx.z, c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;  // rows of W2 = d, cols = h
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const bf16* src = W2 + int64_t(z) * d * h;
+  bf16* dst = W2T + int64_t(z) * d * h;
+  for (int j = ty; j < 32; j += 8)
+    if (r0 + j < d && c0 + tx < h) tile[j][tx] = src[int64_t(r0 + j) * h + c0 + tx];
+  __syncthreads();
+  for (int j = ty; j < 32; j += 8)
+    if (c0 + j < h && r0 + tx < d) dst[int64_t(c0 + j) * d + r0 + tx] = tile[tx][j];
+}
+
+// Key instance-norm, pass 1: per 128-token block and channel, the sum and sum of
+// squares of the chunk's keys (rows past the chunk count as absent).
+__global__ void keystats_kernel(int n, int d, const bf16* K, int64_t k_zs, int t0, float* part) {
+  __shared__ float red[8][2][64];
+  const int z = blockIdx.y, blk = blockIdx.x, nb = gridDim.x;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int c0 = 0; c0 < d; c0 += 64) {
+    float s0 = 0.f, s1 = 0.f, q0 = 0.f, q1 = 0.f;
+    for (int r = blk * 128 + w; r < min(n, blk * 128 + 128); r += 8) {
+      const float2 v = __bfloat1622float2(
+          *reinterpret_cast<const __nv_bfloat162*>(K + z * k_zs + int64_t(t0 + r) * d + c0 + 2 * lane));
+      s0 += v.x;
+      s1 += v.y;
+      q0 += v.x * v.x;
+      q1 += v.y * v.y;
+    }
+    red[w][0][2 * lane] = s0;
+    red[w][0][2 * lane + 1] = s1;
+    red[w][1][2 * lane] = q0;
+    red[w][1][2 * lane + 1] = q1;
+    __syncthreads();
+    if (threadIdx.x < 128) {
+      const int which = threadIdx.x >> 6, ch = threadIdx.x & 63;
+      float t = 0.f;
+      for (int j = 0; j < 8; ++j) t += red[j][which][ch];
+      part[((int64_t(z) * nb + blk) * d + c0 + ch) * 2 + which] = t;
+    }
+    __syncthreads();
+  }
+}
+
+// Pass 2: every CTA combines the block sums of all channels (in double: the biased
+// variance is E[k^2] - E[k]^2) and normalises its 128 tokens: Kn = (k - mean) /
+// sqrt(var + eps), zeros for rows past the chunk.
+__global__ void keynorm_kernel(int n, int d, const bf16* K, int64_t k_zs, int t0, float eps, const float* part,
+                               bf16* Kn, int64_t kn_zs) {
+  extern __shared__ float st[];  // [d] mean, [d] rstd
+  const int z = blockIdx.y, blk = blockIdx.x, nb = gridDim.x;
+  for (int ch = threadIdx.x; ch < d; ch += blockDim.x) {
+    double s = 0.0, q = 0.0;
+    for (int b = 0; b < nb; ++b) {
+      s += part[((int64_t(z) * nb + b) * d + ch) * 2];
+      q += part[((int64_t(z) * nb + b) * d + ch) * 2 + 1];
+    }
+    const double mean = s / n;
+    const double var = fmax(q / n - mean * mean, 0.0);
+    st[ch] = static_cast<float>(mean);
+    st[d + ch] = static_cast<float>(1.0 / sqrt(var + eps));
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int r = blk * 128 + w; r < blk * 128 + 128; r += 8) {
+    for (int c0 = 0; c0 < d; c0 += 64) {
+      const int ch = c0 + 2 * lane;
+      float a = 0.f, b = 0.f;
+      if (r < n) {
+        const float2 v = __bfloat1622float2(
+            *reinterpret_cast<const __nv_bfloat162*>(K + z * k_zs + int64_t(t0 + r) * d + ch));
+        a = (v.x - st[ch]) * st[d + ch];
+        b = (v.y - st[ch + 1]) * st[d + ch + 1];
+      }
+      *reinterpret_cast<__nv_bfloat162*>(Kn + z * kn_zs + int64_t(r) * d + ch) = __floats2bfloat162_rn(a, b);
+    }
+  }
 }
 
 // One warp per gradient row: sum the split-K partials in split order, momentum,
@@ -264,59 +351,6 @@ __global__ void ns_prep_kernel(RowMap rm, int nmat, const float* U, const float*
   for (int j = ty; j < 32; j += 8) {
     const int c = c0 + j, r = r0 + tx;
     if (r < rows_src && c < d) Bt[zk * mn + int64_t(c) * rows_src + r] = tile[tx][j];
-  }
-}
-
-// bf16 key instance-norm over the chunk's tokens: per (z, 64-channel group)
-__global__ void instnorm_bf16_kernel(int n, int Cp, int d, const bf16* K, int64_t k_zs, int t0, float eps, bf16* Kn,
-                                     int64_t kn_zs) {
-  __shared__ float red[8][64];
-  __shared__ float stat[2][64];
-  const int z = blockIdx.y, c0 = blockIdx.x * 64;
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;  // 8 warps; each lane owns channels c0+2l, c0+2l+1
-  const bf16* src = K + z * k_zs + int64_t(t0) * d + c0 + 2 * lane;
-  float s0 = 0.f, s1 = 0.f;
-  for (int r = w; r < n; r += 8) {
-    const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(src + int64_t(r) * d));
-    s0 += v.x;
-    s1 += v.y;
-  }
-  red[w][2 * lane] = s0;
-  red[w][2 * lane + 1] = s1;
-  __syncthreads();
-  if (threadIdx.x < 64) {
-    float t = 0.f;
-    for (int j = 0; j < 8; ++j) t += red[j][threadIdx.x];
-    stat[0][threadIdx.x] = t / float(n);
-  }
-  __syncthreads();
-  const float m0 = stat[0][2 * lane], m1 = stat[0][2 * lane + 1];
-  float q0 = 0.f, q1 = 0.f;
-  for (int r = w; r < n; r += 8) {
-    const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(src + int64_t(r) * d));
-    q0 += (v.x - m0) * (v.x - m0);
-    q1 += (v.y - m1) * (v.y - m1);
-  }
-  __syncthreads();
-  red[w][2 * lane] = q0;
-  red[w][2 * lane + 1] = q1;
-  __syncthreads();
-  if (threadIdx.x < 64) {
-    float t = 0.f;
-    for (int j = 0; j < 8; ++j) t += red[j][threadIdx.x];
-    stat[1][threadIdx.x] = rsqrtf(t / float(n) + eps);
-  }
-  __syncthreads();
-  const float r0 = stat[1][2 * lane], r1 = stat[1][2 * lane + 1];
-  bf16* dst = Kn + z * kn_zs + c0 + 2 * lane;
-  for (int r = w; r < Cp; r += 8) {
-    float a = 0.f, b = 0.f;
-    if (r < n) {
-      const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(src + int64_t(r) * d));
-      a = (v.x - m0) * r0;
-      b = (v.y - m1) * r1;
-    }
-    *reinterpret_cast<__nv_bfloat162*>(dst + int64_t(r) * d) = __floats2bfloat162_rn(a, b);
   }
 }
 
@@ -411,6 +445,19 @@ struct Ctx {
   int bn_first = 0;
 };
 
+// bf16 W2^T from the freshly written bf16 W2 (the token phase's B operand).
+int transpose_w2(Ctx& c) {
+  if (c.p.cfg.inner == TTT_INNER_LINEAR) return TTT_OK;
+  const Dims& D = c.D;
+  cudaStream_t st = c.st;
+  {
+    StageScope _sc(kStageFinish, st);
+    transpose_w2_kernel<<<dim3((D.h + 31) / 32, (D.d + 31) / 32, D.Z), 256, 0, st>>>(
+        D.d, D.h, c.v.at<bf16>(c.p, xW2), c.v.at<bf16>(c.p, xW2T));
+  }
+  return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+
 // update-direction -> weights (+ Newton-Schulz when the optimizer is Muon)
 int optimizer_step(Ctx& c) {
   cudaStream_t st = c.st;
@@ -419,7 +466,7 @@ int optimizer_step(Ctx& c) {
   const ttt_config& cfg = p.cfg;
   const bool mom = cfg.opt == TTT_OPT_MOMENTUM || cfg.opt == TTT_OPT_MOMENTUM_MUON;
   const bool muon = cfg.opt == TTT_OPT_MUON || cfg.opt == TTT_OPT_MOMENTUM_MUON;
-  {
+  if (!D.direct) {
     dim3 g((D.GR + 7) / 8, D.Z);
     {
       StageScope _sc(kStageReduce, st);
@@ -478,7 +525,57 @@ int optimizer_step(Ctx& c) {
                                             c.v.status);
   }
   TRY_CUDA(cudaGetLastError());
-  return TTT_OK;
+  return transpose_w2(c);
+}
+
+// Weight-gradient token reductions of one chunk: problem 0 (rows0 output rows of
+// the gradient layout, from row 0) and, when rows1 > 0, problem 1 (rows1 rows, from
+// row r1), both N = d, K = the chunk's padded tokens.  Split-K writes fp32 partials
+// for reduce_grad_kernel; an unsplit reduction writes U (and M) directly.
+template <class Epi>
+int grad_launch(Ctx& c, const TM& a0, const TM& b0, const TM& a1, const TM& b1, int rows0, int rows1, int b0k,
+                int b1k, const Epi& ep) {
+  const Dims& D = c.D;
+  const int d = D.d, bnd = bn_for(d), kbt = D.Cp / 64;
+  unsigned* status = c.v.status;
+  if (a0.box != 64 || b0.box != 64 || (rows1 > 0 && (a1.box != 64 || b1.box != 64))) return TTT_ERR_INVALID_ARG;
+  if (D.tile_rows == 256 && rows0 % 256 == 0 && rows1 % 256 == 0) {
+    TcGeom gg = geom(rows0 / 256, rows1 / 256, d / bnd, kbt, D.Z, D.splits);
+    gg.b0.k = b0k;
+    gg.b1.k = b1k;
+    StageScope sc(kStageWeightGrad, c.st);
+    cudaError_t e = bnd == 256 ? launch_wgrad<256, 3>(a0.m, b0.m, a1.m, b1.m, gg, ep, status, c.st)
+                    : bnd == 128 ? launch_wgrad<128, 4>(a0.m, b0.m, a1.m, b1.m, gg, ep, status, c.st)
+                                 : launch_wgrad<64, 4>(a0.m, b0.m, a1.m, b1.m, gg, ep, status, c.st);
+    return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+  }
+  TcGeom gg = geom(rows0 / 128, rows1 / 128, d / bnd, kbt, D.Z, D.splits);
+  gg.b0.k = b0k;
+  gg.b1.k = b1k;
+  if (bnd == 256) return gemm<256, 0, true, true, 2, 4, 8>(a0, b0, a1, b1, gg, ep, status, c.st, true);
+  if (bnd == 128) return gemm<128, 0, true, true, 2, 6, 8>(a0, b0, a1, b1, gg, ep, status, c.st, true);
+  return gemm<64, 0, true, true, 2, 4, 8>(a0, b0, a1, b1, gg, ep, status, c.st, true);
+}
+
+int grad_gemm(Ctx& c, const TM& a0, const TM& b0, const TM& a1, const TM& b1, int rows0, int rows1, int r1, int b0k,
+              int b1k) {
+  const Plan& p = c.p;
+  const Dims& D = c.D;
+  const ttt_config& cfg = p.cfg;
+  const int d = D.d;
+  const int64_t pz = int64_t(D.GR) * d;
+  StageCtx stage(kStageWeightGrad);
+  if (!D.direct) {
+    EpiPartial ep{c.v.at<float>(p, xPart), int64_t(D.Z) * pz, pz, d, {0, r1}, {rows0, rows1}};
+    return grad_launch(c, a0, b0, a1, b1, rows0, rows1, b0k, b1k, ep);
+  }
+  const bool mom = cfg.opt == TTT_OPT_MOMENTUM || cfg.opt == TTT_OPT_MOMENTUM_MUON;
+  const bool muon = cfg.opt == TTT_OPT_MUON || cfg.opt == TTT_OPT_MOMENTUM_MUON;
+  float* rowsq = muon ? c.v.at<float>(p, xRowSq) : nullptr;
+  if (rowsq && cudaMemsetAsync(rowsq, 0, size_t(D.Z) * D.GR * 4, c.st) != cudaSuccess) return TTT_ERR_CUDA;
+  EpiGradDirect ep{c.v.at<float>(p, xU), mom ? c.v.at<float>(p, xMom) : nullptr, rowsq, cfg.momentum, pz, d,
+                   {0, r1}, {rows0, rows1}};
+  return grad_launch(c, a0, b0, a1, b1, rows0, rows1, b0k, b1k, ep);
 }
 
 // Token phase of the negative-dot update: activations H' and dZ(13) of chunk
@@ -527,10 +624,16 @@ int update_chunk(Ctx& c, int t0, int n) {
   TM tKn, tKnmn;
   if (cfg.flags & TTT_FLAG_KEY_INSTNORM) {
     bf16* Kn = c.v.at<bf16>(p, xKn);
+    float* kst = c.v.at<float>(p, xKstat);
+    const dim3 gk(Cp / 128, Z);
     {
       StageScope _sc(kStageKeyNorm, st);
-      instnorm_bf16_kernel<<<dim3(d / 64, Z), 256, 0, c.st>>>(n, Cp, d, K, int64_t(D.N) * d, t0, cfg.in_eps, Kn,
-                                                              int64_t(Cp) * d);
+      keystats_kernel<<<gk, 256, 0, c.st>>>(n, d, K, int64_t(D.N) * d, t0, kst);
+    }
+    {
+      StageScope _sc(kStageKeyNorm, st);
+      keynorm_kernel<<<gk, 256, 2 * d * sizeof(float), c.st>>>(n, d, K, int64_t(D.N) * d, t0, cfg.in_eps, kst, Kn,
+                                                               int64_t(Cp) * d);
     }
     TRY_CUDA(cudaGetLastError());
     TRY(tmap(&tKn, Kn, 2, d, Cp, Z, 128));
@@ -543,9 +646,6 @@ int update_chunk(Ctx& c, int t0, int n) {
   bf16* A1 = c.v.at<bf16>(p, xAct1);
   bf16* A2 = c.v.at<bf16>(p, xAct2);
   bf16* DY = c.v.at<bf16>(p, xDY);
-  float* part = c.v.at<float>(p, xPart);
-  const int64_t pz = int64_t(D.GR) * d, ps = int64_t(Z) * pz;
-  const int kbt = Cp / 64;  // token k-blocks of the weight-gradient GEMMs
   const int bnd = bn_for(d);
   unsigned* status = c.v.status;
   const int mt = Cp / 128;
@@ -558,27 +658,13 @@ int update_chunk(Ctx& c, int t0, int n) {
     TM tH, tD;
     TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
     TRY(tmap(&tD, A1, 2, 2 * h, Cp, Z, 64));
-    g_stage = kStageWeightGrad;
-    TcGeom gg = geom(h / 128, 2 * h / 128, d / bnd, kbt, Z, D.splits);
-    gg.b0.k = t0;
-    gg.b1.k = xoff;
-    EpiPartial ep{part, ps, pz, d, {0, h}, {h, 2 * h}};
-    if (bnd == 256) TRY((gemm<256, 0, true, true, 2, 4, 8>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st, true)));
-    else if (bnd == 128) TRY((gemm<128, 0, true, true, 2, 6, 8>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st, true)));
-    else TRY((gemm<64, 0, true, true, 2, 4, 8>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st, true)));
+    TRY(grad_gemm(c, tH, c.tVmn, tD, *tXmn, h, 2 * h, h, t0, xoff));
   } else if (cfg.inner == TTT_INNER_MLP2_GELU && cfg.loss == TTT_LOSS_NEG_DOT) {
     TRY(token_phase(c, *tX, xoff, t0, n, A0, A1, false));
     TM tH, tD;
     TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
     TRY(tmap(&tD, A1, 2, h, Cp, Z, 64));
-    g_stage = kStageWeightGrad;
-    TcGeom gg = geom(h / 128, h / 128, d / bnd, kbt, Z, D.splits);
-    gg.b0.k = t0;
-    gg.b1.k = xoff;
-    EpiPartial ep{part, ps, pz, d, {0, h}, {h, h}};
-    if (bnd == 256) TRY((gemm<256, 0, true, true, 2, 4, 8>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st, true)));
-    else if (bnd == 128) TRY((gemm<128, 0, true, true, 2, 6, 8>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st, true)));
-    else TRY((gemm<64, 0, true, true, 2, 4, 8>(tH, c.tVmn, tD, *tXmn, gg, ep, status, c.st, true)));
+    TRY(grad_gemm(c, tH, c.tVmn, tD, *tXmn, h, h, h, t0, xoff));
   } else if (cfg.inner == TTT_INNER_MLP2_GELU) {  // MSE
     // Z = X W1^T -> H = GELU(Z), G' = GELU'(Z)
     EpiGeluSave e1{A0, A2, h, n, int64_t(Cp) * h};
@@ -605,13 +691,7 @@ int update_chunk(Ctx& c, int t0, int n) {
     TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
     TRY(tmap(&tYmn, DY, 2, d, Cp, Z, 64));
     TRY(tmap(&tD, A1, 2, h, Cp, Z, 64));
-    g_stage = kStageWeightGrad;
-    TcGeom gg = geom(h / 128, h / 128, d / bnd, kbt, Z, D.splits);
-    gg.b1.k = xoff;
-    EpiPartial ep{part, ps, pz, d, {0, h}, {h, h}};
-    if (bnd == 256) TRY((gemm<256, 0, true, true, 2, 4, 8>(tH, tYmn, tD, *tXmn, gg, ep, status, c.st, true)));
-    else if (bnd == 128) TRY((gemm<128, 0, true, true, 2, 6, 8>(tH, tYmn, tD, *tXmn, gg, ep, status, c.st, true)));
-    else TRY((gemm<64, 0, true, true, 2, 4, 8>(tH, tYmn, tD, *tXmn, gg, ep, status, c.st, true)));
+    TRY(grad_gemm(c, tH, tYmn, tD, *tXmn, h, h, h, 0, xoff));
   } else {  // linear
     if (cfg.loss == TTT_LOSS_MSE) {
       EpiMseGrad e2{DY, d, n, int64_t(Cp) * d, V, int64_t(D.N) * d, t0, c.io.eta, D.N, cfg.eta_scalar,
@@ -631,13 +711,7 @@ int update_chunk(Ctx& c, int t0, int n) {
     }
     TM tYmn;
     TRY(tmap(&tYmn, DY, 2, d, Cp, Z, 64));
-    g_stage = kStageWeightGrad;
-    TcGeom gg = geom(d / 128, 0, d / bnd, kbt, Z, D.splits);
-    gg.b0.k = xoff;
-    EpiPartial ep{part, ps, pz, d, {0, 0}, {d, 0}};
-    if (bnd == 256) TRY((gemm<256, 0, true, true, 2, 4, 8>(tYmn, *tXmn, tYmn, *tXmn, gg, ep, status, c.st, true)));
-    else if (bnd == 128) TRY((gemm<128, 0, true, true, 2, 6, 8>(tYmn, *tXmn, tYmn, *tXmn, gg, ep, status, c.st, true)));
-    else TRY((gemm<64, 0, true, true, 2, 4, 8>(tYmn, *tXmn, tYmn, *tXmn, gg, ep, status, c.st, true)));
+    TRY(grad_gemm(c, tYmn, *tXmn, tYmn, *tXmn, d, 0, 0, xoff, 0));
   }
   return optimizer_step(c);
 }
@@ -685,22 +759,28 @@ int apply_rows(Ctx& c, int row0, int rows) {
   return TTT_OK;
 }
 
-int choose_splits(const Plan& p, int Cp) {
+// Weight-gradient launch shape: split-K count and output tile height (256 rows
+// = two accumulators sharing B, when the rows allow it and the tiles alone keep
+// the SMs busy).
+void choose_grad_shape(const Plan& p, int Cp, int* splits, int* tile_rows) {
   const ttt_config& c = p.cfg;
   const int d = c.d, h = c.h;
   const int bnd = bn_for(d);
   const int rows = c.inner == TTT_INNER_LINEAR ? d : c.inner == TTT_INNER_MLP2_GELU ? 2 * h : 3 * h;
-  const int tiles = rows / 128 * (d / bnd) * p.BH;
+  const int r0 = c.inner == TTT_INNER_LINEAR ? d : h;
   const int kblocks = Cp / 64;
+  // each split reduces at least 1024 tokens: below that the fp32 partials it writes
+  // and the reduction reads cost more than the parallelism gains; chunks of at most
+  // 4096 tokens are not split at all (the gradient then goes straight to the optimizer)
+  const int smax = kblocks <= 64 ? 1 : std::min(64, std::max(1, kblocks / 16));
+  const int tiles256 = (r0 % 256 == 0 && rows % 256 == 0) ? rows / 256 * (d / bnd) * p.BH : 0;
+  *tile_rows = (tiles256 > 0 && tiles256 * smax >= 148) ? 256 : 128;
+  const int tiles = rows / *tile_rows * (d / bnd) * p.BH;
   // about two waves of CTAs: long K ranges per split, few partials to reduce
   int s = std::max(1, (2 * 148 + tiles / 2) / tiles);
-  // each split reduces at least 1024 tokens: below that the fp32 partials it writes
-  // and the reduction reads cost more than the parallelism gains
-  s = std::min(s, std::max(1, kblocks / 16));
-  s = std::min(s, 64);
-  // every split must own at least one k-block
-  const int per = (kblocks + s - 1) / s;
-  return (kblocks + per - 1) / per;
+  s = std::min(s, smax);
+  const int per = (kblocks + s - 1) / s;  // every split owns at least one k-block
+  *splits = (kblocks + per - 1) / per;
 }
 
 }  // namespace
@@ -715,7 +795,10 @@ int plan_layout_bf16(Plan* p) {
   const bool muon = c.opt == TTT_OPT_MUON || c.opt == TTT_OPT_MOMENTUM_MUON;
   if (muon && (d % 128 != 0 || (c.inner != TTT_INNER_LINEAR && h % 128 != 0))) return TTT_ERR_UNSUPPORTED;
   const int Cp = (p->chunk + 127) / 128 * 128;
-  p->off[kNumBBuf] = size_t(choose_splits(*p, Cp));
+  int splits = 1, tile_rows = 128;
+  choose_grad_shape(*p, Cp, &splits, &tile_rows);
+  p->off[kNumBBuf] = size_t(splits);
+  p->off[kNumBBuf + 1] = size_t(tile_rows);
   const Dims D = dims_of(*p);
   const int64_t Z = D.Z, P = p->P, GR = D.GR, nm = int64_t(D.m) * D.n, mm = int64_t(D.m) * D.m;
   const int64_t ZK = Z * D.nmat;
@@ -727,7 +810,7 @@ int plan_layout_bf16(Plan* p) {
       Z * GR * d * 4,
       Z * GR * 4,
       ZK * 4,
-      int64_t(D.splits) * Z * GR * d * 4,
+      D.direct ? 0 : int64_t(D.splits) * Z * GR * d * 4,
       Z * D.R1 * d * 2,
       act ? Z * h * d * 2 : 0,
       act ? Z * d * h * 2 : 0,
@@ -737,6 +820,7 @@ int plan_layout_bf16(Plan* p) {
       mlp_mse ? Z * Cp * h * 2 : 0,
       (mlp_mse || !act) ? Z * Cp * d * 2 : 0,
       act ? Z * D.Rq * h * 2 : 0,
+      (c.flags & TTT_FLAG_KEY_INSTNORM) ? Z * (Cp / 128) * d * 2 * 4 : 0,
       muon ? ZK * nm * 4 : 0,
       muon ? ZK * nm * 4 : 0,
       muon ? ZK * nm * 4 : 0,
@@ -792,6 +876,7 @@ int run_bf16(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
                                             false, First, c.v.at<bf16>(p, xW2T), c.v.at<bf16>(p, xW2), c.v.status);
     }
     TRY_CUDA(cudaGetLastError());
+    TRY(transpose_w2(c));
   }
   for (int ci = 0; ci < p.nchunks; ++ci) {
     const int t0 = ci * p.chunk, n = std::min(p.chunk, cfg.N - t0);
