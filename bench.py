@@ -40,8 +40,8 @@ DATASHEET_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # tokens per reference-arm step (bounded CPU sample) and per CPU-baseline sample
 CPU_SAMPLE_TOKENS = {
-    "tiny_mlp2_n196_fp32": 196, "vit3s_1248_mlp2_n6084": 6084, "lact_lm_causal_n32k_c2048": 8192,
-    "lact_nvs_n196k_d512": 32768, "lact_scene_n1m_c131k": 32768,
+    "tiny_mlp2_n196_fp32": 196, "vit3s_1248_mlp2_n6084": 6084, "lact_lm_causal_n32k_c2048": 16384,
+    "lact_nvs_n196k_d512": 65536, "lact_scene_n1m_c131k": 65536,
 }
 
 

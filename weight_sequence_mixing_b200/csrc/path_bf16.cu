@@ -51,7 +51,7 @@ enum BBuf {
 };
 
 struct Dims {
-  int Z, H, N, Nq, d, h, Cp, Rq, GR, R1, nmat, m, n, splits, tile_rows;
+  int Z, H, N, Nq, d, h, Cp, Rq, GR, R1, nmat, m, n, splits, tile_rows, grad_bn;
   bool direct;  // unsplit gradients go straight into U (and M): no partials, no reduction
   bool src_t;  // Newton-Schulz input is the transpose of the gradient-layout source
 };
@@ -80,10 +80,11 @@ Dims dims_of(const Plan& p) {
   D.n = std::max(rows_src, c.d);
   D.splits = int(p.off[kNumBBuf]);
   D.tile_rows = int(p.off[kNumBBuf + 1]);
+  D.grad_bn = int(p.off[kNumBBuf + 2]);
   const bool muon = c.opt == TTT_OPT_MUON || c.opt == TTT_OPT_MOMENTUM_MUON;
   // with Muon the squared row norms are summed over the tiles of a row: allow at
   // most two contributions per row (order-independent)
-  D.direct = D.splits == 1 && !(muon && bn_for(c.d) != c.d);
+  D.direct = D.splits == 1 && !(muon && D.grad_bn != c.d);
   return D;
 }
 
@@ -536,7 +537,7 @@ template <class Epi>
 int grad_launch(Ctx& c, const TM& a0, const TM& b0, const TM& a1, const TM& b1, int rows0, int rows1, int b0k,
                 int b1k, const Epi& ep) {
   const Dims& D = c.D;
-  const int d = D.d, bnd = bn_for(d), kbt = D.Cp / 64;
+  const int d = D.d, bnd = D.grad_bn, kbt = D.Cp / 64;
   unsigned* status = c.v.status;
   if (a0.box != 64 || b0.box != 64 || (rows1 > 0 && (a1.box != 64 || b1.box != 64))) return TTT_ERR_INVALID_ARG;
   if (D.tile_rows == 256 && rows0 % 256 == 0 && rows1 % 256 == 0) {
@@ -762,7 +763,7 @@ int apply_rows(Ctx& c, int row0, int rows) {
 // Weight-gradient launch shape: split-K count and output tile height (256 rows
 // = two accumulators sharing B, when the rows allow it and the tiles alone keep
 // the SMs busy).
-void choose_grad_shape(const Plan& p, int Cp, int* splits, int* tile_rows) {
+void choose_grad_shape(const Plan& p, int Cp, int* splits, int* tile_rows, int* grad_bn) {
   const ttt_config& c = p.cfg;
   const int d = c.d, h = c.h;
   const int bnd = bn_for(d);
@@ -781,6 +782,11 @@ void choose_grad_shape(const Plan& p, int Cp, int* splits, int* tile_rows) {
   s = std::min(s, smax);
   const int per = (kblocks + s - 1) / s;  // every split owns at least one k-block
   *splits = (kblocks + per - 1) / per;
+  // an unsplit reduction that leaves SMs idle uses narrower tiles (twice the CTAs);
+  // not with Muon, whose row norms must then sum over at most two parts of a row
+  const bool muon = c.opt == TTT_OPT_MUON || c.opt == TTT_OPT_MOMENTUM_MUON;
+  *grad_bn = bnd;
+  if (*splits == 1 && !muon && *tile_rows == 128 && tiles < 148 && bnd >= 128) *grad_bn = bnd / 2;
 }
 
 }  // namespace
@@ -795,10 +801,11 @@ int plan_layout_bf16(Plan* p) {
   const bool muon = c.opt == TTT_OPT_MUON || c.opt == TTT_OPT_MOMENTUM_MUON;
   if (muon && (d % 128 != 0 || (c.inner != TTT_INNER_LINEAR && h % 128 != 0))) return TTT_ERR_UNSUPPORTED;
   const int Cp = (p->chunk + 127) / 128 * 128;
-  int splits = 1, tile_rows = 128;
-  choose_grad_shape(*p, Cp, &splits, &tile_rows);
+  int splits = 1, tile_rows = 128, grad_bn = 64;
+  choose_grad_shape(*p, Cp, &splits, &tile_rows, &grad_bn);
   p->off[kNumBBuf] = size_t(splits);
   p->off[kNumBBuf + 1] = size_t(tile_rows);
+  p->off[kNumBBuf + 2] = size_t(grad_bn);
   const Dims D = dims_of(*p);
   const int64_t Z = D.Z, P = p->P, GR = D.GR, nm = int64_t(D.m) * D.n, mm = int64_t(D.m) * D.m;
   const int64_t ZK = Z * D.nmat;
