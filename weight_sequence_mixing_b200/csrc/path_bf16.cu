@@ -21,6 +21,7 @@
 
 #include "epilogues.cuh"
 #include "ns_fused.cuh"
+#include "token_pair.cuh"
 #include "token_phase.cuh"
 #include "ttt_plan.cuh"
 #include "wgrad.cuh"
@@ -54,6 +55,7 @@ struct Dims {
   int Z, H, N, Nq, d, h, Cp, Rq, GR, R1, nmat, m, n, splits, tile_rows, grad_bn;
   bool direct;  // unsplit gradients go straight into U (and M): no partials, no reduction
   bool src_t;  // Newton-Schulz input is the transpose of the gradient-layout source
+  bool token_pairs;  // token phase on CTA pairs
 };
 
 int bn_for(int n) { return n % 256 == 0 ? 256 : n % 128 == 0 ? 128 : 64; }
@@ -85,6 +87,7 @@ Dims dims_of(const Plan& p) {
   // with Muon the squared row norms are summed over the tiles of a row: allow at
   // most two contributions per row (order-independent)
   D.direct = D.splits == 1 && !(muon && D.grad_bn != c.d);
+  D.token_pairs = (c.flags & TTT_FLAG_SINGLE_CTA_TOKENS) == 0;
   return D;
 }
 
@@ -599,13 +602,27 @@ int token_phase(Ctx& c, const TM& tX, int xoff, int t0, int n, bf16* Hp, bf16* d
   g.x_off = xoff;
   g.v_off = t0;
   g.rows_valid = n;
+  g.rows_alloc = Cp;
   g.t0 = t0;
   g.eta = c.io.eta;
   g.eta_zs = D.N;
   g.eta_scalar = c.p.cfg.eta_scalar;
+  // CTA pairs (256-token tiles) when a pair can be resident; each CTA then loads
+  // half of every weight block: [W1_blk; W3_blk] rows by halves, W2^T rows by halves
+  const bool pairs = D.token_pairs && (swiglu ? token_pair_capacity<true>() : token_pair_capacity<false>()) > 0;
   StageScope sc(kStageTokenPhase, c.st);
-  const cudaError_t e = swiglu ? launch_token_dot<true>(tX.m, c.tFirst.m, c.tV.m, c.tW2T.m, sH, sD, g, c.v.status, c.st)
-                               : launch_token_dot<false>(tX.m, c.tFirst.m, c.tV.m, c.tW2T.m, sH, sD, g, c.v.status, c.st);
+  cudaError_t e;
+  if (pairs) {
+    TM fh, wh;
+    TRY(tmap(&fh, c.v.at<bf16>(c.p, xFirst), 2, d, D.R1, Z, swiglu ? 128 : 64));
+    TRY(tmap(&wh, c.v.at<bf16>(c.p, xW2T), 2, d, h, Z, 64));
+    g.m_tiles = (Cp + 255) / 256;
+    e = swiglu ? launch_token_pair<true>(tX.m, fh.m, c.tV.m, wh.m, sH, sD, g, c.v.status, c.st)
+               : launch_token_pair<false>(tX.m, fh.m, c.tV.m, wh.m, sH, sD, g, c.v.status, c.st);
+  } else {
+    e = swiglu ? launch_token_dot<true>(tX.m, c.tFirst.m, c.tV.m, c.tW2T.m, sH, sD, g, c.v.status, c.st)
+               : launch_token_dot<false>(tX.m, c.tFirst.m, c.tV.m, c.tW2T.m, sH, sD, g, c.v.status, c.st);
+  }
   return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
 }
 

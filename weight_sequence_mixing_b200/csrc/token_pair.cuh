@@ -1,0 +1,315 @@
+// Token phase of the negative-dot-loss update on CTA pairs (tcgen05 cta_group::2).
+//
+// Same arithmetic as token_dot_kernel (token_phase.cuh): for every tile of chunk
+// tokens x 128 hidden units it forms P = V W2[:, blk] and Z13 = X [W1_blk; W3_blk]^T
+// and writes H' and dZ13 (MLP2: H' and dZ) for the weight-gradient GEMMs (LaCT
+// analysis, "Nonlinear memory complements local attention").
+//
+// Here a tile is 256 tokens, computed by the two CTAs of a cluster as one M = 256
+// tensor-core operation: each CTA stages its own 128 token rows (A) and one half
+// of the weight block's rows (B), and the even CTA issues MMAs that read both
+// CTAs' shared memory and accumulate its 128 rows in its own TMEM and the other
+// 128 rows in the peer's.  Each CTA therefore brings in half of the weight bytes a
+// single-CTA tile needs for the same multiply-adds: per 64-token-column k-block a
+// CTA loads 16 KB of tokens + 8 KB (P) / 16 KB (Z, SwiGLU) of weights instead of
+// 16 KB + 16 KB / 32 KB, which is what limits the single-CTA kernel (the rate at
+// which an SM can pull operand tiles out of L2).
+//
+// Protocol (CTA 0 of the pair = leader, CTA 1 = peer):
+//   full[s]    (leader only)  the leader's producer arms it with both CTAs' bytes;
+//                             both producers' TMA loads count their bytes on it.
+//   empty[s]   (both)         the leader's MMA commit arrives on both CTAs' copies.
+//   tmem_full  (both)         the leader's commit after a tile's last MMA.
+//   tmem_empty (leader only)  one arrival per epilogue warp of both CTAs.
+// All waits are bounded; the kernel ends with a cluster barrier so that neither CTA
+// leaves (or frees its TMEM) while the other may still touch its shared memory.
+#pragma once
+#include "token_phase.cuh"
+
+namespace ttt {
+
+template <bool SWIGLU>
+struct PairShape {
+  static constexpr int A_BYTES = 128 * 128;         // this CTA's 128 tokens x 64 bf16
+  static constexpr int BZ_ROWS = SWIGLU ? 128 : 64;  // this CTA's half of the first-layer rows
+  static constexpr int BZ_BYTES = BZ_ROWS * 128;
+  static constexpr int BP_ROWS = 64;  // this CTA's half of the 128 W2^T rows
+  static constexpr int BP_BYTES = BP_ROWS * 128;
+  static constexpr int Z_STAGE = A_BYTES + BZ_BYTES;
+  static constexpr int P_STAGE = A_BYTES + BP_BYTES;
+  static constexpr int SLOT = Z_STAGE > P_STAGE ? Z_STAGE : P_STAGE;
+  static constexpr int STAGES = SWIGLU ? 5 : 6;
+  static constexpr int NOUT = SWIGLU ? 3 : 2;
+  static constexpr int EW = 8;
+  static constexpr int STG_BYTES = 2048;
+  static constexpr int STG_WARP = NOUT * STG_BYTES;
+  static constexpr int SMEM = 1024 + STAGES * SLOT + EW * STG_WARP + 256;
+  static constexpr int ZN = SWIGLU ? 256 : 128;  // MMA N of the Z phase (both halves)
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+template <bool SWIGLU>
+__global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
+    token_pair_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__ CUtensorMap tFirst,
+                      const __grid_constant__ CUtensorMap tV, const __grid_constant__ CUtensorMap tW2T,
+                      const __grid_constant__ CUtensorMap tHp, const __grid_constant__ CUtensorMap tDZ,
+                      const TokGeom g, unsigned* status) {
+  using S = PairShape<SWIGLU>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stg = smem + S::STAGES * S::SLOT;
+  uint64_t* full = reinterpret_cast<uint64_t*>(stg + S::EW * S::STG_WARP);
+  uint64_t* empty = full + S::STAGES;
+  uint64_t* tmem_full = empty + S::STAGES;
+  uint64_t* tmem_empty = tmem_full + 1;
+  uint64_t* drain = tmem_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const uint32_t rank = cluster_rank() & 1u;
+  const bool leader = rank == 0;
+  const int warp = threadIdx.x >> 5;
+  const int lane = static_cast<int>(lane_id());
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int total = g.m_tiles * g.n_tiles * g.batches;  // m_tiles counts 256-token tiles
+  const int KB = g.kblocks;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tmem_full, 1);
+    mbar_init(tmem_empty, 2 * S::EW);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  // both CTAs' barriers initialised and the pair's TMEM allocated before any use
+  tc_fence_before();
+  cluster_barrier();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      tma_prefetch_desc(&tX);
+      tma_prefetch_desc(&tFirst);
+      tma_prefetch_desc(&tV);
+      tma_prefetch_desc(&tW2T);
+      const uint32_t full0 = mapa_shared(smem_u32(full), 0);  // the leader's full[0]
+      int it = 0;
+      bool stop = false;
+      for (int t = pair; t < total && !stop; t += npairs) {
+        const int nt = t % g.n_tiles;
+        const int mt = (t / g.n_tiles) % g.m_tiles;
+        const int z = t / (g.n_tiles * g.m_tiles);
+        const int m0 = mt * 256 + static_cast<int>(rank) * 128;
+        for (int phase = 0; phase < 2 && !stop; ++phase) {
+          for (int kb = 0; kb < KB; ++kb, ++it) {
+            const int s = it % S::STAGES;
+            const uint32_t ph = (it / S::STAGES) & 1;
+            if (it >= S::STAGES && !mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
+              stop = true;
+              break;
+            }
+            uint8_t* st = smem + s * S::SLOT;
+            const uint32_t fb = full0 + static_cast<uint32_t>(s) * 8u;
+            if (phase == 0) {
+              if (leader) mbar_arrive_expect_tx(&full[s], 2 * S::P_STAGE);
+              tma_load_3d_pair(st, &tV, fb, kb * 64, m0 + g.v_off, z);
+              tma_load_3d_pair(st + S::A_BYTES, &tW2T, fb, kb * 64, nt * 128 + static_cast<int>(rank) * S::BP_ROWS, z);
+            } else {
+              if (leader) mbar_arrive_expect_tx(&full[s], 2 * S::Z_STAGE);
+              tma_load_3d_pair(st, &tX, fb, kb * 64, m0 + g.x_off, z);
+              tma_load_3d_pair(st + S::A_BYTES, &tFirst, fb, kb * 64,
+                               nt * (2 * S::BZ_ROWS) + static_cast<int>(rank) * S::BZ_ROWS, z);
+            }
+          }
+        }
+      }
+      if (!*abort_flag) {
+        // every stage released: the leader's last commits have landed here
+        for (int j = max(0, it - S::STAGES); j < it; ++j)
+          if (!mbar_wait(&empty[j % S::STAGES], (j / S::STAGES) & 1, abort_flag)) break;
+      }
+      if (*abort_flag) {
+        // loads still in flight complete within microseconds; give them a millisecond
+        const unsigned long long t0 = global_ns();
+        while (global_ns() - t0 < 1000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (leader && elect_one()) {
+      constexpr uint32_t idP = make_idesc(256, 128, 1, false, false);
+      constexpr uint32_t idZ = make_idesc(256, S::ZN, 1, false, false);
+      const uint32_t sbase = smem_u32(smem);
+      int it = 0, j = 0;
+      bool stop = false;
+      for (int t = pair; t < total && !stop; t += npairs, ++j) {
+        const uint32_t pcol = (j & 1) ? 384u : 256u;
+        for (int phase = 0; phase < 2 && !stop; ++phase) {
+          if (phase == 1) {
+            // both CTAs' epilogues must have drained the previous tile's Z (and its P slot)
+            if (j > 0 && !mbar_wait_cluster(tmem_empty, (j - 1) & 1, abort_flag)) {
+              stop = true;
+              break;
+            }
+            tc_fence_after();
+          }
+          const uint32_t dcol = phase == 0 ? pcol : 0u;
+          const uint32_t id = phase == 0 ? idP : idZ;
+          for (int kb = 0; kb < KB; ++kb, ++it) {
+            const int s = it % S::STAGES;
+            const uint32_t ph = (it / S::STAGES) & 1;
+            if (!mbar_wait_cluster(&full[s], ph, abort_flag)) {
+              stop = true;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a = sbase + s * S::SLOT;
+            const uint32_t b = a + S::A_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_pair(tmem_base + dcol, make_sdesc_sw128(a + kk * 32, 16, 1024),
+                           make_sdesc_sw128(b + kk * 32, 16, 1024), id, (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_commit_pair(&empty[s], 0x3);
+          }
+        }
+        if (!stop) mma_commit_pair(tmem_full, 0x3);
+      }
+      // the last tile's epilogue arrivals (some remote) have all landed
+      if (!stop && j > 0) mbar_wait_cluster(tmem_empty, (j - 1) & 1, abort_flag);
+      if (*abort_flag) {
+        volatile int never = 0;
+        mma_commit_pair(drain, 0x1);
+        mbar_wait(drain, 0, &never);
+      }
+    }
+  } else {
+    const int ew = warp - 2;
+    const int q = warp & 3;
+    const int part = ew >> 2;
+    uint8_t* my = stg + ew * S::STG_WARP;
+    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t tmem_empty0 = mapa_shared(smem_u32(tmem_empty), 0);
+    int j = 0;
+    for (int t = pair; t < total; t += npairs, ++j) {
+      const int nt = t % g.n_tiles;
+      const int mt = (t / g.n_tiles) % g.m_tiles;
+      const int z = t / (g.n_tiles * g.m_tiles);
+      const int m0 = mt * 256 + static_cast<int>(rank) * 128;
+      const bool ready = __all_sync(0xffffffffu, mbar_wait_cluster(tmem_full, j & 1, abort_flag));
+      if (!ready) break;
+      tc_fence_after();
+      const int m = m0 + q * 32 + lane;
+      const bool valid = m < g.rows_valid;
+      const float e = valid ? (g.eta ? g.eta[z * g.eta_zs + g.t0 + m] : g.eta_scalar) : 0.0f;
+      const uint32_t pcol = (j & 1) ? 384u : 256u;
+      const int row = m0 + q * 32;
+      const bool store = row < g.rows_alloc;
+#pragma unroll 1
+      for (int ci = 0; ci < 2; ++ci) {
+        const int cc = 32 * part + 64 * ci;
+        uint32_t r1[32], r3[32], rp[32];
+        tmem_ld32_async(taddr + cc, r1);
+        if constexpr (SWIGLU) tmem_ld32_async(taddr + 128 + cc, r3);
+        tmem_ld32_async(taddr + pcol + cc, rp);
+        tmem_wait_regs(r1);
+        if constexpr (SWIGLU) tmem_wait_regs(r3);
+        tmem_wait_regs(rp);
+        if (ci == 1) {  // last TMEM read of this tile by this warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(tmem_empty0);
+        }
+        float hv[32], d1[32], d3[32];
+        token_dot_math<SWIGLU>(e, r1, r3, rp, hv, d1, d3);
+        if (!store) continue;
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+        stage_row_sw64(my, lane, hv);
+        stage_row_sw64(my + S::STG_BYTES, lane, d1);
+        if constexpr (SWIGLU) stage_row_sw64(my + 2 * S::STG_BYTES, lane, d3);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tHp, my, nt * 128 + cc, row, z);
+          if constexpr (SWIGLU) {
+            tma_store_3d(&tDZ, my + S::STG_BYTES, nt * 256 + cc, row, z);
+            tma_store_3d(&tDZ, my + 2 * S::STG_BYTES, nt * 256 + 128 + cc, row, z);
+          } else {
+            tma_store_3d(&tDZ, my + S::STG_BYTES, nt * 128 + cc, row, z);
+          }
+          bulk_commit();
+        }
+      }
+    }
+    if (lane == 0) bulk_wait0();
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  cluster_barrier();
+  tc_fence_after();
+  if (threadIdx.x == 0 && *abort_flag) set_status(status, kStatusTimeout);
+  if (warp == 1) tmem_dealloc_pair(tmem_base, 512);
+}
+
+template <bool SWIGLU>
+cudaLaunchConfig_t pair_launch_config(int pairs, cudaStream_t st, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(64 + 32 * PairShape<SWIGLU>::EW, 1, 1);
+  cfg.dynamicSmemBytes = PairShape<SWIGLU>::SMEM;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+// CTA pairs of this kernel that can be resident at once (0: none, use the single-CTA kernel).
+template <bool SWIGLU>
+int token_pair_capacity() {
+  static int cap = -1;
+  if (cap < 0) {
+    auto kern = token_pair_kernel<SWIGLU>;
+    cap = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairShape<SWIGLU>::SMEM) ==
+        cudaSuccess) {
+      cudaLaunchAttribute attr[1];
+      cudaLaunchConfig_t cfg = pair_launch_config<SWIGLU>(1, nullptr, attr);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) cap = n;
+    }
+    cudaGetLastError();  // a refused query leaves no sticky error behind
+  }
+  return cap;
+}
+
+// g.m_tiles counts 256-token tiles; g.rows_alloc bounds the rows the stores may write.
+template <bool SWIGLU>
+cudaError_t launch_token_pair(const CUtensorMap& tX, const CUtensorMap& tFirstHalf, const CUtensorMap& tV,
+                              const CUtensorMap& tW2THalf, const CUtensorMap& tHp, const CUtensorMap& tDZ,
+                              const TokGeom& g, unsigned* status, cudaStream_t st) {
+  const int cap = token_pair_capacity<SWIGLU>();
+  if (cap <= 0) return cudaErrorInvalidConfiguration;
+  const long long total = static_cast<long long>(g.m_tiles) * g.n_tiles * g.batches;
+  if (total <= 0) return cudaSuccess;
+  if (total > 0x7fffffffLL || g.kblocks <= 0) return cudaErrorInvalidConfiguration;
+  const int pairs = static_cast<int>(std::min<long long>(total, cap));
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pair_launch_config<SWIGLU>(pairs, st, attr);
+  return cudaLaunchKernelEx(&cfg, token_pair_kernel<SWIGLU>, tX, tFirstHalf, tV, tW2THalf, tHp, tDZ, g, status);
+}
+
+}  // namespace ttt

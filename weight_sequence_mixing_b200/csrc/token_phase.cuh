@@ -28,6 +28,7 @@ struct TokGeom {
   int kblocks;                    // d / 64
   int x_off, v_off;               // token offsets of the keys and values maps
   int rows_valid;                 // tokens in the chunk
+  int rows_alloc;                 // rows of the activation buffers (stores stop there)
   int t0;                         // chunk's first token (eta index)
   const float* eta;
   int64_t eta_zs;
@@ -65,6 +66,49 @@ __device__ __forceinline__ void stage_row_sw64(uint8_t* box, int r, const float 
     u.z = pack_bf16x2(v[8 * k + 4], v[8 * k + 5]);
     u.w = pack_bf16x2(v[8 * k + 6], v[8 * k + 7]);
     rowp[k ^ ((r >> 1) & 3)] = u;
+  }
+}
+
+// Epilogue math of one row's 32 columns: z1 (and z3) and p from TMEM, e = eta_t.
+template <bool SWIGLU>
+__device__ __forceinline__ void token_dot_math(float e, const uint32_t (&r1)[32], const uint32_t (&r3)[32],
+                                               const uint32_t (&rp)[32], float (&hv)[32], float (&d1)[32],
+                                               float (&d3)[32]) {
+  if constexpr (SWIGLU) {
+    // pairs of columns with the paired fp32 instructions:
+    //   s = SiLU gate sigma(z1) = (1 + tanh(z1/2))/2, a = z1 s, dh = -eta p
+    //   H' = -eta a z3, dZ3 = dh a, dZ1 = dh z3 s (1 + z1 (1 - s))
+    const float2 ne = make_float2(-e, -e), half = make_float2(0.5f, 0.5f), one = make_float2(1.0f, 1.0f),
+                 mone = make_float2(-1.0f, -1.0f);
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const float2 z1 = make_float2(__uint_as_float(r1[i]), __uint_as_float(r1[i + 1]));
+      const float2 z3 = make_float2(__uint_as_float(r3[i]), __uint_as_float(r3[i + 1]));
+      const float2 p = make_float2(__uint_as_float(rp[i]), __uint_as_float(rp[i + 1]));
+      const float2 hz = mul2(half, z1);
+      const float2 sg = fma2(half, make_float2(tanh_approx(hz.x), tanh_approx(hz.y)), half);
+      const float2 a = mul2(z1, sg);
+      const float2 dh = mul2(ne, p);
+      const float2 h = mul2(mul2(ne, a), z3);
+      const float2 g3 = mul2(dh, a);
+      const float2 u = fma2(z1, fma2(sg, mone, one), one);
+      const float2 g1 = mul2(mul2(dh, z3), mul2(sg, u));
+      hv[i] = h.x;
+      hv[i + 1] = h.y;
+      d3[i] = g3.x;
+      d3[i + 1] = g3.y;
+      d1[i] = g1.x;
+      d1[i + 1] = g1.y;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float z1 = __uint_as_float(r1[i]);
+      const float dh = -e * __uint_as_float(rp[i]);
+      hv[i] = -e * gelu_dev(z1);
+      d1[i] = dh * gelu_grad_dev(z1);
+      d3[i] = 0.0f;
+    }
   }
 }
 
@@ -232,42 +276,7 @@ __global__ void __launch_bounds__(64 + 32 * TokShape<SWIGLU>::EW, 1)
           if (lane == 0) mbar_arrive(tmem_empty);
         }
         float hv[32], d1[32], d3[32];
-        if constexpr (SWIGLU) {
-          // pairs of columns with the paired fp32 instructions:
-          //   s = SiLU gate sigma(z1) = (1 + tanh(z1/2))/2, a = z1 s, dh = -eta p
-          //   H' = -eta a z3, dZ3 = dh a, dZ1 = dh z3 s (1 + z1 (1 - s))
-          const float2 ne = make_float2(-e, -e), half = make_float2(0.5f, 0.5f), one = make_float2(1.0f, 1.0f),
-                       mone = make_float2(-1.0f, -1.0f);
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float2 z1 = make_float2(__uint_as_float(r1[i]), __uint_as_float(r1[i + 1]));
-            const float2 z3 = make_float2(__uint_as_float(r3[i]), __uint_as_float(r3[i + 1]));
-            const float2 p = make_float2(__uint_as_float(rp[i]), __uint_as_float(rp[i + 1]));
-            const float2 hz = mul2(half, z1);
-            const float2 sg = fma2(half, make_float2(tanh_approx(hz.x), tanh_approx(hz.y)), half);
-            const float2 a = mul2(z1, sg);
-            const float2 dh = mul2(ne, p);
-            const float2 h = mul2(mul2(ne, a), z3);
-            const float2 g3 = mul2(dh, a);
-            const float2 u = fma2(z1, fma2(sg, mone, one), one);
-            const float2 g1 = mul2(mul2(dh, z3), mul2(sg, u));
-            hv[i] = h.x;
-            hv[i + 1] = h.y;
-            d3[i] = g3.x;
-            d3[i + 1] = g3.y;
-            d1[i] = g1.x;
-            d1[i + 1] = g1.y;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float z1 = __uint_as_float(r1[i]);
-            const float dh = -e * __uint_as_float(rp[i]);
-            hv[i] = -e * gelu_dev(z1);
-            d1[i] = dh * gelu_grad_dev(z1);
-            d3[i] = 0.0f;
-          }
-        }
+        token_dot_math<SWIGLU>(e, r1, r3, rp, hv, d1, d3);
         // the previous bulk stores must have read the staging boxes
         if (lane == 0) bulk_wait_read0();
         __syncwarp();
