@@ -38,6 +38,11 @@ const char* ttt_stage_name(int stage);
 /* Kernel launches this handle's forward calls have enqueued since it was created. */
 int64_t ttt_launch_count(const ttt_handle* handle);
 
+/* CTA pairs of the token-phase kernel (swiglu != 0: SwiGLU fast weights, else the
+ * GELU MLP) that can be resident at once on the current device; 0 means the pair
+ * kernel cannot run there and the token phase falls back to single CTAs. */
+int ttt_token_pair_capacity(int swiglu);
+
 #ifdef __cplusplus
 }
 #endif

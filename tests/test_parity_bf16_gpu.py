@@ -80,6 +80,15 @@ TOKEN_KERNEL_CASES = [
 ]
 
 
+def test_token_pair_kernel_is_resident():
+    # the pair kernel must fit an SM pair (registers x threads, shared memory), or the
+    # token phase silently runs on single CTAs
+    from weight_sequence_mixing_b200 import binding
+
+    assert binding.token_pair_capacity(True) >= 64
+    assert binding.token_pair_capacity(False) >= 64
+
+
 @pytest.mark.parametrize("kw", TOKEN_KERNEL_CASES, ids=lambda kw: "-".join(f"{v}" for v in kw.values()))
 def test_token_kernels_pair_and_single_cta(kw):
     base = dict(B=2, H=2, dtype="bf16", data="lact", eta_mode="per_token", loss="neg_dot", opt="gd", seed=17)

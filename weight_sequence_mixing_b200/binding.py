@@ -35,7 +35,7 @@ EXPORTED = [
     "ttt_config_init", "ttt_create", "ttt_param_count", "ttt_workspace_size", "ttt_forward",
     "ttt_host_staging_size", "ttt_forward_host", "ttt_query_status", "ttt_destroy", "ttt_status_string",
     "ttt_selftest_gemm", "ttt_profile_enable", "ttt_profile_collect", "ttt_stage_name", "ttt_launch_count",
-    "ttt_forward_noalloc",
+    "ttt_forward_noalloc", "ttt_token_pair_capacity",
 ]
 NUM_STAGES = 8
 
@@ -80,6 +80,7 @@ def _load():
         "ttt_stage_name": (ctypes.c_char_p, [i32]),
         "ttt_launch_count": (i64, [vp]),
         "ttt_forward_noalloc": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "ttt_token_pair_capacity": (i32, [i32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -225,3 +226,8 @@ def selftest_gemm(A, B, elem_bytes, a_mn, b_mn, bn, M, N, K, batches, splits, st
     _check(LIB.ttt_selftest_gemm(elem_bytes, int(a_mn), int(b_mn), bn, M, N, K, batches, splits, _ptr(A), _ptr(B),
                                  _ptr(C), _stream_ptr(stream)), "ttt_selftest_gemm")
     return C
+
+
+def token_pair_capacity(swiglu: bool) -> int:
+    """CTA pairs of the token-phase kernel resident at once on the current device (0: single-CTA fallback)."""
+    return int(LIB.ttt_token_pair_capacity(int(bool(swiglu))))

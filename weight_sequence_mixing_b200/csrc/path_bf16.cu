@@ -23,6 +23,7 @@
 #include "ns_fused.cuh"
 #include "token_pair.cuh"
 #include "token_phase.cuh"
+#include "ttt_diag.h"
 #include "ttt_plan.cuh"
 #include "wgrad.cuh"
 
@@ -914,3 +915,7 @@ int run_bf16(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
 }
 
 }  // namespace ttt
+
+extern "C" int ttt_token_pair_capacity(int swiglu) {
+  return swiglu ? ttt::token_pair_capacity<true>() : ttt::token_pair_capacity<false>();
+}

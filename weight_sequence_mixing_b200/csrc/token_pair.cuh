@@ -15,12 +15,19 @@
 // 16 KB + 16 KB / 32 KB, which is what limits the single-CTA kernel (the rate at
 // which an SM can pull operand tiles out of L2).
 //
+// TMEM per CTA: Z13 in columns [0, 256), P in one of two 128-column slots (256 or
+// 384, alternating by tile), so a tile's P phase overlaps the previous tile's
+// epilogue.  An epilogue warp reads its first 32-column chunk, computes and packs
+// it, reads the second chunk and then releases the tile's TMEM, before any of its
+// stores; the leader's next Z phase waits only for that release.
+//
 // Protocol (CTA 0 of the pair = leader, CTA 1 = peer):
 //   full[s]    (leader only)  the leader's producer arms it with both CTAs' bytes;
 //                             both producers' TMA loads count their bytes on it.
 //   empty[s]   (both)         the leader's MMA commit arrives on both CTAs' copies.
 //   tmem_full  (both)         the leader's commit after a tile's last MMA.
-//   tmem_empty (leader only)  one arrival per epilogue warp of both CTAs.
+//   tmem_empty (leader only)  one arrival per epilogue warp of both CTAs: the tile's
+//                             Z13 and P columns have been read.
 // All waits are bounded; the kernel ends with a cluster barrier so that neither CTA
 // leaves (or frees its TMEM) while the other may still touch its shared memory.
 #pragma once
@@ -39,10 +46,10 @@ struct PairShape {
   static constexpr int P_STAGE = A_BYTES + BP_BYTES;
   static constexpr int SLOT = Z_STAGE > P_STAGE ? Z_STAGE : P_STAGE;
   static constexpr int STAGES = SWIGLU ? 5 : 6;
-  static constexpr int NOUT = SWIGLU ? 3 : 2;
   static constexpr int EW = 8;
-  static constexpr int STG_BYTES = 2048;
-  static constexpr int STG_WARP = NOUT * STG_BYTES;
+  static constexpr int STG_BYTES = 2048;  // one [32 rows][32 bf16] output box
+  static constexpr int STG_BOXES = 4;     // ring of output boxes per epilogue warp
+  static constexpr int STG_WARP = STG_BOXES * STG_BYTES;
   static constexpr int SMEM = 1024 + STAGES * SLOT + EW * STG_WARP + 256;
   static constexpr int ZN = SWIGLU ? 256 : 128;  // MMA N of the Z phase (both halves)
   static_assert(SMEM <= 227 * 1024, "shared memory");
@@ -155,7 +162,7 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
         const uint32_t pcol = (j & 1) ? 384u : 256u;
         for (int phase = 0; phase < 2 && !stop; ++phase) {
           if (phase == 1) {
-            // both CTAs' epilogues must have drained the previous tile's Z (and its P slot)
+            // both CTAs' epilogues have read the previous tile (Z13 and its P slot)
             if (j > 0 && !mbar_wait_cluster(tmem_empty, (j - 1) & 1, abort_flag)) {
               stop = true;
               break;
@@ -198,11 +205,37 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
     uint8_t* my = stg + ew * S::STG_WARP;
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const uint32_t tmem_empty0 = mapa_shared(smem_u32(tmem_empty), 0);
+    int nt = 0, z = 0, row = 0;
+    int box = 0;  // output boxes this warp has staged: a ring of STG_BOXES in shared memory
+    // stage one [32 rows][32 columns] bf16 box and store it with TMA; the ring slot's
+    // previous store (STG_BOXES boxes ago) must have finished reading it
+    auto emit = [&](const uint32_t (&w)[16], const CUtensorMap* m, int c0) {
+      uint8_t* bx = my + (box % S::STG_BOXES) * S::STG_BYTES;
+      if (lane == 0) bulk_wait_read<S::STG_BOXES - 1>();
+      __syncwarp();
+      stage_packed_sw64(bx, lane, w);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(m, bx, c0, row, z);
+        bulk_commit();
+      }
+      ++box;
+    };
+    auto emit_chunk = [&](const uint32_t (&w)[3][16], int cc) {
+      emit(w[0], &tHp, nt * 128 + cc);
+      if constexpr (SWIGLU) {
+        emit(w[1], &tDZ, nt * 256 + cc);
+        emit(w[2], &tDZ, nt * 256 + 128 + cc);
+      } else {
+        emit(w[1], &tDZ, nt * 128 + cc);
+      }
+    };
     int j = 0;
     for (int t = pair; t < total; t += npairs, ++j) {
-      const int nt = t % g.n_tiles;
+      nt = t % g.n_tiles;
       const int mt = (t / g.n_tiles) % g.m_tiles;
-      const int z = t / (g.n_tiles * g.m_tiles);
+      z = t / (g.n_tiles * g.m_tiles);
       const int m0 = mt * 256 + static_cast<int>(rank) * 128;
       const bool ready = __all_sync(0xffffffffu, mbar_wait_cluster(tmem_full, j & 1, abort_flag));
       if (!ready) break;
@@ -211,43 +244,45 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
       const bool valid = m < g.rows_valid;
       const float e = valid ? (g.eta ? g.eta[z * g.eta_zs + g.t0 + m] : g.eta_scalar) : 0.0f;
       const uint32_t pcol = (j & 1) ? 384u : 256u;
-      const int row = m0 + q * 32;
+      row = m0 + q * 32;
       const bool store = row < g.rows_alloc;
-#pragma unroll 1
-      for (int ci = 0; ci < 2; ++ci) {
-        const int cc = 32 * part + 64 * ci;
+      // this warp's two 32-column chunks: cc0 and cc0 + 64.  Chunk 0 is read,
+      // computed and packed to bf16 before chunk 1 is read; then TMEM is released.
+      const int cc0 = 32 * part;
+      uint32_t wa[3][16];
+      {
         uint32_t r1[32], r3[32], rp[32];
-        tmem_ld32_async(taddr + cc, r1);
-        if constexpr (SWIGLU) tmem_ld32_async(taddr + 128 + cc, r3);
-        tmem_ld32_async(taddr + pcol + cc, rp);
+        tmem_ld32_async(taddr + cc0, r1);
+        if constexpr (SWIGLU) tmem_ld32_async(taddr + 128 + cc0, r3);
+        tmem_ld32_async(taddr + pcol + cc0, rp);
         tmem_wait_regs(r1);
         if constexpr (SWIGLU) tmem_wait_regs(r3);
         tmem_wait_regs(rp);
-        if (ci == 1) {  // last TMEM read of this tile by this warp
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(tmem_empty0);
-        }
         float hv[32], d1[32], d3[32];
         token_dot_math<SWIGLU>(e, r1, r3, rp, hv, d1, d3);
-        if (!store) continue;
-        if (lane == 0) bulk_wait_read0();
-        __syncwarp();
-        stage_row_sw64(my, lane, hv);
-        stage_row_sw64(my + S::STG_BYTES, lane, d1);
-        if constexpr (SWIGLU) stage_row_sw64(my + 2 * S::STG_BYTES, lane, d3);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_3d(&tHp, my, nt * 128 + cc, row, z);
-          if constexpr (SWIGLU) {
-            tma_store_3d(&tDZ, my + S::STG_BYTES, nt * 256 + cc, row, z);
-            tma_store_3d(&tDZ, my + 2 * S::STG_BYTES, nt * 256 + 128 + cc, row, z);
-          } else {
-            tma_store_3d(&tDZ, my + S::STG_BYTES, nt * 128 + cc, row, z);
-          }
-          bulk_commit();
-        }
+        pack_row_bf16(hv, wa[0]);
+        pack_row_bf16(d1, wa[1]);
+        if constexpr (SWIGLU) pack_row_bf16(d3, wa[2]);
+      }
+      uint32_t r1[32], r3[32], rp[32];
+      tmem_ld32_async(taddr + cc0 + 64, r1);
+      if constexpr (SWIGLU) tmem_ld32_async(taddr + 128 + cc0 + 64, r3);
+      tmem_ld32_async(taddr + pcol + cc0 + 64, rp);
+      tmem_wait_regs(r1);
+      if constexpr (SWIGLU) tmem_wait_regs(r3);
+      tmem_wait_regs(rp);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tmem_empty0);
+      if (store) emit_chunk(wa, cc0);
+      {
+        float hv[32], d1[32], d3[32];
+        token_dot_math<SWIGLU>(e, r1, r3, rp, hv, d1, d3);
+        uint32_t wb[3][16];
+        pack_row_bf16(hv, wb[0]);
+        pack_row_bf16(d1, wb[1]);
+        if constexpr (SWIGLU) pack_row_bf16(d3, wb[2]);
+        if (store) emit_chunk(wb, cc0 + 64);
       }
     }
     if (lane == 0) bulk_wait0();

@@ -69,6 +69,19 @@ __device__ __forceinline__ void stage_row_sw64(uint8_t* box, int r, const float 
   }
 }
 
+// 32 floats of one row as 16 bf16 pairs (the order stage_row_sw64 stores them in)
+__device__ __forceinline__ void pack_row_bf16(const float (&v)[32], uint32_t (&w)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+}
+
+// 16 packed bf16 pairs of one row into a [32 rows][64 B] box, 64-byte TMA swizzle
+__device__ __forceinline__ void stage_packed_sw64(uint8_t* box, int r, const uint32_t (&w)[16]) {
+  uint4* rowp = reinterpret_cast<uint4*>(box + r * 64);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) rowp[k ^ ((r >> 1) & 3)] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+}
+
 // Epilogue math of one row's 32 columns: z1 (and z3) and p from TMEM, e = eta_t.
 template <bool SWIGLU>
 __device__ __forceinline__ void token_dot_math(float e, const uint32_t (&r1)[32], const uint32_t (&r3)[32],
