@@ -74,8 +74,8 @@ typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
 #define TTT_FLAG_KEY_INSTNORM 1u  /* normalise each key channel over the chunk's tokens */
 #define TTT_FLAG_WEIGHT_L2NORM 2u /* unit L2 norm for every weight row after each update */
 #define TTT_FLAG_DIRECT_LAUNCH 4u /* launch every kernel on each call instead of replaying a cached CUDA graph */
-#define TTT_FLAG_SINGLE_CTA_TOKENS 8u /* token phase on single CTAs (128-token tiles) instead of CTA pairs;
-                                         same results up to fp32 summation order, for comparison and tests */
+#define TTT_FLAG_SINGLE_CTA 8u /* token phase and weight-gradient GEMMs on single CTAs instead of CTA
+                                  pairs; same results up to fp32 summation order, for comparison and tests */
 
 typedef struct ttt_config {
   int32_t B, H;       /* batch entries and heads */

@@ -39,7 +39,7 @@ _TID = {"Q": 1, "K": 2, "V": 3, "eta": 4, "W0": 5}
 _DEFAULTS = dict(
     B=1, H=1, N=128, Nq=None, d=64, h=64, chunk=0, causal=0,
     inner="mlp2_gelu", loss="mse", opt="gd", dtype="bf16",
-    key_instnorm=False, weight_l2norm=False, direct_launch=False, single_cta_tokens=False,
+    key_instnorm=False, weight_l2norm=False, direct_launch=False, single_cta=False,
     eta_mode="scalar",           # "scalar" | "per_token"
     eta_scalar=1.0, lr=1.0, momentum=0.9,
     ns_iters=5, ns_coeff=(3.4445, -4.7750, 2.0315), in_eps=1e-5,

@@ -68,15 +68,17 @@ def test_small_bf16_variants(kw):
         assert v <= tol, f"{k}: relative Frobenius error {v:.3e} > {tol}"
 
 
-# Token phase on single CTAs (128-token tiles) instead of CTA pairs (256-token
-# tiles): both kernels against the oracle, and against each other.  Token counts
-# leave a ragged last pair tile (N = 300: 384 padded rows, the second pair tile's
-# upper half lies past the activation buffers) and several pair tiles per CTA pair.
+# Token phase and weight gradients on single CTAs instead of CTA pairs: both
+# against the oracle, and against each other.  Token counts leave a ragged last
+# pair tile (N = 300: 384 padded rows, the second pair tile's upper half lies past
+# the activation buffers) and several pair tiles per CTA pair.
 TOKEN_KERNEL_CASES = [
     dict(inner="swiglu", d=128, h=256, N=300),
     dict(inner="swiglu", d=256, h=512, N=1200, chunk=640, opt="momentum", weight_l2norm=True),
     dict(inner="swiglu", d=512, h=256, N=520, opt="muon", weight_l2norm=True),
     dict(inner="mlp2_gelu", d=128, h=384, N=700, chunk=384),
+    # enough k-blocks for split weight gradients on 512-row pair tiles (rows 3h = 1536)
+    dict(inner="swiglu", d=256, h=512, N=8192, opt="momentum_muon", weight_l2norm=True),
 ]
 
 
@@ -95,11 +97,11 @@ def test_token_kernels_pair_and_single_cta(kw):
     base.update(kw)
     x = gen_inputs(make_config(**base))
     Op, Wp = run_gpu(make_config(**base), x)
-    Os, Ws = run_gpu(make_config(single_cta_tokens=True, **base), x)
+    Os, Ws = run_gpu(make_config(single_cta=True, **base), x)
     # the two kernels round the same fp32 accumulators to bf16: near-identical results
     assert rel_fro(Op, Os) < 1e-3 and rel_fro(Wp, Ws) < 1e-3
     for single in (False, True):
-        cfg = make_config(single_cta_tokens=single, **base)
+        cfg = make_config(single_cta=single, **base)
         errs = _delta_w_check(cfg, x)
         for k, v in errs.items():
             tol = DW_TOL if k.startswith("d") else TOL

@@ -29,7 +29,7 @@ DTYPE = {"f32": 0, "bf16": 1}
 FLAG_KEY_INSTNORM = 1
 FLAG_WEIGHT_L2NORM = 2
 FLAG_DIRECT_LAUNCH = 4
-FLAG_SINGLE_CTA_TOKENS = 8
+FLAG_SINGLE_CTA = 8
 
 EXPORTED = [
     "ttt_config_init", "ttt_create", "ttt_param_count", "ttt_workspace_size", "ttt_forward",
@@ -124,7 +124,7 @@ def make_config(cfg: dict) -> TTTConfig:
     c.dtype = DTYPE[cfg["dtype"]]
     c.flags = ((FLAG_KEY_INSTNORM if cfg["key_instnorm"] else 0) | (FLAG_WEIGHT_L2NORM if cfg["weight_l2norm"] else 0)
                | (FLAG_DIRECT_LAUNCH if cfg.get("direct_launch") else 0)
-               | (FLAG_SINGLE_CTA_TOKENS if cfg.get("single_cta_tokens") else 0))
+               | (FLAG_SINGLE_CTA if cfg.get("single_cta") else 0))
     c.eta_scalar = float(cfg["eta_scalar"])
     c.lr = float(cfg["lr"])
     c.momentum = float(cfg["momentum"])

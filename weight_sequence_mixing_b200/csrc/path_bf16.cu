@@ -26,6 +26,7 @@
 #include "ttt_diag.h"
 #include "ttt_plan.cuh"
 #include "wgrad.cuh"
+#include "wgrad_pair.cuh"
 
 namespace ttt {
 namespace {
@@ -56,7 +57,7 @@ struct Dims {
   int Z, H, N, Nq, d, h, Cp, Rq, GR, R1, nmat, m, n, splits, tile_rows, grad_bn;
   bool direct;  // unsplit gradients go straight into U (and M): no partials, no reduction
   bool src_t;  // Newton-Schulz input is the transpose of the gradient-layout source
-  bool token_pairs;  // token phase on CTA pairs
+  bool token_pairs;  // token phase (and, with tile_rows 512, weight gradients) on CTA pairs
 };
 
 int bn_for(int n) { return n % 256 == 0 ? 256 : n % 128 == 0 ? 128 : 64; }
@@ -88,7 +89,7 @@ Dims dims_of(const Plan& p) {
   // with Muon the squared row norms are summed over the tiles of a row: allow at
   // most two contributions per row (order-independent)
   D.direct = D.splits == 1 && !(muon && D.grad_bn != c.d);
-  D.token_pairs = (c.flags & TTT_FLAG_SINGLE_CTA_TOKENS) == 0;
+  D.token_pairs = (c.flags & TTT_FLAG_SINGLE_CTA) == 0;
   return D;
 }
 
@@ -544,7 +545,17 @@ int grad_launch(Ctx& c, const TM& a0, const TM& b0, const TM& a1, const TM& b1, 
   const int d = D.d, bnd = D.grad_bn, kbt = D.Cp / 64;
   unsigned* status = c.v.status;
   if (a0.box != 64 || b0.box != 64 || (rows1 > 0 && (a1.box != 64 || b1.box != 64))) return TTT_ERR_INVALID_ARG;
-  if (D.tile_rows == 256 && rows0 % 256 == 0 && rows1 % 256 == 0) {
+  if (D.tile_rows == 512 && rows0 % 512 == 0 && rows1 % 512 == 0 && (bnd == 256 || bnd == 128) &&
+      (bnd == 256 ? wgrad_pair_capacity<256, 4, Epi>() : wgrad_pair_capacity<128, 5, Epi>()) > 0) {
+    TcGeom gg = geom(rows0 / 512, rows1 / 512, d / bnd, kbt, D.Z, D.splits);
+    gg.b0.k = b0k;
+    gg.b1.k = b1k;
+    StageScope sc(kStageWeightGrad, c.st);
+    cudaError_t e = bnd == 256 ? launch_wgrad_pair<256, 4>(a0.m, b0.m, a1.m, b1.m, gg, ep, status, c.st)
+                               : launch_wgrad_pair<128, 5>(a0.m, b0.m, a1.m, b1.m, gg, ep, status, c.st);
+    return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+  }
+  if (D.tile_rows >= 256 && rows0 % 256 == 0 && rows1 % 256 == 0) {
     TcGeom gg = geom(rows0 / 256, rows1 / 256, d / bnd, kbt, D.Z, D.splits);
     gg.b0.k = b0k;
     gg.b1.k = b1k;
@@ -794,9 +805,14 @@ void choose_grad_shape(const Plan& p, int Cp, int* splits, int* tile_rows, int* 
   const int smax = kblocks <= 64 ? 1 : std::min(64, std::max(1, kblocks / 16));
   const int tiles256 = (r0 % 256 == 0 && rows % 256 == 0) ? rows / 256 * (d / bnd) * p.BH : 0;
   *tile_rows = (tiles256 > 0 && tiles256 * smax >= 148) ? 256 : 128;
+  // 512-row tiles on CTA pairs (74 pairs): each CTA brings in a third fewer bytes
+  const bool pairs_ok = (c.flags & TTT_FLAG_SINGLE_CTA) == 0 && bnd >= 128;
+  const int tiles512 = (pairs_ok && r0 % 512 == 0 && rows % 512 == 0) ? rows / 512 * (d / bnd) * p.BH : 0;
+  if (tiles512 > 0 && tiles512 * smax >= 74) *tile_rows = 512;
+  const int units = *tile_rows == 512 ? 74 : 148;  // tiles that run at once
   const int tiles = rows / *tile_rows * (d / bnd) * p.BH;
-  // about two waves of CTAs: long K ranges per split, few partials to reduce
-  int s = std::max(1, (2 * 148 + tiles / 2) / tiles);
+  // about two waves of tiles: long K ranges per split, few partials to reduce
+  int s = std::max(1, (2 * units + tiles / 2) / tiles);
   s = std::min(s, smax);
   const int per = (kblocks + s - 1) / s;  // every split owns at least one k-block
   *splits = (kblocks + per - 1) / per;
@@ -804,7 +820,7 @@ void choose_grad_shape(const Plan& p, int Cp, int* splits, int* tile_rows, int* 
   // not with Muon, whose row norms must then sum over at most two parts of a row
   const bool muon = c.opt == TTT_OPT_MUON || c.opt == TTT_OPT_MOMENTUM_MUON;
   *grad_bn = bnd;
-  if (*splits == 1 && !muon && *tile_rows == 128 && tiles < 148 && bnd >= 128) *grad_bn = bnd / 2;
+  if (*splits == 1 && !muon && *tile_rows == 128 && tiles < units && bnd >= 128) *grad_bn = bnd / 2;
 }
 
 }  // namespace

@@ -17,7 +17,7 @@ int plan_build(const ttt_config& c, Plan* p) {
   if (c.causal && c.Nq != c.N) return TTT_ERR_INVALID_ARG;
   if (c.inner != TTT_INNER_LINEAR && c.h < 1) return TTT_ERR_INVALID_ARG;
   if ((c.flags & ~(TTT_FLAG_KEY_INSTNORM | TTT_FLAG_WEIGHT_L2NORM | TTT_FLAG_DIRECT_LAUNCH |
-                   TTT_FLAG_SINGLE_CTA_TOKENS)) != 0)
+                   TTT_FLAG_SINGLE_CTA)) != 0)
     return TTT_ERR_INVALID_ARG;
   if (c.ns_iters < 0 || c.ns_iters > 100) return TTT_ERR_INVALID_ARG;
   if (!std::isfinite(c.eta_scalar) || !std::isfinite(c.lr) || !std::isfinite(c.momentum) ||
