@@ -90,10 +90,21 @@ def load_peaks() -> tuple[dict, str]:
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_digest() -> str:
+# The sources that define each timed kernel (its launch function included): a DRAM
+# traffic figure recorded for a stage stays valid only while these files are unchanged.
+STAGE_SOURCES = {
+    "token_phase": ["token_pair.cuh", "token_phase.cuh", "epilogues.cuh", "tc_gemm.cuh", "ptx.cuh"],
+    "weight_grad": ["wgrad_pair.cuh", "wgrad.cuh", "epilogues.cuh", "tc_gemm.cuh", "ptx.cuh"],
+    "newton_schulz": ["ns_fused.cuh", "epilogues.cuh", "tc_gemm.cuh", "ptx.cuh"],
+}
+
+
+def source_digest(stage: str) -> str:
     h = hashlib.sha256()
-    files = sorted(glob.glob(os.path.join(ROOT, "weight_sequence_mixing_b200", "csrc", "*")) +
-                   glob.glob(os.path.join(ROOT, "include", "*.h")))
+    csrc = os.path.join(ROOT, "weight_sequence_mixing_b200", "csrc")
+    names = STAGE_SOURCES.get(stage)
+    files = ([os.path.join(csrc, n) for n in names] if names else
+             sorted(glob.glob(os.path.join(csrc, "*")) + glob.glob(os.path.join(ROOT, "include", "*.h"))))
     for f in files:
         with open(f, "rb") as fh:
             h.update(os.path.basename(f).encode())
@@ -106,7 +117,7 @@ def measured_traffic(workload_name: str, stage: str):
     path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(path):
         return None
-    digest = source_digest()
+    digest = source_digest(stage)
     with open(path) as f:
         for line in f:
             parts = line.split()
