@@ -58,13 +58,20 @@ def build(verbose: bool = False, extra_flags: list[str] | None = None) -> str:
             subprocess.run(cmd, check=True)
             changed = True
         objs.append(obj)
-    if changed or not os.path.exists(LIB):
+    # the objects the library was last linked from: relink whenever they differ (a
+    # source reverted to an earlier version finds its old object in the cache)
+    manifest = os.path.join(BUILD, "libttt_b200.objects")
+    listing = "\n".join(os.path.basename(o) for o in objs)
+    linked = open(manifest).read() if os.path.exists(manifest) else None
+    if changed or linked != listing or not os.path.exists(LIB):
         tmp = LIB + ".tmp"
         cmd = [nvcc] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
         subprocess.run(cmd, check=True)
         os.replace(tmp, LIB)
+        with open(manifest, "w") as f:
+            f.write(listing)
     return LIB
 
 
