@@ -16,8 +16,11 @@ using bf16 = __nv_bfloat16;
 
 // ------------------------------------------------------------------ helpers
 __device__ __forceinline__ float gelu_dev(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
-__device__ __forceinline__ float gelu_grad_dev(float x) {
-  return 0.5f * (1.0f + erff(x * 0.70710678118654752f)) + x * 0.39894228040143268f * __expf(-0.5f * x * x);
+// GELU(x) = x Phi(x) and its derivative Phi(x) + x phi(x) with one erf evaluation
+__device__ __forceinline__ void gelu_and_grad(float x, float& g, float& gp) {
+  const float cdf = 0.5f * (1.0f + erff(x * 0.70710678118654752f));
+  g = x * cdf;
+  gp = fmaf(x * 0.39894228040143268f, __expf(-0.5f * x * x), cdf);
 }
 // sigma(x) = (1 + tanh(x/2)) / 2 with the hardware tanh approximation (max rel.
 // error ~2^-11, below the bf16 rounding the results get)
@@ -210,8 +213,10 @@ struct EpiTokenDot {
           d3[j] = dh * a;
           d1[j] = dh * z3[j] * s * (1.0f + z1[j] * (1.0f - s));
         } else {
-          hv[j] = -e * gelu_dev(z1[j]);
-          d1[j] = dh * gelu_grad_dev(z1[j]);
+          float gz, gpz;
+          gelu_and_grad(z1[j], gz, gpz);
+          hv[j] = -e * gz;
+          d1[j] = dh * gpz;
           d3[j] = 0.0f;
         }
       }
@@ -241,8 +246,10 @@ struct EpiGeluSave {
       tmem_ld32(c.taddr + cc, v);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        a[j] = valid ? gelu_dev(v[j]) : 0.0f;
-        g[j] = valid ? gelu_grad_dev(v[j]) : 0.0f;
+        float gz, gpz;
+        gelu_and_grad(v[j], gz, gpz);
+        a[j] = valid ? gz : 0.0f;
+        g[j] = valid ? gpz : 0.0f;
       }
       store_bf16x32(hrow + cc, a);
       store_bf16x32(grow + cc, g);

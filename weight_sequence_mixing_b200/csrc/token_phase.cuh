@@ -118,8 +118,10 @@ __device__ __forceinline__ void token_dot_math(float e, const uint32_t (&r1)[32]
     for (int i = 0; i < 32; ++i) {
       const float z1 = __uint_as_float(r1[i]);
       const float dh = -e * __uint_as_float(rp[i]);
-      hv[i] = -e * gelu_dev(z1);
-      d1[i] = dh * gelu_grad_dev(z1);
+      float gz, gpz;
+      gelu_and_grad(z1, gz, gpz);
+      hv[i] = -e * gz;
+      d1[i] = dh * gpz;
       d3[i] = 0.0f;
     }
   }
