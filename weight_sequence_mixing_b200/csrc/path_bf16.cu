@@ -600,9 +600,14 @@ int token_phase(Ctx& c, const TM& tX, int xoff, int t0, int n, bf16* Hp, bf16* d
   const Dims& D = c.D;
   const int Z = D.Z, d = D.d, h = D.h, Cp = D.Cp;
   const int dzc = swiglu ? 2 * h : h;
+  // CTA pairs (256-token tiles) when a pair can be resident; each CTA then loads
+  // half of every weight block: [W1_blk; W3_blk] rows by halves, W2^T rows by halves
+  const bool pairs = D.token_pairs && (swiglu ? token_pair_capacity<true>() : token_pair_capacity<false>()) > 0;
+  // output boxes: [32 rows][16 columns] (pair kernel) or [32 rows][32 columns]
+  const int bc = pairs ? 16 : 32;
   CUtensorMap sH, sD;
-  if (!make_tmap_ex(&sH, Hp, 2, h, Cp, Z, h, int64_t(Cp) * h, 32, 32, 64) ||
-      !make_tmap_ex(&sD, dZ, 2, dzc, Cp, Z, dzc, int64_t(Cp) * dzc, 32, 32, 64))
+  if (!make_tmap_ex(&sH, Hp, 2, h, Cp, Z, h, int64_t(Cp) * h, bc, 32, 2 * bc) ||
+      !make_tmap_ex(&sD, dZ, 2, dzc, Cp, Z, dzc, int64_t(Cp) * dzc, bc, 32, 2 * bc))
     return TTT_ERR_INVALID_ARG;
   const int bz = swiglu ? 256 : 128;
   if (tX.box != 128 || c.tV.box != 128 || c.tW2T.box != 128 || c.tFirst.box != bz) return TTT_ERR_INVALID_ARG;
@@ -619,9 +624,6 @@ int token_phase(Ctx& c, const TM& tX, int xoff, int t0, int n, bf16* Hp, bf16* d
   g.eta = c.io.eta;
   g.eta_zs = D.N;
   g.eta_scalar = c.p.cfg.eta_scalar;
-  // CTA pairs (256-token tiles) when a pair can be resident; each CTA then loads
-  // half of every weight block: [W1_blk; W3_blk] rows by halves, W2^T rows by halves
-  const bool pairs = D.token_pairs && (swiglu ? token_pair_capacity<true>() : token_pair_capacity<false>()) > 0;
   StageScope sc(kStageTokenPhase, c.st);
   cudaError_t e;
   if (pairs) {

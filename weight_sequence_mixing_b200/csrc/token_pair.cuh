@@ -46,8 +46,8 @@ struct PairShape {
   static constexpr int P_STAGE = A_BYTES + BP_BYTES;
   static constexpr int SLOT = Z_STAGE > P_STAGE ? Z_STAGE : P_STAGE;
   static constexpr int STAGES = SWIGLU ? 5 : 6;
-  static constexpr int EW = 8;
-  static constexpr int STG_BYTES = 2048;  // one [32 rows][32 bf16] output box
+  static constexpr int EW = 16;           // epilogue warps: 4 per TMEM lane quarter
+  static constexpr int STG_BYTES = 1024;  // one [32 rows][16 bf16] output box
   static constexpr int STG_BOXES = 4;     // ring of output boxes per epilogue warp
   static constexpr int STG_WARP = STG_BOXES * STG_BYTES;
   static constexpr int SMEM = 1024 + STAGES * SLOT + EW * STG_WARP + 256;
@@ -199,21 +199,23 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
       }
     }
   } else {
+    // 16 epilogue warps, four per TMEM lane quarter: warp slot s of quarter q owns the
+    // 16-column chunks 16 s and 64 + 16 s of rows 32 q .. 32 q + 31 of every tile
     const int ew = warp - 2;
     const int q = warp & 3;
-    const int part = ew >> 2;
+    const int slot = ew >> 2;
     uint8_t* my = stg + ew * S::STG_WARP;
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const uint32_t tmem_empty0 = mapa_shared(smem_u32(tmem_empty), 0);
     int nt = 0, z = 0, row = 0;
     int box = 0;  // output boxes this warp has staged: a ring of STG_BOXES in shared memory
-    // stage one [32 rows][32 columns] bf16 box and store it with TMA; the ring slot's
+    // stage one [32 rows][16 columns] bf16 box and store it with TMA; the ring slot's
     // previous store (STG_BOXES boxes ago) must have finished reading it
-    auto emit = [&](const uint32_t (&w)[16], const CUtensorMap* m, int c0) {
+    auto emit = [&](const uint32_t (&w)[8], const CUtensorMap* m, int c0) {
       uint8_t* bx = my + (box % S::STG_BOXES) * S::STG_BYTES;
       if (lane == 0) bulk_wait_read<S::STG_BOXES - 1>();
       __syncwarp();
-      stage_packed_sw64(bx, lane, w);
+      stage_packed_sw32(bx, lane, w);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
       }
       ++box;
     };
-    auto emit_chunk = [&](const uint32_t (&w)[3][16], int cc) {
+    auto emit_chunk = [&](const uint32_t (&w)[3][8], int cc) {
       emit(w[0], &tHp, nt * 128 + cc);
       if constexpr (SWIGLU) {
         emit(w[1], &tDZ, nt * 256 + cc);
@@ -246,43 +248,43 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
       const uint32_t pcol = (j & 1) ? 384u : 256u;
       row = m0 + q * 32;
       const bool store = row < g.rows_alloc;
-      // this warp's two 32-column chunks: cc0 and cc0 + 64.  Chunk 0 is read,
-      // computed and packed to bf16 before chunk 1 is read; then TMEM is released.
-      const int cc0 = 32 * part;
-      uint32_t wa[3][16];
+      // chunk a (columns cca) is read, computed and packed to bf16 before chunk b
+      // (cca + 64) is read; then TMEM is released, before any store.
+      const int cca = 16 * slot;
+      uint32_t wa[3][8];
       {
-        uint32_t r1[32], r3[32], rp[32];
-        tmem_ld32_async(taddr + cc0, r1);
-        if constexpr (SWIGLU) tmem_ld32_async(taddr + 128 + cc0, r3);
-        tmem_ld32_async(taddr + pcol + cc0, rp);
+        uint32_t r1[16], r3[16], rp[16];
+        tmem_ld16_async(taddr + cca, r1);
+        if constexpr (SWIGLU) tmem_ld16_async(taddr + 128 + cca, r3);
+        tmem_ld16_async(taddr + pcol + cca, rp);
         tmem_wait_regs(r1);
         if constexpr (SWIGLU) tmem_wait_regs(r3);
         tmem_wait_regs(rp);
-        float hv[32], d1[32], d3[32];
-        token_dot_math<SWIGLU>(e, r1, r3, rp, hv, d1, d3);
+        float hv[16], d1[16], d3[16];
+        token_dot_math<SWIGLU, 16>(e, r1, r3, rp, hv, d1, d3);
         pack_row_bf16(hv, wa[0]);
         pack_row_bf16(d1, wa[1]);
         if constexpr (SWIGLU) pack_row_bf16(d3, wa[2]);
       }
-      uint32_t r1[32], r3[32], rp[32];
-      tmem_ld32_async(taddr + cc0 + 64, r1);
-      if constexpr (SWIGLU) tmem_ld32_async(taddr + 128 + cc0 + 64, r3);
-      tmem_ld32_async(taddr + pcol + cc0 + 64, rp);
+      uint32_t r1[16], r3[16], rp[16];
+      tmem_ld16_async(taddr + cca + 64, r1);
+      if constexpr (SWIGLU) tmem_ld16_async(taddr + 128 + cca + 64, r3);
+      tmem_ld16_async(taddr + pcol + cca + 64, rp);
       tmem_wait_regs(r1);
       if constexpr (SWIGLU) tmem_wait_regs(r3);
       tmem_wait_regs(rp);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tmem_empty0);
-      if (store) emit_chunk(wa, cc0);
+      if (store) emit_chunk(wa, cca);
       {
-        float hv[32], d1[32], d3[32];
-        token_dot_math<SWIGLU>(e, r1, r3, rp, hv, d1, d3);
-        uint32_t wb[3][16];
+        float hv[16], d1[16], d3[16];
+        token_dot_math<SWIGLU, 16>(e, r1, r3, rp, hv, d1, d3);
+        uint32_t wb[3][8];
         pack_row_bf16(hv, wb[0]);
         pack_row_bf16(d1, wb[1]);
         if constexpr (SWIGLU) pack_row_bf16(d3, wb[2]);
-        if (store) emit_chunk(wb, cc0 + 64);
+        if (store) emit_chunk(wb, cca + 64);
       }
     }
     if (lane == 0) bulk_wait0();

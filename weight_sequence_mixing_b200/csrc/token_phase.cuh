@@ -69,10 +69,19 @@ __device__ __forceinline__ void stage_row_sw64(uint8_t* box, int r, const float 
   }
 }
 
-// 32 floats of one row as 16 bf16 pairs (the order stage_row_sw64 stores them in)
-__device__ __forceinline__ void pack_row_bf16(const float (&v)[32], uint32_t (&w)[16]) {
+// N floats of one row as N/2 bf16 pairs (the order stage_row_sw64 stores them in)
+template <int N>
+__device__ __forceinline__ void pack_row_bf16(const float (&v)[N], uint32_t (&w)[N / 2]) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+  for (int i = 0; i < N / 2; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+}
+
+// 8 packed bf16 pairs (16 columns, 32 bytes) of one row into a [32 rows][32 B] box with
+// the 32-byte TMA swizzle (16-byte chunk k of row r sits at chunk k ^ ((r >> 2) & 1))
+__device__ __forceinline__ void stage_packed_sw32(uint8_t* box, int r, const uint32_t (&w)[8]) {
+  uint4* rowp = reinterpret_cast<uint4*>(box + r * 32);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) rowp[k ^ ((r >> 2) & 1)] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
 }
 
 // 16 packed bf16 pairs of one row into a [32 rows][64 B] box, 64-byte TMA swizzle
@@ -82,11 +91,11 @@ __device__ __forceinline__ void stage_packed_sw64(uint8_t* box, int r, const uin
   for (int k = 0; k < 4; ++k) rowp[k ^ ((r >> 1) & 3)] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
 }
 
-// Epilogue math of one row's 32 columns: z1 (and z3) and p from TMEM, e = eta_t.
-template <bool SWIGLU>
-__device__ __forceinline__ void token_dot_math(float e, const uint32_t (&r1)[32], const uint32_t (&r3)[32],
-                                               const uint32_t (&rp)[32], float (&hv)[32], float (&d1)[32],
-                                               float (&d3)[32]) {
+// Epilogue math of N columns of one row: z1 (and z3) and p from TMEM, e = eta_t.
+template <bool SWIGLU, int N = 32>
+__device__ __forceinline__ void token_dot_math(float e, const uint32_t (&r1)[N], const uint32_t (&r3)[N],
+                                               const uint32_t (&rp)[N], float (&hv)[N], float (&d1)[N],
+                                               float (&d3)[N]) {
   if constexpr (SWIGLU) {
     // pairs of columns with the paired fp32 instructions:
     //   s = SiLU gate sigma(z1) = (1 + tanh(z1/2))/2, a = z1 s, dh = -eta p
@@ -94,7 +103,7 @@ __device__ __forceinline__ void token_dot_math(float e, const uint32_t (&r1)[32]
     const float2 ne = make_float2(-e, -e), half = make_float2(0.5f, 0.5f), one = make_float2(1.0f, 1.0f),
                  mone = make_float2(-1.0f, -1.0f);
 #pragma unroll
-    for (int i = 0; i < 32; i += 2) {
+    for (int i = 0; i < N; i += 2) {
       const float2 z1 = make_float2(__uint_as_float(r1[i]), __uint_as_float(r1[i + 1]));
       const float2 z3 = make_float2(__uint_as_float(r3[i]), __uint_as_float(r3[i + 1]));
       const float2 p = make_float2(__uint_as_float(rp[i]), __uint_as_float(rp[i + 1]));
@@ -115,7 +124,7 @@ __device__ __forceinline__ void token_dot_math(float e, const uint32_t (&r1)[32]
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < N; ++i) {
       const float z1 = __uint_as_float(r1[i]);
       const float dh = -e * __uint_as_float(rp[i]);
       float gz, gpz;
