@@ -285,37 +285,18 @@ __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
-// arrive (release at cluster scope) on an mbarrier of any CTA of the cluster
+// Arrive on an mbarrier of any CTA of the cluster (default semantics, release at CTA
+// scope, the form CUTLASS's 2-SM pipelines use).  What the arrival orders across the
+// pair is tcgen05 work: TMEM reads before the arrival (tcgen05.fence::before_thread_sync)
+// against MMAs issued after the matching wait (tcgen05.fence::after_thread_sync).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// bounded wait (as mbar_wait) for a phase completed by arrivals from the other CTA
+// bounded wait (as mbar_wait) for a phase completed by arrivals or TMA bytes that may
+// come from the other CTA of the pair
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const unsigned long long t0 = global_ns();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait_cluster(bar, parity)) return true;
-    if (*abort) return false;
-    if (global_ns() - t0 > kWaitLimitNs) {
-      *abort = 1;
-      return false;
-    }
-  }
+  return mbar_wait(bar, parity, abort);
 }
 
 // Pair TMEM allocation: one warp of each CTA (same warp index, same `dst_smem`
