@@ -168,65 +168,6 @@ struct EpiGradDirect {
   }
 };
 
-// ------------------------------------------------------------------ token phase, dot loss
-// Two products per 128-token tile and 128-wide hidden block j0 = 128*tile_n:
-//   SwiGLU: D0 = X [W1_blk ; W3_blk]^T (256 cols: z1 | z3), D1 = V W2[:, blk] (128 cols: p)
-//   MLP2  : D0 = X W1_blk^T           (128 cols: z),       D1 = V W2[:, blk] (128 cols: p)
-// With dL/dV_hat_t = -eta_t v_t (negative dot loss, LaCT analysis "Nonlinear memory"):
-//   dH = -eta_t p.  SwiGLU: H' = -eta_t SiLU(z1) z3, dZ3 = dH SiLU(z1), dZ1 = dH z3 SiLU'(z1).
-//   MLP2  : H' = -eta_t GELU(z), dZ = dH GELU'(z).
-// H' (so that the W2 gradient is V^T H') goes to Hp [z][t][h]; dZ1/dZ3 to dZ
-// [z][t][2h] blocked as [blk][dZ1 128 | dZ3 128] (SwiGLU) or dZ [z][t][h] (MLP2).
-// Rows t >= rows_valid (past the chunk's last token) are written as zeros.
-template <bool SWIGLU>
-struct EpiTokenDot {
-  bf16* Hp;
-  bf16* dZ;
-  int h;                 // hidden width
-  int rows_valid;        // tokens in the chunk
-  int64_t hp_zs, dz_zs;  // per-z strides (elements)
-  const float* eta;      // [z][N] or null
-  int64_t eta_zs;
-  int t0;                // chunk's first token (eta index)
-  float eta_scalar;
-  template <int BN0, int BN1>
-  __device__ void run(const EpiCtx& c) const {
-    const bool valid = c.m < rows_valid;
-    const float e = valid ? (eta ? eta[c.z * eta_zs + t0 + c.m] : eta_scalar) : 0.0f;
-    const int blk = c.n0 / BN0;
-    bf16* hrow = Hp + c.z * hp_zs + int64_t(c.m) * h + blk * 128;
-    bf16* drow = dZ + c.z * dz_zs + int64_t(c.m) * (SWIGLU ? 2 * h : h) + blk * (SWIGLU ? 256 : 128);
-#pragma unroll 1
-    for (int cc = 32 * c.part; cc < 128; cc += 32 * c.nparts) {
-      float z1[32], z3[32], p[32];
-      tmem_ld32(c.taddr + cc, z1);
-      if constexpr (SWIGLU) tmem_ld32(c.taddr + 128 + cc, z3);
-      tmem_ld32(c.taddr + BN0 + cc, p);
-      float hv[32], d1[32], d3[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float dh = -e * p[j];
-        if constexpr (SWIGLU) {
-          const float s = sigmoid_dev(z1[j]);
-          const float a = z1[j] * s;
-          hv[j] = -e * a * z3[j];
-          d3[j] = dh * a;
-          d1[j] = dh * z3[j] * s * (1.0f + z1[j] * (1.0f - s));
-        } else {
-          float gz, gpz;
-          gelu_and_grad(z1[j], gz, gpz);
-          hv[j] = -e * gz;
-          d1[j] = dh * gpz;
-          d3[j] = 0.0f;
-        }
-      }
-      store_bf16x32(hrow + cc, hv);
-      store_bf16x32(drow + cc, d1);
-      if constexpr (SWIGLU) store_bf16x32(drow + 128 + cc, d3);
-    }
-  }
-};
-
 // ------------------------------------------------------------------ token phase, MSE (MLP2)
 // Z = X W1^T tile: H = GELU(Z) and G' = GELU'(Z) (bf16), zeros past the chunk.
 struct EpiGeluSave {
@@ -374,77 +315,6 @@ struct EpiStoreOut {
       else store_f32x32(reinterpret_cast<float*>(row + cc), v);
     }
     if (bad) set_status(status, kStatusNonFinite);
-  }
-};
-
-// ------------------------------------------------------------------ Newton-Schulz (fp32 / tf32)
-// S = X X^T
-struct EpiStoreF32 {
-  float* out;
-  int ld, rows;
-  int64_t zs;
-  template <int BN0, int BN1>
-  __device__ void run(const EpiCtx& c) const {
-    float* row = out + c.z * zs + int64_t(c.m) * ld + c.n0;
-#pragma unroll 1
-    for (int cc = 32 * c.part; cc < BN0; cc += 32 * c.nparts) {
-      float v[32];
-      tmem_ld32(c.taddr + cc, v);
-      if (c.m < rows && c.n0 + cc < ld) store_f32x32(row + cc, v);
-    }
-  }
-};
-
-// T = b S + c (S S)
-struct EpiNsPoly {
-  float* T;
-  const float* S;
-  int ld, rows;
-  int64_t zs;
-  float b, cc_;
-  template <int BN0, int BN1>
-  __device__ void run(const EpiCtx& c) const {
-    float* trow = T + c.z * zs + int64_t(c.m) * ld + c.n0;
-    const float* srow = S + c.z * zs + int64_t(c.m) * ld + c.n0;
-#pragma unroll 1
-    for (int cc = 32 * c.part; cc < BN0; cc += 32 * c.nparts) {
-      float v[32], s[32];
-      tmem_ld32(c.taddr + cc, v);
-      if (c.m >= rows || c.n0 + cc >= ld) continue;
-      load_f32x32(srow + cc, s);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = b * s[j] + cc_ * v[j];
-      store_f32x32(trow + cc, v);
-    }
-  }
-};
-
-// X' = a X + T X, stored as X' [m][n] and X'^T [n][m]
-struct EpiNsUpdate {
-  float* Xn;
-  float* XnT;
-  const float* X;
-  int m, n;
-  int64_t zs;
-  float a;
-  template <int BN0, int BN1>
-  __device__ void run(const EpiCtx& c) const {
-    const bool valid = c.m < m;
-    float* row = Xn + c.z * zs + int64_t(c.m) * n + c.n0;
-    const float* xrow = X + c.z * zs + int64_t(c.m) * n + c.n0;
-    float* colT = XnT + c.z * zs + int64_t(c.n0) * m + c.m;
-#pragma unroll 1
-    for (int cc = 32 * c.part; cc < BN0; cc += 32 * c.nparts) {
-      float v[32], x[32];
-      tmem_ld32(c.taddr + cc, v);
-      if (!valid || c.n0 + cc >= n) continue;
-      load_f32x32(xrow + cc, x);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = a * x[j] + v[j];
-      store_f32x32(row + cc, v);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) colT[int64_t(cc + j) * m] = v[j];  // coalesced across the warp's rows
-    }
   }
 };
 
