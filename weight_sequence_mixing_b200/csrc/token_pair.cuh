@@ -45,10 +45,10 @@ struct PairShape {
   static constexpr int Z_STAGE = A_BYTES + BZ_BYTES;
   static constexpr int P_STAGE = A_BYTES + BP_BYTES;
   static constexpr int SLOT = Z_STAGE > P_STAGE ? Z_STAGE : P_STAGE;
-  static constexpr int STAGES = SWIGLU ? 5 : 6;
+  static constexpr int STAGES = 6;  // operand ring: the P and Z phases are bound by what is in flight
   static constexpr int EW = 16;           // epilogue warps: 4 per TMEM lane quarter
   static constexpr int STG_BYTES = 1024;  // one [32 rows][16 bf16] output box
-  static constexpr int STG_BOXES = 4;     // ring of output boxes per epilogue warp
+  static constexpr int STG_BOXES = 2;     // ring of output boxes per epilogue warp
   static constexpr int STG_WARP = STG_BOXES * STG_BYTES;
   static constexpr int SMEM = 1024 + STAGES * SLOT + EW * STG_WARP + 256;
   static constexpr int ZN = SWIGLU ? 256 : 128;  // MMA N of the Z phase (both halves)
