@@ -25,6 +25,15 @@ extern "C" {
 int ttt_selftest_gemm(int elem_bytes, int a_mn, int b_mn, int bn, int M, int N, int K, int batches, int splits,
                       const void* A, const void* B, float* C, void* stream);
 
+/* Failure detection without a fault: launches one CTA that waits on an mbarrier no one
+ * arrives at.  The wait gives up after the library's limit (2 s), as every wait of the
+ * path does, records a timeout in the 4-byte device status word `status_word` (any
+ * device buffer of at least 4 bytes, zeroed by the call first) and returns; the CUDA
+ * context stays usable.  Synchronises `stream` and returns what the word maps to:
+ * TTT_ERR_TIMEOUT when the wait ran out (the expected result), TTT_OK otherwise,
+ * TTT_ERR_CUDA / TTT_ERR_INVALID_ARG on a launch or argument error. */
+int ttt_selftest_timeout(void* status_word, cudaStream_t stream);
+
 /* Per-stage timing of a handle's forward calls.  ttt_profile_enable(h, 1)
  * clears earlier records and starts recording a CUDA event pair around every
  * kernel launch of later ttt_forward calls, on the stream the kernel runs on;

@@ -35,7 +35,7 @@ EXPORTED = [
     "ttt_config_init", "ttt_create", "ttt_param_count", "ttt_workspace_size", "ttt_forward",
     "ttt_host_staging_size", "ttt_forward_host", "ttt_query_status", "ttt_destroy", "ttt_status_string",
     "ttt_selftest_gemm", "ttt_profile_enable", "ttt_profile_collect", "ttt_stage_name", "ttt_launch_count",
-    "ttt_forward_noalloc", "ttt_token_pair_capacity",
+    "ttt_forward_noalloc", "ttt_token_pair_capacity", "ttt_selftest_timeout",
 ]
 NUM_STAGES = 8
 
@@ -81,6 +81,7 @@ def _load():
         "ttt_launch_count": (i64, [vp]),
         "ttt_forward_noalloc": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "ttt_token_pair_capacity": (i32, [i32]),
+        "ttt_selftest_timeout": (i32, [vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -231,3 +232,8 @@ def selftest_gemm(A, B, elem_bytes, a_mn, b_mn, bn, M, N, K, batches, splits, st
 def token_pair_capacity(swiglu: bool) -> int:
     """CTA pairs of the token-phase kernel resident at once on the current device (0: single-CTA fallback)."""
     return int(LIB.ttt_token_pair_capacity(int(bool(swiglu))))
+
+
+def selftest_timeout(status_word: torch.Tensor, stream=None) -> int:
+    """Status (TTT_ERR_TIMEOUT expected) of a kernel whose bounded wait runs out; see ttt_diag.h."""
+    return int(LIB.ttt_selftest_timeout(_ptr(status_word), _stream_ptr(stream)))

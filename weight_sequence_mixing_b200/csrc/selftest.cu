@@ -88,3 +88,34 @@ extern "C" int ttt_selftest_gemm(int elem_bytes, int a_mn, int b_mn, int bn, int
   }
   return TTT_ERR_UNSUPPORTED;
 }
+
+namespace ttt {
+namespace {
+
+// An mbarrier that expects one arrival which never comes: the bounded wait runs out.
+__global__ void stuck_wait_kernel(unsigned* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, &abort_flag)) set_status(status, kStatusTimeout);
+}
+
+}  // namespace
+}  // namespace ttt
+
+extern "C" int ttt_selftest_timeout(void* status_word, cudaStream_t stream) {
+  if (!status_word) return TTT_ERR_INVALID_ARG;
+  unsigned* w = static_cast<unsigned*>(status_word);
+  if (cudaMemsetAsync(w, 0, sizeof(unsigned), stream) != cudaSuccess) return TTT_ERR_CUDA;
+  ttt::stuck_wait_kernel<<<1, 32, 0, stream>>>(w);
+  if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
+  unsigned word = 0;
+  if (cudaMemcpyAsync(&word, w, sizeof(word), cudaMemcpyDeviceToHost, stream) != cudaSuccess) return TTT_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return TTT_ERR_CUDA;
+  return (word & ttt::kStatusTimeout) ? TTT_ERR_TIMEOUT : TTT_OK;
+}
