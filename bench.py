@@ -325,13 +325,9 @@ def main():
     layer.profile(False)
     layer.check_status()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(step_ms)
-    if dist:
-        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, "cuda")
     tokens_per_step = cfg["B"] * cfg["N"]
-    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+    value = job_throughput(world, tokens_per_step, args.steps, total_ms)
     ms_per_step = total_ms / args.steps
 
     # ---- end to end through the host-buffer entry point (pinned host memory)
@@ -412,6 +408,21 @@ def main():
         dist.destroy_process_group()
 
 
+def max_over_ranks(ms: float, dist, device: str) -> float:
+    """The slowest rank's device time: every rank takes part (MAX all-reduce)."""
+    if not dist:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_step: int, steps: int, total_ms: float) -> float:
+    """Whole-job tokens/s: every rank runs its own replica of the workload (weak scaling),
+    timed by the slowest rank."""
+    return world * tokens_per_step * steps / (total_ms / 1e3)
+
+
 def run_e2e(args, cfg, layer, x, h2d, d2h, stream, dist, world):
     pin = {k: (v.pin_memory() if v is not None else None) for k, v in x.items()}
     O_h = torch.empty((cfg["B"], cfg["H"], cfg["Nq"], cfg["d"]), dtype=layer.io_dtype).pin_memory()
@@ -435,13 +446,9 @@ def run_e2e(args, cfg, layer, x, h2d, d2h, stream, dist, world):
         call()
         e[i].record(stream)
     torch.cuda.synchronize()
-    total = sum(a.elapsed_time(b) for a, b in zip(s, e))
-    if dist:
-        t = torch.tensor([total], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total = float(t.item())
+    total = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(s, e)), dist, "cuda")
     del staging
-    return {"value": world * cfg["B"] * cfg["N"] * n / (total / 1e3), "unit": "tokens/s",
+    return {"value": job_throughput(world, cfg["B"] * cfg["N"], n, total), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": total / n,
             "api": "ttt_forward_host (pinned host buffers; copies inside the timed region)"}
 
