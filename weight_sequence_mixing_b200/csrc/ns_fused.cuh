@@ -217,7 +217,11 @@ __global__ void __launch_bounds__(192, 1)
             float v[32];
             tmem_ld32(tacc + cc, v);
             if (step == 0) {
-              store_f32x32(g.S + zk * mm + int64_t(row) * g.m + c0 + cc, v);
+              // S is symmetric: write the tile transposed, into the mirrored position, so that
+              // the warp's 32 lanes (consecutive rows) store consecutive addresses
+              float* colS = g.S + zk * mm + int64_t(c0 + cc) * g.m + row;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) colS[int64_t(i) * g.m] = v[i];
             } else {
               // the prefetched fp32 tile: box cc/32, row lrow, 16-byte chunk k at k ^ (lrow & 7)
               const float4* box = reinterpret_cast<const float4*>(ebuf + (cc / 32) * 128 * 128 + lrow * 128);
@@ -231,9 +235,10 @@ __global__ void __launch_bounds__(192, 1)
                 e[4 * k + 3] = f.w;
               }
               if (step == 1) {
+                // T = b S + c S S is symmetric too: transposed, mirrored store as for S
+                float* colT = g.T + zk * mm + int64_t(c0 + cc) * g.m + row;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = g.b * e[i] + g.c * v[i];
-                store_f32x32(g.T + zk * mm + int64_t(row) * g.m + c0 + cc, v);
+                for (int i = 0; i < 32; ++i) colT[int64_t(i) * g.m] = g.b * e[i] + g.c * v[i];
               } else {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = g.a * e[i] + v[i];
