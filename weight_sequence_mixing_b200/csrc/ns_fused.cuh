@@ -12,10 +12,13 @@
 // separates the steps (every step reads what the previous one wrote).
 // X is kept twice, as X [m][n] and X^T [n][m], so every operand is K-major.
 //
+// Stores: S and T (symmetric) are written transposed into their mirrored tiles and
+// X^T column-wise, so a warp's lanes (consecutive rows) store consecutive addresses;
+// X' rows go back into the prefetch buffer and leave by TMA.
 // Memory ordering across a step boundary: epilogue threads write with generic
-// stores, issue fence.proxy.async.global and arrive on the cluster barrier with
-// release semantics; after the acquiring wait the producer fences again before
-// its TMA loads read those values.
+// stores and wait for their TMA stores to complete, issue fence.proxy.async.global
+// and arrive on the cluster barrier with release semantics; after the acquiring
+// wait the producer fences again before its TMA loads read those values.
 #pragma once
 #include "epilogues.cuh"
 
@@ -88,7 +91,8 @@ template <int CS>
 __global__ void __launch_bounds__(192, 1)
     ns_fused_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mXT,
                     const __grid_constant__ CUtensorMap mX2, const __grid_constant__ CUtensorMap mXT2,
-                    const __grid_constant__ CUtensorMap mS, const __grid_constant__ CUtensorMap mT, const NsGeom g,
+                    const __grid_constant__ CUtensorMap mS, const __grid_constant__ CUtensorMap mT,
+                    const __grid_constant__ CUtensorMap sX, const __grid_constant__ CUtensorMap sX2, const NsGeom g,
                     unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -204,8 +208,7 @@ __global__ void __launch_bounds__(192, 1)
           const int r0 = (t / sp.tiles_n) * 128, c0 = (t % sp.tiles_n) * 128;
           const int row = r0 + q * 32 + lane;
           const bool odd = it & 1;
-          float* nx = odd ? g.X : g.X2;  // X of the next iteration
-          float* nxt = odd ? g.XT : g.XT2;
+          float* nxt = odd ? g.XT : g.XT2;  // X^T of the next iteration
           const uint32_t tacc = taddr + static_cast<uint32_t>(buf * 128);
           const int lrow = q * 32 + lane;  // row inside the tile (and the prefetched box)
           if (step > 0) {
@@ -242,11 +245,29 @@ __global__ void __launch_bounds__(192, 1)
               } else {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = g.a * e[i] + v[i];
-                store_f32x32(nx + zk * mn + int64_t(row) * g.n + c0 + cc, v);
+                // X' rows go back into the prefetched tile's place in shared memory (same
+                // swizzled layout) and leave as TMA stores after the last chunk
+                float4* wbox = reinterpret_cast<float4*>(ebuf + (cc / 32) * 128 * 128 + lrow * 128);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                  wbox[k ^ (lrow & 7)] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
                 float* colT = nxt + zk * mn + int64_t(c0 + cc) * g.m + row;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) colT[int64_t(i) * g.m] = v[i];  // coalesced across the warp
               }
+            }
+          }
+          if (step == 2) {
+            // this warp's 32 rows of X' (4 boxes of 32 columns) from shared memory to X;
+            // the prefetch buffer is released once the stores have read it
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              const CUtensorMap* dst = (it & 1) ? &sX : &sX2;
+              for (int bx = 0; bx < 4; ++bx)
+                tma_store_3d(dst, ebuf + bx * 128 * 128 + q * 32 * 128, c0 + 32 * bx, r0 + q * 32, zk);
+              bulk_commit();
+              bulk_wait_read0();
             }
           }
           if (step > 0) {
@@ -259,7 +280,8 @@ __global__ void __launch_bounds__(192, 1)
           if (lane == 0) mbar_arrive(&tmem_empty[buf]);
           ++j_tile;
         }
-        fence_proxy_async_global();  // these generic stores -> the next step's TMA loads
+        if (lane == 0) bulk_wait0();  // the X' stores are complete
+        fence_proxy_async_global();  // these stores -> the next step's TMA loads
       }
       cluster_sync_all();
     }
@@ -280,14 +302,17 @@ __global__ void __launch_bounds__(192, 1)
 // X: Newton-Schulz input (normalised) in g.X / g.XT; result in (g.iters odd ? X2 : X).
 template <int CS>
 cudaError_t launch_ns_fused_cs(int nmat, const NsGeom& g, unsigned* status, cudaStream_t st) {
-  CUtensorMap mX, mXT, mX2, mXT2, mS, mT;
+  CUtensorMap mX, mXT, mX2, mXT2, mS, mT, sX, sX2;
   const int m = g.m, n = g.n;
   if (!make_tmap(&mX, g.X, 4, n, m, nmat, n, int64_t(m) * n, 128) ||
       !make_tmap(&mXT, g.XT, 4, m, n, nmat, m, int64_t(m) * n, 128) ||
       !make_tmap(&mX2, g.X2, 4, n, m, nmat, n, int64_t(m) * n, 128) ||
       !make_tmap(&mXT2, g.XT2, 4, m, n, nmat, m, int64_t(m) * n, 128) ||
       !make_tmap(&mS, g.S, 4, m, m, nmat, m, int64_t(m) * m, 128) ||
-      !make_tmap(&mT, g.T, 4, m, m, nmat, m, int64_t(m) * m, 128))
+      !make_tmap(&mT, g.T, 4, m, m, nmat, m, int64_t(m) * m, 128) ||
+      // stores of one epilogue warp's 32 rows of X'
+      !make_tmap(&sX, g.X, 4, n, m, nmat, n, int64_t(m) * n, 32) ||
+      !make_tmap(&sX2, g.X2, 4, n, m, nmat, n, int64_t(m) * n, 32))
     return cudaErrorInvalidValue;
   auto kern = ns_fused_kernel<CS>;
   static bool configured = false;
@@ -312,7 +337,7 @@ cudaError_t launch_ns_fused_cs(int nmat, const NsGeom& g, unsigned* status, cuda
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, mX, mXT, mX2, mXT2, mS, mT, g, status);
+  return cudaLaunchKernelEx(&cfg, kern, mX, mXT, mX2, mXT2, mS, mT, sX, sX2, g, status);
 }
 
 // Whether a cluster of CS CTAs of this kernel can be resident at all on this device.
