@@ -25,6 +25,17 @@ extern "C" {
 int ttt_selftest_gemm(int elem_bytes, int a_mn, int b_mn, int bn, int M, int N, int K, int batches, int splits,
                       const void* A, const void* B, float* C, void* stream);
 
+/* The execution plan ttt_create chose (host logic only, no GPU needed).  Writes up to
+ * `n` ints into `info`, in this order:
+ *   [0] path: 0 fp32 SIMT, 1 bf16 tensor cores
+ *   [1] chunk length in tokens, [2] number of chunks
+ *   [3] split-K splits of the weight-gradient reductions (bf16 path; 0 on fp32)
+ *   [4] rows per weight-gradient tile: 128 or 256 on single CTAs, 512 on CTA pairs
+ *   [5] output columns per weight-gradient tile
+ *   [6] 1 when unsplit reductions write U (and momentum) directly, without partials
+ * Returns the number of entries written, or TTT_ERR_INVALID_ARG. */
+int ttt_plan_info(const ttt_handle* handle, int* info, int n);
+
 /* Failure detection without a fault: launches one CTA that waits on an mbarrier no one
  * arrives at.  The wait gives up after the library's limit (2 s), as every wait of the
  * path does, records a timeout in the 4-byte device status word `status_word` (any

@@ -35,7 +35,7 @@ EXPORTED = [
     "ttt_config_init", "ttt_create", "ttt_param_count", "ttt_workspace_size", "ttt_forward",
     "ttt_host_staging_size", "ttt_forward_host", "ttt_query_status", "ttt_destroy", "ttt_status_string",
     "ttt_selftest_gemm", "ttt_profile_enable", "ttt_profile_collect", "ttt_stage_name", "ttt_launch_count",
-    "ttt_forward_noalloc", "ttt_token_pair_capacity", "ttt_selftest_timeout",
+    "ttt_forward_noalloc", "ttt_token_pair_capacity", "ttt_selftest_timeout", "ttt_plan_info",
 ]
 NUM_STAGES = 8
 
@@ -82,6 +82,7 @@ def _load():
         "ttt_forward_noalloc": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "ttt_token_pair_capacity": (i32, [i32]),
         "ttt_selftest_timeout": (i32, [vp, vp]),
+        "ttt_plan_info": (i32, [vp, ctypes.POINTER(ctypes.c_int), i32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -237,3 +238,21 @@ def token_pair_capacity(swiglu: bool) -> int:
 def selftest_timeout(status_word: torch.Tensor, stream=None) -> int:
     """Status (TTT_ERR_TIMEOUT expected) of a kernel whose bounded wait runs out; see ttt_diag.h."""
     return int(LIB.ttt_selftest_timeout(_ptr(status_word), _stream_ptr(stream)))
+
+
+PLAN_FIELDS = ("path", "chunk", "nchunks", "splits", "tile_rows", "grad_bn", "direct")
+
+
+def plan_info(cfg: dict) -> dict:
+    """The execution plan ttt_create chooses for `cfg` (host logic; no GPU needed)."""
+    c = make_config(cfg)
+    h = ctypes.c_void_p()
+    _check(LIB.ttt_create(ctypes.byref(c), ctypes.byref(h)), "ttt_create")
+    try:
+        buf = (ctypes.c_int * len(PLAN_FIELDS))()
+        n = LIB.ttt_plan_info(h, buf, len(PLAN_FIELDS))
+        if n < 0:
+            raise TTTError(n, "ttt_plan_info")
+        return dict(zip(PLAN_FIELDS, list(buf)[:n]))
+    finally:
+        LIB.ttt_destroy(h)

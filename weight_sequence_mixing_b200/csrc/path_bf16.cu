@@ -937,3 +937,19 @@ int run_bf16(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
 extern "C" int ttt_token_pair_capacity(int swiglu) {
   return swiglu ? ttt::token_pair_capacity<true>() : ttt::token_pair_capacity<false>();
 }
+
+extern "C" int ttt_plan_info(const ttt_handle* h, int* info, int n) {
+  if (!h || !info || n < 0) return TTT_ERR_INVALID_ARG;
+  const ttt::Plan& p = h->plan;
+  int v[7] = {p.path == ttt::kPathBf16 ? 1 : 0, static_cast<int>(p.chunk), static_cast<int>(p.nchunks), 0, 0, 0, 0};
+  if (p.path == ttt::kPathBf16) {
+    const ttt::Dims D = ttt::dims_of(p);
+    v[3] = D.splits;
+    v[4] = D.tile_rows;
+    v[5] = D.grad_bn;
+    v[6] = D.direct ? 1 : 0;
+  }
+  const int m = n < 7 ? n : 7;
+  for (int i = 0; i < m; ++i) info[i] = v[i];
+  return m;
+}
