@@ -65,10 +65,11 @@ def algorithmic_flops(cfg) -> dict:
         for _, r, c in matrix_shapes(cfg):
             m, n = min(r, c), max(r, c)
             ns += cfg["ns_iters"] * (4 * m * m * n + 2 * m ** 3)
+    ep = max(1, int(cfg.get("epochs", 1)))  # full-batch steps per chunk
     return {
-        "token_phase": float(BH) * N * tok,
-        "weight_grad": float(BH) * N * grad,
-        "newton_schulz": float(BH) * nchunks * ns,
+        "token_phase": float(BH) * N * tok * ep,
+        "weight_grad": float(BH) * N * grad * ep,
+        "newton_schulz": float(BH) * nchunks * ns * ep,
         "apply": float(BH) * Nq * app,
     }
 

@@ -94,6 +94,9 @@ typedef struct ttt_config {
   int32_t ns_iters;   /* Newton-Schulz iterations (default 5) */
   float ns_coeff[3];  /* quintic (a, b, c), default (3.4445, -4.7750, 2.0315) */
   float in_eps;       /* instance-norm epsilon (default 1e-5) */
+  int32_t epochs;     /* full-batch inner steps per chunk, 1..64 (default 1; 0 reads as 1): the
+                         inner model trains for `epochs` passes over each chunk before moving on
+                         (ViT3 digest, inner-training ablation); momentum carries through */
 } ttt_config;
 
 typedef struct ttt_handle ttt_handle;

@@ -255,16 +255,21 @@ def forward_head(cfg, Q, K, V, eta, w0):
     W = unpack(kind, d, h, w0)
     M = {name: np.zeros_like(m) for name, m in W.items()}
     bounds = chunk_bounds(N, cfg["chunk"])
+    # inner epochs: that many full-batch steps on each chunk before the next one
+    # (ViT3 digest, inner-training ablation); momentum carries through them
+    epochs = max(1, int(cfg.get("epochs", 1)))
     if cfg["causal"]:
         if Q.shape[0] != N:
             raise ValueError("causal order needs Nq == N")
         O = np.empty((N, d), dtype=F64)
         for s, e in bounds:
             O[s:e] = inner_forward(kind, W, Q[s:e])[0]
-            update_chunk(cfg, W, M, K[s:e], V[s:e], eta[s:e])
+            for _ in range(epochs):
+                update_chunk(cfg, W, M, K[s:e], V[s:e], eta[s:e])
     else:
         for s, e in bounds:
-            update_chunk(cfg, W, M, K[s:e], V[s:e], eta[s:e])
+            for _ in range(epochs):
+                update_chunk(cfg, W, M, K[s:e], V[s:e], eta[s:e])
         O = inner_forward(kind, W, Q)[0]
     return O, pack(kind, d, h, W)
 

@@ -42,7 +42,7 @@ _DEFAULTS = dict(
     key_instnorm=False, weight_l2norm=False, direct_launch=False, single_cta=False,
     eta_mode="scalar",           # "scalar" | "per_token"
     eta_scalar=1.0, lr=1.0, momentum=0.9,
-    ns_iters=5, ns_coeff=(3.4445, -4.7750, 2.0315), in_eps=1e-5,
+    ns_iters=5, ns_coeff=(3.4445, -4.7750, 2.0315), in_eps=1e-5, epochs=1,
     data="vit", seed=7,
 )
 

@@ -65,7 +65,8 @@ def test_invalid_configurations_are_rejected(bad):
 
 def test_invalid_enum_and_flag_values_are_rejected():
     from weight_sequence_mixing_b200 import binding
-    for field, value in (("inner", 7), ("loss", -1), ("opt", 9), ("dtype", 5), ("flags", 64), ("ns_iters", -1)):
+    for field, value in (("inner", 7), ("loss", -1), ("opt", 9), ("dtype", 5), ("flags", 64), ("ns_iters", -1),
+                         ("epochs", -1), ("epochs", 65)):
         c = binding.make_config(make_config(N=16, d=64, h=128))
         setattr(c, field, value)
         st, h = _create(c)

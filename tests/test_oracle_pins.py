@@ -389,3 +389,27 @@ def test_forward_all_heads_matches_per_head():
                                     x["V"][b, hh].double().numpy(), x["eta"][b, hh].double().numpy(),
                                     x["W0"][hh].double().numpy())
             assert np.array_equal(O[b, hh], o) and np.array_equal(W[b, hh], w)
+
+
+# ---------------------------------------------------------------- inner epochs
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("rownorm", [False, True])
+def test_epochs_are_repeated_full_batch_steps(kind, rownorm):
+    # plain GD (no state carried between calls): E epochs over one chunk equal E calls
+    # that each take one step, the next starting from the previous call's W*
+    d, h, N = 4, 6, 9
+    cfg1 = cfg_for(kind, "mse", d=d, h=h, N=N, weight_l2norm=rownorm)
+    cfg3 = cfg_for(kind, "mse", d=d, h=h, N=N, weight_l2norm=rownorm, epochs=3)
+    Q, K, V, eta = rand(1, 1, N, d), rand(1, 1, N, d), rand(1, 1, N, d), np.abs(rand(1, 1, N, scale=0.3))
+    W = orc.pack(kind, d, h, rand_w(kind, d, h))[None]
+    O3, W3 = orc.forward(cfg3, Q, K, V, eta, W)
+    Wi = W
+    for _ in range(3):
+        Oi, Wstep = orc.forward(cfg1, Q, K, V, eta, Wi)
+        Wi = Wstep[:, 0]
+    assert np.allclose(W3[:, 0], Wi, rtol=1e-12, atol=1e-12)
+    assert np.allclose(O3, Oi, rtol=1e-12, atol=1e-12)
+    # and one epoch is the default
+    O1, W1 = orc.forward(cfg1, Q, K, V, eta, W)
+    O1b, W1b = orc.forward(cfg_for(kind, "mse", d=d, h=h, N=N, weight_l2norm=rownorm, epochs=1), Q, K, V, eta, W)
+    assert np.array_equal(W1, W1b) and np.array_equal(O1, O1b)

@@ -54,6 +54,11 @@ SMALL = [
     dict(inner="mlp2_gelu", loss="neg_dot", opt="momentum", d=128, h=256, N=400, chunk=256, weight_l2norm=True),
     dict(inner="linear", loss="neg_dot", opt="gd", d=128, h=128, N=260),
     dict(inner="linear", loss="mse", opt="momentum_muon", d=128, h=128, N=390, chunk=128, weight_l2norm=True),
+    # inner epochs: repeated full-batch steps per chunk, momentum carried through them
+    dict(inner="swiglu", loss="neg_dot", opt="momentum_muon", d=128, h=256, N=700, chunk=256, Nq=200,
+         weight_l2norm=True, epochs=2),
+    dict(inner="mlp2_gelu", loss="mse", opt="gd", d=64, h=256, N=700, key_instnorm=True, data="vit",
+         eta_mode="scalar", eta_scalar=1.0, epochs=3),
 ]
 
 

@@ -26,6 +26,9 @@ SMALL = [
     dict(inner="swiglu", loss="neg_dot", opt="momentum", chunk=50, causal=1, weight_l2norm=True),
     dict(inner="swiglu", loss="mse", opt="muon", weight_l2norm=True, key_instnorm=True),
     dict(inner="swiglu", loss="neg_dot", opt="momentum_muon", chunk=70, weight_l2norm=True, Nq=33),
+    # inner epochs: repeated full-batch steps per chunk, momentum carried through them
+    dict(inner="mlp2_gelu", loss="mse", opt="momentum", chunk=64, key_instnorm=True, epochs=3),
+    dict(inner="swiglu", loss="neg_dot", opt="momentum", chunk=50, causal=1, weight_l2norm=True, epochs=2),
 ]
 
 

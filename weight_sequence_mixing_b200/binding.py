@@ -47,7 +47,7 @@ class TTTConfig(ctypes.Structure):
         ("inner", ctypes.c_int32), ("loss", ctypes.c_int32), ("opt", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("flags", ctypes.c_uint32), ("eta_scalar", ctypes.c_float), ("lr", ctypes.c_float),
         ("momentum", ctypes.c_float), ("ns_iters", ctypes.c_int32), ("ns_coeff", ctypes.c_float * 3),
-        ("in_eps", ctypes.c_float),
+        ("in_eps", ctypes.c_float), ("epochs", ctypes.c_int32),
     ]
 
 
@@ -134,6 +134,7 @@ def make_config(cfg: dict) -> TTTConfig:
     for i in range(3):
         c.ns_coeff[i] = float(cfg["ns_coeff"][i])
     c.in_eps = float(cfg["in_eps"])
+    c.epochs = int(cfg.get("epochs", 1))
     return c
 
 

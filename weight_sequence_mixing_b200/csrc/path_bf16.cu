@@ -924,7 +924,7 @@ int run_bf16(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
   for (int ci = 0; ci < p.nchunks; ++ci) {
     const int t0 = ci * p.chunk, n = std::min(p.chunk, cfg.N - t0);
     if (cfg.causal) TRY(apply_rows(c, t0, n));
-    TRY(update_chunk(c, t0, n));
+    for (int ep = 0; ep < p.epochs; ++ep) TRY(update_chunk(c, t0, n));
   }
   if (!cfg.causal) TRY(apply_rows(c, 0, cfg.Nq));
   if (io.W_out)

@@ -482,7 +482,7 @@ int run_f32(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
       r = inner_forward(p, v, st, MatRef{Q + int64_t(t0) * d, q_sz, d, 1}, n, O + int64_t(t0) * d, q_sz, d);
       if (r) return r;
     }
-    r = update_chunk(p, v, io, st, t0, n);
+    for (int ep = 0; ep < p.epochs && !r; ++ep) r = update_chunk(p, v, io, st, t0, n);
   }
   if (r) return r;
   if (!c.causal) {

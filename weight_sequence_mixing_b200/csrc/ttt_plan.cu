@@ -20,6 +20,7 @@ int plan_build(const ttt_config& c, Plan* p) {
                    TTT_FLAG_SINGLE_CTA)) != 0)
     return TTT_ERR_INVALID_ARG;
   if (c.ns_iters < 0 || c.ns_iters > 100) return TTT_ERR_INVALID_ARG;
+  if (c.epochs < 0 || c.epochs > 64) return TTT_ERR_INVALID_ARG;
   if (!std::isfinite(c.eta_scalar) || !std::isfinite(c.lr) || !std::isfinite(c.momentum) ||
       !std::isfinite(c.in_eps) || c.in_eps < 0.0f)
     return TTT_ERR_INVALID_ARG;
@@ -29,6 +30,7 @@ int plan_build(const ttt_config& c, Plan* p) {
   if (c.d > 4096 || c.h > 16384) return TTT_ERR_UNSUPPORTED;
 
   p->cfg = c;
+  p->epochs = c.epochs == 0 ? 1 : c.epochs;
   const int64_t d = c.d, h = c.inner == TTT_INNER_LINEAR ? c.d : c.h;
   p->cfg.h = static_cast<int32_t>(h);
   p->P = c.inner == TTT_INNER_LINEAR ? d * d : c.inner == TTT_INNER_MLP2_GELU ? 2 * d * h : 3 * d * h;

@@ -28,6 +28,7 @@ struct Plan {
   int BH = 0;          // B * H
   int chunk = 0;       // tokens per chunk (== N for one chunk)
   int nchunks = 0;
+  int epochs = 1;      // full-batch steps per chunk
   int path = kPathF32;
   size_t ws_bytes = 0;
   // host-staging layout (ttt_forward_host)
