@@ -74,6 +74,10 @@ typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
 #define TTT_FLAG_KEY_INSTNORM 1u  /* normalise each key channel over the chunk's tokens */
 #define TTT_FLAG_WEIGHT_L2NORM 2u /* unit L2 norm for every weight row after each update */
 #define TTT_FLAG_DIRECT_LAUNCH 4u /* launch every kernel on each call instead of replaying a cached CUDA graph */
+#define TTT_FLAG_W0_PER_BATCH 16u /* W0 is [B, H, P], one fast-weight state per batch entry (the W_out
+                                     of the previous call on the same sequences: streaming) */
+#define TTT_FLAG_NO_UPDATE 32u /* read-only: O = F_{W0}(Q) and W_out = W0, no update (LaCT
+                                  "Video and distributed": chunks that only read the state) */
 #define TTT_FLAG_SINGLE_CTA 8u /* token phase and weight-gradient GEMMs on single CTAs instead of CTA
                                   pairs; same results up to fp32 summation order, for comparison and tests */
 

@@ -256,8 +256,9 @@ def forward_head(cfg, Q, K, V, eta, w0):
     M = {name: np.zeros_like(m) for name, m in W.items()}
     bounds = chunk_bounds(N, cfg["chunk"])
     # inner epochs: that many full-batch steps on each chunk before the next one
-    # (ViT3 digest, inner-training ablation); momentum carries through them
-    epochs = max(1, int(cfg.get("epochs", 1)))
+    # (ViT3 digest, inner-training ablation); momentum carries through them.  A
+    # read-only call takes none (LaCT "Video and distributed": chunks that only read).
+    epochs = 0 if cfg.get("no_update", False) else max(1, int(cfg.get("epochs", 1)))
     if cfg["causal"]:
         if Q.shape[0] != N:
             raise ValueError("causal order needs Nq == N")
@@ -294,7 +295,9 @@ def forward(cfg, Q, K, V, eta, W0, heads=None):
     Ws = np.full((B, H, P), np.nan)
     todo = heads if heads is not None else [(b, hh) for b in range(B) for hh in range(H)]
     W0n = _np(W0)
+    per_batch = bool(cfg.get("w0_per_batch", False))  # W0 [B, H, P]: one state per entry
     for b, hh in todo:
         e = None if eta is None else _np(eta[b, hh])
-        O[b, hh], Ws[b, hh] = forward_head(cfg, _np(Q[b, hh]), _np(K[b, hh]), _np(V[b, hh]), e, W0n[hh])
+        w0 = W0n[b, hh] if per_batch else W0n[hh]
+        O[b, hh], Ws[b, hh] = forward_head(cfg, _np(Q[b, hh]), _np(K[b, hh]), _np(V[b, hh]), e, w0)
     return O, Ws

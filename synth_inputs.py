@@ -40,6 +40,7 @@ _DEFAULTS = dict(
     B=1, H=1, N=128, Nq=None, d=64, h=64, chunk=0, causal=0,
     inner="mlp2_gelu", loss="mse", opt="gd", dtype="bf16",
     key_instnorm=False, weight_l2norm=False, direct_launch=False, single_cta=False,
+    w0_per_batch=False, no_update=False,
     eta_mode="scalar",           # "scalar" | "per_token"
     eta_scalar=1.0, lr=1.0, momentum=0.9,
     ns_iters=5, ns_coeff=(3.4445, -4.7750, 2.0315), in_eps=1e-5, epochs=1,

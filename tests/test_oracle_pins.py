@@ -413,3 +413,59 @@ def test_epochs_are_repeated_full_batch_steps(kind, rownorm):
     O1, W1 = orc.forward(cfg1, Q, K, V, eta, W)
     O1b, W1b = orc.forward(cfg_for(kind, "mse", d=d, h=h, N=N, weight_l2norm=rownorm, epochs=1), Q, K, V, eta, W)
     assert np.array_equal(W1, W1b) and np.array_equal(O1, O1b)
+
+
+# ---------------------------------------------------------------- streaming state
+def _data(B, H, N, d, scale=0.3):
+    return (rand(B, H, N, d), rand(B, H, N, d), rand(B, H, N, d), np.abs(rand(B, H, N, scale=scale)))
+
+
+@pytest.mark.parametrize("kind", KINDS)
+def test_w0_per_batch_with_equal_states_matches_shared_w0(kind):
+    d, h, N, B, H = 4, 6, 7, 2, 2
+    Q, K, V, eta = _data(B, H, N, d)
+    W0 = np.stack([orc.pack(kind, d, h, rand_w(kind, d, h)) for _ in range(H)])
+    cfg = dict(B=B, H=H, d=d, h=h, N=N, opt="momentum", weight_l2norm=True)
+    Os, Ws = orc.forward(cfg_for(kind, "neg_dot", **cfg), Q, K, V, eta, W0)
+    Ob, Wb = orc.forward(cfg_for(kind, "neg_dot", w0_per_batch=True, **cfg), Q, K, V, eta,
+                         np.broadcast_to(W0, (B, H, W0.shape[1])))
+    assert np.array_equal(Os, Ob) and np.array_equal(Ws, Wb)
+
+
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("causal", [0, 1])
+def test_no_update_reads_the_initial_weights(kind, causal):
+    d, h, N = 4, 6, 9
+    Q, K, V, eta = _data(1, 1, N, d)
+    w = rand_w(kind, d, h)
+    W0 = orc.pack(kind, d, h, w)[None]
+    cfg = cfg_for(kind, "mse", d=d, h=h, N=N, chunk=4, causal=causal, no_update=True, weight_l2norm=True,
+                  opt="momentum")
+    O, W = orc.forward(cfg, Q, K, V, eta, W0)
+    assert np.array_equal(W[0, 0], W0[0])
+    assert np.allclose(O[0, 0], orc.inner_forward(kind, w, Q[0, 0])[0], rtol=1e-14, atol=1e-14)
+
+
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("causal", [0, 1])
+def test_streaming_two_calls_equal_one_chunked_call(kind, causal):
+    # plain GD: the state is the weights alone, so feeding W_out of a call on the first half
+    # of the tokens back as W0 of a call on the second half gives the one-call result
+    d, h, N, B, H = 4, 6, 12, 2, 1
+    Q, K, V, eta = _data(B, H, N, d)
+    W0 = orc.pack(kind, d, h, rand_w(kind, d, h))[None]
+    half = N // 2
+    base = dict(B=B, H=H, d=d, h=h, weight_l2norm=True, causal=causal)
+    O1, W1 = orc.forward(cfg_for(kind, "neg_dot", N=N, chunk=half, **base), Q, K, V, eta, W0)
+    sl = lambda t, a, b: t[:, :, a:b]
+    qa = sl(Q, 0, half) if causal else Q
+    qb = sl(Q, half, N) if causal else Q
+    Oa, Wa = orc.forward(cfg_for(kind, "neg_dot", N=half, Nq=qa.shape[2], **base), qa, sl(K, 0, half),
+                         sl(V, 0, half), sl(eta, 0, half), W0)
+    Ob, Wb = orc.forward(cfg_for(kind, "neg_dot", N=half, Nq=qb.shape[2], w0_per_batch=True, **base), qb,
+                         sl(K, half, N), sl(V, half, N), sl(eta, half, N), Wa)
+    assert np.allclose(Wb, W1, rtol=1e-12, atol=1e-12)
+    if causal:
+        assert np.allclose(np.concatenate([Oa, Ob], axis=2), O1, rtol=1e-12, atol=1e-12)
+    else:
+        assert np.allclose(Ob, O1, rtol=1e-12, atol=1e-12)

@@ -30,6 +30,8 @@ FLAG_KEY_INSTNORM = 1
 FLAG_WEIGHT_L2NORM = 2
 FLAG_DIRECT_LAUNCH = 4
 FLAG_SINGLE_CTA = 8
+FLAG_W0_PER_BATCH = 16
+FLAG_NO_UPDATE = 32
 
 EXPORTED = [
     "ttt_config_init", "ttt_create", "ttt_param_count", "ttt_workspace_size", "ttt_forward",
@@ -126,7 +128,9 @@ def make_config(cfg: dict) -> TTTConfig:
     c.dtype = DTYPE[cfg["dtype"]]
     c.flags = ((FLAG_KEY_INSTNORM if cfg["key_instnorm"] else 0) | (FLAG_WEIGHT_L2NORM if cfg["weight_l2norm"] else 0)
                | (FLAG_DIRECT_LAUNCH if cfg.get("direct_launch") else 0)
-               | (FLAG_SINGLE_CTA if cfg.get("single_cta") else 0))
+               | (FLAG_SINGLE_CTA if cfg.get("single_cta") else 0)
+               | (FLAG_W0_PER_BATCH if cfg.get("w0_per_batch") else 0)
+               | (FLAG_NO_UPDATE if cfg.get("no_update") else 0))
     c.eta_scalar = float(cfg["eta_scalar"])
     c.lr = float(cfg["lr"])
     c.momentum = float(cfg["momentum"])

@@ -907,8 +907,10 @@ int run_bf16(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
   // W = W0 per batch entry, zero momentum, bf16 copies
   {
     StageScope _sc(kStageOther, st);
+    // W0 [H][P] shared by the batch entries, or [B*H][P] with one state per entry
+    const int w0_rows = (cfg.flags & TTT_FLAG_W0_PER_BATCH) ? Z : cfg.H;
     init_weights_kernel<<<std::min<int64_t>((int64_t(Z) * p.P + 255) / 256, 4096), 256, 0, st>>>(
-        Z, cfg.H, p.P, io.W0, c.v.at<float>(p, xWf));
+        Z, w0_rows, p.P, io.W0, c.v.at<float>(p, xWf));
   }
   TRY_CUDA(cudaMemsetAsync(c.v.at<float>(p, xMom), 0, size_t(Z) * D.GR * d * 4, st));
   {
@@ -924,6 +926,7 @@ int run_bf16(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
   for (int ci = 0; ci < p.nchunks; ++ci) {
     const int t0 = ci * p.chunk, n = std::min(p.chunk, cfg.N - t0);
     if (cfg.causal) TRY(apply_rows(c, t0, n));
+    if (cfg.flags & TTT_FLAG_NO_UPDATE) continue;
     for (int ep = 0; ep < p.epochs; ++ep) TRY(update_chunk(c, t0, n));
   }
   if (!cfg.causal) TRY(apply_rows(c, 0, cfg.Nq));

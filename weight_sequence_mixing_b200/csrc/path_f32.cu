@@ -234,7 +234,7 @@ __global__ void rownorm_kernel(int rows, int cols, float* W, int64_t w_sz) {
   for (int c = threadIdx.x & 31; c < cols; c += 32) row[c] *= inv;
 }
 
-// W[z] = W0[z % H]
+// W[z] = W0[z % H] (H = rows of W0: the heads, or every batch entry and head)
 __global__ void init_weights_kernel(int Z, int H, int64_t P, const float* W0, float* W) {
   const int64_t total = int64_t(Z) * P;
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
@@ -469,7 +469,8 @@ int run_f32(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
   const int64_t P = p.P, Rd = int64_t(p.off[kNumBuf]) * d;
   {
     StageScope _sc(kStageOther, st);
-    init_weights_kernel<<<grid_for(int64_t(Z) * P), 256, 0, st>>>(Z, c.H, P, io.W0, v.b[bW]);
+    const int w0_rows = (c.flags & TTT_FLAG_W0_PER_BATCH) ? Z : c.H;  // W0 [H][P] or [B*H][P]
+    init_weights_kernel<<<grid_for(int64_t(Z) * P), 256, 0, st>>>(Z, w0_rows, P, io.W0, v.b[bW]);
   }
   if (cudaMemsetAsync(v.b[bM], 0, size_t(Z) * P * 4, st) != cudaSuccess) return TTT_ERR_CUDA;
   const float* Q = static_cast<const float*>(io.Q);
@@ -482,6 +483,7 @@ int run_f32(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
       r = inner_forward(p, v, st, MatRef{Q + int64_t(t0) * d, q_sz, d, 1}, n, O + int64_t(t0) * d, q_sz, d);
       if (r) return r;
     }
+    if (c.flags & TTT_FLAG_NO_UPDATE) continue;
     for (int ep = 0; ep < p.epochs && !r; ++ep) r = update_chunk(p, v, io, st, t0, n);
   }
   if (r) return r;

@@ -188,7 +188,7 @@ extern "C" int ttt_forward_host(ttt_handle* h, const void* Q, const void* K, con
   const size_t nq = static_cast<size_t>(p.cfg.B) * p.cfg.H * p.cfg.Nq * p.cfg.d * es;
   const size_t nk = static_cast<size_t>(p.cfg.B) * p.cfg.H * p.cfg.N * p.cfg.d * es;
   const size_t ne = static_cast<size_t>(p.cfg.B) * p.cfg.H * p.cfg.N * 4;
-  const size_t nw0 = static_cast<size_t>(p.cfg.H) * p.P * 4;
+  const size_t nw0 = static_cast<size_t>((p.cfg.flags & TTT_FLAG_W0_PER_BATCH) ? p.BH : p.cfg.H) * p.P * 4;
   const size_t nw = static_cast<size_t>(p.cfg.B) * p.cfg.H * p.P * 4;
   if (cudaMemcpyAsync(dQ, Q, nq, cudaMemcpyHostToDevice, st) != cudaSuccess ||
       cudaMemcpyAsync(dK, K, nk, cudaMemcpyHostToDevice, st) != cudaSuccess ||

@@ -17,7 +17,7 @@ int plan_build(const ttt_config& c, Plan* p) {
   if (c.causal && c.Nq != c.N) return TTT_ERR_INVALID_ARG;
   if (c.inner != TTT_INNER_LINEAR && c.h < 1) return TTT_ERR_INVALID_ARG;
   if ((c.flags & ~(TTT_FLAG_KEY_INSTNORM | TTT_FLAG_WEIGHT_L2NORM | TTT_FLAG_DIRECT_LAUNCH |
-                   TTT_FLAG_SINGLE_CTA)) != 0)
+                   TTT_FLAG_SINGLE_CTA | TTT_FLAG_W0_PER_BATCH | TTT_FLAG_NO_UPDATE)) != 0)
     return TTT_ERR_INVALID_ARG;
   if (c.ns_iters < 0 || c.ns_iters > 100) return TTT_ERR_INVALID_ARG;
   if (c.epochs < 0 || c.epochs > 64) return TTT_ERR_INVALID_ARG;
@@ -46,7 +46,7 @@ int plan_build(const ttt_config& c, Plan* p) {
   p->stg_k = o; o = align_up(o + size_t(p->BH) * c.N * d * es, 256);
   p->stg_v = o; o = align_up(o + size_t(p->BH) * c.N * d * es, 256);
   p->stg_eta = o; o = align_up(o + size_t(p->BH) * c.N * 4, 256);
-  p->stg_w0 = o; o = align_up(o + size_t(c.H) * p->P * 4, 256);
+  p->stg_w0 = o; o = align_up(o + size_t((c.flags & TTT_FLAG_W0_PER_BATCH) ? p->BH : c.H) * p->P * 4, 256);
   p->stg_o = o; o = align_up(o + size_t(p->BH) * c.Nq * d * es, 256);
   p->stg_w = o; o = align_up(o + size_t(p->BH) * p->P * 4, 256);
   p->staging_bytes = o;
