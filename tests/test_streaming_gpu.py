@@ -50,9 +50,7 @@ def test_two_streamed_calls_equal_one_chunked_call(dtype, causal):
     O1, W1 = run_gpu(full, x)
 
     def part(a, b, w0, per_batch):
-        kw = dict(base, N=half)
-        if causal:
-            kw["Nq"] = half
+        kw = dict(base, N=half, Nq=half if causal else N)  # non-causal: the whole query set
         cfg = make_config(chunk=0, w0_per_batch=per_batch, **kw)
         q = x["Q"][:, :, a:b] if causal else x["Q"]
         xi = dict(Q=q.contiguous(), K=x["K"][:, :, a:b].contiguous(), V=x["V"][:, :, a:b].contiguous(),
