@@ -43,7 +43,7 @@ int ttt_plan_info(const ttt_handle* handle, int* info, int n);
  * context stays usable.  Synchronises `stream` and returns what the word maps to:
  * TTT_ERR_TIMEOUT when the wait ran out (the expected result), TTT_OK otherwise,
  * TTT_ERR_CUDA / TTT_ERR_INVALID_ARG on a launch or argument error. */
-int ttt_selftest_timeout(void* status_word, cudaStream_t stream);
+int ttt_selftest_timeout(void* status_word, void* stream);
 
 /* Per-stage timing of a handle's forward calls.  ttt_profile_enable(h, 1)
  * clears earlier records and starts recording a CUDA event pair around every

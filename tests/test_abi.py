@@ -91,3 +91,29 @@ def test_status_strings():
     for s in range(-6, 1):
         assert binding.status_string(s) and binding.status_string(s) != "unknown status"
     assert binding.status_string(-99) == "unknown status"
+
+
+def test_binding_config_struct_matches_the_c_header(tmp_path, repo_root):
+    # the ctypes mirror of ttt_config must have the C layout: compare sizeof and every
+    # field offset with a C program compiled against include/ttt.h
+    import ctypes
+    import shutil
+    import subprocess
+
+    from weight_sequence_mixing_b200 import binding
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    names = [f[0] for f in binding.TTTConfig._fields_]
+    src = tmp_path / "layout.c"
+    # (ttt_diag.h includes ttt.h: both headers must be plain C)
+    src.write_text("#include <stdio.h>\n#include <stddef.h>\n#include \"ttt_diag.h\"\nint main(void) {\n"
+                   + "  printf(\"%zu\\n\", sizeof(ttt_config));\n"
+                   + "".join(f"  printf(\"%zu\\n\", offsetof(ttt_config, {n}));\n" for n in names)
+                   + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-std=c99", "-I", os.path.join(repo_root, "include"), str(src), "-o", str(exe)], check=True)
+    out = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    assert out[0] == ctypes.sizeof(binding.TTTConfig)
+    assert out[1:] == [getattr(binding.TTTConfig, n).offset for n in names]

@@ -108,8 +108,9 @@ __global__ void stuck_wait_kernel(unsigned* status) {
 }  // namespace
 }  // namespace ttt
 
-extern "C" int ttt_selftest_timeout(void* status_word, cudaStream_t stream) {
+extern "C" int ttt_selftest_timeout(void* status_word, void* stream_ptr) {
   if (!status_word) return TTT_ERR_INVALID_ARG;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
   unsigned* w = static_cast<unsigned*>(status_word);
   if (cudaMemsetAsync(w, 0, sizeof(unsigned), stream) != cudaSuccess) return TTT_ERR_CUDA;
   ttt::stuck_wait_kernel<<<1, 32, 0, stream>>>(w);
