@@ -20,15 +20,18 @@
  *                                                    F(x) = (SiLU(x W1^T) * x W3^T) W2^T
  *   - Q [B,H,Nq,d], K [B,H,N,d], V [B,H,N,d] and O [B,H,Nq,d] in `dtype`
  *     (fp32 or bf16); eta [B,H,N] fp32; W0 [H,P] fp32 (shared by every batch
- *     entry); W_out [B,H,P] fp32.
+ *     entry; [B,H,P] with TTT_FLAG_W0_PER_BATCH); W_out [B,H,P] fp32.
  *   - Losses, summed over the chunk's tokens with the per-token learning rate eta_i:
  *        TTT_LOSS_MSE      L = sum_i eta_i ||F(k_i) - v_i||^2 / (n_chunk * d)
  *        TTT_LOSS_NEG_DOT  L = -sum_i eta_i <F(k_i), v_i>
- *   - One step per chunk: G -> [momentum M <- beta M + G] -> [Muon: Newton-Schulz]
+ *   - One step per chunk (cfg.epochs steps when set; none with TTT_FLAG_NO_UPDATE):
+ *     G -> [momentum M <- beta M + G] -> [Muon: Newton-Schulz]
  *     -> W <- W - lr U -> [each row of each matrix scaled to unit L2 norm].
  *   - causal = 1 (needs Nq == N): per chunk, first O_c = F_W(Q_c), then update.
  *     causal = 0: update over every chunk in order, then O = F_{W*}(Q).
- *   - Nothing persists between calls: momentum starts at zero in every call.
+ *   - Nothing persists between calls: momentum starts at zero in every call.  A
+ *     caller streams the weight state by passing a call's W_out as the next call's
+ *     W0 with TTT_FLAG_W0_PER_BATCH.
  *
  * Ownership and threading
  *   The caller owns every buffer (inputs, outputs and the workspace); the handle
@@ -106,7 +109,7 @@ typedef struct ttt_config {
 typedef struct ttt_handle ttt_handle;
 
 /* Fill `cfg` with defaults (lr 1, momentum 0.9, 5 NS iterations with the Muon
- * quintic, in_eps 1e-5, eta_scalar 1); shapes are zero and must be set. */
+ * quintic, in_eps 1e-5, eta_scalar 1, epochs 1); shapes are zero and must be set. */
 void ttt_config_init(ttt_config* cfg);
 
 /* Validate `cfg` and build a handle.  Host only; no device work.  Returns
