@@ -401,6 +401,7 @@ def main():
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches,
+        "plan": dict(binding.plan_info(cfg), token_pair_capacity=binding.token_pair_capacity(cfg["inner"] == "swiglu")),
         "clocks": clocks,
         "step_ms_min_median_max": [min(step_ms), statistics.median(step_ms), max(step_ms)],
     }
