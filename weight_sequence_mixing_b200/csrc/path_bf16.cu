@@ -2,11 +2,14 @@
 // accumulation in TMEM) with the elementwise steps fused into their epilogues.
 //
 // Per chunk c (tokens [t0, t0+n), all heads batched, z = b*H + h):
-//   token phase  : one GEMM launch over 128-token x 128-hidden tiles computes the
-//                  inner forward on the keys and the loss backprop to the hidden
+//   token phase  : one launch over 256-token x 128-hidden tiles on CTA pairs (dot
+//                  loss; 128-token tiles on single CTAs as the fallback) computes
+//                  the inner forward on the keys and the loss backprop to the hidden
 //                  layer (epilogue: SiLU / GELU gating, eta_i folding), writing the
-//                  bf16 activations the weight gradient needs
+//                  bf16 activations the weight gradient needs; the MSE loss runs it
+//                  as three GEMMs with fused epilogues
 //   weight grads : one grouped launch of token-reduction GEMMs (MN-major operands,
+//                  512-row tiles on CTA pairs or 256/128-row tiles on single CTAs,
 //                  split-K over tokens, fp32 partials, deterministic reduction)
 //   optimizer    : split reduction + momentum, [Newton-Schulz on tf32 tensor cores],
 //                  W <- W - lr U, row L2-norm, bf16 copies of the new weights

@@ -1,6 +1,6 @@
 // C ABI of the TTT-layer forward pass: argument validation, workspace sizing,
 // the device status word and the host-buffer wrapper.  The forward pass itself
-// is planned and enqueued by the path selected in ttt_path.cuh.
+// is planned (ttt_plan.cu) and enqueued by the fp32 or bf16 path.
 #include <cstdio>
 #include <cstring>
 #include <new>
