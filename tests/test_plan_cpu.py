@@ -59,3 +59,39 @@ def test_split_heuristic_invariants(d, h, n, opt):
     if opt == "muon" and got["direct"]:
         assert got["grad_bn"] == d
     assert got["direct"] == (1 if got["splits"] == 1 and not (opt == "muon" and got["grad_bn"] != d) else 0)
+
+
+def _sizes(cfg):
+    import ctypes
+    c = binding.make_config(cfg)
+    h = ctypes.c_void_p()
+    assert binding.LIB.ttt_create(ctypes.byref(c), ctypes.byref(h)) == 0
+    try:
+        return int(binding.LIB.ttt_workspace_size(h)), int(binding.LIB.ttt_host_staging_size(h)), \
+            int(binding.LIB.ttt_param_count(h))
+    finally:
+        binding.LIB.ttt_destroy(h)
+
+
+def _up(x, a=256):
+    return (x + a - 1) // a * a
+
+
+@pytest.mark.parametrize("per_batch", [False, True])
+def test_host_staging_holds_every_input_and_output(per_batch):
+    cfg = make_config(B=2, H=3, N=300, Nq=200, d=64, h=128, inner="swiglu", loss="neg_dot", dtype="bf16",
+                      eta_mode="per_token", w0_per_batch=per_batch)
+    _, staging, P = _sizes(cfg)
+    BH = 2 * 3
+    expect = (_up(BH * 200 * 64 * 2) + 2 * _up(BH * 300 * 64 * 2) + _up(BH * 300 * 4)
+              + _up((BH if per_batch else 3) * P * 4) + _up(BH * 200 * 64 * 2) + _up(BH * P * 4))
+    assert staging == expect
+
+
+def test_workspace_grows_with_the_chunk_and_fits_the_static_scratch_when_small():
+    small_ws, _, _ = _sizes(workload("tiny_mlp2_n196_fp32"))
+    big_ws, _, _ = _sizes(workload("lact_nvs_n196k_d512"))
+    assert small_ws <= 32 * 1024 * 1024 < big_ws  # the no-allocation entry takes the first only
+    a, _, _ = _sizes(make_config(B=1, H=2, N=4096, d=128, h=256, inner="swiglu", loss="neg_dot", dtype="bf16"))
+    b, _, _ = _sizes(make_config(B=1, H=2, N=8192, d=128, h=256, inner="swiglu", loss="neg_dot", dtype="bf16"))
+    assert b > a
