@@ -38,6 +38,10 @@
  *   owns only host-side state.  Device pointers must be 16-byte aligned and
  *   contiguous.  ttt_forward only enqueues work on `stream` and returns; it
  *   allocates nothing.  One handle must not be used on two streams at once.
+ *   The library sets its kernels' shared-memory and cluster attributes once per
+ *   process, on the device current at the first call: drive one GPU per process
+ *   (the usual one-rank-per-GPU layout).  A call on a second device of the same
+ *   process is not supported and may return TTT_ERR_CUDA.
  *
  * Errors
  *   Calls return TTT_OK (0) or a negative status.  Argument errors are found on
