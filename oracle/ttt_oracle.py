@@ -16,7 +16,10 @@ What is computed (sources: the pages' text, cited per function):
   linear F(x) = x W^T [ViT3 digest, section 01: linear attention is a d x d layer];
   two-layer GELU MLP F(x) = GELU(x W1^T) W2^T [ViT3 digest, inner-model table;
   TTT vs Sleep, "Side one"]; SwiGLU F(x) = (SiLU(x W1^T) * x W3^T) W2^T with three
-  matrices [LaCT analysis, "Nonlinear memory complements local attention"].
+  matrices [LaCT analysis, "Nonlinear memory complements local attention"];
+  simplified GLU F(x) = (x Wa^T) * SiLU(x Wb^T) with two d x d matrices and no
+  output projection [ViT3 digest, section 03, inner-model table and the F1 module
+  of the ViT3 design].
 * Losses: MSE, and the negative dot product -<F(k_i), v_i> [ViT3 digest, inner-loss
   table; LaCT analysis, "Nonlinear memory"], summed with each token's learning
   rate eta_i [LaCT analysis, "Nonlinear memory"].
@@ -39,7 +42,11 @@ Readings taken where the pages are silent (each is listed in the design doc):
   momentum M <- beta M + G, M0 = 0, carried across chunks, reset per call;
   R10 Muon = Newton-Schulz quintic (a, b, c) on G / (||G||_F + 1e-7), transposed so
   rows <= cols, applied to the momentum buffer when momentum is on; R11 lr scales the
-  update; R12 order G -> momentum -> NS -> W <- W - lr U -> row norm.
+  update; R12 order G -> momentum -> NS -> W <- W - lr U -> row norm; R21 with
+  ``first_layer_only`` only the matrices that read the input (W1, and W3 for SwiGLU;
+  the single matrix of the linear model) take the step, W2 keeps its initial value
+  and is not row-normalised [TTT vs Sleep, "Side one": the first layer is adjusted];
+  R22 the simplified GLU has no biases, Wa is the linear branch, Wb the SiLU gate.
 
 Parity: every part here is pinned by tests in tests/test_oracle_pins.py (closed forms,
 finite differences, SVD, invariances).  The full-size GELU-MLP / SwiGLU / Muon results
@@ -96,6 +103,8 @@ def matrix_shapes(kind: str, d: int, h: int):
         return [("W1", h, d), ("W2", d, h)]
     if kind == "swiglu":
         return [("W1", h, d), ("W3", h, d), ("W2", d, h)]
+    if kind == "glu":
+        return [("Wa", d, d), ("Wb", d, d)]
     raise ValueError(kind)
 
 
@@ -131,6 +140,11 @@ def inner_forward(kind, W, X):
         A = silu(Z1)
         Hh = A * Z3
         return Hh @ W["W2"].T, dict(X=X, Z1=Z1, Z3=Z3, A=A, H=Hh)
+    if kind == "glu":
+        Za = X @ W["Wa"].T
+        Zb = X @ W["Wb"].T
+        S = silu(Zb)
+        return Za * S, dict(X=X, Za=Za, Zb=Zb, S=S)
     raise ValueError(kind)
 
 
@@ -150,6 +164,10 @@ def inner_backward(kind, W, cache, dY):
         dZ3 = dH * cache["A"]
         dZ1 = dH * cache["Z3"] * silu_prime(cache["Z1"])
         return dict(W1=dZ1.T @ X, W3=dZ3.T @ X, W2=G2)
+    if kind == "glu":
+        dZa = dY * cache["S"]
+        dZb = dY * cache["Za"] * silu_prime(cache["Zb"])
+        return dict(Wa=dZa.T @ X, Wb=dZb.T @ X)
     raise ValueError(kind)
 
 
@@ -223,7 +241,11 @@ def update_chunk(cfg, W, M, Kc, Vc, etac):
     dY = loss_grad(cfg["loss"], Vhat, Vc, etac)
     G = inner_backward(kind, W, cache, dY)
     opt = cfg["opt"]
+    # reading R21: the second layer keeps its initial value (no step, no row norm)
+    frozen = {"W2"} if cfg.get("first_layer_only", False) else set()
     for name in W:
+        if name in frozen:
+            continue
         g = G[name]
         if opt in ("momentum", "momentum_muon"):
             M[name] = cfg["momentum"] * M[name] + g

@@ -16,7 +16,7 @@ import oracle as orc
 from synth_inputs import make_config
 
 RNG = np.random.default_rng(12345)
-KINDS = ["linear", "mlp2_gelu", "swiglu"]
+KINDS = ["linear", "mlp2_gelu", "swiglu", "glu"]
 LOSSES = ["mse", "neg_dot"]
 
 
@@ -79,6 +79,10 @@ def _brute_forward(kind, W, x):
     if kind == "mlp2_gelu":
         hid = [gelu(z) for z in matvec(W["W1"].tolist(), x)]
         return matvec(W["W2"].tolist(), hid)
+    if kind == "glu":  # FC(x) * SiLU(FC(x))
+        za = matvec(W["Wa"].tolist(), x)
+        zb = matvec(W["Wb"].tolist(), x)
+        return [a * silu(b) for a, b in zip(za, zb)]
     z1 = matvec(W["W1"].tolist(), x)
     z3 = matvec(W["W3"].tolist(), x)
     hid = [silu(a) * b for a, b in zip(z1, z3)]
@@ -469,3 +473,119 @@ def test_streaming_two_calls_equal_one_chunked_call(kind, causal):
         assert np.allclose(np.concatenate([Oa, Ob], axis=2), O1, rtol=1e-12, atol=1e-12)
     else:
         assert np.allclose(Ob, O1, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- first layer only (SD3.5-T5 layer)
+def _run(cfg, Q, K, V, eta, w0):
+    return orc.forward_head(cfg, Q, K, V, eta, w0)
+
+
+@pytest.mark.parametrize("kind", ["mlp2_gelu", "swiglu"])
+@pytest.mark.parametrize("opt", ["gd", "momentum", "muon", "momentum_muon"])
+@pytest.mark.parametrize("rownorm", [False, True])
+def test_first_layer_only_keeps_w2_and_takes_the_same_first_layer_step(kind, opt, rownorm):
+    # one chunk: every matrix's gradient is taken at W0, so freezing W2 leaves the
+    # first layer's step unchanged; W2 must come back bit for bit
+    d, h, n = 4, 6, 9
+    cfg = cfg_for(kind, "neg_dot", opt=opt, weight_l2norm=rownorm, d=d, h=h, N=n, ns_iters=3)
+    W0 = rand_w(kind, d, h)
+    w0 = orc.pack(kind, d, h, W0)
+    Q, K, V, eta = rand(5, d), rand(n, d), rand(n, d), np.abs(rand(n)) + 0.1
+    _, wf = _run(cfg, Q, K, V, eta, w0)
+    O1, w1 = _run(dict(cfg, first_layer_only=True), Q, K, V, eta, w0)
+    Wf, W1 = orc.unpack(kind, d, h, wf), orc.unpack(kind, d, h, w1)
+    assert np.array_equal(W1["W2"], W0["W2"])
+    for name in W0:
+        if name != "W2":
+            assert np.allclose(W1[name], Wf[name], rtol=1e-13, atol=1e-13), name
+    assert np.allclose(O1, orc.inner_forward(kind, W1, Q)[0], rtol=1e-13, atol=1e-13)
+
+
+def test_first_layer_only_changes_nothing_for_the_linear_model():
+    d, n = 5, 7
+    cfg = cfg_for("linear", "mse", opt="momentum_muon", weight_l2norm=True, d=d, N=n, chunk=3, ns_iters=2)
+    w0 = rand(d * d)
+    Q, K, V, eta = rand(n, d), rand(n, d), rand(n, d), np.abs(rand(n)) + 0.1
+    O0, w_a = _run(cfg, Q, K, V, eta, w0)
+    O1, w_b = _run(dict(cfg, first_layer_only=True), Q, K, V, eta, w0)
+    assert np.array_equal(O0, O1) and np.array_equal(w_a, w_b)
+
+
+@pytest.mark.parametrize("kind", ["mlp2_gelu", "swiglu"])
+@pytest.mark.parametrize("loss", LOSSES)
+def test_first_layer_only_chunks_step_on_finite_difference_gradients(kind, loss):
+    # two chunks of plain gradient steps, checked against central finite differences
+    # of each chunk's loss in the first-layer matrices, with W2 held at W0
+    d, h, n, C = 3, 4, 8, 4
+    cfg = cfg_for(kind, loss, d=d, h=h, N=n, chunk=C)
+    W = rand_w(kind, d, h)
+    w0 = orc.pack(kind, d, h, W)
+    Q, K, V, eta = rand(3, d), rand(n, d), rand(n, d), np.abs(rand(n)) + 0.1
+    _, w_or = _run(dict(cfg, first_layer_only=True), Q, K, V, eta, w0)
+    eps = 1e-6
+    for s in range(0, n, C):
+        Kc, Vc, ec = K[s:s + C], V[s:s + C], eta[s:s + C]
+
+        def L(Wd):
+            return orc.loss_value(loss, orc.inner_forward(kind, Wd, Kc)[0], Vc, ec)
+
+        step = {}
+        for name, M in W.items():
+            if name == "W2":
+                continue
+            g = np.zeros_like(M)
+            for idx in np.ndindex(M.shape):
+                Wp = {k: v.copy() for k, v in W.items()}
+                Wm = {k: v.copy() for k, v in W.items()}
+                Wp[name][idx] += eps
+                Wm[name][idx] -= eps
+                g[idx] = (L(Wp) - L(Wm)) / (2 * eps)
+            step[name] = M - g
+        W.update(step)
+    assert np.allclose(w_or, orc.pack(kind, d, h, W), rtol=1e-7, atol=1e-8)
+
+
+# ---------------------------------------------------------------- simplified GLU (ViT3's F1)
+def _glu_as_swiglu(Wg, d):
+    """The GLU's matrices as a SwiGLU with h = d: W1 = Wb (gate), W3 = Wa, W2 = I."""
+    return {"W1": Wg["Wb"], "W3": Wg["Wa"], "W2": np.eye(d)}
+
+
+@pytest.mark.parametrize("opt", ["gd", "momentum", "muon", "momentum_muon"])
+@pytest.mark.parametrize("causal,chunk,rownorm", [(0, 0, False), (0, 4, True), (1, 3, True), (1, 0, False)])
+def test_glu_is_a_swiglu_with_identity_w2_and_first_layer_only(opt, causal, chunk, rownorm):
+    d, n = 4, 10
+    cfg = cfg_for("glu", "neg_dot", opt=opt, weight_l2norm=rownorm, d=d, h=d, N=n, chunk=chunk, causal=causal,
+                  ns_iters=3)
+    Wg = rand_w("glu", d, d)
+    Q, K, V, eta = rand(n, d), rand(n, d), rand(n, d), np.abs(rand(n)) + 0.1
+    Og, wg = _run(cfg, Q, K, V, eta, orc.pack("glu", d, d, Wg))
+    Ws0 = _glu_as_swiglu(Wg, d)
+    Os, ws = _run(dict(cfg, inner="swiglu", first_layer_only=True), Q, K, V, eta, orc.pack("swiglu", d, d, Ws0))
+    Wgs, Wss = orc.unpack("glu", d, d, wg), orc.unpack("swiglu", d, d, ws)
+    assert np.allclose(Og, Os, rtol=1e-12, atol=1e-12)
+    assert np.allclose(Wss["W1"], Wgs["Wb"], rtol=1e-12, atol=1e-12)
+    assert np.allclose(Wss["W3"], Wgs["Wa"], rtol=1e-12, atol=1e-12)
+    assert np.array_equal(Wss["W2"], np.eye(d))
+
+
+def test_glu_dot_step_in_closed_form():
+    # one GD step of the dot loss written out per token:
+    #   Wa += sum_i eta_i (v_i * SiLU(zb_i)) k_i^T
+    #   Wb += sum_i eta_i (v_i * za_i * SiLU'(zb_i)) k_i^T
+    # with SiLU'(z) from the quotient rule on z / (1 + e^-z), evaluated by math.exp
+    d, n = 3, 6
+    Wg = rand_w("glu", d, d)
+    K, V, eta = rand(n, d), rand(n, d), np.abs(rand(n)) + 0.1
+    Wa, Wb = Wg["Wa"].copy(), Wg["Wb"].copy()
+    for i in range(n):
+        za, zb = Wg["Wa"] @ K[i], Wg["Wb"] @ K[i]
+        s = np.array([z / (1 + math.exp(-z)) for z in zb])
+        ds = np.array([(1 + math.exp(-z) + z * math.exp(-z)) / (1 + math.exp(-z)) ** 2 for z in zb])
+        Wa += eta[i] * np.outer(V[i] * s, K[i])
+        Wb += eta[i] * np.outer(V[i] * za * ds, K[i])
+    cfg = cfg_for("glu", "neg_dot", d=d, h=d, N=n)
+    _, w = _run(cfg, rand(2, d), K, V, eta, orc.pack("glu", d, d, Wg))
+    W = orc.unpack("glu", d, d, w)
+    assert np.allclose(W["Wa"], Wa, rtol=1e-13, atol=1e-13)
+    assert np.allclose(W["Wb"], Wb, rtol=1e-13, atol=1e-13)
