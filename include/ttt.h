@@ -87,6 +87,13 @@ typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
                                   "Video and distributed": chunks that only read the state) */
 #define TTT_FLAG_SINGLE_CTA 8u /* token phase and weight-gradient GEMMs on single CTAs instead of CTA
                                   pairs; same results up to fp32 summation order, for comparison and tests */
+#define TTT_FLAG_FIRST_LAYER_ONLY 64u /* only the matrices that read the input take the step (W1, and
+                                         W3 for SWIGLU); W2 keeps its W0 value and is not row-normalised
+                                         ("Test-Time Training vs Sleep", Side one: the SD3.5-T5 layer
+                                         adjusts the first layer).  No effect on LINEAR.  The simplified GLU
+                                         FC(x) * SiLU(FC(x)) of the ViT3 digest (section 03, inner-model
+                                         table) is a SWIGLU with h = d, W1 = the SiLU gate's matrix, W3 =
+                                         the linear branch's, W2 = I and this flag */
 
 typedef struct ttt_config {
   int32_t B, H;       /* batch entries and heads */

@@ -65,12 +65,29 @@ def test_invalid_configurations_are_rejected(bad):
 
 def test_invalid_enum_and_flag_values_are_rejected():
     from weight_sequence_mixing_b200 import binding
-    for field, value in (("inner", 7), ("loss", -1), ("opt", 9), ("dtype", 5), ("flags", 64), ("ns_iters", -1),
+    for field, value in (("inner", 7), ("loss", -1), ("opt", 9), ("dtype", 5), ("flags", 128), ("ns_iters", -1),
                          ("epochs", -1), ("epochs", 65)):
         c = binding.make_config(make_config(N=16, d=64, h=128))
         setattr(c, field, value)
         st, h = _create(c)
         assert st == binding.TTT_ERR_INVALID_ARG, field
+
+
+@pytest.mark.parametrize("inner", ["linear", "mlp2_gelu", "swiglu"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_first_layer_only_is_accepted_and_leaves_the_plan_alone(inner, dtype):
+    from weight_sequence_mixing_b200 import binding
+    kw = dict(N=300, d=128, h=128, inner=inner, loss="neg_dot", dtype=dtype, opt="momentum_muon",
+              weight_l2norm=True)
+    sizes = []
+    for flo in (False, True):
+        c = binding.make_config(make_config(first_layer_only=flo, **kw))
+        assert bool(c.flags & binding.FLAG_FIRST_LAYER_ONLY) == flo
+        st, h = _create(c)
+        assert st == 0, binding.status_string(st)
+        sizes.append((binding.LIB.ttt_param_count(h), binding.LIB.ttt_workspace_size(h)))
+        binding.LIB.ttt_destroy(h)
+    assert sizes[0] == sizes[1]
 
 
 def test_forward_rejects_null_and_small_workspace_without_touching_the_gpu():

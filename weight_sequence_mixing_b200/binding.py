@@ -32,6 +32,7 @@ FLAG_DIRECT_LAUNCH = 4
 FLAG_SINGLE_CTA = 8
 FLAG_W0_PER_BATCH = 16
 FLAG_NO_UPDATE = 32
+FLAG_FIRST_LAYER_ONLY = 64
 
 EXPORTED = [
     "ttt_config_init", "ttt_create", "ttt_param_count", "ttt_workspace_size", "ttt_forward",
@@ -130,7 +131,8 @@ def make_config(cfg: dict) -> TTTConfig:
                | (FLAG_DIRECT_LAUNCH if cfg.get("direct_launch") else 0)
                | (FLAG_SINGLE_CTA if cfg.get("single_cta") else 0)
                | (FLAG_W0_PER_BATCH if cfg.get("w0_per_batch") else 0)
-               | (FLAG_NO_UPDATE if cfg.get("no_update") else 0))
+               | (FLAG_NO_UPDATE if cfg.get("no_update") else 0)
+               | (FLAG_FIRST_LAYER_ONLY if cfg.get("first_layer_only") else 0))
     c.eta_scalar = float(cfg["eta_scalar"])
     c.lr = float(cfg["lr"])
     c.momentum = float(cfg["momentum"])

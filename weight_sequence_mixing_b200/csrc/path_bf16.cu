@@ -144,9 +144,11 @@ __global__ void init_weights_kernel(int Z, int H, int64_t P, const float* W0, fl
 //   mode 0: no update (initial weights)
 //   mode 1: U from the gradient layout
 //   mode 2: U from the Newton-Schulz result (X [m][n], XT [n][m] per matrix)
-__global__ void finish_rows_kernel(RowMap rm, int mode, float lr, bool rownorm, float* Wf, const float* U,
-                                   const float* X, const float* XT, int m, int n, bool src_t, bf16* First, bf16* W2T,
-                                   bf16* W2, unsigned* status) {
+// hold_w2: the rows of W2 keep their values (first-layer-only updates): no step,
+// no row norm; their bf16 copies are rewritten unchanged.
+__global__ void finish_rows_kernel(RowMap rm, int mode, float lr, bool rownorm, bool hold_w2, float* Wf,
+                                   const float* U, const float* X, const float* XT, int m, int n, bool src_t,
+                                   bf16* First, bf16* W2T, bf16* W2, unsigned* status) {
   const int z = blockIdx.y;
   const int R = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   if (R >= rm.nrows()) return;
@@ -157,6 +159,10 @@ __global__ void finish_rows_kernel(RowMap rm, int mode, float lr, bool rownorm, 
   float* w = Wf + z * rm.P + off + int64_t(r) * len;
   const bool w2 = rm.is_w2(k);
   const int nmat = rm.inner == TTT_INNER_LINEAR ? 1 : rm.inner == TTT_INNER_MLP2_GELU ? 2 : 3;
+  if (w2 && hold_w2) {
+    mode = 0;
+    rownorm = false;
+  }
   if (mode == 1) {
     const float* Uz = U + int64_t(z) * rm.GR * rm.d;
     if (!w2) {
@@ -529,9 +535,9 @@ int optimizer_step(Ctx& c) {
   {
     StageScope _sc(kStageFinish, st);
     finish_rows_kernel<<<g, 256, 0, c.st>>>(c.rm, muon ? 2 : 1, cfg.lr, (cfg.flags & TTT_FLAG_WEIGHT_L2NORM) != 0,
-                                            c.v.at<float>(p, xWf), c.v.at<float>(p, xU), X, XT, D.m, D.n, D.src_t,
-                                            c.v.at<bf16>(p, xFirst), c.v.at<bf16>(p, xW2T), c.v.at<bf16>(p, xW2),
-                                            c.v.status);
+                                            (cfg.flags & TTT_FLAG_FIRST_LAYER_ONLY) != 0, c.v.at<float>(p, xWf),
+                                            c.v.at<float>(p, xU), X, XT, D.m, D.n, D.src_t, c.v.at<bf16>(p, xFirst),
+                                            c.v.at<bf16>(p, xW2T), c.v.at<bf16>(p, xW2), c.v.status);
   }
   TRY_CUDA(cudaGetLastError());
   return transpose_w2(c);
@@ -920,8 +926,9 @@ int run_bf16(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
     dim3 g((c.rm.nrows() + 7) / 8, Z);
     {
       StageScope _sc(kStageFinish, st);
-      finish_rows_kernel<<<g, 256, 0, st>>>(c.rm, 0, 0.f, false, c.v.at<float>(p, xWf), nullptr, nullptr, nullptr, 0, 0,
-                                            false, First, c.v.at<bf16>(p, xW2T), c.v.at<bf16>(p, xW2), c.v.status);
+      finish_rows_kernel<<<g, 256, 0, st>>>(c.rm, 0, 0.f, false, false, c.v.at<float>(p, xWf), nullptr, nullptr,
+                                            nullptr, 0, 0, false, First, c.v.at<bf16>(p, xW2T), c.v.at<bf16>(p, xW2),
+                                            c.v.status);
     }
     TRY_CUDA(cudaGetLastError());
     TRY(transpose_w2(c));

@@ -420,8 +420,11 @@ int update_chunk(const Plan& p, const F32View& v, const Io& io, cudaStream_t st,
   if (mom) momentum_kernel<<<grid_for(int64_t(Z) * P), 256, 0, st>>>(int64_t(Z) * P, c.momentum, v.b[bM], G);
   Mat mats[3];
   const int nm = matrices(p, mats);
+  const bool hold_w2 = (c.flags & TTT_FLAG_FIRST_LAYER_ONLY) != 0;
   for (int i = 0; i < nm; ++i) {
     const Mat& m = mats[i];
+    // first-layer-only updates: W2 (the last matrix of MLP2 / SwiGLU) keeps its value
+    if (hold_w2 && c.inner != TTT_INNER_LINEAR && i == nm - 1) continue;
     MatRef U{G + m.off, P, m.cols, 1};
     if (muon) {
       r = newton_schulz(p, v, st, U, m.rows, m.cols, &U);

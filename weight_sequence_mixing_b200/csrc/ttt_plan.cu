@@ -17,7 +17,8 @@ int plan_build(const ttt_config& c, Plan* p) {
   if (c.causal && c.Nq != c.N) return TTT_ERR_INVALID_ARG;
   if (c.inner != TTT_INNER_LINEAR && c.h < 1) return TTT_ERR_INVALID_ARG;
   if ((c.flags & ~(TTT_FLAG_KEY_INSTNORM | TTT_FLAG_WEIGHT_L2NORM | TTT_FLAG_DIRECT_LAUNCH |
-                   TTT_FLAG_SINGLE_CTA | TTT_FLAG_W0_PER_BATCH | TTT_FLAG_NO_UPDATE)) != 0)
+                   TTT_FLAG_SINGLE_CTA | TTT_FLAG_W0_PER_BATCH | TTT_FLAG_NO_UPDATE |
+                   TTT_FLAG_FIRST_LAYER_ONLY)) != 0)
     return TTT_ERR_INVALID_ARG;
   if (c.ns_iters < 0 || c.ns_iters > 100) return TTT_ERR_INVALID_ARG;
   if (c.epochs < 0 || c.epochs > 64) return TTT_ERR_INVALID_ARG;
