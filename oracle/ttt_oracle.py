@@ -259,11 +259,14 @@ def update_chunk(cfg, W, M, Kc, Vc, etac):
             W[name] = row_l2_normalize(W[name])
 
 
-def forward_head(cfg, Q, K, V, eta, w0):
-    """One (batch, head): returns (O [Nq, d], W* packed [P]) in fp64.
+def forward_head(cfg, Q, K, V, eta, w0, m0=None, return_m=False):
+    """One (batch, head): returns (O [Nq, d], W* packed [P]) in fp64, and with
+    ``return_m`` also the momentum buffer after the last step (packed [P]).
 
     Non-causal: update over every chunk in order, then O = F_{W*}(Q).
     Causal (Nq == N): for each chunk, first O_c = F_W(Q_c), then update with chunk c.
+    ``m0`` (packed [P]) is the momentum a previous call on the same sequence ended
+    with (streamed state, LaCT "Video and distributed"); None means zero (R9).
     """
     kind, d, h = cfg["inner"], cfg["d"], cfg["h"]
     Q = np.asarray(Q, dtype=F64)
@@ -275,7 +278,7 @@ def forward_head(cfg, Q, K, V, eta, w0):
     else:
         eta = np.asarray(eta, dtype=F64)
     W = unpack(kind, d, h, w0)
-    M = {name: np.zeros_like(m) for name, m in W.items()}
+    M = unpack(kind, d, h, m0) if m0 is not None else {name: np.zeros_like(m) for name, m in W.items()}
     bounds = chunk_bounds(N, cfg["chunk"])
     # inner epochs: that many full-batch steps on each chunk before the next one
     # (ViT3 digest, inner-training ablation); momentum carries through them.  A
@@ -294,6 +297,8 @@ def forward_head(cfg, Q, K, V, eta, w0):
             for _ in range(epochs):
                 update_chunk(cfg, W, M, K[s:e], V[s:e], eta[s:e])
         O = inner_forward(kind, W, Q)[0]
+    if return_m:
+        return O, pack(kind, d, h, W), pack(kind, d, h, M)
     return O, pack(kind, d, h, W)
 
 
@@ -305,21 +310,29 @@ def _np(t):
     return np.asarray(t, dtype=F64)
 
 
-def forward(cfg, Q, K, V, eta, W0, heads=None):
+def forward(cfg, Q, K, V, eta, W0, heads=None, M0=None, return_m=False):
     """All (batch, head) pairs, or the listed ``heads`` [(b, h), ...].
 
-    Returns O [B, H, Nq, d] and W* [B, H, P] in fp64 (entries of unlisted heads are NaN).
+    Returns O [B, H, Nq, d] and W* [B, H, P] in fp64 (entries of unlisted heads are NaN);
+    with ``return_m`` also the final momentum buffers [B, H, P].  ``M0`` [B, H, P]
+    is the momentum carried in from a previous call (None: zero).
     """
     B, H = cfg["B"], cfg["H"]
     Nq, d = cfg["Nq"], cfg["d"]
     P = sum(r * c for _, r, c in matrix_shapes(cfg["inner"], d, cfg["h"]))
     O = np.full((B, H, Nq, d), np.nan)
     Ws = np.full((B, H, P), np.nan)
+    Ms = np.full((B, H, P), np.nan)
+    M0n = _np(M0)
     todo = heads if heads is not None else [(b, hh) for b in range(B) for hh in range(H)]
     W0n = _np(W0)
     per_batch = bool(cfg.get("w0_per_batch", False))  # W0 [B, H, P]: one state per entry
     for b, hh in todo:
         e = None if eta is None else _np(eta[b, hh])
         w0 = W0n[b, hh] if per_batch else W0n[hh]
-        O[b, hh], Ws[b, hh] = forward_head(cfg, _np(Q[b, hh]), _np(K[b, hh]), _np(V[b, hh]), e, w0)
+        m0 = None if M0n is None else M0n[b, hh]
+        O[b, hh], Ws[b, hh], Ms[b, hh] = forward_head(cfg, _np(Q[b, hh]), _np(K[b, hh]), _np(V[b, hh]), e, w0,
+                                                      m0=m0, return_m=True)
+    if return_m:
+        return O, Ws, Ms
     return O, Ws

@@ -475,6 +475,55 @@ def test_streaming_two_calls_equal_one_chunked_call(kind, causal):
         assert np.allclose(Ob, O1, rtol=1e-12, atol=1e-12)
 
 
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("causal", [0, 1])
+@pytest.mark.parametrize("opt", ["momentum", "momentum_muon"])
+def test_streaming_with_momentum_state_equals_one_chunked_call(kind, causal, opt):
+    # with momentum the state is (W, M): handing both to the call on the second half
+    # gives the one-call result, as momentum is carried across chunks (reading R9)
+    d, h, N, B, H = 4, 6, 12, 2, 1
+    Q, K, V, eta = _data(B, H, N, d)
+    W0 = orc.pack(kind, d, h, rand_w(kind, d, h))[None]
+    half = N // 2
+    base = dict(B=B, H=H, d=d, h=h, weight_l2norm=True, causal=causal, opt=opt, ns_iters=3)
+    O1, W1, M1 = orc.forward(cfg_for(kind, "neg_dot", N=N, chunk=half, **base), Q, K, V, eta, W0, return_m=True)
+    sl = lambda t, a, b: t[:, :, a:b]
+    qa = sl(Q, 0, half) if causal else Q
+    qb = sl(Q, half, N) if causal else Q
+    Oa, Wa, Ma = orc.forward(cfg_for(kind, "neg_dot", N=half, Nq=qa.shape[2], **base), qa, sl(K, 0, half),
+                             sl(V, 0, half), sl(eta, 0, half), W0, return_m=True)
+    Ob, Wb, Mb = orc.forward(cfg_for(kind, "neg_dot", N=half, Nq=qb.shape[2], w0_per_batch=True, **base), qb,
+                             sl(K, half, N), sl(V, half, N), sl(eta, half, N), Wa, M0=Ma, return_m=True)
+    assert np.allclose(Wb, W1, rtol=1e-12, atol=1e-12) and np.allclose(Mb, M1, rtol=1e-12, atol=1e-12)
+    O2 = np.concatenate([Oa, Ob], axis=2) if causal else Ob
+    assert np.allclose(O2, O1, rtol=1e-12, atol=1e-12)
+    # without the momentum handed over the second call restarts it at zero: a different result
+    _, Wc = orc.forward(cfg_for(kind, "neg_dot", N=half, Nq=qb.shape[2], w0_per_batch=True, **base), qb,
+                        sl(K, half, N), sl(V, half, N), sl(eta, half, N), Wa)
+    assert not np.allclose(Wc, W1, rtol=1e-6, atol=1e-9)
+
+
+def test_momentum_state_of_the_linear_dot_layer_in_closed_form():
+    # linear + dot: every chunk's gradient is -sum_i eta_i v_i k_i^T whatever W is, so
+    # M after chunks 1 and 2 is beta (-V1^T E1 K1) + (-V2^T E2 K2), token by token
+    d, N, C, beta = 3, 10, 4, 0.7
+    Q, K, V, eta = rand(2, d), rand(N, d), rand(N, d), np.abs(rand(N)) + 0.1
+    M0 = rand(d * d)
+    cfg = cfg_for("linear", "neg_dot", opt="momentum", momentum=beta, d=d, N=N, chunk=C)
+    _, _, m = orc.forward_head(cfg, Q, K, V, eta, rand(d * d), m0=M0, return_m=True)
+    M = M0.reshape(d, d).copy()
+    for s in range(0, N, C):
+        G = np.zeros((d, d))
+        for i in range(s, min(s + C, N)):
+            for r in range(d):
+                for c in range(d):
+                    G[r, c] -= eta[i] * V[i, r] * K[i, c]
+        M = beta * M + G
+    assert np.allclose(m, M.reshape(-1), rtol=1e-13, atol=1e-13)
+    _, _, mg = orc.forward_head(dict(cfg, opt="gd"), Q, K, V, eta, rand(d * d), return_m=True)
+    assert np.array_equal(mg, np.zeros(d * d))
+
+
 # ---------------------------------------------------------------- first layer only (SD3.5-T5 layer)
 def _run(cfg, Q, K, V, eta, w0):
     return orc.forward_head(cfg, Q, K, V, eta, w0)
