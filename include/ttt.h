@@ -31,7 +31,7 @@
  *     causal = 0: update over every chunk in order, then O = F_{W*}(Q).
  *   - Nothing persists between calls: momentum starts at zero in every call.  A
  *     caller streams the weight state by passing a call's W_out as the next call's
- *     W0 with TTT_FLAG_W0_PER_BATCH.
+ *     W0 with TTT_FLAG_W0_PER_BATCH, and the momentum through ttt_forward_state.
  *
  * Ownership and threading
  *   The caller owns every buffer (inputs, outputs and the workspace); the handle
@@ -145,6 +145,25 @@ size_t ttt_workspace_size(const ttt_handle* handle);
 int ttt_forward(ttt_handle* handle, const void* Q, const void* K, const void* V, const float* eta,
                 const float* W0, void* O, float* W_out, void* workspace, size_t workspace_bytes,
                 void* stream);
+
+/* Streaming with momentum (LaCT analysis, "Video and distributed": the fast-weight
+ * state is carried from one call to the next).  With a momentum optimizer the state
+ * of a sequence is (W, M); W travels as W_out -> W0 (TTT_FLAG_W0_PER_BATCH) and M as
+ * an opaque device blob of ttt_state_size() bytes: the heavy-ball buffer of every
+ * (batch entry, head) after the call's last step, in the library's own layout.
+ *   - state_in: the state_out of an earlier call, or NULL (momentum starts at zero,
+ *     as in ttt_forward).  state_out: written at the end of the pass, or NULL.
+ *     They may be the same buffer.  Both 16-byte aligned device memory.
+ *   - A blob is valid between handles with the same B, H, d, h, inner, opt and
+ *     dtype; N, Nq, chunk, causal and the flags may differ.  A read-only call
+ *     (TTT_FLAG_NO_UPDATE) hands the state on unchanged.
+ *   - Without momentum ttt_state_size() is 0 and the state pointers are ignored.
+ * Two calls over consecutive token ranges with (W, M) handed on give the result
+ * of one call with those ranges as chunks.  Otherwise as ttt_forward. */
+size_t ttt_state_size(const ttt_handle* handle);
+int ttt_forward_state(ttt_handle* handle, const void* Q, const void* K, const void* V, const float* eta,
+                      const float* W0, void* O, float* W_out, const void* state_in, void* state_out,
+                      void* workspace, size_t workspace_bytes, void* stream);
 
 /* The same pass on HOST buffers (pinned memory gives asynchronous copies):
  * copies the inputs into the front of `device_staging`, runs ttt_forward and

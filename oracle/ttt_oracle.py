@@ -39,7 +39,8 @@ Readings taken where the pages are silent (each is listed in the design doc):
   branch, W2 = down projection; R6 no biases; R7 instance norm per channel over the
   chunk's tokens, biased variance, eps, no affine, keys only, the target V stays raw;
   R8 each [out,in] row scaled to unit L2 norm after every update; R9 heavy-ball
-  momentum M <- beta M + G, M0 = 0, carried across chunks, reset per call;
+  momentum M <- beta M + G, M0 = 0 (or the momentum a previous call on the same
+  sequence ended with), carried across chunks;
   R10 Muon = Newton-Schulz quintic (a, b, c) on G / (||G||_F + 1e-7), transposed so
   rows <= cols, applied to the momentum buffer when momentum is on; R11 lr scales the
   update; R12 order G -> momentum -> NS -> W <- W - lr U -> row norm; R21 with

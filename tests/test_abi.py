@@ -90,6 +90,42 @@ def test_first_layer_only_is_accepted_and_leaves_the_plan_alone(inner, dtype):
     assert sizes[0] == sizes[1]
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("opt", ["gd", "momentum", "muon", "momentum_muon"])
+def test_momentum_state_size(dtype, opt):
+    from weight_sequence_mixing_b200 import binding
+    B, H, d, h = 2, 3, 128, 256
+    cfg = make_config(B=B, H=H, N=300, d=d, h=h, inner="swiglu", loss="neg_dot", dtype=dtype, opt=opt)
+    st, hd = _create(binding.make_config(cfg))
+    assert st == 0
+    n = binding.LIB.ttt_state_size(hd)
+    binding.LIB.ttt_destroy(hd)
+    if opt in ("gd", "muon"):
+        assert n == 0
+    else:  # the momentum of every matrix of every (batch entry, head), fp32
+        assert n == B * H * 3 * d * h * 4
+    # the blob does not depend on the token counts, chunking or flags
+    st, hd = _create(binding.make_config(dict(cfg, N=1000, Nq=40, chunk=256, weight_l2norm=True,
+                                              w0_per_batch=True)))
+    assert st == 0 and binding.LIB.ttt_state_size(hd) == n
+    binding.LIB.ttt_destroy(hd)
+
+
+def test_forward_state_checks_state_alignment_without_touching_the_gpu():
+    from weight_sequence_mixing_b200 import binding
+    st, h = _create(binding.make_config(make_config(N=16, d=64, h=128, opt="momentum")))
+    assert st == 0
+    lib = binding.LIB
+    fake = ctypes.c_void_p(4096)
+    bad = ctypes.c_void_p(4096 + 4)
+    for a, b in ((bad, None), (None, bad)):
+        assert lib.ttt_forward_state(h, fake, fake, fake, None, fake, fake, None, a, b, fake, 1 << 30,
+                                     None) == binding.TTT_ERR_INVALID_ARG
+    assert lib.ttt_forward_state(h, None, fake, fake, None, fake, fake, None, None, None, fake, 1 << 30,
+                                 None) == binding.TTT_ERR_INVALID_ARG
+    lib.ttt_destroy(h)
+
+
 def test_forward_rejects_null_and_small_workspace_without_touching_the_gpu():
     from weight_sequence_mixing_b200 import binding
     st, h = _create(binding.make_config(make_config(N=16, d=64, h=128)))

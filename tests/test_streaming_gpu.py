@@ -62,3 +62,46 @@ def test_two_streamed_calls_equal_one_chunked_call(dtype, causal):
     assert rel_fro(Wb, W1) < 1e-5
     O2 = torch.cat([torch.from_numpy(Oa), torch.from_numpy(Ob)], dim=2).numpy() if causal else Ob
     assert rel_fro(O2, O1) < 1e-5
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("causal", [0, 1])
+@pytest.mark.parametrize("opt", ["momentum", "momentum_muon"])
+def test_two_streamed_calls_with_momentum_state_equal_one_chunked_call(dtype, causal, opt):
+    # (W, M) handed on: W_out -> W0 and the opaque momentum blob state_out -> state_in
+    from weight_sequence_mixing_b200 import binding
+    import oracle as orc
+
+    base = dict(opt=opt, weight_l2norm=True, data="lact", eta_mode="per_token", seed=47, causal=causal,
+                **BASE[dtype])
+    N = base["N"]
+    half = N // 2
+    full = make_config(chunk=half, **base)
+    x = gen_inputs(full)
+    O1, W1 = run_gpu(full, x)
+
+    def part(a, b, w0, per_batch, state_in, state_out):
+        kw = dict(base, N=half, Nq=half if causal else N)
+        layer = binding.TTTLayer(make_config(chunk=0, w0_per_batch=per_batch, **kw))
+        q = x["Q"][:, :, a:b] if causal else x["Q"]
+        dev = lambda t: t.contiguous().cuda()
+        O, W = layer.forward_state(dev(q), dev(x["K"][:, :, a:b]), dev(x["V"][:, :, a:b]),
+                                   dev(x["eta"][:, :, a:b]), dev(w0), state_in=state_in, state_out=state_out)
+        torch.cuda.synchronize()
+        out = O.double().cpu(), W
+        layer.close()
+        return out
+
+    probe = binding.TTTLayer(make_config(chunk=0, **dict(base, N=half, Nq=half if causal else N)))
+    assert probe.state_size > 0
+    state = probe.new_state()
+    probe.close()
+    Oa, Wa = part(0, half, x["W0"], False, None, state)
+    Ob, Wb = part(half, N, Wa, True, state, state)
+    Wb = Wb.double().cpu().numpy()
+    assert rel_fro(Wb, W1) < 1e-5
+    O2 = torch.cat([Oa, Ob], dim=2).numpy() if causal else Ob.numpy()
+    assert rel_fro(O2, O1) < 1e-5
+    # and against the oracle's one chunked call
+    Or, Wr = orc.forward(full, x["Q"], x["K"], x["V"], x["eta"], x["W0"])
+    assert rel_fro(O2, Or) <= TOL[dtype] and rel_fro(Wb, Wr) <= TOL[dtype]

@@ -39,6 +39,7 @@ EXPORTED = [
     "ttt_host_staging_size", "ttt_forward_host", "ttt_query_status", "ttt_destroy", "ttt_status_string",
     "ttt_selftest_gemm", "ttt_profile_enable", "ttt_profile_collect", "ttt_stage_name", "ttt_launch_count",
     "ttt_forward_noalloc", "ttt_token_pair_capacity", "ttt_selftest_timeout", "ttt_plan_info",
+    "ttt_state_size", "ttt_forward_state",
 ]
 NUM_STAGES = 8
 
@@ -86,6 +87,8 @@ def _load():
         "ttt_token_pair_capacity": (i32, [i32]),
         "ttt_selftest_timeout": (i32, [vp, vp]),
         "ttt_plan_info": (i32, [vp, ctypes.POINTER(ctypes.c_int), i32]),
+        "ttt_state_size": (sz, [vp]),
+        "ttt_forward_state": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -190,6 +193,35 @@ class TTTLayer:
         st = _stream_ptr(stream)
         _check(LIB.ttt_forward(self._handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W0), _ptr(O), _ptr(W_out),
                                _ptr(self.workspace), self.workspace.numel(), st), "ttt_forward")
+        if check:
+            self.check_status(stream)
+        return O, W_out
+
+    @property
+    def state_size(self) -> int:
+        """Bytes of the momentum state a call hands on (0 without momentum)."""
+        return int(LIB.ttt_state_size(self._handle))
+
+    def new_state(self):
+        """A device buffer for the momentum state (at least 16 bytes)."""
+        return torch.zeros(max(self.state_size, 16), dtype=torch.uint8, device=self.device)
+
+    def forward_state(self, Q, K, V, eta, W0, state_in=None, state_out=None, O=None, W_out=None, stream=None,
+                      check=True):
+        """As forward, carrying the momentum state in (state_in, or None: zero) and out
+        (state_out, or None); both uint8 device buffers of at least state_size bytes."""
+        c = self.cfg
+        if O is None:
+            O = torch.empty((c["B"], c["H"], c["Nq"], c["d"]), dtype=self.io_dtype, device=self.device)
+        if W_out is None:
+            W_out = torch.empty((c["B"], c["H"], self.P), dtype=torch.float32, device=self.device)
+        for t in (state_in, state_out):
+            if t is not None and t.numel() * t.element_size() < self.state_size:
+                raise ValueError("state buffer smaller than state_size")
+        st = _stream_ptr(stream)
+        _check(LIB.ttt_forward_state(self._handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W0), _ptr(O),
+                                     _ptr(W_out), _ptr(state_in), _ptr(state_out), _ptr(self.workspace),
+                                     self.workspace.numel(), st), "ttt_forward_state")
         if check:
             self.check_status(stream)
         return O, W_out

@@ -886,6 +886,8 @@ int plan_layout_bf16(Plan* p) {
     o += (size_t(bytes[i]) + 1023) / 1024 * 1024;
   }
   p->ws_bytes = o;
+  // the momentum buffer, in its gradient layout, is the state a call hands on
+  p->state_bytes = (c.opt == TTT_OPT_MOMENTUM || c.opt == TTT_OPT_MOMENTUM_MUON) ? size_t(bytes[xMom]) : 0;
   return TTT_OK;
 }
 
@@ -921,7 +923,10 @@ int run_bf16(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
     init_weights_kernel<<<std::min<int64_t>((int64_t(Z) * p.P + 255) / 256, 4096), 256, 0, st>>>(
         Z, w0_rows, p.P, io.W0, c.v.at<float>(p, xWf));
   }
-  TRY_CUDA(cudaMemsetAsync(c.v.at<float>(p, xMom), 0, size_t(Z) * D.GR * d * 4, st));
+  if (io.M_in && p.state_bytes)
+    TRY_CUDA(cudaMemcpyAsync(c.v.at<float>(p, xMom), io.M_in, p.state_bytes, cudaMemcpyDeviceToDevice, st));
+  else
+    TRY_CUDA(cudaMemsetAsync(c.v.at<float>(p, xMom), 0, size_t(Z) * D.GR * d * 4, st));
   {
     dim3 g((c.rm.nrows() + 7) / 8, Z);
     {
@@ -942,6 +947,8 @@ int run_bf16(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
   if (!cfg.causal) TRY(apply_rows(c, 0, cfg.Nq));
   if (io.W_out)
     TRY_CUDA(cudaMemcpyAsync(io.W_out, c.v.at<float>(p, xWf), size_t(Z) * p.P * 4, cudaMemcpyDeviceToDevice, st));
+  if (io.M_out && p.state_bytes)
+    TRY_CUDA(cudaMemcpyAsync(io.M_out, c.v.at<float>(p, xMom), p.state_bytes, cudaMemcpyDeviceToDevice, st));
   return TTT_OK;
 }
 

@@ -462,6 +462,8 @@ int plan_layout_f32(Plan* p) {
   }
   p->off[kNumBuf] = size_t(R);  // rows reserved per head
   p->ws_bytes = o;
+  // the momentum buffer [Z][P] is the state a call hands on
+  p->state_bytes = (c.opt == TTT_OPT_MOMENTUM || c.opt == TTT_OPT_MOMENTUM_MUON) ? size_t(Z * P) * 4 : 0;
   return TTT_OK;
 }
 
@@ -475,7 +477,12 @@ int run_f32(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
     const int w0_rows = (c.flags & TTT_FLAG_W0_PER_BATCH) ? Z : c.H;  // W0 [H][P] or [B*H][P]
     init_weights_kernel<<<grid_for(int64_t(Z) * P), 256, 0, st>>>(Z, w0_rows, P, io.W0, v.b[bW]);
   }
-  if (cudaMemsetAsync(v.b[bM], 0, size_t(Z) * P * 4, st) != cudaSuccess) return TTT_ERR_CUDA;
+  if (io.M_in && p.state_bytes) {
+    if (cudaMemcpyAsync(v.b[bM], io.M_in, p.state_bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return TTT_ERR_CUDA;
+  } else if (cudaMemsetAsync(v.b[bM], 0, size_t(Z) * P * 4, st) != cudaSuccess) {
+    return TTT_ERR_CUDA;
+  }
   const float* Q = static_cast<const float*>(io.Q);
   float* O = static_cast<float*>(io.O);
   const int64_t q_sz = int64_t(c.Nq) * d;
@@ -502,6 +509,9 @@ int run_f32(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
   (void)Rd;
   if (io.W_out &&
       cudaMemcpyAsync(io.W_out, v.b[bW], size_t(Z) * P * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return TTT_ERR_CUDA;
+  if (io.M_out && p.state_bytes &&
+      cudaMemcpyAsync(io.M_out, v.b[bM], p.state_bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return TTT_ERR_CUDA;
   {
     StageScope _sc(kStageOther, st);

@@ -43,7 +43,7 @@ struct GraphInstance {
 };
 
 struct GraphEntry {
-  const void* key[9] = {};
+  const void* key[11] = {};
   bool profiled = false;
   long long launches = 0;  // kernel launches one replay performs
   GraphInstance inst[2];

@@ -94,11 +94,11 @@ int capture_instance(ttt_handle* h, const Io& io, void* ws, cudaStream_t st, ttt
 // Replay the cached graph of this pointer set (capturing it on first use).
 int forward_graph(ttt_handle* h, const Io& io, void* ws, cudaStream_t st) {
   Profiler& pr = h->prof;
-  const void* key[9] = {io.Q, io.K, io.V, io.eta, io.W0, io.O, io.W_out, ws, st};
+  const void* key[11] = {io.Q, io.K, io.V, io.eta, io.W0, io.O, io.W_out, io.M_in, io.M_out, ws, st};
   GraphEntry* hit = nullptr;
   for (GraphEntry& e : pr.graphs) {
     bool same = e.profiled == pr.on;
-    for (int i = 0; i < 9 && same; ++i) same = e.key[i] == key[i];
+    for (int i = 0; i < 11 && same; ++i) same = e.key[i] == key[i];
     if (same) {
       hit = &e;
       break;
@@ -115,7 +115,7 @@ int forward_graph(ttt_handle* h, const Io& io, void* ws, cudaStream_t st) {
       pr.graphs.erase(pr.graphs.begin() + static_cast<long>(old));
     }
     GraphEntry e;
-    for (int i = 0; i < 9; ++i) e.key[i] = key[i];
+    for (int i = 0; i < 11; ++i) e.key[i] = key[i];
     e.profiled = pr.on;
     e.ninst = pr.on ? 2 : 1;
     for (int i = 0; i < e.ninst; ++i) {
@@ -138,18 +138,14 @@ int forward_graph(ttt_handle* h, const Io& io, void* ws, cudaStream_t st) {
   return TTT_OK;
 }
 
-}  // namespace
-
-extern "C" int ttt_forward(ttt_handle* h, const void* Q, const void* K, const void* V, const float* eta,
-                           const float* W0, void* O, float* W_out, void* workspace, size_t workspace_bytes,
-                           void* stream) {
-  if (!h || !Q || !K || !V || !W0 || !O) return TTT_ERR_INVALID_ARG;
-  const void* ptrs[] = {Q, K, V, eta, W0, O, W_out};
+// Validate and enqueue one forward pass (ttt_forward, ttt_forward_state).
+int forward_impl(ttt_handle* h, const Io& io, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!h || !io.Q || !io.K || !io.V || !io.W0 || !io.O) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {io.Q, io.K, io.V, io.eta, io.W0, io.O, io.W_out, io.M_in, io.M_out};
   for (const void* p : ptrs)
     if (p && (reinterpret_cast<uintptr_t>(p) & 15) != 0) return TTT_ERR_INVALID_ARG;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) != 0 || workspace_bytes < h->plan.ws_bytes)
     return TTT_ERR_WORKSPACE;
-  Io io{Q, K, V, eta, W0, O, W_out};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // Replay a cached graph unless the caller asked for direct launches, the stream
   // is the legacy default stream (not capturable), or the caller is capturing
@@ -164,6 +160,26 @@ extern "C" int ttt_forward(ttt_handle* h, const void* Q, const void* K, const vo
   const int r = graph ? forward_graph(h, io, workspace, st) : plan_run(h->plan, io, workspace, st);
   g_prof = nullptr;
   return r;
+}
+
+}  // namespace
+
+extern "C" int ttt_forward(ttt_handle* h, const void* Q, const void* K, const void* V, const float* eta,
+                           const float* W0, void* O, float* W_out, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  const Io io{Q, K, V, eta, W0, O, W_out};
+  return forward_impl(h, io, workspace, workspace_bytes, stream);
+}
+
+extern "C" size_t ttt_state_size(const ttt_handle* h) { return h ? h->plan.state_bytes : 0; }
+
+extern "C" int ttt_forward_state(ttt_handle* h, const void* Q, const void* K, const void* V, const float* eta,
+                                 const float* W0, void* O, float* W_out, const void* state_in, void* state_out,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  // without momentum there is no state: the state pointers are ignored
+  const bool has = h && h->plan.state_bytes > 0;
+  const Io io{Q, K, V, eta, W0, O, W_out, has ? state_in : nullptr, has ? state_out : nullptr};
+  return forward_impl(h, io, workspace, workspace_bytes, stream);
 }
 
 extern "C" size_t ttt_host_staging_size(const ttt_handle* h) { return h ? h->plan.staging_bytes : 0; }

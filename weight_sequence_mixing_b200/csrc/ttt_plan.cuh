@@ -18,6 +18,8 @@ struct Io {
   const float* W0;
   void* O;
   float* W_out;
+  const void* M_in = nullptr;  // momentum state carried in (ttt_forward_state), or null: zero
+  void* M_out = nullptr;       // momentum state carried out, or null
 };
 
 enum PathKind : int { kPathF32 = 0, kPathBf16 = 1 };
@@ -31,6 +33,7 @@ struct Plan {
   int epochs = 1;      // full-batch steps per chunk
   int path = kPathF32;
   size_t ws_bytes = 0;
+  size_t state_bytes = 0;  // momentum state (0 without momentum)
   // host-staging layout (ttt_forward_host)
   size_t staging_bytes = 0, stg_q = 0, stg_k = 0, stg_v = 0, stg_eta = 0, stg_w0 = 0, stg_o = 0, stg_w = 0;
   // workspace layout: byte offsets into the caller's workspace
