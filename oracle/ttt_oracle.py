@@ -20,9 +20,9 @@ What is computed (sources: the pages' text, cited per function):
   simplified GLU F(x) = (x Wa^T) * SiLU(x Wb^T) with two d x d matrices and no
   output projection [ViT3 digest, section 03, inner-model table and the F1 module
   of the ViT3 design].
-* Losses: MSE, and the negative dot product -<F(k_i), v_i> [ViT3 digest, inner-loss
-  table; LaCT analysis, "Nonlinear memory"], summed with each token's learning
-  rate eta_i [LaCT analysis, "Nonlinear memory"].
+* Losses: MSE, RMSE = sqrt(MSE), and the negative dot product -<F(k_i), v_i> [ViT3
+  digest, inner-loss table; LaCT analysis, "Nonlinear memory"], summed with each
+  token's learning rate eta_i [LaCT analysis, "Nonlinear memory"].
 * One full-batch step per chunk [ViT3 digest, guideline 2]; large chunks and
   apply-then-update order for causal data, update-then-apply otherwise
   [LaCT analysis, "Fast weights" and "Order of operations"].
@@ -47,7 +47,9 @@ Readings taken where the pages are silent (each is listed in the design doc):
   ``first_layer_only`` only the matrices that read the input (W1, and W3 for SwiGLU;
   the single matrix of the linear model) take the step, W2 keeps its initial value
   and is not row-normalised [TTT vs Sleep, "Side one": the first layer is adjusted];
-  R22 the simplified GLU has no biases, Wa is the linear branch, Wb the SiLU gate.
+  R22 the simplified GLU has no biases, Wa is the linear branch, Wb the SiLU gate;
+  R23 RMSE is the square root of the R2 MSE of the chunk (eta inside the root); its
+  gradient is the MSE gradient over 2 sqrt(MSE), and zero where the MSE is zero.
 
 Parity: every part here is pinned by tests in tests/test_oracle_pins.py (closed forms,
 finite differences, SVD, invariances).  The full-size GELU-MLP / SwiGLU / Muon results
@@ -180,6 +182,8 @@ def loss_value(loss, Vhat, V, eta):
     n, d = V.shape
     if loss == "mse":
         return float(np.sum(eta[:, None] * (Vhat - V) ** 2) / (n * d))
+    if loss == "rmse":
+        return float(np.sqrt(np.sum(eta[:, None] * (Vhat - V) ** 2) / (n * d)))
     if loss == "neg_dot":
         return float(-np.sum(eta[:, None] * Vhat * V))
     raise ValueError(loss)
@@ -190,6 +194,11 @@ def loss_grad(loss, Vhat, V, eta):
     n, d = V.shape
     if loss == "mse":
         return 2.0 * eta[:, None] * (Vhat - V) / (n * d)
+    if loss == "rmse":
+        mse = np.sum(eta[:, None] * (Vhat - V) ** 2) / (n * d)
+        if mse == 0.0:
+            return np.zeros_like(V)
+        return eta[:, None] * (Vhat - V) / (n * d * np.sqrt(mse))
     if loss == "neg_dot":
         return -eta[:, None] * V
     raise ValueError(loss)

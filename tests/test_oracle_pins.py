@@ -17,7 +17,7 @@ from synth_inputs import make_config
 
 RNG = np.random.default_rng(12345)
 KINDS = ["linear", "mlp2_gelu", "swiglu", "glu"]
-LOSSES = ["mse", "neg_dot"]
+LOSSES = ["mse", "neg_dot", "rmse"]
 
 
 def rand(*shape, scale=1.0):
@@ -638,3 +638,33 @@ def test_glu_dot_step_in_closed_form():
     W = orc.unpack("glu", d, d, w)
     assert np.allclose(W["Wa"], Wa, rtol=1e-13, atol=1e-13)
     assert np.allclose(W["Wb"], Wb, rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------- RMSE loss (ViT3 inner-loss table)
+def test_rmse_textbook_value():
+    # errors 1, 2, 3, 4 over n = 2 tokens, d = 2 channels: sqrt((1 + 4 + 9 + 16) / 4)
+    Vhat = np.array([[1.0, 2.0], [3.0, 4.0]])
+    V = np.zeros((2, 2))
+    assert orc.loss_value("rmse", Vhat, V, np.ones(2)) == math.sqrt(7.5)
+    # eta weights each token's squared error inside the root
+    assert abs(orc.loss_value("rmse", Vhat, V, np.array([2.0, 0.0])) - math.sqrt(2 * 5 / 4)) < 1e-15
+
+
+def test_rmse_gradient_has_norm_one_over_sqrt_nd():
+    # with eta = 1, dL/dV_hat = (V_hat - V) / (n d RMSE), whose Frobenius norm is
+    # ||V_hat - V|| / (n d ||V_hat - V|| / sqrt(n d)) = 1 / sqrt(n d) for any data
+    for n, d in ((3, 5), (17, 4)):
+        g = orc.loss_grad("rmse", rand(n, d), rand(n, d), np.ones(n))
+        assert abs(np.linalg.norm(g) - 1.0 / math.sqrt(n * d)) < 1e-14
+
+
+@pytest.mark.parametrize("kind", KINDS)
+def test_rmse_at_zero_error_takes_no_step(kind):
+    # values the inner model already reproduces exactly: the MSE is 0 and the step is 0
+    d, h, n = 4, 6, 7
+    W = rand_w(kind, d, h)
+    K = rand(n, d)
+    V = orc.inner_forward(kind, W, K)[0]
+    cfg = cfg_for(kind, "rmse", d=d, h=h, N=n)
+    _, w = orc.forward_head(cfg, rand(2, d), K, V, np.abs(rand(n)) + 0.1, orc.pack(kind, d, h, W))
+    assert np.array_equal(w, orc.pack(kind, d, h, W))
