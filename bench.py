@@ -54,10 +54,10 @@ def algorithmic_flops(cfg) -> dict:
     if kind == "swiglu":  # token phase: Z1, Z3, V W2; weight grads: G2, G1, G3
         tok, grad, app = 6 * d * h, 6 * d * h, 6 * d * h
     elif kind == "mlp2_gelu":  # token phase: Z, [V_hat], dH; grads: G2, G1
-        tok = (6 if loss == "mse" else 4) * d * h
+        tok = (6 if loss in ("mse", "rmse") else 4) * d * h
         grad, app = 4 * d * h, 4 * d * h
     else:  # linear: [V_hat]; grad G
-        tok, grad, app = (2 * d * d if loss == "mse" else 0), 2 * d * d, 2 * d * d
+        tok, grad, app = (2 * d * d if loss in ("mse", "rmse") else 0), 2 * d * d, 2 * d * d
     chunk = cfg["chunk"] if 0 < cfg["chunk"] < N else N
     nchunks = math.ceil(N / chunk)
     ns = 0

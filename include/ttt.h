@@ -69,7 +69,12 @@ extern "C" {
 #define TTT_ERR_WORKSPACE (-6)   /* workspace too small or misaligned */
 
 typedef enum { TTT_INNER_LINEAR = 0, TTT_INNER_MLP2_GELU = 1, TTT_INNER_SWIGLU = 2 } ttt_inner_kind;
-typedef enum { TTT_LOSS_MSE = 0, TTT_LOSS_NEG_DOT = 1 } ttt_loss_kind;
+typedef enum {
+  TTT_LOSS_MSE = 0,      /* sum_i eta_i ||F(k_i) - v_i||^2 / (n d) over the chunk's n tokens */
+  TTT_LOSS_NEG_DOT = 1,  /* -sum_i eta_i <F(k_i), v_i> */
+  TTT_LOSS_RMSE = 2      /* sqrt of the MSE (ViT3 digest, section 03, inner-loss table); no step where
+                            the MSE is 0.  fp32 path only: TTT_BF16 returns TTT_ERR_UNSUPPORTED */
+} ttt_loss_kind;
 typedef enum {
   TTT_OPT_GD = 0,            /* U = G */
   TTT_OPT_MOMENTUM = 1,      /* M <- beta M + G; U = M */

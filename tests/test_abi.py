@@ -65,7 +65,7 @@ def test_invalid_configurations_are_rejected(bad):
 
 def test_invalid_enum_and_flag_values_are_rejected():
     from weight_sequence_mixing_b200 import binding
-    for field, value in (("inner", 7), ("loss", -1), ("opt", 9), ("dtype", 5), ("flags", 128), ("ns_iters", -1),
+    for field, value in (("inner", 7), ("loss", -1), ("loss", 3), ("opt", 9), ("dtype", 5), ("flags", 128), ("ns_iters", -1),
                          ("epochs", -1), ("epochs", 65)):
         c = binding.make_config(make_config(N=16, d=64, h=128))
         setattr(c, field, value)
@@ -124,6 +124,17 @@ def test_forward_state_checks_state_alignment_without_touching_the_gpu():
     assert lib.ttt_forward_state(h, None, fake, fake, None, fake, fake, None, None, None, fake, 1 << 30,
                                  None) == binding.TTT_ERR_INVALID_ARG
     lib.ttt_destroy(h)
+
+
+@pytest.mark.parametrize("inner", ["linear", "mlp2_gelu", "swiglu"])
+def test_rmse_loss_runs_on_the_fp32_path_only(inner):
+    from weight_sequence_mixing_b200 import binding
+    kw = dict(N=300, d=128, h=128, inner=inner, loss="rmse")
+    st, h = _create(binding.make_config(make_config(dtype="f32", **kw)))
+    assert st == 0, binding.status_string(st)
+    binding.LIB.ttt_destroy(h)
+    st, h = _create(binding.make_config(make_config(dtype="bf16", **kw)))
+    assert st == binding.TTT_ERR_UNSUPPORTED and not h.value
 
 
 def test_forward_rejects_null_and_small_workspace_without_touching_the_gpu():

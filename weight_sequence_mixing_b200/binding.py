@@ -23,7 +23,7 @@ TTT_ERR_TIMEOUT = -5
 TTT_ERR_WORKSPACE = -6
 
 INNER = {"linear": 0, "mlp2_gelu": 1, "swiglu": 2}
-LOSS = {"mse": 0, "neg_dot": 1}
+LOSS = {"mse": 0, "neg_dot": 1, "rmse": 2}
 OPT = {"gd": 0, "momentum": 1, "muon": 2, "momentum_muon": 3}
 DTYPE = {"f32": 0, "bf16": 1}
 FLAG_KEY_INSTNORM = 1

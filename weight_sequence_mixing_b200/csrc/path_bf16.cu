@@ -839,7 +839,8 @@ void choose_grad_shape(const Plan& p, int Cp, int* splits, int* tile_rows, int* 
 int plan_layout_bf16(Plan* p) {
   const ttt_config& c = p->cfg;
   const int d = c.d, h = c.h;
-  // supported shapes of the tensor-core path
+  // supported shapes and losses of the tensor-core path
+  if (c.loss == TTT_LOSS_RMSE) return TTT_ERR_UNSUPPORTED;
   if (d % 64 != 0) return TTT_ERR_UNSUPPORTED;
   if (c.inner != TTT_INNER_LINEAR && h % 128 != 0) return TTT_ERR_UNSUPPORTED;
   if (c.inner == TTT_INNER_SWIGLU && c.loss != TTT_LOSS_NEG_DOT) return TTT_ERR_UNSUPPORTED;

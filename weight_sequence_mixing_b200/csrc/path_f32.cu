@@ -128,9 +128,32 @@ __global__ void swiglu_back_kernel(int64_t n, float* Z1, const float* Z3, float*
   }
 }
 
-// dY = dL/dV_hat for the chunk; Vhat [Z][n][d] (overwritten), V rows t0.. of [Z][N][d]
+// RMSE of the chunk per z: sqrt(sum_i eta_i ||Vhat_i - V_i||^2 / (n d)); one CTA of
+// 256 threads per z, fixed-order tree reduction.
+__global__ void rmse_kernel(int n, int d, const float* Y, int64_t y_sz, const float* V, int64_t v_sz, int t0,
+                            const float* eta, int64_t eta_sz, float eta_scalar, float* rms) {
+  __shared__ float red[256];
+  const int z = blockIdx.x;
+  float s = 0.f;
+  for (int64_t i = threadIdx.x; i < int64_t(n) * d; i += blockDim.x) {
+    const int r = int(i / d), c = int(i % d);
+    const float e = eta ? eta[z * eta_sz + t0 + r] : eta_scalar;
+    const float diff = Y[z * y_sz + i] - V[z * v_sz + int64_t(t0 + r) * d + c];
+    s += e * diff * diff;
+  }
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) rms[z] = sqrtf(red[0] / (float(n) * float(d)));
+}
+
+// dY = dL/dV_hat for the chunk; Vhat [Z][n][d] (overwritten), V rows t0.. of [Z][N][d].
+// RMSE: the MSE gradient over 2 RMSE (rms [Z] from rmse_kernel), zero where RMSE = 0.
 __global__ void loss_grad_kernel(int loss, int Z, int n, int d, float* Y, int64_t y_sz, const float* V, int64_t v_sz,
-                                 int t0, const float* eta, int64_t eta_sz, float eta_scalar) {
+                                 int t0, const float* eta, int64_t eta_sz, float eta_scalar, const float* rms) {
   const int64_t total = int64_t(Z) * n * d;
   const float mse_coef = 2.0f / (float(n) * float(d));
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
@@ -139,7 +162,14 @@ __global__ void loss_grad_kernel(int loss, int Z, int n, int d, float* Y, int64_
     const float v = V[z * v_sz + int64_t(t0 + r) * d + c];
     const float e = eta ? eta[z * eta_sz + t0 + r] : eta_scalar;
     float* y = Y + z * y_sz + int64_t(r) * d + c;
-    *y = loss == TTT_LOSS_MSE ? mse_coef * e * (*y - v) : -e * v;
+    if (loss == TTT_LOSS_NEG_DOT) {
+      *y = -e * v;
+    } else if (loss == TTT_LOSS_MSE) {
+      *y = mse_coef * e * (*y - v);
+    } else {
+      const float q = rms[z];
+      *y = q > 0.f ? e * (*y - v) / (float(n) * float(d) * q) : 0.f;
+    }
   }
 }
 
@@ -253,7 +283,7 @@ __global__ void nonfinite_kernel(int64_t n, const float* x, unsigned* status) {
 int grid_for(int64_t n) { return int(std::min<int64_t>((n + 255) / 256, 148 * 16)); }
 
 // ------------------------------------------------------------------ workspace
-enum Buf { bW, bM, bG, bXn, bZ1, bZ3, bA, bH, bdH, bY, bNX, bNX2, bNS, bNT, kNumBuf };
+enum Buf { bW, bM, bG, bXn, bZ1, bZ3, bA, bH, bdH, bY, bNX, bNX2, bNS, bNT, bRms, kNumBuf };
 
 struct F32View {
   float* b[kNumBuf];
@@ -375,10 +405,15 @@ int update_chunk(const Plan& p, const F32View& v, const Io& io, cudaStream_t st,
   r = inner_forward(p, v, st, X, n, v.b[bY], Rd, d);
   if (r) return r;
   const int64_t tot = int64_t(Z) * n * d;
+  if (c.loss == TTT_LOSS_RMSE) {
+    StageScope _sc(kStageOther, st);
+    rmse_kernel<<<Z, 256, 0, st>>>(n, d, v.b[bY], Rd, V, int64_t(N) * d, t0, io.eta, int64_t(N), c.eta_scalar,
+                                   v.b[bRms]);
+  }
   {
     StageScope _sc(kStageOther, st);
     loss_grad_kernel<<<grid_for(tot), 256, 0, st>>>(c.loss, Z, n, d, v.b[bY], Rd, V, int64_t(N) * d, t0, io.eta,
-                                                     int64_t(N), c.eta_scalar);
+                                                     int64_t(N), c.eta_scalar, v.b[bRms]);
   }
   // backprop into the gradient buffer G [Z][P]
   float* G = v.b[bG];
@@ -453,8 +488,9 @@ int plan_layout_f32(Plan* p) {
   const int64_t Z = p->BH, d = c.d, h = c.h, P = p->P;
   const int64_t R = std::max<int64_t>(p->chunk, c.Nq);  // rows per head in the activation buffers
   const int64_t m = std::min(d, h), n = std::max(d, h);
-  const int64_t sizes[kNumBuf] = {Z * P, Z * P, Z * P, Z * R * d, Z * R * h, Z * R * h, Z * R * h,
-                                  Z * R * h, Z * R * h, Z * R * d, Z * m * n, Z * m * n, Z * m * m, Z * m * m};
+  const int64_t sizes[kNumBuf] = {Z * P,     Z * P,     Z * P,     Z * R * d, Z * R * h, Z * R * h,
+                                  Z * R * h, Z * R * h, Z * R * h, Z * R * d, Z * m * n, Z * m * n,
+                                  Z * m * m, Z * m * m, Z};
   size_t o = 256;
   for (int i = 0; i < kNumBuf; ++i) {
     p->off[i] = o;

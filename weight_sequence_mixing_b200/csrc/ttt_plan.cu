@@ -10,7 +10,7 @@ static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int plan_build(const ttt_config& c, Plan* p) {
   if (c.B < 1 || c.H < 1 || c.N < 1 || c.Nq < 1 || c.d < 1) return TTT_ERR_INVALID_ARG;
   if (c.inner < TTT_INNER_LINEAR || c.inner > TTT_INNER_SWIGLU) return TTT_ERR_INVALID_ARG;
-  if (c.loss < TTT_LOSS_MSE || c.loss > TTT_LOSS_NEG_DOT) return TTT_ERR_INVALID_ARG;
+  if (c.loss < TTT_LOSS_MSE || c.loss > TTT_LOSS_RMSE) return TTT_ERR_INVALID_ARG;
   if (c.opt < TTT_OPT_GD || c.opt > TTT_OPT_MOMENTUM_MUON) return TTT_ERR_INVALID_ARG;
   if (c.dtype != TTT_F32 && c.dtype != TTT_BF16) return TTT_ERR_INVALID_ARG;
   if (c.causal != 0 && c.causal != 1) return TTT_ERR_INVALID_ARG;
