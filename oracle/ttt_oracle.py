@@ -19,7 +19,9 @@ What is computed (sources: the pages' text, cited per function):
   matrices [LaCT analysis, "Nonlinear memory complements local attention"];
   simplified GLU F(x) = (x Wa^T) * SiLU(x Wb^T) with two d x d matrices and no
   output projection [ViT3 digest, section 03, inner-model table and the F1 module
-  of the ViT3 design].
+  of the ViT3 design]; depthwise convolution DWConv(x) over the token grid, one k x k
+  kernel per channel [ViT3 digest, section 03, guideline 6 and the inner-model table;
+  the F2 module of the ViT3 design].
 * Losses: MSE, RMSE = sqrt(MSE), and the negative dot product -<F(k_i), v_i> [ViT3
   digest, inner-loss table; LaCT analysis, "Nonlinear memory"], summed with each
   token's learning rate eta_i [LaCT analysis, "Nonlinear memory"].
@@ -49,7 +51,11 @@ Readings taken where the pages are silent (each is listed in the design doc):
   and is not row-normalised [TTT vs Sleep, "Side one": the first layer is adjusted];
   R22 the simplified GLU has no biases, Wa is the linear branch, Wb the SiLU gate;
   R23 RMSE is the square root of the R2 MSE of the chunk (eta inside the root); its
-  gradient is the MSE gradient over 2 sqrt(MSE), and zero where the MSE is zero.
+  gradient is the MSE gradient over 2 sqrt(MSE), and zero where the MSE is zero;
+  R24 DWConv: tokens in raster order on a grid_h x grid_w grid, a 'same' depthwise
+  cross-correlation with zero padding, odd k (3 by default, the size of the pages'
+  convolution row), no bias, weights [d][k*k] (PyTorch's [d, 1, k, k]); the whole grid
+  is one chunk (non-causal) and the queries lie on the same grid.
 
 Parity: every part here is pinned by tests in tests/test_oracle_pins.py (closed forms,
 finite differences, SVD, invariances).  The full-size GELU-MLP / SwiGLU / Muon results
@@ -99,7 +105,7 @@ def silu_prime(x):
 # ---------------------------------------------------------------------------
 # fast-weight packing ([out, in] matrices, concatenated per head)
 # ---------------------------------------------------------------------------
-def matrix_shapes(kind: str, d: int, h: int):
+def matrix_shapes(kind: str, d: int, h: int, ksize: int = 3):
     if kind == "linear":
         return [("W", d, d)]
     if kind == "mlp2_gelu":
@@ -108,29 +114,68 @@ def matrix_shapes(kind: str, d: int, h: int):
         return [("W1", h, d), ("W3", h, d), ("W2", d, h)]
     if kind == "glu":
         return [("Wa", d, d), ("Wb", d, d)]
+    if kind == "dwconv":
+        return [("Wc", d, ksize * ksize)]
     raise ValueError(kind)
 
 
-def unpack(kind, d, h, flat):
+def unpack(kind, d, h, flat, ksize=3):
     flat = np.asarray(flat, dtype=F64)
     out, off = {}, 0
-    for name, r, c in matrix_shapes(kind, d, h):
+    for name, r, c in matrix_shapes(kind, d, h, ksize):
         out[name] = flat[off:off + r * c].reshape(r, c).copy()
         off += r * c
     assert off == flat.size
     return out
 
 
-def pack(kind, d, h, W):
-    return np.concatenate([W[name].reshape(-1) for name, _, _ in matrix_shapes(kind, d, h)])
+def pack(kind, d, h, W, ksize=3):
+    return np.concatenate([W[name].reshape(-1) for name, _, _ in matrix_shapes(kind, d, h, ksize)])
+
+
+# ---------------------------------------------------------------------------
+# depthwise convolution over the token grid (reading R24)
+# ---------------------------------------------------------------------------
+def _pad_grid(X, grid, r):
+    gh, gw = grid
+    Xp = np.zeros((gh + 2 * r, gw + 2 * r, X.shape[1]), dtype=F64)
+    Xp[r:r + gh, r:r + gw] = X.reshape(gh, gw, X.shape[1])
+    return Xp
+
+
+def dwconv_apply(Wc, X, grid):
+    """Y[(y, x), c] = sum_{a, b < k} Wc[c, a k + b] X[(y + a - r, x + b - r), c], r = k // 2,
+    zero outside the grid.  X [gh * gw, d] in raster order."""
+    gh, gw = grid
+    k = int(round(np.sqrt(Wc.shape[1])))
+    Xp = _pad_grid(X, grid, k // 2)
+    Y = np.zeros((gh, gw, X.shape[1]), dtype=F64)
+    for a in range(k):
+        for b in range(k):
+            Y += Wc[:, a * k + b] * Xp[a:a + gh, b:b + gw]
+    return Y.reshape(gh * gw, X.shape[1])
+
+
+def dwconv_weight_grad(X, dY, grid, k):
+    """Gradient of sum(dY * dwconv_apply(Wc, X)) in Wc: for each channel and tap, the sum
+    over the grid of dY times the input shifted by that tap."""
+    gh, gw = grid
+    Xp = _pad_grid(X, grid, k // 2)
+    dYg = dY.reshape(gh, gw, dY.shape[1])
+    G = np.zeros((dY.shape[1], k * k), dtype=F64)
+    for a in range(k):
+        for b in range(k):
+            G[:, a * k + b] = np.sum(dYg * Xp[a:a + gh, b:b + gw], axis=(0, 1))
+    return G
 
 
 # ---------------------------------------------------------------------------
 # inner model: forward and hand-derived backward
 # [ViT3 digest section 02; LaCT analysis "Nonlinear memory"]
 # ---------------------------------------------------------------------------
-def inner_forward(kind, W, X):
-    """Returns (F_W(X), cache).  X is [n, d] (rows are tokens)."""
+def inner_forward(kind, W, X, grid=None):
+    """Returns (F_W(X), cache).  X is [n, d] (rows are tokens; for DWConv the n = gh * gw
+    tokens of the grid ``grid`` = (gh, gw) in raster order)."""
     if kind == "linear":
         return X @ W["W"].T, dict(X=X)
     if kind == "mlp2_gelu":
@@ -148,6 +193,8 @@ def inner_forward(kind, W, X):
         Zb = X @ W["Wb"].T
         S = silu(Zb)
         return Za * S, dict(X=X, Za=Za, Zb=Zb, S=S)
+    if kind == "dwconv":
+        return dwconv_apply(W["Wc"], X, grid), dict(X=X, grid=grid)
     raise ValueError(kind)
 
 
@@ -171,6 +218,9 @@ def inner_backward(kind, W, cache, dY):
         dZa = dY * cache["S"]
         dZb = dY * cache["Za"] * silu_prime(cache["Zb"])
         return dict(Wa=dZa.T @ X, Wb=dZb.T @ X)
+    if kind == "dwconv":
+        k = int(round(np.sqrt(W["Wc"].shape[1])))
+        return dict(Wc=dwconv_weight_grad(X, dY, cache["grid"], k))
     raise ValueError(kind)
 
 
@@ -247,7 +297,7 @@ def update_chunk(cfg, W, M, Kc, Vc, etac):
     """One full-batch gradient step on one chunk (W, M updated in place)."""
     kind = cfg["inner"]
     X = instance_norm(Kc, cfg["in_eps"]) if cfg["key_instnorm"] else Kc
-    Vhat, cache = inner_forward(kind, W, X)
+    Vhat, cache = inner_forward(kind, W, X, _grid(cfg))
     dY = loss_grad(cfg["loss"], Vhat, Vc, etac)
     G = inner_backward(kind, W, cache, dY)
     opt = cfg["opt"]
@@ -269,6 +319,10 @@ def update_chunk(cfg, W, M, Kc, Vc, etac):
             W[name] = row_l2_normalize(W[name])
 
 
+def _grid(cfg):
+    return (int(cfg["grid_h"]), int(cfg["grid_w"])) if cfg["inner"] == "dwconv" else None
+
+
 def forward_head(cfg, Q, K, V, eta, w0, m0=None, return_m=False):
     """One (batch, head): returns (O [Nq, d], W* packed [P]) in fp64, and with
     ``return_m`` also the momentum buffer after the last step (packed [P]).
@@ -279,6 +333,8 @@ def forward_head(cfg, Q, K, V, eta, w0, m0=None, return_m=False):
     with (streamed state, LaCT "Video and distributed"); None means zero (R9).
     """
     kind, d, h = cfg["inner"], cfg["d"], cfg["h"]
+    ks = int(cfg.get("ksize", 3))
+    grid = _grid(cfg)
     Q = np.asarray(Q, dtype=F64)
     K = np.asarray(K, dtype=F64)
     V = np.asarray(V, dtype=F64)
@@ -287,9 +343,12 @@ def forward_head(cfg, Q, K, V, eta, w0, m0=None, return_m=False):
         eta = np.full((N,), float(cfg["eta_scalar"]), dtype=F64)
     else:
         eta = np.asarray(eta, dtype=F64)
-    W = unpack(kind, d, h, w0)
-    M = unpack(kind, d, h, m0) if m0 is not None else {name: np.zeros_like(m) for name, m in W.items()}
+    W = unpack(kind, d, h, w0, ks)
+    M = unpack(kind, d, h, m0, ks) if m0 is not None else {name: np.zeros_like(m) for name, m in W.items()}
     bounds = chunk_bounds(N, cfg["chunk"])
+    if grid is not None:  # reading R24: the whole grid is one non-causal chunk, queries on it too
+        if grid[0] * grid[1] != N or Q.shape[0] != N or len(bounds) != 1 or cfg["causal"] or ks % 2 == 0:
+            raise ValueError("DWConv needs one non-causal chunk over a grid_h x grid_w grid, Nq == N, odd k")
     # inner epochs: that many full-batch steps on each chunk before the next one
     # (ViT3 digest, inner-training ablation); momentum carries through them.  A
     # read-only call takes none (LaCT "Video and distributed": chunks that only read).
@@ -299,17 +358,17 @@ def forward_head(cfg, Q, K, V, eta, w0, m0=None, return_m=False):
             raise ValueError("causal order needs Nq == N")
         O = np.empty((N, d), dtype=F64)
         for s, e in bounds:
-            O[s:e] = inner_forward(kind, W, Q[s:e])[0]
+            O[s:e] = inner_forward(kind, W, Q[s:e], grid)[0]
             for _ in range(epochs):
                 update_chunk(cfg, W, M, K[s:e], V[s:e], eta[s:e])
     else:
         for s, e in bounds:
             for _ in range(epochs):
                 update_chunk(cfg, W, M, K[s:e], V[s:e], eta[s:e])
-        O = inner_forward(kind, W, Q)[0]
+        O = inner_forward(kind, W, Q, grid)[0]
     if return_m:
-        return O, pack(kind, d, h, W), pack(kind, d, h, M)
-    return O, pack(kind, d, h, W)
+        return O, pack(kind, d, h, W, ks), pack(kind, d, h, M, ks)
+    return O, pack(kind, d, h, W, ks)
 
 
 def _np(t):
@@ -329,7 +388,7 @@ def forward(cfg, Q, K, V, eta, W0, heads=None, M0=None, return_m=False):
     """
     B, H = cfg["B"], cfg["H"]
     Nq, d = cfg["Nq"], cfg["d"]
-    P = sum(r * c for _, r, c in matrix_shapes(cfg["inner"], d, cfg["h"]))
+    P = sum(r * c for _, r, c in matrix_shapes(cfg["inner"], d, cfg["h"], int(cfg.get("ksize", 3))))
     O = np.full((B, H, Nq, d), np.nan)
     Ws = np.full((B, H, P), np.nan)
     Ms = np.full((B, H, P), np.nan)

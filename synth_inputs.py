@@ -15,6 +15,7 @@ Tensor layouts (row-major, contiguous):
     swiglu    [W1 (h x d) | W3 (h x d) | W2 (d x h)]
     glu       [Wa (d x d) | Wb (d x d)]   (oracle only; the CUDA path runs it as a
               SwiGLU with h = d, W1 = Wb, W3 = Wa, W2 = I and the first-layer-only flag)
+    dwconv    [Wc (d x k*k)]              (oracle only: one k x k kernel per channel)
 
 Data recipes (the pages' workloads use image / text / multi-view data that is
 not available here; seeded Gaussians of the same shapes stand in for them):
@@ -43,6 +44,7 @@ _DEFAULTS = dict(
     inner="mlp2_gelu", loss="mse", opt="gd", dtype="bf16",
     key_instnorm=False, weight_l2norm=False, direct_launch=False, single_cta=False,
     w0_per_batch=False, no_update=False, first_layer_only=False,
+    grid_h=0, grid_w=0, ksize=3,  # DWConv: token grid and kernel size
     eta_mode="scalar",           # "scalar" | "per_token"
     eta_scalar=1.0, lr=1.0, momentum=0.9,
     ns_iters=5, ns_coeff=(3.4445, -4.7750, 2.0315), in_eps=1e-5, epochs=1,
@@ -112,6 +114,8 @@ def matrix_shapes(cfg) -> list[tuple[str, int, int]]:
         return [("W1", h, d), ("W3", h, d), ("W2", d, h)]
     if kind == "glu":
         return [("Wa", d, d), ("Wb", d, d)]
+    if kind == "dwconv":
+        return [("Wc", d, cfg["ksize"] * cfg["ksize"])]
     raise ValueError(kind)
 
 

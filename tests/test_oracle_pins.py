@@ -668,3 +668,106 @@ def test_rmse_at_zero_error_takes_no_step(kind):
     cfg = cfg_for(kind, "rmse", d=d, h=h, N=n)
     _, w = orc.forward_head(cfg, rand(2, d), K, V, np.abs(rand(n)) + 0.1, orc.pack(kind, d, h, W))
     assert np.array_equal(w, orc.pack(kind, d, h, W))
+
+
+# ---------------------------------------------------------------- DWConv (ViT3's F2 module)
+def _dw_cfg(loss, gh, gw, d, k=3, **kw):
+    return cfg_for("dwconv", loss, d=d, h=d, N=gh * gw, grid_h=gh, grid_w=gw, ksize=k, **kw)
+
+
+def _brute_dwconv(Wc, X, gh, gw, k):
+    """Scalar loops: every output pixel and channel sums its k x k neighbours that lie on the grid."""
+    r = k // 2
+    out = []
+    for y in range(gh):
+        for x in range(gw):
+            row = []
+            for c in range(X.shape[1]):
+                s = 0.0
+                for a in range(k):
+                    for b in range(k):
+                        yy, xx = y + a - r, x + b - r
+                        if 0 <= yy < gh and 0 <= xx < gw:
+                            s += float(Wc[c, a * k + b]) * float(X[yy * gw + xx, c])
+                row.append(s)
+            out.append(row)
+    return np.array(out)
+
+
+@pytest.mark.parametrize("gh,gw,k", [(4, 5, 3), (1, 7, 3), (3, 3, 5), (2, 6, 1)])
+def test_dwconv_forward_matches_scalar_loops(gh, gw, k):
+    d = 3
+    Wc, X = rand(d, k * k), rand(gh * gw, d)
+    Y = orc.inner_forward("dwconv", {"Wc": Wc}, X, (gh, gw))[0]
+    assert np.allclose(Y, _brute_dwconv(Wc, X, gh, gw, k), rtol=1e-13, atol=1e-13)
+
+
+def test_dwconv_forward_and_weight_gradient_match_scipy_correlate2d():
+    # per channel: the layer is a 'same' 2-D cross-correlation with zero fill, and the kernel
+    # gradient is the 'valid' cross-correlation of the zero-padded input with dL/dY
+    from scipy.signal import correlate2d
+
+    gh, gw, d, k = 5, 6, 4, 3
+    Wc, X, dY = rand(d, k * k), rand(gh * gw, d), rand(gh * gw, d)
+    Y = orc.inner_forward("dwconv", {"Wc": Wc}, X, (gh, gw))[0]
+    G = orc.inner_backward("dwconv", {"Wc": Wc}, {"X": X, "grid": (gh, gw)}, dY)["Wc"]
+    for c in range(d):
+        Xc = X[:, c].reshape(gh, gw)
+        ref = correlate2d(Xc, Wc[c].reshape(k, k), mode="same", boundary="fill", fillvalue=0.0)
+        assert np.allclose(Y[:, c].reshape(gh, gw), ref, rtol=1e-13, atol=1e-13)
+        Xpad = np.pad(Xc, 1)
+        gref = correlate2d(Xpad, dY[:, c].reshape(gh, gw), mode="valid")
+        assert np.allclose(G[c].reshape(k, k), gref, rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("loss", LOSSES)
+def test_dwconv_gradients_by_central_finite_differences(loss):
+    gh, gw, d, k = 3, 4, 2, 3
+    W = {"Wc": rand(d, k * k)}
+    X, V = rand(gh * gw, d), rand(gh * gw, d)
+    eta = np.abs(rand(gh * gw)) + 0.1
+    grid = (gh, gw)
+
+    def L(Wd):
+        return orc.loss_value(loss, orc.inner_forward("dwconv", Wd, X, grid)[0], V, eta)
+
+    Vhat, cache = orc.inner_forward("dwconv", W, X, grid)
+    G = orc.inner_backward("dwconv", W, cache, orc.loss_grad(loss, Vhat, V, eta))["Wc"]
+    fd = np.zeros_like(G)
+    eps = 1e-6
+    for idx in np.ndindex(G.shape):
+        Wp, Wm = {"Wc": W["Wc"].copy()}, {"Wc": W["Wc"].copy()}
+        Wp["Wc"][idx] += eps
+        Wm["Wc"][idx] -= eps
+        fd[idx] = (L(Wp) - L(Wm)) / (2 * eps)
+    assert np.linalg.norm(fd - G) / np.linalg.norm(G) < 1e-7
+
+
+@pytest.mark.parametrize("loss", LOSSES)
+def test_dwconv_with_one_tap_is_the_diagonal_of_the_linear_model(loss):
+    # k = 1: each channel is scaled by its own weight, i.e. the linear model with a diagonal W;
+    # one gradient step moves the diagonal of the linear model's W by the same amount
+    gh, gw, d = 3, 5, 4
+    w0 = rand(d)
+    Q, K, V, eta = rand(gh * gw, d), rand(gh * gw, d), rand(gh * gw, d), np.abs(rand(gh * gw)) + 0.1
+    Od, wd = orc.forward_head(_dw_cfg(loss, gh, gw, d, k=1), Q, K, V, eta, w0)
+    _, wl = orc.forward_head(cfg_for("linear", loss, d=d, N=gh * gw), Q, K, V, eta, np.diag(w0).reshape(-1))
+    assert np.allclose(wd, np.diag(wl.reshape(d, d)), rtol=1e-13, atol=1e-13)
+    assert np.allclose(Od, Q * wd, rtol=1e-13, atol=1e-13)
+
+
+def test_dwconv_layer_reads_the_grid_once_as_one_chunk():
+    gh, gw, d = 3, 4, 2
+    Q, K, V, eta = rand(gh * gw, d), rand(gh * gw, d), rand(gh * gw, d), np.abs(rand(gh * gw)) + 0.1
+    w0 = rand(d * 9)
+    with pytest.raises(ValueError):
+        orc.forward_head(_dw_cfg("neg_dot", gh, gw, d, chunk=4), Q, K, V, eta, w0)
+    with pytest.raises(ValueError):
+        orc.forward_head(_dw_cfg("neg_dot", gh, gw, d, causal=1), Q, K, V, eta, w0)
+    with pytest.raises(ValueError):
+        orc.forward_head(_dw_cfg("neg_dot", gh, gw + 1, d), Q, K, V, eta, w0)
+    # the ViT3 recipe: dot loss, one full-batch step, rate 1 -> W* = W0 + sum_p eta_p v_p (x) shifted k_p
+    O, w = orc.forward_head(_dw_cfg("neg_dot", gh, gw, d, eta_mode="scalar"), Q, K, V, None, w0)
+    G = orc.dwconv_weight_grad(K, -V, (gh, gw), 3)
+    assert np.allclose(w, w0 - G.reshape(-1), rtol=1e-13, atol=1e-13)
+    assert np.allclose(O, _brute_dwconv(w.reshape(d, 9), Q, gh, gw, 3), rtol=1e-13, atol=1e-13)
