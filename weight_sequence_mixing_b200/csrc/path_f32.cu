@@ -507,7 +507,7 @@ int run_f32(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
   const ttt_config& c = p.cfg;
   const F32View v = view(p, ws);
   const int Z = p.BH, d = c.d;
-  const int64_t P = p.P, Rd = int64_t(p.off[kNumBuf]) * d;
+  const int64_t P = p.P;
   {
     StageScope _sc(kStageOther, st);
     const int w0_rows = (c.flags & TTT_FLAG_W0_PER_BATCH) ? Z : c.H;  // W0 [H][P] or [B*H][P]
@@ -542,7 +542,6 @@ int run_f32(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
     }
     if (r) return r;
   }
-  (void)Rd;
   if (io.W_out &&
       cudaMemcpyAsync(io.W_out, v.b[bW], size_t(Z) * P * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return TTT_ERR_CUDA;
