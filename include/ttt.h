@@ -18,6 +18,10 @@
  *        TTT_INNER_MLP2_GELU  [W1 (h x d) | W2 (d x h)]         F(x) = GELU(x W1^T) W2^T
  *        TTT_INNER_SWIGLU     [W1 (h x d) | W3 (h x d) | W2 (d x h)]
  *                                                    F(x) = (SiLU(x W1^T) * x W3^T) W2^T
+ *        TTT_INNER_DWCONV     [Wc (d x k*k)]  one k x k kernel per channel (PyTorch [d,1,k,k]):
+ *                             F(X)[(y,x),c] = sum_{a,b<k} Wc[c][a k + b] X[(y+a-k/2, x+b-k/2), c]
+ *                             over the grid_h x grid_w token grid (raster order), zero outside
+ *                             (ViT3 digest, section 03, guideline 6 and inner-model table)
  *   - Q [B,H,Nq,d], K [B,H,N,d], V [B,H,N,d] and O [B,H,Nq,d] in `dtype`
  *     (fp32 or bf16); eta [B,H,N] fp32; W0 [H,P] fp32 (shared by every batch
  *     entry; [B,H,P] with TTT_FLAG_W0_PER_BATCH); W_out [B,H,P] fp32.
@@ -68,7 +72,14 @@ extern "C" {
 #define TTT_ERR_TIMEOUT (-5)     /* a bounded device-side wait ran out (device status word) */
 #define TTT_ERR_WORKSPACE (-6)   /* workspace too small or misaligned */
 
-typedef enum { TTT_INNER_LINEAR = 0, TTT_INNER_MLP2_GELU = 1, TTT_INNER_SWIGLU = 2 } ttt_inner_kind;
+typedef enum {
+  TTT_INNER_LINEAR = 0,
+  TTT_INNER_MLP2_GELU = 1,
+  TTT_INNER_SWIGLU = 2,
+  TTT_INNER_DWCONV = 3 /* the whole grid is one non-causal chunk (Nq == N, queries on the same grid);
+                          loss MSE or NEG_DOT, optimizer GD or MOMENTUM, no key instance-norm;
+                          other combinations return TTT_ERR_UNSUPPORTED */
+} ttt_inner_kind;
 typedef enum {
   TTT_LOSS_MSE = 0,      /* sum_i eta_i ||F(k_i) - v_i||^2 / (n d) over the chunk's n tokens */
   TTT_LOSS_NEG_DOT = 1,  /* -sum_i eta_i <F(k_i), v_i> */
@@ -120,6 +131,8 @@ typedef struct ttt_config {
   int32_t epochs;     /* full-batch inner steps per chunk, 1..64 (default 1; 0 reads as 1): the
                          inner model trains for `epochs` passes over each chunk before moving on
                          (ViT3 digest, inner-training ablation); momentum carries through */
+  int32_t grid_h, grid_w; /* TTT_INNER_DWCONV: the token grid, grid_h * grid_w == N (else ignored) */
+  int32_t ksize;          /* TTT_INNER_DWCONV: odd kernel size 1..7 (default 3; else ignored) */
 } ttt_config;
 
 typedef struct ttt_handle ttt_handle;

@@ -137,6 +137,37 @@ def test_rmse_loss_runs_on_the_fp32_path_only(inner):
     assert st == binding.TTT_ERR_UNSUPPORTED and not h.value
 
 
+def _dw(**kw):
+    base = dict(B=2, H=3, N=20, d=64, inner="dwconv", loss="neg_dot", opt="gd", dtype="bf16", grid_h=4, grid_w=5)
+    base.update(kw)
+    return make_config(**base)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("k", [1, 3, 5, 7])
+def test_dwconv_configuration_is_accepted(dtype, k):
+    from weight_sequence_mixing_b200 import binding
+    st, h = _create(binding.make_config(_dw(dtype=dtype, ksize=k, opt="momentum", loss="mse", weight_l2norm=True)))
+    assert st == 0, binding.status_string(st)
+    assert binding.LIB.ttt_param_count(h) == 64 * k * k
+    assert binding.LIB.ttt_state_size(h) == 2 * 3 * 64 * k * k * 4
+    binding.LIB.ttt_destroy(h)
+    assert binding.plan_info(_dw(dtype=dtype, ksize=k))["path"] == 2
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(grid_w=4), "invalid"), (dict(ksize=2), "invalid"), (dict(ksize=9), "invalid"), (dict(grid_h=0), "invalid"),
+    (dict(Nq=10), "invalid"), (dict(causal=1), "unsupported"), (dict(chunk=10), "unsupported"),
+    (dict(key_instnorm=True), "unsupported"), (dict(loss="rmse"), "unsupported"), (dict(opt="muon"), "unsupported"),
+    (dict(opt="momentum_muon"), "unsupported"),
+])
+def test_dwconv_configurations_outside_the_built_set_are_rejected(bad, status):
+    from weight_sequence_mixing_b200 import binding
+    st, h = _create(binding.make_config(_dw(**bad)))
+    want = binding.TTT_ERR_INVALID_ARG if status == "invalid" else binding.TTT_ERR_UNSUPPORTED
+    assert st == want and not h.value
+
+
 def test_forward_rejects_null_and_small_workspace_without_touching_the_gpu():
     from weight_sequence_mixing_b200 import binding
     st, h = _create(binding.make_config(make_config(N=16, d=64, h=128)))

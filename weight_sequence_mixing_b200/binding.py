@@ -22,7 +22,7 @@ TTT_ERR_NONFINITE = -4
 TTT_ERR_TIMEOUT = -5
 TTT_ERR_WORKSPACE = -6
 
-INNER = {"linear": 0, "mlp2_gelu": 1, "swiglu": 2}
+INNER = {"linear": 0, "mlp2_gelu": 1, "swiglu": 2, "dwconv": 3}
 LOSS = {"mse": 0, "neg_dot": 1, "rmse": 2}
 OPT = {"gd": 0, "momentum": 1, "muon": 2, "momentum_muon": 3}
 DTYPE = {"f32": 0, "bf16": 1}
@@ -52,6 +52,7 @@ class TTTConfig(ctypes.Structure):
         ("flags", ctypes.c_uint32), ("eta_scalar", ctypes.c_float), ("lr", ctypes.c_float),
         ("momentum", ctypes.c_float), ("ns_iters", ctypes.c_int32), ("ns_coeff", ctypes.c_float * 3),
         ("in_eps", ctypes.c_float), ("epochs", ctypes.c_int32),
+        ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32), ("ksize", ctypes.c_int32),
     ]
 
 
@@ -144,6 +145,9 @@ def make_config(cfg: dict) -> TTTConfig:
         c.ns_coeff[i] = float(cfg["ns_coeff"][i])
     c.in_eps = float(cfg["in_eps"])
     c.epochs = int(cfg.get("epochs", 1))
+    c.grid_h = int(cfg.get("grid_h", 0))
+    c.grid_w = int(cfg.get("grid_w", 0))
+    c.ksize = int(cfg.get("ksize", 3))
     return c
 
 

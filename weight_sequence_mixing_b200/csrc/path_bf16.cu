@@ -962,7 +962,7 @@ extern "C" int ttt_token_pair_capacity(int swiglu) {
 extern "C" int ttt_plan_info(const ttt_handle* h, int* info, int n) {
   if (!h || !info || n < 0) return TTT_ERR_INVALID_ARG;
   const ttt::Plan& p = h->plan;
-  int v[7] = {p.path == ttt::kPathBf16 ? 1 : 0, static_cast<int>(p.chunk), static_cast<int>(p.nchunks), 0, 0, 0, 0};
+  int v[7] = {static_cast<int>(p.path), static_cast<int>(p.chunk), static_cast<int>(p.nchunks), 0, 0, 0, 0};
   if (p.path == ttt::kPathBf16) {
     const ttt::Dims D = ttt::dims_of(p);
     v[3] = D.splits;

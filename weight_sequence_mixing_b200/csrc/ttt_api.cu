@@ -28,6 +28,7 @@ extern "C" void ttt_config_init(ttt_config* c) {
   c->momentum = 0.9f;
   c->ns_iters = 5;
   c->epochs = 1;
+  c->ksize = 3;
   c->ns_coeff[0] = 3.4445f;
   c->ns_coeff[1] = -4.7750f;
   c->ns_coeff[2] = 2.0315f;

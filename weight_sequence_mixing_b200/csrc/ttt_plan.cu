@@ -9,13 +9,23 @@ static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int plan_build(const ttt_config& c, Plan* p) {
   if (c.B < 1 || c.H < 1 || c.N < 1 || c.Nq < 1 || c.d < 1) return TTT_ERR_INVALID_ARG;
-  if (c.inner < TTT_INNER_LINEAR || c.inner > TTT_INNER_SWIGLU) return TTT_ERR_INVALID_ARG;
+  if (c.inner < TTT_INNER_LINEAR || c.inner > TTT_INNER_DWCONV) return TTT_ERR_INVALID_ARG;
   if (c.loss < TTT_LOSS_MSE || c.loss > TTT_LOSS_RMSE) return TTT_ERR_INVALID_ARG;
   if (c.opt < TTT_OPT_GD || c.opt > TTT_OPT_MOMENTUM_MUON) return TTT_ERR_INVALID_ARG;
   if (c.dtype != TTT_F32 && c.dtype != TTT_BF16) return TTT_ERR_INVALID_ARG;
   if (c.causal != 0 && c.causal != 1) return TTT_ERR_INVALID_ARG;
   if (c.causal && c.Nq != c.N) return TTT_ERR_INVALID_ARG;
-  if (c.inner != TTT_INNER_LINEAR && c.h < 1) return TTT_ERR_INVALID_ARG;
+  const bool dw = c.inner == TTT_INNER_DWCONV;
+  if ((c.inner == TTT_INNER_MLP2_GELU || c.inner == TTT_INNER_SWIGLU) && c.h < 1) return TTT_ERR_INVALID_ARG;
+  if (dw) {
+    if (c.ksize < 1 || c.ksize > 7 || c.ksize % 2 == 0 || c.grid_h < 1 || c.grid_w < 1 ||
+        static_cast<int64_t>(c.grid_h) * c.grid_w != c.N || c.Nq != c.N)
+      return TTT_ERR_INVALID_ARG;
+    // the grid is one non-causal chunk; the combinations built for it
+    if (c.causal || (c.chunk > 0 && c.chunk < c.N) || (c.flags & TTT_FLAG_KEY_INSTNORM) ||
+        (c.loss != TTT_LOSS_MSE && c.loss != TTT_LOSS_NEG_DOT) || (c.opt != TTT_OPT_GD && c.opt != TTT_OPT_MOMENTUM))
+      return TTT_ERR_UNSUPPORTED;
+  }
   if ((c.flags & ~(TTT_FLAG_KEY_INSTNORM | TTT_FLAG_WEIGHT_L2NORM | TTT_FLAG_DIRECT_LAUNCH |
                    TTT_FLAG_SINGLE_CTA | TTT_FLAG_W0_PER_BATCH | TTT_FLAG_NO_UPDATE |
                    TTT_FLAG_FIRST_LAYER_ONLY)) != 0)
@@ -28,17 +38,19 @@ int plan_build(const ttt_config& c, Plan* p) {
   for (float v : c.ns_coeff)
     if (!std::isfinite(v)) return TTT_ERR_INVALID_ARG;
   if (static_cast<int64_t>(c.B) * c.H > 65535) return TTT_ERR_UNSUPPORTED;
-  if (c.d > 4096 || c.h > 16384) return TTT_ERR_UNSUPPORTED;
+  if (c.d > 4096 || ((c.inner == TTT_INNER_MLP2_GELU || c.inner == TTT_INNER_SWIGLU) && c.h > 16384))
+    return TTT_ERR_UNSUPPORTED;
 
   p->cfg = c;
   p->epochs = c.epochs == 0 ? 1 : c.epochs;
-  const int64_t d = c.d, h = c.inner == TTT_INNER_LINEAR ? c.d : c.h;
+  const int64_t d = c.d, h = (c.inner == TTT_INNER_LINEAR || dw) ? c.d : c.h;
   p->cfg.h = static_cast<int32_t>(h);
-  p->P = c.inner == TTT_INNER_LINEAR ? d * d : c.inner == TTT_INNER_MLP2_GELU ? 2 * d * h : 3 * d * h;
+  p->P = dw ? d * c.ksize * c.ksize
+            : c.inner == TTT_INNER_LINEAR ? d * d : c.inner == TTT_INNER_MLP2_GELU ? 2 * d * h : 3 * d * h;
   p->BH = c.B * c.H;
   p->chunk = (c.chunk <= 0 || c.chunk >= c.N) ? c.N : c.chunk;
   p->nchunks = (c.N + p->chunk - 1) / p->chunk;
-  p->path = c.dtype == TTT_F32 ? kPathF32 : kPathBf16;
+  p->path = dw ? kPathDwconv : c.dtype == TTT_F32 ? kPathF32 : kPathBf16;
 
   // host staging: inputs then outputs, each 256-byte aligned
   const size_t es = c.dtype == TTT_F32 ? 4 : 2;
@@ -52,13 +64,16 @@ int plan_build(const ttt_config& c, Plan* p) {
   p->stg_w = o; o = align_up(o + size_t(p->BH) * p->P * 4, 256);
   p->staging_bytes = o;
 
-  int st = p->path == kPathF32 ? plan_layout_f32(p) : plan_layout_bf16(p);
-  return st;
+  return p->path == kPathDwconv ? plan_layout_dwconv(p)
+         : p->path == kPathF32  ? plan_layout_f32(p)
+                                : plan_layout_bf16(p);
 }
 
 int plan_run(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
   if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return TTT_ERR_CUDA;  // status word
-  return p.path == kPathF32 ? run_f32(p, io, ws, st) : run_bf16(p, io, ws, st);
+  return p.path == kPathDwconv ? run_dwconv(p, io, ws, st)
+         : p.path == kPathF32  ? run_f32(p, io, ws, st)
+                               : run_bf16(p, io, ws, st);
 }
 
 }  // namespace ttt

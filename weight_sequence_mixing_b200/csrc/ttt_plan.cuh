@@ -22,7 +22,7 @@ struct Io {
   void* M_out = nullptr;       // momentum state carried out, or null
 };
 
-enum PathKind : int { kPathF32 = 0, kPathBf16 = 1 };
+enum PathKind : int { kPathF32 = 0, kPathBf16 = 1, kPathDwconv = 2 };
 
 struct Plan {
   ttt_config cfg{};
@@ -46,8 +46,10 @@ int plan_run(const Plan& plan, const Io& io, void* workspace, cudaStream_t st);
 // per-path workspace layout and launch sequence
 int plan_layout_f32(Plan* plan);
 int plan_layout_bf16(Plan* plan);
+int plan_layout_dwconv(Plan* plan);
 int run_f32(const Plan& plan, const Io& io, void* workspace, cudaStream_t st);
 int run_bf16(const Plan& plan, const Io& io, void* workspace, cudaStream_t st);
+int run_dwconv(const Plan& plan, const Io& io, void* workspace, cudaStream_t st);
 
 }  // namespace ttt
 
