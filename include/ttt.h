@@ -84,7 +84,7 @@ typedef enum {
   TTT_LOSS_MSE = 0,      /* sum_i eta_i ||F(k_i) - v_i||^2 / (n d) over the chunk's n tokens */
   TTT_LOSS_NEG_DOT = 1,  /* -sum_i eta_i <F(k_i), v_i> */
   TTT_LOSS_RMSE = 2      /* sqrt of the MSE (ViT3 digest, section 03, inner-loss table); no step where
-                            the MSE is 0.  fp32 path only: TTT_BF16 returns TTT_ERR_UNSUPPORTED */
+                            the MSE is 0.  Like MSE, not built for SWIGLU with TTT_BF16 */
 } ttt_loss_kind;
 typedef enum {
   TTT_OPT_GD = 0,            /* U = G */

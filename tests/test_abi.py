@@ -127,14 +127,17 @@ def test_forward_state_checks_state_alignment_without_touching_the_gpu():
 
 
 @pytest.mark.parametrize("inner", ["linear", "mlp2_gelu", "swiglu"])
-def test_rmse_loss_runs_on_the_fp32_path_only(inner):
+def test_rmse_loss_is_built_where_mse_is(inner):
     from weight_sequence_mixing_b200 import binding
-    kw = dict(N=300, d=128, h=128, inner=inner, loss="rmse")
-    st, h = _create(binding.make_config(make_config(dtype="f32", **kw)))
-    assert st == 0, binding.status_string(st)
-    binding.LIB.ttt_destroy(h)
-    st, h = _create(binding.make_config(make_config(dtype="bf16", **kw)))
-    assert st == binding.TTT_ERR_UNSUPPORTED and not h.value
+    for dtype in ("f32", "bf16"):
+        for loss in ("mse", "rmse"):
+            st, h = _create(binding.make_config(make_config(N=300, d=128, h=128, inner=inner, loss=loss,
+                                                            dtype=dtype)))
+            if dtype == "bf16" and inner == "swiglu":
+                assert st == binding.TTT_ERR_UNSUPPORTED and not h.value
+            else:
+                assert st == 0, binding.status_string(st)
+                binding.LIB.ttt_destroy(h)
 
 
 def _dw(**kw):

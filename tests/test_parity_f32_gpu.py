@@ -43,19 +43,3 @@ def test_eta_scalar_and_single_head_edge():
     _check(compare(make_config(B=1, H=1, N=1, d=8, h=8, dtype="f32", inner="mlp2_gelu", loss="mse",
                                eta_mode="scalar", eta_scalar=0.7)))
 
-
-# RMSE inner loss (fp32 path only): the chunk's RMSE is reduced on the device first,
-# then scales the MSE gradient
-RMSE_CASES = [
-    dict(inner="linear", loss="rmse", opt="gd"),
-    dict(inner="mlp2_gelu", loss="rmse", opt="gd", key_instnorm=True, data="vit", eta_mode="scalar"),
-    dict(inner="swiglu", loss="rmse", opt="momentum_muon", chunk=70, weight_l2norm=True, Nq=33),
-    dict(inner="mlp2_gelu", loss="rmse", opt="momentum", chunk=50, causal=1),
-]
-
-
-@pytest.mark.parametrize("kw", RMSE_CASES, ids=lambda kw: "-".join(str(v) for v in kw.values()))
-def test_rmse_loss(kw):
-    base = dict(B=2, H=3, N=161, d=24, h=40, dtype="f32", data="lact", eta_mode="per_token", seed=83)
-    base.update(kw)
-    _check(compare(make_config(**base)))

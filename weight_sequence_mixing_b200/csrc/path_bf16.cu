@@ -384,6 +384,33 @@ __global__ void neg_eta_rows_kernel(int n, int Cp, int d, const bf16* V, int64_t
   }
 }
 
+// RMSE loss: the MSE gradient dY = 2 eta (V_hat - V) / (n d) is already in DY (bf16,
+// rows [0, n) of each z).  Per z, L = sqrt(sum eta (V_hat - V)^2 / (n d)), recovered from
+// dY as sqrt(sum_{eta != 0} dY^2 / eta * n d / 4); then dY <- dY / (2 L), the RMSE
+// gradient (zero where L = 0).  One CTA of 256 threads per z, fixed-order reduction.
+__global__ void rmse_scale_kernel(int n, int d, bf16* DY, int64_t y_zs, int t0, const float* eta, int64_t eta_zs,
+                                  float eta_scalar) {
+  __shared__ float red[256];
+  const int z = blockIdx.x;
+  bf16* y = DY + z * y_zs;
+  const int64_t total = int64_t(n) * d;
+  float s = 0.f;
+  for (int64_t i = threadIdx.x; i < total; i += blockDim.x) {
+    const float e = eta ? eta[z * eta_zs + t0 + int(i / d)] : eta_scalar;
+    const float v = __bfloat162float(y[i]);
+    if (e != 0.f) s += v * v / e;
+  }
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  const float L = sqrtf(fmaxf(red[0] * (float(n) * float(d) * 0.25f), 0.f));
+  const float scale = L > 0.f ? 0.5f / L : 0.f;
+  for (int64_t i = threadIdx.x; i < total; i += blockDim.x) y[i] = __float2bfloat16_rn(__bfloat162float(y[i]) * scale);
+}
+
 // ------------------------------------------------------------------ host helpers
 struct BView {
   uint8_t* base;
@@ -603,6 +630,16 @@ int grad_gemm(Ctx& c, const TM& a0, const TM& b0, const TM& a1, const TM& b1, in
   return grad_launch(c, a0, b0, a1, b1, rows0, rows1, b0k, b1k, ep);
 }
 
+// RMSE: rescale the chunk's MSE gradient in DY by 1/(2 RMSE) per head.
+int rmse_scale(Ctx& c, bf16* DY, int t0, int n) {
+  {
+    StageScope _sc(kStageKeyNorm, c.st);
+    rmse_scale_kernel<<<c.D.Z, 256, 0, c.st>>>(n, c.D.d, DY, int64_t(c.D.Cp) * c.D.d, t0, c.io.eta, c.D.N,
+                                               c.p.cfg.eta_scalar);
+  }
+  return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+
 // Token phase of the negative-dot update: activations H' and dZ(13) of chunk
 // tokens [t0, t0+n) for the weight-gradient GEMMs (token_phase.cuh).
 int token_phase(Ctx& c, const TM& tX, int xoff, int t0, int n, bf16* Hp, bf16* dZ, bool swiglu) {
@@ -722,6 +759,7 @@ int update_chunk(Ctx& c, int t0, int n) {
     if (bnd == 256) TRY((gemm<256, 0, false, false, 2, 4, 8>(tHk, c.tW2, tHk, c.tW2, g2, e2, status, c.st, true)));
     else if (bnd == 128) TRY((gemm<128, 0, false, false, 2, 4, 8>(tHk, c.tW2, tHk, c.tW2, g2, e2, status, c.st, true)));
     else TRY((gemm<64, 0, false, false, 2, 4, 8>(tHk, c.tW2, tHk, c.tW2, g2, e2, status, c.st, true)));
+    if (cfg.loss == TTT_LOSS_RMSE) TRY(rmse_scale(c, DY, t0, n));
     // dH = dY W2 -> dZ = dH G'
     TRY(tmap(&tY, DY, 2, d, Cp, Z, 128));
     EpiMulSaved e3{A1, A2, h, int64_t(Cp) * h};
@@ -734,7 +772,7 @@ int update_chunk(Ctx& c, int t0, int n) {
     TRY(tmap(&tD, A1, 2, h, Cp, Z, 64));
     TRY(grad_gemm(c, tH, tYmn, tD, *tXmn, h, h, h, 0, xoff));
   } else {  // linear
-    if (cfg.loss == TTT_LOSS_MSE) {
+    if (cfg.loss != TTT_LOSS_NEG_DOT) {  // MSE, RMSE
       EpiMseGrad e2{DY, d, n, int64_t(Cp) * d, V, int64_t(D.N) * d, t0, c.io.eta, D.N, cfg.eta_scalar,
                     2.0f / (float(n) * float(d))};
       TcGeom g2 = geom(mt, 0, d / bnd, d / 64, Z, 1);
@@ -742,6 +780,7 @@ int update_chunk(Ctx& c, int t0, int n) {
       if (bnd == 256) TRY((gemm<256, 0, false, false, 2, 4, 8>(*tX, c.tFirst, *tX, c.tFirst, g2, e2, status, c.st, true)));
       else if (bnd == 128) TRY((gemm<128, 0, false, false, 2, 4, 8>(*tX, c.tFirst, *tX, c.tFirst, g2, e2, status, c.st, true)));
       else TRY((gemm<64, 0, false, false, 2, 4, 8>(*tX, c.tFirst, *tX, c.tFirst, g2, e2, status, c.st, true)));
+      if (cfg.loss == TTT_LOSS_RMSE) TRY(rmse_scale(c, DY, t0, n));
     } else {
       {
         StageScope _sc(kStageKeyNorm, st);
@@ -839,8 +878,7 @@ void choose_grad_shape(const Plan& p, int Cp, int* splits, int* tile_rows, int* 
 int plan_layout_bf16(Plan* p) {
   const ttt_config& c = p->cfg;
   const int d = c.d, h = c.h;
-  // supported shapes and losses of the tensor-core path
-  if (c.loss == TTT_LOSS_RMSE) return TTT_ERR_UNSUPPORTED;
+  // supported shapes of the tensor-core path
   if (d % 64 != 0) return TTT_ERR_UNSUPPORTED;
   if (c.inner != TTT_INNER_LINEAR && h % 128 != 0) return TTT_ERR_UNSUPPORTED;
   if (c.inner == TTT_INNER_SWIGLU && c.loss != TTT_LOSS_NEG_DOT) return TTT_ERR_UNSUPPORTED;
@@ -855,7 +893,7 @@ int plan_layout_bf16(Plan* p) {
   const Dims D = dims_of(*p);
   const int64_t Z = D.Z, P = p->P, GR = D.GR, nm = int64_t(D.m) * D.n, mm = int64_t(D.m) * D.m;
   const int64_t ZK = Z * D.nmat;
-  const bool mlp_mse = c.inner == TTT_INNER_MLP2_GELU && c.loss == TTT_LOSS_MSE;
+  const bool mlp_mse = c.inner == TTT_INNER_MLP2_GELU && c.loss != TTT_LOSS_NEG_DOT;  // MSE, RMSE
   const bool act = c.inner != TTT_INNER_LINEAR;
   const int64_t bytes[kNumBBuf] = {
       Z * P * 4,
