@@ -28,9 +28,11 @@
  *   - Losses, summed over the chunk's tokens with the per-token learning rate eta_i:
  *        TTT_LOSS_MSE      L = sum_i eta_i ||F(k_i) - v_i||^2 / (n_chunk * d)
  *        TTT_LOSS_NEG_DOT  L = -sum_i eta_i <F(k_i), v_i>
+ *        TTT_LOSS_RMSE     L = sqrt(MSE)
  *   - One step per chunk (cfg.epochs steps when set; none with TTT_FLAG_NO_UPDATE):
  *     G -> [momentum M <- beta M + G] -> [Muon: Newton-Schulz]
- *     -> W <- W - lr U -> [each row of each matrix scaled to unit L2 norm].
+ *     -> W <- W - lr U -> [each row of each matrix scaled to unit L2 norm; for
+ *     DWCONV each channel's kernel].  TTT_FLAG_FIRST_LAYER_ONLY holds W2.
  *   - causal = 1 (needs Nq == N): per chunk, first O_c = F_W(Q_c), then update.
  *     causal = 0: update over every chunk in order, then O = F_{W*}(Q).
  *   - Nothing persists between calls: momentum starts at zero in every call.  A
