@@ -171,6 +171,19 @@ def test_dwconv_configurations_outside_the_built_set_are_rejected(bad, status):
     assert st == want and not h.value
 
 
+@pytest.mark.parametrize("d,ok", [(64, False), (192, False), (128, True), (256, True)])
+def test_bf16_linear_model_needs_whole_128_row_gradient_tiles(d, ok):
+    # d = 64 once divided by zero in the gradient-shape heuristic (a crash of ttt_create)
+    from weight_sequence_mixing_b200 import binding
+    st, h = _create(binding.make_config(make_config(N=500, d=d, inner="linear", dtype="bf16", loss="neg_dot")))
+    assert st == (0 if ok else binding.TTT_ERR_UNSUPPORTED)
+    if ok:
+        binding.LIB.ttt_destroy(h)
+    st, h = _create(binding.make_config(make_config(N=500, d=d, inner="linear", dtype="f32", loss="neg_dot")))
+    assert st == 0
+    binding.LIB.ttt_destroy(h)
+
+
 def test_forward_rejects_null_and_small_workspace_without_touching_the_gpu():
     from weight_sequence_mixing_b200 import binding
     st, h = _create(binding.make_config(make_config(N=16, d=64, h=128)))

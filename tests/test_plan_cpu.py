@@ -95,3 +95,74 @@ def test_workspace_grows_with_the_chunk_and_fits_the_static_scratch_when_small()
     a, _, _ = _sizes(make_config(B=1, H=2, N=4096, d=128, h=256, inner="swiglu", loss="neg_dot", dtype="bf16"))
     b, _, _ = _sizes(make_config(B=1, H=2, N=8192, d=128, h=256, inner="swiglu", loss="neg_dot", dtype="bf16"))
     assert b > a
+
+
+# ---------------------------------------------------------------- random configurations
+# Any configuration, valid or not, gets a defined status from ttt_create (host only), and
+# an accepted one has sizes that agree with their definitions.
+from hypothesis import HealthCheck, given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+_INNER = ["linear", "mlp2_gelu", "swiglu", "dwconv"]
+
+
+@st.composite
+def _configs(draw):
+    inner = draw(st.sampled_from(_INNER))
+    dtype = draw(st.sampled_from(["f32", "bf16"]))
+    d = draw(st.sampled_from([1, 8, 24, 64, 96, 128, 256, 512]))
+    h = draw(st.sampled_from([1, 40, 128, 256, 384, 1024]))
+    N = draw(st.integers(1, 1 << 20))
+    kw = dict(B=draw(st.integers(1, 8)), H=draw(st.integers(1, 8)), N=N, d=d, h=h, inner=inner, dtype=dtype,
+              loss=draw(st.sampled_from(["mse", "neg_dot", "rmse"])),
+              opt=draw(st.sampled_from(["gd", "momentum", "muon", "momentum_muon"])),
+              chunk=draw(st.sampled_from([0, 1, 64, 100, 2048, N, N + 5])),
+              causal=draw(st.sampled_from([0, 1])),
+              weight_l2norm=draw(st.booleans()), key_instnorm=draw(st.booleans()),
+              w0_per_batch=draw(st.booleans()), epochs=draw(st.integers(0, 3)))
+    kw["Nq"] = N if kw["causal"] or inner == "dwconv" else draw(st.integers(1, 5000))
+    if inner == "dwconv":
+        gh = draw(st.integers(1, 64))
+        kw.update(N=gh * draw(st.integers(1, 64)), grid_h=gh, ksize=draw(st.sampled_from([1, 2, 3, 5, 7, 9])))
+        kw["grid_w"] = kw["N"] // gh
+        kw["Nq"] = kw["N"]
+        kw["chunk"] = draw(st.sampled_from([0, kw["N"], 7]))
+    return make_config(**kw)
+
+
+@settings(max_examples=300, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(_configs())
+def test_random_configurations_get_a_status_and_consistent_sizes(cfg):
+    import ctypes
+
+    c = binding.make_config(cfg)
+    h = ctypes.c_void_p()
+    st_ = binding.LIB.ttt_create(ctypes.byref(c), ctypes.byref(h))
+    assert st_ in (binding.TTT_OK, binding.TTT_ERR_INVALID_ARG, binding.TTT_ERR_UNSUPPORTED)
+    if st_ != binding.TTT_OK:
+        assert not h.value
+        return
+    try:
+        d, hh, k = cfg["d"], cfg["h"], cfg["ksize"]
+        P = {"linear": d * d, "mlp2_gelu": 2 * d * hh, "swiglu": 3 * d * hh, "dwconv": d * k * k}[cfg["inner"]]
+        assert binding.LIB.ttt_param_count(h) == P
+        Z = cfg["B"] * cfg["H"]
+        mom = cfg["opt"] in ("momentum", "momentum_muon")
+        state = binding.LIB.ttt_state_size(h)
+        assert (state > 0) == mom and state % 4 == 0 and (state == 0 or state >= Z * P * 4)
+        es = 4 if cfg["dtype"] == "f32" else 2
+        io = (2 * Z * cfg["Nq"] * d * es + 2 * Z * cfg["N"] * d * es + Z * cfg["N"] * 4
+              + (Z if cfg["w0_per_batch"] else cfg["H"]) * P * 4 + Z * P * 4)
+        assert binding.LIB.ttt_host_staging_size(h) >= io
+        assert binding.LIB.ttt_workspace_size(h) >= 256 + Z * P * 4
+        buf = (ctypes.c_int * len(binding.PLAN_FIELDS))()
+        binding.LIB.ttt_plan_info(h, buf, len(binding.PLAN_FIELDS))
+        info = dict(zip(binding.PLAN_FIELDS, buf))
+        N, chunk = cfg["N"], cfg["chunk"]
+        assert info["chunk"] == (N if chunk <= 0 or chunk >= N else chunk)
+        assert info["nchunks"] == -(-N // info["chunk"])
+        assert info["path"] == (2 if cfg["inner"] == "dwconv" else 0 if cfg["dtype"] == "f32" else 1)
+        if info["path"] == 1:
+            assert info["splits"] >= 1 and info["tile_rows"] in (128, 256, 512) and info["grad_bn"] in (32, 64, 128, 256)
+    finally:
+        binding.LIB.ttt_destroy(h)

@@ -862,7 +862,7 @@ void choose_grad_shape(const Plan& p, int Cp, int* splits, int* tile_rows, int* 
   const int units = *tile_rows == 512 ? 74 : 148;  // tiles that run at once
   const int tiles = rows / *tile_rows * (d / bnd) * p.BH;
   // about two waves of tiles: long K ranges per split, few partials to reduce
-  int s = std::max(1, (2 * units + tiles / 2) / tiles);
+  int s = tiles > 0 ? std::max(1, (2 * units + tiles / 2) / tiles) : 1;
   s = std::min(s, smax);
   const int per = (kblocks + s - 1) / s;  // every split owns at least one k-block
   *splits = (kblocks + per - 1) / per;
@@ -881,6 +881,9 @@ int plan_layout_bf16(Plan* p) {
   // supported shapes of the tensor-core path
   if (d % 64 != 0) return TTT_ERR_UNSUPPORTED;
   if (c.inner != TTT_INNER_LINEAR && h % 128 != 0) return TTT_ERR_UNSUPPORTED;
+  // the weight-gradient GEMMs tile their output rows (h per matrix, d for the linear
+  // model) by 128
+  if (c.inner == TTT_INNER_LINEAR && d % 128 != 0) return TTT_ERR_UNSUPPORTED;
   if (c.inner == TTT_INNER_SWIGLU && c.loss != TTT_LOSS_NEG_DOT) return TTT_ERR_UNSUPPORTED;
   const bool muon = c.opt == TTT_OPT_MUON || c.opt == TTT_OPT_MOMENTUM_MUON;
   if (muon && (d % 128 != 0 || (c.inner != TTT_INNER_LINEAR && h % 128 != 0))) return TTT_ERR_UNSUPPORTED;
