@@ -112,7 +112,7 @@ def _configs(draw):
     dtype = draw(st.sampled_from(["f32", "bf16"]))
     d = draw(st.sampled_from([1, 8, 24, 64, 96, 128, 256, 512]))
     h = draw(st.sampled_from([1, 40, 128, 256, 384, 1024]))
-    N = draw(st.integers(1, 1 << 20))
+    N = draw(st.one_of(st.integers(1, 1 << 20), st.integers((1 << 30) - 300, (1 << 31) - 1)))
     kw = dict(B=draw(st.integers(1, 8)), H=draw(st.integers(1, 8)), N=N, d=d, h=h, inner=inner, dtype=dtype,
               loss=draw(st.sampled_from(["mse", "neg_dot", "rmse"])),
               opt=draw(st.sampled_from(["gd", "momentum", "muon", "momentum_muon"])),
@@ -139,6 +139,8 @@ def test_random_configurations_get_a_status_and_consistent_sizes(cfg):
     h = ctypes.c_void_p()
     st_ = binding.LIB.ttt_create(ctypes.byref(c), ctypes.byref(h))
     assert st_ in (binding.TTT_OK, binding.TTT_ERR_INVALID_ARG, binding.TTT_ERR_UNSUPPORTED)
+    if max(cfg["N"], cfg["Nq"]) > (1 << 30):
+        assert st_ != binding.TTT_OK
     if st_ != binding.TTT_OK:
         assert not h.value
         return

@@ -38,6 +38,9 @@ int plan_build(const ttt_config& c, Plan* p) {
   for (float v : c.ns_coeff)
     if (!std::isfinite(v)) return TTT_ERR_INVALID_ARG;
   if (static_cast<int64_t>(c.B) * c.H > 65535) return TTT_ERR_UNSUPPORTED;
+  // token counts: 2^30 keys of even 64 bf16 channels already outgrow HBM; the bound keeps
+  // every padded token count inside int32
+  if (c.N > (1 << 30) || c.Nq > (1 << 30)) return TTT_ERR_UNSUPPORTED;
   if (c.d > 4096 || ((c.inner == TTT_INNER_MLP2_GELU || c.inner == TTT_INNER_SWIGLU) && c.h > 16384))
     return TTT_ERR_UNSUPPORTED;
 
@@ -49,7 +52,7 @@ int plan_build(const ttt_config& c, Plan* p) {
             : c.inner == TTT_INNER_LINEAR ? d * d : c.inner == TTT_INNER_MLP2_GELU ? 2 * d * h : 3 * d * h;
   p->BH = c.B * c.H;
   p->chunk = (c.chunk <= 0 || c.chunk >= c.N) ? c.N : c.chunk;
-  p->nchunks = (c.N + p->chunk - 1) / p->chunk;
+  p->nchunks = static_cast<int>((static_cast<int64_t>(c.N) + p->chunk - 1) / p->chunk);
   p->path = dw ? kPathDwconv : c.dtype == TTT_F32 ? kPathF32 : kPathBf16;
 
   // host staging: inputs then outputs, each 256-byte aligned
