@@ -771,3 +771,71 @@ def test_dwconv_layer_reads_the_grid_once_as_one_chunk():
     G = orc.dwconv_weight_grad(K, -V, (gh, gw), 3)
     assert np.allclose(w, w0 - G.reshape(-1), rtol=1e-13, atol=1e-13)
     assert np.allclose(O, _brute_dwconv(w.reshape(d, 9), Q, gh, gw, 3), rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------- the same identities on drawn shapes
+from hypothesis import given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+@settings(max_examples=60, deadline=None)
+@given(d=st.integers(1, 7), n=st.integers(1, 30), chunk=st.integers(0, 35), causal=st.booleans(),
+       seed=st.integers(0, 2**31 - 1))
+def test_linear_dot_is_chunkwise_linear_attention_on_drawn_shapes(d, n, chunk, causal, seed):
+    # W_c = W0 + sum of eta_i v_i k_i^T over the tokens of the chunks before c (causal reads),
+    # or over all tokens (non-causal), accumulated one outer product at a time
+    rng = np.random.default_rng(seed)
+    Q, K, V = rng.standard_normal((n, d)), rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    eta, W0 = np.abs(rng.standard_normal(n)), rng.standard_normal((d, d))
+    cfg = cfg_for("linear", "neg_dot", d=d, h=d, N=n, chunk=chunk, causal=int(causal))
+    O, Ws = orc.forward_head(cfg, Q, K, V, eta, W0.reshape(-1))
+    C = n if chunk <= 0 or chunk >= n else chunk
+    W = W0.copy()
+    Oref = np.zeros((n, d))
+    for s in range(0, n, C):
+        if causal:
+            Oref[s:s + C] = Q[s:s + C] @ W.T
+        for i in range(s, min(s + C, n)):
+            W += eta[i] * np.outer(V[i], K[i])
+    if not causal:
+        Oref = Q @ W.T
+    assert np.allclose(Ws.reshape(d, d), W, rtol=1e-11, atol=1e-11)
+    assert np.allclose(O, Oref, rtol=1e-11, atol=1e-11)
+
+
+@settings(max_examples=40, deadline=None)
+@given(d=st.integers(1, 5), n=st.integers(1, 12), opt=st.sampled_from(["gd", "momentum", "muon", "momentum_muon"]),
+       chunk=st.integers(0, 14), causal=st.booleans(), rownorm=st.booleans(), seed=st.integers(0, 2**31 - 1))
+def test_glu_is_a_swiglu_with_identity_w2_on_drawn_shapes(d, n, opt, chunk, causal, rownorm, seed):
+    rng = np.random.default_rng(seed)
+    Wg = {"Wa": rng.standard_normal((d, d)) * 0.5, "Wb": rng.standard_normal((d, d)) * 0.5}
+    Q, K, V = rng.standard_normal((n, d)), rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    eta = np.abs(rng.standard_normal(n)) + 0.1
+    cfg = cfg_for("glu", "neg_dot", opt=opt, weight_l2norm=rownorm, d=d, h=d, N=n, chunk=chunk, causal=int(causal),
+                  ns_iters=2)
+    Og, wg = orc.forward_head(cfg, Q, K, V, eta, orc.pack("glu", d, d, Wg))
+    Ws0 = {"W1": Wg["Wb"], "W3": Wg["Wa"], "W2": np.eye(d)}
+    Os, ws = orc.forward_head(dict(cfg, inner="swiglu", first_layer_only=True), Q, K, V, eta,
+                              orc.pack("swiglu", d, d, Ws0))
+    Wgs, Wss = orc.unpack("glu", d, d, wg), orc.unpack("swiglu", d, d, ws)
+    assert np.allclose(Og, Os, rtol=1e-10, atol=1e-10)
+    assert np.allclose(Wss["W1"], Wgs["Wb"], rtol=1e-10, atol=1e-10)
+    assert np.allclose(Wss["W3"], Wgs["Wa"], rtol=1e-10, atol=1e-10)
+
+
+@settings(max_examples=40, deadline=None)
+@given(gh=st.integers(1, 9), gw=st.integers(1, 9), d=st.integers(1, 4), k=st.sampled_from([1, 3, 5, 7]),
+       seed=st.integers(0, 2**31 - 1))
+def test_dwconv_matches_scipy_correlate2d_on_drawn_shapes(gh, gw, d, k, seed):
+    from scipy.signal import correlate2d
+
+    rng = np.random.default_rng(seed)
+    Wc, X, dY = rng.standard_normal((d, k * k)), rng.standard_normal((gh * gw, d)), rng.standard_normal((gh * gw, d))
+    Y = orc.dwconv_apply(Wc, X, (gh, gw))
+    G = orc.dwconv_weight_grad(X, dY, (gh, gw), k)
+    for c in range(d):
+        Xc = X[:, c].reshape(gh, gw)
+        ref = correlate2d(Xc, Wc[c].reshape(k, k), mode="same", boundary="fill", fillvalue=0.0)
+        assert np.allclose(Y[:, c].reshape(gh, gw), ref, rtol=1e-12, atol=1e-12)
+        gref = correlate2d(np.pad(Xc, k // 2), dY[:, c].reshape(gh, gw), mode="valid")
+        assert np.allclose(G[c].reshape(k, k), gref, rtol=1e-12, atol=1e-12)
