@@ -228,3 +228,34 @@ def test_binding_config_struct_matches_the_c_header(tmp_path, repo_root):
     out = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
     assert out[0] == ctypes.sizeof(binding.TTTConfig)
     assert out[1:] == [getattr(binding.TTTConfig, n).offset for n in names]
+
+
+def test_binding_refuses_buffers_of_the_wrong_size_dtype_or_place():
+    # the library reads and writes buffers by the configured sizes: the binding checks them first
+    import torch
+
+    from weight_sequence_mixing_b200 import binding
+    cfg = make_config(B=2, H=3, N=40, Nq=24, d=64, h=128, inner="swiglu", loss="neg_dot", dtype="bf16",
+                      eta_mode="per_token")
+    layer = binding.TTTLayer(cfg, device="cpu")
+    P = layer.P
+    ok = dict(Q=torch.zeros(2, 3, 24, 64, dtype=torch.bfloat16), K=torch.zeros(2, 3, 40, 64, dtype=torch.bfloat16),
+              V=torch.zeros(2, 3, 40, 64, dtype=torch.bfloat16), eta=torch.zeros(2, 3, 40),
+              W0=torch.zeros(3, P), O=torch.zeros(2, 3, 24, 64, dtype=torch.bfloat16), W_out=torch.zeros(2, 3, P))
+    layer.check_buffers("cpu", **ok)  # right sizes on the host: accepted
+    layer.check_buffers("cpu", **dict(ok, eta=None, W_out=None))
+    bad = [dict(K=torch.zeros(2, 3, 39, 64, dtype=torch.bfloat16)), dict(Q=torch.zeros(2, 3, 24, 64)),
+           dict(eta=torch.zeros(2, 3, 40, dtype=torch.float64)), dict(W0=torch.zeros(2, 3, P)),
+           dict(O=torch.zeros(2, 3, 64, 24, dtype=torch.bfloat16).transpose(2, 3)), dict(V=None)]
+    for b in bad:
+        with pytest.raises(ValueError):
+            layer.check_buffers("cpu", **dict(ok, **b))
+    with pytest.raises(ValueError):
+        layer.check_buffers("cuda", **ok)  # host tensors where device memory is expected
+    layer.close()
+    # one state per batch entry: W0 is [B, H, P]
+    per = binding.TTTLayer(dict(cfg, w0_per_batch=True), device="cpu")
+    per.check_buffers("cpu", **dict(ok, W0=torch.zeros(2, 3, P)))
+    with pytest.raises(ValueError):
+        per.check_buffers("cpu", **ok)
+    per.close()

@@ -183,6 +183,28 @@ class TTTLayer:
     def io_dtype(self):
         return torch.float32 if self.cfg["dtype"] == "f32" else torch.bfloat16
 
+    def check_buffers(self, device_type: str, **bufs):
+        """Element counts, dtypes and layout of a call's buffers: the library reads and
+        writes them by the configured sizes, so a short buffer is refused here."""
+        c = self.cfg
+        BH = c["B"] * c["H"]
+        q = BH * c["Nq"] * c["d"]
+        kv = BH * c["N"] * c["d"]
+        want = {"Q": (q, self.io_dtype), "K": (kv, self.io_dtype), "V": (kv, self.io_dtype),
+                "eta": (BH * c["N"], torch.float32),
+                "W0": ((BH if c.get("w0_per_batch") else c["H"]) * self.P, torch.float32),
+                "O": (q, self.io_dtype), "W_out": (BH * self.P, torch.float32)}
+        for name, t in bufs.items():
+            if t is None:
+                if name in ("Q", "K", "V", "W0", "O"):
+                    raise ValueError(f"{name} is required")
+                continue
+            n, dt = want[name]
+            if t.numel() != n or t.dtype != dt:
+                raise ValueError(f"{name}: expected {n} elements of {dt}, got shape {tuple(t.shape)} of {t.dtype}")
+            if not t.is_contiguous() or t.device.type != device_type:
+                raise ValueError(f"{name}: must be a contiguous {device_type} tensor")
+
     def forward(self, Q, K, V, eta, W0, O=None, W_out=None, stream=None, check=True):
         """Enqueue the layer on `stream`; returns (O, W_out).  With check=True the
         stream is synchronised and the device status word is checked."""
@@ -191,9 +213,7 @@ class TTTLayer:
             O = torch.empty((c["B"], c["H"], c["Nq"], c["d"]), dtype=self.io_dtype, device=self.device)
         if W_out is None:
             W_out = torch.empty((c["B"], c["H"], self.P), dtype=torch.float32, device=self.device)
-        for t in (Q, K, V, W0, O, W_out) + ((eta,) if eta is not None else ()):
-            if not t.is_contiguous() or t.device.type != "cuda":
-                raise ValueError("tensors must be contiguous CUDA tensors")
+        self.check_buffers("cuda", Q=Q, K=K, V=V, eta=eta, W0=W0, O=O, W_out=W_out)
         st = _stream_ptr(stream)
         _check(LIB.ttt_forward(self._handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W0), _ptr(O), _ptr(W_out),
                                _ptr(self.workspace), self.workspace.numel(), st), "ttt_forward")
@@ -219,9 +239,10 @@ class TTTLayer:
             O = torch.empty((c["B"], c["H"], c["Nq"], c["d"]), dtype=self.io_dtype, device=self.device)
         if W_out is None:
             W_out = torch.empty((c["B"], c["H"], self.P), dtype=torch.float32, device=self.device)
+        self.check_buffers("cuda", Q=Q, K=K, V=V, eta=eta, W0=W0, O=O, W_out=W_out)
         for t in (state_in, state_out):
-            if t is not None and t.numel() * t.element_size() < self.state_size:
-                raise ValueError("state buffer smaller than state_size")
+            if t is not None and (t.numel() * t.element_size() < self.state_size or t.device.type != "cuda"):
+                raise ValueError("state buffer smaller than state_size or not on the GPU")
         st = _stream_ptr(stream)
         _check(LIB.ttt_forward_state(self._handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W0), _ptr(O),
                                      _ptr(W_out), _ptr(state_in), _ptr(state_out), _ptr(self.workspace),
@@ -236,6 +257,7 @@ class TTTLayer:
     def forward_noalloc(self, Q, K, V, eta, W0, O, W_out=None, status=None, stream=None):
         """The layer without a workspace argument: the library's own static device
         scratch stands in for it (for callers that cannot allocate; see ttt.h)."""
+        self.check_buffers("cuda", Q=Q, K=K, V=V, eta=eta, W0=W0, O=O, W_out=W_out)
         _check(LIB.ttt_forward_noalloc(self._handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W0), _ptr(O),
                                        _ptr(W_out), _ptr(status), _stream_ptr(stream)), "ttt_forward_noalloc")
 
@@ -259,6 +281,9 @@ class TTTLayer:
 
     def forward_host(self, Q, K, V, eta, W0, O, W_out, staging, stream=None):
         """Host (ideally pinned) CPU tensors in and out; enqueued on `stream`."""
+        self.check_buffers("cpu", Q=Q, K=K, V=V, eta=eta, W0=W0, O=O, W_out=W_out)
+        if staging.numel() < int(LIB.ttt_host_staging_size(self._handle)) or staging.device.type != "cuda":
+            raise ValueError("staging must be a device buffer of at least ttt_host_staging_size bytes")
         st = _stream_ptr(stream)
         _check(LIB.ttt_forward_host(self._handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W0), _ptr(O),
                                     _ptr(W_out), _ptr(staging), staging.numel(), _ptr(self.workspace),
