@@ -778,7 +778,7 @@ from hypothesis import given, settings  # noqa: E402
 from hypothesis import strategies as st  # noqa: E402
 
 
-@settings(max_examples=60, deadline=None)
+@settings(max_examples=60, deadline=None, derandomize=True)
 @given(d=st.integers(1, 7), n=st.integers(1, 30), chunk=st.integers(0, 35), causal=st.booleans(),
        seed=st.integers(0, 2**31 - 1))
 def test_linear_dot_is_chunkwise_linear_attention_on_drawn_shapes(d, n, chunk, causal, seed):
@@ -803,7 +803,7 @@ def test_linear_dot_is_chunkwise_linear_attention_on_drawn_shapes(d, n, chunk, c
     assert np.allclose(O, Oref, rtol=1e-11, atol=1e-11)
 
 
-@settings(max_examples=40, deadline=None)
+@settings(max_examples=40, deadline=None, derandomize=True)
 @given(d=st.integers(1, 5), n=st.integers(1, 12), opt=st.sampled_from(["gd", "momentum", "muon", "momentum_muon"]),
        chunk=st.integers(0, 14), causal=st.booleans(), rownorm=st.booleans(), seed=st.integers(0, 2**31 - 1))
 def test_glu_is_a_swiglu_with_identity_w2_on_drawn_shapes(d, n, opt, chunk, causal, rownorm, seed):
@@ -823,7 +823,7 @@ def test_glu_is_a_swiglu_with_identity_w2_on_drawn_shapes(d, n, opt, chunk, caus
     assert np.allclose(Wss["W3"], Wgs["Wa"], rtol=1e-10, atol=1e-10)
 
 
-@settings(max_examples=40, deadline=None)
+@settings(max_examples=40, deadline=None, derandomize=True)
 @given(gh=st.integers(1, 9), gw=st.integers(1, 9), d=st.integers(1, 4), k=st.sampled_from([1, 3, 5, 7]),
        seed=st.integers(0, 2**31 - 1))
 def test_dwconv_matches_scipy_correlate2d_on_drawn_shapes(gh, gw, d, k, seed):

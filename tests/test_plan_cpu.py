@@ -130,7 +130,7 @@ def _configs(draw):
     return make_config(**kw)
 
 
-@settings(max_examples=300, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@settings(max_examples=300, deadline=None, derandomize=True, suppress_health_check=[HealthCheck.too_slow])
 @given(_configs())
 def test_random_configurations_get_a_status_and_consistent_sizes(cfg):
     import ctypes
