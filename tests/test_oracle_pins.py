@@ -839,3 +839,25 @@ def test_dwconv_matches_scipy_correlate2d_on_drawn_shapes(gh, gw, d, k, seed):
         assert np.allclose(Y[:, c].reshape(gh, gw), ref, rtol=1e-12, atol=1e-12)
         gref = correlate2d(np.pad(Xc, k // 2), dY[:, c].reshape(gh, gw), mode="valid")
         assert np.allclose(G[c].reshape(k, k), gref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("name", ["neg_dot", "mse"])
+def test_hand_worked_dwconv_example(repo_root, name):
+    g = json.load(open(os.path.join(repo_root, "tests", "golden", "dwconv_row_of_three.json")))
+    gh, gw = g["grid"]
+    col = lambda key: np.array(g[key], float)[:, None]  # one channel
+    cfg = cfg_for("dwconv", name, d=1, h=1, N=gh * gw, grid_h=gh, grid_w=gw, ksize=g["ksize"])
+    O, Ws = orc.forward_head(cfg, col("Q"), col("K"), col("V"), np.array(g["eta"], float), np.array(g["W0"], float))
+    case = g["cases"][name]
+    assert np.allclose(Ws, np.array(case["W_star"]), rtol=0, atol=1e-14)
+    assert np.allclose(O[:, 0], np.array(case["O"]), rtol=0, atol=1e-14)
+
+
+def test_hand_worked_glu_example(repo_root):
+    g = json.load(open(os.path.join(repo_root, "tests", "golden", "glu_two_tokens.json")))
+    col = lambda key: np.array(g[key], float)[:, None]
+    cfg = cfg_for("glu", "neg_dot", d=1, h=1, N=2, Nq=1)
+    O, Ws = orc.forward_head(cfg, col("q"), col("K"), col("V"), np.array(g["eta"], float),
+                             np.array([g["Wa0"], g["Wb0"]], float))
+    assert np.allclose(Ws, [g["Wa_star"], g["Wb_star"]], rtol=0, atol=1e-14)
+    assert abs(O[0, 0] - 14.0 / (1.0 + math.exp(-7.0))) < 1e-13 and abs(O[0, 0] - g["O"]) < 1e-13
