@@ -193,7 +193,7 @@ def test_linear_mse_eta_is_a_rescaling_of_k_and_v():
     assert np.allclose(O1, O2, rtol=1e-12, atol=1e-12)
 
 
-@pytest.mark.parametrize("name", ["neg_dot", "mse"])
+@pytest.mark.parametrize("name", ["neg_dot", "mse", "rmse"])
 def test_hand_worked_linear_example(repo_root, name):
     g = json.load(open(os.path.join(repo_root, "tests", "golden", "linear_two_tokens.json")))
     d = g["d"]
