@@ -80,3 +80,14 @@ def test_lact_w0_fan_in_scale():
 def test_scene_workload_has_a_partial_last_chunk():
     cfg = workload("lact_scene_n1m_c131k")
     assert cfg["N"] == 7 * 131072 + 111616 and cfg["chunk"] == 131072
+
+
+@pytest.mark.parametrize("kind,k", [("glu", 3), ("dwconv", 1), ("dwconv", 3), ("dwconv", 7)])
+def test_packing_of_the_ablation_inner_models(kind, k):
+    # GLU: [Wa (d x d) | Wb (d x d)]; DWConv: [Wc (d x k*k)]; W0 has one row of P per head
+    cfg = make_config(B=1, H=3, N=20, d=8, h=8, inner=kind, ksize=k, grid_h=4, grid_w=5)
+    P = 2 * 8 * 8 if kind == "glu" else 8 * k * k
+    assert param_count(cfg) == P
+    W0 = gen_w0(cfg)
+    assert W0.shape == (3, P) and torch.isfinite(W0).all()
+    assert not torch.equal(W0[0], W0[1])  # each head draws its own weights
