@@ -41,7 +41,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # tokens per reference-arm step (bounded CPU sample) and per CPU-baseline sample
 CPU_SAMPLE_TOKENS = {
     "tiny_mlp2_n196_fp32": 196, "vit3s_1248_mlp2_n6084": 6084, "lact_lm_causal_n32k_c2048": 16384,
-    "lact_nvs_n196k_d512": 65536, "lact_scene_n1m_c131k": 65536,
+    "lact_nvs_n196k_d512": 65536, "lact_scene_n1m_c131k": 65536, "vit3s_1248_dwconv_n6084": 8 * 6084,
 }
 
 
@@ -51,6 +51,12 @@ def algorithmic_flops(cfg) -> dict:
     B, H, N, Nq, d, h = cfg["B"], cfg["H"], cfg["N"], cfg["Nq"], cfg["d"], cfg["h"]
     BH = B * H
     kind, loss = cfg["inner"], cfg["loss"]
+    ep = max(1, int(cfg.get("epochs", 1)))  # full-batch steps per chunk
+    if kind == "dwconv":  # k*k taps per (token, channel): gradient (and the MSE forward), apply
+        kk = cfg["ksize"] ** 2
+        return {"token_phase": 0.0, "newton_schulz": 0.0,
+                "weight_grad": float(BH) * N * 2 * kk * d * (2 if loss in ("mse", "rmse") else 1) * ep,
+                "apply": float(BH) * Nq * 2 * kk * d}
     if kind == "swiglu":  # token phase: Z1, Z3, V W2; weight grads: G2, G1, G3
         tok, grad, app = 6 * d * h, 6 * d * h, 6 * d * h
     elif kind == "mlp2_gelu":  # token phase: Z, [V_hat], dH; grads: G2, G1
@@ -65,13 +71,22 @@ def algorithmic_flops(cfg) -> dict:
         for _, r, c in matrix_shapes(cfg):
             m, n = min(r, c), max(r, c)
             ns += cfg["ns_iters"] * (4 * m * m * n + 2 * m ** 3)
-    ep = max(1, int(cfg.get("epochs", 1)))  # full-batch steps per chunk
     return {
         "token_phase": float(BH) * N * tok * ep,
         "weight_grad": float(BH) * N * grad * ep,
         "newton_schulz": float(BH) * nchunks * ns * ep,
         "apply": float(BH) * Nq * app,
     }
+
+
+def algorithmic_bytes(cfg) -> dict:
+    """HBM bytes per stage of a bandwidth-bound path (DWConv): every input read once and
+    every output written once.  Tap gradients: K and V (and eta); apply: Q in, O out."""
+    es = 4 if cfg["dtype"] == "f32" else 2
+    BH, N, Nq, d = cfg["B"] * cfg["H"], cfg["N"], cfg["Nq"], cfg["d"]
+    ep = max(1, int(cfg.get("epochs", 1)))
+    eta = 4 * N if cfg["eta_mode"] == "per_token" else 0
+    return {"weight_grad": float(BH) * (2 * N * d * es + eta) * ep, "apply": float(BH) * 2 * Nq * d * es}
 
 
 def io_bytes(cfg) -> tuple[int, int]:
@@ -186,9 +201,13 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------- CPU oracle timing
 def cpu_sample_config(cfg, tokens):
-    """The workload cut to its first `tokens` key/value tokens (one update), Nq scaled alike."""
+    """The workload cut to its first `tokens` key/value tokens (one update), Nq scaled alike;
+    a DWConv layer keeps whole grids and is cut to its first tokens // N batch entries."""
     import copy
     s = copy.deepcopy(cfg)
+    if cfg["inner"] == "dwconv":
+        s["B"] = max(1, min(cfg["B"], tokens // cfg["N"]))
+        return s
     S = min(tokens, cfg["N"])
     s["N"] = S
     s["Nq"] = S if cfg["causal"] else max(1, round(cfg["Nq"] * S / cfg["N"]))
@@ -217,9 +236,15 @@ def time_oracle(cfg, tokens, reps=1):
         t0 = time.perf_counter()
         oracle.forward(s, x["Q"], x["K"], x["V"], x["eta"], x["W0"])
         times.append(time.perf_counter() - t0)
-    sample = (f"first {s['N']} of {cfg['N']} tokens of all {cfg['B'] * cfg['H']} heads, Nq {s['Nq']}, "
-              f"chunk {s['chunk'] or s['N']}, fp64 numpy oracle")
-    return s, times, sample
+    return s, times, sample_text(cfg, s)
+
+
+def sample_text(cfg, s) -> str:
+    if cfg["inner"] == "dwconv":
+        return (f"{s['B']} of {cfg['B']} batch entries (whole {cfg['grid_h']}x{cfg['grid_w']} grids), "
+                f"fp64 numpy oracle")
+    return (f"first {s['N']} of {cfg['N']} tokens of all {cfg['B'] * cfg['H']} heads, Nq {s['Nq']}, "
+            f"chunk {s['chunk'] or s['N']}, fp64 numpy oracle")
 
 
 # ---------------------------------------------------------------------------- main
@@ -355,6 +380,18 @@ def main():
     burst = bool(clocks) and clocks["sm_mhz"] >= 0.95 * clocks["sm_max_mhz"]
     peak_key = "bf16_tflops" if burst else "bf16_tflops_sustained"
     roof = None
+    if cfg["inner"] == "dwconv":  # SIMT and bandwidth-bound: the roofline is HBM, not the tensor pipe
+        nbytes = algorithmic_bytes(cfg)
+        dom = max((n for n in stages if nbytes.get(n, 0) > 0), key=lambda n: stages[n][0], default=None)
+        if dom:
+            ms, cnt = stages[dom]
+            per_launch = nbytes[dom] * args.steps / cnt
+            achieved = per_launch / (ms / cnt / 1e3) / 1e9
+            peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+            roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                    "frac": achieved / peak, "traffic": measured_traffic(args.workload, dom),
+                    "bytes_per_launch": per_launch, "launches": cnt, "peak_source": f"{peak_src} HBM copy bandwidth"}
+        dom = None
     if dom:
         ms, cnt = stages[dom]
         per_launch = flops[dom] * args.steps / cnt
@@ -469,8 +506,7 @@ def run_reference(args, cfg, world):
         times.append(time.perf_counter() - t0)
     total = sum(times)
     value = s["B"] * s["N"] * args.steps / total
-    sample = (f"first {s['N']} of {cfg['N']} tokens of all {cfg['B'] * cfg['H']} heads, Nq {s['Nq']}, "
-              f"chunk {s['chunk'] or s['N']}, fp64 numpy oracle")
+    sample = sample_text(cfg, s)
     line = {
         "impl": "reference",
         "metric": METRIC,

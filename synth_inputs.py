@@ -78,6 +78,11 @@ WORKLOADS = {
                                  inner="swiglu", loss="neg_dot", opt="momentum_muon", momentum=0.9,
                                  dtype="bf16", weight_l2norm=True, eta_mode="per_token",
                                  data="lact", seed=5000),
+    # the DWConv head of a ViT^3-S-like 1248^2 layer: B8, one head, the 78 x 78 token grid,
+    # d64, 3 x 3 depthwise kernels, the ViT^3 recipe (dot loss, one full-batch step, eta = 1)
+    "vit3s_1248_dwconv_n6084": dict(B=8, H=1, N=6084, grid_h=78, grid_w=78, ksize=3, d=64, h=64,
+                                    inner="dwconv", loss="neg_dot", opt="gd", dtype="bf16",
+                                    eta_mode="scalar", eta_scalar=1.0, data="vit", seed=6000),
 }
 
 
