@@ -27,9 +27,9 @@ int ttt_selftest_gemm(int elem_bytes, int a_mn, int b_mn, int bn, int M, int N, 
 
 /* The execution plan ttt_create chose (host logic only, no GPU needed).  Writes up to
  * `n` ints into `info`, in this order:
- *   [0] path: 0 fp32 SIMT, 1 bf16 tensor cores
+ *   [0] path: 0 fp32 SIMT, 1 bf16 tensor cores, 2 DWConv (SIMT, either dtype)
  *   [1] chunk length in tokens, [2] number of chunks
- *   [3] split-K splits of the weight-gradient reductions (bf16 path; 0 on fp32)
+ *   [3] split-K splits of the weight-gradient reductions (bf16 path; 0 on the others)
  *   [4] rows per weight-gradient tile: 128 or 256 on single CTAs, 512 on CTA pairs
  *   [5] output columns per weight-gradient tile
  *   [6] 1 when unsplit reductions write U (and momentum) directly, without partials
