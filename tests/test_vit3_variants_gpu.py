@@ -119,6 +119,13 @@ def test_dwconv_against_the_oracle(kw):
     _check(compare(cfg), TOL[cfg["dtype"]])
 
 
+def test_dwconv_bench_workload_at_full_size():
+    # the workload bench.py times (B8, a 78 x 78 grid, d64), in its launch configuration
+    from synth_inputs import workload
+
+    _check(compare(workload("vit3s_1248_dwconv_n6084")), TOL["bf16"])
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_dwconv_state_handed_on_equals_more_epochs(dtype):
     # two calls of one step each, (W, M) handed on, equal one call of two steps
