@@ -260,3 +260,42 @@ def test_binding_refuses_buffers_of_the_wrong_size_dtype_or_place():
     with pytest.raises(ValueError):
         per.check_buffers("cpu", **ok)
     per.close()
+
+
+def test_every_entry_point_refuses_a_null_handle_or_buffer_without_gpu_work():
+    import ctypes
+
+    from weight_sequence_mixing_b200 import binding
+    lib = binding.LIB
+    inv = binding.TTT_ERR_INVALID_ARG
+    fake = ctypes.c_void_p(4096)
+    assert lib.ttt_create(None, None) == inv
+    out = ctypes.c_void_p(1234)
+    assert lib.ttt_create(None, ctypes.byref(out)) == inv and not out.value  # *out cleared
+    assert lib.ttt_param_count(None) == 0 and lib.ttt_workspace_size(None) == 0
+    assert lib.ttt_state_size(None) == 0 and lib.ttt_host_staging_size(None) == 0
+    assert lib.ttt_launch_count(None) == 0
+    assert lib.ttt_forward(None, fake, fake, fake, None, fake, fake, None, fake, 1 << 30, None) == inv
+    assert lib.ttt_forward_state(None, fake, fake, fake, None, fake, fake, None, None, None, fake, 1 << 30,
+                                 None) == inv
+    assert lib.ttt_forward_host(None, fake, fake, fake, None, fake, fake, None, fake, 1 << 30, fake, 1 << 30,
+                                None) == inv
+    assert lib.ttt_forward_noalloc(None, fake, fake, fake, None, fake, fake, None, None, None) == inv
+    assert lib.ttt_query_status(None, fake, None) == inv
+    assert lib.ttt_profile_enable(None, 1) == inv
+    ms, cnt = (ctypes.c_float * 8)(), (ctypes.c_int * 8)()
+    assert lib.ttt_profile_collect(None, 8, ms, cnt) == inv
+    info = (ctypes.c_int * 7)()
+    assert lib.ttt_plan_info(None, info, 7) == inv
+    assert lib.ttt_selftest_timeout(None, None) == inv
+    assert lib.ttt_selftest_gemm(2, 0, 0, 64, 128, 64, 64, 1, 1, None, fake, fake, None) == inv
+    lib.ttt_destroy(None)  # a no-op
+    assert lib.ttt_stage_name(99) == b"unknown"
+    # a real handle: null outputs and a null workspace are refused too
+    st, h = _create(binding.make_config(make_config(N=16, d=64, h=128)))
+    assert st == 0
+    assert lib.ttt_query_status(h, None, None) == inv
+    assert lib.ttt_profile_collect(h, 0, ms, cnt) == inv and lib.ttt_plan_info(h, None, 7) == inv
+    assert lib.ttt_forward_host(h, fake, fake, fake, None, fake, None, None, fake, 1 << 30, fake, 1 << 30,
+                                None) == inv
+    lib.ttt_destroy(h)
