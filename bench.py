@@ -151,7 +151,9 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.idx = device_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        # the raw samples (the JSON line carries their summary); TTT_BENCH_OUT picks the folder
+        out = os.environ.get("TTT_BENCH_OUT", os.path.join(ROOT, "bench_out"))
+        self.path = os.path.join(out, f"clocks_rank{device_index}.csv")
 
     def __enter__(self):
         try:

@@ -34,7 +34,7 @@ What is computed (sources: the pages' text, cited per function):
 * Key instance normalisation over tokens [TTT vs Sleep, "Side one": keys carry a
   constant shift that must be removed].
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent (numbered R1-R24 wherever they are cited):
   R1 every fast-weight matrix is updated; R2 MSE is the mean over the chunk's
   (token, channel) elements, weighted per token by eta_i; R3 the dot loss is a sum
   over tokens with no 1/n; R4 exact erf GELU; R5 SwiGLU W1 = SiLU gate, W3 = linear
