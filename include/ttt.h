@@ -68,7 +68,7 @@ extern "C" {
 
 #define TTT_OK 0
 #define TTT_ERR_INVALID_ARG (-1) /* null pointer, bad shape, causal with Nq != N, ... */
-#define TTT_ERR_UNSUPPORTED (-2) /* a valid combination this build does not implement */
+#define TTT_ERR_UNSUPPORTED (-2) /* a valid combination the library does not implement */
 #define TTT_ERR_CUDA (-3)        /* a CUDA runtime call failed */
 #define TTT_ERR_NONFINITE (-4)   /* O or W* holds Inf or NaN (device status word) */
 #define TTT_ERR_TIMEOUT (-5)     /* a bounded device-side wait ran out (device status word) */
