@@ -33,7 +33,7 @@ import torch  # noqa: E402
 
 from synth_inputs import WORKLOADS, gen_inputs, matrix_shapes, param_count, workload  # noqa: E402
 
-DEFAULT_WORKLOAD = "lact_nvs_n196k_d512"
+DEFAULT_WORKLOAD = "lact_scene_n1m_c131k"
 METRIC = "TTT-layer tokens/s (update+apply) and % of B200 bf16 dense tensor peak, 1 GPU"
 L2_BYTES = 126 * 1024 * 1024
 DATASHEET_BF16_TFLOPS = 2250.0
@@ -41,7 +41,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # tokens per reference-arm step (bounded CPU sample) and per CPU-baseline sample
 CPU_SAMPLE_TOKENS = {
     "tiny_mlp2_n196_fp32": 196, "vit3s_1248_mlp2_n6084": 6084, "lact_lm_causal_n32k_c2048": 16384,
-    "lact_nvs_n196k_d512": 65536, "lact_scene_n1m_c131k": 65536, "vit3s_1248_dwconv_n6084": 8 * 6084,
+    "lact_nvs_n196k_d512": 65536, "lact_scene_n1m_c131k": 32768, "vit3s_1248_dwconv_n6084": 8 * 6084,
 }
 
 

@@ -44,10 +44,10 @@
  *   owns only host-side state.  Device pointers must be 16-byte aligned and
  *   contiguous.  ttt_forward only enqueues work on `stream` and returns; it
  *   allocates nothing.  One handle must not be used on two streams at once.
- *   The library sets its kernels' shared-memory and cluster attributes once per
- *   process, on the device current at the first call: drive one GPU per process
- *   (the usual one-rank-per-GPU layout).  A call on a second device of the same
- *   process is not supported and may return TTT_ERR_CUDA.
+ *   Calls run on the device current in the calling thread.  The library sets
+ *   its kernels' shared-memory and cluster attributes, and asks how many CTA
+ *   pairs fit, once per device, the first time a kernel runs there; one process
+ *   may drive layers on several GPUs (handles hold no device state).
  *
  * Errors
  *   Calls return TTT_OK (0) or a negative status.  Argument errors are found on
@@ -207,6 +207,9 @@ int ttt_forward_host(ttt_handle* handle, const void* Q, const void* K, const voi
  *     routine).  The caller passes inputs and outputs exactly as for ttt_forward.
  *   - The first call on a device looks up the address of that device's array with
  *     that device current; make that first call before any stream capture begins.
+ *     The address is kept for the life of the process: after cudaDeviceReset (or
+ *     any other end of the device's primary context) the array is gone and this
+ *     entry must not be called again on that device.
  *   - Every call on a device shares the one array.  Each call clears what must
  *     start at zero, but calls whose GPU work overlaps (other streams, other host
  *     threads) race on the array: serialise them.

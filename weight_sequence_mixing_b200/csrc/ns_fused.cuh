@@ -315,16 +315,13 @@ cudaError_t launch_ns_fused_cs(int nmat, const NsGeom& g, unsigned* status, cuda
       !make_tmap(&sX2, g.X2, 4, n, m, nmat, n, int64_t(m) * n, 32))
     return cudaErrorInvalidValue;
   auto kern = ns_fused_kernel<CS>;
-  static bool configured = false;
-  if (!configured) {
+  static OncePerDevice configured;
+  const int set = configured.run(current_device(), [&] {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kNsSmem);
-    if (e != cudaSuccess) return e;
-    if (CS > 8) {
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      if (e != cudaSuccess) return e;
-    }
-    configured = true;
-  }
+    if (e == cudaSuccess && CS > 8) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    return e;
+  });
+  if (set != 0) return static_cast<cudaError_t>(set);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nmat * CS, 1, 1);
   cfg.blockDim = dim3(192, 1, 1);
@@ -343,10 +340,10 @@ cudaError_t launch_ns_fused_cs(int nmat, const NsGeom& g, unsigned* status, cuda
 // Whether a cluster of CS CTAs of this kernel can be resident at all on this device.
 template <int CS>
 bool ns_cluster_fits() {
-  static int fits = -1;
-  if (fits < 0) {
+  static IntPerDevice fit;
+  return fit.get(current_device(), [] {
     auto kern = ns_fused_kernel<CS>;
-    fits = 0;
+    int fits = 0;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kNsSmem) == cudaSuccess &&
         (CS <= 8 || cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess)) {
       cudaLaunchConfig_t cfg = {};
@@ -364,8 +361,8 @@ bool ns_cluster_fits() {
       if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) fits = 1;
     }
     cudaGetLastError();  // a refused query leaves no sticky error behind
-  }
-  return fits == 1;
+    return fits;
+  }) == 1;
 }
 
 // Cluster size: one CTA per 128 x 128 tile of the largest step (T' X), at most 16

@@ -854,12 +854,12 @@ void choose_grad_shape(const Plan& p, int Cp, int* splits, int* tile_rows, int* 
   // 4096 tokens are not split at all (the gradient then goes straight to the optimizer)
   const int smax = kblocks <= 64 ? 1 : std::min(64, std::max(1, kblocks / 16));
   const int tiles256 = (r0 % 256 == 0 && rows % 256 == 0) ? rows / 256 * (d / bnd) * p.BH : 0;
-  *tile_rows = (tiles256 > 0 && tiles256 * smax >= 148) ? 256 : 128;
+  *tile_rows = (tiles256 > 0 && tiles256 * smax >= kPlanSMs) ? 256 : 128;
   // 512-row tiles on CTA pairs (74 pairs): each CTA brings in a third fewer bytes
   const bool pairs_ok = (c.flags & TTT_FLAG_SINGLE_CTA) == 0 && bnd >= 128;
   const int tiles512 = (pairs_ok && r0 % 512 == 0 && rows % 512 == 0) ? rows / 512 * (d / bnd) * p.BH : 0;
-  if (tiles512 > 0 && tiles512 * smax >= 74) *tile_rows = 512;
-  const int units = *tile_rows == 512 ? 74 : 148;  // tiles that run at once
+  if (tiles512 > 0 && tiles512 * smax >= kPlanSMs / 2) *tile_rows = 512;
+  const int units = *tile_rows == 512 ? kPlanSMs / 2 : kPlanSMs;  // tiles that run at once
   const int tiles = rows / *tile_rows * (d / bnd) * p.BH;
   // about two waves of tiles: long K ranges per split, few partials to reduce
   int s = tiles > 0 ? std::max(1, (2 * units + tiles / 2) / tiles) : 1;

@@ -185,7 +185,7 @@ DwGeom geom_of(const Plan& p) {
   return g;
 }
 
-int grid_1d(int64_t n) { return int(std::min<int64_t>((n + 255) / 256, 148 * 16)); }
+int grid_1d(int64_t n) { return int(std::min<int64_t>((n + 255) / 256, int64_t(sm_count()) * 16)); }
 
 template <int K, class T>
 int run_k(const Plan& p, const Io& io, uint8_t* ws, cudaStream_t st) {
@@ -254,7 +254,7 @@ int plan_layout_dwconv(Plan* p) {
   // token blocks: about four CTAs per SM over all (z, channel group) pairs, at least
   // 64 tokens per block; every block non-empty
   const int64_t groups = Z * ((d + 127) / 128);
-  const int64_t want = std::max<int64_t>(1, (4 * 148 + groups - 1) / groups);
+  const int64_t want = std::max<int64_t>(1, (4 * kPlanSMs + groups - 1) / groups);
   const int64_t blocks0 = std::max<int64_t>(1, std::min<int64_t>(want, (c.N + 63) / 64));
   const int64_t per = (c.N + blocks0 - 1) / blocks0;
   const int64_t blocks = (c.N + per - 1) / per;

@@ -280,7 +280,7 @@ __global__ void nonfinite_kernel(int64_t n, const float* x, unsigned* status) {
   if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, kStatusNonFinite);
 }
 
-int grid_for(int64_t n) { return int(std::min<int64_t>((n + 255) / 256, 148 * 16)); }
+int grid_for(int64_t n) { return int(std::min<int64_t>((n + 255) / 256, int64_t(sm_count()) * 16)); }
 
 // ------------------------------------------------------------------ workspace
 enum Buf { bW, bM, bG, bXn, bZ1, bZ3, bA, bH, bdH, bY, bNX, bNX2, bNS, bNT, bRms, kNumBuf };

@@ -25,6 +25,7 @@
 #pragma once
 #include <algorithm>
 
+#include "per_device.h"
 #include "ptx.cuh"
 
 namespace ttt {
@@ -318,7 +319,10 @@ bool make_tmap(CUtensorMap* out, const void* base, int eb, int64_t cols, int64_t
 bool make_tmap_ex(CUtensorMap* out, const void* base, int eb, int64_t cols, int64_t rows, int64_t batches,
                   int64_t row_pitch_elems, int64_t batch_pitch_elems, int box_cols, int box_rows, int swizzle);
 
+// SMs of the current device (queried once per device)
 int sm_count();
+// the current device's ordinal, or -1 when it cannot be read
+int current_device();
 
 // persistent = true: at most (SMs x resident CTAs per SM) CTAs loop over the tiles;
 // otherwise one CTA per tile.
@@ -340,12 +344,11 @@ cudaError_t launch_tc_gemm(const CUtensorMap& a0, const CUtensorMap& b0, const C
   constexpr int kCtasPerSm = kSmemPerSM / (kSmem + kReservedPerCta) < kMaxCtas
                                  ? kSmemPerSM / (kSmem + kReservedPerCta)
                                  : kMaxCtas;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static OncePerDevice configured;
+  const int set = configured.run(current_device(), [&] {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  });
+  if (set != 0) return static_cast<cudaError_t>(set);
   const long long total = static_cast<long long>(g.m_tiles0 + g.m_tiles1) * g.n_tiles * g.batches * g.splits;
   if (total <= 0) return cudaSuccess;
   if (total > 0x7fffffffLL) return cudaErrorInvalidConfiguration;

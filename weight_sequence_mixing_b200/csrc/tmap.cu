@@ -16,15 +16,20 @@ PFN_tmapEncodeTiled tmap_encoder() {
   return fn;
 }
 
+int current_device() {
+  int dev = -1;
+  return cudaGetDevice(&dev) == cudaSuccess ? dev : -1;
+}
+
 int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        n <= 0)
-      n = 148;
-  }
-  return n;
+  static IntPerDevice counts;
+  const int dev = current_device();
+  return counts.get(dev, [dev] {
+    int n = 0;
+    if (dev < 0 || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;  // a B200's count, if the device cannot be asked
+    return n;
+  });
 }
 
 bool make_tmap(CUtensorMap* out, const void* base, int eb, int64_t cols, int64_t rows, int64_t batches,

@@ -317,10 +317,10 @@ cudaLaunchConfig_t pair_launch_config(int pairs, cudaStream_t st, cudaLaunchAttr
 // CTA pairs of this kernel that can be resident at once (0: none, use the single-CTA kernel).
 template <bool SWIGLU>
 int token_pair_capacity() {
-  static int cap = -1;
-  if (cap < 0) {
+  static IntPerDevice caps;
+  return caps.get(current_device(), [] {
     auto kern = token_pair_kernel<SWIGLU>;
-    cap = 0;
+    int cap = 0;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairShape<SWIGLU>::SMEM) ==
         cudaSuccess) {
       cudaLaunchAttribute attr[1];
@@ -329,8 +329,8 @@ int token_pair_capacity() {
       if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) cap = n;
     }
     cudaGetLastError();  // a refused query leaves no sticky error behind
-  }
-  return cap;
+    return cap;
+  });
 }
 
 // g.m_tiles counts 256-token tiles; g.rows_alloc bounds the rows the stores may write.

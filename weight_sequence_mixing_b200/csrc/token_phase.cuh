@@ -338,12 +338,11 @@ cudaError_t launch_token_dot(const CUtensorMap& tX, const CUtensorMap& tFirst, c
                              const TokGeom& g, unsigned* status, cudaStream_t st) {
   using S = TokShape<SWIGLU>;
   auto kern = token_dot_kernel<SWIGLU>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static OncePerDevice configured;
+  const int set = configured.run(current_device(), [&] {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+  });
+  if (set != 0) return static_cast<cudaError_t>(set);
   const long long total = static_cast<long long>(g.m_tiles) * g.n_tiles * g.batches;
   if (total <= 0) return cudaSuccess;
   if (total > 0x7fffffffLL || g.kblocks <= 0) return cudaErrorInvalidConfiguration;

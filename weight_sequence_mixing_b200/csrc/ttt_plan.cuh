@@ -41,6 +41,11 @@ struct Plan {
 };
 
 int plan_build(const ttt_config& cfg, Plan* plan);
+// SMs of the current device (launch-time grid sizing; tmap.cu)
+int sm_count();
+// B200's SM count: the planner sizes its work splits with it, since ttt_create runs
+// on the host without a device
+constexpr int kPlanSMs = 148;
 int plan_run(const Plan& plan, const Io& io, void* workspace, cudaStream_t st);
 
 // per-path workspace layout and launch sequence

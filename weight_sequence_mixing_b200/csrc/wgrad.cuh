@@ -201,12 +201,11 @@ cudaError_t launch_wgrad(const CUtensorMap& a0, const CUtensorMap& b0, const CUt
   auto kern = wgrad_kernel<BN, STAGES, Epi>;
   // one CTA per SM: the accumulators may take all 512 TMEM columns
   constexpr int kSmem = S::SMEM > 116 * 1024 ? S::SMEM : 116 * 1024;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static OncePerDevice configured;
+  const int set = configured.run(current_device(), [&] {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  });
+  if (set != 0) return static_cast<cudaError_t>(set);
   const long long total = static_cast<long long>(g.m_tiles0 + g.m_tiles1) * g.n_tiles * g.batches * g.splits;
   if (total <= 0) return cudaSuccess;
   if (total > 0x7fffffffLL) return cudaErrorInvalidConfiguration;

@@ -234,10 +234,10 @@ cudaLaunchConfig_t wgrad_pair_config(int pairs, cudaStream_t st, cudaLaunchAttri
 // CTA pairs of this instantiation that can be resident at once (0: use wgrad_kernel).
 template <int BN, int STAGES, class Epi>
 int wgrad_pair_capacity() {
-  static int cap = -1;
-  if (cap < 0) {
+  static IntPerDevice caps;
+  return caps.get(current_device(), [] {
     auto kern = wgrad_pair_kernel<BN, STAGES, Epi>;
-    cap = 0;
+    int cap = 0;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, WgPairShape<BN, STAGES>::SMEM) ==
         cudaSuccess) {
       cudaLaunchAttribute attr[1];
@@ -246,8 +246,8 @@ int wgrad_pair_capacity() {
       if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) cap = n;
     }
     cudaGetLastError();
-  }
-  return cap;
+    return cap;
+  });
 }
 
 // g.m_tiles0 / m_tiles1 count 512-row tiles.
