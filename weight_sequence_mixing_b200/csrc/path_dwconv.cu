@@ -60,13 +60,19 @@ __device__ __forceinline__ void gather_taps(const T* Xz, const DwGeom& g, int p,
   }
 }
 
+// Tap gradients of one token block: CTA (block, z, channel chunk) with threads
+// (channel, slot); slot s takes the block's tokens p0 + s, p0 + s + S, ...  The S
+// slots' register sums are added in slot order through shared memory, so the
+// partial of a block does not depend on timing.
 template <int K, class T>
-__global__ void __launch_bounds__(128) dw_tapgrad_kernel(DwGeom g, const T* X, const T* V, const float* eta,
+__global__ void __launch_bounds__(256) dw_tapgrad_kernel(DwGeom g, const T* X, const T* V, const float* eta,
                                                           const float* W, float* part) {
   constexpr int KK = K * K;
+  extern __shared__ float red[];  // [S][blockDim.x][KK]
   const int z = blockIdx.y;
-  const int c = blockIdx.z * blockDim.x + threadIdx.x;
-  if (c >= g.d) return;  // no block-wide synchronisation below
+  const int cx = threadIdx.x, slot = threadIdx.y, S = blockDim.y;
+  const int c = blockIdx.z * blockDim.x + cx;
+  const bool live = c < g.d;
   const int tb = blockIdx.x;
   const int p0 = tb * g.tok_per_block, p1 = min(g.N, p0 + g.tok_per_block);
   const T* Xz = X + int64_t(z) * g.N * g.d;
@@ -74,88 +80,121 @@ __global__ void __launch_bounds__(128) dw_tapgrad_kernel(DwGeom g, const T* X, c
   const bool mse = g.loss == TTT_LOSS_MSE;
   float w[KK];
 #pragma unroll
-  for (int t = 0; t < KK; ++t) w[t] = mse ? W[(int64_t(z) * g.d + c) * KK + t] : 0.f;
+  for (int t = 0; t < KK; ++t) w[t] = (mse && live) ? W[(int64_t(z) * g.d + c) * KK + t] : 0.f;
   float acc[KK];
 #pragma unroll
   for (int t = 0; t < KK; ++t) acc[t] = 0.f;
-  for (int p = p0; p < p1; ++p) {
-    float nb[KK];
-    gather_taps<K>(Xz, g, p, c, nb);
-    const float e = eta ? eta[int64_t(z) * g.N + p] : g.eta_scalar;
-    const float v = to_f(Vz[int64_t(p) * g.d + c]);
-    float dy;
-    if (mse) {
-      float f = 0.f;
+  if (live) {
+    for (int p = p0 + slot; p < p1; p += S) {
+      float nb[KK];
+      gather_taps<K>(Xz, g, p, c, nb);
+      const float e = eta ? eta[int64_t(z) * g.N + p] : g.eta_scalar;
+      const float v = to_f(Vz[int64_t(p) * g.d + c]);
+      float dy;
+      if (mse) {
+        float f = 0.f;
 #pragma unroll
-      for (int t = 0; t < KK; ++t) f += w[t] * nb[t];
-      dy = g.mse_coef * e * (f - v);
-    } else {
-      dy = -e * v;
+        for (int t = 0; t < KK; ++t) f += w[t] * nb[t];
+        dy = g.mse_coef * e * (f - v);
+      } else {
+        dy = -e * v;
+      }
+#pragma unroll
+      for (int t = 0; t < KK; ++t) acc[t] += dy * nb[t];
     }
-#pragma unroll
-    for (int t = 0; t < KK; ++t) acc[t] += dy * nb[t];
   }
-  float* out = part + ((int64_t(z) * g.blocks + tb) * g.d + c) * KK;
+  float* mine = red + (int64_t(slot) * blockDim.x + cx) * KK;
 #pragma unroll
-  for (int t = 0; t < KK; ++t) out[t] = acc[t];
+  for (int t = 0; t < KK; ++t) mine[t] = acc[t];
+  __syncthreads();
+  // slot-order sum: thread (cx, s) sums tap t = s, s + S, ... of channel cx
+  if (live) {
+    float* out = part + ((int64_t(z) * g.blocks + tb) * g.d + c) * KK;
+    for (int t = slot; t < KK; t += S) {
+      float u = 0.f;
+      for (int j = 0; j < S; ++j) u += red[(int64_t(j) * blockDim.x + cx) * KK + t];
+      out[t] = u;
+    }
+  }
 }
 
+// One warp per (z, channel): the lanes sum the token blocks' partials (lane l takes
+// blocks l, l + 32, ...), a fixed butterfly adds the lanes, then momentum, the step
+// and the kernel's L2 norm.
 template <int K>
 __global__ void dw_update_kernel(DwGeom g, const float* part, float* W, float* M, bool momentum, float beta, float lr,
                                  bool rownorm, unsigned* status) {
   constexpr int KK = K * K;
-  const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
-  if (i >= int64_t(g.Z) * g.d) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t i = blockIdx.x * int64_t(blockDim.x / 32) + threadIdx.x / 32;
+  if (i >= int64_t(g.Z) * g.d) return;  // whole warps leave together
   const int z = int(i / g.d), c = int(i % g.d);
   float u[KK];
 #pragma unroll
   for (int t = 0; t < KK; ++t) u[t] = 0.f;
-  for (int b = 0; b < g.blocks; ++b) {
+  for (int b = lane; b < g.blocks; b += 32) {
     const float* pb = part + ((int64_t(z) * g.blocks + b) * g.d + c) * KK;
 #pragma unroll
     for (int t = 0; t < KK; ++t) u[t] += pb[t];
   }
+#pragma unroll
+  for (int t = 0; t < KK; ++t)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) u[t] += __shfl_xor_sync(0xffffffffu, u[t], o);
   float* w = W + i * KK;
   float* m = M + i * KK;
+  float wt[KK];
   float s = 0.f;
 #pragma unroll
   for (int t = 0; t < KK; ++t) {
     float ut = u[t];
-    if (momentum) {
-      ut = beta * m[t] + ut;
-      m[t] = ut;
-    }
-    const float wt = w[t] - lr * ut;
-    w[t] = wt;
-    s += wt * wt;
+    if (momentum) ut = beta * m[t] + ut;
+    wt[t] = w[t] - lr * ut;
+    s += wt[t] * wt[t];
+    u[t] = ut;
   }
-  bool bad = false;
+  __syncwarp();
   const float inv = rownorm ? 1.0f / fmaxf(sqrtf(s), 1e-12f) : 1.0f;
+  bool bad = false;
+  for (int t = lane; t < KK; t += 32) {
+    float wv = 0.f, uv = 0.f;
 #pragma unroll
-  for (int t = 0; t < KK; ++t) {
-    const float wt = w[t] * inv;
-    w[t] = wt;
-    bad |= !isfinite(wt);
+    for (int q = 0; q < KK; ++q)
+      if (q == t) {
+        wv = wt[q];
+        uv = u[q];
+      }
+    if (momentum) m[t] = uv;
+    w[t] = wv * inv;
+    bad |= !isfinite(wv * inv);
   }
-  if (bad) set_status(status, kStatusNonFinite);
+  if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(status, kStatusNonFinite);
 }
 
+// O = sum_tap Wc * Q_{p+tap}: CTA (token chunk, z, channel chunk) with threads
+// (channel, slot); the channel's k*k weights stay in registers while the slots walk
+// the chunk's tokens.
 template <int K, class T>
-__global__ void dw_apply_kernel(DwGeom g, const T* Q, const float* W, T* O, unsigned* status) {
+__global__ void __launch_bounds__(256) dw_apply_kernel(DwGeom g, int tok_per_cta, const T* Q, const float* W, T* O,
+                                                        unsigned* status) {
   constexpr int KK = K * K;
-  const int64_t total = int64_t(g.Z) * g.N * g.d;
+  const int z = blockIdx.y;
+  const int c = blockIdx.z * blockDim.x + threadIdx.x;
+  if (c >= g.d) return;  // no block-wide synchronisation below
+  const int p0 = blockIdx.x * tok_per_cta, p1 = min(g.N, p0 + tok_per_cta);
+  float w[KK];
+#pragma unroll
+  for (int t = 0; t < KK; ++t) w[t] = W[(int64_t(z) * g.d + c) * KK + t];
+  const T* Qz = Q + int64_t(z) * g.N * g.d;
+  T* Oz = O + int64_t(z) * g.N * g.d;
   bool bad = false;
-  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
-    const int c = int(i % g.d);
-    const int64_t zp = i / g.d;
-    const int p = int(zp % g.N), z = int(zp / g.N);
+  for (int p = p0 + threadIdx.y; p < p1; p += blockDim.y) {
     float nb[KK];
-    gather_taps<K>(Q + int64_t(z) * g.N * g.d, g, p, c, nb);
-    const float* w = W + (int64_t(z) * g.d + c) * KK;
+    gather_taps<K>(Qz, g, p, c, nb);
     float s = 0.f;
 #pragma unroll
     for (int t = 0; t < KK; ++t) s += w[t] * nb[t];
-    O[i] = from_f<T>(s);
+    Oz[int64_t(p) * g.d + c] = from_f<T>(s);
     bad |= !isfinite(s);
   }
   if (bad) set_status(status, kStatusNonFinite);
@@ -209,23 +248,34 @@ int run_k(const Plan& p, const Io& io, uint8_t* ws, cudaStream_t st) {
   const bool momentum = c.opt == TTT_OPT_MOMENTUM;
   const bool rownorm = (c.flags & TTT_FLAG_WEIGHT_L2NORM) != 0;
   const int epochs = (c.flags & TTT_FLAG_NO_UPDATE) ? 0 : p.epochs;
-  const dim3 tg(g.blocks, g.Z, (g.d + 127) / 128);
+  // threads (channel, slot): up to 128 channels of a chunk, 256 threads per CTA
+  // (the slot sums of the tap pass stay within the default 48 KB of shared memory)
+  const int cx = std::min(g.d, 128);
+  const int slots = std::max(1, std::min(256 / cx, 49152 / (cx * K * K * int(sizeof(float)))));
+  const dim3 blk(cx, slots);
+  const int cchunks = (g.d + cx - 1) / cx;
+  const dim3 tg(g.blocks, g.Z, cchunks);
+  const size_t red_bytes = size_t(slots) * cx * (K * K) * sizeof(float);
   for (int ep = 0; ep < epochs; ++ep) {
     {
       StageScope _sc(kStageWeightGrad, st);
-      dw_tapgrad_kernel<K, T><<<tg, 128, 0, st>>>(g, static_cast<const T*>(io.K), static_cast<const T*>(io.V), io.eta,
-                                                   W, part);
+      dw_tapgrad_kernel<K, T><<<tg, blk, red_bytes, st>>>(g, static_cast<const T*>(io.K), static_cast<const T*>(io.V),
+                                                          io.eta, W, part);
     }
     {
       StageScope _sc(kStageFinish, st);
-      dw_update_kernel<K><<<int((int64_t(g.Z) * g.d + 255) / 256), 256, 0, st>>>(g, part, W, M, momentum, c.momentum,
-                                                                                  c.lr, rownorm, status);
+      dw_update_kernel<K><<<int((int64_t(g.Z) * g.d + 7) / 8), 256, 0, st>>>(g, part, W, M, momentum, c.momentum, c.lr,
+                                                                             rownorm, status);
     }
   }
   {
     StageScope _sc(kStageApply, st);
-    dw_apply_kernel<K, T><<<grid_1d(int64_t(g.Z) * g.N * g.d), 256, 0, st>>>(g, static_cast<const T*>(io.Q), W,
-                                                                              static_cast<T*>(io.O), status);
+    // about eight CTAs per SM over (token chunk, z, channel chunk)
+    const int64_t want = std::max<int64_t>(1, (int64_t(sm_count()) * 8 + int64_t(g.Z) * cchunks - 1) /
+                                                  (int64_t(g.Z) * cchunks));
+    const int tok = int(std::max<int64_t>(slots, (g.N + want - 1) / want));
+    const dim3 ag((g.N + tok - 1) / tok, g.Z, cchunks);
+    dw_apply_kernel<K, T><<<ag, blk, 0, st>>>(g, tok, static_cast<const T*>(io.Q), W, static_cast<T*>(io.O), status);
   }
   if (io.W_out && cudaMemcpyAsync(io.W_out, W, size_t(ZP) * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return TTT_ERR_CUDA;
