@@ -33,8 +33,6 @@ int ttt_selftest_gemm(int elem_bytes, int a_mn, int b_mn, int bn, int M, int N, 
  *   [4] rows per weight-gradient tile: 128 or 256 on single CTAs, 512 on CTA pairs
  *   [5] output columns per weight-gradient tile
  *   [6] 1 when unsplit reductions write U (and momentum) directly, without partials
- *   [7] 1 when the weight-gradient epilogue also takes the step, normalises the rows
- *       and writes the weights (no separate optimizer launches)
  * Returns the number of entries written, or TTT_ERR_INVALID_ARG. */
 int ttt_plan_info(const ttt_handle* handle, int* info, int n);
 

@@ -13,17 +13,14 @@ EXPECTED = {
     "tiny_mlp2_n196_fp32": dict(path=0, chunk=196, nchunks=1),
     # d = 64: 256-row single-CTA tiles of 64 columns, 3 splits of 2048 tokens
     "vit3s_1248_mlp2_n6084": dict(path=1, chunk=6084, nchunks=1, splits=3, tile_rows=256, grad_bn=64, direct=0),
-    # 2048-token chunks are not split, and with d = h = 256 a 256-column tile holds whole
-    # weight rows: the gradient epilogue takes the momentum step, normalises the rows
-    # and writes the weights itself
-    "lact_lm_causal_n32k_c2048": dict(path=1, chunk=2048, nchunks=16, splits=1, tile_rows=128, grad_bn=256,
-                                      direct=1, fused_finish=1),
+    # 2048-token chunks are not split: gradients go straight into U and the momentum;
+    # 128-column tiles give the 96 CTAs the 256-column tiles would halve
+    "lact_lm_causal_n32k_c2048": dict(path=1, chunk=2048, nchunks=16, splits=1, tile_rows=128, grad_bn=128,
+                                      direct=1),
     # one 196608-token chunk: 512-row pair tiles (24 of them), 6 splits (144 pair tiles)
-    "lact_nvs_n196k_d512": dict(path=1, chunk=196608, nchunks=1, splits=6, tile_rows=512, grad_bn=256, direct=0,
-                                fused_finish=0),
+    "lact_nvs_n196k_d512": dict(path=1, chunk=196608, nchunks=1, splits=6, tile_rows=512, grad_bn=256, direct=0),
     # 8 chunks of 131072 (the last one 111616): 12 pair tiles x 12 splits
-    "lact_scene_n1m_c131k": dict(path=1, chunk=131072, nchunks=8, splits=12, tile_rows=512, grad_bn=256, direct=0,
-                                 fused_finish=0),
+    "lact_scene_n1m_c131k": dict(path=1, chunk=131072, nchunks=8, splits=12, tile_rows=512, grad_bn=256, direct=0),
 }
 
 
@@ -62,12 +59,6 @@ def test_split_heuristic_invariants(d, h, n, opt):
     if opt == "muon" and got["direct"]:
         assert got["grad_bn"] == d
     assert got["direct"] == (1 if got["splits"] == 1 and not (opt == "muon" and got["grad_bn"] != d) else 0)
-    # the weights are finished in the gradient epilogue exactly when a tile holds whole
-    # rows of every matrix of an unsplit, Muon-free update
-    fused = got["splits"] == 1 and opt != "muon" and got["tile_rows"] == 128 and d == h and d in (128, 256)
-    assert got["fused_finish"] == (1 if fused else 0)
-    if got["fused_finish"]:
-        assert got["grad_bn"] == d and got["direct"] == 1
 
 
 def _sizes(cfg):

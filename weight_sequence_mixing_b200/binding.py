@@ -308,7 +308,7 @@ def selftest_timeout(status_word: torch.Tensor, stream=None) -> int:
     return int(LIB.ttt_selftest_timeout(_ptr(status_word), _stream_ptr(stream)))
 
 
-PLAN_FIELDS = ("path", "chunk", "nchunks", "splits", "tile_rows", "grad_bn", "direct", "fused_finish")
+PLAN_FIELDS = ("path", "chunk", "nchunks", "splits", "tile_rows", "grad_bn", "direct")
 
 
 def plan_info(cfg: dict) -> dict:

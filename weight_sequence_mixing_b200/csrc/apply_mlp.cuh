@@ -1,0 +1,311 @@
+// Apply on the queries, O = F_W(Q), as one kernel with the hidden layer kept on chip
+// (ViT3 digest section 02: the queries read the updated fast weights; LaCT analysis,
+// "Nonlinear memory complements local attention": SwiGLU F(x) = (SiLU(x W1^T) * x W3^T) W2^T).
+//
+// A CTA owns 128 query rows of one head at a time (persistent over tiles).  The row
+// tile of Q stays in shared memory; for every block of 128 hidden units
+//   Z   = Q [W1_blk; W3_blk]^T (SwiGLU: z1 | z3, 256 TMEM columns; GELU MLP: z, 128)
+//   H   = SiLU(z1) z3  (or GELU(z)), bf16, written by the epilogue warps straight into
+//         shared memory in the 128-byte-swizzled K-major layout an MMA operand needs
+//   O  += H W2[:, blk]^T  (d TMEM columns, accumulated over the hidden blocks)
+// and after the last block the epilogue writes O.  The next block's Z MMAs overlap
+// the gating of the current one (Z is read out of TMEM before the gating math).
+// d <= 256 (O and Z together fit the 512 TMEM columns).
+//
+// Warps: 0 TMA producer, 1 MMA issuer, 2..9 epilogue (two per TMEM lane quarter; warp
+// half j of a quarter owns hidden columns [64 j, 64 j + 64) of a block, which is
+// k-block j of the H operand, and half of O's columns).  Every wait is bounded.
+#pragma once
+#include "epilogues.cuh"
+
+namespace ttt {
+
+struct ApplyGeom {
+  int m_tiles, batches;  // 128-row query tiles per head, heads (z)
+  int hblocks;           // h / 128
+  int rows_valid;        // query rows of each head
+  int row0;              // first query row of this call (causal chunks) in Q and O
+  int64_t o_zs;          // elements between heads in O
+};
+
+template <bool SWIGLU, int D>
+struct ApplyShape {
+  static constexpr int KB = D / 64;                  // k-blocks of Q (64 channels each)
+  static constexpr int ZN = SWIGLU ? 256 : 128;      // first-layer rows per hidden block
+  static constexpr int Q_BYTES = KB * 128 * 128;     // 128 rows x D bf16
+  static constexpr int H_BYTES = 2 * 128 * 128;      // 128 rows x 128 hidden bf16
+  static constexpr int STAGE = (ZN > D ? ZN : D) * 128;  // one B k-block (64 K elements)
+  static constexpr int STAGES = 3;
+  static constexpr int EW = 8;
+  static constexpr int SMEM = 1024 + Q_BYTES + H_BYTES + STAGES * STAGE + 256;
+  static constexpr uint32_t Z_COL = 256;             // Z accumulator columns [256, 256 + ZN)
+  static_assert(D == 64 || D == 128 || D == 256, "d");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+template <bool SWIGLU, int D>
+__global__ void __launch_bounds__(64 + 32 * ApplyShape<SWIGLU, D>::EW, 1)
+    apply_mlp_kernel(const __grid_constant__ CUtensorMap tQ, const __grid_constant__ CUtensorMap tFirst,
+                     const __grid_constant__ CUtensorMap tW2, const ApplyGeom g, bf16* O, unsigned* status) {
+  using S = ApplyShape<SWIGLU, D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* qs = smem;
+  uint8_t* hs = qs + S::Q_BYTES;
+  uint8_t* ring = hs + S::H_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + S::STAGES * S::STAGE);
+  uint64_t* empty = full + S::STAGES;
+  uint64_t* qfull = empty + S::STAGES;  // the tile's Q rows landed
+  uint64_t* qempty = qfull + 1;         // the tile's MMAs are done with them
+  uint64_t* zfull = qempty + 1;         // Z of a hidden block is in TMEM
+  uint64_t* zempty = zfull + 1;         // the epilogue has read it
+  uint64_t* hfull = zempty + 1;         // H of the block is in shared memory
+  uint64_t* hempty = hfull + 1;         // the O MMAs reading H are done
+  uint64_t* ofull = hempty + 1;         // O of the tile is complete
+  uint64_t* oempty = ofull + 1;         // the epilogue has read O
+  uint64_t* drain = oempty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = static_cast<int>(lane_id());
+  const int total = g.m_tiles * g.batches;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(qfull, 1);
+    mbar_init(qempty, 1);
+    mbar_init(zfull, 1);
+    mbar_init(zempty, S::EW);
+    mbar_init(hfull, S::EW);
+    mbar_init(hempty, 1);
+    mbar_init(ofull, 1);
+    mbar_init(oempty, S::EW);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      tma_prefetch_desc(&tQ);
+      tma_prefetch_desc(&tFirst);
+      tma_prefetch_desc(&tW2);
+      int it = 0, j = 0;
+      bool stop = false;
+      for (int t = blockIdx.x; t < total && !stop; t += gridDim.x, ++j) {
+        const int mt = t % g.m_tiles, z = t / g.m_tiles;
+        // the previous tile's MMAs have finished reading Q
+        if (j > 0 && !mbar_wait(qempty, (j - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(qfull, S::Q_BYTES);
+        for (int kb = 0; kb < S::KB; ++kb) tma_load_3d(qs + kb * 128 * 128, &tQ, qfull, kb * 64, g.row0 + mt * 128, z);
+        for (int hb = 0; hb < g.hblocks && !stop; ++hb) {
+          // first-layer rows of the block (K = d), then W2's columns of the block (K = hidden)
+          for (int i = 0; i < S::KB + 2; ++i, ++it) {
+            const int s = it % S::STAGES;
+            const uint32_t ph = (it / S::STAGES) & 1;
+            if (it >= S::STAGES && !mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
+              stop = true;
+              break;
+            }
+            uint8_t* st = ring + s * S::STAGE;
+            if (i < S::KB) {
+              mbar_arrive_expect_tx(&full[s], S::ZN * 128);
+              tma_load_3d(st, &tFirst, &full[s], i * 64, hb * S::ZN, z);
+            } else {
+              mbar_arrive_expect_tx(&full[s], D * 128);
+              tma_load_3d(st, &tW2, &full[s], hb * 128 + (i - S::KB) * 64, 0, z);
+            }
+          }
+        }
+      }
+      if (*abort_flag) {
+        // copies already in flight land within microseconds; give them a millisecond
+        const unsigned long long t0 = global_ns();
+        while (global_ns() - t0 < 1000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      constexpr uint32_t idZ = make_idesc(128, S::ZN, 1, false, false);
+      constexpr uint32_t idO = make_idesc(128, D, 1, false, false);
+      const uint32_t qbase = smem_u32(qs), hbase = smem_u32(hs), rbase = smem_u32(ring);
+      int it = 0, j = 0, nz = 0;  // ring position, tiles, hidden blocks issued
+      bool stop = false;
+      for (int t = blockIdx.x; t < total && !stop; t += gridDim.x, ++j) {
+        if (!mbar_wait(qfull, j & 1, abort_flag)) break;
+        tc_fence_after();
+        for (int hb = 0; hb < g.hblocks && !stop; ++hb, ++nz) {
+          // Z of the previous block has been read out of TMEM
+          if (nz > 0 && !mbar_wait(zempty, (nz - 1) & 1, abort_flag)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          for (int kb = 0; kb < S::KB; ++kb, ++it) {
+            const int s = it % S::STAGES;
+            if (!mbar_wait(&full[s], (it / S::STAGES) & 1, abort_flag)) {
+              stop = true;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a = qbase + kb * 128 * 128, b = rbase + s * S::STAGE;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16(tmem_base + S::Z_COL, make_sdesc_sw128(a + kk * 32, 16, 1024),
+                      make_sdesc_sw128(b + kk * 32, 16, 1024), idZ, (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&empty[s]);
+          }
+          if (stop) break;
+          mma_commit(zfull);
+          // H of this block written by the epilogue (and, for the tile's first block,
+          // O of the previous tile read out of TMEM)
+          if (!mbar_wait(hfull, nz & 1, abort_flag)) {
+            stop = true;
+            break;
+          }
+          if (hb == 0 && j > 0 && !mbar_wait(oempty, (j - 1) & 1, abort_flag)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          for (int kh = 0; kh < 2; ++kh, ++it) {
+            const int s = it % S::STAGES;
+            if (!mbar_wait(&full[s], (it / S::STAGES) & 1, abort_flag)) {
+              stop = true;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a = hbase + kh * 128 * 128, b = rbase + s * S::STAGE;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16(tmem_base, make_sdesc_sw128(a + kk * 32, 16, 1024), make_sdesc_sw128(b + kk * 32, 16, 1024),
+                      idO, (hb > 0 || kh > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&empty[s]);
+          }
+          if (stop) break;
+          mma_commit(hempty);
+        }
+        if (stop) break;
+        mma_commit(ofull);
+        mma_commit(qempty);
+      }
+      if (*abort_flag) {
+        volatile int never = 0;
+        mma_commit(drain);
+        mbar_wait(drain, 0, &never);
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;  // hidden columns [64 half, 64 half + 64) of a block
+    const int row = q * 32 + lane;
+    const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    uint8_t* hk = hs + half * 128 * 128 + row * 128;  // this thread's row of H's k-block `half`
+    int j = 0, nz = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++j) {
+      const int mt = t % g.m_tiles, z = t / g.m_tiles;
+      for (int hb = 0; hb < g.hblocks; ++hb, ++nz) {
+        ok = __all_sync(0xffffffffu, mbar_wait(zfull, nz & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        // read this thread's 64 hidden columns of Z (and z3), then release the TMEM
+        uint32_t packed[32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float z1[32], z3[32];
+          tmem_ld32(tq + S::Z_COL + half * 64 + c * 32, z1);
+          if constexpr (SWIGLU) tmem_ld32(tq + S::Z_COL + 128 + half * 64 + c * 32, z3);
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float a, b;
+            if constexpr (SWIGLU) {
+              a = z1[i] * sigmoid_dev(z1[i]) * z3[i];
+              b = z1[i + 1] * sigmoid_dev(z1[i + 1]) * z3[i + 1];
+            } else {
+              a = gelu_dev(z1[i]);
+              b = gelu_dev(z1[i + 1]);
+            }
+            packed[c * 16 + i / 2] = pack_bf16x2(a, b);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(zempty);
+        // the previous block's O MMAs are done reading H
+        if (nz > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(hempty, (nz - 1) & 1, abort_flag));
+          if (!ok) break;
+        }
+        // 64 bf16 = 8 chunks of 16 bytes; chunk k of row r sits at k ^ (r & 7)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          *reinterpret_cast<uint4*>(hk + 16 * (k ^ (row & 7))) =
+              make_uint4(packed[4 * k], packed[4 * k + 1], packed[4 * k + 2], packed[4 * k + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(hfull);
+      }
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(ofull, j & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const int m = mt * 128 + row;
+      const bool valid = m < g.rows_valid;
+      bf16* orow = O + z * g.o_zs + int64_t(g.row0 + m) * D;
+      bool bad = false;
+#pragma unroll 1
+      for (int cc = half * (D / 2); cc < (half + 1) * (D / 2); cc += 32) {
+        float v[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + cc, v);
+        if (!valid) continue;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) bad |= !isfinite(v[i]);
+        store_bf16x32(orow + cc, v);
+      }
+      if (bad) set_status(status, kStatusNonFinite);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(oempty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0 && *abort_flag) set_status(status, kStatusTimeout);
+  if (warp == 1) tmem_dealloc(tmem_base, 512);
+}
+
+template <bool SWIGLU, int D>
+cudaError_t launch_apply_mlp(const CUtensorMap& tQ, const CUtensorMap& tFirst, const CUtensorMap& tW2,
+                             const ApplyGeom& g, bf16* O, unsigned* status, cudaStream_t st) {
+  using S = ApplyShape<SWIGLU, D>;
+  auto kern = apply_mlp_kernel<SWIGLU, D>;
+  static OncePerDevice configured;
+  const int set = configured.run(current_device(), [&] {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+  });
+  if (set != 0) return static_cast<cudaError_t>(set);
+  const long long total = static_cast<long long>(g.m_tiles) * g.batches;
+  if (total <= 0) return cudaSuccess;
+  if (total > 0x7fffffffLL || g.hblocks <= 0) return cudaErrorInvalidConfiguration;
+  const int grid = static_cast<int>(std::min<long long>(total, sm_count()));
+  kern<<<grid, 64 + 32 * S::EW, S::SMEM, st>>>(tQ, tFirst, tW2, g, O, status);
+  return cudaGetLastError();
+}
+
+}  // namespace ttt

@@ -48,45 +48,6 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
   return r;
 }
 
-// Hand-off of a split-K partial tile to the other CTA of a pair (distributed shared
-// memory): stores into the peer's buffer, a release at cluster scope by each lane, and
-// an arrival on the peer's mbarrier; the peer waits with acquire at cluster scope.
-__device__ __forceinline__ void st_cluster_f4(uint32_t addr, float4 v) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
-               "f"(v.w)
-               : "memory");
-}
-__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait_cluster_acq(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// bounded like mbar_wait (kWaitLimitNs), acquiring what the peer released
-__device__ __forceinline__ bool mbar_wait_peer(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait_cluster_acq(bar, parity)) return true;
-  const unsigned long long t0 = global_ns();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait_cluster_acq(bar, parity)) return true;
-    if (*abort) return false;
-    if (global_ns() - t0 > kWaitLimitNs) {
-      *abort = 1;
-      return false;
-    }
-  }
-}
-
 // The three steps of one iteration as tile problems.
 struct NsStep {
   const CUtensorMap* A;
@@ -94,11 +55,8 @@ struct NsStep {
   int tiles_n;  // output tiles per tile row
   int tiles;    // output tiles in all
   int kblocks;  // K / 32
-  int split;    // 2: each tile's K range is cut in halves over two CTAs of the cluster
-  int items;    // tiles * split
 };
 
-template <int CS>
 __device__ __forceinline__ NsStep ns_step(int step, int it, const NsGeom& g, const CUtensorMap* mX,
                                           const CUtensorMap* mXT, const CUtensorMap* mX2, const CUtensorMap* mXT2,
                                           const CUtensorMap* mS, const CUtensorMap* mT) {
@@ -126,11 +84,6 @@ __device__ __forceinline__ NsStep ns_step(int step, int it, const NsGeom& g, con
     s.tiles = tm * tn;
     s.kblocks = g.m / 32;
   }
-  // S and T have fewer tiles than the cluster has CTAs when m is small: each tile is
-  // then computed by CTAs 2i (first half of K) and 2i + 1 (second half), which adds the
-  // first one's partial, handed over through distributed shared memory.
-  s.split = (step < 2 && 2 * s.tiles <= CS && s.kblocks % 2 == 0) ? 2 : 1;
-  s.items = s.tiles * s.split;
   return s;
 }
 
@@ -151,8 +104,7 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* drain = tmem_empty + 2;
   uint64_t* efull = drain + 1;   // epilogue operand tile landed
   uint64_t* eempty = efull + 1;  // epilogue done with it
-  uint64_t* rx = eempty + 1;     // split-K: the partner's partial has landed in ebuf
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rx + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(eempty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -173,7 +125,6 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(drain, 1);
     mbar_init(efull, 1);
     mbar_init(eempty, 4);
-    mbar_init(rx, 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -185,25 +136,20 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // every CTA's barriers are initialised before a partner may arrive on them
-  cluster_sync_all();
 
   int it_ring = 0;  // producer / MMA position in the smem ring (lane 0 of warps 0 and 1)
   int j_tile = 0;   // tiles this CTA has computed (TMEM phases)
   int e_use = 0;    // epilogue operand tiles loaded (producer) / consumed (epilogue)
-  int rx_use = 0;   // partials received from the partner (epilogue)
   for (int it = 0; it < g.iters; ++it) {
     for (int step = 0; step < 3; ++step) {
-      const NsStep sp = ns_step<CS>(step, it, g, &mX, &mXT, &mX2, &mXT2, &mS, &mT);
+      const NsStep sp = ns_step(step, it, g, &mX, &mXT, &mX2, &mXT2, &mS, &mT);
       if (warp == 0) {
         if (lane == 0 && !*abort_flag) {
           fence_proxy_async_global();  // the previous step's generic stores -> these TMA loads
           const CUtensorMap* eop = step == 1 ? &mS : ((it & 1) ? &mX2 : &mX);  // S for T, X for X'
-          for (int w = rank; w < sp.items && !*abort_flag; w += CS) {
-            const int t = w / sp.split, half = w % sp.split;
-            const int kb0 = half * (sp.kblocks / sp.split), kb1 = kb0 + sp.kblocks / sp.split;
+          for (int t = rank; t < sp.tiles && !*abort_flag; t += CS) {
             const int r0 = (t / sp.tiles_n) * 128, c0 = (t % sp.tiles_n) * 128;
-            for (int kb = kb0; kb < kb1; ++kb, ++it_ring) {
+            for (int kb = 0; kb < sp.kblocks; ++kb, ++it_ring) {
               const int s = it_ring % kNsStages;
               const uint32_t ph = (it_ring / kNsStages) & 1;
               if (it_ring >= kNsStages && !mbar_wait(&empty[s], ph ^ 1, abort_flag)) break;
@@ -214,8 +160,7 @@ __global__ void __launch_bounds__(192, 1)
             }
             // after the tile's operands (so waiting for the previous epilogue never holds
             // them back): the fp32 tile its epilogue adds, S for T = b S + c S S, X for a X + T X
-            // (a split tile's second half adds its partner's partial instead: no prefetch)
-            if (step > 0 && half == 0 && !*abort_flag) {
+            if (step > 0 && !*abort_flag) {
               if (e_use > 0 && !mbar_wait(eempty, (e_use - 1) & 1, abort_flag)) break;
               mbar_arrive_expect_tx(efull, kNsEbuf);
               for (int bx = 0; bx < 4; ++bx) tma_load_3d(ebuf + bx * 128 * 128, eop, efull, c0 + 32 * bx, r0, zk);
@@ -228,15 +173,13 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0 && !*abort_flag) {
           constexpr uint32_t id = make_idesc(128, 128, 2, false, false);
           const uint32_t sbase = smem_u32(smem);
-          for (int w = rank; w < sp.items && !*abort_flag; w += CS) {
-            const int half = w % sp.split;
-            const int kb0 = half * (sp.kblocks / sp.split), kb1 = kb0 + sp.kblocks / sp.split;
+          for (int t = rank; t < sp.tiles && !*abort_flag; t += CS) {
             const int buf = j_tile & 1;
             // buffer `buf` last held tile j_tile - 2: its epilogue must have drained it
             if (j_tile >= 2 && !mbar_wait(&tmem_empty[buf], ((j_tile - 2) >> 1) & 1, abort_flag)) break;
             tc_fence_after();
             const uint32_t dacc = tmem_base + static_cast<uint32_t>(buf * 128);
-            for (int kb = kb0; kb < kb1; ++kb, ++it_ring) {
+            for (int kb = 0; kb < sp.kblocks; ++kb, ++it_ring) {
               const int s = it_ring % kNsStages;
               const uint32_t ph = (it_ring / kNsStages) & 1;
               if (!mbar_wait(&full[s], ph, abort_flag)) break;
@@ -246,7 +189,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
                 mma_tf32(dacc, make_sdesc_sw128(a + kk * 32, 16, 1024), make_sdesc_sw128(b + kk * 32, 16, 1024), id,
-                         (kb > kb0 || kk > 0) ? 1u : 0u);
+                         (kb > 0 || kk > 0) ? 1u : 0u);
               mma_commit(&empty[s]);
             }
             mma_commit(&tmem_full[buf]);
@@ -257,10 +200,7 @@ __global__ void __launch_bounds__(192, 1)
       } else {
         const int q = warp & 3;
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-        for (int w = rank; w < sp.items; w += CS) {
-          const int t = w / sp.split, half = w % sp.split;
-          const bool sender = sp.split == 2 && half == 0;    // first K half: hands its partial over
-          const bool receiver = sp.split == 2 && half == 1;  // second K half: adds it and stores
+        for (int t = rank; t < sp.tiles; t += CS) {
           const int buf = j_tile & 1;
           const bool ready = __all_sync(0xffffffffu, mbar_wait(&tmem_full[buf], (j_tile >> 1) & 1, abort_flag));
           if (!ready) break;
@@ -271,53 +211,14 @@ __global__ void __launch_bounds__(192, 1)
           float* nxt = odd ? g.XT : g.XT2;  // X^T of the next iteration
           const uint32_t tacc = taddr + static_cast<uint32_t>(buf * 128);
           const int lrow = q * 32 + lane;  // row inside the tile (and the prefetched box)
-          if (step > 0 && !receiver) {
+          if (step > 0) {
             const bool landed = __all_sync(0xffffffffu, mbar_wait(efull, e_use & 1, abort_flag));
             if (!landed) break;
           }
-          if (receiver) {
-            const bool got = __all_sync(0xffffffffu, mbar_wait_peer(rx, rx_use & 1, abort_flag));
-            ++rx_use;
-            if (!got) break;
-          }
-          // the partner's copy of this thread's row of ebuf (same swizzled layout)
-          const uint32_t peer_row = sender ? mapa_shared(smem_u32(ebuf + lrow * 128), rank + 1) : 0u;
 #pragma unroll 1
           for (int cc = 0; cc < 128; cc += 32) {
             float v[32];
             tmem_ld32(tacc + cc, v);
-            if (sender || receiver) {
-              // box cc/32, row lrow, 16-byte chunk k at k ^ (lrow & 7)
-              float e[32];
-              if (step == 1 || receiver) {
-                const float4* box = reinterpret_cast<const float4*>(ebuf + (cc / 32) * 128 * 128 + lrow * 128);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                  const float4 f = box[k ^ (lrow & 7)];
-                  e[4 * k] = f.x;
-                  e[4 * k + 1] = f.y;
-                  e[4 * k + 2] = f.z;
-                  e[4 * k + 3] = f.w;
-                }
-              }
-              if (sender) {
-                // S: the first half's sum; T: b S + c (first half of S S)
-                if (step == 1) {
-#pragma unroll
-                  for (int i = 0; i < 32; ++i) v[i] = g.b * e[i] + g.c * v[i];
-                }
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                  st_cluster_f4(peer_row + (cc / 32) * 128 * 128 + 16 * (k ^ (lrow & 7)),
-                                make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]));
-              } else {
-                const float cf = step == 0 ? 1.0f : g.c;
-                float* col = (step == 0 ? g.S : g.T) + zk * mm + int64_t(c0 + cc) * g.m + row;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) col[int64_t(i) * g.m] = e[i] + cf * v[i];  // mirrored, as below
-              }
-              continue;
-            }
             if (step == 0) {
               // S is symmetric: write the tile transposed, into the mirrored position, so that
               // the warp's 32 lanes (consecutive rows) store consecutive addresses
@@ -356,12 +257,6 @@ __global__ void __launch_bounds__(192, 1)
               }
             }
           }
-          if (sender) {
-            // every lane's stores into the partner's buffer, then one arrival per warp
-            fence_acq_rel_cluster();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(rx), rank + 1));
-          }
           if (step == 2) {
             // this warp's 32 rows of X' (4 boxes of 32 columns) from shared memory to X;
             // the prefetch buffer is released once the stores have read it
@@ -375,7 +270,7 @@ __global__ void __launch_bounds__(192, 1)
               bulk_wait_read0();
             }
           }
-          if (step > 0 && !receiver) {
+          if (step > 0) {
             __syncwarp();
             if (lane == 0) mbar_arrive(eempty);
             ++e_use;

@@ -22,7 +22,7 @@
 // momentum / Muon, L2 normalisation) and "Order of operations".
 #include <algorithm>
 
-#include "epi_finish.cuh"
+#include "apply_mlp.cuh"
 #include "epilogues.cuh"
 #include "ns_fused.cuh"
 #include "token_pair.cuh"
@@ -62,7 +62,6 @@ struct Dims {
   bool direct;  // unsplit gradients go straight into U (and M): no partials, no reduction
   bool src_t;  // Newton-Schulz input is the transpose of the gradient-layout source
   bool token_pairs;  // token phase (and, with tile_rows 512, weight gradients) on CTA pairs
-  bool fused_finish;  // the weight-gradient epilogue also takes the step and writes the weights
 };
 
 int bn_for(int n) { return n % 256 == 0 ? 256 : n % 128 == 0 ? 128 : 64; }
@@ -95,7 +94,6 @@ Dims dims_of(const Plan& p) {
   // most two contributions per row (order-independent)
   D.direct = D.splits == 1 && !(muon && D.grad_bn != c.d);
   D.token_pairs = (c.flags & TTT_FLAG_SINGLE_CTA) == 0;
-  D.fused_finish = p.off[kNumBBuf + 3] != 0;
   return D;
 }
 
@@ -643,42 +641,6 @@ int rmse_scale(Ctx& c, bf16* DY, int t0, int n) {
   return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
 }
 
-// Unsplit weight gradients whose epilogue also finishes the weights (EpiGradFinish):
-// problem 0 = G2 = V^T H' (rows of W2), problem 1 = G13 = dZ13^T X; N = d = h.
-int grad_finish(Ctx& c, const TM& tH, const TM& tD, const TM& tXmn, int rows1, int t0, int xoff) {
-  const Plan& p = c.p;
-  const Dims& D = c.D;
-  const ttt_config& cfg = p.cfg;
-  const bool mom = cfg.opt == TTT_OPT_MOMENTUM;
-  EpiGradFinish ep;
-  ep.Wf = c.v.at<float>(p, xWf);
-  ep.M = mom ? c.v.at<float>(p, xMom) : nullptr;
-  ep.First = c.v.at<bf16>(p, xFirst);
-  ep.W2 = c.v.at<bf16>(p, xW2);
-  ep.W2T = c.v.at<bf16>(p, xW2T);
-  ep.status = c.v.status;
-  ep.P = p.P;
-  ep.d = D.d;
-  ep.h = D.h;
-  ep.R1 = D.R1;
-  ep.GR = D.GR;
-  ep.swiglu = cfg.inner == TTT_INNER_SWIGLU;
-  ep.beta = cfg.momentum;
-  ep.lr = cfg.lr;
-  ep.rownorm = (cfg.flags & TTT_FLAG_WEIGHT_L2NORM) != 0;
-  ep.hold_w2 = (cfg.flags & TTT_FLAG_FIRST_LAYER_ONLY) != 0;
-  ep.row0[0] = 0;
-  ep.row0[1] = D.h;
-  ep.rows[0] = D.d;
-  ep.rows[1] = rows1;
-  TcGeom g = geom(D.d / 128, rows1 / 128, 1, D.Cp / 64, D.Z, 1);
-  g.a0.k = t0;    // V rows of the chunk
-  g.b1.k = xoff;  // keys (or their normalised copy)
-  StageCtx stage(kStageWeightGrad);
-  if (D.d == 256) return gemm<256, 0, true, true, 2, 4, 4>(c.tVmn, tH, tD, tXmn, g, ep, c.v.status, c.st, true);
-  return gemm<128, 0, true, true, 2, 6, 4>(c.tVmn, tH, tD, tXmn, g, ep, c.v.status, c.st, true);
-}
-
 // Token phase of the negative-dot update: activations H' and dZ(13) of chunk
 // tokens [t0, t0+n) for the weight-gradient GEMMs (token_phase.cuh).
 int token_phase(Ctx& c, const TM& tX, int xoff, int t0, int n, bf16* Hp, bf16* dZ, bool swiglu) {
@@ -775,14 +737,12 @@ int update_chunk(Ctx& c, int t0, int n) {
     TM tH, tD;
     TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
     TRY(tmap(&tD, A1, 2, 2 * h, Cp, Z, 64));
-    if (D.fused_finish) return grad_finish(c, tH, tD, *tXmn, 2 * h, t0, xoff);
     TRY(grad_gemm(c, tH, c.tVmn, tD, *tXmn, h, 2 * h, h, t0, xoff));
   } else if (cfg.inner == TTT_INNER_MLP2_GELU && cfg.loss == TTT_LOSS_NEG_DOT) {
     TRY(token_phase(c, *tX, xoff, t0, n, A0, A1, false));
     TM tH, tD;
     TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
     TRY(tmap(&tD, A1, 2, h, Cp, Z, 64));
-    if (D.fused_finish) return grad_finish(c, tH, tD, *tXmn, h, t0, xoff);
     TRY(grad_gemm(c, tH, c.tVmn, tD, *tXmn, h, h, h, t0, xoff));
   } else if (cfg.inner == TTT_INNER_MLP2_GELU) {  // MSE
     // Z = X W1^T -> H = GELU(Z), G' = GELU'(Z)
@@ -857,6 +817,33 @@ int apply_rows(Ctx& c, int row0, int rows) {
     else TRY((gemm<64, 0, false, false, 2, 4, 8>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, eo, status, c.st, true)));
     return TTT_OK;
   }
+  if (d == 64 || d == 128 || d == 256) {
+    // one kernel, hidden layer on chip (apply_mlp.cuh)
+    const bool swiglu = cfg.inner == TTT_INNER_SWIGLU;
+    TM tf, tw;
+    TRY(tmap(&tf, c.v.at<bf16>(p, xFirst), 2, d, D.R1, Z, swiglu ? 256 : 128));
+    TRY(tmap(&tw, c.v.at<bf16>(p, xW2), 2, h, d, Z, d));
+    if (c.tQ.box != 128) return TTT_ERR_INVALID_ARG;
+    ApplyGeom ag;
+    ag.m_tiles = mt;
+    ag.batches = Z;
+    ag.hblocks = h / 128;
+    ag.rows_valid = rows;
+    ag.row0 = row0;
+    ag.o_zs = int64_t(D.Nq) * d;
+    StageScope sc(kStageApply, c.st);
+    cudaError_t e = cudaErrorInvalidValue;
+    if (swiglu) {
+      e = d == 256 ? launch_apply_mlp<true, 256>(c.tQ.m, tf.m, tw.m, ag, O, status, c.st)
+          : d == 128 ? launch_apply_mlp<true, 128>(c.tQ.m, tf.m, tw.m, ag, O, status, c.st)
+                     : launch_apply_mlp<true, 64>(c.tQ.m, tf.m, tw.m, ag, O, status, c.st);
+    } else {
+      e = d == 256 ? launch_apply_mlp<false, 256>(c.tQ.m, tf.m, tw.m, ag, O, status, c.st)
+          : d == 128 ? launch_apply_mlp<false, 128>(c.tQ.m, tf.m, tw.m, ag, O, status, c.st)
+                     : launch_apply_mlp<false, 64>(c.tQ.m, tf.m, tw.m, ag, O, status, c.st);
+    }
+    return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+  }
   bf16* Hq = c.v.at<bf16>(p, xHq);
   if (cfg.inner == TTT_INNER_SWIGLU) {
     EpiApplyAct<true> e{Hq, h, rows, int64_t(D.Rq) * h};
@@ -883,7 +870,7 @@ int apply_rows(Ctx& c, int row0, int rows) {
 // Weight-gradient launch shape: split-K count and output tile height (256 rows
 // = two accumulators sharing B, when the rows allow it and the tiles alone keep
 // the SMs busy).
-void choose_grad_shape(const Plan& p, int Cp, int* splits, int* tile_rows, int* grad_bn, int* fused) {
+void choose_grad_shape(const Plan& p, int Cp, int* splits, int* tile_rows, int* grad_bn) {
   const ttt_config& c = p.cfg;
   const int d = c.d, h = c.h;
   const int bnd = bn_for(d);
@@ -912,14 +899,6 @@ void choose_grad_shape(const Plan& p, int Cp, int* splits, int* tile_rows, int* 
   const bool muon = c.opt == TTT_OPT_MUON || c.opt == TTT_OPT_MOMENTUM_MUON;
   *grad_bn = bnd;
   if (*splits == 1 && !muon && *tile_rows == 128 && tiles < units && bnd >= 128) *grad_bn = bnd / 2;
-  // Unsplit, Muon-free negative-dot updates whose rows fit one tile (d = h <= 256) finish
-  // the weights in the gradient epilogue: one launch instead of three per chunk.
-  *fused = 0;
-  const bool token_path = c.loss == TTT_LOSS_NEG_DOT && (c.inner == TTT_INNER_SWIGLU || c.inner == TTT_INNER_MLP2_GELU);
-  if (token_path && *splits == 1 && !muon && *tile_rows == 128 && d == h && (d == 128 || d == 256)) {
-    *fused = 1;
-    *grad_bn = d;
-  }
 }
 
 }  // namespace
@@ -937,12 +916,11 @@ int plan_layout_bf16(Plan* p) {
   const bool muon = c.opt == TTT_OPT_MUON || c.opt == TTT_OPT_MOMENTUM_MUON;
   if (muon && (d % 128 != 0 || (c.inner != TTT_INNER_LINEAR && h % 128 != 0))) return TTT_ERR_UNSUPPORTED;
   const int Cp = (p->chunk + 127) / 128 * 128;
-  int splits = 1, tile_rows = 128, grad_bn = 64, fused = 0;
-  choose_grad_shape(*p, Cp, &splits, &tile_rows, &grad_bn, &fused);
+  int splits = 1, tile_rows = 128, grad_bn = 64;
+  choose_grad_shape(*p, Cp, &splits, &tile_rows, &grad_bn);
   p->off[kNumBBuf] = size_t(splits);
   p->off[kNumBBuf + 1] = size_t(tile_rows);
   p->off[kNumBBuf + 2] = size_t(grad_bn);
-  p->off[kNumBBuf + 3] = size_t(fused);
   const Dims D = dims_of(*p);
   const int64_t Z = D.Z, P = p->P, GR = D.GR, nm = int64_t(D.m) * D.n, mm = int64_t(D.m) * D.m;
   const int64_t ZK = Z * D.nmat;
@@ -963,7 +941,7 @@ int plan_layout_bf16(Plan* p) {
       act ? Z * Cp * 2 * h * 2 : 0,
       mlp_mse ? Z * Cp * h * 2 : 0,
       (mlp_mse || !act) ? Z * Cp * d * 2 : 0,
-      act ? Z * D.Rq * h * 2 : 0,
+      (act && d != 64 && d != 128 && d != 256) ? Z * D.Rq * h * 2 : 0,  // two-GEMM apply only (d = 512)
       (c.flags & TTT_FLAG_KEY_INSTNORM) ? Z * (Cp / 128) * d * 2 * 4 : 0,
       muon ? ZK * nm * 4 : 0,
       muon ? ZK * nm * 4 : 0,
@@ -1053,16 +1031,15 @@ extern "C" int ttt_token_pair_capacity(int swiglu) {
 extern "C" int ttt_plan_info(const ttt_handle* h, int* info, int n) {
   if (!h || !info || n < 0) return TTT_ERR_INVALID_ARG;
   const ttt::Plan& p = h->plan;
-  int v[8] = {static_cast<int>(p.path), static_cast<int>(p.chunk), static_cast<int>(p.nchunks), 0, 0, 0, 0, 0};
+  int v[7] = {static_cast<int>(p.path), static_cast<int>(p.chunk), static_cast<int>(p.nchunks), 0, 0, 0, 0};
   if (p.path == ttt::kPathBf16) {
     const ttt::Dims D = ttt::dims_of(p);
     v[3] = D.splits;
     v[4] = D.tile_rows;
     v[5] = D.grad_bn;
     v[6] = D.direct ? 1 : 0;
-    v[7] = D.fused_finish ? 1 : 0;
   }
-  const int m = n < 8 ? n : 8;
+  const int m = n < 7 ? n : 7;
   for (int i = 0; i < m; ++i) info[i] = v[i];
   return m;
 }
