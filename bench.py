@@ -42,6 +42,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 CPU_SAMPLE_TOKENS = {
     "tiny_mlp2_n196_fp32": 196, "vit3s_1248_mlp2_n6084": 6084, "lact_lm_causal_n32k_c2048": 16384,
     "lact_nvs_n196k_d512": 65536, "lact_scene_n1m_c131k": 32768, "vit3s_1248_dwconv_n6084": 8 * 6084,
+    "vit3s_1248_glu_n6084": 6084,
 }
 
 
@@ -59,6 +60,8 @@ def algorithmic_flops(cfg) -> dict:
                 "apply": float(BH) * Nq * 2 * kk * d}
     if kind == "swiglu":  # token phase: Z1, Z3, V W2; weight grads: G2, G1, G3
         tok, grad, app = 6 * d * h, 6 * d * h, 6 * d * h
+    elif kind == "glu":  # token phase: [Zb | Za] = X [Wb; Wa]^T; grads: [Gb; Ga] = dZ^T X; apply: Q [Wb; Wa]^T
+        tok, grad, app = 4 * d * d, 4 * d * d, 4 * d * d
     elif kind == "mlp2_gelu":  # token phase: Z, [V_hat], dH; grads: G2, G1
         tok = (6 if loss in ("mse", "rmse") else 4) * d * h
         grad, app = 4 * d * h, 4 * d * h

@@ -22,6 +22,9 @@
  *                             F(X)[(y,x),c] = sum_{a,b<k} Wc[c][a k + b] X[(y+a-k/2, x+b-k/2), c]
  *                             over the grid_h x grid_w token grid (raster order), zero outside
  *                             (ViT3 digest, section 03, guideline 6 and inner-model table)
+ *        TTT_INNER_GLU        [Wa (d x d) | Wb (d x d)]        F(x) = (x Wa^T) * SiLU(x Wb^T)
+ *                             the simplified GLU (ViT3 digest, section 03, inner-model table;
+ *                             no biases, no output projection; Wa the linear branch, Wb the gate)
  *   - Q [B,H,Nq,d], K [B,H,N,d], V [B,H,N,d] and O [B,H,Nq,d] in `dtype`
  *     (fp32 or bf16); eta [B,H,N] fp32; W0 [H,P] fp32 (shared by every batch
  *     entry; [B,H,P] with TTT_FLAG_W0_PER_BATCH); W_out [B,H,P] fp32.
@@ -78,9 +81,11 @@ typedef enum {
   TTT_INNER_LINEAR = 0,
   TTT_INNER_MLP2_GELU = 1,
   TTT_INNER_SWIGLU = 2,
-  TTT_INNER_DWCONV = 3 /* the whole grid is one non-causal chunk (Nq == N, queries on the same grid);
-                          loss MSE or NEG_DOT, optimizer GD or MOMENTUM, no key instance-norm;
-                          other combinations return TTT_ERR_UNSUPPORTED */
+  TTT_INNER_DWCONV = 3, /* the whole grid is one non-causal chunk (Nq == N, queries on the same grid);
+                           loss MSE or NEG_DOT, optimizer GD or MOMENTUM, no key instance-norm;
+                           other combinations return TTT_ERR_UNSUPPORTED */
+  TTT_INNER_GLU = 4      /* bf16 only; loss MSE or NEG_DOT, optimizer GD or MOMENTUM; h is ignored
+                           (other combinations return TTT_ERR_UNSUPPORTED) */
 } ttt_inner_kind;
 typedef enum {
   TTT_LOSS_MSE = 0,      /* sum_i eta_i ||F(k_i) - v_i||^2 / (n d) over the chunk's n tokens */

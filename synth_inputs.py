@@ -13,7 +13,7 @@ Tensor layouts (row-major, contiguous):
     linear    [W  (d x d)]
     mlp2_gelu [W1 (h x d) | W2 (d x h)]
     swiglu    [W1 (h x d) | W3 (h x d) | W2 (d x h)]
-    glu       [Wa (d x d) | Wb (d x d)]   (oracle only; the CUDA path runs it as a
+    glu       [Wa (d x d) | Wb (d x d)]   (bf16: TTT_INNER_GLU; the fp32 path runs it as a
               SwiGLU with h = d, W1 = Wb, W3 = Wa, W2 = I and the first-layer-only flag)
     dwconv    [Wc (d x k*k)]              (oracle only: one k x k kernel per channel)
 
@@ -78,6 +78,11 @@ WORKLOADS = {
                                  inner="swiglu", loss="neg_dot", opt="momentum_muon", momentum=0.9,
                                  dtype="bf16", weight_l2norm=True, eta_mode="per_token",
                                  data="lact", seed=5000),
+    # the GLU heads of a ViT^3-S-like 1248^2 layer: B8, 5 heads (the sixth is the DWConv head),
+    # N6084, d64, F(x) = (x Wa^T) * SiLU(x Wb^T), the ViT^3 recipe (dot loss, one full-batch step,
+    # eta = 1)
+    "vit3s_1248_glu_n6084": dict(B=8, H=5, N=6084, d=64, h=64, inner="glu", loss="neg_dot", opt="gd",
+                                 dtype="bf16", eta_mode="scalar", eta_scalar=1.0, data="vit", seed=7000),
     # the DWConv head of a ViT^3-S-like 1248^2 layer: B8, one head, the 78 x 78 token grid,
     # d64, 3 x 3 depthwise kernels, the ViT^3 recipe (dot loss, one full-batch step, eta = 1)
     "vit3s_1248_dwconv_n6084": dict(B=8, H=1, N=6084, grid_h=78, grid_w=78, ksize=3, d=64, h=64,

@@ -44,7 +44,7 @@ def test_every_workload_configuration_is_accepted(name):
     st, h = _create(binding.make_config(cfg))
     assert st == 0, binding.status_string(st)
     P = binding.LIB.ttt_param_count(h)
-    expect = ({"linear": 1, "mlp2_gelu": 2, "swiglu": 3}[cfg["inner"]] * cfg["d"] * cfg["h"]
+    expect = ({"linear": 1, "mlp2_gelu": 2, "swiglu": 3, "glu": 2}[cfg["inner"]] * cfg["d"] * cfg["h"]
               if cfg["inner"] != "dwconv" else cfg["d"] * cfg["ksize"] ** 2)
     assert P == expect
     assert binding.LIB.ttt_workspace_size(h) >= 256

@@ -22,6 +22,9 @@ CLOSED_FORM_GFLOP = {
     # B1 H4 N1029120 (8 chunks) Nq8040 d256 h512, SwiGLU + dot, momentum + Muon on 256 x 512
     "lact_scene_n1m_c131k": 4 * (12 * 1029120 * 256 * 512 + 6 * 8040 * 256 * 512
                                  + 8 * 3 * 5 * (4 * 256 ** 2 * 512 + 2 * 256 ** 3)) / 1e9,
+    # B8 H5 N6084 d64, GLU + dot: two d x d products on the keys (4 N d^2), their gradients
+    # (4 N d^2) and two on the queries (4 Nq d^2)
+    "vit3s_1248_glu_n6084": 40 * (8 * 6084 * 64 * 64 + 4 * 6084 * 64 * 64) / 1e9,
     # B8 H1 N6084 d64, 3 x 3 DWConv + dot: tap gradients 2 k^2 N d, apply 2 k^2 Nq d
     "vit3s_1248_dwconv_n6084": 8 * (2 * 9 * 6084 * 64 * 2) / 1e9,
 }

@@ -168,3 +168,27 @@ def test_random_configurations_get_a_status_and_consistent_sizes(cfg):
             assert info["splits"] >= 1 and info["tile_rows"] in (128, 256, 512) and info["grad_bn"] in (32, 64, 128, 256)
     finally:
         binding.LIB.ttt_destroy(h)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dtype="bf16"), 0),
+    (dict(dtype="bf16", loss="mse", opt="momentum", chunk=256, causal=1), 0),
+    (dict(dtype="f32"), -2),                   # the fp32 path runs the GLU in its SwiGLU form
+    (dict(dtype="bf16", opt="muon"), -2),
+    (dict(dtype="bf16", opt="momentum_muon"), -2),
+    (dict(dtype="bf16", loss="rmse"), -2),
+    (dict(dtype="bf16", d=96), -2),            # channels in whole 64-channel blocks
+])
+def test_glu_combinations(kw, status):
+    import ctypes
+    base = dict(B=1, H=2, N=1024, d=128, h=7, inner="glu", loss="neg_dot", opt="gd")
+    base.update(kw)
+    cfg = make_config(**base)
+    c = binding.make_config(cfg)
+    h = ctypes.c_void_p()
+    st = binding.LIB.ttt_create(ctypes.byref(c), ctypes.byref(h))
+    assert st == status, binding.status_string(st)
+    if st == 0:
+        # two d x d matrices (h is ignored), 64-channel blocks of gate and linear rows
+        assert binding.LIB.ttt_param_count(h) == 2 * cfg["d"] ** 2
+        binding.LIB.ttt_destroy(h)

@@ -3,10 +3,12 @@
 modules of the ViT3 design).  fp32 inputs within 1e-4, bf16 inputs within 2e-2
 (relative Frobenius error per output and per weight tensor).
 
-* The simplified GLU FC(x) * SiLU(FC(x)) (F1) runs as a SwiGLU with h = d, W1 = the
-  gate's matrix Wb, W3 = the linear branch's Wa, W2 = I and the first-layer-only flag;
-  it is checked against the oracle's own GLU model, with the ViT3 recipe (dot loss,
-  one full-batch step, learning rate 1) and with momentum + Muon over several chunks.
+* The simplified GLU FC(x) * SiLU(FC(x)) (F1): as its own inner model on the tensor
+  cores (bf16, any multiple of 64 channels, ViT3's 64 included), and in its SwiGLU form
+  (h = d, W1 = the gate's matrix Wb, W3 = the linear branch's Wa, W2 = I and the
+  first-layer-only flag) on both dtypes; both against the oracle's own GLU model, with
+  the ViT3 recipe (dot loss, one full-batch step, learning rate 1) and with momentum
+  (+ Muon in the SwiGLU form) over several chunks.
 * DWConv (F2): a 'same' depthwise k x k cross-correlation over the token grid whose
   kernels take the layer's gradient step.
 * The RMSE inner loss: the chunk's RMSE is reduced on the device, then scales the MSE
@@ -65,6 +67,53 @@ def test_glu_as_swiglu_against_the_oracle_glu(kw):
     _check(errs, tol)
     assert np.isfinite(Og).all()
     assert np.array_equal(Wg[..., 2 * P:], np.broadcast_to(np.eye(d).reshape(-1), Wg[..., 2 * P:].shape))
+
+
+# The GLU as its own inner model on the tensor cores (TTT_INNER_GLU, bf16): 64-channel
+# blocks [Wb rows | Wa rows] per GEMM tile, so ViT3's own 64-channel heads run there, and
+# no W2 = I products.  Against the oracle's GLU.
+GLU_NATIVE_CASES = [
+    # the ViT3 recipe at ViT3's head width
+    dict(d=64, N=600, opt="gd", eta_mode="scalar", eta_scalar=1.0, data="vit"),
+    dict(d=64, N=333, Nq=150, opt="gd", eta_mode="scalar", eta_scalar=1.0, data="vit", key_instnorm=True),
+    dict(d=128, N=700, opt="momentum", chunk=256, weight_l2norm=True, eta_mode="per_token"),
+    dict(d=64, N=450, opt="momentum", chunk=128, causal=1, weight_l2norm=True, eta_mode="per_token"),
+    dict(d=192, N=520, opt="gd", loss="mse", eta_mode="scalar", eta_scalar=1.0, data="vit"),
+    dict(d=64, N=300, opt="momentum", loss="mse", chunk=128, eta_mode="per_token", epochs=2),
+]
+
+
+@pytest.mark.parametrize("kw", GLU_NATIVE_CASES, ids=lambda kw: "-".join(f"{v}" for v in kw.values()))
+def test_glu_inner_model_against_the_oracle(kw):
+    base = dict(B=2, H=2, inner="glu", loss="neg_dot", dtype="bf16", data="lact", seed=81)
+    base.update(kw)
+    base["h"] = base["d"]
+    cfg = make_config(**base)
+    _check(compare(cfg), TOL["bf16"])
+
+
+def test_glu_matches_its_swiglu_form_on_the_gpu():
+    # the native GLU and its SwiGLU form (W1 = Wb, W3 = Wa, W2 = I, first layer only) run
+    # different kernels on the same bf16 inputs: their results agree to bf16 rounding
+    kw = dict(B=1, H=2, N=500, d=128, h=128, loss="neg_dot", opt="gd", dtype="bf16", data="vit",
+              eta_mode="scalar", eta_scalar=1.0, seed=83)
+    cfg_glu = make_config(inner="glu", **kw)
+    x = gen_inputs(cfg_glu)
+    d, P = 128, 128 * 128
+    Og, Wg = run_gpu(cfg_glu, x)
+    xs = dict(x)
+    xs["W0"] = torch.cat([x["W0"][:, P:], x["W0"][:, :P], torch.eye(d).reshape(1, -1).expand(2, -1)], dim=1).contiguous()
+    Os, Ws = run_gpu(make_config(inner="swiglu", first_layer_only=True, **kw), xs)
+    assert rel_fro(Og, Os) < 1e-2
+    assert rel_fro(Wg[..., :P], Ws[..., P:2 * P]) < 1e-2 and rel_fro(Wg[..., P:], Ws[..., :P]) < 1e-2
+
+
+def test_glu_bench_workload_at_full_size():
+    # the GLU heads of the ViT3-S-like 1248^2 layer (B8 H5 N6084 d64): every head
+    from synth_inputs import workload
+    errs = compare(workload("vit3s_1248_glu_n6084"))
+    print({k: f"{v:.2e}" for k, v in errs.items()})
+    _check(errs, TOL["bf16"])
 
 
 # ---------------------------------------------------------------- RMSE loss

@@ -22,7 +22,7 @@ TTT_ERR_NONFINITE = -4
 TTT_ERR_TIMEOUT = -5
 TTT_ERR_WORKSPACE = -6
 
-INNER = {"linear": 0, "mlp2_gelu": 1, "swiglu": 2, "dwconv": 3}
+INNER = {"linear": 0, "mlp2_gelu": 1, "swiglu": 2, "dwconv": 3, "glu": 4}
 LOSS = {"mse": 0, "neg_dot": 1, "rmse": 2}
 OPT = {"gd": 0, "momentum": 1, "muon": 2, "momentum_muon": 3}
 DTYPE = {"f32": 0, "bf16": 1}

@@ -23,6 +23,7 @@
 #include <algorithm>
 
 #include "apply_mlp.cuh"
+#include "epi_glu.cuh"
 #include "epilogues.cuh"
 #include "ns_fused.cuh"
 #include "token_pair.cuh"
@@ -52,7 +53,7 @@ enum BBuf {
   xAct2,   // bf16 [Z][Cp][h]  (GELU' for MSE)
   xDY,     // bf16 [Z][Cp][d]  (dL/dV_hat for MSE / linear)
   xHq,     // bf16 apply hidden [Z][Rq][h]
-  xKstat,  // fp32 key-norm partial sums [Z][Cp/128][d][2]
+  xKstat,  // fp32 key-norm partial sums [Z][Cp/128][d][2], then [Z][d][2] mean and 1/std
   xNX, xNXT, xNX2, xNXT2, xNS, xNT,  // fp32 Newton-Schulz buffers [Z*nmat][...]
   kNumBBuf
 };
@@ -80,6 +81,7 @@ Dims dims_of(const Plan& p) {
   switch (c.inner) {
     case TTT_INNER_LINEAR: D.GR = c.d; D.R1 = c.d; D.nmat = 1; break;
     case TTT_INNER_MLP2_GELU: D.GR = 2 * c.h; D.R1 = c.h; D.nmat = 2; break;
+    case TTT_INNER_GLU: D.GR = 2 * c.d; D.R1 = 2 * c.d; D.nmat = 2; break;
     default: D.GR = 3 * c.h; D.R1 = 2 * c.h; D.nmat = 3; break;
   }
   const int rows_src = c.inner == TTT_INNER_LINEAR ? c.d : c.h;
@@ -105,11 +107,16 @@ struct RowMap {
   int inner, d, h, GR;
   int64_t P;
   __host__ __device__ int nrows() const {
-    return inner == TTT_INNER_LINEAR ? d : inner == TTT_INNER_MLP2_GELU ? h + d : 2 * h + d;
+    return inner == TTT_INNER_LINEAR ? d : inner == TTT_INNER_MLP2_GELU ? h + d : inner == TTT_INNER_GLU ? 2 * d
+                                                                                                          : 2 * h + d;
   }
   // matrix index k, row inside it, row length, offset of the matrix in the packed layout
   __device__ void locate(int R, int& k, int& r, int& len, int64_t& off) const {
     if (inner == TTT_INNER_LINEAR) { k = 0; r = R; len = d; off = 0; return; }
+    if (inner == TTT_INNER_GLU) {  // [Wa | Wb], both d x d
+      k = R < d ? 0 : 1; r = R < d ? R : R - d; len = d; off = int64_t(k) * d * d;
+      return;
+    }
     if (inner == TTT_INNER_MLP2_GELU) {
       if (R < h) { k = 0; r = R; len = d; off = 0; }
       else { k = 1; r = R - h; len = h; off = int64_t(h) * d; }
@@ -119,16 +126,20 @@ struct RowMap {
     else if (R < 2 * h) { k = 1; r = R - h; len = d; off = int64_t(h) * d; }
     else { k = 2; r = R - 2 * h; len = h; off = 2 * int64_t(h) * d; }
   }
-  __device__ bool is_w2(int k) const { return inner != TTT_INNER_LINEAR && k == (inner == TTT_INNER_SWIGLU ? 2 : 1); }
+  __device__ bool is_w2(int k) const {
+    return (inner == TTT_INNER_MLP2_GELU || inner == TTT_INNER_SWIGLU) && k == (inner == TTT_INNER_SWIGLU ? 2 : 1);
+  }
   // gradient-layout row of row r of a first-layer matrix k (W1, W3 or linear W)
   __device__ int grad_row(int k, int r) const {
     if (inner == TTT_INNER_LINEAR) return r;
+    if (inner == TTT_INNER_GLU) return 128 * (r / 64) + (k == 0 ? 64 : 0) + (r % 64);  // [Wb 64 | Wa 64] blocks
     if (inner == TTT_INNER_MLP2_GELU) return h + r;
     return h + 256 * (r / 128) + (k == 1 ? 128 : 0) + (r % 128);
   }
   // bf16 first-layer row of row r of matrix k
   __device__ int first_row(int k, int r) const {
     if (inner == TTT_INNER_SWIGLU) return 256 * (r / 128) + (k == 1 ? 128 : 0) + (r % 128);
+    if (inner == TTT_INNER_GLU) return 128 * (r / 64) + (k == 0 ? 64 : 0) + (r % 64);
     return r;
   }
 };
@@ -164,13 +175,17 @@ __global__ void finish_rows_kernel(RowMap rm, int mode, float lr, bool rownorm, 
     mode = 0;
     rownorm = false;
   }
+  // rows of up to 1024 stay in registers (lane element q is column lane + 32 q), so every
+  // load of the row is issued before the norm's reduction
+  const float* u = nullptr;  // the update row (stride 1), or W2's column of the gradient layout
+  int64_t ustride = 1;
   if (mode == 1) {
     const float* Uz = U + int64_t(z) * rm.GR * rm.d;
     if (!w2) {
-      const float* u = Uz + int64_t(rm.grad_row(k, r)) * rm.d;
-      for (int i = lane; i < len; i += 32) w[i] -= lr * u[i];
+      u = Uz + int64_t(rm.grad_row(k, r)) * rm.d;
     } else {  // W2 row r = column r of the G2^T rows [0, h)
-      for (int i = lane; i < len; i += 32) w[i] -= lr * Uz[int64_t(i) * rm.d + r];
+      u = Uz + r;
+      ustride = rm.d;
     }
   } else if (mode == 2) {
     const int64_t mn = int64_t(m) * n;
@@ -178,34 +193,64 @@ __global__ void finish_rows_kernel(RowMap rm, int mode, float lr, bool rownorm, 
     const float* XTk = XT + (int64_t(z) * nmat + k) * mn;
     // result in the source orientation is (src_t ? XT : X); W2 rows are its columns
     const float* src = w2 ? (src_t ? Xk : XTk) : (src_t ? XTk : Xk);
-    const float* u = src + int64_t(r) * len;
-    for (int i = lane; i < len; i += 32) w[i] -= lr * u[i];
+    u = src + int64_t(r) * len;
   }
-  float inv = 1.0f;
-  if (rownorm) {
-    float s = 0.f;
-    for (int i = lane; i < len; i += 32) s += w[i] * w[i];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    inv = 1.0f / fmaxf(sqrtf(s), 1e-12f);
-  }
+  const int r1 = rm.inner == TTT_INNER_SWIGLU ? 2 * rm.h
+                 : rm.inner == TTT_INNER_GLU   ? 2 * rm.d
+                 : rm.inner == TTT_INNER_LINEAR ? rm.d
+                                                : rm.h;
+  bf16* dst = !w2 ? First + (int64_t(z) * r1 +
+                             rm.first_row(k, r)) * rm.d
+                  : W2 + (int64_t(z) * rm.d + r) * rm.h;
+  float s = 0.f;
   bool bad = false;
-  if (!w2) {
-    bf16* f = First + (int64_t(z) * (rm.inner == TTT_INNER_SWIGLU ? 2 * rm.h : (rm.inner == TTT_INNER_LINEAR ? rm.d : rm.h)) +
-                       rm.first_row(k, r)) * rm.d;
-    for (int i = lane; i < len; i += 32) {
-      const float v = w[i] * inv;
-      w[i] = v;
-      bad |= !isfinite(v);
-      f[i] = __float2bfloat16_rn(v);
+  if (len <= 1024) {
+    float wv[32];
+#pragma unroll
+    for (int q = 0; q < 32; ++q) {
+      const int i = lane + 32 * q;
+      wv[q] = 0.f;
+      if (i < len) {
+        float x = w[i];
+        if (u) x -= lr * u[int64_t(i) * ustride];
+        wv[q] = x;
+        s += x * x;
+      }
     }
-  } else {
-    bf16* w2row = W2 + (int64_t(z) * rm.d + r) * rm.h;
+    float inv = 1.0f;
+    if (rownorm) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      inv = 1.0f / fmaxf(sqrtf(s), 1e-12f);
+    }
+#pragma unroll
+    for (int q = 0; q < 32; ++q) {
+      const int i = lane + 32 * q;
+      if (i < len) {
+        const float v = wv[q] * inv;
+        w[i] = v;
+        bad |= !isfinite(v);
+        dst[i] = __float2bfloat16_rn(v);
+      }
+    }
+  } else {  // longer rows: the step in place, then the norm and the copies
+    for (int i = lane; i < len; i += 32) {
+      float x = w[i];
+      if (u) x -= lr * u[int64_t(i) * ustride];
+      w[i] = x;
+      s += x * x;
+    }
+    float inv = 1.0f;
+    if (rownorm) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      inv = 1.0f / fmaxf(sqrtf(s), 1e-12f);
+    }
     for (int i = lane; i < len; i += 32) {
       const float v = w[i] * inv;
       w[i] = v;
       bad |= !isfinite(v);
-      w2row[i] = __float2bfloat16_rn(v);
+      dst[i] = __float2bfloat16_rn(v);
     }
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(status, kStatusNonFinite);
@@ -256,23 +301,31 @@ __global__ void keystats_kernel(int n, int d, const bf16* K, int64_t k_zs, int t
   }
 }
 
-// Pass 2: every CTA combines the block sums of all channels (in double: the biased
-// variance is E[k^2] - E[k]^2) and normalises its 128 tokens: Kn = (k - mean) /
-// sqrt(var + eps), zeros for rows past the chunk.
-__global__ void keynorm_kernel(int n, int d, const bf16* K, int64_t k_zs, int t0, float eps, const float* part,
-                               bf16* Kn, int64_t kn_zs) {
+// Pass 2: per (z, channel), the block sums combined in block order (in double: the
+// biased variance is E[k^2] - E[k]^2) into the mean and 1/sqrt(var + eps).
+__global__ void keystats_final_kernel(int n, int d, int nb, float eps, const float* part, float* stats) {
+  const int z = blockIdx.y;
+  const int ch = blockIdx.x * blockDim.x + threadIdx.x;
+  if (ch >= d) return;
+  double s = 0.0, q = 0.0;
+  for (int b = 0; b < nb; ++b) {
+    s += part[((int64_t(z) * nb + b) * d + ch) * 2];
+    q += part[((int64_t(z) * nb + b) * d + ch) * 2 + 1];
+  }
+  const double mean = s / n;
+  const double var = fmax(q / n - mean * mean, 0.0);
+  stats[(int64_t(z) * d + ch) * 2] = static_cast<float>(mean);
+  stats[(int64_t(z) * d + ch) * 2 + 1] = static_cast<float>(1.0 / sqrt(var + eps));
+}
+
+// Pass 3: normalise the chunk's keys, Kn = (k - mean) * rstd, zeros for rows past the chunk.
+__global__ void keynorm_kernel(int n, int d, const bf16* K, int64_t k_zs, int t0, const float* stats, bf16* Kn,
+                               int64_t kn_zs) {
   extern __shared__ float st[];  // [d] mean, [d] rstd
-  const int z = blockIdx.y, blk = blockIdx.x, nb = gridDim.x;
+  const int z = blockIdx.y, blk = blockIdx.x;
   for (int ch = threadIdx.x; ch < d; ch += blockDim.x) {
-    double s = 0.0, q = 0.0;
-    for (int b = 0; b < nb; ++b) {
-      s += part[((int64_t(z) * nb + b) * d + ch) * 2];
-      q += part[((int64_t(z) * nb + b) * d + ch) * 2 + 1];
-    }
-    const double mean = s / n;
-    const double var = fmax(q / n - mean * mean, 0.0);
-    st[ch] = static_cast<float>(mean);
-    st[d + ch] = static_cast<float>(1.0 / sqrt(var + eps));
+    st[ch] = stats[(int64_t(z) * d + ch) * 2];
+    st[d + ch] = stats[(int64_t(z) * d + ch) * 2 + 1];
   }
   __syncthreads();
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -488,9 +541,14 @@ struct Ctx {
   int bn_first = 0;
 };
 
-// bf16 W2^T from the freshly written bf16 W2 (the token phase's B operand).
+// bf16 W2^T from the freshly written bf16 W2: the B operand of the single-CTA token
+// kernel and of the MSE path's dH = dY W2.  The pair token kernel reads W2 itself.
 int transpose_w2(Ctx& c) {
-  if (c.p.cfg.inner == TTT_INNER_LINEAR) return TTT_OK;
+  const ttt_config& cfg = c.p.cfg;
+  if (cfg.inner == TTT_INNER_LINEAR || cfg.inner == TTT_INNER_GLU) return TTT_OK;
+  if (cfg.loss == TTT_LOSS_NEG_DOT && c.D.token_pairs &&
+      (cfg.inner == TTT_INNER_SWIGLU ? token_pair_capacity<true>() : token_pair_capacity<false>()) > 0)
+    return TTT_OK;
   const Dims& D = c.D;
   cudaStream_t st = c.st;
   {
@@ -676,7 +734,7 @@ int token_phase(Ctx& c, const TM& tX, int xoff, int t0, int n, bf16* Hp, bf16* d
   if (pairs) {
     TM fh, wh;
     TRY(tmap(&fh, c.v.at<bf16>(c.p, xFirst), 2, d, D.R1, Z, swiglu ? 128 : 64));
-    TRY(tmap(&wh, c.v.at<bf16>(c.p, xW2T), 2, d, h, Z, 64));
+    TRY(tmap(&wh, c.v.at<bf16>(c.p, xW2), 2, h, d, Z, 64));  // W2 [d][h], MN-major 64 x 64 boxes
     g.m_tiles = (Cp + 255) / 256;
     e = swiglu ? launch_token_pair<true>(tX.m, fh.m, c.tV.m, wh.m, sH, sD, g, c.v.status, c.st)
                : launch_token_pair<false>(tX.m, fh.m, c.tV.m, wh.m, sH, sD, g, c.v.status, c.st);
@@ -709,9 +767,14 @@ int update_chunk(Ctx& c, int t0, int n) {
       StageScope _sc(kStageKeyNorm, st);
       keystats_kernel<<<gk, 256, 0, c.st>>>(n, d, K, int64_t(D.N) * d, t0, kst);
     }
+    float* kfin = kst + size_t(Z) * (Cp / 128) * d * 2;  // [Z][d][2] mean, rstd
     {
       StageScope _sc(kStageKeyNorm, st);
-      keynorm_kernel<<<gk, 256, 2 * d * sizeof(float), c.st>>>(n, d, K, int64_t(D.N) * d, t0, cfg.in_eps, kst, Kn,
+      keystats_final_kernel<<<dim3((d + 127) / 128, Z), 128, 0, c.st>>>(n, d, Cp / 128, cfg.in_eps, kst, kfin);
+    }
+    {
+      StageScope _sc(kStageKeyNorm, st);
+      keynorm_kernel<<<gk, 256, 2 * d * sizeof(float), c.st>>>(n, d, K, int64_t(D.N) * d, t0, kfin, Kn,
                                                                int64_t(Cp) * d);
     }
     TRY_CUDA(cudaGetLastError());
@@ -772,6 +835,16 @@ int update_chunk(Ctx& c, int t0, int n) {
     TRY(tmap(&tYmn, DY, 2, d, Cp, Z, 64));
     TRY(tmap(&tD, A1, 2, h, Cp, Z, 64));
     TRY(grad_gemm(c, tH, tYmn, tD, *tXmn, h, h, h, 0, xoff));
+  } else if (cfg.inner == TTT_INNER_GLU) {
+    // Z = X [Wb_blk; Wa_blk]^T per 64-channel block -> dZ (gate, linear), then G = dZ^T X
+    EpiGluGrad eg{A1, d, n, int64_t(Cp) * 2 * d, V, int64_t(D.N) * d, t0, c.io.eta, D.N, cfg.eta_scalar,
+                  cfg.loss == TTT_LOSS_MSE ? 1 : 0, 2.0f / (float(n) * float(d))};
+    TcGeom gz = geom(mt, 0, (2 * d) / 128, d / 64, Z, 1);
+    gz.a0.mn = xoff;
+    TRY((gemm<128, 0, false, false, 2, 4, 8>(*tX, c.tFirst, *tX, c.tFirst, gz, eg, status, c.st, true)));
+    TM tD;
+    TRY(tmap(&tD, A1, 2, 2 * d, Cp, Z, 64));
+    TRY(grad_gemm(c, tD, *tXmn, tD, *tXmn, 2 * d, 0, 0, xoff, 0));
   } else {  // linear
     if (cfg.loss != TTT_LOSS_NEG_DOT) {  // MSE, RMSE
       EpiMseGrad e2{DY, d, n, int64_t(Cp) * d, V, int64_t(D.N) * d, t0, c.io.eta, D.N, cfg.eta_scalar,
@@ -815,6 +888,13 @@ int apply_rows(Ctx& c, int row0, int rows) {
     if (bnd == 256) TRY((gemm<256, 0, false, false, 2, 4, 8>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, eo, status, c.st, true)));
     else if (bnd == 128) TRY((gemm<128, 0, false, false, 2, 4, 8>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, eo, status, c.st, true)));
     else TRY((gemm<64, 0, false, false, 2, 4, 8>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, eo, status, c.st, true)));
+    return TTT_OK;
+  }
+  if (cfg.inner == TTT_INNER_GLU) {  // O = za * SiLU(zb) straight from the first-layer tiles
+    EpiGluOut eo2{O, d, rows, row0, int64_t(D.Nq) * d, status};
+    TcGeom g = geom(mt, 0, (2 * d) / 128, d / 64, Z, 1);
+    g.a0.mn = row0;
+    TRY((gemm<128, 0, false, false, 2, 4, 8>(c.tQ, c.tFirst, c.tQ, c.tFirst, g, eo2, status, c.st, true)));
     return TTT_OK;
   }
   if (d == 64 || d == 128 || d == 256) {
@@ -874,8 +954,11 @@ void choose_grad_shape(const Plan& p, int Cp, int* splits, int* tile_rows, int* 
   const ttt_config& c = p.cfg;
   const int d = c.d, h = c.h;
   const int bnd = bn_for(d);
-  const int rows = c.inner == TTT_INNER_LINEAR ? d : c.inner == TTT_INNER_MLP2_GELU ? 2 * h : 3 * h;
-  const int r0 = c.inner == TTT_INNER_LINEAR ? d : h;
+  const int rows = c.inner == TTT_INNER_LINEAR ? d
+                   : c.inner == TTT_INNER_GLU ? 2 * d
+                   : c.inner == TTT_INNER_MLP2_GELU ? 2 * h
+                                                    : 3 * h;
+  const int r0 = c.inner == TTT_INNER_LINEAR ? d : c.inner == TTT_INNER_GLU ? 2 * d : h;
   const int kblocks = Cp / 64;
   // each split reduces at least 1024 tokens: below that the fp32 partials it writes
   // and the reduction reads cost more than the parallelism gains; chunks of at most
@@ -908,7 +991,12 @@ int plan_layout_bf16(Plan* p) {
   const int d = c.d, h = c.h;
   // supported shapes of the tensor-core path
   if (d % 64 != 0) return TTT_ERR_UNSUPPORTED;
-  if (c.inner != TTT_INNER_LINEAR && h % 128 != 0) return TTT_ERR_UNSUPPORTED;
+  const bool glu = c.inner == TTT_INNER_GLU;
+  if (c.inner != TTT_INNER_LINEAR && !glu && h % 128 != 0) return TTT_ERR_UNSUPPORTED;
+  // GLU: the plain and momentum steps with the dot or MSE loss (RMSE needs the chunk's whole
+  // loss before any gradient; Muon is not built for it)
+  if (glu && (c.loss == TTT_LOSS_RMSE || c.opt == TTT_OPT_MUON || c.opt == TTT_OPT_MOMENTUM_MUON))
+    return TTT_ERR_UNSUPPORTED;
   // the weight-gradient GEMMs tile their output rows (h per matrix, d for the linear
   // model) by 128
   if (c.inner == TTT_INNER_LINEAR && d % 128 != 0) return TTT_ERR_UNSUPPORTED;
@@ -925,7 +1013,7 @@ int plan_layout_bf16(Plan* p) {
   const int64_t Z = D.Z, P = p->P, GR = D.GR, nm = int64_t(D.m) * D.n, mm = int64_t(D.m) * D.m;
   const int64_t ZK = Z * D.nmat;
   const bool mlp_mse = c.inner == TTT_INNER_MLP2_GELU && c.loss != TTT_LOSS_NEG_DOT;  // MSE, RMSE
-  const bool act = c.inner != TTT_INNER_LINEAR;
+  const bool act = c.inner != TTT_INNER_LINEAR && !glu;  // a hidden layer and W2
   const int64_t bytes[kNumBBuf] = {
       Z * P * 4,
       Z * GR * d * 4,
@@ -938,11 +1026,11 @@ int plan_layout_bf16(Plan* p) {
       act ? Z * d * h * 2 : 0,
       (c.flags & TTT_FLAG_KEY_INSTNORM) ? Z * Cp * d * 2 : 0,
       act ? Z * Cp * h * 2 : 0,
-      act ? Z * Cp * 2 * h * 2 : 0,
+      (act || glu) ? Z * Cp * 2 * h * 2 : 0,  // dZ13 / dZ (GLU: h = d)
       mlp_mse ? Z * Cp * h * 2 : 0,
       (mlp_mse || !act) ? Z * Cp * d * 2 : 0,
       (act && d != 64 && d != 128 && d != 256) ? Z * D.Rq * h * 2 : 0,  // two-GEMM apply only (d = 512)
-      (c.flags & TTT_FLAG_KEY_INSTNORM) ? Z * (Cp / 128) * d * 2 * 4 : 0,
+      (c.flags & TTT_FLAG_KEY_INSTNORM) ? Z * (Cp / 128 + 1) * d * 2 * 4 : 0,  // block sums, then mean / rstd
       muon ? ZK * nm * 4 : 0,
       muon ? ZK * nm * 4 : 0,
       muon ? ZK * nm * 4 : 0,
@@ -976,12 +1064,13 @@ int run_bf16(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
   TRY(tmap(&c.tQ, io.Q, 2, d, D.Nq, Z, 128));
   bf16* First = c.v.at<bf16>(p, xFirst);
   const int bn_first = cfg.inner == TTT_INNER_SWIGLU ? 256
+                       : cfg.inner == TTT_INNER_GLU  ? 128
                        : cfg.inner == TTT_INNER_MLP2_GELU
                            ? (cfg.loss == TTT_LOSS_NEG_DOT ? 128 : bn_for(h))
                            : bn_for(d);
   c.bn_first = bn_first;
   TRY(tmap(&c.tFirst, First, 2, d, D.R1, Z, bn_first));
-  if (cfg.inner != TTT_INNER_LINEAR) {
+  if (cfg.inner == TTT_INNER_MLP2_GELU || cfg.inner == TTT_INNER_SWIGLU) {
     TRY(tmap(&c.tW2T, c.v.at<bf16>(p, xW2T), 2, d, h, Z, cfg.loss == TTT_LOSS_NEG_DOT ? 128 : bn_for(h)));
     TRY(tmap(&c.tW2, c.v.at<bf16>(p, xW2), 2, h, d, Z, bn_for(d)));
   }

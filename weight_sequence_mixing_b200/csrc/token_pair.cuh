@@ -2,6 +2,8 @@
 //
 // Same arithmetic as token_dot_kernel (token_phase.cuh): for every tile of chunk
 // tokens x 128 hidden units it forms P = V W2[:, blk] and Z13 = X [W1_blk; W3_blk]^T
+// (W2's columns are read straight from W2 [d][h] as an MN-major operand, so no W2^T
+// copy is needed)
 // and writes H' and dZ13 (MLP2: H' and dZ) for the weight-gradient GEMMs (LaCT
 // analysis, "Nonlinear memory complements local attention").
 //
@@ -40,7 +42,7 @@ struct PairShape {
   static constexpr int A_BYTES = 128 * 128;         // this CTA's 128 tokens x 64 bf16
   static constexpr int BZ_ROWS = SWIGLU ? 128 : 64;  // this CTA's half of the first-layer rows
   static constexpr int BZ_BYTES = BZ_ROWS * 128;
-  static constexpr int BP_ROWS = 64;  // this CTA's half of the 128 W2^T rows
+  static constexpr int BP_ROWS = 64;  // this CTA's half of the block's 128 W2 columns
   static constexpr int BP_BYTES = BP_ROWS * 128;
   static constexpr int Z_STAGE = A_BYTES + BZ_BYTES;
   static constexpr int P_STAGE = A_BYTES + BP_BYTES;
@@ -58,7 +60,7 @@ struct PairShape {
 template <bool SWIGLU>
 __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
     token_pair_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__ CUtensorMap tFirst,
-                      const __grid_constant__ CUtensorMap tV, const __grid_constant__ CUtensorMap tW2T,
+                      const __grid_constant__ CUtensorMap tV, const __grid_constant__ CUtensorMap tW2,
                       const __grid_constant__ CUtensorMap tHp, const __grid_constant__ CUtensorMap tDZ,
                       const TokGeom g, unsigned* status) {
   using S = PairShape<SWIGLU>;
@@ -107,7 +109,7 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
       tma_prefetch_desc(&tX);
       tma_prefetch_desc(&tFirst);
       tma_prefetch_desc(&tV);
-      tma_prefetch_desc(&tW2T);
+      tma_prefetch_desc(&tW2);
       const uint32_t full0 = mapa_shared(smem_u32(full), 0);  // the leader's full[0]
       int it = 0;
       bool stop = false;
@@ -129,7 +131,8 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
             if (phase == 0) {
               if (leader) mbar_arrive_expect_tx(&full[s], 2 * S::P_STAGE);
               tma_load_3d_pair(st, &tV, fb, kb * 64, m0 + g.v_off, z);
-              tma_load_3d_pair(st + S::A_BYTES, &tW2T, fb, kb * 64, nt * 128 + static_cast<int>(rank) * S::BP_ROWS, z);
+              // W2 [d][h]: 64 of the block's columns (N) x the k-block's 64 rows (K), MN-major
+              tma_load_3d_pair(st + S::A_BYTES, &tW2, fb, nt * 128 + static_cast<int>(rank) * S::BP_ROWS, kb * 64, z);
             } else {
               if (leader) mbar_arrive_expect_tx(&full[s], 2 * S::Z_STAGE);
               tma_load_3d_pair(st, &tX, fb, kb * 64, m0 + g.x_off, z);
@@ -153,7 +156,7 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
     }
   } else if (warp == 1) {
     if (leader && elect_one()) {
-      constexpr uint32_t idP = make_idesc(256, 128, 1, false, false);
+      constexpr uint32_t idP = make_idesc(256, 128, 1, false, true);
       constexpr uint32_t idZ = make_idesc(256, S::ZN, 1, false, false);
       const uint32_t sbase = smem_u32(smem);
       int it = 0, j = 0;
@@ -182,9 +185,13 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
             const uint32_t a = sbase + s * S::SLOT;
             const uint32_t b = a + S::A_BYTES;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16_pair(tmem_base + dcol, make_sdesc_sw128(a + kk * 32, 16, 1024),
-                           make_sdesc_sw128(b + kk * 32, 16, 1024), id, (kb > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              // P phase: B is MN-major (16 K-rows of 128 bytes per step); Z phase: K-major
+              const uint64_t db = phase == 0 ? make_sdesc_sw128(b + kk * 16 * 128, 8192, 1024)
+                                             : make_sdesc_sw128(b + kk * 32, 16, 1024);
+              mma_f16_pair(tmem_base + dcol, make_sdesc_sw128(a + kk * 32, 16, 1024), db, id,
+                           (kb > 0 || kk > 0) ? 1u : 0u);
+            }
             mma_commit_pair(&empty[s], 0x3);
           }
         }
@@ -336,7 +343,7 @@ int token_pair_capacity() {
 // g.m_tiles counts 256-token tiles; g.rows_alloc bounds the rows the stores may write.
 template <bool SWIGLU>
 cudaError_t launch_token_pair(const CUtensorMap& tX, const CUtensorMap& tFirstHalf, const CUtensorMap& tV,
-                              const CUtensorMap& tW2THalf, const CUtensorMap& tHp, const CUtensorMap& tDZ,
+                              const CUtensorMap& tW2Mn, const CUtensorMap& tHp, const CUtensorMap& tDZ,
                               const TokGeom& g, unsigned* status, cudaStream_t st) {
   const int cap = token_pair_capacity<SWIGLU>();
   if (cap <= 0) return cudaErrorInvalidConfiguration;
@@ -346,7 +353,7 @@ cudaError_t launch_token_pair(const CUtensorMap& tX, const CUtensorMap& tFirstHa
   const int pairs = static_cast<int>(std::min<long long>(total, cap));
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = pair_launch_config<SWIGLU>(pairs, st, attr);
-  return cudaLaunchKernelEx(&cfg, token_pair_kernel<SWIGLU>, tX, tFirstHalf, tV, tW2THalf, tHp, tDZ, g, status);
+  return cudaLaunchKernelEx(&cfg, token_pair_kernel<SWIGLU>, tX, tFirstHalf, tV, tW2Mn, tHp, tDZ, g, status);
 }
 
 }  // namespace ttt

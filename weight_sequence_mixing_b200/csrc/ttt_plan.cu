@@ -9,7 +9,7 @@ static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int plan_build(const ttt_config& c, Plan* p) {
   if (c.B < 1 || c.H < 1 || c.N < 1 || c.Nq < 1 || c.d < 1) return TTT_ERR_INVALID_ARG;
-  if (c.inner < TTT_INNER_LINEAR || c.inner > TTT_INNER_DWCONV) return TTT_ERR_INVALID_ARG;
+  if (c.inner < TTT_INNER_LINEAR || c.inner > TTT_INNER_GLU) return TTT_ERR_INVALID_ARG;
   if (c.loss < TTT_LOSS_MSE || c.loss > TTT_LOSS_RMSE) return TTT_ERR_INVALID_ARG;
   if (c.opt < TTT_OPT_GD || c.opt > TTT_OPT_MOMENTUM_MUON) return TTT_ERR_INVALID_ARG;
   if (c.dtype != TTT_F32 && c.dtype != TTT_BF16) return TTT_ERR_INVALID_ARG;
@@ -17,6 +17,9 @@ int plan_build(const ttt_config& c, Plan* p) {
   if (c.causal && c.Nq != c.N) return TTT_ERR_INVALID_ARG;
   const bool dw = c.inner == TTT_INNER_DWCONV;
   if ((c.inner == TTT_INNER_MLP2_GELU || c.inner == TTT_INNER_SWIGLU) && c.h < 1) return TTT_ERR_INVALID_ARG;
+  // the GLU runs on the tensor-core path only (the fp32 path runs it as a SwiGLU with h = d,
+  // W2 = I and TTT_FLAG_FIRST_LAYER_ONLY)
+  if (c.inner == TTT_INNER_GLU && c.dtype != TTT_BF16) return TTT_ERR_UNSUPPORTED;
   if (dw) {
     if (c.ksize < 1 || c.ksize > 7 || c.ksize % 2 == 0 || c.grid_h < 1 || c.grid_w < 1 ||
         static_cast<int64_t>(c.grid_h) * c.grid_w != c.N || c.Nq != c.N)
@@ -46,10 +49,13 @@ int plan_build(const ttt_config& c, Plan* p) {
 
   p->cfg = c;
   p->epochs = c.epochs == 0 ? 1 : c.epochs;
-  const int64_t d = c.d, h = (c.inner == TTT_INNER_LINEAR || dw) ? c.d : c.h;
+  const int64_t d = c.d, h = (c.inner == TTT_INNER_LINEAR || c.inner == TTT_INNER_GLU || dw) ? c.d : c.h;
   p->cfg.h = static_cast<int32_t>(h);
   p->P = dw ? d * c.ksize * c.ksize
-            : c.inner == TTT_INNER_LINEAR ? d * d : c.inner == TTT_INNER_MLP2_GELU ? 2 * d * h : 3 * d * h;
+            : c.inner == TTT_INNER_LINEAR ? d * d
+            : c.inner == TTT_INNER_GLU    ? 2 * d * d
+            : c.inner == TTT_INNER_MLP2_GELU ? 2 * d * h
+                                             : 3 * d * h;
   p->BH = c.B * c.H;
   p->chunk = (c.chunk <= 0 || c.chunk >= c.N) ? c.N : c.chunk;
   p->nchunks = static_cast<int>((static_cast<int64_t>(c.N) + p->chunk - 1) / p->chunk);
