@@ -25,6 +25,7 @@
 #include "apply_mlp.cuh"
 #include "epi_glu.cuh"
 #include "epilogues.cuh"
+#include "mse_token.cuh"
 #include "ns_fused.cuh"
 #include "token_pair.cuh"
 #include "token_phase.cuh"
@@ -175,17 +176,13 @@ __global__ void finish_rows_kernel(RowMap rm, int mode, float lr, bool rownorm, 
     mode = 0;
     rownorm = false;
   }
-  // rows of up to 1024 stay in registers (lane element q is column lane + 32 q), so every
-  // load of the row is issued before the norm's reduction
-  const float* u = nullptr;  // the update row (stride 1), or W2's column of the gradient layout
-  int64_t ustride = 1;
   if (mode == 1) {
     const float* Uz = U + int64_t(z) * rm.GR * rm.d;
     if (!w2) {
-      u = Uz + int64_t(rm.grad_row(k, r)) * rm.d;
+      const float* u = Uz + int64_t(rm.grad_row(k, r)) * rm.d;
+      for (int i = lane; i < len; i += 32) w[i] -= lr * u[i];
     } else {  // W2 row r = column r of the G2^T rows [0, h)
-      u = Uz + r;
-      ustride = rm.d;
+      for (int i = lane; i < len; i += 32) w[i] -= lr * Uz[int64_t(i) * rm.d + r];
     }
   } else if (mode == 2) {
     const int64_t mn = int64_t(m) * n;
@@ -193,64 +190,37 @@ __global__ void finish_rows_kernel(RowMap rm, int mode, float lr, bool rownorm, 
     const float* XTk = XT + (int64_t(z) * nmat + k) * mn;
     // result in the source orientation is (src_t ? XT : X); W2 rows are its columns
     const float* src = w2 ? (src_t ? Xk : XTk) : (src_t ? XTk : Xk);
-    u = src + int64_t(r) * len;
+    const float* u = src + int64_t(r) * len;
+    for (int i = lane; i < len; i += 32) w[i] -= lr * u[i];
   }
-  const int r1 = rm.inner == TTT_INNER_SWIGLU ? 2 * rm.h
-                 : rm.inner == TTT_INNER_GLU   ? 2 * rm.d
-                 : rm.inner == TTT_INNER_LINEAR ? rm.d
-                                                : rm.h;
-  bf16* dst = !w2 ? First + (int64_t(z) * r1 +
-                             rm.first_row(k, r)) * rm.d
-                  : W2 + (int64_t(z) * rm.d + r) * rm.h;
-  float s = 0.f;
+  float inv = 1.0f;
+  if (rownorm) {
+    float s = 0.f;
+    for (int i = lane; i < len; i += 32) s += w[i] * w[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    inv = 1.0f / fmaxf(sqrtf(s), 1e-12f);
+  }
   bool bad = false;
-  if (len <= 1024) {
-    float wv[32];
-#pragma unroll
-    for (int q = 0; q < 32; ++q) {
-      const int i = lane + 32 * q;
-      wv[q] = 0.f;
-      if (i < len) {
-        float x = w[i];
-        if (u) x -= lr * u[int64_t(i) * ustride];
-        wv[q] = x;
-        s += x * x;
-      }
-    }
-    float inv = 1.0f;
-    if (rownorm) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      inv = 1.0f / fmaxf(sqrtf(s), 1e-12f);
-    }
-#pragma unroll
-    for (int q = 0; q < 32; ++q) {
-      const int i = lane + 32 * q;
-      if (i < len) {
-        const float v = wv[q] * inv;
-        w[i] = v;
-        bad |= !isfinite(v);
-        dst[i] = __float2bfloat16_rn(v);
-      }
-    }
-  } else {  // longer rows: the step in place, then the norm and the copies
-    for (int i = lane; i < len; i += 32) {
-      float x = w[i];
-      if (u) x -= lr * u[int64_t(i) * ustride];
-      w[i] = x;
-      s += x * x;
-    }
-    float inv = 1.0f;
-    if (rownorm) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      inv = 1.0f / fmaxf(sqrtf(s), 1e-12f);
-    }
+  if (!w2) {
+    const int r1 = rm.inner == TTT_INNER_SWIGLU ? 2 * rm.h
+                   : rm.inner == TTT_INNER_GLU   ? 2 * rm.d
+                   : rm.inner == TTT_INNER_LINEAR ? rm.d
+                                                  : rm.h;
+    bf16* f = First + (int64_t(z) * r1 + rm.first_row(k, r)) * rm.d;
     for (int i = lane; i < len; i += 32) {
       const float v = w[i] * inv;
       w[i] = v;
       bad |= !isfinite(v);
-      dst[i] = __float2bfloat16_rn(v);
+      f[i] = __float2bfloat16_rn(v);
+    }
+  } else {
+    bf16* w2row = W2 + (int64_t(z) * rm.d + r) * rm.h;
+    for (int i = lane; i < len; i += 32) {
+      const float v = w[i] * inv;
+      w[i] = v;
+      bad |= !isfinite(v);
+      w2row[i] = __float2bfloat16_rn(v);
     }
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(status, kStatusNonFinite);
@@ -807,7 +777,41 @@ int update_chunk(Ctx& c, int t0, int n) {
     TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
     TRY(tmap(&tD, A1, 2, h, Cp, Z, 64));
     TRY(grad_gemm(c, tH, c.tVmn, tD, *tXmn, h, h, h, t0, xoff));
-  } else if (cfg.inner == TTT_INNER_MLP2_GELU) {  // MSE
+  } else if (cfg.inner == TTT_INNER_MLP2_GELU && cfg.loss == TTT_LOSS_MSE && d == 64 && (h == 128 || h == 256)) {
+    // one kernel for Z, GELU, V_hat, the MSE gradient and dH (mse_token.cuh) -> H, dY, dZ
+    TM tw1, tw2;
+    TRY(tmap(&tw1, c.v.at<bf16>(p, xFirst), 2, d, h, Z, h));
+    TRY(tmap(&tw2, c.v.at<bf16>(p, xW2), 2, h, d, Z, 64));
+    if (tX->box != 128 || c.tV.box != 128) return TTT_ERR_INVALID_ARG;
+    MseGeom mg;
+    mg.m_tiles = mt;
+    mg.batches = Z;
+    mg.rows_valid = n;
+    mg.x_off = xoff;
+    mg.v_off = t0;
+    mg.t0 = t0;
+    mg.eta = c.io.eta;
+    mg.eta_zs = D.N;
+    mg.eta_scalar = cfg.eta_scalar;
+    mg.coef = 2.0f / (float(n) * float(d));
+    mg.H = A0;
+    mg.dY = DY;
+    mg.dZ = A1;
+    mg.h_zs = int64_t(Cp) * h;
+    mg.y_zs = int64_t(Cp) * d;
+    {
+      StageScope sc(kStageTokenPhase, c.st);
+      const cudaError_t e = h == 256 ? launch_mse_token<256>(tX->m, c.tV.m, tw1.m, tw2.m, mg, status, c.st)
+                                     : launch_mse_token<128>(tX->m, c.tV.m, tw1.m, tw2.m, mg, status, c.st);
+      TRY_CUDA(e);
+    }
+    // G2^T = H^T dY (rows [0,h)), G1 = dZ^T X (rows [h,2h))
+    TM tH, tYmn, tD;
+    TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
+    TRY(tmap(&tYmn, DY, 2, d, Cp, Z, 64));
+    TRY(tmap(&tD, A1, 2, h, Cp, Z, 64));
+    TRY(grad_gemm(c, tH, tYmn, tD, *tXmn, h, h, h, 0, xoff));
+  } else if (cfg.inner == TTT_INNER_MLP2_GELU) {  // MSE, RMSE
     // Z = X W1^T -> H = GELU(Z), G' = GELU'(Z)
     EpiGeluSave e1{A0, A2, h, n, int64_t(Cp) * h};
     TcGeom g1 = geom(mt, 0, h / bn_for(h), d / 64, Z, 1);
