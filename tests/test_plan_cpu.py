@@ -17,10 +17,11 @@ EXPECTED = {
     # 128-column tiles give the 96 CTAs the 256-column tiles would halve
     "lact_lm_causal_n32k_c2048": dict(path=1, chunk=2048, nchunks=16, splits=1, tile_rows=128, grad_bn=128,
                                       direct=1),
-    # one 196608-token chunk: 512-row pair tiles (24 of them), 6 splits (144 pair tiles)
-    "lact_nvs_n196k_d512": dict(path=1, chunk=196608, nchunks=1, splits=6, tile_rows=512, grad_bn=256, direct=0),
-    # 8 chunks of 131072 (the last one 111616): 12 pair tiles x 12 splits
-    "lact_scene_n1m_c131k": dict(path=1, chunk=131072, nchunks=8, splits=12, tile_rows=512, grad_bn=256, direct=0),
+    # one 196608-token chunk: 512-row pair tiles (24 of them), 3 splits (72 pair tiles: one
+    # wave of the 74 pairs)
+    "lact_nvs_n196k_d512": dict(path=1, chunk=196608, nchunks=1, splits=3, tile_rows=512, grad_bn=256, direct=0),
+    # 8 chunks of 131072 (the last one 111616): 12 pair tiles x 6 splits, one wave
+    "lact_scene_n1m_c131k": dict(path=1, chunk=131072, nchunks=8, splits=6, tile_rows=512, grad_bn=256, direct=0),
 }
 
 
@@ -34,6 +35,12 @@ def test_workload_plans(name):
 def test_single_cta_flag_keeps_gradient_tiles_on_single_ctas():
     got = binding.plan_info(workload("lact_nvs_n196k_d512", single_cta=True))
     assert got["tile_rows"] == 256 and got["splits"] == 6
+    # pair tiles split only as far as one wave of the 74 CTA pairs holds
+    for name in ("lact_nvs_n196k_d512", "lact_scene_n1m_c131k"):
+        cfg = workload(name)
+        info = binding.plan_info(cfg)
+        tiles = 3 * cfg["h"] // 512 * (cfg["d"] // info["grad_bn"]) * cfg["B"] * cfg["H"]
+        assert info["tile_rows"] == 512 and tiles * info["splits"] <= 74 < tiles * (info["splits"] + 1)
 
 
 CASES = list(itertools.product([128, 256, 512], [128, 256, 1024], [1024, 4096, 8192, 65536], ["gd", "momentum", "muon"]))

@@ -12,9 +12,10 @@
 // the gating of the current one (Z is read out of TMEM before the gating math).
 // d <= 256 (O and Z together fit the 512 TMEM columns).
 //
-// Warps: 0 TMA producer, 1 MMA issuer, 2..9 epilogue (two per TMEM lane quarter; warp
-// half j of a quarter owns hidden columns [64 j, 64 j + 64) of a block, which is
-// k-block j of the H operand, and half of O's columns).  Every wait is bounded.
+// Warps: 0 TMA producer, 1 MMA issuer, then EW epilogue warps (EW / 4 per TMEM lane
+// quarter; warp part j of a quarter owns 128 / (EW / 4) adjacent hidden columns of a block,
+// inside one 64-column k-block of the H operand, and the matching share of O's columns).
+// Every wait is bounded.
 #pragma once
 #include "epilogues.cuh"
 
@@ -28,7 +29,7 @@ struct ApplyGeom {
   int64_t o_zs;          // elements between heads in O
 };
 
-template <bool SWIGLU, int D>
+template <bool SWIGLU, int D, int EPIW = 8>
 struct ApplyShape {
   static constexpr int KB = D / 64;                  // k-blocks of Q (64 channels each)
   static constexpr int ZN = SWIGLU ? 256 : 128;      // first-layer rows per hidden block
@@ -36,18 +37,21 @@ struct ApplyShape {
   static constexpr int H_BYTES = 2 * 128 * 128;      // 128 rows x 128 hidden bf16
   static constexpr int STAGE = (ZN > D ? ZN : D) * 128;  // one B k-block (64 K elements)
   static constexpr int STAGES = 3;
-  static constexpr int EW = 8;
+  static constexpr int EW = EPIW;                    // epilogue warps: EW / 4 per TMEM lane quarter
+  static constexpr int NQ = EW / 4;
+  static constexpr int HC = 128 / NQ;                // hidden columns of a block per epilogue thread
+  static_assert(EW == 8 || EW == 16, "epilogue warps");
   static constexpr int SMEM = 1024 + Q_BYTES + H_BYTES + STAGES * STAGE + 256;
   static constexpr uint32_t Z_COL = 256;             // Z accumulator columns [256, 256 + ZN)
   static_assert(D == 64 || D == 128 || D == 256, "d");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
-template <bool SWIGLU, int D>
-__global__ void __launch_bounds__(64 + 32 * ApplyShape<SWIGLU, D>::EW, 1)
+template <bool SWIGLU, int D, int EPIW>
+__global__ void __launch_bounds__(64 + 32 * ApplyShape<SWIGLU, D, EPIW>::EW, 1)
     apply_mlp_kernel(const __grid_constant__ CUtensorMap tQ, const __grid_constant__ CUtensorMap tFirst,
                      const __grid_constant__ CUtensorMap tW2, const ApplyGeom g, bf16* O, unsigned* status) {
-  using S = ApplyShape<SWIGLU, D>;
+  using S = ApplyShape<SWIGLU, D, EPIW>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* qs = smem;
@@ -210,10 +214,13 @@ __global__ void __launch_bounds__(64 + 32 * ApplyShape<SWIGLU, D>::EW, 1)
     }
   } else {
     const int q = warp & 3;
-    const int half = (warp - 2) >> 2;  // hidden columns [64 half, 64 half + 64) of a block
+    const int part = (warp - 2) >> 2;  // hidden columns [HC part, HC part + HC) of a block
+    const int hc0 = part * S::HC;
     const int row = q * 32 + lane;
     const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    uint8_t* hk = hs + half * 128 * 128 + row * 128;  // this thread's row of H's k-block `half`
+    // this thread's row of H's k-block hc0 / 64, from 16-byte chunk (hc0 % 64) / 8 on
+    uint8_t* hk = hs + (hc0 / 64) * 128 * 128 + row * 128;
+    const int k0 = (hc0 % 64) / 8;
     int j = 0, nz = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++j) {
@@ -222,13 +229,13 @@ __global__ void __launch_bounds__(64 + 32 * ApplyShape<SWIGLU, D>::EW, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(zfull, nz & 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
-        // read this thread's 64 hidden columns of Z (and z3), then release the TMEM
-        uint32_t packed[32];
+        // read this thread's HC hidden columns of Z (and z3), then release the TMEM
+        uint32_t packed[S::HC / 2];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < S::HC / 32; ++c) {
           float z1[32], z3[32];
-          tmem_ld32(tq + S::Z_COL + half * 64 + c * 32, z1);
-          if constexpr (SWIGLU) tmem_ld32(tq + S::Z_COL + 128 + half * 64 + c * 32, z3);
+          tmem_ld32(tq + S::Z_COL + hc0 + c * 32, z1);
+          if constexpr (SWIGLU) tmem_ld32(tq + S::Z_COL + 128 + hc0 + c * 32, z3);
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             float a, b;
@@ -250,10 +257,10 @@ __global__ void __launch_bounds__(64 + 32 * ApplyShape<SWIGLU, D>::EW, 1)
           ok = __all_sync(0xffffffffu, mbar_wait(hempty, (nz - 1) & 1, abort_flag));
           if (!ok) break;
         }
-        // 64 bf16 = 8 chunks of 16 bytes; chunk k of row r sits at k ^ (r & 7)
+        // HC bf16 = HC / 8 chunks of 16 bytes; chunk k of row r sits at k ^ (r & 7)
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          *reinterpret_cast<uint4*>(hk + 16 * (k ^ (row & 7))) =
+        for (int k = 0; k < S::HC / 8; ++k)
+          *reinterpret_cast<uint4*>(hk + 16 * ((k0 + k) ^ (row & 7))) =
               make_uint4(packed[4 * k], packed[4 * k + 1], packed[4 * k + 2], packed[4 * k + 3]);
         fence_proxy_async_smem();
         __syncwarp();
@@ -267,14 +274,34 @@ __global__ void __launch_bounds__(64 + 32 * ApplyShape<SWIGLU, D>::EW, 1)
       const bool valid = m < g.rows_valid;
       bf16* orow = O + z * g.o_zs + int64_t(g.row0 + m) * D;
       bool bad = false;
+      // O columns [part D / NQ, (part + 1) D / NQ) of this thread's row
+      constexpr int OC = D / S::NQ;
+      if constexpr (OC >= 32) {
 #pragma unroll 1
-      for (int cc = half * (D / 2); cc < (half + 1) * (D / 2); cc += 32) {
-        float v[32];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + cc, v);
-        if (!valid) continue;
+        for (int cc = part * OC; cc < (part + 1) * OC; cc += 32) {
+          float v[32];
+          tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + cc, v);
+          if (!valid) continue;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) bad |= !isfinite(v[i]);
-        store_bf16x32(orow + cc, v);
+          for (int i = 0; i < 32; ++i) bad |= !isfinite(v[i]);
+          store_bf16x32(orow + cc, v);
+        }
+      } else {  // 16 columns
+        uint32_t r[16];
+        tmem_ld16_async(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + part * OC, r);
+        tmem_wait_regs(r);
+        if (valid) {
+          uint32_t w[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float a = __uint_as_float(r[2 * i]), b = __uint_as_float(r[2 * i + 1]);
+            bad |= !isfinite(a) || !isfinite(b);
+            w[i] = pack_bf16x2(a, b);
+          }
+          uint4* o4 = reinterpret_cast<uint4*>(orow + part * OC);
+          o4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          o4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        }
       }
       if (bad) set_status(status, kStatusNonFinite);
       tc_fence_before();
@@ -290,11 +317,13 @@ __global__ void __launch_bounds__(64 + 32 * ApplyShape<SWIGLU, D>::EW, 1)
   if (warp == 1) tmem_dealloc(tmem_base, 512);
 }
 
+// The GELU MLP's epilogue (an erf per hidden unit) is the slower one: it gets 16 warps.
 template <bool SWIGLU, int D>
 cudaError_t launch_apply_mlp(const CUtensorMap& tQ, const CUtensorMap& tFirst, const CUtensorMap& tW2,
                              const ApplyGeom& g, bf16* O, unsigned* status, cudaStream_t st) {
-  using S = ApplyShape<SWIGLU, D>;
-  auto kern = apply_mlp_kernel<SWIGLU, D>;
+  constexpr int EPIW = SWIGLU ? 8 : 16;
+  using S = ApplyShape<SWIGLU, D, EPIW>;
+  auto kern = apply_mlp_kernel<SWIGLU, D, EPIW>;
   static OncePerDevice configured;
   const int set = configured.run(current_device(), [&] {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);

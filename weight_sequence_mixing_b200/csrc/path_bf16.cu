@@ -43,7 +43,6 @@ enum BBuf {
   xMom,    // fp32 momentum, gradient layout [Z][GR][d]
   xU,      // fp32 update direction, gradient layout [Z][GR][d]
   xRowSq,  // fp32 [Z][GR] squared row norms of U
-  xInvN,   // fp32 [Z][nmat] 1/(||U_k||_F + 1e-7)
   xPart,   // fp32 split-K partials [S][Z][GR][d]
   xFirst,  // bf16 first-layer weights [Z][R1][d] (SwiGLU: blocks [W1 128 | W3 128])
   xW2T,    // bf16 W2^T [Z][h][d]
@@ -345,35 +344,30 @@ __global__ void reduce_grad_kernel(int Z, int GR, int d, int splits, const float
   if (lane == 0 && rowsq) rowsq[int64_t(z) * GR + g] = sq;
 }
 
-// 1/(||U_k||_F + 1e-7) per (z, matrix k), summing row norms in a fixed order.
-__global__ void ns_norm_kernel(RowMap rm, int nmat, const float* rowsq, float* invn) {
-  __shared__ float red[256];
-  const int z = blockIdx.x / nmat, k = blockIdx.x % nmat;
-  const int rows_src = rm.inner == TTT_INNER_LINEAR ? rm.d : rm.h;
-  const bool w2 = rm.is_w2(k);
-  float s = 0.f;
-  for (int r = threadIdx.x; r < rows_src; r += blockDim.x)
-    s += rowsq[int64_t(z) * rm.GR + (w2 ? r : rm.grad_row(k, r))];
-  red[threadIdx.x] = s;
-  __syncthreads();
-  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
-    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) invn[blockIdx.x] = 1.0f / (sqrtf(red[0]) + 1e-7f);
-}
-
 // Newton-Schulz input of matrix k: its gradient-layout source M_src [rows_src][d]
-// scaled by invn, written in source orientation to A and transposed to B.
-// (X0, X0^T) = src_t ? (B, A) : (A, B).
-__global__ void ns_prep_kernel(RowMap rm, int nmat, const float* U, const float* invn, float* A, float* Bt) {
+// scaled by 1/(||M_src||_F + 1e-7), written in source orientation to A and transposed
+// to B.  (X0, X0^T) = src_t ? (B, A) : (A, B).  Every CTA of the matrix sums the squared
+// row norms (rowsq) itself, in the same fixed order, so all of them scale by the same value.
+__global__ void ns_prep_kernel(RowMap rm, int nmat, const float* U, const float* rowsq, float* A, float* Bt) {
   __shared__ float tile[32][33];
+  __shared__ float red[256];
   const int zk = blockIdx.z, z = zk / nmat, k = zk % nmat;
   const int rows_src = rm.inner == TTT_INNER_LINEAR ? rm.d : rm.h;
   const int d = rm.d;
   const bool w2 = rm.is_w2(k);
   const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
-  const float s = invn[zk];
+  {
+    float q = 0.f;
+    for (int r = threadIdx.x; r < rows_src; r += blockDim.x)
+      q += rowsq[int64_t(z) * rm.GR + (w2 ? r : rm.grad_row(k, r))];
+    red[threadIdx.x] = q;
+    __syncthreads();
+    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+      if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+      __syncthreads();
+    }
+  }
+  const float s = 1.0f / (sqrtf(red[0]) + 1e-7f);
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8 threads
   const int64_t mn = int64_t(rows_src) * d;
   for (int j = ty; j < 32; j += 8) {
@@ -551,17 +545,13 @@ int optimizer_step(Ctx& c) {
   float* XT = c.v.at<float>(p, xNXT);
   if (muon) {
     const int ZK = D.Z * D.nmat;
-    {
-      StageScope _sc(kStageNewtonSchulz, st);
-      ns_norm_kernel<<<ZK, 256, 0, c.st>>>(c.rm, D.nmat, c.v.at<float>(p, xRowSq), c.v.at<float>(p, xInvN));
-    }
     const int rows_src = cfg.inner == TTT_INNER_LINEAR ? D.d : D.h;
     dim3 g((D.d + 31) / 32, (rows_src + 31) / 32, ZK);
     float* A = D.src_t ? XT : X;
     float* B = D.src_t ? X : XT;
     {
       StageScope _sc(kStageNewtonSchulz, st);
-      ns_prep_kernel<<<g, 256, 0, c.st>>>(c.rm, D.nmat, c.v.at<float>(p, xU), c.v.at<float>(p, xInvN), A, B);
+      ns_prep_kernel<<<g, 256, 0, c.st>>>(c.rm, D.nmat, c.v.at<float>(p, xU), c.v.at<float>(p, xRowSq), A, B);
     }
     TRY_CUDA(cudaGetLastError());
     // all Newton-Schulz iterations of every matrix in one clustered launch
@@ -976,8 +966,12 @@ void choose_grad_shape(const Plan& p, int Cp, int* splits, int* tile_rows, int* 
   if (tiles512 > 0 && tiles512 * smax >= kPlanSMs / 2) *tile_rows = 512;
   const int units = *tile_rows == 512 ? kPlanSMs / 2 : kPlanSMs;  // tiles that run at once
   const int tiles = rows / *tile_rows * (d / bnd) * p.BH;
-  // about two waves of tiles: long K ranges per split, few partials to reduce
-  int s = tiles > 0 ? std::max(1, (2 * units + tiles / 2) / tiles) : 1;
+  // single CTAs: about two waves of tiles (long K ranges per split, few partials to
+  // reduce); CTA pairs: as many splits as fit one wave of the pairs (two waves measured
+  // 1.2% slower on the million-token scene layer: twice the partials to write and reduce)
+  int s = tiles <= 0 ? 1
+          : *tile_rows == 512 ? std::max(1, units / tiles)
+                              : std::max(1, (2 * units + tiles / 2) / tiles);
   s = std::min(s, smax);
   const int per = (kblocks + s - 1) / s;  // every split owns at least one k-block
   *splits = (kblocks + per - 1) / per;
@@ -1023,7 +1017,6 @@ int plan_layout_bf16(Plan* p) {
       Z * GR * d * 4,
       Z * GR * d * 4,
       Z * GR * 4,
-      ZK * 4,
       D.direct ? 0 : int64_t(D.splits) * Z * GR * d * 4,
       Z * D.R1 * d * 2,
       act ? Z * h * d * 2 : 0,
