@@ -11,6 +11,7 @@ import torch
 
 import oracle as orc
 from synth_inputs import gen_inputs, make_config, matrix_shapes, workload
+from weight_sequence_mixing_b200 import binding
 from tests.parity_util import compare, rel_fro, run_gpu
 
 pytestmark = pytest.mark.gpu
@@ -51,6 +52,9 @@ SMALL = [
          eta_mode="scalar", eta_scalar=1.0),
     dict(inner="mlp2_gelu", loss="mse", opt="momentum", d=64, h=128, N=333, chunk=128, key_instnorm=True,
          data="vit", eta_mode="scalar"),
+    # fused MSE kernel: 4 tile ranges per head, the last chunk's 2 tiles leave two ranges empty
+    dict(inner="mlp2_gelu", loss="mse", opt="momentum", d=64, h=256, N=700, chunk=512, key_instnorm=True,
+         data="vit"),
     dict(inner="mlp2_gelu", loss="neg_dot", opt="momentum", d=128, h=256, N=400, chunk=256, weight_l2norm=True),
     dict(inner="linear", loss="neg_dot", opt="gd", d=128, h=128, N=260),
     dict(inner="linear", loss="mse", opt="momentum_muon", d=128, h=128, N=390, chunk=128, weight_l2norm=True),
@@ -101,16 +105,23 @@ def test_token_kernels_pair_and_single_cta(kw):
     base = dict(B=2, H=2, dtype="bf16", data="lact", eta_mode="per_token", loss="neg_dot", opt="gd", seed=17)
     base.update(kw)
     x = gen_inputs(make_config(**base))
-    Op, Wp = run_gpu(make_config(**base), x)
-    Os, Ws = run_gpu(make_config(single_cta=True, **base), x)
-    # the two kernels round the same fp32 accumulators to bf16: near-identical results
-    assert rel_fro(Op, Os) < 1e-3 and rel_fro(Wp, Ws) < 1e-3
     for single in (False, True):
         cfg = make_config(single_cta=single, **base)
         errs = _delta_w_check(cfg, x)
         for k, v in errs.items():
             tol = DW_TOL if k.startswith("d") else TOL
             assert v <= tol, f"single={single} {k}: relative Frobenius error {v:.3e} > {tol}"
+    Op, Wp = run_gpu(make_config(**base), x)
+    Os, Ws = run_gpu(make_config(single_cta=True, **base), x)
+    # With the same split-K count the two kernels round the same fp32 accumulators to
+    # bf16: near-identical results.  With different counts the gradient sums run in another
+    # order, and Muon's Newton-Schulz map (slope about 3.4 per step near a zero singular
+    # value) magnifies that rounding noise in the weak directions: a looser bound.
+    same = binding.plan_info(make_config(**base))["splits"] == \
+        binding.plan_info(make_config(single_cta=True, **base))["splits"]
+    muon = base["opt"] in ("muon", "momentum_muon")
+    near = 1e-3 if same or not muon else 1e-2
+    assert rel_fro(Op, Os) < near and rel_fro(Wp, Ws) < near
 
 
 def test_causal_chunk_n_equals_single_chunk_weights_on_gpu():

@@ -503,6 +503,7 @@ struct Ctx {
   RowMap rm;
   TM tK, tV, tKmn, tVmn, tQ, tFirst, tW2T, tW2;
   int bn_first = 0;
+  bool apply_pending = false;  // an apply on io.aux still reads the bf16 weight copies
 };
 
 // bf16 W2^T from the freshly written bf16 W2: the B operand of the single-CTA token
@@ -526,6 +527,11 @@ int transpose_w2(Ctx& c) {
 // update-direction -> weights (+ Newton-Schulz when the optimizer is Muon)
 int optimizer_step(Ctx& c) {
   cudaStream_t st = c.st;
+  // the chunk's apply on the side stream reads the bf16 weights this step rewrites
+  if (c.apply_pending) {
+    TRY_CUDA(cudaStreamWaitEvent(st, c.io.ev_join, 0));
+    c.apply_pending = false;
+  }
   const Plan& p = c.p;
   const Dims& D = c.D;
   const ttt_config& cfg = p.cfg;
@@ -1094,12 +1100,27 @@ int run_bf16(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
     TRY_CUDA(cudaGetLastError());
     TRY(transpose_w2(c));
   }
+  // causal with a side stream: chunk c's apply (reads W_c) runs beside chunk c's token
+  // phase and gradient GEMMs (read W_c too); the optimizer step that replaces W_c waits for it
+  const bool overlap = cfg.causal && io.aux && io.ev_fork && io.ev_join;
   for (int ci = 0; ci < p.nchunks; ++ci) {
     const int t0 = ci * p.chunk, n = std::min(p.chunk, cfg.N - t0);
-    if (cfg.causal) TRY(apply_rows(c, t0, n));
+    if (cfg.causal && overlap) {
+      TRY_CUDA(cudaEventRecord(io.ev_fork, st));
+      TRY_CUDA(cudaStreamWaitEvent(io.aux, io.ev_fork, 0));
+      c.st = io.aux;
+      const int r = apply_rows(c, t0, n);
+      c.st = st;
+      TRY(r);
+      TRY_CUDA(cudaEventRecord(io.ev_join, io.aux));
+      c.apply_pending = true;
+    } else if (cfg.causal) {
+      TRY(apply_rows(c, t0, n));
+    }
     if (cfg.flags & TTT_FLAG_NO_UPDATE) continue;
     for (int ep = 0; ep < p.epochs; ++ep) TRY(update_chunk(c, t0, n));
   }
+  if (overlap) TRY_CUDA(cudaStreamWaitEvent(st, io.ev_join, 0));  // join the side stream
   if (!cfg.causal) TRY(apply_rows(c, 0, cfg.Nq));
   if (io.W_out)
     TRY_CUDA(cudaMemcpyAsync(io.W_out, c.v.at<float>(p, xWf), size_t(Z) * p.P * 4, cudaMemcpyDeviceToDevice, st));

@@ -66,6 +66,16 @@ void destroy_entry(ttt::GraphEntry& e) {
   }
 }
 
+// The side stream and events of a handle (see forward_impl).
+void release_aux(ttt_handle* h) {
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+  if (h->ev_join) cudaEventDestroy(h->ev_join);
+  if (h->aux) cudaStreamDestroy(h->aux);
+  h->aux = nullptr;
+  h->ev_fork = h->ev_join = nullptr;
+  h->aux_dev = -1;
+}
+
 // Capture one replayable instance of the layer's launch sequence on `st`.
 int capture_instance(ttt_handle* h, const Io& io, void* ws, cudaStream_t st, ttt::GraphInstance* gi,
                      long long* launches) {
@@ -157,8 +167,35 @@ int forward_impl(ttt_handle* h, const Io& io, void* workspace, size_t workspace_
     if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return TTT_ERR_CUDA;
     graph = cs == cudaStreamCaptureStatusNone;
   }
+  // The causal bf16 layer applies each chunk on a side stream while the main stream
+  // computes the chunk's update; the stream and its events are made outside any capture.
+  Io run = io;
+  const Plan& pl = h->plan;
+  if (pl.path == kPathBf16 && pl.cfg.causal && pl.nchunks > 1) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TTT_ERR_CUDA;
+    if (h->aux_dev != dev) {
+      cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+      const bool capturing = st && cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs != cudaStreamCaptureStatusNone;
+      if (!capturing) {
+        release_aux(h);
+        if (cudaStreamCreateWithFlags(&h->aux, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) != cudaSuccess) {
+          release_aux(h);
+          return TTT_ERR_CUDA;
+        }
+        h->aux_dev = dev;
+      }
+    }
+    if (h->aux_dev == dev) {
+      run.aux = h->aux;
+      run.ev_fork = h->ev_fork;
+      run.ev_join = h->ev_join;
+    }
+  }
   g_prof = &h->prof;
-  const int r = graph ? forward_graph(h, io, workspace, st) : plan_run(h->plan, io, workspace, st);
+  const int r = graph ? forward_graph(h, run, workspace, st) : plan_run(h->plan, run, workspace, st);
   g_prof = nullptr;
   return r;
 }
@@ -244,6 +281,7 @@ extern "C" void ttt_destroy(ttt_handle* h) {
     cudaEventDestroy(q.b);
   }
   for (cudaEvent_t e : p.pool) cudaEventDestroy(e);
+  release_aux(h);
   delete h;
 }
 

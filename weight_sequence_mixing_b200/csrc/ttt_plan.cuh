@@ -20,6 +20,11 @@ struct Io {
   float* W_out;
   const void* M_in = nullptr;  // momentum state carried in (ttt_forward_state), or null: zero
   void* M_out = nullptr;       // momentum state carried out, or null
+  // a second stream of the calling device for work that may overlap the main stream's
+  // (the causal layer's apply on a chunk runs beside that chunk's update), with the
+  // events that fork it from and join it back into the main stream; null: no overlap
+  cudaStream_t aux = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
 };
 
 enum PathKind : int { kPathF32 = 0, kPathBf16 = 1, kPathDwconv = 2 };
@@ -61,4 +66,9 @@ int run_dwconv(const Plan& plan, const Io& io, void* workspace, cudaStream_t st)
 struct ttt_handle {
   ttt::Plan plan;
   ttt::Profiler prof;
+  // the side stream and fork / join events of Io::aux, made for the device they were first
+  // needed on (remade if a later call runs on another device)
+  int aux_dev = -1;
+  cudaStream_t aux = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
 };
