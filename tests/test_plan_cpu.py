@@ -11,8 +11,9 @@ binding = pytest.importorskip("weight_sequence_mixing_b200.binding")
 EXPECTED = {
     # fp32 SIMT path: one chunk of 196 tokens
     "tiny_mlp2_n196_fp32": dict(path=0, chunk=196, nchunks=1),
-    # d = 64: 256-row single-CTA tiles of 64 columns, 3 splits of 2048 tokens
-    "vit3s_1248_mlp2_n6084": dict(path=1, chunk=6084, nchunks=1, splits=3, tile_rows=256, grad_bn=64, direct=0),
+    # d = 64 GELU MLP with the MSE loss: token phase and gradients in one kernel, one CTA
+    # per (head, third of the 48 token tiles): 144 CTAs, 3 split partials per head
+    "vit3s_1248_mlp2_n6084": dict(path=1, chunk=6084, nchunks=1, splits=3, tile_rows=128, grad_bn=64, direct=0),
     # 2048-token chunks are not split: gradients go straight into U and the momentum;
     # 128-column tiles give the 96 CTAs the 256-column tiles would halve
     "lact_lm_causal_n32k_c2048": dict(path=1, chunk=2048, nchunks=16, splits=1, tile_rows=128, grad_bn=128,
@@ -199,3 +200,16 @@ def test_glu_combinations(kw, status):
         # two d x d matrices (h is ignored), 64-channel blocks of gate and linear rows
         assert binding.LIB.ttt_param_count(h) == 2 * cfg["d"] ** 2
         binding.LIB.ttt_destroy(h)
+
+
+@pytest.mark.parametrize("B,H,N,chunk,h", [(8, 6, 6084, 0, 256), (1, 1, 300, 0, 128), (2, 2, 700, 512, 256),
+                                           (1, 200, 1000, 0, 256), (4, 1, 65536, 0, 128)])
+def test_fused_mse_plan(B, H, N, chunk, h):
+    # one CTA per (head, token-tile range): at most one wave of 148 CTAs, every range at
+    # least one tile of a full chunk, split partials always reduced (never direct)
+    cfg = make_config(B=B, H=H, N=N, chunk=chunk, d=64, h=h, inner="mlp2_gelu", loss="mse", opt="gd",
+                      dtype="bf16")
+    got = binding.plan_info(cfg)
+    tiles = -(-got["chunk"] // 128)
+    assert got["direct"] == 0 and got["tile_rows"] == 128
+    assert got["splits"] == max(1, min(tiles, 148 // (B * H)))

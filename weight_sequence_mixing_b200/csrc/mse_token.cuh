@@ -1,53 +1,58 @@
-// Token phase of the GELU-MLP update with the MSE loss in one kernel (d = 64; h = 128 or
-// 256: the ViT3-like heads).  For every 128-token tile of a chunk (ViT3 digest section 02:
-// forward on the keys, loss backward):
+// Token phase and weight gradients of the GELU-MLP update with the MSE loss in one kernel
+// (d = 64; h = 128 or 256: the ViT3-like heads).  For every 128-token tile of a chunk
+// (ViT3 digest section 02: forward on the keys, loss backward, gradients of W1 and W2):
 //   Z    = X W1^T                      (TMEM columns [0, h))
-//   H    = GELU(Z), G' = GELU'(Z)      (H -> shared memory as the next MMA's operand and
-//                                       to HBM for the weight gradients; G' stays in the
-//                                       epilogue threads' registers)
-//   V^   = H W2^T                      (TMEM columns [256, 320))
-//   dY   = 2 eta_t (V^ - V) / (n d)    (-> shared memory and HBM)
-//   dH   = dY W2                       (TMEM columns [256, 256 + h): W2 [d][h] read as an
-//                                       MN-major operand from the same tile as for V^)
-//   dZ   = dH * G'                     (-> HBM)
-// H, dY and dZ are what the weight-gradient reductions read (G2^T = H^T dY, G1 = dZ^T X);
-// rows past the chunk are written as zeros.  The three GEMMs of a tile are chained
-// through TMEM and shared memory: neither Z nor G' nor V^ reaches HBM, and the next
-// tile's Z overlaps this tile's later phases (Z and V^ / dH use separate TMEM columns).
+//   H    = GELU(Z), G' = GELU'(Z)      (H -> shared memory; G' stays in the epilogue
+//                                       threads' registers)
+//   V^   = H W2^T                      (TMEM columns [0, 64): Z has been read by then)
+//   dY   = 2 eta_t (V^ - V) / (n d)    (-> shared memory)
+//   G2^T += H^T dY                     (TMEM accumulators, see below)
+//   dH   = dY W2                       (TMEM columns [0, h): W2 [d][h] read as an MN-major
+//                                       operand from the same tile as for V^)
+//   dZ   = dH * G'                     (-> shared memory, over H)
+//   G1   += dZ^T X                     (TMEM accumulators)
+// Nothing of a tile reaches HBM: the gradients of W2 (as G2^T [h][d]) and W1 [h][d] stay
+// in TMEM columns [256, 256 + 128 h / 64) as 128-row x 64-column accumulators, summed
+// over the CTA's tiles, and are written once, as fp32 split partials in the gradient
+// layout [split][z][2h][d] (rows [0, h) G2^T, rows [h, 2h) G1), for the split reduction.
 //
-// Warps: 0 TMA producer (keys and values of two tiles in flight; W1, W2 of the current
-// head resident), 1 MMA issuer, 2..17 epilogue (four per TMEM lane quarter; warp slot s
-// owns hidden columns [s h/4, (s+1) h/4) and 16 of the 64 output channels).  Every wait
-// is bounded.
+// A CTA owns one head z and one contiguous range of its token tiles (split sp of the
+// chunk's tiles), so the head's weights are loaded once.  Tiles run one after another:
+// a tile's TMEM-chained steps leave no room in TMEM for a second tile.  Rows past the
+// chunk are zero in H, dY and dZ, so they add nothing.
+//
+// Warps: 0 TMA producer (keys and values of two tiles in flight), 1 MMA issuer, 2..17
+// epilogue (four per TMEM lane quarter; warp slot s owns hidden columns [s h/4, (s+1) h/4)
+// and 16 of the 64 output channels).  Every wait is bounded.
 #pragma once
 #include "epilogues.cuh"
 
 namespace ttt {
 
 struct MseGeom {
-  int m_tiles, batches;  // 128-token tiles per head, heads (z)
-  int rows_valid;        // tokens in the chunk
-  int x_off, v_off;      // token offsets of the key and value maps
-  int t0;                // chunk's first token (eta index)
+  int m_tiles;          // 128-token tiles of the chunk holding keys (ceil(n / 128))
+  int batches, splits;  // heads (z), token-tile ranges per head: one CTA each
+  int rows_valid;       // tokens in the chunk
+  int x_off, v_off;     // token offsets of the key and value maps
+  int t0;               // chunk's first token (eta index)
   const float* eta;
   int64_t eta_zs;
   float eta_scalar, coef;  // coef = 2 / (n d)
-  bf16* H;                 // [z][Cp][h]
-  bf16* dY;                // [z][Cp][d]
-  bf16* dZ;                // [z][Cp][h]
-  int64_t h_zs, y_zs;      // elements per head of H (and dZ) and of dY
+  float* part;             // [splits][z][2h][64] fp32 gradient partials
 };
 
 template <int HID>
 struct MseShape {
   static constexpr int D = 64;
-  static constexpr int TILE = 128 * 128;              // 128 rows x 64 bf16
-  static constexpr int W1_BYTES = HID * 128;          // [HID][64]
+  static constexpr int TILE = 128 * 128;                  // 128 rows x 64 bf16
+  static constexpr int W1_BYTES = HID * 128;              // [HID][64]
   static constexpr int W2_BYTES = (HID / 64) * 64 * 128;  // [64][HID] as HID/64 blocks of 64 columns
-  static constexpr int H_BYTES = (HID / 64) * TILE;   // [128][HID] as HID/64 k-blocks
+  static constexpr int H_BYTES = (HID / 64) * TILE;       // [128][HID] as HID/64 k-blocks (H, then dZ)
   static constexpr int EW = 16;
   static constexpr int SMEM = 1024 + 2 * 2 * TILE + W1_BYTES + W2_BYTES + H_BYTES + TILE + 256;
-  static constexpr int COLS = HID / 4;                // hidden columns per epilogue thread
+  static constexpr int COLS = HID / 4;          // hidden columns per epilogue thread
+  static constexpr int NACC = 2 * (HID / 128);  // 128 x 64 gradient accumulators
+  static constexpr uint32_t GCOL = 256;         // first TMEM column of the accumulators
   static_assert(HID == 128 || HID == 256, "h");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
@@ -55,6 +60,15 @@ struct MseShape {
 // 16-byte chunk k of row r of a 128-byte-row, 128-byte-swizzled tile sits at k ^ (r & 7)
 __device__ __forceinline__ uint4* sw128_chunk(uint8_t* tile, int r, int k) {
   return reinterpret_cast<uint4*>(tile + r * 128 + 16 * (k ^ (r & 7)));
+}
+
+// 16 values of this thread's row as bf16 into columns [k0 8, k0 8 + 16) of a swizzled k-block
+__device__ __forceinline__ void put_row16(uint8_t* kb, int row, int k0, const float (&v)[16]) {
+#pragma unroll
+  for (int k = 0; k < 2; ++k)
+    *sw128_chunk(kb, row, k0 + k) =
+        make_uint4(pack_bf16x2(v[8 * k], v[8 * k + 1]), pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
+                   pack_bf16x2(v[8 * k + 4], v[8 * k + 5]), pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
 }
 
 template <int HID>
@@ -65,29 +79,30 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
   using S = MseShape<HID>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* xv = smem;                       // [slot][X tile | V tile]
+  uint8_t* xv = smem;  // [slot][X tile | V tile]
   uint8_t* w1s = xv + 2 * 2 * S::TILE;
   uint8_t* w2s = w1s + S::W1_BYTES;
   uint8_t* hs = w2s + S::W2_BYTES;
   uint8_t* dys = hs + S::H_BYTES;
   uint64_t* xfull = reinterpret_cast<uint64_t*>(dys + S::TILE);  // [2]
-  uint64_t* xempty = xfull + 2;   // [2]: the Z MMAs (commit) and the dY epilogue are done with the slot
-  uint64_t* wfull = xempty + 2;   // the head's weights landed
-  uint64_t* wrelease = wfull + 1;  // the last MMA reading a head's weights completed
-  uint64_t* zfull = wrelease + 1;
-  uint64_t* zempty = zfull + 1;
-  uint64_t* hfull = zempty + 1;
-  uint64_t* vfull = hfull + 1;
-  uint64_t* dyfull = vfull + 1;
-  uint64_t* dhfull = dyfull + 1;
-  uint64_t* dhempty = dhfull + 1;
-  uint64_t* drain = dhempty + 1;
+  uint64_t* xempty = xfull + 2;  // [2]: G1 (commit) and the dY epilogue are done with the slot
+  uint64_t* wfull = xempty + 2;  // the head's weights landed
+  uint64_t* zfull = wfull + 1;   // Z in TMEM (every earlier MMA, the previous tile's G1 too, done)
+  uint64_t* hfull = zfull + 1;   // H in shared memory, Z read
+  uint64_t* vfull = hfull + 1;   // V^ in TMEM
+  uint64_t* dyfull = vfull + 1;  // dY in shared memory, V^ read
+  uint64_t* dhfull = dyfull + 1;  // dH in TMEM, the tile's G2^T done (H no longer read)
+  uint64_t* dzfull = dhfull + 1;  // dZ in shared memory, dH read
+  uint64_t* gdone = dzfull + 1;   // the last tile's G1 done: the accumulators are final
+  uint64_t* drain = gdone + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = static_cast<int>(lane_id());
-  const int total = g.m_tiles * g.batches;
+  const int z = blockIdx.x / g.splits, sp = blockIdx.x % g.splits;
+  const int mt0 = static_cast<int>(int64_t(sp) * g.m_tiles / g.splits);
+  const int ntiles = static_cast<int>(int64_t(sp + 1) * g.m_tiles / g.splits) - mt0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -95,14 +110,13 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
       mbar_init(&xempty[s], 1 + S::EW);
     }
     mbar_init(wfull, 1);
-    mbar_init(wrelease, 1);
     mbar_init(zfull, 1);
-    mbar_init(zempty, S::EW);
     mbar_init(hfull, S::EW);
     mbar_init(vfull, 1);
     mbar_init(dyfull, S::EW);
     mbar_init(dhfull, 1);
-    mbar_init(dhempty, S::EW);
+    mbar_init(dzfull, S::EW);
+    mbar_init(gdone, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -117,25 +131,16 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    if (elect_one()) {
+    if (elect_one() && ntiles > 0) {
       tma_prefetch_desc(&tX);
       tma_prefetch_desc(&tV);
       tma_prefetch_desc(&tW1);
       tma_prefetch_desc(&tW2);
-      int j = 0, zw = -1, nw = 0;  // tiles, head of the resident weights, weight loads
-      for (int t = blockIdx.x; t < total; t += gridDim.x, ++j) {
-        const int mt = t % g.m_tiles, z = t / g.m_tiles;
-        if (z != zw) {
-          // the MMAs of the previous head must be done reading its weights (one release per
-          // head change, in order: the phases alternate)
-          if (nw > 0 && !mbar_wait(wrelease, (nw - 1) & 1, abort_flag)) break;
-          mbar_arrive_expect_tx(wfull, S::W1_BYTES + S::W2_BYTES);
-          tma_load_3d(w1s, &tW1, wfull, 0, 0, z);
-          for (int b = 0; b < HID / 64; ++b) tma_load_3d(w2s + b * 64 * 128, &tW2, wfull, 64 * b, 0, z);
-          zw = z;
-          ++nw;
-        }
-        const int s = j & 1;
+      mbar_arrive_expect_tx(wfull, S::W1_BYTES + S::W2_BYTES);
+      tma_load_3d(w1s, &tW1, wfull, 0, 0, z);
+      for (int b = 0; b < HID / 64; ++b) tma_load_3d(w2s + b * 64 * 128, &tW2, wfull, 64 * b, 0, z);
+      for (int j = 0; j < ntiles; ++j) {
+        const int s = j & 1, mt = mt0 + j;
         if (j >= 2 && !mbar_wait(&xempty[s], ((j - 2) >> 1) & 1, abort_flag)) break;
         uint8_t* slot = xv + s * 2 * S::TILE;
         mbar_arrive_expect_tx(&xfull[s], 2 * S::TILE);
@@ -149,23 +154,34 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
       }
     }
   } else if (warp == 1) {
-    if (elect_one()) {
+    if (elect_one() && ntiles > 0) {
       constexpr uint32_t idZ = make_idesc(128, HID, 1, false, false);
       constexpr uint32_t idV = make_idesc(128, 64, 1, false, false);
       constexpr uint32_t idH = make_idesc(128, HID, 1, false, true);  // B = W2 [d][h], MN-major
+      constexpr uint32_t idG = make_idesc(128, 64, 1, true, true);    // A = H^T / dZ^T, B = dY / X
       const uint32_t w1a = smem_u32(w1s), w2a = smem_u32(w2s), ha = smem_u32(hs), dya = smem_u32(dys);
-      int j = 0, zw = -1, nw = 0;
-      for (int t = blockIdx.x; t < total; t += gridDim.x, ++j) {
-        const int z = t / g.m_tiles;
+      // G1 += dZ^T X of tile jj (keys in slot jj & 1), one 128-row block of h at a time; the
+      // operands are read MN-major: 64-column runs of h 16 KB apart, 16-token steps of 2 KB
+      auto issue_g1 = [&](int jj) {
+        const uint32_t xa = smem_u32(xv + (jj & 1) * 2 * S::TILE);
+        for (int blk = 0; blk < HID / 128; ++blk)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_f16(tmem_base + S::GCOL + 64 * (HID / 128 + blk),
+                    make_sdesc_sw128(ha + blk * 2 * S::TILE + kk * 2048, S::TILE, 1024),
+                    make_sdesc_sw128(xa + kk * 2048, S::TILE, 1024), idG, (jj > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&xempty[jj & 1]);
+      };
+      bool ok = mbar_wait(wfull, 0, abort_flag);
+      for (int j = 0; j < ntiles && ok; ++j) {
         const int s = j & 1;
-        if (z != zw) {
-          if (!mbar_wait(wfull, nw & 1, abort_flag)) break;
-          zw = z;
-          ++nw;
+        if (j > 0) {
+          // dZ of the previous tile in shared memory and its dH read out of TMEM
+          if (!(ok = mbar_wait(dzfull, (j - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_g1(j - 1);
         }
-        // Z of the previous tile read out of TMEM; this tile's keys landed
-        if (j > 0 && !mbar_wait(zempty, (j - 1) & 1, abort_flag)) break;
-        if (!mbar_wait(&xfull[s], (j >> 1) & 1, abort_flag)) break;
+        if (!(ok = mbar_wait(&xfull[s], (j >> 1) & 1, abort_flag))) break;
         tc_fence_after();
         const uint32_t xa = smem_u32(xv + s * 2 * S::TILE);
 #pragma unroll
@@ -173,28 +189,33 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
           mma_f16(tmem_base, make_sdesc_sw128(xa + kk * 32, 16, 1024), make_sdesc_sw128(w1a + kk * 32, 16, 1024), idZ,
                   kk > 0 ? 1u : 0u);
         mma_commit(zfull);
-        mma_commit(&xempty[s]);
-        // V^ = H W2^T once H is in shared memory and the previous tile's dH has been read
-        if (!mbar_wait(hfull, j & 1, abort_flag)) break;
-        if (j > 0 && !mbar_wait(dhempty, (j - 1) & 1, abort_flag)) break;
+        // V^ = H W2^T once H is in shared memory (Z has been read)
+        if (!(ok = mbar_wait(hfull, j & 1, abort_flag))) break;
         tc_fence_after();
         for (int kb = 0; kb < HID / 64; ++kb)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_f16(tmem_base + 256, make_sdesc_sw128(ha + kb * S::TILE + kk * 32, 16, 1024),
+            mma_f16(tmem_base, make_sdesc_sw128(ha + kb * S::TILE + kk * 32, 16, 1024),
                     make_sdesc_sw128(w2a + kb * 64 * 128 + kk * 32, 16, 1024), idV, (kb > 0 || kk > 0) ? 1u : 0u);
         mma_commit(vfull);
-        // dH = dY W2 once dY is in shared memory (V^ has been read by then)
-        if (!mbar_wait(dyfull, j & 1, abort_flag)) break;
+        // dY in shared memory (V^ has been read): G2^T += H^T dY, then dH = dY W2
+        if (!(ok = mbar_wait(dyfull, j & 1, abort_flag))) break;
         tc_fence_after();
+        for (int blk = 0; blk < HID / 128; ++blk)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_f16(tmem_base + S::GCOL + 64 * blk, make_sdesc_sw128(ha + blk * 2 * S::TILE + kk * 2048, S::TILE, 1024),
+                    make_sdesc_sw128(dya + kk * 2048, S::TILE, 1024), idG, (j > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_f16(tmem_base + 256, make_sdesc_sw128(dya + kk * 32, 16, 1024),
+          mma_f16(tmem_base, make_sdesc_sw128(dya + kk * 32, 16, 1024),
                   make_sdesc_sw128(w2a + kk * 16 * 128, 64 * 128, 1024), idH, kk > 0 ? 1u : 0u);
         mma_commit(dhfull);
-        // the next tile of this CTA reads another head's weights: release these
-        const int tn = t + static_cast<int>(gridDim.x);
-        if (tn < total && tn / g.m_tiles != z) mma_commit(wrelease);
+      }
+      if (ok && mbar_wait(dzfull, (ntiles - 1) & 1, abort_flag)) {
+        tc_fence_after();
+        issue_g1(ntiles - 1);
+        mma_commit(gdone);
       }
       if (*abort_flag) {
         volatile int never = 0;
@@ -208,27 +229,28 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
     const int row = q * 32 + lane;
     const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const int c0 = slot * S::COLS;  // hidden columns [c0, c0 + COLS)
-    int j = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++j) {
-      const int mt = t % g.m_tiles, z = t / g.m_tiles;
+    for (int j = 0; j < ntiles && ok; ++j) {
       const int s = j & 1;
-      const int m = mt * 128 + row;
+      const int m = (mt0 + j) * 128 + row;
       const bool valid = m < g.rows_valid;
-      bf16* hrow = g.H + z * g.h_zs + int64_t(m) * HID + c0;
-      bf16* zrow = g.dZ + z * g.h_zs + int64_t(m) * HID + c0;
-      bf16* yrow = g.dY + z * g.y_zs + int64_t(m) * S::D + slot * 16;
-      // ---- E1: H = GELU(Z), G' kept packed in registers
+      // ---- E1: H = GELU(Z) into shared memory (the previous tile's G1, which read dZ
+      // there, completed before Z did), G' kept packed in registers
       ok = __all_sync(0xffffffffu, mbar_wait(zfull, j & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       uint32_t gp[S::COLS / 2];
 #pragma unroll
-      for (int cc = 0; cc < S::COLS; cc += 32) {
-        float zv[32], hv[32];
-        tmem_ld32(tq + c0 + cc, zv);
+      for (int cc = 0; cc < S::COLS; cc += 16) {
+        uint32_t zr[16];
+        float hv[16];
+        tmem_ld16_async(tq + c0 + cc, zr);
+        tmem_wait_regs(zr);
+        float zv[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
+        for (int i = 0; i < 16; ++i) zv[i] = __uint_as_float(zr[i]);
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
           float g0, g1, p0, p1;
           gelu_and_grad(zv[i], g0, p0);
           gelu_and_grad(zv[i + 1], g1, p1);
@@ -236,30 +258,19 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
           hv[i + 1] = valid ? g1 : 0.f;
           gp[(cc + i) / 2] = pack_bf16x2(p0, p1);
         }
-        // H: the k-block of column c0 + cc in shared memory (next MMA's operand) and HBM
-        uint8_t* kb = hs + ((c0 + cc) / 64) * S::TILE;
-        const int k0 = ((c0 + cc) % 64) / 8;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          *sw128_chunk(kb, row, k0 + k) =
-              make_uint4(pack_bf16x2(hv[8 * k], hv[8 * k + 1]), pack_bf16x2(hv[8 * k + 2], hv[8 * k + 3]),
-                         pack_bf16x2(hv[8 * k + 4], hv[8 * k + 5]), pack_bf16x2(hv[8 * k + 6], hv[8 * k + 7]));
-        if (m < g.m_tiles * 128) store_bf16x32(hrow + cc, hv);
+        put_row16(hs + ((c0 + cc) / 64) * S::TILE, row, ((c0 + cc) % 64) / 8, hv);
       }
       tc_fence_before();
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(zempty);
-        mbar_arrive(hfull);
-      }
+      if (lane == 0) mbar_arrive(hfull);
       // ---- E2: dY = coef eta (V^ - V) on this warp's 16 output channels
       ok = __all_sync(0xffffffffu, mbar_wait(vfull, j & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       {
         uint32_t vr[16];
-        tmem_ld16_async(tq + 256 + slot * 16, vr);
+        tmem_ld16_async(tq + slot * 16, vr);
         tmem_wait_regs(vr);
         const float e = valid ? (g.eta ? g.eta[z * g.eta_zs + g.t0 + m] : g.eta_scalar) * g.coef : 0.f;
         const uint8_t* vt = xv + s * 2 * S::TILE + S::TILE;  // the V tile (128-byte swizzled rows)
@@ -280,11 +291,6 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
         for (int i = 0; i < 8; ++i) yp[i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
         *sw128_chunk(dys, row, slot * 2) = make_uint4(yp[0], yp[1], yp[2], yp[3]);
         *sw128_chunk(dys, row, slot * 2 + 1) = make_uint4(yp[4], yp[5], yp[6], yp[7]);
-        if (m < g.m_tiles * 128) {
-          uint4* yd = reinterpret_cast<uint4*>(yrow);
-          yd[0] = make_uint4(yp[0], yp[1], yp[2], yp[3]);
-          yd[1] = make_uint4(yp[4], yp[5], yp[6], yp[7]);
-        }
       }
       tc_fence_before();
       fence_proxy_async_smem();
@@ -293,25 +299,53 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
         mbar_arrive(dyfull);
         mbar_arrive(&xempty[s]);
       }
-      // ---- E3: dZ = dH * G'
+      // ---- E3: dZ = dH * G' into shared memory over H (G2^T, its last reader, is done)
       ok = __all_sync(0xffffffffu, mbar_wait(dhfull, j & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
-      for (int cc = 0; cc < S::COLS; cc += 32) {
-        float dh[32];
-        tmem_ld32(tq + 256 + c0 + cc, dh);
+      for (int cc = 0; cc < S::COLS; cc += 16) {
+        uint32_t dr[16];
+        tmem_ld16_async(tq + c0 + cc, dr);
+        tmem_wait_regs(dr);
+        float dh[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
+        for (int i = 0; i < 16; ++i) dh[i] = __uint_as_float(dr[i]);
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
           const float2 gpf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gp[(cc + i) / 2]));
           dh[i] = valid ? dh[i] * gpf.x : 0.f;
           dh[i + 1] = valid ? dh[i + 1] * gpf.y : 0.f;
         }
-        if (m < g.m_tiles * 128) store_bf16x32(zrow + cc, dh);
+        put_row16(hs + ((c0 + cc) / 64) * S::TILE, row, ((c0 + cc) % 64) / 8, dh);
       }
       tc_fence_before();
+      fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(dhempty);
+      if (lane == 0) mbar_arrive(dzfull);
+    }
+    // ---- the CTA's gradient partials: accumulator columns [slot PER, (slot + 1) PER)
+    if (ok && ntiles > 0) ok = __all_sync(0xffffffffu, mbar_wait(gdone, 0, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      constexpr int PER = 16 * S::NACC;  // columns per warp slot (64 or 32)
+      const int a0 = slot * PER;
+      const int acc = a0 / 64, col0 = a0 % 64;
+      const int grow = (acc < S::NACC / 2 ? 128 * acc : HID + 128 * (acc - S::NACC / 2)) + row;
+      float* dst = g.part + ((int64_t(sp) * g.batches + z) * (2 * HID) + grow) * 64 + col0;
+#pragma unroll
+      for (int cc = 0; cc < PER; cc += 32) {
+        float v[32];
+        if (ntiles > 0) {
+          tmem_ld32(tq + S::GCOL + a0 + cc, v);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(dst + cc + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      }
     }
   }
 
@@ -332,11 +366,10 @@ cudaError_t launch_mse_token(const CUtensorMap& tX, const CUtensorMap& tV, const
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
   });
   if (set != 0) return static_cast<cudaError_t>(set);
-  const long long total = static_cast<long long>(g.m_tiles) * g.batches;
-  if (total <= 0) return cudaSuccess;
-  if (total > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  const int grid = static_cast<int>(std::min<long long>(total, sm_count()));
-  kern<<<grid, 64 + 32 * S::EW, S::SMEM, st>>>(tX, tV, tW1, tW2, g, status);
+  if (g.splits < 1 || g.batches < 1 || g.m_tiles < 1) return cudaErrorInvalidValue;
+  const long long grid = static_cast<long long>(g.batches) * g.splits;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  kern<<<static_cast<int>(grid), 64 + 32 * S::EW, S::SMEM, st>>>(tX, tV, tW1, tW2, g, status);
   return cudaGetLastError();
 }
 

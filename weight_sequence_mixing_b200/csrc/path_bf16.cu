@@ -53,7 +53,8 @@ enum BBuf {
   xAct2,   // bf16 [Z][Cp][h]  (GELU' for MSE)
   xDY,     // bf16 [Z][Cp][d]  (dL/dV_hat for MSE / linear)
   xHq,     // bf16 apply hidden [Z][Rq][h]
-  xKstat,  // fp32 key-norm partial sums [Z][Cp/128][d][2], then [Z][d][2] mean and 1/std
+  xKstat,  // fp32 key-norm partial sums [Z][Cp/128][d][2], then [Z][d][2] mean and 1/std, then
+           // [Z] u32 counters of the blocks done (zero between launches)
   xNX, xNXT, xNX2, xNXT2, xNS, xNT,  // fp32 Newton-Schulz buffers [Z*nmat][...]
   kNumBBuf
 };
@@ -66,6 +67,13 @@ struct Dims {
 };
 
 int bn_for(int n) { return n % 256 == 0 ? 256 : n % 128 == 0 ? 128 : 64; }
+
+// The GELU MLP with the MSE loss at d = 64 and h = 128 or 256 runs its token phase and
+// weight gradients in one kernel (mse_token.cuh), one CTA per head and token-tile range,
+// which writes split partials of the gradients.
+bool mse_token_path(const ttt_config& c) {
+  return c.inner == TTT_INNER_MLP2_GELU && c.loss == TTT_LOSS_MSE && c.d == 64 && (c.h == 128 || c.h == 256);
+}
 
 Dims dims_of(const Plan& p) {
   const ttt_config& c = p.cfg;
@@ -94,7 +102,7 @@ Dims dims_of(const Plan& p) {
   const bool muon = c.opt == TTT_OPT_MUON || c.opt == TTT_OPT_MOMENTUM_MUON;
   // with Muon the squared row norms are summed over the tiles of a row: allow at
   // most two contributions per row (order-independent)
-  D.direct = D.splits == 1 && !(muon && D.grad_bn != c.d);
+  D.direct = D.splits == 1 && !(muon && D.grad_bn != c.d) && !mse_token_path(c);
   D.token_pairs = (c.flags & TTT_FLAG_SINGLE_CTA) == 0;
   return D;
 }
@@ -144,23 +152,19 @@ struct RowMap {
   }
 };
 
-__global__ void init_weights_kernel(int Z, int H, int64_t P, const float* W0, float* W) {
-  const int64_t total = int64_t(Z) * P;
-  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x)
-    W[i] = W0[int64_t(int(i / P) % H) * P + i % P];
-}
-
 // One warp per canonical weight row: [W -= lr U] -> [row L2-norm] -> bf16 copies
 // (+ the non-finite check of the layer's weights).  W2^T is made from the bf16 W2
 // afterwards by transpose_w2_kernel.
-//   mode 0: no update (initial weights)
+//   mode 0: no update (initial weights: W = W0 first when W0 is given; W0 [w0_rows][P],
+//           row z % w0_rows for batch-head z)
 //   mode 1: U from the gradient layout
 //   mode 2: U from the Newton-Schulz result (X [m][n], XT [n][m] per matrix)
 // hold_w2: the rows of W2 keep their values (first-layer-only updates): no step,
 // no row norm; their bf16 copies are rewritten unchanged.
 __global__ void finish_rows_kernel(RowMap rm, int mode, float lr, bool rownorm, bool hold_w2, float* Wf,
                                    const float* U, const float* X, const float* XT, int m, int n, bool src_t,
-                                   bf16* First, bf16* W2T, bf16* W2, unsigned* status) {
+                                   bf16* First, bf16* W2T, bf16* W2, unsigned* status, const float* W0 = nullptr,
+                                   int w0_rows = 1) {
   const int z = blockIdx.y;
   const int R = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   if (R >= rm.nrows()) return;
@@ -174,6 +178,10 @@ __global__ void finish_rows_kernel(RowMap rm, int mode, float lr, bool rownorm, 
   if (w2 && hold_w2) {
     mode = 0;
     rownorm = false;
+  }
+  if (mode == 0 && W0) {
+    const float* src = W0 + int64_t(z % w0_rows) * rm.P + off + int64_t(r) * len;
+    for (int i = lane; i < len; i += 32) w[i] = src[i];
   }
   if (mode == 1) {
     const float* Uz = U + int64_t(z) * rm.GR * rm.d;
@@ -239,55 +247,78 @@ __global__ void transpose_w2_kernel(int d, int h, const bf16* W2, bf16* W2T) {
     if (c0 + j < h && r0 + tx < d) dst[int64_t(c0 + j) * d + r0 + tx] = tile[tx][j];
 }
 
-// Key instance-norm, pass 1: per 128-token block and channel, the sum and sum of
-// squares of the chunk's keys (rows past the chunk count as absent).
-__global__ void keystats_kernel(int n, int d, const bf16* K, int64_t k_zs, int t0, float* part) {
-  __shared__ float red[8][2][64];
+// Key instance-norm (per head, per channel, over the chunk's tokens).  Both passes
+// move the keys in 16-byte pieces of 8 channels: thread t owns piece t % cpr of a row
+// (cpr = channels / 8 of the current window of at most 2048 channels) and rows
+// t / cpr, t / cpr + 256 / cpr, ...
+//
+// Pass 1: per (z, 128-token block), channel sums and sums of squares -> part[z][blk][ch][2].
+// The block that finishes last for its head (a counter per head, reset by that block)
+// combines the block sums in block order, in double (the biased variance is
+// E[k^2] - E[k]^2), into the mean and 1/sqrt(var + eps) -> stats[z][ch][2].
+__global__ void keystats_kernel(int n, int d, const bf16* K, int64_t k_zs, int t0, float eps, float* part,
+                                float* stats, unsigned* done) {
+  __shared__ float red[2][2048];  // [sum | sum of squares][row group x channel of the window]
+  __shared__ bool last;
   const int z = blockIdx.y, blk = blockIdx.x, nb = gridDim.x;
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  for (int c0 = 0; c0 < d; c0 += 64) {
-    float s0 = 0.f, s1 = 0.f, q0 = 0.f, q1 = 0.f;
-    for (int r = blk * 128 + w; r < min(n, blk * 128 + 128); r += 8) {
-      const float2 v = __bfloat1622float2(
-          *reinterpret_cast<const __nv_bfloat162*>(K + z * k_zs + int64_t(t0 + r) * d + c0 + 2 * lane));
-      s0 += v.x;
-      s1 += v.y;
-      q0 += v.x * v.x;
-      q1 += v.y * v.y;
+  const int tid = threadIdx.x;
+  const int rows = min(n - blk * 128, 128);
+  for (int c0 = 0; c0 < d; c0 += 2048) {
+    const int w = min(d - c0, 2048), cpr = w / 8, groups = 256 / cpr;
+    const int piece = tid % cpr, grp = tid / cpr;
+    float s[8] = {}, q[8] = {};
+    if (grp < groups) {
+      const bf16* base = K + z * k_zs + int64_t(t0 + blk * 128) * d + c0 + 8 * piece;
+#pragma unroll 4
+      for (int r = grp; r < rows; r += groups) {
+        const uint4 u = *reinterpret_cast<const uint4*>(base + int64_t(r) * d);
+        const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wd[i]));
+          s[2 * i] += f.x;
+          s[2 * i + 1] += f.y;
+          q[2 * i] = fmaf(f.x, f.x, q[2 * i]);
+          q[2 * i + 1] = fmaf(f.y, f.y, q[2 * i + 1]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        red[0][grp * w + 8 * piece + i] = s[i];
+        red[1][grp * w + 8 * piece + i] = q[i];
+      }
     }
-    red[w][0][2 * lane] = s0;
-    red[w][0][2 * lane + 1] = s1;
-    red[w][1][2 * lane] = q0;
-    red[w][1][2 * lane + 1] = q1;
     __syncthreads();
-    if (threadIdx.x < 128) {
-      const int which = threadIdx.x >> 6, ch = threadIdx.x & 63;
+    for (int e = tid; e < 2 * w; e += blockDim.x) {
+      const int which = e / w, ch = e % w;
       float t = 0.f;
-      for (int j = 0; j < 8; ++j) t += red[j][which][ch];
+      for (int gi = 0; gi < groups; ++gi) t += red[which][gi * w + ch];
       part[((int64_t(z) * nb + blk) * d + c0 + ch) * 2 + which] = t;
     }
     __syncthreads();
   }
-}
-
-// Pass 2: per (z, channel), the block sums combined in block order (in double: the
-// biased variance is E[k^2] - E[k]^2) into the mean and 1/sqrt(var + eps).
-__global__ void keystats_final_kernel(int n, int d, int nb, float eps, const float* part, float* stats) {
-  const int z = blockIdx.y;
-  const int ch = blockIdx.x * blockDim.x + threadIdx.x;
-  if (ch >= d) return;
-  double s = 0.0, q = 0.0;
-  for (int b = 0; b < nb; ++b) {
-    s += part[((int64_t(z) * nb + b) * d + ch) * 2];
-    q += part[((int64_t(z) * nb + b) * d + ch) * 2 + 1];
+  // the last block of head z to finish finalises its statistics
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) last = atomicAdd(&done[z], 1u) == static_cast<unsigned>(nb - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  for (int ch = tid; ch < d; ch += blockDim.x) {
+    double sum = 0.0, sq = 0.0;
+    for (int b = 0; b < nb; ++b) {
+      sum += __ldcg(part + ((int64_t(z) * nb + b) * d + ch) * 2);
+      sq += __ldcg(part + ((int64_t(z) * nb + b) * d + ch) * 2 + 1);
+    }
+    const double mean = sum / n;
+    const double var = fmax(sq / n - mean * mean, 0.0);
+    stats[(int64_t(z) * d + ch) * 2] = static_cast<float>(mean);
+    stats[(int64_t(z) * d + ch) * 2 + 1] = static_cast<float>(1.0 / sqrt(var + eps));
   }
-  const double mean = s / n;
-  const double var = fmax(q / n - mean * mean, 0.0);
-  stats[(int64_t(z) * d + ch) * 2] = static_cast<float>(mean);
-  stats[(int64_t(z) * d + ch) * 2 + 1] = static_cast<float>(1.0 / sqrt(var + eps));
+  if (tid == 0) done[z] = 0u;
 }
 
-// Pass 3: normalise the chunk's keys, Kn = (k - mean) * rstd, zeros for rows past the chunk.
+// Pass 2: normalise the chunk's keys, Kn = (k - mean) * rstd, zeros for rows past the chunk.
 __global__ void keynorm_kernel(int n, int d, const bf16* K, int64_t k_zs, int t0, const float* stats, bf16* Kn,
                                int64_t kn_zs) {
   extern __shared__ float st[];  // [d] mean, [d] rstd
@@ -297,19 +328,27 @@ __global__ void keynorm_kernel(int n, int d, const bf16* K, int64_t k_zs, int t0
     st[d + ch] = stats[(int64_t(z) * d + ch) * 2 + 1];
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  for (int r = blk * 128 + w; r < blk * 128 + 128; r += 8) {
-    for (int c0 = 0; c0 < d; c0 += 64) {
-      const int ch = c0 + 2 * lane;
-      float a = 0.f, b = 0.f;
-      if (r < n) {
-        const float2 v = __bfloat1622float2(
-            *reinterpret_cast<const __nv_bfloat162*>(K + z * k_zs + int64_t(t0 + r) * d + ch));
-        a = (v.x - st[ch]) * st[d + ch];
-        b = (v.y - st[ch + 1]) * st[d + ch + 1];
+  const int cpr = d / 8;  // 16-byte pieces per row
+  const int total = 128 * cpr;
+#pragma unroll 4
+  for (int e = threadIdx.x; e < total; e += blockDim.x) {
+    const int r = e / cpr, ch = 8 * (e % cpr);
+    const int row = blk * 128 + r;
+    uint4 out = make_uint4(0u, 0u, 0u, 0u);
+    if (row < n) {
+      const uint4 u = *reinterpret_cast<const uint4*>(K + z * k_zs + int64_t(t0 + row) * d + ch);
+      const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wd[i]));
+        const int c = ch + 2 * i;
+        const __nv_bfloat162 b = __floats2bfloat162_rn((f.x - st[c]) * st[d + c], (f.y - st[c + 1]) * st[d + c + 1]);
+        o[i] = *reinterpret_cast<const uint32_t*>(&b);
       }
-      *reinterpret_cast<__nv_bfloat162*>(Kn + z * kn_zs + int64_t(r) * d + ch) = __floats2bfloat162_rn(a, b);
+      out = make_uint4(o[0], o[1], o[2], o[3]);
     }
+    *reinterpret_cast<uint4*>(Kn + z * kn_zs + int64_t(row) * d + ch) = out;
   }
 }
 
@@ -507,10 +546,11 @@ struct Ctx {
 };
 
 // bf16 W2^T from the freshly written bf16 W2: the B operand of the single-CTA token
-// kernel and of the MSE path's dH = dY W2.  The pair token kernel reads W2 itself.
+// kernel and of the generic MSE path's dH = dY W2.  The pair token kernel, the fused MSE
+// token kernel and the apply read W2 itself.
 int transpose_w2(Ctx& c) {
   const ttt_config& cfg = c.p.cfg;
-  if (cfg.inner == TTT_INNER_LINEAR || cfg.inner == TTT_INNER_GLU) return TTT_OK;
+  if (cfg.inner == TTT_INNER_LINEAR || cfg.inner == TTT_INNER_GLU || mse_token_path(cfg)) return TTT_OK;
   if (cfg.loss == TTT_LOSS_NEG_DOT && c.D.token_pairs &&
       (cfg.inner == TTT_INNER_SWIGLU ? token_pair_capacity<true>() : token_pair_capacity<false>()) > 0)
     return TTT_OK;
@@ -728,15 +768,13 @@ int update_chunk(Ctx& c, int t0, int n) {
   if (cfg.flags & TTT_FLAG_KEY_INSTNORM) {
     bf16* Kn = c.v.at<bf16>(p, xKn);
     float* kst = c.v.at<float>(p, xKstat);
+    const int nb = (n + 127) / 128;  // token blocks holding keys of the chunk
     const dim3 gk(Cp / 128, Z);
+    float* kfin = kst + size_t(Z) * (Cp / 128) * d * 2;                   // [Z][d][2] mean, rstd
+    unsigned* kdone = reinterpret_cast<unsigned*>(kfin + size_t(Z) * d * 2);  // [Z] blocks finished
     {
       StageScope _sc(kStageKeyNorm, st);
-      keystats_kernel<<<gk, 256, 0, c.st>>>(n, d, K, int64_t(D.N) * d, t0, kst);
-    }
-    float* kfin = kst + size_t(Z) * (Cp / 128) * d * 2;  // [Z][d][2] mean, rstd
-    {
-      StageScope _sc(kStageKeyNorm, st);
-      keystats_final_kernel<<<dim3((d + 127) / 128, Z), 128, 0, c.st>>>(n, d, Cp / 128, cfg.in_eps, kst, kfin);
+      keystats_kernel<<<dim3(nb, Z), 256, 0, c.st>>>(n, d, K, int64_t(D.N) * d, t0, cfg.in_eps, kst, kfin, kdone);
     }
     {
       StageScope _sc(kStageKeyNorm, st);
@@ -773,15 +811,17 @@ int update_chunk(Ctx& c, int t0, int n) {
     TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
     TRY(tmap(&tD, A1, 2, h, Cp, Z, 64));
     TRY(grad_gemm(c, tH, c.tVmn, tD, *tXmn, h, h, h, t0, xoff));
-  } else if (cfg.inner == TTT_INNER_MLP2_GELU && cfg.loss == TTT_LOSS_MSE && d == 64 && (h == 128 || h == 256)) {
-    // one kernel for Z, GELU, V_hat, the MSE gradient and dH (mse_token.cuh) -> H, dY, dZ
+  } else if (mse_token_path(cfg)) {
+    // one kernel: Z, GELU, V_hat, the MSE gradient, dH, dZ and the gradient reductions
+    // G2^T = H^T dY, G1 = dZ^T X per (head, token-tile range) -> split partials (mse_token.cuh)
     TM tw1, tw2;
     TRY(tmap(&tw1, c.v.at<bf16>(p, xFirst), 2, d, h, Z, h));
     TRY(tmap(&tw2, c.v.at<bf16>(p, xW2), 2, h, d, Z, 64));
-    if (tX->box != 128 || c.tV.box != 128) return TTT_ERR_INVALID_ARG;
+    if (tX->box != 128 || c.tV.box != 128 || D.direct) return TTT_ERR_INVALID_ARG;
     MseGeom mg;
-    mg.m_tiles = mt;
+    mg.m_tiles = (n + 127) / 128;
     mg.batches = Z;
+    mg.splits = D.splits;
     mg.rows_valid = n;
     mg.x_off = xoff;
     mg.v_off = t0;
@@ -790,23 +830,13 @@ int update_chunk(Ctx& c, int t0, int n) {
     mg.eta_zs = D.N;
     mg.eta_scalar = cfg.eta_scalar;
     mg.coef = 2.0f / (float(n) * float(d));
-    mg.H = A0;
-    mg.dY = DY;
-    mg.dZ = A1;
-    mg.h_zs = int64_t(Cp) * h;
-    mg.y_zs = int64_t(Cp) * d;
+    mg.part = c.v.at<float>(p, xPart);
     {
       StageScope sc(kStageTokenPhase, c.st);
       const cudaError_t e = h == 256 ? launch_mse_token<256>(tX->m, c.tV.m, tw1.m, tw2.m, mg, status, c.st)
                                      : launch_mse_token<128>(tX->m, c.tV.m, tw1.m, tw2.m, mg, status, c.st);
       TRY_CUDA(e);
     }
-    // G2^T = H^T dY (rows [0,h)), G1 = dZ^T X (rows [h,2h))
-    TM tH, tYmn, tD;
-    TRY(tmap(&tH, A0, 2, h, Cp, Z, 64));
-    TRY(tmap(&tYmn, DY, 2, d, Cp, Z, 64));
-    TRY(tmap(&tD, A1, 2, h, Cp, Z, 64));
-    TRY(grad_gemm(c, tH, tYmn, tD, *tXmn, h, h, h, 0, xoff));
   } else if (cfg.inner == TTT_INNER_MLP2_GELU) {  // MSE, RMSE
     // Z = X W1^T -> H = GELU(Z), G' = GELU'(Z)
     EpiGeluSave e1{A0, A2, h, n, int64_t(Cp) * h};
@@ -960,6 +990,13 @@ void choose_grad_shape(const Plan& p, int Cp, int* splits, int* tile_rows, int* 
                                                     : 3 * h;
   const int r0 = c.inner == TTT_INNER_LINEAR ? d : c.inner == TTT_INNER_GLU ? 2 * d : h;
   const int kblocks = Cp / 64;
+  if (mse_token_path(c)) {
+    // the fused MSE kernel: one CTA per (head, token-tile range), one wave of them
+    *splits = std::max(1, std::min(Cp / 128, kPlanSMs / std::max(1, p.BH)));
+    *tile_rows = 128;
+    *grad_bn = 64;
+    return;
+  }
   // each split reduces at least 1024 tokens: below that the fp32 partials it writes
   // and the reduction reads cost more than the parallelism gains; chunks of at most
   // 4096 tokens are not split at all (the gradient then goes straight to the optimizer)
@@ -1018,6 +1055,7 @@ int plan_layout_bf16(Plan* p) {
   const int64_t ZK = Z * D.nmat;
   const bool mlp_mse = c.inner == TTT_INNER_MLP2_GELU && c.loss != TTT_LOSS_NEG_DOT;  // MSE, RMSE
   const bool act = c.inner != TTT_INNER_LINEAR && !glu;  // a hidden layer and W2
+  const bool spill = !mse_token_path(c);                   // activations go through HBM
   const int64_t bytes[kNumBBuf] = {
       Z * P * 4,
       Z * GR * d * 4,
@@ -1028,12 +1066,12 @@ int plan_layout_bf16(Plan* p) {
       act ? Z * h * d * 2 : 0,
       act ? Z * d * h * 2 : 0,
       (c.flags & TTT_FLAG_KEY_INSTNORM) ? Z * Cp * d * 2 : 0,
-      act ? Z * Cp * h * 2 : 0,
-      (act || glu) ? Z * Cp * 2 * h * 2 : 0,  // dZ13 / dZ (GLU: h = d)
-      mlp_mse ? Z * Cp * h * 2 : 0,
-      (mlp_mse || !act) ? Z * Cp * d * 2 : 0,
+      (act && spill) ? Z * Cp * h * 2 : 0,
+      ((act && spill) || glu) ? Z * Cp * 2 * h * 2 : 0,  // dZ13 / dZ (GLU: h = d)
+      (mlp_mse && spill) ? Z * Cp * h * 2 : 0,
+      ((mlp_mse && spill) || !act) ? Z * Cp * d * 2 : 0,
       (act && d != 64 && d != 128 && d != 256) ? Z * D.Rq * h * 2 : 0,  // two-GEMM apply only (d = 512)
-      (c.flags & TTT_FLAG_KEY_INSTNORM) ? Z * (Cp / 128 + 1) * d * 2 * 4 : 0,  // block sums, then mean / rstd
+      (c.flags & TTT_FLAG_KEY_INSTNORM) ? Z * (Cp / 128 + 1) * d * 2 * 4 + Z * 4 : 0,  // block sums, mean / rstd, counters
       muon ? ZK * nm * 4 : 0,
       muon ? ZK * nm * 4 : 0,
       muon ? ZK * nm * 4 : 0,
@@ -1077,25 +1115,24 @@ int run_bf16(const Plan& p, const Io& io, void* ws, cudaStream_t st) {
     TRY(tmap(&c.tW2T, c.v.at<bf16>(p, xW2T), 2, d, h, Z, cfg.loss == TTT_LOSS_NEG_DOT ? 128 : bn_for(h)));
     TRY(tmap(&c.tW2, c.v.at<bf16>(p, xW2), 2, h, d, Z, bn_for(d)));
   }
-  // W = W0 per batch entry, zero momentum, bf16 copies
-  {
-    StageScope _sc(kStageOther, st);
-    // W0 [H][P] shared by the batch entries, or [B*H][P] with one state per entry
-    const int w0_rows = (cfg.flags & TTT_FLAG_W0_PER_BATCH) ? Z : cfg.H;
-    init_weights_kernel<<<std::min<int64_t>((int64_t(Z) * p.P + 255) / 256, 4096), 256, 0, st>>>(
-        Z, w0_rows, p.P, io.W0, c.v.at<float>(p, xWf));
-  }
+  // W = W0 per batch entry (W0 [H][P] shared by the batch entries, or [B*H][P] with one
+  // state per entry) and its bf16 copies in one pass; zero momentum
+  const int w0_rows = (cfg.flags & TTT_FLAG_W0_PER_BATCH) ? Z : cfg.H;
   if (io.M_in && p.state_bytes)
     TRY_CUDA(cudaMemcpyAsync(c.v.at<float>(p, xMom), io.M_in, p.state_bytes, cudaMemcpyDeviceToDevice, st));
   else
     TRY_CUDA(cudaMemsetAsync(c.v.at<float>(p, xMom), 0, size_t(Z) * D.GR * d * 4, st));
+  if (cfg.flags & TTT_FLAG_KEY_INSTNORM) {  // the key-statistics counters start at zero
+    float* kfin = c.v.at<float>(p, xKstat) + size_t(Z) * (D.Cp / 128) * d * 2;
+    TRY_CUDA(cudaMemsetAsync(kfin + size_t(Z) * d * 2, 0, size_t(Z) * 4, st));
+  }
   {
     dim3 g((c.rm.nrows() + 7) / 8, Z);
     {
       StageScope _sc(kStageFinish, st);
       finish_rows_kernel<<<g, 256, 0, st>>>(c.rm, 0, 0.f, false, false, c.v.at<float>(p, xWf), nullptr, nullptr,
                                             nullptr, 0, 0, false, First, c.v.at<bf16>(p, xW2T), c.v.at<bf16>(p, xW2),
-                                            c.v.status);
+                                            c.v.status, io.W0, w0_rows);
     }
     TRY_CUDA(cudaGetLastError());
     TRY(transpose_w2(c));
