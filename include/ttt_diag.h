@@ -25,6 +25,16 @@ extern "C" {
 int ttt_selftest_gemm(int elem_bytes, int a_mn, int b_mn, int bn, int M, int N, int K, int batches, int splits,
                       const void* A, const void* B, float* C, void* stream);
 
+/* The activation functions the epilogues use, elementwise on n fp32 device values:
+ *   kind 0: y = GELU(x) = x Phi(x), dy = GELU'(x) = Phi(x) + x phi(x) (Phi, phi: the standard
+ *           normal CDF and density; erf from Abramowitz & Stegun 7.1.26, |error| <= 1.5e-7)
+ *   kind 1: y = SiLU(x) = x sigma(x), dy = sigma(x) (1 + x (1 - sigma(x))) (sigma from the
+ *           hardware tanh approximation, relative error about 2^-11)
+ * (the GELU of the ViT3 MLP inner model and the SiLU of the SwiGLU / GLU inner models).
+ * x, y, dy: device buffers of n floats, caller-owned.  Enqueued on `stream`;
+ * TTT_ERR_INVALID_ARG for an unknown kind or missing buffers, TTT_ERR_CUDA if the launch fails. */
+int ttt_selftest_activation(int kind, int64_t n, const float* x, float* y, float* dy, void* stream);
+
 /* The execution plan ttt_create chose (host logic only, no GPU needed).  Writes up to
  * `n` ints into `info`, in this order:
  *   [0] path: 0 fp32 SIMT, 1 bf16 tensor cores, 2 DWConv (SIMT, either dtype)

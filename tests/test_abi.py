@@ -288,6 +288,10 @@ def test_every_entry_point_refuses_a_null_handle_or_buffer_without_gpu_work():
     info = (ctypes.c_int * 7)()
     assert lib.ttt_plan_info(None, info, 7) == inv
     assert lib.ttt_selftest_timeout(None, None) == inv
+    assert lib.ttt_selftest_activation(2, 16, fake, fake, fake, None) == inv  # unknown kind
+    assert lib.ttt_selftest_activation(0, 16, None, fake, fake, None) == inv
+    assert lib.ttt_selftest_activation(0, -1, fake, fake, fake, None) == inv
+    assert lib.ttt_selftest_activation(0, 0, None, None, None, None) == 0  # nothing to do
     assert lib.ttt_selftest_gemm(2, 0, 0, 64, 128, 64, 64, 1, 1, None, fake, fake, None) == inv
     lib.ttt_destroy(None)  # a no-op
     assert lib.ttt_stage_name(99) == b"unknown"

@@ -39,7 +39,7 @@ EXPORTED = [
     "ttt_host_staging_size", "ttt_forward_host", "ttt_query_status", "ttt_destroy", "ttt_status_string",
     "ttt_selftest_gemm", "ttt_profile_enable", "ttt_profile_collect", "ttt_stage_name", "ttt_launch_count",
     "ttt_forward_noalloc", "ttt_token_pair_capacity", "ttt_selftest_timeout", "ttt_plan_info",
-    "ttt_state_size", "ttt_forward_state",
+    "ttt_state_size", "ttt_forward_state", "ttt_selftest_activation",
 ]
 NUM_STAGES = 8
 
@@ -87,6 +87,7 @@ def _load():
         "ttt_forward_noalloc": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "ttt_token_pair_capacity": (i32, [i32]),
         "ttt_selftest_timeout": (i32, [vp, vp]),
+        "ttt_selftest_activation": (i32, [i32, i64, vp, vp, vp, vp]),
         "ttt_plan_info": (i32, [vp, ctypes.POINTER(ctypes.c_int), i32]),
         "ttt_state_size": (sz, [vp]),
         "ttt_forward_state": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -306,6 +307,16 @@ def token_pair_capacity(swiglu: bool) -> int:
 def selftest_timeout(status_word: torch.Tensor, stream=None) -> int:
     """Status (TTT_ERR_TIMEOUT expected) of a kernel whose bounded wait runs out; see ttt_diag.h."""
     return int(LIB.ttt_selftest_timeout(_ptr(status_word), _stream_ptr(stream)))
+
+
+def selftest_activation(kind: str, x: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """The epilogues' activation ("gelu" or "silu") and its derivative on fp32 device values; see ttt_diag.h."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous fp32 CUDA tensor")
+    y, dy = torch.empty_like(x), torch.empty_like(x)
+    _check(LIB.ttt_selftest_activation({"gelu": 0, "silu": 1}[kind], x.numel(), _ptr(x), _ptr(y), _ptr(dy),
+                                       _stream_ptr(stream)), "ttt_selftest_activation")
+    return y, dy
 
 
 PLAN_FIELDS = ("path", "chunk", "nchunks", "splits", "tile_rows", "grad_bn", "direct")

@@ -15,12 +15,55 @@ namespace ttt {
 using bf16 = __nv_bfloat16;
 
 // ------------------------------------------------------------------ helpers
-__device__ __forceinline__ float gelu_dev(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
-// GELU(x) = x Phi(x) and its derivative Phi(x) + x phi(x) with one erf evaluation
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// Standard normal CDF Phi(x) = (1 + erf(x / sqrt 2)) / 2 and density phi(x), with erf from
+// Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26:
+//   erf(u) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-u^2),  t = 1 / (1 + p u),  u >= 0,
+// absolute error <= 1.5e-7, far below the bf16 rounding of every GELU output.  With
+// u = |x| / sqrt 2, exp(-u^2) = exp(-x^2 / 2) is also the density's exponential, so one
+// evaluation serves both.  The coefficients are the published ones; here a1..a5 carry Phi's
+// factor 1/2 and p the 1/sqrt 2 of u.
+namespace normal_as {
+constexpr float kP = 0.3275911f * 0.70710678118654752f;
+constexpr float kA1 = 0.5f * 0.254829592f, kA2 = 0.5f * -0.284496736f, kA3 = 0.5f * 1.421413741f,
+                kA4 = 0.5f * -1.453152027f, kA5 = 0.5f * 1.061405429f;
+constexpr float kNegHalfLog2e = -0.72134752044448170f;  // -log2(e) / 2: exp(-x^2/2) = 2^(x^2 kNegHalfLog2e)
+constexpr float kInvSqrt2Pi = 0.39894228040143268f;
+}  // namespace normal_as
+__device__ __forceinline__ void normal_cdf_pdf(float x, float& cdf, float& pdf) {
+  using namespace normal_as;
+  const float t = rcp_approx(fmaf(kP, fabsf(x), 1.0f));
+  float y = fmaf(kA5, t, kA4);
+  y = fmaf(y, t, kA3);
+  y = fmaf(y, t, kA2);
+  y = fmaf(y, t, kA1);
+  y *= t;
+  const float e = ex2_approx(x * x * kNegHalfLog2e);
+  const float q = y * e;  // Phi(-|x|)
+  cdf = x >= 0.0f ? 1.0f - q : q;
+  pdf = e * kInvSqrt2Pi;
+}
+// GELU(x) = x Phi(x)
+__device__ __forceinline__ float gelu_dev(float x) {
+  float c, p;
+  normal_cdf_pdf(x, c, p);
+  return x * c;
+}
+// GELU(x) and its derivative Phi(x) + x phi(x)
 __device__ __forceinline__ void gelu_and_grad(float x, float& g, float& gp) {
-  const float cdf = 0.5f * (1.0f + erff(x * 0.70710678118654752f));
-  g = x * cdf;
-  gp = fmaf(x * 0.39894228040143268f, __expf(-0.5f * x * x), cdf);
+  float c, p;
+  normal_cdf_pdf(x, c, p);
+  g = x * c;
+  gp = fmaf(x, p, c);
 }
 // sigma(x) = (1 + tanh(x/2)) / 2 with the hardware tanh approximation (max rel.
 // error ~2^-11, below the bf16 rounding the results get)

@@ -2,6 +2,7 @@
 // TTT path uses, so the operand layouts (K-major / MN-major, bf16 / tf32),
 // ragged edges, batching and split-K can be checked against a library matmul.
 #include "../../include/ttt_diag.h"
+#include "epilogues.cuh"
 #include "tc_gemm.cuh"
 
 namespace ttt {
@@ -105,8 +106,35 @@ __global__ void stuck_wait_kernel(unsigned* status) {
   if (threadIdx.x == 0 && !mbar_wait(&bar, 0, &abort_flag)) set_status(status, kStatusTimeout);
 }
 
+// The activation functions of the epilogues, elementwise: kind 0 GELU and its derivative,
+// kind 1 SiLU and its derivative.
+__global__ void activation_kernel(int kind, int64_t n, const float* x, float* y, float* dy) {
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    const float v = x[i];
+    float f, g;
+    if (kind == 0) {
+      gelu_and_grad(v, f, g);
+    } else {
+      const float s = sigmoid_dev(v);
+      f = v * s;
+      g = s * fmaf(v, 1.0f - s, 1.0f);
+    }
+    y[i] = f;
+    dy[i] = g;
+  }
+}
+
 }  // namespace
 }  // namespace ttt
+
+extern "C" int ttt_selftest_activation(int kind, int64_t n, const float* x, float* y, float* dy, void* stream_ptr) {
+  if ((kind != 0 && kind != 1) || n < 0 || (n > 0 && (!x || !y || !dy))) return TTT_ERR_INVALID_ARG;
+  if (n == 0) return TTT_OK;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, 4096));
+  ttt::activation_kernel<<<grid, 256, 0, stream>>>(kind, n, x, y, dy);
+  return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
 
 extern "C" int ttt_selftest_timeout(void* status_word, void* stream_ptr) {
   if (!status_word) return TTT_ERR_INVALID_ARG;
