@@ -243,8 +243,9 @@ __global__ void __launch_bounds__(64 + 32 * ApplyShape<SWIGLU, D, EPIW>::EW, 1)
               a = z1[i] * sigmoid_dev(z1[i]) * z3[i];
               b = z1[i + 1] * sigmoid_dev(z1[i + 1]) * z3[i + 1];
             } else {
-              a = gelu_dev(z1[i]);
-              b = gelu_dev(z1[i + 1]);
+              const float2 gv = gelu2(make_float2(z1[i], z1[i + 1]));
+              a = gv.x;
+              b = gv.y;
             }
             packed[c * 16 + i / 2] = pack_bf16x2(a, b);
           }

@@ -96,6 +96,36 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
   return bits_f2(r);
 }
 
+// Two GELUs (and derivatives) at once: the same arithmetic as normal_cdf_pdf lane by lane
+// (fma.rn / mul.rn per lane give bit-identical results), with the multiplies and adds
+// issued as paired fp32 instructions; the reciprocal and exp2 stay per lane.
+__device__ __forceinline__ void normal_cdf_pdf2(float2 x, float2& cdf, float2& pdf) {
+  using namespace normal_as;
+  const float2 den = fma2(make_float2(kP, kP), make_float2(fabsf(x.x), fabsf(x.y)), make_float2(1.0f, 1.0f));
+  const float2 t = make_float2(rcp_approx(den.x), rcp_approx(den.y));
+  float2 y = fma2(make_float2(kA5, kA5), t, make_float2(kA4, kA4));
+  y = fma2(y, t, make_float2(kA3, kA3));
+  y = fma2(y, t, make_float2(kA2, kA2));
+  y = fma2(y, t, make_float2(kA1, kA1));
+  y = mul2(y, t);
+  const float2 a = mul2(mul2(x, x), make_float2(kNegHalfLog2e, kNegHalfLog2e));
+  const float2 e = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+  const float2 q = mul2(y, e);
+  cdf = make_float2(x.x >= 0.0f ? 1.0f - q.x : q.x, x.y >= 0.0f ? 1.0f - q.y : q.y);
+  pdf = mul2(e, make_float2(kInvSqrt2Pi, kInvSqrt2Pi));
+}
+__device__ __forceinline__ float2 gelu2(float2 x) {
+  float2 c, p;
+  normal_cdf_pdf2(x, c, p);
+  return mul2(x, c);
+}
+__device__ __forceinline__ void gelu_and_grad2(float2 x, float2& g, float2& gp) {
+  float2 c, p;
+  normal_cdf_pdf2(x, c, p);
+  g = mul2(x, c);
+  gp = fma2(x, p, c);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -251,12 +251,11 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
         for (int i = 0; i < 16; ++i) zv[i] = __uint_as_float(zr[i]);
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
-          float g0, g1, p0, p1;
-          gelu_and_grad(zv[i], g0, p0);
-          gelu_and_grad(zv[i + 1], g1, p1);
-          hv[i] = valid ? g0 : 0.f;
-          hv[i + 1] = valid ? g1 : 0.f;
-          gp[(cc + i) / 2] = pack_bf16x2(p0, p1);
+          float2 gv, pv;
+          gelu_and_grad2(make_float2(zv[i], zv[i + 1]), gv, pv);
+          hv[i] = valid ? gv.x : 0.f;
+          hv[i + 1] = valid ? gv.y : 0.f;
+          gp[(cc + i) / 2] = pack_bf16x2(pv.x, pv.y);
         }
         put_row16(hs + ((c0 + cc) / 64) * S::TILE, row, ((c0 + cc) % 64) / 8, hv);
       }

@@ -306,9 +306,23 @@ __global__ void keystats_kernel(int n, int d, const bf16* K, int64_t k_zs, int t
   __threadfence();
   for (int ch = tid; ch < d; ch += blockDim.x) {
     double sum = 0.0, sq = 0.0;
-    for (int b = 0; b < nb; ++b) {
-      sum += __ldcg(part + ((int64_t(z) * nb + b) * d + ch) * 2);
-      sq += __ldcg(part + ((int64_t(z) * nb + b) * d + ch) * 2 + 1);
+    const float2* pz = reinterpret_cast<const float2*>(part) + int64_t(z) * nb * d + ch;
+    int b = 0;
+    // eight blocks' sums in flight at a time, added in block order
+    for (; b + 8 <= nb; b += 8) {
+      float2 v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = __ldcg(pz + int64_t(b + i) * d);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        sum += v[i].x;
+        sq += v[i].y;
+      }
+    }
+    for (; b < nb; ++b) {
+      const float2 v = __ldcg(pz + int64_t(b) * d);
+      sum += v.x;
+      sq += v.y;
     }
     const double mean = sum / n;
     const double var = fmax(sq / n - mean * mean, 0.0);
