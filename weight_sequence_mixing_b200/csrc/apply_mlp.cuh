@@ -101,38 +101,62 @@ __global__ void __launch_bounds__(64 + 32 * ApplyShape<SWIGLU, D, EPIW>::EW, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // The CTA's hidden blocks in order, across its tiles: block nb is block nb % hblocks of
+  // the CTA's tile nb / hblocks.  The MMA issuer runs one block ahead: Z of block nb + 1 is
+  // issued as soon as the epilogue has read Z of block nb out of TMEM, before the O
+  // MMAs of block nb (which wait for its gating), so the next block's Z is ready when
+  // the epilogue gets to it; the next tile's Q is loaded as soon as the current tile's
+  // last Z MMA has read Q.  The producer fills the operand ring in the same order:
+  // [Q(0)] Z(0), then per block nb: [Q(next tile)] Z(nb + 1), O(nb).
+  const int ntiles_cta = total > static_cast<int>(blockIdx.x) ? (total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const int nblocks = ntiles_cta * g.hblocks;
+  auto tile_of = [&](int jt) { return static_cast<int>(blockIdx.x) + jt * static_cast<int>(gridDim.x); };
+
   if (warp == 0) {
-    if (elect_one()) {
+    if (elect_one() && nblocks > 0) {
       tma_prefetch_desc(&tQ);
       tma_prefetch_desc(&tFirst);
       tma_prefetch_desc(&tW2);
-      int it = 0, j = 0;
+      int it = 0;
       bool stop = false;
-      for (int t = blockIdx.x; t < total && !stop; t += gridDim.x, ++j) {
-        const int mt = t % g.m_tiles, z = t / g.m_tiles;
-        // the previous tile's MMAs have finished reading Q
-        if (j > 0 && !mbar_wait(qempty, (j - 1) & 1, abort_flag)) break;
+      // one ring slot per k-block: the first-layer rows of a block (K = d) or W2's columns (K = hidden)
+      auto ring_load = [&](bool first_layer, int i, int hb, int z) {
+        const int s = it % S::STAGES;
+        const uint32_t ph = (it / S::STAGES) & 1;
+        if (it >= S::STAGES && !mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
+          stop = true;
+          return;
+        }
+        uint8_t* st = ring + s * S::STAGE;
+        if (first_layer) {
+          mbar_arrive_expect_tx(&full[s], S::ZN * 128);
+          tma_load_3d(st, &tFirst, &full[s], i * 64, hb * S::ZN, z);
+        } else {
+          mbar_arrive_expect_tx(&full[s], D * 128);
+          tma_load_3d(st, &tW2, &full[s], hb * 128 + i * 64, 0, z);
+        }
+        ++it;
+      };
+      // Q of the CTA's tile jt (after the previous tile's Z MMAs have read Q)
+      auto q_load = [&](int jt) {
+        if (jt > 0 && !mbar_wait(qempty, (jt - 1) & 1, abort_flag)) {
+          stop = true;
+          return;
+        }
+        const int t = tile_of(jt), mt = t % g.m_tiles, z = t / g.m_tiles;
         mbar_arrive_expect_tx(qfull, S::Q_BYTES);
         for (int kb = 0; kb < S::KB; ++kb) tma_load_3d(qs + kb * 128 * 128, &tQ, qfull, kb * 64, g.row0 + mt * 128, z);
-        for (int hb = 0; hb < g.hblocks && !stop; ++hb) {
-          // first-layer rows of the block (K = d), then W2's columns of the block (K = hidden)
-          for (int i = 0; i < S::KB + 2; ++i, ++it) {
-            const int s = it % S::STAGES;
-            const uint32_t ph = (it / S::STAGES) & 1;
-            if (it >= S::STAGES && !mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
-              stop = true;
-              break;
-            }
-            uint8_t* st = ring + s * S::STAGE;
-            if (i < S::KB) {
-              mbar_arrive_expect_tx(&full[s], S::ZN * 128);
-              tma_load_3d(st, &tFirst, &full[s], i * 64, hb * S::ZN, z);
-            } else {
-              mbar_arrive_expect_tx(&full[s], D * 128);
-              tma_load_3d(st, &tW2, &full[s], hb * 128 + (i - S::KB) * 64, 0, z);
-            }
-          }
-        }
+      };
+      auto z_loads = [&](int nb) {
+        const int jt = nb / g.hblocks, hb = nb % g.hblocks, z = tile_of(jt) / g.m_tiles;
+        if (hb == 0) q_load(jt);
+        for (int i = 0; i < S::KB && !stop; ++i) ring_load(true, i, hb, z);
+      };
+      z_loads(0);
+      for (int nb = 0; nb < nblocks && !stop; ++nb) {
+        if (nb + 1 < nblocks) z_loads(nb + 1);
+        const int hb = nb % g.hblocks, z = tile_of(nb / g.hblocks) / g.m_tiles;
+        for (int i = 0; i < 2 && !stop; ++i) ring_load(false, i, hb, z);
       }
       if (*abort_flag) {
         // copies already in flight land within microseconds; give them a millisecond
@@ -142,69 +166,58 @@ __global__ void __launch_bounds__(64 + 32 * ApplyShape<SWIGLU, D, EPIW>::EW, 1)
       }
     }
   } else if (warp == 1) {
-    if (elect_one()) {
+    if (elect_one() && nblocks > 0) {
       constexpr uint32_t idZ = make_idesc(128, S::ZN, 1, false, false);
       constexpr uint32_t idO = make_idesc(128, D, 1, false, false);
       const uint32_t qbase = smem_u32(qs), hbase = smem_u32(hs), rbase = smem_u32(ring);
-      int it = 0, j = 0, nz = 0;  // ring position, tiles, hidden blocks issued
-      bool stop = false;
-      for (int t = blockIdx.x; t < total && !stop; t += gridDim.x, ++j) {
-        if (!mbar_wait(qfull, j & 1, abort_flag)) break;
+      int it = 0;
+      bool ok = true;
+      // Z = Q [W1_blk; W3_blk]^T of block nb (Z has been read out of TMEM by then)
+      auto issue_z = [&](int nb) {
+        const int jt = nb / g.hblocks, hb = nb % g.hblocks;
+        if (hb == 0 && !(ok = mbar_wait(qfull, jt & 1, abort_flag))) return;
         tc_fence_after();
-        for (int hb = 0; hb < g.hblocks && !stop; ++hb, ++nz) {
-          // Z of the previous block has been read out of TMEM
-          if (nz > 0 && !mbar_wait(zempty, (nz - 1) & 1, abort_flag)) {
-            stop = true;
-            break;
-          }
+        for (int kb = 0; kb < S::KB; ++kb, ++it) {
+          const int s = it % S::STAGES;
+          if (!(ok = mbar_wait(&full[s], (it / S::STAGES) & 1, abort_flag))) return;
           tc_fence_after();
-          for (int kb = 0; kb < S::KB; ++kb, ++it) {
-            const int s = it % S::STAGES;
-            if (!mbar_wait(&full[s], (it / S::STAGES) & 1, abort_flag)) {
-              stop = true;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t a = qbase + kb * 128 * 128, b = rbase + s * S::STAGE;
+          const uint32_t a = qbase + kb * 128 * 128, b = rbase + s * S::STAGE;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16(tmem_base + S::Z_COL, make_sdesc_sw128(a + kk * 32, 16, 1024),
-                      make_sdesc_sw128(b + kk * 32, 16, 1024), idZ, (kb > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(&empty[s]);
-          }
-          if (stop) break;
-          mma_commit(zfull);
-          // H of this block written by the epilogue (and, for the tile's first block,
-          // O of the previous tile read out of TMEM)
-          if (!mbar_wait(hfull, nz & 1, abort_flag)) {
-            stop = true;
-            break;
-          }
-          if (hb == 0 && j > 0 && !mbar_wait(oempty, (j - 1) & 1, abort_flag)) {
-            stop = true;
-            break;
-          }
-          tc_fence_after();
-          for (int kh = 0; kh < 2; ++kh, ++it) {
-            const int s = it % S::STAGES;
-            if (!mbar_wait(&full[s], (it / S::STAGES) & 1, abort_flag)) {
-              stop = true;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t a = hbase + kh * 128 * 128, b = rbase + s * S::STAGE;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16(tmem_base, make_sdesc_sw128(a + kk * 32, 16, 1024), make_sdesc_sw128(b + kk * 32, 16, 1024),
-                      idO, (hb > 0 || kh > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(&empty[s]);
-          }
-          if (stop) break;
-          mma_commit(hempty);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16(tmem_base + S::Z_COL, make_sdesc_sw128(a + kk * 32, 16, 1024),
+                    make_sdesc_sw128(b + kk * 32, 16, 1024), idZ, (kb > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&empty[s]);
         }
-        if (stop) break;
-        mma_commit(ofull);
-        mma_commit(qempty);
+        mma_commit(zfull);
+        if (hb == g.hblocks - 1) mma_commit(qempty);  // the tile's last read of Q
+      };
+      issue_z(0);
+      for (int nb = 0; nb < nblocks && ok; ++nb) {
+        const int jt = nb / g.hblocks, hb = nb % g.hblocks;
+        if (nb + 1 < nblocks) {
+          if (!(ok = mbar_wait(zempty, nb & 1, abort_flag))) break;
+          issue_z(nb + 1);
+          if (!ok) break;
+        }
+        // H of block nb written by the epilogue (and, for a tile's first block, O of the
+        // previous tile read out of TMEM): O += H W2[:, blk]^T
+        if (!(ok = mbar_wait(hfull, nb & 1, abort_flag))) break;
+        if (hb == 0 && jt > 0 && !(ok = mbar_wait(oempty, (jt - 1) & 1, abort_flag))) break;
+        tc_fence_after();
+        for (int kh = 0; kh < 2 && ok; ++kh, ++it) {
+          const int s = it % S::STAGES;
+          if (!(ok = mbar_wait(&full[s], (it / S::STAGES) & 1, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t a = hbase + kh * 128 * 128, b = rbase + s * S::STAGE;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16(tmem_base, make_sdesc_sw128(a + kk * 32, 16, 1024), make_sdesc_sw128(b + kk * 32, 16, 1024),
+                    idO, (hb > 0 || kh > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(hempty);
+        if (hb == g.hblocks - 1) mma_commit(ofull);
       }
       if (*abort_flag) {
         volatile int never = 0;
