@@ -21,9 +21,13 @@
 // a tile's TMEM-chained steps leave no room in TMEM for a second tile.  Rows past the
 // chunk are zero in H, dY and dZ, so they add nothing.
 //
-// Warps: 0 TMA producer (keys and values of two tiles in flight), 1 MMA issuer, 2..17
-// epilogue (four per TMEM lane quarter; warp slot s owns hidden columns [s h/4, (s+1) h/4)
-// and 16 of the 64 output channels).  Every wait is bounded.
+// Key instance-norm (kstats given): the keys arrive raw and warp 0 normalises each tile in
+// shared memory, x_hat = (x - mean) rstd per channel, before the Z MMAs read it (and G1
+// then reduces against the normalised keys), so no normalised copy of K goes through HBM.
+//
+// Warps: 0 TMA producer (keys and values of two tiles in flight; all its lanes normalise
+// the keys), 1 MMA issuer, 2..17 epilogue (four per TMEM lane quarter; warp slot s owns
+// hidden columns [s h/4, (s+1) h/4) and 16 of the 64 output channels).  Every wait is bounded.
 #pragma once
 #include "epilogues.cuh"
 
@@ -39,6 +43,7 @@ struct MseGeom {
   int64_t eta_zs;
   float eta_scalar, coef;  // coef = 2 / (n d)
   float* part;             // [splits][z][2h][64] fp32 gradient partials
+  const float* kstats;     // [z][64][2] mean, 1/std of the chunk's keys per channel, or null
 };
 
 template <int HID>
@@ -49,7 +54,7 @@ struct MseShape {
   static constexpr int W2_BYTES = (HID / 64) * 64 * 128;  // [64][HID] as HID/64 blocks of 64 columns
   static constexpr int H_BYTES = (HID / 64) * TILE;       // [128][HID] as HID/64 k-blocks (H, then dZ)
   static constexpr int EW = 16;
-  static constexpr int SMEM = 1024 + 2 * 2 * TILE + W1_BYTES + W2_BYTES + H_BYTES + TILE + 256;
+  static constexpr int SMEM = 1024 + 2 * 2 * TILE + W1_BYTES + W2_BYTES + H_BYTES + TILE + 2 * 64 * 4 + 256;
   static constexpr int COLS = HID / 4;          // hidden columns per epilogue thread
   static constexpr int NACC = 2 * (HID / 128);  // 128 x 64 gradient accumulators
   static constexpr uint32_t GCOL = 256;         // first TMEM column of the accumulators
@@ -84,7 +89,8 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
   uint8_t* w2s = w1s + S::W1_BYTES;
   uint8_t* hs = w2s + S::W2_BYTES;
   uint8_t* dys = hs + S::H_BYTES;
-  uint64_t* xfull = reinterpret_cast<uint64_t*>(dys + S::TILE);  // [2]
+  float* nsc = reinterpret_cast<float*>(dys + S::TILE);  // [64] rstd, [64] -mean rstd
+  uint64_t* xfull = reinterpret_cast<uint64_t*>(nsc + 2 * 64);  // [2]
   uint64_t* xempty = xfull + 2;  // [2]: G1 (commit) and the dY epilogue are done with the slot
   uint64_t* wfull = xempty + 2;  // the head's weights landed
   uint64_t* zfull = wfull + 1;   // Z in TMEM (every earlier MMA, the previous tile's G1 too, done)
@@ -94,7 +100,8 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
   uint64_t* dhfull = dyfull + 1;  // dH in TMEM, the tile's G2^T done (H no longer read)
   uint64_t* dzfull = dhfull + 1;  // dZ in shared memory, dH read
   uint64_t* gdone = dzfull + 1;   // the last tile's G1 done: the accumulators are final
-  uint64_t* drain = gdone + 1;
+  uint64_t* xnorm = gdone + 1;    // [2]: the slot's keys normalised (key instance-norm only)
+  uint64_t* drain = xnorm + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -108,6 +115,7 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&xfull[s], 1);
       mbar_init(&xempty[s], 1 + S::EW);
+      mbar_init(&xnorm[s], 1);
     }
     mbar_init(wfull, 1);
     mbar_init(zfull, 1);
@@ -131,21 +139,56 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    if (elect_one() && ntiles > 0) {
-      tma_prefetch_desc(&tX);
-      tma_prefetch_desc(&tV);
-      tma_prefetch_desc(&tW1);
-      tma_prefetch_desc(&tW2);
-      mbar_arrive_expect_tx(wfull, S::W1_BYTES + S::W2_BYTES);
-      tma_load_3d(w1s, &tW1, wfull, 0, 0, z);
-      for (int b = 0; b < HID / 64; ++b) tma_load_3d(w2s + b * 64 * 128, &tW2, wfull, 64 * b, 0, z);
+    const bool norm = g.kstats != nullptr;
+    if (norm) {
+      for (int c = lane; c < 64; c += 32) {
+        const float mean = g.kstats[(int64_t(z) * 64 + c) * 2], rstd = g.kstats[(int64_t(z) * 64 + c) * 2 + 1];
+        nsc[c] = rstd;
+        nsc[64 + c] = -mean * rstd;
+      }
+      __syncwarp();
+    }
+    if (ntiles > 0) {
+      if (lane == 0) {
+        tma_prefetch_desc(&tX);
+        tma_prefetch_desc(&tV);
+        tma_prefetch_desc(&tW1);
+        tma_prefetch_desc(&tW2);
+        mbar_arrive_expect_tx(wfull, S::W1_BYTES + S::W2_BYTES);
+        tma_load_3d(w1s, &tW1, wfull, 0, 0, z);
+        for (int b = 0; b < HID / 64; ++b) tma_load_3d(w2s + b * 64 * 128, &tW2, wfull, 64 * b, 0, z);
+      }
       for (int j = 0; j < ntiles; ++j) {
         const int s = j & 1, mt = mt0 + j;
-        if (j >= 2 && !mbar_wait(&xempty[s], ((j - 2) >> 1) & 1, abort_flag)) break;
+        if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&xempty[s], ((j - 2) >> 1) & 1, abort_flag))) break;
         uint8_t* slot = xv + s * 2 * S::TILE;
-        mbar_arrive_expect_tx(&xfull[s], 2 * S::TILE);
-        tma_load_3d(slot, &tX, &xfull[s], 0, g.x_off + mt * 128, z);
-        tma_load_3d(slot + S::TILE, &tV, &xfull[s], 0, g.v_off + mt * 128, z);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&xfull[s], 2 * S::TILE);
+          tma_load_3d(slot, &tX, &xfull[s], 0, g.x_off + mt * 128, z);
+          tma_load_3d(slot + S::TILE, &tV, &xfull[s], 0, g.v_off + mt * 128, z);
+        }
+        if (!norm) continue;
+        // normalise the 128 x 64 key tile in place: 16-byte chunk p of row r holds channels
+        // 8 (p ^ (r & 7)) .. + 7 (128-byte swizzle); lane l takes chunk l % 8 of rows l / 8 + 4 i
+        if (!__all_sync(0xffffffffu, mbar_wait(&xfull[s], (j >> 1) & 1, abort_flag))) break;
+#pragma unroll 4
+        for (int i = 0; i < 32; ++i) {
+          const int r = lane / 8 + 4 * i, p = lane % 8, c0 = 8 * (p ^ (r & 7));
+          uint4* ch = reinterpret_cast<uint4*>(slot + r * 128 + 16 * p);
+          const uint4 u = *ch;
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+            const int c = c0 + 2 * e;
+            o[e] = pack_bf16x2(fmaf(f.x, nsc[c], nsc[64 + c]), fmaf(f.y, nsc[c + 1], nsc[64 + c + 1]));
+          }
+          *ch = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xnorm[s]);
       }
       if (*abort_flag) {
         const unsigned long long t0 = global_ns();
@@ -181,7 +224,7 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
           tc_fence_after();
           issue_g1(j - 1);
         }
-        if (!(ok = mbar_wait(&xfull[s], (j >> 1) & 1, abort_flag))) break;
+        if (!(ok = mbar_wait(g.kstats ? &xnorm[s] : &xfull[s], (j >> 1) & 1, abort_flag))) break;
         tc_fence_after();
         const uint32_t xa = smem_u32(xv + s * 2 * S::TILE);
 #pragma unroll

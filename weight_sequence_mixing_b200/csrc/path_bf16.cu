@@ -779,20 +779,25 @@ int update_chunk(Ctx& c, int t0, int n) {
   const TM* tXmn = &c.tKmn;
   int xoff = t0;
   TM tKn, tKnmn;
+  const float* kstats = nullptr;  // per-channel key statistics the fused MSE kernel applies itself
   if (cfg.flags & TTT_FLAG_KEY_INSTNORM) {
-    bf16* Kn = c.v.at<bf16>(p, xKn);
     float* kst = c.v.at<float>(p, xKstat);
     const int nb = (n + 127) / 128;  // token blocks holding keys of the chunk
-    const dim3 gk(Cp / 128, Z);
     float* kfin = kst + size_t(Z) * (Cp / 128) * d * 2;                   // [Z][d][2] mean, rstd
     unsigned* kdone = reinterpret_cast<unsigned*>(kfin + size_t(Z) * d * 2);  // [Z] blocks finished
     {
       StageScope _sc(kStageKeyNorm, st);
       keystats_kernel<<<dim3(nb, Z), 256, 0, c.st>>>(n, d, K, int64_t(D.N) * d, t0, cfg.in_eps, kst, kfin, kdone);
     }
+    TRY_CUDA(cudaGetLastError());
+    kstats = kfin;
+  }
+  if ((cfg.flags & TTT_FLAG_KEY_INSTNORM) && !mse_token_path(cfg)) {
+    bf16* Kn = c.v.at<bf16>(p, xKn);
+    const dim3 gk(Cp / 128, Z);
     {
       StageScope _sc(kStageKeyNorm, st);
-      keynorm_kernel<<<gk, 256, 2 * d * sizeof(float), c.st>>>(n, d, K, int64_t(D.N) * d, t0, kfin, Kn,
+      keynorm_kernel<<<gk, 256, 2 * d * sizeof(float), c.st>>>(n, d, K, int64_t(D.N) * d, t0, kstats, Kn,
                                                                int64_t(Cp) * d);
     }
     TRY_CUDA(cudaGetLastError());
@@ -845,6 +850,7 @@ int update_chunk(Ctx& c, int t0, int n) {
     mg.eta_scalar = cfg.eta_scalar;
     mg.coef = 2.0f / (float(n) * float(d));
     mg.part = c.v.at<float>(p, xPart);
+    mg.kstats = kstats;  // key instance-norm applied to the raw key tiles in the kernel
     {
       StageScope sc(kStageTokenPhase, c.st);
       const cudaError_t e = h == 256 ? launch_mse_token<256>(tX->m, c.tV.m, tw1.m, tw2.m, mg, status, c.st)
@@ -1079,7 +1085,7 @@ int plan_layout_bf16(Plan* p) {
       Z * D.R1 * d * 2,
       act ? Z * h * d * 2 : 0,
       act ? Z * d * h * 2 : 0,
-      (c.flags & TTT_FLAG_KEY_INSTNORM) ? Z * Cp * d * 2 : 0,
+      ((c.flags & TTT_FLAG_KEY_INSTNORM) && !mse_token_path(c)) ? Z * Cp * d * 2 : 0,
       (act && spill) ? Z * Cp * h * 2 : 0,
       ((act && spill) || glu) ? Z * Cp * 2 * h * 2 : 0,  // dZ13 / dZ (GLU: h = d)
       (mlp_mse && spill) ? Z * Cp * h * 2 : 0,
