@@ -17,9 +17,13 @@
 // layout [split][z][2h][d] (rows [0, h) G2^T, rows [h, 2h) G1), for the split reduction.
 //
 // A CTA owns one head z and one contiguous range of its token tiles (split sp of the
-// chunk's tiles), so the head's weights are loaded once.  Tiles run one after another:
-// a tile's TMEM-chained steps leave no room in TMEM for a second tile.  Rows past the
-// chunk are zero in H, dY and dZ, so they add nothing.
+// chunk's tiles), so the head's weights are loaded once.  Tiles run one after another
+// (a tile's TMEM-chained steps leave no room in TMEM for a second tile), but each step is
+// staggered by 64-column k-blocks of the hidden layer: Z is issued as h/64 MMAs of 64
+// columns, the gating starts on the first while the others run, V^ accumulates k-block by
+// k-block as the gating finishes them; dH likewise feeds dZ, and G1 of a 128-row block of h
+// and the next tile's Z k-blocks go as soon as their dZ k-blocks are written.  Rows past
+// the chunk are zero in H, dY and dZ, so they add nothing.
 //
 // Key instance-norm (kstats given): the keys arrive raw and warp 0 normalises each tile in
 // shared memory, x_hat = (x - mean) rstd per channel, before the Z MMAs read it (and G1
@@ -27,7 +31,8 @@
 //
 // Warps: 0 TMA producer (keys and values of two tiles in flight; all its lanes normalise
 // the keys), 1 MMA issuer, 2..17 epilogue (four per TMEM lane quarter; warp slot s owns
-// hidden columns [s h/4, (s+1) h/4) and 16 of the 64 output channels).  Every wait is bounded.
+// hidden columns [64 k + 16 s, 64 k + 16 s + 16) of every k-block k and 16 of the 64 output
+// channels).  Every wait is bounded.
 #pragma once
 #include "epilogues.cuh"
 
@@ -56,6 +61,7 @@ struct MseShape {
   static constexpr int EW = 16;
   static constexpr int SMEM = 1024 + 2 * 2 * TILE + W1_BYTES + W2_BYTES + H_BYTES + TILE + 2 * 64 * 4 + 256;
   static constexpr int COLS = HID / 4;          // hidden columns per epilogue thread
+  static constexpr int KB = HID / 64;           // 64-column k-blocks of the hidden layer
   static constexpr int NACC = 2 * (HID / 128);  // 128 x 64 gradient accumulators
   static constexpr uint32_t GCOL = 256;         // first TMEM column of the accumulators
   static_assert(HID == 128 || HID == 256, "h");
@@ -93,13 +99,13 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
   uint64_t* xfull = reinterpret_cast<uint64_t*>(nsc + 2 * 64);  // [2]
   uint64_t* xempty = xfull + 2;  // [2]: G1 (commit) and the dY epilogue are done with the slot
   uint64_t* wfull = xempty + 2;  // the head's weights landed
-  uint64_t* zfull = wfull + 1;   // Z in TMEM (every earlier MMA, the previous tile's G1 too, done)
-  uint64_t* hfull = zfull + 1;   // H in shared memory, Z read
-  uint64_t* vfull = hfull + 1;   // V^ in TMEM
+  uint64_t* zk = wfull + 1;      // [KB] Z k-block in TMEM (the previous tile's G1 of its rows done)
+  uint64_t* hk = zk + S::KB;     // [KB] H k-block in shared memory, its Z read
+  uint64_t* vfull = hk + S::KB;  // V^ in TMEM
   uint64_t* dyfull = vfull + 1;  // dY in shared memory, V^ read
-  uint64_t* dhfull = dyfull + 1;  // dH in TMEM, the tile's G2^T done (H no longer read)
-  uint64_t* dzfull = dhfull + 1;  // dZ in shared memory, dH read
-  uint64_t* gdone = dzfull + 1;   // the last tile's G1 done: the accumulators are final
+  uint64_t* dhk = dyfull + 1;    // [KB] dH k-block in TMEM, the tile's G2^T done (H no longer read)
+  uint64_t* dzk = dhk + S::KB;   // [KB] dZ k-block in shared memory, its dH read
+  uint64_t* gdone = dzk + S::KB;  // the last tile's G1 done: the accumulators are final
   uint64_t* xnorm = gdone + 1;    // [2]: the slot's keys normalised (key instance-norm only)
   uint64_t* drain = xnorm + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -118,12 +124,14 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
       mbar_init(&xnorm[s], 1);
     }
     mbar_init(wfull, 1);
-    mbar_init(zfull, 1);
-    mbar_init(hfull, S::EW);
+    for (int k = 0; k < S::KB; ++k) {
+      mbar_init(&zk[k], 1);
+      mbar_init(&hk[k], S::EW);
+      mbar_init(&dhk[k], 1);
+      mbar_init(&dzk[k], S::EW);
+    }
     mbar_init(vfull, 1);
     mbar_init(dyfull, S::EW);
-    mbar_init(dhfull, 1);
-    mbar_init(dzfull, S::EW);
     mbar_init(gdone, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -198,50 +206,53 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
     }
   } else if (warp == 1) {
     if (elect_one() && ntiles > 0) {
-      constexpr uint32_t idZ = make_idesc(128, HID, 1, false, false);
+      constexpr uint32_t idZ = make_idesc(128, 64, 1, false, false);  // one 64-column k-block of Z
       constexpr uint32_t idV = make_idesc(128, 64, 1, false, false);
-      constexpr uint32_t idH = make_idesc(128, HID, 1, false, true);  // B = W2 [d][h], MN-major
+      constexpr uint32_t idH = make_idesc(128, 64, 1, false, true);   // B = a W2 [d][h] block, MN-major
       constexpr uint32_t idG = make_idesc(128, 64, 1, true, true);    // A = H^T / dZ^T, B = dY / X
       const uint32_t w1a = smem_u32(w1s), w2a = smem_u32(w2s), ha = smem_u32(hs), dya = smem_u32(dys);
-      // G1 += dZ^T X of tile jj (keys in slot jj & 1), one 128-row block of h at a time; the
-      // operands are read MN-major: 64-column runs of h 16 KB apart, 16-token steps of 2 KB
-      auto issue_g1 = [&](int jj) {
+      // Z k-block kb of tile jj: X W1[64 kb .. 64 kb + 64)^T into TMEM columns [64 kb, 64 kb + 64)
+      auto issue_z = [&](int jj, int kb) {
         const uint32_t xa = smem_u32(xv + (jj & 1) * 2 * S::TILE);
-        for (int blk = 0; blk < HID / 128; ++blk)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_f16(tmem_base + S::GCOL + 64 * (HID / 128 + blk),
-                    make_sdesc_sw128(ha + blk * 2 * S::TILE + kk * 2048, S::TILE, 1024),
-                    make_sdesc_sw128(xa + kk * 2048, S::TILE, 1024), idG, (jj > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&xempty[jj & 1]);
-      };
-      bool ok = mbar_wait(wfull, 0, abort_flag);
-      for (int j = 0; j < ntiles && ok; ++j) {
-        const int s = j & 1;
-        if (j > 0) {
-          // dZ of the previous tile in shared memory and its dH read out of TMEM
-          if (!(ok = mbar_wait(dzfull, (j - 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          issue_g1(j - 1);
-        }
-        if (!(ok = mbar_wait(g.kstats ? &xnorm[s] : &xfull[s], (j >> 1) & 1, abort_flag))) break;
-        tc_fence_after();
-        const uint32_t xa = smem_u32(xv + s * 2 * S::TILE);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_f16(tmem_base, make_sdesc_sw128(xa + kk * 32, 16, 1024), make_sdesc_sw128(w1a + kk * 32, 16, 1024), idZ,
-                  kk > 0 ? 1u : 0u);
-        mma_commit(zfull);
-        // V^ = H W2^T once H is in shared memory (Z has been read)
-        if (!(ok = mbar_wait(hfull, j & 1, abort_flag))) break;
+          mma_f16(tmem_base + 64 * kb, make_sdesc_sw128(xa + kk * 32, 16, 1024),
+                  make_sdesc_sw128(w1a + kb * 64 * 128 + kk * 32, 16, 1024), idZ, kk > 0 ? 1u : 0u);
+        mma_commit(&zk[kb]);
+      };
+      // G1 rows [128 blk, 128 blk + 128) += dZ^T X of tile jj (keys in slot jj & 1); the
+      // operands are read MN-major: 64-column runs of h 16 KB apart, 16-token steps of 2 KB
+      auto issue_g1 = [&](int jj, int blk) {
+        const uint32_t xa = smem_u32(xv + (jj & 1) * 2 * S::TILE);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_f16(tmem_base + S::GCOL + 64 * (HID / 128 + blk),
+                  make_sdesc_sw128(ha + blk * 2 * S::TILE + kk * 2048, S::TILE, 1024),
+                  make_sdesc_sw128(xa + kk * 2048, S::TILE, 1024), idG, (jj > 0 || kk > 0) ? 1u : 0u);
+      };
+      auto keys_ready = [&](int jj) {
+        return mbar_wait(g.kstats ? &xnorm[jj & 1] : &xfull[jj & 1], (jj >> 1) & 1, abort_flag);
+      };
+      bool ok = mbar_wait(wfull, 0, abort_flag) && keys_ready(0);
+      if (ok) {
         tc_fence_after();
-        for (int kb = 0; kb < HID / 64; ++kb)
+        for (int kb = 0; kb < S::KB; ++kb) issue_z(0, kb);
+      }
+      for (int j = 0; j < ntiles && ok; ++j) {
+        const int s = j & 1;
+        // V^ = H W2^T, one k-block of H at a time as the gating writes them (V^ takes TMEM
+        // columns [0, 64), Z's first k-block, which has been read by then)
+        for (int kb = 0; kb < S::KB && ok; ++kb) {
+          if (!(ok = mbar_wait(&hk[kb], j & 1, abort_flag))) break;
+          tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_f16(tmem_base, make_sdesc_sw128(ha + kb * S::TILE + kk * 32, 16, 1024),
                     make_sdesc_sw128(w2a + kb * 64 * 128 + kk * 32, 16, 1024), idV, (kb > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (!ok) break;
         mma_commit(vfull);
-        // dY in shared memory (V^ has been read): G2^T += H^T dY, then dH = dY W2
+        // dY in shared memory (V^ has been read): G2^T += H^T dY, then dH = dY W2 by k-blocks
         if (!(ok = mbar_wait(dyfull, j & 1, abort_flag))) break;
         tc_fence_after();
         for (int blk = 0; blk < HID / 128; ++blk)
@@ -249,17 +260,33 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
           for (int kk = 0; kk < 8; ++kk)
             mma_f16(tmem_base + S::GCOL + 64 * blk, make_sdesc_sw128(ha + blk * 2 * S::TILE + kk * 2048, S::TILE, 1024),
                     make_sdesc_sw128(dya + kk * 2048, S::TILE, 1024), idG, (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kb = 0; kb < S::KB; ++kb) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f16(tmem_base, make_sdesc_sw128(dya + kk * 32, 16, 1024),
-                  make_sdesc_sw128(w2a + kk * 16 * 128, 64 * 128, 1024), idH, kk > 0 ? 1u : 0u);
-        mma_commit(dhfull);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16(tmem_base + 64 * kb, make_sdesc_sw128(dya + kk * 32, 16, 1024),
+                    make_sdesc_sw128(w2a + kb * 64 * 128 + kk * 16 * 128, 64 * 128, 1024), idH, kk > 0 ? 1u : 0u);
+          mma_commit(&dhk[kb]);
+        }
+        // per 128-row block of h, once its two dZ k-blocks are written (and their dH read):
+        // G1 of this tile, then the next tile's Z k-blocks in the freed TMEM columns (their
+        // completion tells the gating that G1 has finished reading those k-blocks of dZ)
+        const bool next = j + 1 < ntiles;
+        for (int blk = 0; blk < HID / 128 && ok; ++blk) {
+          if (!(ok = mbar_wait(&dzk[2 * blk], j & 1, abort_flag) && mbar_wait(&dzk[2 * blk + 1], j & 1, abort_flag)))
+            break;
+          tc_fence_after();
+          issue_g1(j, blk);
+          if (next) {
+            if (blk == 0 && !(ok = keys_ready(j + 1))) break;
+            tc_fence_after();
+            issue_z(j + 1, 2 * blk);
+            issue_z(j + 1, 2 * blk + 1);
+          }
+        }
+        if (!ok) break;
+        mma_commit(&xempty[s]);
       }
-      if (ok && mbar_wait(dzfull, (ntiles - 1) & 1, abort_flag)) {
-        tc_fence_after();
-        issue_g1(ntiles - 1);
-        mma_commit(gdone);
-      }
+      if (ok) mma_commit(gdone);
       if (*abort_flag) {
         volatile int never = 0;
         mma_commit(drain);
@@ -271,41 +298,38 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
     const int slot = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    const int c0 = slot * S::COLS;  // hidden columns [c0, c0 + COLS)
     bool ok = true;
     for (int j = 0; j < ntiles && ok; ++j) {
       const int s = j & 1;
       const int m = (mt0 + j) * 128 + row;
       const bool valid = m < g.rows_valid;
-      // ---- E1: H = GELU(Z) into shared memory (the previous tile's G1, which read dZ
-      // there, completed before Z did), G' kept packed in registers
-      ok = __all_sync(0xffffffffu, mbar_wait(zfull, j & 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
+      // ---- E1, k-block by k-block: H = GELU(Z) into shared memory (the previous tile's G1,
+      // which read dZ there, completed before this k-block of Z did), G' kept packed in registers
       uint32_t gp[S::COLS / 2];
 #pragma unroll
-      for (int cc = 0; cc < S::COLS; cc += 16) {
+      for (int kb = 0; kb < S::KB; ++kb) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&zk[kb], j & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
         uint32_t zr[16];
         float hv[16];
-        tmem_ld16_async(tq + c0 + cc, zr);
+        tmem_ld16_async(tq + 64 * kb + 16 * slot, zr);
         tmem_wait_regs(zr);
-        float zv[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) zv[i] = __uint_as_float(zr[i]);
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
           float2 gv, pv;
-          gelu_and_grad2(make_float2(zv[i], zv[i + 1]), gv, pv);
+          gelu_and_grad2(make_float2(__uint_as_float(zr[i]), __uint_as_float(zr[i + 1])), gv, pv);
           hv[i] = valid ? gv.x : 0.f;
           hv[i + 1] = valid ? gv.y : 0.f;
-          gp[(cc + i) / 2] = pack_bf16x2(pv.x, pv.y);
+          gp[kb * 8 + i / 2] = pack_bf16x2(pv.x, pv.y);
         }
-        put_row16(hs + ((c0 + cc) / 64) * S::TILE, row, ((c0 + cc) % 64) / 8, hv);
+        put_row16(hs + kb * S::TILE, row, 2 * slot, hv);
+        tc_fence_before();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&hk[kb]);
       }
-      tc_fence_before();
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(hfull);
+      if (!ok) break;
       // ---- E2: dY = coef eta (V^ - V) on this warp's 16 output channels
       ok = __all_sync(0xffffffffu, mbar_wait(vfull, j & 1, abort_flag));
       if (!ok) break;
@@ -341,30 +365,29 @@ __global__ void __launch_bounds__(64 + 32 * MseShape<HID>::EW, 1)
         mbar_arrive(dyfull);
         mbar_arrive(&xempty[s]);
       }
-      // ---- E3: dZ = dH * G' into shared memory over H (G2^T, its last reader, is done)
-      ok = __all_sync(0xffffffffu, mbar_wait(dhfull, j & 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
+      // ---- E3, k-block by k-block: dZ = dH * G' into shared memory over H (G2^T, its last
+      // reader, is done)
 #pragma unroll
-      for (int cc = 0; cc < S::COLS; cc += 16) {
+      for (int kb = 0; kb < S::KB; ++kb) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&dhk[kb], j & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
         uint32_t dr[16];
-        tmem_ld16_async(tq + c0 + cc, dr);
+        tmem_ld16_async(tq + 64 * kb + 16 * slot, dr);
         tmem_wait_regs(dr);
         float dh[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) dh[i] = __uint_as_float(dr[i]);
-#pragma unroll
         for (int i = 0; i < 16; i += 2) {
-          const float2 gpf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gp[(cc + i) / 2]));
-          dh[i] = valid ? dh[i] * gpf.x : 0.f;
-          dh[i + 1] = valid ? dh[i + 1] * gpf.y : 0.f;
+          const float2 gpf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gp[kb * 8 + i / 2]));
+          dh[i] = valid ? __uint_as_float(dr[i]) * gpf.x : 0.f;
+          dh[i + 1] = valid ? __uint_as_float(dr[i + 1]) * gpf.y : 0.f;
         }
-        put_row16(hs + ((c0 + cc) / 64) * S::TILE, row, ((c0 + cc) % 64) / 8, dh);
+        put_row16(hs + kb * S::TILE, row, 2 * slot, dh);
+        tc_fence_before();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dzk[kb]);
       }
-      tc_fence_before();
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(dzfull);
     }
     // ---- the CTA's gradient partials: accumulator columns [slot PER, (slot + 1) PER)
     if (ok && ntiles > 0) ok = __all_sync(0xffffffffu, mbar_wait(gdone, 0, abort_flag));
