@@ -505,7 +505,12 @@ def run_e2e(args, cfg, layer, x, h2d, d2h, stream, dist, world):
 def run_reference(args, cfg, world):
     """The fp64 CPU oracle, as it stands, on a bounded sample per step (rank 0 only)."""
     import oracle
-    s = cpu_sample_config(cfg, CPU_SAMPLE_TOKENS[args.workload])
+    # about ten full samples of CPU work in all (10-30 s each): a run of many steps times a
+    # proportionally smaller sample per step, so that any --steps K --warmup W ends in minutes
+    full = CPU_SAMPLE_TOKENS[args.workload]
+    scale = min(1.0, 10.0 / max(1, args.steps + args.warmup))
+    tokens = full if scale >= 1.0 else max(min(full, 256), int(full * scale) // 128 * 128)
+    s = cpu_sample_config(cfg, tokens)
     x = gen_inputs(s)
     for _ in range(args.warmup):
         oracle.forward(s, x["Q"], x["K"], x["V"], x["eta"], x["W0"])

@@ -166,14 +166,16 @@ def test_vit3s_full_size_weight_change():
         assert v <= tol, f"{k}: relative Frobenius error {v:.3e} > {tol}"
 
 
-@pytest.mark.parametrize("profiled", [False, True])
-def test_graph_replay_matches_direct_launch(profiled):
+@pytest.mark.parametrize("profiled,causal", [(False, 0), (True, 0), (False, 1), (True, 1)])
+def test_graph_replay_matches_direct_launch(profiled, causal):
     # on a non-default stream ttt_forward captures its launches into a CUDA graph on the
     # first call and replays it afterwards (two alternating instances when profiling);
-    # every replay must give the bits the direct launches give.
+    # every replay must give the bits the direct launches give.  Causal: each chunk's apply
+    # runs on the handle's second stream, forked and joined inside the graph too.
     from weight_sequence_mixing_b200 import binding
-    kw = dict(B=1, H=2, N=640, chunk=256, Nq=300, d=128, h=256, inner="swiglu", loss="neg_dot",
-              opt="momentum_muon", weight_l2norm=True, dtype="bf16", data="lact", eta_mode="per_token", seed=8)
+    kw = dict(B=1, H=2, N=640, chunk=256, Nq=640 if causal else 300, causal=causal, d=128, h=256,
+              inner="swiglu", loss="neg_dot", opt="momentum_muon", weight_l2norm=True, dtype="bf16", data="lact",
+              eta_mode="per_token", seed=8)
     x = gen_inputs(make_config(**kw))
     d = {k: (v.cuda() if v is not None else None) for k, v in x.items()}
     direct = binding.TTTLayer(make_config(direct_launch=True, **kw))
