@@ -63,6 +63,13 @@ SMALL = [
          weight_l2norm=True, epochs=2),
     dict(inner="mlp2_gelu", loss="mse", opt="gd", d=64, h=256, N=700, key_instnorm=True, data="vit",
          eta_mode="scalar", eta_scalar=1.0, epochs=3),
+    # split-K partials with momentum: reduced by their own pass (models with W2), or summed by
+    # the row finish (linear, GLU)
+    dict(inner="swiglu", loss="neg_dot", opt="momentum", d=128, h=256, N=6000, weight_l2norm=True),
+    dict(inner="mlp2_gelu", loss="neg_dot", opt="momentum", d=128, h=256, N=6000, chunk=4608, epochs=2),
+    dict(inner="linear", loss="neg_dot", opt="momentum", d=128, h=128, N=6000, weight_l2norm=True),
+    dict(inner="glu", loss="mse", opt="momentum", d=64, h=64, N=6000, chunk=4608, data="vit", eta_mode="scalar",
+         eta_scalar=1.0, epochs=2),
 ]
 
 

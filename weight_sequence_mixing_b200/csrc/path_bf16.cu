@@ -159,12 +159,16 @@ struct RowMap {
 //           row z % w0_rows for batch-head z)
 //   mode 1: U from the gradient layout
 //   mode 2: U from the Newton-Schulz result (X [m][n], XT [n][m] per matrix)
+//   mode 3: U summed here from the split-K partials part[splits][z][GR][d] (in split order,
+//           as the split reduction would), with momentum M = beta M + U when Mom is given:
+//           every element of the gradient layout belongs to exactly one row of one matrix
 // hold_w2: the rows of W2 keep their values (first-layer-only updates): no step,
 // no row norm; their bf16 copies are rewritten unchanged.
 __global__ void finish_rows_kernel(RowMap rm, int mode, float lr, bool rownorm, bool hold_w2, float* Wf,
                                    const float* U, const float* X, const float* XT, int m, int n, bool src_t,
                                    bf16* First, bf16* W2T, bf16* W2, unsigned* status, const float* W0 = nullptr,
-                                   int w0_rows = 1) {
+                                   int w0_rows = 1, const float* part = nullptr, int splits = 0, float* Mom = nullptr,
+                                   float beta = 0.f) {
   const int z = blockIdx.y;
   const int R = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   if (R >= rm.nrows()) return;
@@ -190,6 +194,24 @@ __global__ void finish_rows_kernel(RowMap rm, int mode, float lr, bool rownorm, 
       for (int i = lane; i < len; i += 32) w[i] -= lr * u[i];
     } else {  // W2 row r = column r of the G2^T rows [0, h)
       for (int i = lane; i < len; i += 32) w[i] -= lr * Uz[int64_t(i) * rm.d + r];
+    }
+  } else if (mode == 3) {
+    const int64_t zoff = int64_t(z) * rm.GR * rm.d, sstride = int64_t(gridDim.y) * rm.GR * rm.d;
+    auto grad = [&](int64_t idx) {
+      float u = part[zoff + idx];
+      for (int sp = 1; sp < splits; ++sp) u += part[sp * sstride + zoff + idx];
+      if (Mom) {
+        const float mm = beta * Mom[zoff + idx] + u;
+        Mom[zoff + idx] = mm;
+        u = mm;
+      }
+      return u;
+    };
+    if (!w2) {
+      const int64_t g0 = int64_t(rm.grad_row(k, r)) * rm.d;
+      for (int i = lane; i < len; i += 32) w[i] -= lr * grad(g0 + i);
+    } else {  // W2 row r = column r of the G2^T rows [0, h)
+      for (int i = lane; i < len; i += 32) w[i] -= lr * grad(int64_t(i) * rm.d + r);
     }
   } else if (mode == 2) {
     const int64_t mn = int64_t(m) * n;
@@ -252,24 +274,24 @@ __global__ void transpose_w2_kernel(int d, int h, const bf16* W2, bf16* W2T) {
 // (cpr = channels / 8 of the current window of at most 2048 channels) and rows
 // t / cpr, t / cpr + 256 / cpr, ...
 //
-// Pass 1: per (z, 128-token block), channel sums and sums of squares -> part[z][blk][ch][2].
+// Pass 1: per (z, block of rb tokens), channel sums and sums of squares -> part[z][blk][ch][2].
 // The block that finishes last for its head (a counter per head, reset by that block)
 // combines the block sums in block order, in double (the biased variance is
 // E[k^2] - E[k]^2), into the mean and 1/sqrt(var + eps) -> stats[z][ch][2].
-__global__ void keystats_kernel(int n, int d, const bf16* K, int64_t k_zs, int t0, float eps, float* part,
+__global__ void keystats_kernel(int n, int d, int rb, const bf16* K, int64_t k_zs, int t0, float eps, float* part,
                                 float* stats, unsigned* done) {
   __shared__ float red[2][2048];  // [sum | sum of squares][row group x channel of the window]
   __shared__ bool last;
   const int z = blockIdx.y, blk = blockIdx.x, nb = gridDim.x;
   const int tid = threadIdx.x;
-  const int rows = min(n - blk * 128, 128);
+  const int rows = min(n - blk * rb, rb);
   for (int c0 = 0; c0 < d; c0 += 2048) {
     const int w = min(d - c0, 2048), cpr = w / 8, groups = 256 / cpr;
     const int piece = tid % cpr, grp = tid / cpr;
     float s[8] = {}, q[8] = {};
     if (grp < groups) {
-      const bf16* base = K + z * k_zs + int64_t(t0 + blk * 128) * d + c0 + 8 * piece;
-#pragma unroll 4
+      const bf16* base = K + z * k_zs + int64_t(t0 + int64_t(blk) * rb) * d + c0 + 8 * piece;
+#pragma unroll 8
       for (int r = grp; r < rows; r += groups) {
         const uint4 u = *reinterpret_cast<const uint4*>(base + int64_t(r) * d);
         const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
@@ -591,7 +613,13 @@ int optimizer_step(Ctx& c) {
   const ttt_config& cfg = p.cfg;
   const bool mom = cfg.opt == TTT_OPT_MOMENTUM || cfg.opt == TTT_OPT_MOMENTUM_MUON;
   const bool muon = cfg.opt == TTT_OPT_MUON || cfg.opt == TTT_OPT_MOMENTUM_MUON;
-  if (!D.direct) {
+  const bool hold_w2 = (cfg.flags & TTT_FLAG_FIRST_LAYER_ONLY) != 0;
+  // plain and momentum steps of models without W2 (linear, GLU) sum the split partials
+  // inside the row finish (no separate reduction pass).  Not with W2: its rows' updates are
+  // strided columns of G2^T, and summing the partials there costs more than the reduction
+  // saves; nor with Muon, which needs the reduced rows and their norms first.
+  const bool fold = !D.direct && !muon && !hold_w2 && (cfg.inner == TTT_INNER_LINEAR || cfg.inner == TTT_INNER_GLU);
+  if (!D.direct && !fold) {
     dim3 g((D.GR + 7) / 8, D.Z);
     {
       StageScope _sc(kStageReduce, st);
@@ -640,10 +668,12 @@ int optimizer_step(Ctx& c) {
   dim3 g((c.rm.nrows() + 7) / 8, D.Z);
   {
     StageScope _sc(kStageFinish, st);
-    finish_rows_kernel<<<g, 256, 0, c.st>>>(c.rm, muon ? 2 : 1, cfg.lr, (cfg.flags & TTT_FLAG_WEIGHT_L2NORM) != 0,
-                                            (cfg.flags & TTT_FLAG_FIRST_LAYER_ONLY) != 0, c.v.at<float>(p, xWf),
+    finish_rows_kernel<<<g, 256, 0, c.st>>>(c.rm, muon ? 2 : fold ? 3 : 1, cfg.lr,
+                                            (cfg.flags & TTT_FLAG_WEIGHT_L2NORM) != 0, hold_w2, c.v.at<float>(p, xWf),
                                             c.v.at<float>(p, xU), X, XT, D.m, D.n, D.src_t, c.v.at<bf16>(p, xFirst),
-                                            c.v.at<bf16>(p, xW2T), c.v.at<bf16>(p, xW2), c.v.status);
+                                            c.v.at<bf16>(p, xW2T), c.v.at<bf16>(p, xW2), c.v.status, nullptr, 1,
+                                            c.v.at<float>(p, xPart), D.splits, mom ? c.v.at<float>(p, xMom) : nullptr,
+                                            cfg.momentum);
   }
   TRY_CUDA(cudaGetLastError());
   return transpose_w2(c);
@@ -782,12 +812,15 @@ int update_chunk(Ctx& c, int t0, int n) {
   const float* kstats = nullptr;  // per-channel key statistics the fused MSE kernel applies itself
   if (cfg.flags & TTT_FLAG_KEY_INSTNORM) {
     float* kst = c.v.at<float>(p, xKstat);
-    const int nb = (n + 127) / 128;  // token blocks holding keys of the chunk
+    // blocks of rb tokens: about two blocks per SM over all heads, each with many loads in flight
+    const int rb = static_cast<int>(std::max<int64_t>(128, std::min<int64_t>(1024, (int64_t(n) * Z / (2 * kPlanSMs) + 127) / 128 * 128)));
+    const int nb = (n + rb - 1) / rb;
     float* kfin = kst + size_t(Z) * (Cp / 128) * d * 2;                   // [Z][d][2] mean, rstd
     unsigned* kdone = reinterpret_cast<unsigned*>(kfin + size_t(Z) * d * 2);  // [Z] blocks finished
     {
       StageScope _sc(kStageKeyNorm, st);
-      keystats_kernel<<<dim3(nb, Z), 256, 0, c.st>>>(n, d, K, int64_t(D.N) * d, t0, cfg.in_eps, kst, kfin, kdone);
+      keystats_kernel<<<dim3(nb, Z), 256, 0, c.st>>>(n, d, rb, K, int64_t(D.N) * d, t0, cfg.in_eps, kst, kfin,
+                                                     kdone);
     }
     TRY_CUDA(cudaGetLastError());
     kstats = kfin;
