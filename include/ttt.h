@@ -46,11 +46,16 @@
  *   The caller owns every buffer (inputs, outputs and the workspace); the handle
  *   owns only host-side state.  Device pointers must be 16-byte aligned and
  *   contiguous.  ttt_forward only enqueues work on `stream` and returns; it
- *   allocates nothing.  One handle must not be used on two streams at once.
+ *   allocates no device memory.  A causal call with more than one chunk runs each
+ *   chunk's apply on a second stream beside the chunk's update (forked from and
+ *   joined back into `stream`, inside a captured graph too): the handle creates
+ *   that stream and two events the first time it needs them on a device, outside
+ *   any stream capture, and ttt_destroy releases them.  One handle must not be
+ *   used on two streams, or by two threads, at once.
  *   Calls run on the device current in the calling thread.  The library sets
  *   its kernels' shared-memory and cluster attributes, and asks how many CTA
  *   pairs fit, once per device, the first time a kernel runs there; one process
- *   may drive layers on several GPUs (handles hold no device state).
+ *   may drive layers on several GPUs (handles hold no device memory).
  *
  * Errors
  *   Calls return TTT_OK (0) or a negative status.  Argument errors are found on
