@@ -216,10 +216,16 @@ struct EpiGradDirect {
   int64_t z_stride;  // elements per batch entry (GR * ld)
   int ld;            // d
   int row0[2], rows[2];
+  // > 0: problem 0 is G2^T (rows [0, w2t_h) of the gradient layout) and its update goes into
+  // the same h * d elements of U transposed, as [d][h] (W2's orientation), so that the row
+  // finish reads W2's update rows contiguously; the momentum keeps the gradient layout.  The
+  // lanes of a warp hold consecutive rows, so each transposed store is one 128-byte run.
+  int w2t_h;
   template <int BN0, int BN1>
   __device__ void run(const EpiCtx& c) const {
     const bool ok = c.m < rows[c.problem];
     const int64_t off = c.z * z_stride + int64_t(row0[c.problem] + c.m) * ld + c.n0;
+    const bool w2t = w2t_h > 0 && c.problem == 0;
     float sq = 0.0f;
 #pragma unroll 1
     for (int cc = 32 * c.part; cc < BN0; cc += 32 * c.nparts) {
@@ -233,7 +239,13 @@ struct EpiGradDirect {
         for (int j = 0; j < 32; ++j) v[j] = beta * mv[j] + v[j];
         store_f32x32(M + off + cc, v);
       }
-      store_f32x32(U + off + cc, v);
+      if (w2t) {
+        float* ut = U + c.z * z_stride + int64_t(c.n0 + cc) * w2t_h + row0[0] + c.m;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) ut[int64_t(j) * w2t_h] = v[j];
+      } else {
+        store_f32x32(U + off + cc, v);
+      }
 #pragma unroll
       for (int j = 0; j < 32; ++j) sq += v[j] * v[j];
     }

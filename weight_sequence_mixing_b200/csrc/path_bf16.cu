@@ -157,7 +157,7 @@ struct RowMap {
 // afterwards by transpose_w2_kernel.
 //   mode 0: no update (initial weights: W = W0 first when W0 is given; W0 [w0_rows][P],
 //           row z % w0_rows for batch-head z)
-//   mode 1: U from the gradient layout
+//   mode 1: U from the gradient layout (w2t_u: W2's rows of it stored as [d][h] instead)
 //   mode 2: U from the Newton-Schulz result (X [m][n], XT [n][m] per matrix)
 //   mode 3: U summed here from the split-K partials part[splits][z][GR][d] (in split order,
 //           as the split reduction would), with momentum M = beta M + U when Mom is given:
@@ -168,7 +168,7 @@ __global__ void finish_rows_kernel(RowMap rm, int mode, float lr, bool rownorm, 
                                    const float* U, const float* X, const float* XT, int m, int n, bool src_t,
                                    bf16* First, bf16* W2T, bf16* W2, unsigned* status, const float* W0 = nullptr,
                                    int w0_rows = 1, const float* part = nullptr, int splits = 0, float* Mom = nullptr,
-                                   float beta = 0.f) {
+                                   float beta = 0.f, bool w2t_u = false) {
   const int z = blockIdx.y;
   const int R = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   if (R >= rm.nrows()) return;
@@ -191,6 +191,9 @@ __global__ void finish_rows_kernel(RowMap rm, int mode, float lr, bool rownorm, 
     const float* Uz = U + int64_t(z) * rm.GR * rm.d;
     if (!w2) {
       const float* u = Uz + int64_t(rm.grad_row(k, r)) * rm.d;
+      for (int i = lane; i < len; i += 32) w[i] -= lr * u[i];
+    } else if (w2t_u) {  // W2's update stored as [d][h]: row r is contiguous
+      const float* u = Uz + int64_t(r) * rm.h;
       for (int i = lane; i < len; i += 32) w[i] -= lr * u[i];
     } else {  // W2 row r = column r of the G2^T rows [0, h)
       for (int i = lane; i < len; i += 32) w[i] -= lr * Uz[int64_t(i) * rm.d + r];
@@ -581,6 +584,14 @@ struct Ctx {
   bool apply_pending = false;  // an apply on io.aux still reads the bf16 weight copies
 };
 
+// An unsplit plain or momentum step of a model with W2 stores W2's update (G2^T) in U
+// transposed, as [d][h] (EpiGradDirect::w2t_h): nothing else reads those rows of U then.
+bool w2_update_transposed(const Ctx& c) {
+  const ttt_config& cfg = c.p.cfg;
+  const bool muon = cfg.opt == TTT_OPT_MUON || cfg.opt == TTT_OPT_MOMENTUM_MUON;
+  return c.D.direct && !muon && (cfg.inner == TTT_INNER_MLP2_GELU || cfg.inner == TTT_INNER_SWIGLU);
+}
+
 // bf16 W2^T from the freshly written bf16 W2: the B operand of the single-CTA token
 // kernel and of the generic MSE path's dH = dY W2.  The pair token kernel, the fused MSE
 // token kernel and the apply read W2 itself.
@@ -673,7 +684,7 @@ int optimizer_step(Ctx& c) {
                                             c.v.at<float>(p, xU), X, XT, D.m, D.n, D.src_t, c.v.at<bf16>(p, xFirst),
                                             c.v.at<bf16>(p, xW2T), c.v.at<bf16>(p, xW2), c.v.status, nullptr, 1,
                                             c.v.at<float>(p, xPart), D.splits, mom ? c.v.at<float>(p, xMom) : nullptr,
-                                            cfg.momentum);
+                                            cfg.momentum, w2_update_transposed(c));
   }
   TRY_CUDA(cudaGetLastError());
   return transpose_w2(c);
@@ -735,7 +746,7 @@ int grad_gemm(Ctx& c, const TM& a0, const TM& b0, const TM& a1, const TM& b1, in
   float* rowsq = muon ? c.v.at<float>(p, xRowSq) : nullptr;
   if (rowsq && cudaMemsetAsync(rowsq, 0, size_t(D.Z) * D.GR * 4, c.st) != cudaSuccess) return TTT_ERR_CUDA;
   EpiGradDirect ep{c.v.at<float>(p, xU), mom ? c.v.at<float>(p, xMom) : nullptr, rowsq, cfg.momentum, pz, d,
-                   {0, r1}, {rows0, rows1}};
+                   {0, r1}, {rows0, rows1}, w2_update_transposed(c) ? D.h : 0};
   return grad_launch(c, a0, b0, a1, b1, rows0, rows1, b0k, b1k, ep);
 }
 
