@@ -213,3 +213,13 @@ def test_fused_mse_plan(B, H, N, chunk, h):
     tiles = -(-got["chunk"] // 128)
     assert got["direct"] == 0 and got["tile_rows"] == 128
     assert got["splits"] == max(1, min(tiles, 148 // (B * H)))
+
+
+@pytest.mark.parametrize("B,H,N,chunk,loss", [(8, 5, 6084, 0, "neg_dot"), (2, 2, 700, 512, "mse"), (1, 1, 300, 0, "neg_dot")])
+def test_fused_glu_plan(B, H, N, chunk, loss):
+    # d = 64 GLU: token GEMM, gating gradient and gradient reduction in one kernel, one CTA
+    # per (head, token-tile range), split partials summed by the row finish
+    cfg = make_config(B=B, H=H, N=N, chunk=chunk, d=64, h=64, inner="glu", loss=loss, opt="gd", dtype="bf16")
+    got = binding.plan_info(cfg)
+    tiles = -(-got["chunk"] // 128)
+    assert got["direct"] == 0 and got["splits"] == max(1, min(tiles, 148 // (B * H)))

@@ -25,6 +25,7 @@
 #include "apply_mlp.cuh"
 #include "epi_glu.cuh"
 #include "epilogues.cuh"
+#include "glu_update.cuh"
 #include "mse_token.cuh"
 #include "ns_fused.cuh"
 #include "token_pair.cuh"
@@ -75,6 +76,13 @@ bool mse_token_path(const ttt_config& c) {
   return c.inner == TTT_INNER_MLP2_GELU && c.loss == TTT_LOSS_MSE && c.d == 64 && (c.h == 128 || c.h == 256);
 }
 
+// The GLU at d = 64 (ViT3's heads) likewise: token GEMM, gating gradient and the gradient
+// reduction in one kernel (glu_update.cuh).
+bool glu_update_path(const ttt_config& c) { return c.inner == TTT_INNER_GLU && c.d == 64; }
+
+// Either fused update: one CTA per (head, token-tile range), split partials reduced by the finish.
+bool fused_update_path(const ttt_config& c) { return mse_token_path(c) || glu_update_path(c); }
+
 Dims dims_of(const Plan& p) {
   const ttt_config& c = p.cfg;
   Dims D{};
@@ -102,7 +110,7 @@ Dims dims_of(const Plan& p) {
   const bool muon = c.opt == TTT_OPT_MUON || c.opt == TTT_OPT_MOMENTUM_MUON;
   // with Muon the squared row norms are summed over the tiles of a row: allow at
   // most two contributions per row (order-independent)
-  D.direct = D.splits == 1 && !(muon && D.grad_bn != c.d) && !mse_token_path(c);
+  D.direct = D.splits == 1 && !(muon && D.grad_bn != c.d) && !fused_update_path(c);
   D.token_pairs = (c.flags & TTT_FLAG_SINGLE_CTA) == 0;
   return D;
 }
@@ -929,6 +937,30 @@ int update_chunk(Ctx& c, int t0, int n) {
     TRY(tmap(&tYmn, DY, 2, d, Cp, Z, 64));
     TRY(tmap(&tD, A1, 2, h, Cp, Z, 64));
     TRY(grad_gemm(c, tH, tYmn, tD, *tXmn, h, h, h, 0, xoff));
+  } else if (glu_update_path(cfg)) {
+    // one kernel: Z = X [Wb; Wa]^T, the gating gradient and G = dZ^T X per (head, token-tile
+    // range) -> split partials (glu_update.cuh)
+    TM tw;
+    TRY(tmap(&tw, c.v.at<bf16>(p, xFirst), 2, d, 2 * d, Z, 128));
+    if (tX->box != 128 || c.tV.box != 128 || D.direct) return TTT_ERR_INVALID_ARG;
+    GluGeom gg;
+    gg.m_tiles = (n + 127) / 128;
+    gg.batches = Z;
+    gg.splits = D.splits;
+    gg.rows_valid = n;
+    gg.x_off = xoff;
+    gg.v_off = t0;
+    gg.t0 = t0;
+    gg.eta = c.io.eta;
+    gg.eta_zs = D.N;
+    gg.eta_scalar = cfg.eta_scalar;
+    gg.mse = cfg.loss == TTT_LOSS_MSE ? 1 : 0;
+    gg.coef = 2.0f / (float(n) * float(d));
+    gg.part = c.v.at<float>(p, xPart);
+    {
+      StageScope sc(kStageTokenPhase, c.st);
+      TRY_CUDA(launch_glu_update(tX->m, c.tV.m, tw.m, gg, status, c.st));
+    }
   } else if (cfg.inner == TTT_INNER_GLU) {
     // Z = X [Wb_blk; Wa_blk]^T per 64-channel block -> dZ (gate, linear), then G = dZ^T X
     EpiGluGrad eg{A1, d, n, int64_t(Cp) * 2 * d, V, int64_t(D.N) * d, t0, c.io.eta, D.N, cfg.eta_scalar,
@@ -1054,8 +1086,8 @@ void choose_grad_shape(const Plan& p, int Cp, int* splits, int* tile_rows, int* 
                                                     : 3 * h;
   const int r0 = c.inner == TTT_INNER_LINEAR ? d : c.inner == TTT_INNER_GLU ? 2 * d : h;
   const int kblocks = Cp / 64;
-  if (mse_token_path(c)) {
-    // the fused MSE kernel: one CTA per (head, token-tile range), one wave of them
+  if (fused_update_path(c)) {
+    // the fused update kernels: one CTA per (head, token-tile range), one wave of them
     *splits = std::max(1, std::min(Cp / 128, kPlanSMs / std::max(1, p.BH)));
     *tile_rows = 128;
     *grad_bn = 64;
@@ -1131,7 +1163,7 @@ int plan_layout_bf16(Plan* p) {
       act ? Z * d * h * 2 : 0,
       ((c.flags & TTT_FLAG_KEY_INSTNORM) && !mse_token_path(c)) ? Z * Cp * d * 2 : 0,
       (act && spill) ? Z * Cp * h * 2 : 0,
-      ((act && spill) || glu) ? Z * Cp * 2 * h * 2 : 0,  // dZ13 / dZ (GLU: h = d)
+      ((act && spill) || (glu && !glu_update_path(c))) ? Z * Cp * 2 * h * 2 : 0,  // dZ13 / dZ (GLU: h = d)
       (mlp_mse && spill) ? Z * Cp * h * 2 : 0,
       ((mlp_mse && spill) || !act) ? Z * Cp * d * 2 : 0,
       (act && d != 64 && d != 128 && d != 256) ? Z * D.Rq * h * 2 : 0,  // two-GEMM apply only (d = 512)
