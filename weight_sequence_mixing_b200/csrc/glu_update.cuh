@@ -12,10 +12,12 @@
 //
 // Pipelining: Z of the next tile is issued before G of the current one, into the other Z
 // buffer; dZ has two shared-memory buffers, so the gating of tile j + 1 overlaps G of tile j.
+// A key/value slot stays busy until G of its tile has read the keys, so four slots keep the
+// loads of the next tiles in flight across that chain.
 //
-// Warps: 0 TMA producer (keys and values of two tiles in flight, the head's weights once),
-// 1 MMA issuer, 2..9 epilogue (two per TMEM lane quarter; warp part p owns channels
-// [32 p, 32 p + 32)).  Every wait is bounded.
+// Warps: 0 TMA producer (keys and values of four tiles in flight, the head's weights once),
+// 1 MMA issuer, 2..17 epilogue (four per TMEM lane quarter; warp part p owns channels
+// [16 p, 16 p + 16)).  Every wait is bounded.
 #pragma once
 #include "epi_glu.cuh"
 #include "mse_token.cuh"
@@ -40,8 +42,10 @@ struct GluShape {
   static constexpr int TILE = 128 * 128;  // 128 rows x 64 bf16
   static constexpr int W_BYTES = TILE;    // [Wb 64 rows | Wa 64 rows] x 64
   static constexpr int DZ_BYTES = 2 * TILE;  // [128 tokens][gate 64 | linear 64] as two k-blocks
-  static constexpr int EW = 8;
-  static constexpr int SMEM = 1024 + 2 * 2 * TILE + W_BYTES + 2 * DZ_BYTES + 256;
+  static constexpr int NSLOT = 4;  // key/value slots
+  static constexpr int EW = 16;
+  static constexpr int CH = 64 / (EW / 4);  // channels per epilogue thread
+  static constexpr int SMEM = 1024 + NSLOT * 2 * TILE + W_BYTES + 2 * DZ_BYTES + 256;
   static constexpr uint32_t GCOL = 256;  // TMEM columns of G
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
@@ -53,11 +57,11 @@ __global__ void __launch_bounds__(64 + 32 * GluShape::EW, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xv = smem;  // [slot][X tile | V tile]
-  uint8_t* ws = xv + 2 * 2 * S::TILE;
+  uint8_t* ws = xv + S::NSLOT * 2 * S::TILE;
   uint8_t* dzs = ws + S::W_BYTES;  // [buffer][2 k-blocks]
-  uint64_t* xfull = reinterpret_cast<uint64_t*>(dzs + 2 * S::DZ_BYTES);  // [2]
-  uint64_t* xempty = xfull + 2;   // [2]: G (commit) and the epilogue's V reads are done with the slot
-  uint64_t* zfull = xempty + 2;   // [2] Z buffer written
+  uint64_t* xfull = reinterpret_cast<uint64_t*>(dzs + 2 * S::DZ_BYTES);  // [NSLOT]
+  uint64_t* xempty = xfull + S::NSLOT;  // [NSLOT]: G (commit) and the epilogue's V reads are done with the slot
+  uint64_t* zfull = xempty + S::NSLOT;  // [2] Z buffer written
   uint64_t* zempty = zfull + 2;   // [2] Z buffer read
   uint64_t* dzfull = zempty + 2;  // [2] dZ buffer written
   uint64_t* dzempty = dzfull + 2;  // [2] G done reading the dZ buffer
@@ -74,9 +78,11 @@ __global__ void __launch_bounds__(64 + 32 * GluShape::EW, 1)
   const int ntiles = static_cast<int>(int64_t(sp + 1) * g.m_tiles / g.splits) - mt0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < S::NSLOT; ++s) {
       mbar_init(&xfull[s], 1);
       mbar_init(&xempty[s], 1 + S::EW);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&zfull[s], 1);
       mbar_init(&zempty[s], S::EW);
       mbar_init(&dzfull[s], S::EW);
@@ -105,8 +111,8 @@ __global__ void __launch_bounds__(64 + 32 * GluShape::EW, 1)
       mbar_arrive_expect_tx(wfull, S::W_BYTES);
       tma_load_3d(ws, &tW, wfull, 0, 0, z);
       for (int j = 0; j < ntiles; ++j) {
-        const int s = j & 1, mt = mt0 + j;
-        if (j >= 2 && !mbar_wait(&xempty[s], ((j - 2) >> 1) & 1, abort_flag)) break;
+        const int s = j % S::NSLOT, mt = mt0 + j;
+        if (j >= S::NSLOT && !mbar_wait(&xempty[s], ((j - S::NSLOT) / S::NSLOT) & 1, abort_flag)) break;
         uint8_t* slot = xv + s * 2 * S::TILE;
         mbar_arrive_expect_tx(&xfull[s], 2 * S::TILE);
         tma_load_3d(slot, &tX, &xfull[s], 0, g.x_off + mt * 128, z);
@@ -124,28 +130,29 @@ __global__ void __launch_bounds__(64 + 32 * GluShape::EW, 1)
       constexpr uint32_t idG = make_idesc(128, 64, 1, true, true);     // G = dZ^T X, both MN-major
       const uint32_t wa = smem_u32(ws);
       // G += dZ^T X of tile jj: A = dZ buffer jj & 1 read MN-major (64-column runs of the 128
-      // rows 16 KB apart, 16-token steps of 2 KB), B = the keys of slot jj & 1
+      // rows 16 KB apart, 16-token steps of 2 KB), B = the keys of slot jj % NSLOT
       auto issue_g = [&](int jj) -> bool {
         const int b = jj & 1;
         if (!mbar_wait(&dzfull[b], (jj >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t da = smem_u32(dzs + b * S::DZ_BYTES), xa = smem_u32(xv + b * 2 * S::TILE);
+        const int xs = jj % S::NSLOT;
+        const uint32_t da = smem_u32(dzs + b * S::DZ_BYTES), xa = smem_u32(xv + xs * 2 * S::TILE);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_f16(tmem_base + S::GCOL, make_sdesc_sw128(da + kk * 2048, S::TILE, 1024),
                   make_sdesc_sw128(xa + kk * 2048, S::TILE, 1024), idG, (jj > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&dzempty[b]);
-        mma_commit(&xempty[b]);
+        mma_commit(&xempty[xs]);
         return true;
       };
       bool ok = mbar_wait(wfull, 0, abort_flag);
       for (int j = 0; j < ntiles && ok; ++j) {
-        const int b = j & 1;
-        if (!(ok = mbar_wait(&xfull[b], (j >> 1) & 1, abort_flag))) break;
+        const int b = j & 1, xs = j % S::NSLOT;
+        if (!(ok = mbar_wait(&xfull[xs], (j / S::NSLOT) & 1, abort_flag))) break;
         // Z buffer b was last read by the epilogue of tile j - 2
         if (j >= 2 && !(ok = mbar_wait(&zempty[b], ((j - 2) >> 1) & 1, abort_flag))) break;
         tc_fence_after();
-        const uint32_t xa = smem_u32(xv + b * 2 * S::TILE);
+        const uint32_t xa = smem_u32(xv + xs * 2 * S::TILE);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_f16(tmem_base + b * 128, make_sdesc_sw128(xa + kk * 32, 16, 1024),
@@ -162,29 +169,37 @@ __global__ void __launch_bounds__(64 + 32 * GluShape::EW, 1)
     }
   } else {
     const int q = warp & 3;
-    const int part = (warp - 2) >> 2;  // channels [32 part, 32 part + 32)
+    const int part = (warp - 2) >> 2;  // channels [CH part, CH part + CH)
     const int row = q * 32 + lane;
     const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     bool ok = true;
     for (int j = 0; j < ntiles && ok; ++j) {
-      const int b = j & 1;
+      const int b = j & 1, xs = j % S::NSLOT;
       const int m = (mt0 + j) * 128 + row;
       const bool valid = m < g.rows_valid;
       ok = __all_sync(0xffffffffu, mbar_wait(&zfull[b], (j >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      float zb[32], za[32];
-      tmem_ld32(tq + b * 128 + 32 * part, zb);
-      tmem_ld32(tq + b * 128 + 64 + 32 * part, za);
+      uint32_t rb[S::CH], ra[S::CH];
+      tmem_ld16_async(tq + b * 128 + S::CH * part, rb);
+      tmem_ld16_async(tq + b * 128 + 64 + S::CH * part, ra);
+      tmem_wait_regs(rb);
+      tmem_wait_regs(ra);
+      float zb[S::CH], za[S::CH];
+#pragma unroll
+      for (int i = 0; i < S::CH; ++i) {
+        zb[i] = __uint_as_float(rb[i]);
+        za[i] = __uint_as_float(ra[i]);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&zempty[b]);
       // this row's 32 values of V from the slot's V tile (128-byte swizzled rows)
-      const uint8_t* vt = xv + b * 2 * S::TILE + S::TILE;
-      float v[32];
+      const uint8_t* vt = xv + xs * 2 * S::TILE + S::TILE;
+      float v[S::CH];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint4 u = *sw128_chunk(const_cast<uint8_t*>(vt), row, 4 * part + k);
+      for (int k = 0; k < S::CH / 8; ++k) {
+        const uint4 u = *sw128_chunk(const_cast<uint8_t*>(vt), row, (S::CH / 8) * part + k);
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -194,10 +209,10 @@ __global__ void __launch_bounds__(64 + 32 * GluShape::EW, 1)
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&xempty[b]);
+      if (lane == 0) mbar_arrive(&xempty[xs]);
       const float e = valid ? (g.eta ? g.eta[z * g.eta_zs + g.t0 + m] : g.eta_scalar) : 0.0f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < S::CH; ++i) {
         const float s = sigmoid_dev(zb[i]);
         const float silu = zb[i] * s;
         const float df = g.mse ? g.coef * e * (za[i] * silu - v[i]) : -e * v[i];
@@ -213,11 +228,11 @@ __global__ void __launch_bounds__(64 + 32 * GluShape::EW, 1)
       }
       uint8_t* dz = dzs + b * S::DZ_BYTES;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        *sw128_chunk(dz, row, 4 * part + k) =
+      for (int k = 0; k < S::CH / 8; ++k) {
+        *sw128_chunk(dz, row, (S::CH / 8) * part + k) =
             make_uint4(pack_bf16x2(zb[8 * k], zb[8 * k + 1]), pack_bf16x2(zb[8 * k + 2], zb[8 * k + 3]),
                        pack_bf16x2(zb[8 * k + 4], zb[8 * k + 5]), pack_bf16x2(zb[8 * k + 6], zb[8 * k + 7]));
-        *sw128_chunk(dz + S::TILE, row, 4 * part + k) =
+        *sw128_chunk(dz + S::TILE, row, (S::CH / 8) * part + k) =
             make_uint4(pack_bf16x2(za[8 * k], za[8 * k + 1]), pack_bf16x2(za[8 * k + 2], za[8 * k + 3]),
                        pack_bf16x2(za[8 * k + 4], za[8 * k + 5]), pack_bf16x2(za[8 * k + 6], za[8 * k + 7]));
       }
@@ -225,21 +240,23 @@ __global__ void __launch_bounds__(64 + 32 * GluShape::EW, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&dzfull[b]);
     }
-    // the CTA's partial of G: this warp's 32 columns of rows 32 q .. 32 q + 31
+    // the CTA's partial of G: this warp's CH columns of rows 32 q .. 32 q + 31
     if (ok && ntiles > 0) ok = __all_sync(0xffffffffu, mbar_wait(gdone, 0, abort_flag));
     if (ok) {
       tc_fence_after();
-      float gv[32];
+      uint32_t gr[S::CH];
       if (ntiles > 0) {
-        tmem_ld32(tq + S::GCOL + 32 * part, gv);
+        tmem_ld16_async(tq + S::GCOL + S::CH * part, gr);
+        tmem_wait_regs(gr);
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) gv[i] = 0.f;
+        for (int i = 0; i < S::CH; ++i) gr[i] = 0u;
       }
-      float* dst = g.part + ((int64_t(sp) * g.batches + z) * 128 + row) * 64 + 32 * part;
+      float* dst = g.part + ((int64_t(sp) * g.batches + z) * 128 + row) * 64 + S::CH * part;
 #pragma unroll
-      for (int i = 0; i < 32; i += 4)
-        *reinterpret_cast<float4*>(dst + i) = make_float4(gv[i], gv[i + 1], gv[i + 2], gv[i + 3]);
+      for (int i = 0; i < S::CH; i += 4)
+        *reinterpret_cast<float4*>(dst + i) = make_float4(__uint_as_float(gr[i]), __uint_as_float(gr[i + 1]),
+                                                          __uint_as_float(gr[i + 2]), __uint_as_float(gr[i + 3]));
     }
   }
 
