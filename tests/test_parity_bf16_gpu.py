@@ -95,6 +95,10 @@ TOKEN_KERNEL_CASES = [
     dict(inner="mlp2_gelu", d=128, h=384, N=700, chunk=384),
     # enough k-blocks for split weight gradients on 512-row pair tiles (rows 3h = 1536)
     dict(inner="swiglu", d=256, h=512, N=8192, opt="momentum_muon", weight_l2norm=True),
+    # enough token tiles per pair for resident weight blocks: the pairs' token-tile ranges
+    # cross from one head into the next (a weight reload) and end on a ragged tile
+    dict(inner="swiglu", d=256, h=512, N=5000, opt="momentum", weight_l2norm=True),
+    dict(inner="mlp2_gelu", d=128, h=256, N=9800),
 ]
 
 

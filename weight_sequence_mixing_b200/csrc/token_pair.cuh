@@ -17,6 +17,17 @@
 // 16 KB + 16 KB / 32 KB, which is what limits the single-CTA kernel (the rate at
 // which an SM can pull operand tiles out of L2).
 //
+// Two ways to feed the weights.  Streaming (any d): every operand stage carries a k-block
+// of tokens and the matching k-block of the weight block, and consecutive tiles of a pair
+// step through the hidden blocks.  Resident (d <= 256): a pair keeps its half of one
+// hidden block's weights (W2 columns and [W1; W3] rows, 96 KB per CTA for SwiGLU at
+// d = 256) in shared memory and walks a range of token tiles; the stages carry tokens
+// only, so a CTA pulls 128 instead of 224 KB per tile out of L2.  The pairs come in
+// groups of h / 128, one per hidden block, that walk the same token tiles, so every key
+// and value tile still crosses HBM once and is read from L2 by the rest of its group.
+// The weights are reloaded when the range crosses into the next head, after every MMA
+// that read them has completed (the last stage's release).
+//
 // TMEM per CTA: Z13 in columns [0, 256), P in one of two 128-column slots (256 or
 // 384, alternating by tile), so a tile's P phase overlaps the previous tile's
 // epilogue.  An epilogue warp reads its first 32-column chunk, computes and packs
@@ -27,6 +38,7 @@
 //   full[s]    (leader only)  the leader's producer arms it with both CTAs' bytes;
 //                             both producers' TMA loads count their bytes on it.
 //   empty[s]   (both)         the leader's MMA commit arrives on both CTAs' copies.
+//   wfull      (leader only)  resident weights: both CTAs' weight bytes of a head.
 //   tmem_full  (both)         the leader's commit after a tile's last MMA.
 //   tmem_empty (leader only)  one arrival per epilogue warp of both CTAs: the tile's
 //                             Z13 and P columns have been read.
@@ -37,7 +49,7 @@
 
 namespace ttt {
 
-template <bool SWIGLU>
+template <bool SWIGLU, bool RESB>
 struct PairShape {
   static constexpr int A_BYTES = 128 * 128;         // this CTA's 128 tokens x 64 bf16
   static constexpr int BZ_ROWS = SWIGLU ? 128 : 64;  // this CTA's half of the first-layer rows
@@ -46,33 +58,78 @@ struct PairShape {
   static constexpr int BP_BYTES = BP_ROWS * 128;
   static constexpr int Z_STAGE = A_BYTES + BZ_BYTES;
   static constexpr int P_STAGE = A_BYTES + BP_BYTES;
-  static constexpr int SLOT = Z_STAGE > P_STAGE ? Z_STAGE : P_STAGE;
-  static constexpr int STAGES = 6;  // operand ring: the P and Z phases are bound by what is in flight
+  // streaming: a stage holds a k-block of tokens and one of weights; resident: tokens only
+  static constexpr int SLOT = RESB ? A_BYTES : (Z_STAGE > P_STAGE ? Z_STAGE : P_STAGE);
+  static constexpr int KB_RES = 4;  // resident weights: up to 4 k-blocks (d <= 256)
+  static constexpr int WP_BYTES = RESB ? KB_RES * BP_BYTES : 0;  // resident W2 columns [kb]
+  static constexpr int WZ_BYTES = RESB ? KB_RES * BZ_BYTES : 0;  // resident first-layer rows [kb]
+  // operand ring: the P and Z phases are bound by what is in flight
+  static constexpr int STAGES = RESB ? (SWIGLU ? 6 : 8) : 6;
   static constexpr int EW = 16;           // epilogue warps: 4 per TMEM lane quarter
   static constexpr int STG_BYTES = 1024;  // one [32 rows][16 bf16] output box
   static constexpr int STG_BOXES = 2;     // ring of output boxes per epilogue warp
   static constexpr int STG_WARP = STG_BOXES * STG_BYTES;
-  static constexpr int SMEM = 1024 + STAGES * SLOT + EW * STG_WARP + 256;
+  static constexpr int SMEM = 1024 + WP_BYTES + WZ_BYTES + STAGES * SLOT + EW * STG_WARP + 256;
   static constexpr int ZN = SWIGLU ? 256 : 128;  // MMA N of the Z phase (both halves)
   static_assert(SMEM <= 227 * 1024, "shared memory");
+  static_assert(2 * STAGES + 4 <= 30, "barrier area");
 };
 
-template <bool SWIGLU>
-__global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
+// The tiles of one pair, in processing order.  Streaming: tile k is t = pair + k npairs
+// of the (z, token tile, hidden block) sequence, hidden block fastest.  Resident: the
+// pair owns hidden block pair % n_tiles and the range of (z, token tile) pairs of its group.
+template <bool RESB>
+struct PairTiles {
+  int count, u0, nt;
+  __device__ PairTiles(const TokGeom& g, int pair, int npairs) {
+    if constexpr (RESB) {
+      const int groups = npairs / g.n_tiles, gi = pair / g.n_tiles;
+      const int64_t U = int64_t(g.batches) * g.m_tiles;
+      nt = pair % g.n_tiles;
+      u0 = gi < groups ? static_cast<int>(gi * U / groups) : 0;
+      count = gi < groups ? static_cast<int>((gi + 1) * U / groups) - u0 : 0;
+    } else {
+      const int total = g.m_tiles * g.n_tiles * g.batches;
+      nt = 0;
+      u0 = pair;
+      count = pair < total ? (total - pair + npairs - 1) / npairs : 0;
+    }
+  }
+  __device__ void at(const TokGeom& g, int npairs, int k, int& z, int& mt, int& n) const {
+    if constexpr (RESB) {
+      const int u = u0 + k;
+      z = u / g.m_tiles;
+      mt = u % g.m_tiles;
+      n = nt;
+    } else {
+      const int t = u0 + k * npairs;
+      n = t % g.n_tiles;
+      mt = (t / g.n_tiles) % g.m_tiles;
+      z = t / (g.n_tiles * g.m_tiles);
+    }
+  }
+};
+
+template <bool SWIGLU, bool RESB>
+__global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU, RESB>::EW, 1)
     token_pair_kernel(const __grid_constant__ CUtensorMap tX, const __grid_constant__ CUtensorMap tFirst,
                       const __grid_constant__ CUtensorMap tV, const __grid_constant__ CUtensorMap tW2,
                       const __grid_constant__ CUtensorMap tHp, const __grid_constant__ CUtensorMap tDZ,
                       const TokGeom g, unsigned* status) {
-  using S = PairShape<SWIGLU>;
+  using S = PairShape<SWIGLU, RESB>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* wp = base;                  // resident W2 columns (RESB)
+  uint8_t* wz = wp + S::WP_BYTES;      // resident first-layer rows (RESB)
+  uint8_t* smem = wz + S::WZ_BYTES;    // operand ring
   uint8_t* stg = smem + S::STAGES * S::SLOT;
   uint64_t* full = reinterpret_cast<uint64_t*>(stg + S::EW * S::STG_WARP);
   uint64_t* empty = full + S::STAGES;
   uint64_t* tmem_full = empty + S::STAGES;
   uint64_t* tmem_empty = tmem_full + 1;
   uint64_t* drain = tmem_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* wfull = drain + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wfull + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t rank = cluster_rank() & 1u;
@@ -80,7 +137,7 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = static_cast<int>(lane_id());
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  const int total = g.m_tiles * g.n_tiles * g.batches;  // m_tiles counts 256-token tiles
+  const PairTiles<RESB> tiles(g, pair, npairs);  // m_tiles counts 256-token tiles
   const int KB = g.kblocks;
 
   if (threadIdx.x == 0) {
@@ -91,6 +148,7 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
     mbar_init(tmem_full, 1);
     mbar_init(tmem_empty, 2 * S::EW);
     mbar_init(drain, 1);
+    mbar_init(wfull, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -111,13 +169,29 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
       tma_prefetch_desc(&tV);
       tma_prefetch_desc(&tW2);
       const uint32_t full0 = mapa_shared(smem_u32(full), 0);  // the leader's full[0]
-      int it = 0;
+      const uint32_t wfull0 = mapa_shared(smem_u32(wfull), 0);
+      int it = 0, wz_head = -1;
       bool stop = false;
-      for (int t = pair; t < total && !stop; t += npairs) {
-        const int nt = t % g.n_tiles;
-        const int mt = (t / g.n_tiles) % g.m_tiles;
-        const int z = t / (g.n_tiles * g.m_tiles);
+      for (int k = 0; k < tiles.count && !stop; ++k) {
+        int z, mt, nt;
+        tiles.at(g, npairs, k, z, mt, nt);
         const int m0 = mt * 256 + static_cast<int>(rank) * 128;
+        if (RESB && z != wz_head) {
+          // every MMA that read the previous head's weights has completed: the last
+          // stage it issued has been released
+          if (it > 0 && !mbar_wait(&empty[(it - 1) % S::STAGES], ((it - 1) / S::STAGES) & 1, abort_flag)) {
+            stop = true;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(wfull, 2 * KB * (S::BP_BYTES + S::BZ_BYTES));
+          for (int kb = 0; kb < KB; ++kb) {
+            tma_load_3d_pair(wp + kb * S::BP_BYTES, &tW2, wfull0, nt * 128 + static_cast<int>(rank) * S::BP_ROWS,
+                             kb * 64, z);
+            tma_load_3d_pair(wz + kb * S::BZ_BYTES, &tFirst, wfull0, kb * 64,
+                             nt * (2 * S::BZ_ROWS) + static_cast<int>(rank) * S::BZ_ROWS, z);
+          }
+          wz_head = z;
+        }
         for (int phase = 0; phase < 2 && !stop; ++phase) {
           for (int kb = 0; kb < KB; ++kb, ++it) {
             const int s = it % S::STAGES;
@@ -129,15 +203,18 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
             uint8_t* st = smem + s * S::SLOT;
             const uint32_t fb = full0 + static_cast<uint32_t>(s) * 8u;
             if (phase == 0) {
-              if (leader) mbar_arrive_expect_tx(&full[s], 2 * S::P_STAGE);
+              if (leader) mbar_arrive_expect_tx(&full[s], 2 * (RESB ? S::A_BYTES : S::P_STAGE));
               tma_load_3d_pair(st, &tV, fb, kb * 64, m0 + g.v_off, z);
               // W2 [d][h]: 64 of the block's columns (N) x the k-block's 64 rows (K), MN-major
-              tma_load_3d_pair(st + S::A_BYTES, &tW2, fb, nt * 128 + static_cast<int>(rank) * S::BP_ROWS, kb * 64, z);
+              if (!RESB)
+                tma_load_3d_pair(st + S::A_BYTES, &tW2, fb, nt * 128 + static_cast<int>(rank) * S::BP_ROWS, kb * 64,
+                                 z);
             } else {
-              if (leader) mbar_arrive_expect_tx(&full[s], 2 * S::Z_STAGE);
+              if (leader) mbar_arrive_expect_tx(&full[s], 2 * (RESB ? S::A_BYTES : S::Z_STAGE));
               tma_load_3d_pair(st, &tX, fb, kb * 64, m0 + g.x_off, z);
-              tma_load_3d_pair(st + S::A_BYTES, &tFirst, fb, kb * 64,
-                               nt * (2 * S::BZ_ROWS) + static_cast<int>(rank) * S::BZ_ROWS, z);
+              if (!RESB)
+                tma_load_3d_pair(st + S::A_BYTES, &tFirst, fb, kb * 64,
+                                 nt * (2 * S::BZ_ROWS) + static_cast<int>(rank) * S::BZ_ROWS, z);
             }
           }
         }
@@ -158,11 +235,24 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
     if (leader && elect_one()) {
       constexpr uint32_t idP = make_idesc(256, 128, 1, false, true);
       constexpr uint32_t idZ = make_idesc(256, S::ZN, 1, false, false);
-      const uint32_t sbase = smem_u32(smem);
-      int it = 0, j = 0;
+      const uint32_t sbase = smem_u32(smem), wpbase = smem_u32(wp), wzbase = smem_u32(wz);
+      int it = 0, j = 0, wz_head = -1, wloads = 0;
       bool stop = false;
-      for (int t = pair; t < total && !stop; t += npairs, ++j) {
+      for (; j < tiles.count && !stop; ++j) {
         const uint32_t pcol = (j & 1) ? 384u : 256u;
+        if (RESB) {
+          int z, mt, nt;
+          tiles.at(g, npairs, j, z, mt, nt);
+          if (z != wz_head) {  // this head's weights have landed in both CTAs
+            if (!mbar_wait_cluster(wfull, wloads & 1, abort_flag)) {
+              stop = true;
+              break;
+            }
+            tc_fence_after();
+            ++wloads;
+            wz_head = z;
+          }
+        }
         for (int phase = 0; phase < 2 && !stop; ++phase) {
           if (phase == 1) {
             // both CTAs' epilogues have read the previous tile (Z13 and its P slot)
@@ -183,7 +273,8 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
             }
             tc_fence_after();
             const uint32_t a = sbase + s * S::SLOT;
-            const uint32_t b = a + S::A_BYTES;
+            const uint32_t b = RESB ? (phase == 0 ? wpbase + kb * S::BP_BYTES : wzbase + kb * S::BZ_BYTES)
+                                    : a + S::A_BYTES;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               // P phase: B is MN-major (16 K-rows of 128 bytes per step); Z phase: K-major
@@ -240,11 +331,9 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
         emit(w[1], &tDZ, nt * 128 + cc);
       }
     };
-    int j = 0;
-    for (int t = pair; t < total; t += npairs, ++j) {
-      nt = t % g.n_tiles;
-      const int mt = (t / g.n_tiles) % g.m_tiles;
-      z = t / (g.n_tiles * g.m_tiles);
+    for (int j = 0; j < tiles.count; ++j) {
+      int mt;
+      tiles.at(g, npairs, j, z, mt, nt);
       const int m0 = mt * 256 + static_cast<int>(rank) * 128;
       const bool ready = __all_sync(0xffffffffu, mbar_wait_cluster(tmem_full, j & 1, abort_flag));
       if (!ready) break;
@@ -305,12 +394,12 @@ __global__ void __launch_bounds__(64 + 32 * PairShape<SWIGLU>::EW, 1)
   if (warp == 1) tmem_dealloc_pair(tmem_base, 512);
 }
 
-template <bool SWIGLU>
+template <bool SWIGLU, bool RESB>
 cudaLaunchConfig_t pair_launch_config(int pairs, cudaStream_t st, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(64 + 32 * PairShape<SWIGLU>::EW, 1, 1);
-  cfg.dynamicSmemBytes = PairShape<SWIGLU>::SMEM;
+  cfg.blockDim = dim3(64 + 32 * PairShape<SWIGLU, RESB>::EW, 1, 1);
+  cfg.dynamicSmemBytes = PairShape<SWIGLU, RESB>::SMEM;
   cfg.stream = st;
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -321,17 +410,17 @@ cudaLaunchConfig_t pair_launch_config(int pairs, cudaStream_t st, cudaLaunchAttr
   return cfg;
 }
 
-// CTA pairs of this kernel that can be resident at once (0: none, use the single-CTA kernel).
-template <bool SWIGLU>
-int token_pair_capacity() {
+// CTA pairs of one form of this kernel that can be resident at once (0: none).
+template <bool SWIGLU, bool RESB>
+int token_pair_capacity_of() {
   static IntPerDevice caps;
   return caps.get(current_device(), [] {
-    auto kern = token_pair_kernel<SWIGLU>;
+    auto kern = token_pair_kernel<SWIGLU, RESB>;
     int cap = 0;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairShape<SWIGLU>::SMEM) ==
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairShape<SWIGLU, RESB>::SMEM) ==
         cudaSuccess) {
       cudaLaunchAttribute attr[1];
-      cudaLaunchConfig_t cfg = pair_launch_config<SWIGLU>(1, nullptr, attr);
+      cudaLaunchConfig_t cfg = pair_launch_config<SWIGLU, RESB>(1, nullptr, attr);
       int n = 0;
       if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) cap = n;
     }
@@ -340,20 +429,41 @@ int token_pair_capacity() {
   });
 }
 
+// CTA pairs of the streaming form (the one every d accepts) that can be resident at
+// once (0: none, use the single-CTA kernel).
+template <bool SWIGLU>
+int token_pair_capacity() {
+  return token_pair_capacity_of<SWIGLU, false>();
+}
+
 // g.m_tiles counts 256-token tiles; g.rows_alloc bounds the rows the stores may write.
+// Resident weights when d <= 256 and every pair of a full wave of groups (h / 128 pairs
+// each) gets at least kResMinTiles token tiles to spread its weight load over (the
+// causal language layer's 2048-token chunks give a pair one or two: streaming measured
+// faster there); the streaming form otherwise.
+constexpr int kResMinTiles = 4;
 template <bool SWIGLU>
 cudaError_t launch_token_pair(const CUtensorMap& tX, const CUtensorMap& tFirstHalf, const CUtensorMap& tV,
                               const CUtensorMap& tW2Mn, const CUtensorMap& tHp, const CUtensorMap& tDZ,
                               const TokGeom& g, unsigned* status, cudaStream_t st) {
-  const int cap = token_pair_capacity<SWIGLU>();
-  if (cap <= 0) return cudaErrorInvalidConfiguration;
   const long long total = static_cast<long long>(g.m_tiles) * g.n_tiles * g.batches;
   if (total <= 0) return cudaSuccess;
   if (total > 0x7fffffffLL || g.kblocks <= 0) return cudaErrorInvalidConfiguration;
-  const int pairs = static_cast<int>(std::min<long long>(total, cap));
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = pair_launch_config<SWIGLU>(pairs, st, attr);
-  return cudaLaunchKernelEx(&cfg, token_pair_kernel<SWIGLU>, tX, tFirstHalf, tV, tW2Mn, tHp, tDZ, g, status);
+  if (g.kblocks <= PairShape<SWIGLU, true>::KB_RES) {
+    const int cap = token_pair_capacity_of<SWIGLU, true>();
+    const long long groups = cap / g.n_tiles, U = static_cast<long long>(g.m_tiles) * g.batches;
+    if (groups > 0 && U >= kResMinTiles * groups) {
+      cudaLaunchConfig_t cfg = pair_launch_config<SWIGLU, true>(static_cast<int>(groups * g.n_tiles), st, attr);
+      return cudaLaunchKernelEx(&cfg, token_pair_kernel<SWIGLU, true>, tX, tFirstHalf, tV, tW2Mn, tHp, tDZ, g,
+                                status);
+    }
+  }
+  const int cap = token_pair_capacity<SWIGLU>();
+  if (cap <= 0) return cudaErrorInvalidConfiguration;
+  const int pairs = static_cast<int>(std::min<long long>(total, cap));
+  cudaLaunchConfig_t cfg = pair_launch_config<SWIGLU, false>(pairs, st, attr);
+  return cudaLaunchKernelEx(&cfg, token_pair_kernel<SWIGLU, false>, tX, tFirstHalf, tV, tW2Mn, tHp, tDZ, g, status);
 }
 
 }  // namespace ttt
