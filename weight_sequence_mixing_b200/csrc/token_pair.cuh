@@ -63,11 +63,13 @@ struct PairShape {
   static constexpr int KB_RES = 4;  // resident weights: up to 4 k-blocks (d <= 256)
   static constexpr int WP_BYTES = RESB ? KB_RES * BP_BYTES : 0;  // resident W2 columns [kb]
   static constexpr int WZ_BYTES = RESB ? KB_RES * BZ_BYTES : 0;  // resident first-layer rows [kb]
-  // operand ring: the P and Z phases are bound by what is in flight
-  static constexpr int STAGES = RESB ? (SWIGLU ? 6 : 8) : 6;
+  // operand ring: the P and Z phases are bound by what is in flight.  Resident SwiGLU
+  // weights leave room for 7 stages only with one output box per warp: the stages pay
+  // more than the box (7 stages and 1 box ran 3% faster than 6 and 2, 5 and 3, 4 and 4)
+  static constexpr int STAGES = RESB ? (SWIGLU ? 7 : 8) : 6;
   static constexpr int EW = 16;           // epilogue warps: 4 per TMEM lane quarter
   static constexpr int STG_BYTES = 1024;  // one [32 rows][16 bf16] output box
-  static constexpr int STG_BOXES = 2;     // ring of output boxes per epilogue warp
+  static constexpr int STG_BOXES = RESB && SWIGLU ? 1 : 2;  // ring of output boxes per epilogue warp
   static constexpr int STG_WARP = STG_BOXES * STG_BYTES;
   static constexpr int SMEM = 1024 + WP_BYTES + WZ_BYTES + STAGES * SLOT + EW * STG_WARP + 256;
   static constexpr int ZN = SWIGLU ? 256 : 128;  // MMA N of the Z phase (both halves)
