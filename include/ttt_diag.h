@@ -73,6 +73,21 @@ int64_t ttt_launch_count(const ttt_handle* handle);
  * kernel cannot run there and the token phase falls back to single CTAs. */
 int ttt_token_pair_capacity(int swiglu);
 
+/* The token phase's CTA-pair tile schedule (host logic only, no GPU needed; LaCT analysis,
+ * "Nonlinear memory complements local attention": the chunk's forward and backprop through
+ * the fast weights, tile by tile).  Geometry: m_tiles 256-token tiles per head, n_tiles
+ * hidden blocks of 128 units, batches heads, kblocks = d / 64.  cap_resident and
+ * cap_streaming: CTA pairs of the resident-weight and the streaming form that fit the
+ * device.  Chooses the form and the number of pairs as the launch does and writes them to
+ * *resident (1 resident, 0 streaming) and *pairs; then, pair by pair, counts[p] = the tiles
+ * of pair p and its tiles in processing order as (head, token tile, hidden block) int
+ * triples in `tiles`, at most max_tiles triples (`counts` holds at least
+ * max(cap_resident, cap_streaming) ints; all buffers caller-owned host memory).  Returns the
+ * number of triples written; TTT_ERR_INVALID_ARG on bad arguments or a too small `tiles`,
+ * TTT_ERR_UNSUPPORTED when no pair fits. */
+int ttt_pair_schedule(int m_tiles, int n_tiles, int batches, int kblocks, int cap_resident, int cap_streaming,
+                      int* resident, int* pairs, int* counts, int* tiles, int64_t max_tiles);
+
 #ifdef __cplusplus
 }
 #endif

@@ -39,7 +39,7 @@ EXPORTED = [
     "ttt_host_staging_size", "ttt_forward_host", "ttt_query_status", "ttt_destroy", "ttt_status_string",
     "ttt_selftest_gemm", "ttt_profile_enable", "ttt_profile_collect", "ttt_stage_name", "ttt_launch_count",
     "ttt_forward_noalloc", "ttt_token_pair_capacity", "ttt_selftest_timeout", "ttt_plan_info",
-    "ttt_state_size", "ttt_forward_state", "ttt_selftest_activation",
+    "ttt_state_size", "ttt_forward_state", "ttt_selftest_activation", "ttt_pair_schedule",
 ]
 NUM_STAGES = 8
 
@@ -88,6 +88,7 @@ def _load():
         "ttt_token_pair_capacity": (i32, [i32]),
         "ttt_selftest_timeout": (i32, [vp, vp]),
         "ttt_selftest_activation": (i32, [i32, i64, vp, vp, vp, vp]),
+        "ttt_pair_schedule": (i32, [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, i64]),
         "ttt_plan_info": (i32, [vp, ctypes.POINTER(ctypes.c_int), i32]),
         "ttt_state_size": (sz, [vp]),
         "ttt_forward_state": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -302,6 +303,21 @@ def selftest_gemm(A, B, elem_bytes, a_mn, b_mn, bn, M, N, K, batches, splits, st
 def token_pair_capacity(swiglu: bool) -> int:
     """CTA pairs of the token-phase kernel resident at once on the current device (0: single-CTA fallback)."""
     return int(LIB.ttt_token_pair_capacity(int(bool(swiglu))))
+
+
+def pair_schedule(m_tiles: int, n_tiles: int, batches: int, kblocks: int, cap_resident: int,
+                  cap_streaming: int) -> tuple[bool, int, list[int], list[tuple[int, int, int]]]:
+    """The token phase's CTA-pair tile schedule (host logic; see ttt_diag.h): (resident form,
+    pairs, tiles per pair, (head, token tile, hidden block) of every tile pair by pair)."""
+    total = m_tiles * n_tiles * batches
+    counts = (ctypes.c_int * max(cap_resident, cap_streaming, 1))()
+    tiles = (ctypes.c_int * (3 * max(total, 1)))()
+    res, pairs = ctypes.c_int(), ctypes.c_int()
+    n = LIB.ttt_pair_schedule(m_tiles, n_tiles, batches, kblocks, cap_resident, cap_streaming, ctypes.byref(res),
+                              ctypes.byref(pairs), counts, tiles, total)
+    if n < 0:
+        raise TTTError(n, "ttt_pair_schedule")
+    return bool(res.value), pairs.value, list(counts[:pairs.value]), [tuple(tiles[3 * i:3 * i + 3]) for i in range(n)]
 
 
 def selftest_timeout(status_word: torch.Tensor, stream=None) -> int:

@@ -1268,6 +1268,44 @@ extern "C" int ttt_token_pair_capacity(int swiglu) {
   return swiglu ? ttt::token_pair_capacity<true>() : ttt::token_pair_capacity<false>();
 }
 
+namespace {
+template <bool RESB>
+int64_t list_pair_tiles(const ttt::TokGeom& g, int pairs, int* counts, int* tiles, int64_t max_tiles) {
+  int64_t listed = 0;
+  for (int p = 0; p < pairs; ++p) {
+    const ttt::PairTiles<RESB> t(g, p, pairs);
+    counts[p] = t.count;
+    for (int k = 0; k < t.count; ++k, ++listed) {
+      if (listed >= max_tiles) return -1;
+      t.at(g, pairs, k, tiles[3 * listed], tiles[3 * listed + 1], tiles[3 * listed + 2]);
+    }
+  }
+  return listed;
+}
+}  // namespace
+
+extern "C" int ttt_pair_schedule(int m_tiles, int n_tiles, int batches, int kblocks, int cap_resident,
+                                 int cap_streaming, int* resident, int* pairs, int* counts, int* tiles,
+                                 int64_t max_tiles) {
+  if (m_tiles < 1 || n_tiles < 1 || batches < 1 || kblocks < 1 || cap_resident < 0 || cap_streaming < 0 ||
+      !resident || !pairs || !counts || max_tiles < 0 || (!tiles && max_tiles > 0))
+    return TTT_ERR_INVALID_ARG;
+  if (static_cast<long long>(m_tiles) * n_tiles * batches > 0x7fffffffLL) return TTT_ERR_INVALID_ARG;
+  ttt::TokGeom g{};
+  g.m_tiles = m_tiles;
+  g.n_tiles = n_tiles;
+  g.batches = batches;
+  g.kblocks = kblocks;
+  bool resb = false;
+  int np = 0;
+  if (!ttt::pair_grid(g, cap_resident, cap_streaming, resb, np)) return TTT_ERR_UNSUPPORTED;
+  *resident = resb ? 1 : 0;
+  *pairs = np;
+  const int64_t n = resb ? list_pair_tiles<true>(g, np, counts, tiles, max_tiles)
+                         : list_pair_tiles<false>(g, np, counts, tiles, max_tiles);
+  return n < 0 ? TTT_ERR_INVALID_ARG : static_cast<int>(n);
+}
+
 extern "C" int ttt_plan_info(const ttt_handle* h, int* info, int n) {
   if (!h || !info || n < 0) return TTT_ERR_INVALID_ARG;
   const ttt::Plan& p = h->plan;

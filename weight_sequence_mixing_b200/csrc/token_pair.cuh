@@ -49,6 +49,12 @@
 
 namespace ttt {
 
+constexpr int kPairResMaxKb = 4;  // resident weights: up to 4 k-blocks (d <= 256)
+// Resident weights only when every pair of a full wave of groups gets at least this many
+// token tiles to spread its weight load over (the causal language layer's 2048-token chunks
+// give a pair one or two: streaming measured faster there).
+constexpr int kResMinTiles = 4;
+
 template <bool SWIGLU, bool RESB>
 struct PairShape {
   static constexpr int A_BYTES = 128 * 128;         // this CTA's 128 tokens x 64 bf16
@@ -60,7 +66,7 @@ struct PairShape {
   static constexpr int P_STAGE = A_BYTES + BP_BYTES;
   // streaming: a stage holds a k-block of tokens and one of weights; resident: tokens only
   static constexpr int SLOT = RESB ? A_BYTES : (Z_STAGE > P_STAGE ? Z_STAGE : P_STAGE);
-  static constexpr int KB_RES = 4;  // resident weights: up to 4 k-blocks (d <= 256)
+  static constexpr int KB_RES = kPairResMaxKb;
   static constexpr int WP_BYTES = RESB ? KB_RES * BP_BYTES : 0;  // resident W2 columns [kb]
   static constexpr int WZ_BYTES = RESB ? KB_RES * BZ_BYTES : 0;  // resident first-layer rows [kb]
   // operand ring: the P and Z phases are bound by what is in flight.  Resident SwiGLU
@@ -83,7 +89,7 @@ struct PairShape {
 template <bool RESB>
 struct PairTiles {
   int count, u0, nt;
-  __device__ PairTiles(const TokGeom& g, int pair, int npairs) {
+  __host__ __device__ PairTiles(const TokGeom& g, int pair, int npairs) {
     if constexpr (RESB) {
       const int groups = npairs / g.n_tiles, gi = pair / g.n_tiles;
       const int64_t U = int64_t(g.batches) * g.m_tiles;
@@ -97,7 +103,7 @@ struct PairTiles {
       count = pair < total ? (total - pair + npairs - 1) / npairs : 0;
     }
   }
-  __device__ void at(const TokGeom& g, int npairs, int k, int& z, int& mt, int& n) const {
+  __host__ __device__ void at(const TokGeom& g, int npairs, int k, int& z, int& mt, int& n) const {
     if constexpr (RESB) {
       const int u = u0 + k;
       z = u / g.m_tiles;
@@ -438,12 +444,27 @@ int token_pair_capacity() {
   return token_pair_capacity_of<SWIGLU, false>();
 }
 
+// Form and grid of the pair kernel for geometry g (host logic): resident weights when
+// d <= 256 and a full wave of groups (cap_res / n_tiles groups of n_tiles pairs) gives every
+// pair at least kResMinTiles token tiles; streaming on min(tiles, cap_str) pairs otherwise.
+// cap_res, cap_str: pairs of each form that fit the device.  false: no pair fits.
+inline bool pair_grid(const TokGeom& g, int cap_res, int cap_str, bool& resb, int& pairs) {
+  const long long total = static_cast<long long>(g.m_tiles) * g.n_tiles * g.batches;
+  if (g.kblocks <= kPairResMaxKb && g.n_tiles > 0) {
+    const long long groups = cap_res / g.n_tiles, U = static_cast<long long>(g.m_tiles) * g.batches;
+    if (groups > 0 && U >= kResMinTiles * groups) {
+      resb = true;
+      pairs = static_cast<int>(groups * g.n_tiles);
+      return true;
+    }
+  }
+  if (cap_str <= 0) return false;
+  resb = false;
+  pairs = static_cast<int>(std::min<long long>(total, cap_str));
+  return true;
+}
+
 // g.m_tiles counts 256-token tiles; g.rows_alloc bounds the rows the stores may write.
-// Resident weights when d <= 256 and every pair of a full wave of groups (h / 128 pairs
-// each) gets at least kResMinTiles token tiles to spread its weight load over (the
-// causal language layer's 2048-token chunks give a pair one or two: streaming measured
-// faster there); the streaming form otherwise.
-constexpr int kResMinTiles = 4;
 template <bool SWIGLU>
 cudaError_t launch_token_pair(const CUtensorMap& tX, const CUtensorMap& tFirstHalf, const CUtensorMap& tV,
                               const CUtensorMap& tW2Mn, const CUtensorMap& tHp, const CUtensorMap& tDZ,
@@ -451,19 +472,15 @@ cudaError_t launch_token_pair(const CUtensorMap& tX, const CUtensorMap& tFirstHa
   const long long total = static_cast<long long>(g.m_tiles) * g.n_tiles * g.batches;
   if (total <= 0) return cudaSuccess;
   if (total > 0x7fffffffLL || g.kblocks <= 0) return cudaErrorInvalidConfiguration;
+  const int cap_res = g.kblocks <= kPairResMaxKb ? token_pair_capacity_of<SWIGLU, true>() : 0;
+  bool resb = false;
+  int pairs = 0;
+  if (!pair_grid(g, cap_res, token_pair_capacity<SWIGLU>(), resb, pairs)) return cudaErrorInvalidConfiguration;
   cudaLaunchAttribute attr[1];
-  if (g.kblocks <= PairShape<SWIGLU, true>::KB_RES) {
-    const int cap = token_pair_capacity_of<SWIGLU, true>();
-    const long long groups = cap / g.n_tiles, U = static_cast<long long>(g.m_tiles) * g.batches;
-    if (groups > 0 && U >= kResMinTiles * groups) {
-      cudaLaunchConfig_t cfg = pair_launch_config<SWIGLU, true>(static_cast<int>(groups * g.n_tiles), st, attr);
-      return cudaLaunchKernelEx(&cfg, token_pair_kernel<SWIGLU, true>, tX, tFirstHalf, tV, tW2Mn, tHp, tDZ, g,
-                                status);
-    }
+  if (resb) {
+    cudaLaunchConfig_t cfg = pair_launch_config<SWIGLU, true>(pairs, st, attr);
+    return cudaLaunchKernelEx(&cfg, token_pair_kernel<SWIGLU, true>, tX, tFirstHalf, tV, tW2Mn, tHp, tDZ, g, status);
   }
-  const int cap = token_pair_capacity<SWIGLU>();
-  if (cap <= 0) return cudaErrorInvalidConfiguration;
-  const int pairs = static_cast<int>(std::min<long long>(total, cap));
   cudaLaunchConfig_t cfg = pair_launch_config<SWIGLU, false>(pairs, st, attr);
   return cudaLaunchKernelEx(&cfg, token_pair_kernel<SWIGLU, false>, tX, tFirstHalf, tV, tW2Mn, tHp, tDZ, g, status);
 }
