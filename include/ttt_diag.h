@@ -30,6 +30,8 @@ int ttt_selftest_gemm(int elem_bytes, int a_mn, int b_mn, int bn, int M, int N, 
  *           normal CDF and density; erf from Abramowitz & Stegun 7.1.26, |error| <= 1.5e-7)
  *   kind 1: y = SiLU(x) = x sigma(x), dy = sigma(x) (1 + x (1 - sigma(x))) (sigma from the
  *           hardware tanh approximation, relative error about 2^-11)
+ *   kind 2: y = GELU(x) as the fused apply evaluates it (erf from Abramowitz & Stegun 7.1.28,
+ *           |error| <= 3e-7, one reciprocal and no exponential), dy = 0
  * (the GELU of the ViT3 MLP inner model and the SiLU of the SwiGLU / GLU inner models).
  * x, y, dy: device buffers of n floats, caller-owned.  Enqueued on `stream`;
  * TTT_ERR_INVALID_ARG for an unknown kind or missing buffers, TTT_ERR_CUDA if the launch fails. */

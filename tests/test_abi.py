@@ -288,7 +288,8 @@ def test_every_entry_point_refuses_a_null_handle_or_buffer_without_gpu_work():
     info = (ctypes.c_int * 7)()
     assert lib.ttt_plan_info(None, info, 7) == inv
     assert lib.ttt_selftest_timeout(None, None) == inv
-    assert lib.ttt_selftest_activation(2, 16, fake, fake, fake, None) == inv  # unknown kind
+    assert lib.ttt_selftest_activation(3, 16, fake, fake, fake, None) == inv  # unknown kind
+    assert lib.ttt_selftest_activation(-1, 16, fake, fake, fake, None) == inv
     assert lib.ttt_selftest_activation(0, 16, None, fake, fake, None) == inv
     assert lib.ttt_selftest_activation(0, -1, fake, fake, fake, None) == inv
     assert lib.ttt_selftest_activation(0, 0, None, None, None, None) == 0  # nothing to do

@@ -326,11 +326,12 @@ def selftest_timeout(status_word: torch.Tensor, stream=None) -> int:
 
 
 def selftest_activation(kind: str, x: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
-    """The epilogues' activation ("gelu" or "silu") and its derivative on fp32 device values; see ttt_diag.h."""
+    """The epilogues' activation ("gelu" or "silu") and its derivative, or the apply's GELU alone
+    ("gelu_fwd", derivative 0), on fp32 device values; see ttt_diag.h."""
     if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
         raise ValueError("x must be a contiguous fp32 CUDA tensor")
     y, dy = torch.empty_like(x), torch.empty_like(x)
-    _check(LIB.ttt_selftest_activation({"gelu": 0, "silu": 1}[kind], x.numel(), _ptr(x), _ptr(y), _ptr(dy),
+    _check(LIB.ttt_selftest_activation({"gelu": 0, "silu": 1, "gelu_fwd": 2}[kind], x.numel(), _ptr(x), _ptr(y), _ptr(dy),
                                        _stream_ptr(stream)), "ttt_selftest_activation")
     return y, dy
 

@@ -18,6 +18,7 @@
 // Every wait is bounded.
 #pragma once
 #include "epilogues.cuh"
+#include "gelu_fwd.cuh"
 
 namespace ttt {
 
@@ -256,7 +257,7 @@ __global__ void __launch_bounds__(64 + 32 * ApplyShape<SWIGLU, D, EPIW>::EW, 1)
               a = z1[i] * sigmoid_dev(z1[i]) * z3[i];
               b = z1[i + 1] * sigmoid_dev(z1[i + 1]) * z3[i + 1];
             } else {
-              const float2 gv = gelu2(make_float2(z1[i], z1[i + 1]));
+              const float2 gv = gelu_fwd2(make_float2(z1[i], z1[i + 1]));
               a = gv.x;
               b = gv.y;
             }

@@ -3,6 +3,7 @@
 // ragged edges, batching and split-K can be checked against a library matmul.
 #include "../../include/ttt_diag.h"
 #include "epilogues.cuh"
+#include "gelu_fwd.cuh"
 #include "tc_gemm.cuh"
 
 namespace ttt {
@@ -107,13 +108,16 @@ __global__ void stuck_wait_kernel(unsigned* status) {
 }
 
 // The activation functions of the epilogues, elementwise: kind 0 GELU and its derivative,
-// kind 1 SiLU and its derivative.
+// kind 1 SiLU and its derivative, kind 2 the apply's GELU alone (dy = 0).
 __global__ void activation_kernel(int kind, int64_t n, const float* x, float* y, float* dy) {
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
     const float v = x[i];
     float f, g;
     if (kind == 0) {
       gelu_and_grad(v, f, g);
+    } else if (kind == 2) {
+      f = gelu_fwd2(make_float2(v, v)).x;
+      g = 0.0f;
     } else {
       const float s = sigmoid_dev(v);
       f = v * s;
@@ -128,7 +132,7 @@ __global__ void activation_kernel(int kind, int64_t n, const float* x, float* y,
 }  // namespace ttt
 
 extern "C" int ttt_selftest_activation(int kind, int64_t n, const float* x, float* y, float* dy, void* stream_ptr) {
-  if ((kind != 0 && kind != 1) || n < 0 || (n > 0 && (!x || !y || !dy))) return TTT_ERR_INVALID_ARG;
+  if (kind < 0 || kind > 2 || n < 0 || (n > 0 && (!x || !y || !dy))) return TTT_ERR_INVALID_ARG;
   if (n == 0) return TTT_OK;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
   const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, 4096));
