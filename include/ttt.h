@@ -124,8 +124,8 @@ typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
                                          the linear branch's, W2 = I and this flag */
 
 typedef struct ttt_config {
-  int32_t B, H;       /* batch entries and heads */
-  int32_t N, Nq;      /* key/value tokens and query tokens */
+  int32_t B, H;       /* batch entries and heads (each >= 1) */
+  int32_t N, Nq;      /* key/value tokens and query tokens (each >= 1; above 2^30: unsupported) */
   int32_t d, h;       /* head dim and inner hidden width (ignored for LINEAR) */
   int32_t chunk;      /* tokens per update; <= 0 or >= N means one chunk of N */
   int32_t causal;     /* 1: apply-then-update per chunk (needs Nq == N) */

@@ -53,7 +53,7 @@ def test_every_workload_configuration_is_accepted(name):
 
 
 @pytest.mark.parametrize("bad", [
-    dict(B=0), dict(N=0), dict(d=0), dict(causal=1, Nq=7),
+    dict(B=0), dict(H=0), dict(N=0), dict(Nq=0), dict(d=0), dict(causal=1, Nq=7),
 ])
 def test_invalid_configurations_are_rejected(bad):
     from weight_sequence_mixing_b200 import binding
